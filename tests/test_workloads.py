@@ -1,0 +1,62 @@
+"""Seeded input generator: determinism, prefix property, distributions, bf16 rounding (CPU)."""
+import numpy as np
+import torch
+
+from transformer_norm_rope_b200 import workloads as wl
+
+
+def test_bf16_rounding_matches_torch():
+    a = np.random.default_rng(0).standard_normal(100_000).astype(np.float32) * 100
+    a[:4] = [1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -0.0, 65504.0]  # ties go to even
+    ref = torch.from_numpy(a).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(wl.bf16_bits(a), ref)
+    np.testing.assert_array_equal(wl.bf16_to_f32(ref), torch.from_numpy(a).to(torch.bfloat16).float().numpy())
+
+
+def test_streams_are_deterministic_and_prefix_stable():
+    a = wl.normal(0, wl.S_X, 3 * wl.CHUNK + 17)
+    b = wl.normal(0, wl.S_X, wl.CHUNK + 5)
+    np.testing.assert_array_equal(a[: b.size], b)
+    c = wl.normal(1, wl.S_X, 100)
+    assert not np.array_equal(a[:100], c)
+    d = wl.normal(0, wl.S_DY, 100)
+    assert not np.array_equal(a[:100], d)
+
+
+def test_rmsnorm_recipe():
+    d = wl.rmsnorm(M=1000, N=256)
+    x = wl.bf16_to_f32(d["x"])
+    rms = np.sqrt((x.astype(np.float64) ** 2).mean(1))
+    big = rms > 10
+    assert big.sum() == 10  # floor(1% of 1000) rows scaled by 50
+    np.testing.assert_allclose(rms[big].mean(), 50, rtol=0.05)
+    np.testing.assert_allclose(rms[~big].mean(), 1, rtol=0.05)
+    w = wl.bf16_to_f32(d["w"])
+    assert abs(w.mean() - 1) < 0.03 and abs(w.std() - 0.1) < 0.02
+    g = wl.rmsnorm(M=10, N=256, gemma=True)
+    assert abs(wl.bf16_to_f32(g["w"]).mean()) < 0.03
+
+
+def test_layernorm_recipe():
+    d = wl.layernorm(M=400, N=512)
+    x = wl.bf16_to_f32(d["x"]).astype(np.float64)
+    mu, sd = x.mean(1), x.std(1)
+    assert mu.min() > -2.3 and mu.max() < 2.3 and mu.max() - mu.min() > 3
+    assert sd.min() > 0.4 and sd.max() < 3.3
+    assert abs(wl.bf16_to_f32(d["b"]).std() - 0.1) < 0.02
+
+
+def test_rope_tables():
+    cos, sin = wl.rope_tables(300, 128)
+    assert cos.shape == (300, 64) and cos.dtype == np.float32
+    assert np.all(cos[0] == 1) and np.all(sin[0] == 0)
+    # row p, pair i: angle p * 10000^(-2i/128); pair 0 has frequency 1
+    np.testing.assert_allclose(cos[:, 0], np.cos(np.arange(300)), atol=1e-7)
+    np.testing.assert_allclose(sin[7, 32], np.sin(7 * 10000 ** -0.5), atol=1e-7)
+
+
+def test_qknorm_recipe_shapes():
+    d = wl.qknorm_rope(B=2, S=16, H=4, D=128)
+    assert d["q"].shape == (2, 16, 4, 128) and d["q"].dtype == np.uint16
+    assert d["dq_out"].shape == d["q"].shape and d["wq"].shape == (128,)
+    assert not np.array_equal(d["q"], d["k"])
