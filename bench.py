@@ -1,0 +1,567 @@
+#!/usr/bin/env python3
+"""Benchmark of the fused norm + RoPE hot path on B200 (one JSON line on stdout).
+
+A step is one pass of the whole path over the bf16 long-sequence workloads, every kernel
+launched through the C ABI of libgn:
+
+  RMSNorm x[15360, 5120] fwd + bwd, plain and Gemma weight offset (1% outlier rows x50)
+  LayerNorm + tanh-GeLU x[32768, 5120] fwd + bwd
+  interleaved RoPE in place on q, k [1, 32760, 40, 128] fwd + bwd (sin negated)
+  qk-norm + RoPE on q, k [2, 76800, 40, 128] fwd + bwd
+
+`value` is the algorithmic HBM bytes of a step (each input read once, each output written
+once) divided by the device time of a step, in GB/s (1e9 bytes), summed over all ranks.
+Every input is larger than the 126 MB L2, and consecutive kernels touch different tensors,
+so no L2 flush is inserted. Launch with torchrun for several GPUs: each rank runs the same
+per-GPU workload on its own seeded data (weak scaling, no collective on the data path).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--only KERNEL[,KERNEL]] [--scale F] [--no-e2e] [--no-cpu-baseline]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from transformer_norm_rope_b200 import workloads as wl  # noqa: E402
+
+METRIC = "achieved HBM GB/s (% of B200 peak) for norm+RoPE fwd/bwd, bf16, 1 GPU"
+ORDER = ["rmsnorm_fwd", "layernorm_fwd", "rmsnorm_gemma_fwd", "rope_fwd", "qknorm_rope_fwd",
+         "rmsnorm_bwd", "layernorm_bwd", "rmsnorm_gemma_bwd", "rope_bwd", "qknorm_rope_bwd"]
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--only", default="", help="comma list of kernels to time (default: all)")
+    ap.add_argument("--scale", type=float, default=1.0, help="fraction of rows/tokens (profiling)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seed", type=int, default=0)
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------- workload and byte counts
+
+def sizes(scale):
+    s = lambda n: max(1, int(round(n * scale)))  # noqa: E731
+    return {
+        "rms": dict(M=s(wl.RMSNORM_MAIN["M"]), N=wl.RMSNORM_MAIN["N"]),
+        "ln": dict(M=s(wl.LAYERNORM_MAIN["M"]), N=wl.LAYERNORM_MAIN["N"]),
+        "rope": dict(B=1, S=s(wl.ROPE_MAIN["S"]), H=40, D=128),
+        "qk": dict(B=2, S=s(wl.QKNORM_MAIN["S"]), H=40, D=128),
+    }
+
+
+def algorithmic_bytes(z):
+    """Minimum HBM bytes per launch: every input read once, every output written once."""
+    e = 2  # bf16
+    M, N = z["rms"]["M"], z["rms"]["N"]
+    rms_f = 2 * M * N * e + 4 * M + N * e
+    rms_b = 3 * M * N * e + 4 * M + N * e + 4 * N
+    M, N = z["ln"]["M"], z["ln"]["N"]
+    ln_f = 2 * M * N * e + 8 * M + 2 * N * e
+    ln_b = 3 * M * N * e + 8 * M + 2 * N * e + 8 * N
+    r = z["rope"]
+    E = r["B"] * r["S"] * r["H"] * r["D"]
+    rope = 2 * 2 * E * e + 2 * r["S"] * r["D"] // 2 * 4
+    q = z["qk"]
+    E = q["B"] * q["S"] * q["H"] * q["D"]
+    R = q["B"] * q["S"] * q["H"]
+    tab = 2 * q["S"] * q["D"] // 2 * 4
+    qk_f = 2 * (2 * E * e + 4 * R + q["D"] * e) + tab
+    qk_b = 2 * (3 * E * e + 4 * R + q["D"] * e + 4 * q["D"]) + tab
+    return {"rmsnorm_fwd": rms_f, "rmsnorm_gemma_fwd": rms_f, "rmsnorm_bwd": rms_b, "rmsnorm_gemma_bwd": rms_b,
+            "layernorm_fwd": ln_f, "layernorm_bwd": ln_b, "rope_fwd": rope, "rope_bwd": rope,
+            "qknorm_rope_fwd": qk_f, "qknorm_rope_bwd": qk_b}
+
+
+def rows_of(z):
+    return {"rmsnorm_fwd": z["rms"]["M"], "rmsnorm_gemma_fwd": z["rms"]["M"], "rmsnorm_bwd": z["rms"]["M"],
+            "rmsnorm_gemma_bwd": z["rms"]["M"], "layernorm_fwd": z["ln"]["M"], "layernorm_bwd": z["ln"]["M"],
+            "rope_fwd": 2 * z["rope"]["S"] * z["rope"]["H"], "rope_bwd": 2 * z["rope"]["S"] * z["rope"]["H"],
+            "qknorm_rope_fwd": 2 * z["qk"]["B"] * z["qk"]["S"] * z["qk"]["H"],
+            "qknorm_rope_bwd": 2 * z["qk"]["B"] * z["qk"]["S"] * z["qk"]["H"]}
+
+
+def workload_config(z, l2_note=True):
+    return {
+        "workload": "norm+RoPE bf16 suite: RMSNorm fwd+bwd plain and Gemma x[%d,%d]; LayerNorm+tanh-GeLU "
+                    "fwd+bwd x[%d,%d]; interleaved RoPE fwd+bwd in place q,k[1,%d,40,128]; qk-norm+RoPE "
+                    "fwd+bwd q,k[2,%d,40,128]" % (z["rms"]["M"], z["rms"]["N"], z["ln"]["M"], z["ln"]["N"],
+                                                  z["rope"]["S"], z["qk"]["S"]),
+        "l2": "no flush: every input tensor is larger than the 126 MB L2 and consecutive kernels touch "
+              "different tensors" if l2_note else "n/a",
+        "seed": "seed = rank",
+    }
+
+
+def gen_inputs(z, seed):
+    r, l, o, q = z["rms"], z["ln"], z["rope"], z["qk"]
+    d = {"rms": wl.rmsnorm(M=r["M"], N=r["N"], dtype="bf16", seed=seed)}
+    d["rms_gemma_w"] = wl.normal(seed, wl.S_W, r["N"], "bf16", scale=0.1)
+    d["ln"] = wl.layernorm(M=l["M"], N=l["N"], dtype="bf16", seed=seed)
+    d["rope"] = wl.rope(**o, dtype="bf16", seed=seed)
+    d["qk"] = wl.qknorm_rope(**q, dtype="bf16", seed=seed)
+    return d
+
+
+# ---------------------------------------------------------------- our arm
+
+class Suite:
+    """Device buffers and C-ABI launch closures for one step of the path."""
+
+    def __init__(self, gn, torch, z, host, dev):
+        self.gn, self.torch, self.z, self.dev = gn, torch, z, dev
+        T = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)  # noqa
+        F = lambda a: torch.from_numpy(np.ascontiguousarray(a))  # noqa: E731
+        self.h = {  # host tensors (pageable); inputs of the step
+            "rx": T(host["rms"]["x"]), "rdy": T(host["rms"]["dy"]), "rw": T(host["rms"]["w"]),
+            "rwg": T(host["rms_gemma_w"]),
+            "lx": T(host["ln"]["x"]), "ldy": T(host["ln"]["dy"]), "lw": T(host["ln"]["w"]), "lb": T(host["ln"]["b"]),
+            "oq": T(host["rope"]["q"]), "ok": T(host["rope"]["k"]), "ocos": F(host["rope"]["cos"]),
+            "osin": F(host["rope"]["sin"]),
+            "qq": T(host["qk"]["q"]), "qk": T(host["qk"]["k"]), "qwq": T(host["qk"]["wq"]), "qwk": T(host["qk"]["wk"]),
+            "qcos": F(host["qk"]["cos"]), "qsin": F(host["qk"]["sin"]), "qdq": T(host["qk"]["dq_out"]),
+            "qdk": T(host["qk"]["dk_out"]),
+        }
+        self.inputs = list(self.h)
+        self.d = {k: v.to(dev) for k, v in self.h.items()}
+        E = lambda ref, dt=None: torch.empty_like(ref) if dt is None else torch.empty(ref.shape[:-1], dtype=dt, device=dev)  # noqa
+        d = self.d
+        f32 = torch.float32
+        d.update({
+            "ry": E(d["rx"]), "rr": E(d["rx"], f32), "rdx": E(d["rx"]), "rdw": torch.empty(z["rms"]["N"], dtype=f32, device=dev),
+            "ryg": E(d["rx"]), "rrg": E(d["rx"], f32), "rdxg": E(d["rx"]), "rdwg": torch.empty(z["rms"]["N"], dtype=f32, device=dev),
+            "ly": E(d["lx"]), "lmu": E(d["lx"], f32), "lrs": E(d["lx"], f32), "ldx": E(d["lx"]),
+            "ldw": torch.empty(z["ln"]["N"], dtype=f32, device=dev), "ldb": torch.empty(z["ln"]["N"], dtype=f32, device=dev),
+            "qqo": E(d["qq"]), "qko": E(d["qk"]), "qrq": E(d["qq"], f32), "qrk": E(d["qk"], f32),
+            "qdxq": E(d["qq"]), "qdxk": E(d["qk"]), "qdwq": torch.empty(128, dtype=f32, device=dev),
+            "qdwk": torch.empty(128, dtype=f32, device=dev),
+        })
+        r, l, q = z["rms"], z["ln"], z["qk"]
+        self.ws_r = gn.gn_rmsnorm_bwd_workspace(r["M"], r["N"], gn.GN_BF16)
+        self.ws_l = gn.gn_layernorm_bwd_workspace(l["M"], l["N"], gn.GN_BF16)
+        self.ws_q = gn.gn_qknorm_rope_bwd_workspace(q["B"], q["S"], q["H"], q["D"], gn.GN_BF16)
+        self.ws = torch.empty(max(self.ws_r, self.ws_l, self.ws_q, 16), dtype=torch.uint8, device=dev)
+        # outputs read back by the end-to-end measurement (final value of each output tensor)
+        self.outputs = ["ry", "rr", "rdx", "rdw", "ryg", "rrg", "rdxg", "rdwg", "ly", "lmu", "lrs", "ldx", "ldw",
+                        "ldb", "oq", "ok", "qqo", "qko", "qrq", "qrk", "qdxq", "qdxk", "qdwq", "qdwk"]
+        self.stream = torch.cuda.current_stream(dev)
+
+    def launch(self, name):
+        gn, d, z, s = self.gn, self.d, self.z, self.stream.cuda_stream
+        P = lambda k: d[k].data_ptr()  # noqa: E731
+        r, l, o, q = z["rms"], z["ln"], z["rope"], z["qk"]
+        bf = gn.GN_BF16
+        if name in ("rmsnorm_fwd", "rmsnorm_gemma_fwd"):
+            g = name == "rmsnorm_gemma_fwd"
+            st = gn.gn_rmsnorm_fwd(P("rx"), P("rwg" if g else "rw"), P("ryg" if g else "ry"), P("rrg" if g else "rr"),
+                                   r["M"], r["N"], r["N"], r["N"], 1e-6, int(g), 0, bf, s)
+        elif name in ("rmsnorm_bwd", "rmsnorm_gemma_bwd"):
+            g = name == "rmsnorm_gemma_bwd"
+            st = gn.gn_rmsnorm_bwd(P("rx"), P("rwg" if g else "rw"), P("rrg" if g else "rr"), P("rdy"),
+                                   P("rdxg" if g else "rdx"), P("rdwg" if g else "rdw"), self.ws.data_ptr(),
+                                   self.ws_r, r["M"], r["N"], r["N"], r["N"], r["N"], int(g), 0, bf, s)
+        elif name == "layernorm_fwd":
+            st = gn.gn_layernorm_fwd(P("lx"), P("lw"), P("lb"), P("ly"), P("lmu"), P("lrs"), l["M"], l["N"], l["N"],
+                                     l["N"], 1e-5, gn.GN_EPI_GELU_TANH, bf, s)
+        elif name == "layernorm_bwd":
+            st = gn.gn_layernorm_bwd(P("lx"), P("lw"), P("lb"), P("lmu"), P("lrs"), P("ldy"), P("ldx"), P("ldw"),
+                                     P("ldb"), self.ws.data_ptr(), self.ws_l, l["M"], l["N"], l["N"], l["N"], l["N"],
+                                     gn.GN_EPI_GELU_TANH, bf, s)
+        elif name in ("rope_fwd", "rope_bwd"):
+            st = gn.gn_rope_apply_inplace(P("oq"), P("ok"), P("ocos"), P("osin"), o["B"], o["S"], o["H"], o["D"],
+                                          1 if name == "rope_fwd" else -1, bf, s)
+        elif name == "qknorm_rope_fwd":
+            st = gn.gn_qknorm_rope_fwd(P("qq"), P("qk"), P("qwq"), P("qwk"), P("qcos"), P("qsin"), P("qqo"),
+                                       P("qko"), P("qrq"), P("qrk"), q["B"], q["S"], q["H"], q["D"], 1e-6, 0, bf, s)
+        elif name == "qknorm_rope_bwd":
+            st = gn.gn_qknorm_rope_bwd(P("qq"), P("qk"), P("qwq"), P("qwk"), P("qcos"), P("qsin"), P("qrq"),
+                                       P("qrk"), P("qdq"), P("qdk"), P("qdxq"), P("qdxk"), P("qdwq"), P("qdwk"),
+                                       self.ws.data_ptr(), self.ws_q, q["B"], q["S"], q["H"], q["D"], 0, bf, s)
+        else:
+            raise KeyError(name)
+        gn.check(st, name)
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index):
+        self.samples, self.reasons, self.max_mhz, self.ok = [], set(), None, False
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # noqa: BLE001 - clocks are reported as unavailable
+            self.err = str(e)
+
+    def __enter__(self):
+        self.stop = threading.Event()
+        if self.ok:
+            self.t = threading.Thread(target=self.run, daemon=True)
+            self.t.start()
+        return self
+
+    def run(self):
+        while not self.stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                m = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.reasons |= {n for b, n in self.REASONS.items() if m & b and n != "gpu_idle"}
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(0.01)
+
+    def __exit__(self, *a):
+        self.stop.set()
+        if self.ok:
+            self.t.join()
+
+    def report(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        return float(json.load(open(p))["hbm_gbs"]), "measured"
+    except Exception:  # noqa: BLE001
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def ncu_traffic(kernel, z):
+    """dram bytes per launch of `kernel` from the committed ncu summary, scaled to this
+    workload, or None when there is none or the kernel sources changed since the capture."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        t = json.load(open(p))
+        from transformer_norm_rope_b200 import _build
+
+        if t.get("sources_sha") != _build.sources_digest():
+            return None
+        e = t["kernels"][kernel]
+        return e["dram_bytes_per_launch"] * (algorithmic_bytes(z)[kernel] / e["algorithmic_bytes"])
+    except Exception:  # noqa: BLE001
+        return None
+
+
+def dist_setup(args):
+    import torch
+
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=torch.device("cuda", local))
+    return ws, rank, local
+
+
+def barrier(ws, device):
+    """All ranks meet; the device is idle on return."""
+    import torch
+
+    if ws > 1:
+        import torch.distributed as dist
+
+        if device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+    if device.type == "cuda":
+        torch.cuda.synchronize(device)
+
+
+def reduce_over_ranks(v, ws, device, op):
+    """Combine one float over the ranks ("max" or "sum")."""
+    import torch
+
+    if ws == 1:
+        return float(v)
+    import torch.distributed as dist
+
+    t = torch.tensor([float(v)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def throughput_gbs(bytes_per_rank, elapsed_s, ws, device):
+    """Whole-job GB/s: the bytes all ranks processed over the slowest rank's device time."""
+    tot = reduce_over_ranks(bytes_per_rank, ws, device, "sum")
+    el = reduce_over_ranks(elapsed_s, ws, device, "max")
+    return tot / el / 1e9, el
+
+
+def run_ours(args):
+    import torch
+
+    import transformer_norm_rope_b200 as gn
+
+    ws, rank, local = dist_setup(args)
+    dev = torch.device("cuda", local)
+
+    torch.cuda.set_device(dev)
+    gn.load()
+    z = sizes(args.scale)
+    kernels = [k for k in ORDER if not args.only or k in args.only.split(",")]
+    host = gen_inputs(z, args.seed + rank)
+    suite = Suite(gn, torch, z, host, dev)
+    nbytes = algorithmic_bytes(z)
+    step_bytes = sum(nbytes[k] for k in kernels)
+    # the backward kernels read the forward statistics: run each forward once before timing
+    for k in ORDER:
+        if k.endswith("_fwd") and k.replace("_fwd", "_bwd") in kernels and k not in kernels:
+            suite.launch(k)
+    stream = suite.stream
+
+    def step(ev=None):
+        for i, k in enumerate(kernels):
+            if ev is not None:
+                ev[i][0].record(stream)
+            suite.launch(k)
+            if ev is not None:
+                ev[i][1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+        if "rope_fwd" in kernels and "rope_bwd" not in kernels:  # keep rotated tensors bounded
+            suite.launch("rope_bwd")
+    barrier(ws, dev)
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in kernels]
+          for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n0 = gn.gn_launch_count()
+    with ClockSampler(dev.index) as clk:
+        barrier(ws, dev)
+        t0.record(stream)
+        for i in range(args.steps):
+            step(ev[i])
+        t1.record(stream)
+        t1.synchronize()
+        barrier(ws, dev)
+    launches = gn.gn_launch_count() - n0
+    value, elapsed = throughput_gbs(step_bytes * args.steps, t0.elapsed_time(t1) * 1e-3, ws, dev)
+    per_kernel = {k: statistics.mean(ev[i][j][0].elapsed_time(ev[i][j][1]) for i in range(args.steps)) * 1e-3
+                  for j, k in enumerate(kernels)}
+    peak, peak_kind = peaks()
+    dom = max(kernels, key=lambda k: per_kernel[k])
+    ach = nbytes[dom] / per_kernel[dom] / 1e9
+    traffic = ncu_traffic(dom, z)
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(elapsed / args.steps * 1e3, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded generator, seed = rank)",
+        "config": dict(workload_config(z), parallelism=f"replica per GPU x{ws} (weak, no collective)",
+                       bytes_per_step_per_gpu=step_bytes),
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(ach / peak, 4), "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs"},
+        "kernels": {k: {"ms": round(per_kernel[k] * 1e3, 4), "GB_s": round(nbytes[k] / per_kernel[k] / 1e9, 1),
+                        "frac_of_peak": round(nbytes[k] / per_kernel[k] / 1e9 / peak, 4),
+                        "rows_per_s": round(rows_of(z)[k] / per_kernel[k], 1)} for k in kernels},
+        "frac_of_peak": round(value / ws / peak, 4),
+        "frac_of_8TBs": round(value / ws / 8000.0, 4),
+        "clocks": clk.report(),
+        "gpu_launches": int(launches),
+    }
+    if not args.no_e2e:
+        out["e2e"] = e2e(args, suite, kernels, step_bytes, ws, dev)
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(host, z, kernels, budget_s=15.0)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+def e2e(args, suite, kernels, step_bytes, ws, dev):
+    """Same metric through host buffers: each step copies its inputs from pinned host memory,
+    runs the path, and copies every output back to pinned host memory."""
+    import torch
+
+    steps = max(1, min(args.steps, 5))
+    need = set()
+    for k in kernels:
+        need |= set(INPUTS[k])
+    ins = [k for k in suite.inputs if k in need]
+    outs = [k for k in suite.outputs if any(k in OUTPUTS[x] for x in kernels)]
+    pin_in = {k: suite.h[k].pin_memory() for k in ins}
+    pin_out = {k: torch.empty(suite.d[k].shape, dtype=suite.d[k].dtype, pin_memory=True) for k in outs}
+    h2d = sum(v.numel() * v.element_size() for v in pin_in.values())
+    d2h = sum(v.numel() * v.element_size() for v in pin_out.values())
+    stream = suite.stream
+
+    def one():
+        for k in ins:
+            suite.d[k].copy_(pin_in[k], non_blocking=True)
+        for k in kernels:
+            suite.launch(k)
+        for k in outs:
+            pin_out[k].copy_(suite.d[k], non_blocking=True)
+
+    one()
+    barrier(ws, dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        one()
+    b.record(stream)
+    b.synchronize()
+    barrier(ws, dev)
+    v, _ = throughput_gbs(step_bytes * steps, a.elapsed_time(b) * 1e-3, ws, dev)
+    return {"value": round(v, 2), "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "steps": steps}
+
+
+INPUTS = {
+    "rmsnorm_fwd": ["rx", "rw"], "rmsnorm_gemma_fwd": ["rx", "rwg"],
+    "rmsnorm_bwd": ["rx", "rw", "rdy"], "rmsnorm_gemma_bwd": ["rx", "rwg", "rdy"],
+    "layernorm_fwd": ["lx", "lw", "lb"], "layernorm_bwd": ["lx", "lw", "lb", "ldy"],
+    "rope_fwd": ["oq", "ok", "ocos", "osin"], "rope_bwd": ["ocos", "osin"],
+    "qknorm_rope_fwd": ["qq", "qk", "qwq", "qwk", "qcos", "qsin"],
+    "qknorm_rope_bwd": ["qq", "qk", "qwq", "qwk", "qcos", "qsin", "qdq", "qdk"],
+}
+OUTPUTS = {
+    "rmsnorm_fwd": ["ry", "rr"], "rmsnorm_gemma_fwd": ["ryg", "rrg"], "rmsnorm_bwd": ["rdx", "rdw"],
+    "rmsnorm_gemma_bwd": ["rdxg", "rdwg"], "layernorm_fwd": ["ly", "lmu", "lrs"], "layernorm_bwd": ["ldx", "ldw", "ldb"],
+    "rope_fwd": [], "rope_bwd": ["oq", "ok"], "qknorm_rope_fwd": ["qqo", "qko", "qrq", "qrk"],
+    "qknorm_rope_bwd": ["qdxq", "qdxk", "qdwq", "qdwk"],
+}
+
+
+# ---------------------------------------------------------------- the fp64 CPU oracle arm
+
+def oracle_step(host, z, kernels, frac):
+    """Runs the oracle on the first `frac` of the rows/tokens of each kernel; returns
+    (seconds, algorithmic bytes of the sample)."""
+    import oracle
+
+    nb = algorithmic_bytes(z)
+    done, t = 0.0, 0.0
+    r, l, o, q = host["rms"], host["ln"], host["rope"], host["qk"]
+    for k in kernels:
+        if k.startswith("rmsnorm"):
+            M = z["rms"]["M"]
+            m = max(1, int(M * frac))
+            w = host["rms_gemma_w"] if "gemma" in k else r["w"]
+            g = "gemma" in k
+            s = time.perf_counter()
+            if k.endswith("fwd"):
+                oracle.rmsnorm_fwd(r["x"][:m], w, 1e-6, gemma=g)
+            else:
+                oracle.rmsnorm_bwd(r["x"][:m], w, r["dy"][:m], 1e-6, gemma=g)
+            t += time.perf_counter() - s
+            done += nb[k] * m / M
+        elif k.startswith("layernorm"):
+            M = z["ln"]["M"]
+            m = max(1, int(M * frac))
+            s = time.perf_counter()
+            if k.endswith("fwd"):
+                oracle.layernorm_fwd(l["x"][:m], l["w"], l["b"], 1e-5, act="gelu_tanh")
+            else:
+                oracle.layernorm_bwd(l["x"][:m], l["w"], l["b"], l["dy"][:m], 1e-5, act="gelu_tanh")
+            t += time.perf_counter() - s
+            done += nb[k] * m / M
+        elif k.startswith("rope"):
+            S = z["rope"]["S"]
+            m = max(1, int(S * frac))
+            sign = 1 if k == "rope_fwd" else -1
+            s = time.perf_counter()
+            oracle.rope(o["q"][:, :m], o["cos"][:m], o["sin"][:m], sign)
+            oracle.rope(o["k"][:, :m], o["cos"][:m], o["sin"][:m], sign)
+            t += time.perf_counter() - s
+            done += nb[k] * m / S
+        else:
+            S = z["qk"]["S"]
+            m = max(1, int(S * frac))
+            s = time.perf_counter()
+            for x, w, dy in (("q", "wq", "dq_out"), ("k", "wk", "dk_out")):
+                if k.endswith("fwd"):
+                    oracle.qknorm_rope_fwd(q[x][:, :m], q[w], q["cos"][:m], q["sin"][:m], 1e-6)
+                else:
+                    oracle.qknorm_rope_bwd(q[x][:, :m], q[w], q["cos"][:m], q["sin"][:m], q[dy][:, :m], 1e-6)
+            t += time.perf_counter() - s
+            done += nb[k] * m / S
+    return t, done
+
+
+def cpu_baseline(host, z, kernels, budget_s):
+    t, done = oracle_step(host, z, kernels, 1.0 / 4096)
+    frac = min(1.0, (1.0 / 4096) * max(1.0, budget_s / max(t, 1e-3)))
+    t, done = oracle_step(host, z, kernels, frac)
+    return {"value": round(done / t / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"first {frac:.5f} of the rows/tokens of every kernel of the step ({t:.1f} s of fp64 C oracle, "
+                      "single thread, same seeded inputs)"}
+
+
+def run_reference(args):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    z = sizes(args.scale)
+    kernels = [k for k in ORDER if not args.only or k in args.only.split(",")]
+    host = gen_inputs(z, args.seed)
+    # size each step's sample so that warmup + steps stay within about two minutes
+    t, _ = oracle_step(host, z, kernels, 1.0 / 8192)
+    frac = (1.0 / 8192) * max(1.0, min(64.0, 120.0 / max(1, args.steps + args.warmup) / max(t, 1e-3)))
+    for _ in range(args.warmup):
+        oracle_step(host, z, kernels, frac)
+    tot_t, tot_b = 0.0, 0.0
+    for _ in range(args.steps):
+        t, b = oracle_step(host, z, kernels, frac)
+        tot_t += t
+        tot_b += b
+    v = tot_b / tot_t / 1e9
+    sample = f"first {frac:.6f} of the rows/tokens of every kernel per step (fp64 C oracle, single thread)"
+    out = {"metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": round(tot_t / args.steps * 1e3, 3), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded generator, seed 0)",
+           "config": dict(workload_config(z), parallelism="host oracle, rank 0 only"), "impl": "reference",
+           "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+           "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,196 @@
+/*
+ * gn.h - C ABI of libgn: fused row normalization and interleaved rotary position embedding
+ * for NVIDIA B200 (sm_100a).
+ *
+ * Sources of the operations (page title, section):
+ *   [H] "Helios 性能优化全解析: 3 个 Triton 自定义内核如何让实时长视频生成提速 16%"
+ *       - "内核一 FlashNorm": RMSNorm / LayerNorm with mean, variance and scaling in one
+ *         memory pass per row, one thread block per row, the per-row inverse statistic saved
+ *         by the forward and reused by the backward, a Gemma-style +1 weight offset handled by
+ *         a compile-time branch in the same kernel.
+ *       - "内核二 FlashRoPE": rotary embedding on an interleaved even/odd layout, pair i read
+ *         at offsets 2i and 2i+1, rotated in place without intermediate tensors; the backward
+ *         is the same kernel with sin negated.
+ *       - "基准实测": FlashNorm and FlashRoPE applied together (the fused qk-norm + RoPE entry
+ *         points combine them per attention head).
+ *   [L] "LLM层的优化算子", section "编写定制融合算子": LayerNorm fused with a tanh-GeLU epilogue
+ *       (centre, biased variance, divide by sqrt(var + eps), times weight plus bias, GeLU).
+ *   [J] "Janus-Pro-7B模型推理加速实战", section 4.1: LayerNorm fused with SiLU = x * sigmoid(x).
+ *
+ * Conventions for every entry point:
+ *   - Pointers are DEVICE pointers owned by the caller, except where stated. The library
+ *     allocates nothing, frees nothing and never synchronizes; each call enqueues its kernels
+ *     on `stream` (a cudaStream_t; NULL = the legacy default stream) and returns.
+ *   - Matrices are row-major. `ld_*` is the distance in ELEMENTS between consecutive rows.
+ *     Rotary tensors are contiguous [B, S, H, D]; tables are contiguous fp32 [S, D/2].
+ *   - `dt` selects the element type of x, y, dy, dx, w, b, q, k (GN_F32 or GN_BF16).
+ *     Saved statistics (inv_rms, mean, rstd), weight gradients and tables are always fp32.
+ *   - Arithmetic is fp32 with one round-to-nearest-even per stored bf16 element.
+ *   - Arguments are checked before anything is enqueued. A check that fails returns its
+ *     status and enqueues nothing:
+ *       GN_ERR_NULL         a required pointer is NULL
+ *       GN_ERR_SHAPE        a size is negative or zero where it must be positive, ld < hidden,
+ *                           D odd or not a multiple of 8, sign not +1/-1
+ *       GN_ERR_ALIGN        a row/tensor base pointer or a row stride in bytes is not a
+ *                           multiple of 16
+ *       GN_ERR_DTYPE        unknown dtype or epilogue
+ *       GN_ERR_WORKSPACE    ws is NULL or ws_bytes below the size the *_workspace query gives
+ *       GN_ERR_UNSUPPORTED  a row does not fit the kernel's shared-memory stage (see each call)
+ *       GN_ERR_CUDA         the CUDA runtime reported an error while querying the device or
+ *                           launching (the kernels' own faults surface at the next sync)
+ *   - rows == 0 (or B*S*H == 0) is valid once the other sizes check out: nothing is launched,
+ *     data pointers may be NULL, and weight gradients that are not NULL are set to zero.
+ *   - A kernel never spins without bound: each wait for an asynchronous copy gives up after
+ *     one second, records GN_DEVERR_WAIT_TIMEOUT in the device error word (gn_device_error)
+ *     and returns.
+ *   - Calls are thread-safe and keep no state between calls apart from the launch counter
+ *     and the device error word.
+ */
+#ifndef GN_H
+#define GN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GN_OK = 0,
+  GN_ERR_NULL = 1,
+  GN_ERR_SHAPE = 2,
+  GN_ERR_ALIGN = 3,
+  GN_ERR_DTYPE = 4,
+  GN_ERR_WORKSPACE = 5,
+  GN_ERR_UNSUPPORTED = 6,
+  GN_ERR_CUDA = 7
+} gn_status;
+
+typedef enum { GN_F32 = 0, GN_BF16 = 1 } gn_dtype;
+
+/* epilogue applied to z = normalized * weight (+ bias) before the store */
+typedef enum { GN_EPI_NONE = 0, GN_EPI_GELU_TANH = 1, GN_EPI_SILU = 2 } gn_epilogue;
+
+/* device error word bits */
+#define GN_DEVERR_WAIT_TIMEOUT 1u
+
+/* Human-readable name of a status. Never NULL. */
+const char* gn_status_string(gn_status s);
+
+/* ---------------------------------------------------------------- RMSNorm ([H] FlashNorm)
+ * Forward, per row m of x[rows, hidden]:
+ *   r = 1 / sqrt(mean_j(x[m,j]^2) + eps)            (eps inside the root)
+ *   w'_j = w_j, or 1 + w_j when gemma != 0          (formed in fp32, not rounded to dt)
+ *   y[m,j] = epi(x[m,j] * r * w'_j)
+ *   inv_rms[m] = r                                  (fp32; may be NULL: not saved)
+ * x, y: device, dt, rows of `hidden` elements with strides ld_x, ld_y (16-byte aligned).
+ * w: device, dt, [hidden], required. y may alias x when ld_y == ld_x (in place).
+ * Limit: hidden <= 16384 (bf16) / 8192 (fp32), else GN_ERR_UNSUPPORTED (each thread keeps
+ * its share of the row in registers between the reduction and the store). */
+gn_status gn_rmsnorm_fwd(const void* x, const void* w, void* y, float* inv_rms, int64_t rows,
+                         int64_t hidden, int64_t ld_x, int64_t ld_y, float eps, int gemma,
+                         gn_epilogue epi, gn_dtype dt, void* stream);
+
+/* Workspace in bytes that gn_rmsnorm_bwd needs for these sizes on the current device
+ * (per-block fp32 partial sums of dw). 0 on error or when rows == 0. */
+size_t gn_rmsnorm_bwd_workspace(int64_t rows, int64_t hidden, gn_dtype dt);
+
+/* Backward of gn_rmsnorm_fwd, reusing the saved inv_rms instead of recomputing it:
+ *   z = x r w', g = dy * epi'(z), xhat = x r
+ *   dx[m,j] = r * (g_j w'_j - xhat_j * mean_k(g_k w'_k xhat_k))
+ *   dw[j]   = sum_m g[m,j] xhat[m,j]            (fp32, deterministic fixed-order reduction;
+ *                                              the same for gemma since d w'/d w = 1)
+ * inv_rms: fp32 [rows] from the forward (required). dy, dx: dt rows with ld_dy, ld_dx.
+ * dw: fp32 [hidden], may be NULL (weight gradient skipped, ws then unused and may be NULL).
+ * ws: device scratch of at least gn_rmsnorm_bwd_workspace(rows, hidden, dt) bytes, 16-byte
+ * aligned, owned by the caller, contents ignored on entry. dx may alias dy.
+ * Limit: hidden <= 8192 (bf16) / 4096 (fp32), else GN_ERR_UNSUPPORTED. */
+gn_status gn_rmsnorm_bwd(const void* x, const void* w, const float* inv_rms, const void* dy,
+                         void* dx, float* dw, void* ws, size_t ws_bytes, int64_t rows,
+                         int64_t hidden, int64_t ld_x, int64_t ld_dy, int64_t ld_dx, int gemma,
+                         gn_epilogue epi, gn_dtype dt, void* stream);
+
+/* ---------------------------------------------------------------- LayerNorm ([H] FlashNorm, [L], [J])
+ * Forward, per row m:
+ *   mu = mean_j x[m,j];  var = mean_j (x[m,j] - mu)^2  (biased);  s = 1 / sqrt(var + eps)
+ *   y[m,j] = epi((x[m,j] - mu) * s * w_j + b_j)
+ *   mean[m] = mu, rstd[m] = s                          (fp32; each may be NULL)
+ * w, b: dt [hidden]; w == NULL means 1, b == NULL means 0. Same layout rules and limits as
+ * gn_rmsnorm_fwd. */
+gn_status gn_layernorm_fwd(const void* x, const void* w, const void* b, void* y, float* mean,
+                           float* rstd, int64_t rows, int64_t hidden, int64_t ld_x, int64_t ld_y,
+                           float eps, gn_epilogue epi, gn_dtype dt, void* stream);
+
+size_t gn_layernorm_bwd_workspace(int64_t rows, int64_t hidden, gn_dtype dt);
+
+/* Backward of gn_layernorm_fwd from the saved mean and rstd:
+ *   xhat = (x - mu) s, z = xhat w + b, g = dy * epi'(z)
+ *   dx[m,j] = s * (g_j w_j - mean_k(g_k w_k) - xhat_j * mean_k(g_k w_k xhat_k))
+ *   dw[j] = sum_m g xhat,  db[j] = sum_m g         (fp32; each may be NULL)
+ * mean, rstd: fp32 [rows], required. b is read only to recompute z for an epilogue.
+ * ws as for gn_rmsnorm_bwd (may be NULL when dw and db are both NULL). */
+gn_status gn_layernorm_bwd(const void* x, const void* w, const void* b, const float* mean,
+                           const float* rstd, const void* dy, void* dx, float* dw, float* db,
+                           void* ws, size_t ws_bytes, int64_t rows, int64_t hidden, int64_t ld_x,
+                           int64_t ld_dy, int64_t ld_dx, gn_epilogue epi, gn_dtype dt,
+                           void* stream);
+
+/* ---------------------------------------------------------------- RoPE ([H] FlashRoPE)
+ * In-place rotary embedding of q and (optionally) k, both contiguous [B, S, H, D] of dt.
+ * For every (b, s, h) and pair i < D/2, with c = cos[s, i], t = sign * sin[s, i]:
+ *   (x[2i], x[2i+1]) <- (x[2i] c - x[2i+1] t,  x[2i] t + x[2i+1] c)
+ * cos, sin: fp32 [S, D/2], row s serving token s of every batch entry and head.
+ * sign = +1: forward rotation; sign = -1: its inverse, which is the backward (apply it to
+ * dq, dk in place). k may be NULL. D must be even and a multiple of 8. */
+gn_status gn_rope_apply_inplace(void* q, void* k, const float* cos, const float* sin, int64_t B,
+                                int64_t S, int64_t H, int64_t D, int sign, gn_dtype dt,
+                                void* stream);
+
+/* ---------------------------------------------------------------- qk-norm + RoPE ([H] FlashNorm + FlashRoPE)
+ * For q (and k when not NULL), contiguous [B, S, H, D] of dt, per head row (b, s, h):
+ *   r = 1 / sqrt(mean_d x_d^2 + eps); n_d = x_d r w'_d   (w' = w or 1 + w with gemma)
+ *   out = rope(n, cos[s], sin[s], +1)                      (out of place)
+ *   inv_rms[b, s, h] = r                                   (fp32 [B, S, H]; may be NULL)
+ * wq, wk: dt [D] (one weight per tensor shared by all heads). D/8 (bf16) or D/4 (fp32) must
+ * be a power of two <= 32 (D in {8,...,256} bf16, {8,...,128} fp32), else
+ * GN_ERR_UNSUPPORTED. */
+gn_status gn_qknorm_rope_fwd(const void* q, const void* k, const void* wq, const void* wk,
+                             const float* cos, const float* sin, void* q_out, void* k_out,
+                             float* inv_rms_q, float* inv_rms_k, int64_t B, int64_t S, int64_t H,
+                             int64_t D, float eps, int gemma, gn_dtype dt, void* stream);
+
+size_t gn_qknorm_rope_bwd_workspace(int64_t B, int64_t S, int64_t H, int64_t D, gn_dtype dt);
+
+/* Backward of gn_qknorm_rope_fwd from the pre-norm inputs and the saved inv_rms:
+ *   u = rope(dy, cos[s], sin[s], -1)                       (inverse rotation of the gradient)
+ *   dx_d = r (u_d w'_d - xhat_d mean_e(u_e w'_e xhat_e)),  xhat = x r
+ *   dw_d = sum over all head rows of u_d xhat_d            (fp32, fixed-order reduction)
+ * dq_out, dk_out: gradients of q_out, k_out (dt). dq, dk: outputs (dt, may alias dq_out /
+ * dk_out). dwq, dwk: fp32 [D], may be NULL. ws as for gn_rmsnorm_bwd. */
+gn_status gn_qknorm_rope_bwd(const void* q, const void* k, const void* wq, const void* wk,
+                             const float* cos, const float* sin, const float* inv_rms_q,
+                             const float* inv_rms_k, const void* dq_out, const void* dk_out,
+                             void* dq, void* dk, float* dwq, float* dwk, void* ws,
+                             size_t ws_bytes, int64_t B, int64_t S, int64_t H, int64_t D,
+                             int gemma, gn_dtype dt, void* stream);
+
+/* ---------------------------------------------------------------- runtime queries
+ * Number of kernels this process has launched through libgn (all devices, all threads). */
+uint64_t gn_launch_count(void);
+
+/* Reads (and with clear != 0 then zeroes) the device error word of the current device into
+ * *word. Synchronizes the device. GN_ERR_NULL if word is NULL, GN_ERR_CUDA on a runtime
+ * error. */
+gn_status gn_device_error(unsigned* word, int clear);
+
+/* Tuning knobs of the launch planner, for benchmarking sweeps. key is one of "stages",
+ * "ctas_per_sm", "vpt", "unit_bytes", "group_rows"; value 0 restores the default. Returns
+ * GN_ERR_SHAPE for an unknown key or a negative value. Not thread-safe with concurrent
+ * launches. */
+gn_status gn_tune(const char* key, int value);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GN_H */

@@ -153,13 +153,14 @@ def rope(x, cos, sin, sign=+1):
     return out
 
 
-def qknorm_rope_fwd(x, w, cos, sin, eps, gemma=False):
-    """out[B,S,H,D], inv_rms[B,S,H]: per-head RMSNorm then the forward rotary embedding."""
+def qknorm_rope_fwd(x, w, cos, sin, eps, gemma=False, want_out=True):
+    """out[B,S,H,D] (None unless want_out), inv_rms[B,S,H]: per-head RMSNorm then the forward
+    rotary embedding."""
     x, xd = _in(x)
     w, wd = _in(w)
     cos, sin, td = _tables(cos, sin)
     B, S, H, D = x.shape
-    out = np.empty(x.shape)
+    out = np.empty(x.shape) if want_out else None
     r = np.empty((B, S, H))
     _load().oracle_qknorm_rope_fwd(_p(x), xd, _p(w), wd, _p(cos), _p(sin), td, B, S, H, D, eps,
                                    int(gemma), _p(out), _p(r))

@@ -1,0 +1,83 @@
+"""Host logic of the benchmark (CPU): byte accounting, the multi-rank timing reduction over a
+world of 2 gloo ranks, and the oracle (reference) arm's JSON line on a tiny sample."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_algorithmic_bytes_match_the_workload_table():
+    b = bench.algorithmic_bytes(bench.sizes(1.0))
+    mb = {k: round(v / 1e6, 1) for k, v in b.items()}
+    assert mb["rmsnorm_fwd"] == 314.6 and mb["rmsnorm_bwd"] == 472.0
+    assert mb["layernorm_fwd"] == 671.4 and mb["layernorm_bwd"] == 1007.0
+    assert mb["rope_fwd"] == 1358.6 and mb["rope_bwd"] == 1358.6
+    assert mb["qknorm_rope_fwd"] == 6379.9 and mb["qknorm_rope_bwd"] == 9525.7
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _worker(rank, ws, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=ws)
+    try:
+        dev = torch.device("cpu")
+        bench.barrier(ws, dev)
+        # rank r processed 1e9*(r+1) bytes in (r+1) seconds: the job moved 3e9 bytes and the
+        # slowest rank took 2 s, so the whole-job figure is 1.5 GB/s (not the mean of ratios)
+        v, el = bench.throughput_gbs(1e9 * (rank + 1), float(rank + 1), ws, dev)
+        mx = bench.reduce_over_ranks(rank * 10.0, ws, dev, "max")
+        q.put((rank, v, el, mx))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_timing_reduction_over_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(2))
+    for rank, v, el, mx in res:
+        assert v == pytest.approx(1.5) and el == 2.0 and mx == 10.0
+
+
+def test_reference_arm_prints_one_json_line():
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0")
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--scale", "0.002", "--steps", "2",
+                        "--warmup", "1"], cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    out = json.loads(lines[0])
+    assert out["impl"] == "reference" and out["unit"] == "GB/s" and out["value"] > 0
+    assert out["cpu_baseline"]["kind"] == "oracle" and out["cpu_baseline"]["cores"] == 1
+    assert out["e2e"]["h2d_bytes_per_step"] == 0 and out["metric"] == bench.METRIC
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    env = dict(os.environ, WORLD_SIZE="2", RANK="1")
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--scale", "0.001", "--steps", "1",
+                        "--warmup", "0"], cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and r.stdout.strip() == ""

@@ -1,0 +1,185 @@
+"""GPU parity of the RMSNorm and LayerNorm kernels against the fp64 oracle.
+
+Small cases span several CTAs and row tiles, ragged tails (hidden not a multiple of the
+16-byte vector), both launch shapes (lane group per row for short rows, CTA per row with the
+TMA pipeline for long rows), strided rows, in-place outputs and empty inputs. The full-size
+cases run the exact launch configuration the benchmark times and compare sampled rows, every
+saved statistic and the complete weight gradients.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from transformer_norm_rope_b200 import workloads as wl
+from tests._util import assert_close, grad_tol, io_tol, to_dev, to_np, wgrad_tol
+
+
+def to_rows(a):
+    """Generator matrix -> device tensor whose rows start on 16-byte boundaries (row stride
+    padded when the width is ragged, as the C ABI requires)."""
+    import transformer_norm_rope_b200 as gn
+
+    t = to_dev(a)
+    out = gn.empty_rows(t.shape, t.dtype, t.device)
+    out.copy_(t)
+    return out
+
+pytestmark = pytest.mark.gpu
+
+EPIS = ["none", "gelu_tanh", "silu"]
+# (rows, hidden): PR1 shape; group path (short rows, incl. lanes < 32 and ragged tails);
+# CTA path (long rows, ragged tails, more rows than the persistent grid)
+SHAPES = [(256, 1024), (33, 72), (129, 1000), (5, 9), (65, 2051), (300, 5120), (3, 8192), (1200, 1536)]
+
+
+def rms_case(rows, hidden, dtype, gemma, seed=0):
+    d = wl.rmsnorm(M=rows, N=hidden, dtype=dtype, gemma=gemma, seed=seed, outliers=rows >= 100)
+    return d
+
+
+@pytest.mark.parametrize("rows,hidden", SHAPES)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_rmsnorm_fwd_bwd(gpu, rows, hidden, dtype):
+    if dtype == "f32" and hidden > 4096:
+        hidden = 4096  # fp32 backward rows stop at 4096
+    for gemma, epi in ((False, "none"), (True, "gelu_tanh"), (False, "silu")):
+        d = rms_case(rows, hidden, dtype, gemma)
+        x, w, dy = to_rows(d["x"]), to_dev(d["w"]), to_rows(d["dy"])
+        y, r = gpu.rmsnorm_fwd(x, w, d["eps"], gemma=gemma, epilogue=epi)
+        dx, dw = gpu.rmsnorm_bwd(x, w, r, dy, gemma=gemma, epilogue=epi)
+        torch.cuda.synchronize()
+        ry, rr = oracle.rmsnorm_fwd(d["x"], d["w"], d["eps"], gemma=gemma, act=epi)
+        rdx, rdw = oracle.rmsnorm_bwd(d["x"], d["w"], d["dy"], d["eps"], gemma=gemma, act=epi)
+        tag = f"rms {dtype} {rows}x{hidden} gemma={gemma} {epi}"
+        assert_close(to_np(y), ry, io_tol(dtype), tag + " y")
+        assert_close(to_np(r), rr, "stat", tag + " inv_rms")
+        assert_close(to_np(dx), rdx, grad_tol(dtype), tag + " dx")
+        assert_close(to_np(dw), rdw, wgrad_tol(dtype, rdw), tag + " dw")
+
+
+@pytest.mark.parametrize("rows,hidden", SHAPES)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_layernorm_fwd_bwd(gpu, rows, hidden, dtype):
+    if dtype == "f32" and hidden > 4096:
+        hidden = 4096
+    for epi, affine in (("gelu_tanh", True), ("none", True), ("silu", False)):
+        d = wl.layernorm(M=rows, N=hidden, dtype=dtype)
+        w = d["w"] if affine else None
+        b = d["b"] if affine else None
+        x, dy = to_rows(d["x"]), to_rows(d["dy"])
+        wt = to_dev(w) if affine else None
+        bt = to_dev(b) if affine else None
+        y, mu, rs = gpu.layernorm_fwd(x, wt, bt, d["eps"], epilogue=epi)
+        dx, dw, db = gpu.layernorm_bwd(x, wt, bt, mu, rs, dy, epilogue=epi)
+        torch.cuda.synchronize()
+        ry, rmu, rrs = oracle.layernorm_fwd(d["x"], w, b, d["eps"], act=epi)
+        rdx, rdw, rdb = oracle.layernorm_bwd(d["x"], w, b, d["dy"], d["eps"], act=epi)
+        tag = f"ln {dtype} {rows}x{hidden} {epi} affine={affine}"
+        assert_close(to_np(y), ry, io_tol(dtype), tag + " y")
+        # the mean is compared with an absolute floor: rows are centred anywhere in (-2, 2)
+        assert_close(to_np(mu), rmu, (1e-5, 1e-6), tag + " mean")
+        assert_close(to_np(rs), rrs, "stat", tag + " rstd")
+        assert_close(to_np(dx), rdx, grad_tol(dtype), tag + " dx")
+        assert_close(to_np(dw), rdw, wgrad_tol(dtype, rdw), tag + " dw")
+        assert_close(to_np(db), rdb, wgrad_tol(dtype, rdb), tag + " db")
+
+
+@pytest.mark.parametrize("hidden", [72, 5120])
+def test_strided_rows_and_in_place(gpu, hidden):
+    rows, ld = 40, hidden + 64
+    d = wl.rmsnorm(M=rows, N=hidden, dtype="bf16", outliers=False)
+    base = torch.zeros(rows, ld, dtype=torch.bfloat16, device="cuda")
+    base[:, :hidden] = to_dev(d["x"])
+    xs = base[:, :hidden]
+    w = to_dev(d["w"])
+    y, r = gpu.rmsnorm_fwd(xs, w, d["eps"])
+    ry, rr = oracle.rmsnorm_fwd(d["x"], d["w"], d["eps"])
+    assert_close(to_np(y), ry, "bf16", "strided rms y")
+    gpu.rmsnorm_fwd(xs, w, d["eps"], out=xs)  # in place on a strided view
+    assert_close(to_np(xs), ry, "bf16", "in-place rms y")
+    assert torch.all(base[:, hidden:] == 0), "padding between rows was written"
+    dl = wl.layernorm(M=rows, N=hidden, dtype="bf16")
+    x = to_dev(dl["x"])
+    gpu.layernorm_fwd(x, to_dev(dl["w"]), to_dev(dl["b"]), dl["eps"], epilogue="gelu_tanh", out=x)
+    ry, _, _ = oracle.layernorm_fwd(dl["x"], dl["w"], dl["b"], dl["eps"], act="gelu_tanh")
+    assert_close(to_np(x), ry, "bf16", "in-place ln y")
+
+
+def test_empty_rows(gpu):
+    x = torch.empty(0, 512, dtype=torch.bfloat16, device="cuda")
+    w = torch.ones(512, dtype=torch.bfloat16, device="cuda")
+    y, r = gpu.rmsnorm_fwd(x, w)
+    assert y.shape == (0, 512)
+    dx, dw = gpu.rmsnorm_bwd(x, w, r, x)
+    dxl, dwl, dbl = gpu.layernorm_bwd(x, w, None, r, r, x)
+    torch.cuda.synchronize()
+    assert torch.all(dw == 0) and torch.all(dwl == 0) and torch.all(dbl == 0)
+
+
+def test_unsupported_hidden_is_reported(gpu):
+    x = torch.zeros(2, 40000, dtype=torch.bfloat16, device="cuda")
+    w = torch.ones(40000, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(gpu.GnError) as e:
+        gpu.rmsnorm_bwd(x, w, torch.ones(2, device="cuda"), x)
+    assert e.value.status == gpu.GN_ERR_UNSUPPORTED
+
+
+def test_deterministic_weight_gradients(gpu):
+    d = wl.rmsnorm(M=3000, N=5120, dtype="bf16")
+    x, w, dy = to_dev(d["x"]), to_dev(d["w"]), to_dev(d["dy"])
+    _, r = gpu.rmsnorm_fwd(x, w, d["eps"])
+    a = gpu.rmsnorm_bwd(x, w, r, dy)
+    b = gpu.rmsnorm_bwd(x, w, r, dy)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def _sample_rows(M, outlier_scale, k=48, seed=7):
+    rows = set(np.random.default_rng(seed).choice(M, k, replace=False).tolist())
+    rows |= {0, 1, M - 1}
+    rows |= set(np.nonzero(outlier_scale > 1)[0][:8].tolist())
+    return np.array(sorted(rows))
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("gemma", [False, True])
+def test_rmsnorm_full_size(gpu, gemma):
+    cfg = wl.RMSNORM_MAIN
+    d = wl.rmsnorm(M=cfg["M"], N=cfg["N"], dtype="bf16", gemma=gemma)
+    x, w, dy = to_dev(d["x"]), to_dev(d["w"]), to_dev(d["dy"])
+    y, r = gpu.rmsnorm_fwd(x, w, d["eps"], gemma=gemma)
+    dx, dw = gpu.rmsnorm_bwd(x, w, r, dy, gemma=gemma)
+    torch.cuda.synchronize()
+    rows = _sample_rows(cfg["M"], wl.outlier_rows(0, cfg["M"]))
+    ry, _ = oracle.rmsnorm_fwd(d["x"][rows], d["w"], d["eps"], gemma=gemma)
+    rdx, _ = oracle.rmsnorm_bwd(d["x"][rows], d["w"], d["dy"][rows], d["eps"], gemma=gemma)
+    _, rr = oracle.rmsnorm_fwd(d["x"], d["w"], d["eps"], gemma=gemma)
+    _, rdw = oracle.rmsnorm_bwd(d["x"], d["w"], d["dy"], d["eps"], gemma=gemma, want_dx=False)
+    idx = torch.from_numpy(rows).cuda()
+    assert_close(to_np(y[idx]), ry, "bf16", "full rms y")
+    assert_close(to_np(dx[idx]), rdx, "grad_bf16", "full rms dx")
+    assert_close(to_np(r), rr, "stat", "full rms inv_rms (all rows)")
+    assert_close(to_np(dw), rdw, "grad_bf16", "full rms dw")
+
+
+@pytest.mark.slow
+def test_layernorm_full_size(gpu):
+    cfg = wl.LAYERNORM_MAIN
+    d = wl.layernorm(M=cfg["M"], N=cfg["N"], dtype="bf16")
+    x, w, b, dy = (to_dev(d[k]) for k in ("x", "w", "b", "dy"))
+    y, mu, rs = gpu.layernorm_fwd(x, w, b, d["eps"], epilogue="gelu_tanh")
+    dx, dw, db = gpu.layernorm_bwd(x, w, b, mu, rs, dy, epilogue="gelu_tanh")
+    torch.cuda.synchronize()
+    rows = _sample_rows(cfg["M"], np.ones(cfg["M"]))
+    ry, _, _ = oracle.layernorm_fwd(d["x"][rows], d["w"], d["b"], d["eps"], act="gelu_tanh")
+    rdx, _, _ = oracle.layernorm_bwd(d["x"][rows], d["w"], d["b"], d["dy"][rows], d["eps"], act="gelu_tanh")
+    _, rmu, rrs = oracle.layernorm_fwd(d["x"], d["w"], d["b"], d["eps"], act="gelu_tanh")
+    _, rdw, rdb = oracle.layernorm_bwd(d["x"], d["w"], d["b"], d["dy"], d["eps"], act="gelu_tanh",
+                                       want_dx=False)
+    idx = torch.from_numpy(rows).cuda()
+    assert_close(to_np(y[idx]), ry, "bf16", "full ln y")
+    assert_close(to_np(dx[idx]), rdx, "grad_bf16", "full ln dx")
+    assert_close(to_np(mu), rmu, (1e-5, 1e-6), "full ln mean")
+    assert_close(to_np(rs), rrs, "stat", "full ln rstd")
+    assert_close(to_np(dw), rdw, "grad_bf16", "full ln dw")
+    assert_close(to_np(db), rdb, "grad_bf16", "full ln db")

@@ -1,0 +1,166 @@
+"""GPU parity of the in-place interleaved RoPE and the fused qk-norm + RoPE against the oracle.
+
+Small cases cover several units per CTA and several CTAs, one or two tensors (k may be
+absent), head dims from 8 to 264 (including widths whose lanes per head are not a power of
+two, for the plain rotation), slabs split across heads (the backward stages four tensors),
+and empty inputs. The full-size cases run the benchmark's launch configuration and compare
+sampled tokens, every saved statistic and the complete weight gradients.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from transformer_norm_rope_b200 import workloads as wl
+from tests._util import assert_close, grad_tol, io_tol, to_dev, to_np, wgrad_tol
+
+pytestmark = pytest.mark.gpu
+
+ROPE_SHAPES = [(1, 256, 8, 128, "f32"), (2, 37, 5, 64, "bf16"), (1, 300, 40, 128, "bf16"),
+               (3, 11, 2, 8, "bf16"), (1, 17, 3, 96, "bf16"), (2, 9, 2, 264, "bf16"), (1, 40, 6, 72, "f32")]
+
+
+@pytest.mark.parametrize("B,S,H,D,dtype", ROPE_SHAPES)
+@pytest.mark.parametrize("with_k", [True, False])
+def test_rope_fwd_bwd_in_place(gpu, B, S, H, D, dtype, with_k):
+    d = wl.rope(B=B, S=S, H=H, D=D, dtype=dtype)
+    q, k = to_dev(d["q"]), to_dev(d["k"]) if with_k else None
+    cos, sin = to_dev(d["cos"]), to_dev(d["sin"])
+    gpu.rope_apply_(q, k, cos, sin, +1)
+    torch.cuda.synchronize()
+    tol = io_tol(dtype)
+    assert_close(to_np(q), oracle.rope(d["q"], d["cos"], d["sin"], +1), tol, "rope fwd q")
+    if with_k:
+        assert_close(to_np(k), oracle.rope(d["k"], d["cos"], d["sin"], +1), tol, "rope fwd k")
+    # the backward is the same call with sin negated, applied in place to the gradient
+    qf = q.clone()
+    gpu.rope_apply_(q, k, cos, sin, -1)
+    torch.cuda.synchronize()
+    qf_np = qf.cpu().view(torch.int16).numpy().view(np.uint16) if dtype == "bf16" else qf.cpu().numpy()
+    assert_close(to_np(q), oracle.rope(qf_np, d["cos"], d["sin"], -1), tol, "rope bwd q")
+    # and it undoes the forward up to the output rounding
+    assert_close(to_np(q), wl.bf16_to_f32(d["q"]) if dtype == "bf16" else d["q"], tol, "rope bwd(fwd)")
+
+
+def test_rope_position_zero_is_identity(gpu):
+    d = wl.rope(B=2, S=4, H=3, D=128, dtype="bf16")
+    q = to_dev(d["q"])
+    gpu.rope_apply_(q, None, to_dev(d["cos"]), to_dev(d["sin"]), +1)
+    torch.cuda.synchronize()
+    assert torch.equal(q[:, 0], to_dev(d["q"])[:, 0])  # cos = 1, sin = 0: bit-exact
+
+
+def test_rope_empty(gpu):
+    q = torch.empty(1, 0, 4, 128, dtype=torch.bfloat16, device="cuda")
+    t = torch.empty(0, 64, device="cuda")
+    gpu.rope_apply_(q, None, t, t, +1)
+
+
+QK_SHAPES = [(2, 37, 5, 128, "bf16"), (1, 64, 40, 128, "bf16"), (1, 50, 8, 128, "f32"), (2, 21, 3, 64, "bf16"),
+             (1, 30, 4, 8, "bf16"), (1, 19, 7, 32, "f32")]
+
+
+def _bits(t, dtype):
+    return t.cpu().view(torch.int16).numpy().view(np.uint16) if dtype == "bf16" else t.cpu().numpy()
+
+
+@pytest.mark.parametrize("B,S,H,D,dtype", QK_SHAPES)
+@pytest.mark.parametrize("gemma", [False, True])
+def test_qknorm_rope_fwd_bwd(gpu, B, S, H, D, dtype, gemma):
+    d = wl.qknorm_rope(B=B, S=S, H=H, D=D, dtype=dtype)
+    if gemma:  # Gemma weights sit around 0: w' = 1 + w
+        d["wq"] = wl.normal(0, wl.S_WQ, D, dtype, scale=0.1)
+        d["wk"] = wl.normal(0, wl.S_WK, D, dtype, scale=0.1)
+    q, k, wq, wk = (to_dev(d[n]) for n in ("q", "k", "wq", "wk"))
+    cos, sin = to_dev(d["cos"]), to_dev(d["sin"])
+    qo, ko, rq, rk = gpu.qknorm_rope_fwd(q, k, wq, wk, cos, sin, d["eps"], gemma=gemma)
+    dq, dk, dwq, dwk = gpu.qknorm_rope_bwd(q, k, wq, wk, cos, sin, rq, rk, to_dev(d["dq_out"]),
+                                           to_dev(d["dk_out"]), gemma=gemma)
+    torch.cuda.synchronize()
+    for name, x, w, dy, out, r, dx, dw in (("q", d["q"], d["wq"], d["dq_out"], qo, rq, dq, dwq),
+                                           ("k", d["k"], d["wk"], d["dk_out"], ko, rk, dk, dwk)):
+        ro, rr = oracle.qknorm_rope_fwd(x, w, d["cos"], d["sin"], d["eps"], gemma=gemma)
+        rdx, rdw = oracle.qknorm_rope_bwd(x, w, d["cos"], d["sin"], dy, d["eps"], gemma=gemma)
+        tag = f"qk {name} {dtype} {B}x{S}x{H}x{D} gemma={gemma}"
+        assert_close(to_np(out), ro, io_tol(dtype), tag + " out")
+        assert_close(to_np(r), rr, "stat", tag + " inv_rms")
+        assert_close(to_np(dx), rdx, grad_tol(dtype), tag + " dx")
+        assert_close(to_np(dw), rdw, wgrad_tol(dtype, rdw), tag + " dw")
+
+
+def test_qknorm_rope_without_k(gpu):
+    d = wl.qknorm_rope(B=1, S=33, H=6, D=128, dtype="bf16")
+    q, wq = to_dev(d["q"]), to_dev(d["wq"])
+    cos, sin = to_dev(d["cos"]), to_dev(d["sin"])
+    qo, ko, rq, rk = gpu.qknorm_rope_fwd(q, None, wq, None, cos, sin, d["eps"])
+    dq, dk, dwq, dwk = gpu.qknorm_rope_bwd(q, None, wq, None, cos, sin, rq, None, to_dev(d["dq_out"]), None)
+    torch.cuda.synchronize()
+    assert ko is None and dk is None and dwk is None
+    ro, _ = oracle.qknorm_rope_fwd(d["q"], d["wq"], d["cos"], d["sin"], d["eps"])
+    rdx, rdw = oracle.qknorm_rope_bwd(d["q"], d["wq"], d["cos"], d["sin"], d["dq_out"], d["eps"])
+    assert_close(to_np(qo), ro, "bf16", "q only out")
+    assert_close(to_np(dq), rdx, "grad_bf16", "q only dx")
+    assert_close(to_np(dwq), rdw, "grad_bf16", "q only dw")
+
+
+def test_qknorm_unsupported_head_dim(gpu):
+    q = torch.zeros(1, 2, 2, 96, dtype=torch.bfloat16, device="cuda")
+    w = torch.ones(96, dtype=torch.bfloat16, device="cuda")
+    t = torch.zeros(2, 48, device="cuda")
+    with pytest.raises(gpu.GnError) as e:
+        gpu.qknorm_rope_fwd(q, None, w, None, t, t)
+    assert e.value.status == gpu.GN_ERR_UNSUPPORTED
+
+
+def _sample_tokens(B, S, k=24, seed=11):
+    rng = np.random.default_rng(seed)
+    toks = {(0, 0), (B - 1, S - 1), (0, 1)}
+    toks |= {(int(b), int(s)) for b, s in zip(rng.integers(0, B, k), rng.integers(0, S, k))}
+    return sorted(toks)
+
+
+@pytest.mark.slow
+def test_rope_full_size(gpu):
+    c = wl.ROPE_MAIN
+    d = wl.rope(**c)
+    q, k = to_dev(d["q"]), to_dev(d["k"])
+    cos, sin = to_dev(d["cos"]), to_dev(d["sin"])
+    gpu.rope_apply_(q, k, cos, sin, +1)
+    torch.cuda.synchronize()
+    for b, s in _sample_tokens(c["B"], c["S"]):
+        for name, t in (("q", q), ("k", k)):
+            ref = oracle.rope(d[name][b:b + 1, s:s + 1], d["cos"][s:s + 1], d["sin"][s:s + 1], +1)
+            assert_close(to_np(t[b:b + 1, s:s + 1]), ref, "bf16", f"full rope {name} token {b},{s}")
+    # the backward call restores every element to within the output rounding
+    gpu.rope_apply_(q, k, cos, sin, -1)
+    torch.cuda.synchronize()
+    for name, t in (("q", q), ("k", k)):
+        diff = (t.float() - to_dev(d[name]).float()).abs()
+        bound = 1.6e-2 * to_dev(d[name]).float().abs() + 1e-2
+        assert bool((diff <= bound).all()), f"full rope bwd(fwd) {name}"
+
+
+@pytest.mark.slow
+def test_qknorm_rope_full_size(gpu):
+    c = wl.QKNORM_MAIN
+    d = wl.qknorm_rope(**c)
+    q, k, wq, wk = (to_dev(d[n]) for n in ("q", "k", "wq", "wk"))
+    cos, sin = to_dev(d["cos"]), to_dev(d["sin"])
+    qo, ko, rq, rk = gpu.qknorm_rope_fwd(q, k, wq, wk, cos, sin, d["eps"])
+    dq, dk, dwq, dwk = gpu.qknorm_rope_bwd(q, k, wq, wk, cos, sin, rq, rk, to_dev(d["dq_out"]), to_dev(d["dk_out"]))
+    torch.cuda.synchronize()
+    for name, x, w, dy, out, r, dx, dw in (("q", "q", "wq", "dq_out", qo, rq, dq, dwq),
+                                           ("k", "k", "wk", "dk_out", ko, rk, dk, dwk)):
+        for b, s in _sample_tokens(c["B"], c["S"]):
+            xs = d[x][b:b + 1, s:s + 1]
+            ro, rr = oracle.qknorm_rope_fwd(xs, d[w], d["cos"][s:s + 1], d["sin"][s:s + 1], d["eps"])
+            rdx, _ = oracle.qknorm_rope_bwd(xs, d[w], d["cos"][s:s + 1], d["sin"][s:s + 1], d[dy][b:b + 1, s:s + 1],
+                                            d["eps"])
+            tag = f"full qk {name} token {b},{s}"
+            assert_close(to_np(out[b:b + 1, s:s + 1]), ro, "bf16", tag + " out")
+            assert_close(to_np(r[b:b + 1, s:s + 1]), rr, "stat", tag + " inv_rms")
+            assert_close(to_np(dx[b:b + 1, s:s + 1]), rdx, "grad_bf16", tag + " dx")
+        _, rr_all = oracle.qknorm_rope_fwd(d[x], d[w], d["cos"], d["sin"], d["eps"], want_out=False)
+        assert_close(to_np(r), rr_all, "stat", f"full qk {name} inv_rms (all rows)")
+        _, rdw = oracle.qknorm_rope_bwd(d[x], d[w], d["cos"], d["sin"], d[dy], d["eps"], want_dx=False)
+        assert_close(to_np(dw), rdw, "grad_bf16", f"full qk {name} dw")

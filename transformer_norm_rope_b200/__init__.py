@@ -1,0 +1,282 @@
+"""Python binding of libgn: fused row normalization and interleaved RoPE on B200 (sm_100a).
+
+Two layers, both argument marshalling only (every step of the computation runs in the CUDA
+kernels of ``libgn.so``):
+
+* ``gn_*`` functions with the names and argument lists of the C ABI in ``include/gn.h``
+  (pointers as Python ints, ``stream`` as an int handle). They return the ``gn_status`` code.
+* torch-tensor helpers (``rmsnorm_fwd``, ``rope_apply_``, ...) that allocate outputs with
+  torch, pass ``data_ptr()`` values and the current CUDA stream, and raise ``GnError`` on a
+  non-zero status.
+
+There is no fallback: if ``libgn.so`` is missing or cannot be loaded, every call raises.
+Build it with ``python -m transformer_norm_rope_b200._build``.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgn.so")
+
+GN_OK, GN_ERR_NULL, GN_ERR_SHAPE, GN_ERR_ALIGN, GN_ERR_DTYPE, GN_ERR_WORKSPACE, \
+    GN_ERR_UNSUPPORTED, GN_ERR_CUDA = range(8)
+GN_F32, GN_BF16 = 0, 1
+GN_EPI_NONE, GN_EPI_GELU_TANH, GN_EPI_SILU = 0, 1, 2
+GN_DEVERR_WAIT_TIMEOUT = 1
+EPILOGUES = {"none": GN_EPI_NONE, "gelu_tanh": GN_EPI_GELU_TANH, "silu": GN_EPI_SILU}
+
+_vp, _i64, _f32, _int, _sz = C.c_void_p, C.c_int64, C.c_float, C.c_int, C.c_size_t
+_st = C.c_int
+
+# name -> (restype, argtypes), in the order of include/gn.h
+SIGNATURES = {
+    "gn_status_string": (C.c_char_p, [_st]),
+    "gn_rmsnorm_fwd": (_st, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _f32, _int, _int, _int, _vp]),
+    "gn_rmsnorm_bwd_workspace": (_sz, [_i64, _i64, _int]),
+    "gn_rmsnorm_bwd": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _i64, _i64, _i64, _i64, _i64,
+                             _int, _int, _int, _vp]),
+    "gn_layernorm_fwd": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _f32, _int, _int,
+                               _vp]),
+    "gn_layernorm_bwd_workspace": (_sz, [_i64, _i64, _int]),
+    "gn_layernorm_bwd": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _i64, _i64, _i64,
+                               _i64, _i64, _int, _int, _vp]),
+    "gn_rope_apply_inplace": (_st, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _int, _int, _vp]),
+    "gn_qknorm_rope_fwd": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
+                                 _i64, _f32, _int, _int, _vp]),
+    "gn_qknorm_rope_bwd_workspace": (_sz, [_i64, _i64, _i64, _i64, _int]),
+    "gn_qknorm_rope_bwd": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                 _vp, _sz, _i64, _i64, _i64, _i64, _int, _int, _vp]),
+    "gn_launch_count": (C.c_uint64, []),
+    "gn_device_error": (_st, [C.POINTER(C.c_uint), _int]),
+    "gn_tune": (_st, [C.c_char_p, _int]),
+}
+
+_lib = None
+
+
+class GnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+def load():
+    """Load libgn.so (once). Raises if it is missing: there is no fallback path."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing; build it with "
+                               "`python -m transformer_norm_rope_b200._build`")
+        lib = C.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(lib, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def _c(name):
+    def call(*args):
+        return getattr(load(), name)(*args)
+
+    call.__name__ = name
+    call.__doc__ = f"Direct call of the C entry point {name} (see include/gn.h)."
+    return call
+
+
+for _name in SIGNATURES:
+    globals()[_name] = _c(_name)
+del _name
+
+
+def status_string(status: int) -> str:
+    try:
+        return load().gn_status_string(status).decode()
+    except Exception:  # noqa: BLE001 - message helper must not mask the original error
+        return f"gn_status {status}"
+
+
+def check(status: int, where: str = "libgn") -> None:
+    if status != GN_OK:
+        raise GnError(status, where)
+
+
+# ---------------------------------------------------------------- torch helpers
+
+def _torch():
+    import torch
+
+    return torch
+
+
+def _dt(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return GN_BF16
+    if t.dtype == torch.float32:
+        return GN_F32
+    raise TypeError(f"unsupported dtype {t.dtype} (bfloat16 or float32)")
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream=None) -> int:
+    torch = _torch()
+    return (stream or torch.cuda.current_stream()).cuda_stream
+
+
+def _epi(epi) -> int:
+    return EPILOGUES[epi] if isinstance(epi, str) else int(epi)
+
+
+def _rows(x):
+    """(rows, hidden, ld) of a tensor whose last dim is contiguous and whose leading dims
+    collapse to one row stride."""
+    if x.dim() < 1 or x.stride(-1) != 1:
+        raise ValueError("last dimension must be contiguous")
+    hidden = x.shape[-1]
+    x2 = x.reshape(-1, hidden) if x.dim() != 2 else x
+    if x2.data_ptr() != x.data_ptr():
+        raise ValueError("rows of x must form one strided matrix")
+    ld = x2.stride(0) if x2.shape[0] > 1 else hidden
+    return x2.shape[0], hidden, ld
+
+
+def empty_rows(shape, dtype, device):
+    """Uninitialised tensor of `shape` whose rows start on 16-byte boundaries: the row stride
+    is the last dimension rounded up to 16 bytes (a strided view when that adds padding)."""
+    torch = _torch()
+    shape = tuple(shape)
+    hidden = shape[-1]
+    es = torch.empty((), dtype=dtype).element_size()
+    ld = (hidden * es + 15) // 16 * 16 // es
+    rows = 1
+    for n in shape[:-1]:
+        rows *= n
+    strides, acc = [1], ld
+    for n in reversed(shape[:-1]):
+        strides.insert(0, acc)
+        acc *= n
+    base = torch.empty(rows * ld, dtype=dtype, device=device)
+    return base.as_strided(shape, strides)
+
+
+def rmsnorm_fwd(x, w, eps=1e-6, gemma=False, epilogue="none", out=None, save_stats=True, stream=None):
+    """y = epi(x * rsqrt(mean(x^2) + eps) * w') -> (y, inv_rms[rows] fp32 or None)."""
+    torch = _torch()
+    rows, hidden, ld = _rows(x)
+    y = empty_rows(x.shape, x.dtype, x.device) if out is None else out
+    _, _, ldy = _rows(y)
+    r = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device) if save_stats else None
+    check(gn_rmsnorm_fwd(_ptr(x), _ptr(w), _ptr(y), _ptr(r), rows, hidden, ld, ldy, eps, int(gemma),
+                         _epi(epilogue), _dt(x), _stream(stream)), "gn_rmsnorm_fwd")
+    return y, r
+
+
+def rmsnorm_bwd(x, w, inv_rms, dy, gemma=False, epilogue="none", want_dw=True, stream=None):
+    """-> (dx, dw fp32 or None)."""
+    torch = _torch()
+    rows, hidden, ld = _rows(x)
+    _, _, lddy = _rows(dy)
+    dx = empty_rows(x.shape, x.dtype, x.device)
+    _, _, lddx = _rows(dx)
+    dw = torch.empty(hidden, dtype=torch.float32, device=x.device) if want_dw else None
+    nws = gn_rmsnorm_bwd_workspace(rows, hidden, _dt(x)) if want_dw else 0
+    ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=x.device) if want_dw else None
+    check(gn_rmsnorm_bwd(_ptr(x), _ptr(w), _ptr(inv_rms), _ptr(dy), _ptr(dx), _ptr(dw), _ptr(ws), nws,
+                         rows, hidden, ld, lddy, lddx, int(gemma), _epi(epilogue), _dt(x),
+                         _stream(stream)), "gn_rmsnorm_bwd")
+    return dx, dw
+
+
+def layernorm_fwd(x, w=None, b=None, eps=1e-5, epilogue="none", out=None, save_stats=True, stream=None):
+    """y = epi((x - mean) * rstd * w + b) -> (y, mean, rstd)."""
+    torch = _torch()
+    rows, hidden, ld = _rows(x)
+    y = empty_rows(x.shape, x.dtype, x.device) if out is None else out
+    _, _, ldy = _rows(y)
+    mk = (lambda: torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device))
+    mu, rs = (mk(), mk()) if save_stats else (None, None)
+    check(gn_layernorm_fwd(_ptr(x), _ptr(w), _ptr(b), _ptr(y), _ptr(mu), _ptr(rs), rows, hidden, ld, ldy,
+                           eps, _epi(epilogue), _dt(x), _stream(stream)), "gn_layernorm_fwd")
+    return y, mu, rs
+
+
+def layernorm_bwd(x, w, b, mean, rstd, dy, epilogue="none", want_wgrad=True, stream=None):
+    """-> (dx, dw, db) (dw, db fp32 or None)."""
+    torch = _torch()
+    rows, hidden, ld = _rows(x)
+    _, _, lddy = _rows(dy)
+    dx = empty_rows(x.shape, x.dtype, x.device)
+    _, _, lddx = _rows(dx)
+    mk = (lambda: torch.empty(hidden, dtype=torch.float32, device=x.device))
+    dw, db = (mk(), mk()) if want_wgrad else (None, None)
+    nws = gn_layernorm_bwd_workspace(rows, hidden, _dt(x)) if want_wgrad else 0
+    ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=x.device) if want_wgrad else None
+    check(gn_layernorm_bwd(_ptr(x), _ptr(w), _ptr(b), _ptr(mean), _ptr(rstd), _ptr(dy), _ptr(dx), _ptr(dw),
+                           _ptr(db), _ptr(ws), nws, rows, hidden, ld, lddy, lddx, _epi(epilogue), _dt(x),
+                           _stream(stream)), "gn_layernorm_bwd")
+    return dx, dw, db
+
+
+def _bshd(q):
+    if q.dim() != 4 or not q.is_contiguous():
+        raise ValueError("rotary tensors must be contiguous [B, S, H, D]")
+    return q.shape
+
+
+def rope_apply_(q, k, cos, sin, sign=+1, stream=None):
+    """In-place interleaved RoPE of q (and k, may be None); sign=-1 is the backward."""
+    B, S, H, D = _bshd(q)
+    if k is not None and k.shape != q.shape:
+        raise ValueError("q and k must have the same shape")
+    check(gn_rope_apply_inplace(_ptr(q), _ptr(k), _ptr(cos), _ptr(sin), B, S, H, D, int(sign), _dt(q),
+                                _stream(stream)), "gn_rope_apply_inplace")
+    return q, k
+
+
+def qknorm_rope_fwd(q, k, wq, wk, cos, sin, eps=1e-6, gemma=False, stream=None):
+    """-> (q_out, k_out, inv_rms_q, inv_rms_k); k may be None."""
+    torch = _torch()
+    B, S, H, D = _bshd(q)
+    qo = torch.empty_like(q)
+    ko = torch.empty_like(k) if k is not None else None
+    rq = torch.empty((B, S, H), dtype=torch.float32, device=q.device)
+    rk = torch.empty((B, S, H), dtype=torch.float32, device=q.device) if k is not None else None
+    check(gn_qknorm_rope_fwd(_ptr(q), _ptr(k), _ptr(wq), _ptr(wk), _ptr(cos), _ptr(sin), _ptr(qo), _ptr(ko),
+                             _ptr(rq), _ptr(rk), B, S, H, D, eps, int(gemma), _dt(q), _stream(stream)),
+          "gn_qknorm_rope_fwd")
+    return qo, ko, rq, rk
+
+
+def qknorm_rope_bwd(q, k, wq, wk, cos, sin, inv_rms_q, inv_rms_k, dq_out, dk_out, gemma=False,
+                    want_dw=True, stream=None):
+    """-> (dq, dk, dwq, dwk)."""
+    torch = _torch()
+    B, S, H, D = _bshd(q)
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k) if k is not None else None
+    dwq = torch.empty(D, dtype=torch.float32, device=q.device) if want_dw else None
+    dwk = torch.empty(D, dtype=torch.float32, device=q.device) if (want_dw and k is not None) else None
+    nws = gn_qknorm_rope_bwd_workspace(B, S, H, D, _dt(q)) if want_dw else 0
+    ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=q.device) if want_dw else None
+    check(gn_qknorm_rope_bwd(_ptr(q), _ptr(k), _ptr(wq), _ptr(wk), _ptr(cos), _ptr(sin), _ptr(inv_rms_q),
+                             _ptr(inv_rms_k), _ptr(dq_out), _ptr(dk_out), _ptr(dq), _ptr(dk), _ptr(dwq),
+                             _ptr(dwk), _ptr(ws), nws, B, S, H, D, int(gemma), _dt(q), _stream(stream)),
+          "gn_qknorm_rope_bwd")
+    return dq, dk, dwq, dwk
+
+
+def device_error(clear: bool = False) -> int:
+    w = C.c_uint(0)
+    check(gn_device_error(C.byref(w), int(clear)), "gn_device_error")
+    return w.value
+
+
+def tune(key: str, value: int) -> None:
+    check(gn_tune(key.encode(), int(value)), "gn_tune")

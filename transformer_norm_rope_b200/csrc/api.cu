@@ -1,0 +1,174 @@
+// api.cu - runtime pieces of libgn shared by all entry points: status strings, the launch
+// counter, the device error word, device property caches, the tuning knobs and the
+// deterministic column reduction that finishes every weight gradient.
+#include <atomic>
+#include <cstring>
+#include <mutex>
+
+#include "gn_host.h"
+
+namespace gn {
+
+Tuning g_tune = {0, 0, 0, 0, 0};
+
+static std::atomic<uint64_t> g_launches{0};
+
+void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+// One error word per device. Kernels receive its address as an argument.
+__device__ unsigned g_device_error_word;
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+unsigned* g_err_ptr[kMaxDevices];
+int g_sms[kMaxDevices];
+size_t g_smem[kMaxDevices];
+
+int current_device() {
+  int d = -1;
+  if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= kMaxDevices) return -1;
+  return d;
+}
+}  // namespace
+
+unsigned* device_err_word() {
+  const int d = current_device();
+  if (d < 0) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_err_ptr[d]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error_word) != cudaSuccess) return nullptr;
+    g_err_ptr[d] = static_cast<unsigned*>(p);
+  }
+  return g_err_ptr[d];
+}
+
+int sm_count() {
+  const int d = current_device();
+  if (d < 0) return 0;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_sms[d]) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, d) != cudaSuccess) return 0;
+    g_sms[d] = v;
+  }
+  return g_sms[d];
+}
+
+size_t smem_optin() {
+  const int d = current_device();
+  if (d < 0) return 0;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_smem[d]) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, d) != cudaSuccess) return 0;
+    g_smem[d] = (size_t)v;
+  }
+  return g_smem[d];
+}
+
+gn_status launch_status() { return cudaGetLastError() == cudaSuccess ? GN_OK : GN_ERR_CUDA; }
+
+int persistent_grid(const void* kernel, int threads, size_t smem, int cap) {
+  const int sms = sm_count();
+  if (sms <= 0) return 0;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return 0;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) != cudaSuccess) return 0;
+  if (per_sm <= 0) return 0;
+  if (cap > 0 && per_sm > cap) per_sm = cap;
+  return per_sm * sms;
+}
+
+// ---------------------------------------------------------------- column reduction
+// Block = 32 columns x 8 slices of the partial rows. Slice k sums rows g = k, k+8, ... in
+// order, then slice 0 adds the 8 slice sums in order: a fixed order for a given G, so the
+// result is the same on every run.
+__global__ void __launch_bounds__(256) colsum_kernel(const float* __restrict__ ws, int64_t G,
+                                                     int64_t ncols, int64_t split,
+                                                     float* __restrict__ out0,
+                                                     float* __restrict__ out1) {
+  __shared__ float part[8][33];
+  const int cl = threadIdx.x & 31, sl = threadIdx.x >> 5;
+  const int64_t c = (int64_t)blockIdx.x * 32 + cl;
+  float acc = 0.f;
+  if (c < ncols) {
+#pragma unroll 4
+    for (int64_t g = sl; g < G; g += 8) acc += ws[g * ncols + c];
+  }
+  part[sl][cl] = acc;
+  __syncthreads();
+  if (sl == 0 && c < ncols) {
+    float t = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) t += part[k][cl];
+    if (c < split) {
+      if (out0) out0[c] = t;
+    } else if (out1) {
+      out1[c - split] = t;
+    }
+  }
+}
+
+gn_status launch_colsum(const float* ws, int64_t G, int64_t ncols, int64_t split, float* out0,
+                        float* out1, cudaStream_t s) {
+  if (!out0 && !out1) return GN_OK;
+  const int64_t blocks = (ncols + 31) / 32;
+  colsum_kernel<<<(unsigned)blocks, 256, 0, s>>>(ws, G, ncols, split, out0, out1);
+  count_launches(1);
+  return launch_status();
+}
+
+}  // namespace gn
+
+using namespace gn;
+
+extern "C" const char* gn_status_string(gn_status s) {
+  switch (s) {
+    case GN_OK: return "GN_OK";
+    case GN_ERR_NULL: return "GN_ERR_NULL: a required pointer is NULL";
+    case GN_ERR_SHAPE: return "GN_ERR_SHAPE: invalid size, stride or sign";
+    case GN_ERR_ALIGN: return "GN_ERR_ALIGN: pointer or row stride not 16-byte aligned";
+    case GN_ERR_DTYPE: return "GN_ERR_DTYPE: unknown dtype or epilogue";
+    case GN_ERR_WORKSPACE: return "GN_ERR_WORKSPACE: workspace missing or too small";
+    case GN_ERR_UNSUPPORTED: return "GN_ERR_UNSUPPORTED: row does not fit the kernel";
+    case GN_ERR_CUDA: return "GN_ERR_CUDA: CUDA runtime error";
+  }
+  return "unknown gn_status";
+}
+
+extern "C" uint64_t gn_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+extern "C" gn_status gn_device_error(unsigned* word, int clear) {
+  if (!word) return GN_ERR_NULL;
+  unsigned* p = device_err_word();
+  if (!p) return GN_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return GN_ERR_CUDA;
+  if (cudaMemcpy(word, p, sizeof(unsigned), cudaMemcpyDeviceToHost) != cudaSuccess) return GN_ERR_CUDA;
+  if (clear && cudaMemset(p, 0, sizeof(unsigned)) != cudaSuccess) return GN_ERR_CUDA;
+  if (clear && cudaDeviceSynchronize() != cudaSuccess) return GN_ERR_CUDA;
+  return GN_OK;
+}
+
+extern "C" gn_status gn_tune(const char* key, int value) {
+  if (!key || value < 0) return GN_ERR_SHAPE;
+  if (!strcmp(key, "stages")) {
+    if (value > 16) return GN_ERR_SHAPE;
+    g_tune.stages = value;
+  } else if (!strcmp(key, "ctas_per_sm")) {
+    g_tune.ctas_per_sm = value;
+  } else if (!strcmp(key, "vpt")) {
+    if (value != 0 && value != 1 && value != 2 && value != 4 && value != 8) return GN_ERR_SHAPE;
+    g_tune.vpt = value;
+  } else if (!strcmp(key, "unit_bytes")) {
+    g_tune.unit_bytes = value;
+  } else if (!strcmp(key, "group_rows")) {
+    g_tune.group_rows = value;
+  } else {
+    return GN_ERR_SHAPE;
+  }
+  return GN_OK;
+}

@@ -1,0 +1,215 @@
+// gn_common.cuh - device building blocks shared by the sm_100a kernels of libgn.
+//
+// * 16-byte vector I/O: 8 bf16 or 4 fp32 per access, widened to fp32 in registers.
+// * 1-D TMA bulk copies (cp.async.bulk global -> shared, completion counted on an mbarrier)
+//   for the row pipeline, with a bounded wait: a wait that runs past kWaitLimitNs records
+//   the wait-timeout bit in the caller's error word and returns false instead of spinning.
+// * warp reductions and the tanh-GeLU / SiLU epilogues with their derivatives.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gn {
+
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s: far above any real copy latency
+constexpr unsigned kDevErrWaitTimeout = 1u;  // GN_DEVERR_WAIT_TIMEOUT in gn.h
+
+// ---------------------------------------------------------------- element traits
+
+template <typename T>
+struct Vec;
+
+template <>
+struct Vec<float> {
+  static constexpr int N = 4;  // elements per 16-byte vector
+  __device__ __forceinline__ static void unpack(const uint4& u, float (&f)[4]) {
+    f[0] = __uint_as_float(u.x);
+    f[1] = __uint_as_float(u.y);
+    f[2] = __uint_as_float(u.z);
+    f[3] = __uint_as_float(u.w);
+  }
+  __device__ __forceinline__ static uint4 pack(const float (&f)[4]) {
+    return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                      __float_as_uint(f[3]));
+  }
+  __device__ __forceinline__ static float load1(const float* p) { return *p; }
+  __device__ __forceinline__ static void store1(float* p, float v) { *p = v; }
+};
+
+template <>
+struct Vec<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ __forceinline__ static void split(uint32_t w, float& lo, float& hi) {
+    lo = __uint_as_float(w << 16);
+    hi = __uint_as_float(w & 0xffff0000u);
+  }
+  __device__ __forceinline__ static void unpack(const uint4& u, float (&f)[8]) {
+    split(u.x, f[0], f[1]);
+    split(u.y, f[2], f[3]);
+    split(u.z, f[4], f[5]);
+    split(u.w, f[6], f[7]);
+  }
+  __device__ __forceinline__ static uint32_t join(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // round to nearest even, both halves
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+  __device__ __forceinline__ static uint4 pack(const float (&f)[8]) {
+    return make_uint4(join(f[0], f[1]), join(f[2], f[3]), join(f[4], f[5]), join(f[6], f[7]));
+  }
+  __device__ __forceinline__ static float load1(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+  __device__ __forceinline__ static void store1(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
+};
+
+// streaming 16-byte global access (read-once / write-once data)
+__device__ __forceinline__ uint4 ld_stream(const void* p) { return __ldcs(reinterpret_cast<const uint4*>(p)); }
+__device__ __forceinline__ void st_stream(void* p, const uint4& v) { __stcs(reinterpret_cast<uint4*>(p), v); }
+
+// element i of a weight vector, widened (w == nullptr -> dflt)
+template <typename T>
+__device__ __forceinline__ float ld_param(const T* w, int64_t i, float dflt) {
+  return w ? Vec<T>::load1(w + i) : dflt;
+}
+
+// ---------------------------------------------------------------- mbarrier + bulk copy
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+// make the initialised barriers visible to the async (TMA) proxy; call before __syncthreads
+__device__ __forceinline__ void mbar_fence_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for phase `parity` of `bar` to complete, for at most kWaitLimitNs. On timeout the
+// error word gets GN_DEVERR_WAIT_TIMEOUT and the function returns false.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (err) atomicOr(err, kDevErrWaitTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
+// 1-D bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned) from global to
+// this CTA's shared memory; completion is counted on `bar` as transaction bytes.
+__device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_addr(dst_smem)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// ---------------------------------------------------------------- reductions
+
+template <int WIDTH = 32>
+__device__ __forceinline__ float group_sum(float v) {
+#pragma unroll
+  for (int o = WIDTH / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o, WIDTH);
+  return v;
+}
+
+// runtime-width variant (width a power of two <= 32); every lane gets the same total
+__device__ __forceinline__ float group_sum_rt(float v, int width) {
+  for (int o = width / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o, width);
+  return v;
+}
+
+// ---------------------------------------------------------------- epilogues
+// tanh-GeLU: 0.5 z (1 + tanh(k (z + 0.044715 z^3))), k = sqrt(2/pi). SiLU: z * sigmoid(z).
+// bf16 outputs use the hardware tanh.approx / ex2-based __expf (error far below bf16
+// rounding); fp32 outputs use the accurate tanhf / expf.
+
+enum Epi { EPI_NONE = 0, EPI_GELU_TANH = 1, EPI_SILU = 2 };
+
+constexpr float kGeluK = 0.7978845608028654f;  // sqrt(2/pi)
+constexpr float kGeluC = 0.044715f;
+
+template <bool FAST>
+__device__ __forceinline__ float tanh_f(float x) {
+  if constexpr (FAST) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+  } else {
+    return tanhf(x);
+  }
+}
+
+template <bool FAST>
+__device__ __forceinline__ float sigmoid_f(float x) {
+  if constexpr (FAST) {
+    return __frcp_rn(1.0f + __expf(-x));
+  } else {
+    return 1.0f / (1.0f + expf(-x));
+  }
+}
+
+template <int EPI, bool FAST>
+__device__ __forceinline__ float epi_fwd(float z) {
+  if constexpr (EPI == EPI_GELU_TANH) {
+    const float t = tanh_f<FAST>(kGeluK * fmaf(kGeluC * z, z * z, z));
+    return 0.5f * z * (1.0f + t);
+  } else if constexpr (EPI == EPI_SILU) {
+    return z * sigmoid_f<FAST>(z);
+  } else {
+    return z;
+  }
+}
+
+// d epi / dz
+template <int EPI, bool FAST>
+__device__ __forceinline__ float epi_grad(float z) {
+  if constexpr (EPI == EPI_GELU_TANH) {
+    const float z2 = z * z;
+    const float t = tanh_f<FAST>(kGeluK * fmaf(kGeluC * z, z2, z));
+    return 0.5f * (1.0f + t) + 0.5f * z * (1.0f - t * t) * kGeluK * fmaf(3.0f * kGeluC, z2, 1.0f);
+  } else if constexpr (EPI == EPI_SILU) {
+    const float s = sigmoid_f<FAST>(z);
+    return s * fmaf(z, 1.0f - s, 1.0f);
+  } else {
+    return 1.0f;
+  }
+}
+
+template <typename T>
+constexpr bool fast_math_for() {
+  return sizeof(T) == 2;  // bf16 I/O
+}
+
+}  // namespace gn

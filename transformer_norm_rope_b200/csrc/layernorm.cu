@@ -1,0 +1,658 @@
+// layernorm.cu - LayerNorm forward and backward with an optional tanh-GeLU or SiLU epilogue
+// (Helios kernels article, section "内核一 FlashNorm": mean, variance and scaling in one
+// memory pass per row, statistics saved for the backward; "LLM层的优化算子", section
+// "编写定制融合算子": centre, biased variance, divide by sqrt(var + eps), times weight plus
+// bias, tanh-GeLU in the same kernel; Janus-Pro-7B article section 4.1: SiLU epilogue).
+//
+//   forward : mu = mean(x), var = mean((x - mu)^2), s = rsqrt(var + eps),
+//             y = epi((x - mu) s w + b), mean = mu, rstd = s
+//   backward: xhat = (x - mu) s, g = dy epi'(xhat w + b),
+//             dx = s (g w - mean(g w) - xhat mean(g w xhat)), dw = sum g xhat, db = sum g
+//
+// The row is read from HBM once and kept in registers, so the variance is taken around the
+// mean (no E[x^2] - E[x]^2 cancellation): every thread forms (count, mean, M2) of its own
+// elements in two register passes, and the triples are combined with Chan et al.'s pairwise
+// update (warp tree, then the per-warp results in warp order after one CTA barrier).
+#include "norm_plan.h"
+
+namespace gn {
+namespace {
+
+struct LnFwdArgs {
+  const void* x;
+  const void* w;
+  const void* b;
+  void* y;
+  float* mean;
+  float* rstd;
+  int64_t rows;
+  int64_t ldx, ldy;
+  int N;
+  float eps;
+  int stages;
+  unsigned* err;
+};
+
+struct LnBwdArgs {
+  const void* x;
+  const void* w;
+  const void* b;
+  const float* mean;
+  const float* rstd;
+  const void* dy;
+  void* dx;
+  float* ws;  // [gridDim.x, 2N]: dw partials then db partials, or null
+  int64_t rows;
+  int64_t ldx, lddy, lddx;
+  int N;
+  int stages;
+  unsigned* err;
+};
+
+// Chan et al. pairwise combination of (count, mean, M2) summaries.
+__device__ __forceinline__ void chan_merge(float& n, float& m, float& M2, float nb, float mb, float M2b) {
+  if (nb == 0.0f) return;
+  if (n == 0.0f) {
+    n = nb;
+    m = mb;
+    M2 = M2b;
+    return;
+  }
+  const float nn = n + nb;
+  const float d = mb - m;
+  const float f = nb / nn;
+  m = fmaf(d, f, m);
+  M2 = M2 + M2b + d * d * n * f;
+  n = nn;
+}
+
+// Summary of this thread's elements of the row: xv[j][0..E) valid for the first cnt[j].
+template <int VPT, int E>
+__device__ __forceinline__ void thread_stats(const float (&xv)[VPT][E], const int (&cnt)[VPT], float& n,
+                                             float& m, float& M2) {
+  float s = 0.0f;
+  int c = 0;
+#pragma unroll
+  for (int j = 0; j < VPT; ++j) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) s += xv[j][e];  // invalid elements are 0
+    c += cnt[j];
+  }
+  n = (float)c;
+  m = c ? s / (float)c : 0.0f;
+  float q = 0.0f;
+#pragma unroll
+  for (int j = 0; j < VPT; ++j)
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const float d = xv[j][e] - m;
+      q = e < cnt[j] ? fmaf(d, d, q) : q;
+    }
+  M2 = q;
+}
+
+// tree-combine the summaries of a group of `width` lanes into its first lane
+__device__ __forceinline__ void group_stats(float& n, float& m, float& M2, int width) {
+  const int li = threadIdx.x & (width - 1);
+  for (int off = width / 2; off > 0; off >>= 1) {
+    const float nb = __shfl_down_sync(0xffffffffu, n, off, width);
+    const float mb = __shfl_down_sync(0xffffffffu, m, off, width);
+    const float qb = __shfl_down_sync(0xffffffffu, M2, off, width);
+    if (li < off) chan_merge(n, m, M2, nb, mb, qb);
+  }
+}
+
+template <typename T, int VPT>
+__device__ __forceinline__ void load_affine(const LnFwdArgs& a, int base, int stride, float (&wr)[VPT][Vec<T>::N],
+                                            float (&br)[VPT][Vec<T>::N]) {
+  constexpr int E = Vec<T>::N;
+#pragma unroll
+  for (int j = 0; j < VPT; ++j)
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int col = (base + j * stride) * E + e;
+      const bool in = col < a.N;
+      wr[j][e] = in ? ld_param(static_cast<const T*>(a.w), col, 1.0f) : 0.0f;
+      br[j][e] = in ? ld_param(static_cast<const T*>(a.b), col, 0.0f) : 0.0f;
+    }
+}
+
+// ---------------------------------------------------------------- CTA path
+
+template <typename T, int VPT, int EPI>
+__global__ void __launch_bounds__(norm_max_threads(VPT)) ln_fwd_cta(const LnFwdArgs a) {
+  using V = Vec<T>;
+  constexpr int E = V::N;
+  constexpr bool FAST = fast_math_for<T>();
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int tid = threadIdx.x, NT = blockDim.x, lane = tid & 31, warp = tid >> 5;
+  const int nwarps = NT >> 5;
+  const int N = a.N, nfull = N / E, nvec = (N + E - 1) / E;
+  const RowPipe pipe(smem, a.stages, 1, (int64_t)N * sizeof(T));
+  const int64_t step = gridDim.x;
+  const T* x = static_cast<const T*>(a.x);
+  T* y = static_cast<T*>(a.y);
+
+  if (tid == 0) pipe.init();
+  __syncthreads();
+  if (tid == 0) {
+    int64_t m = blockIdx.x;
+    for (int s = 0; s < a.stages && m < a.rows; ++s, m += step) pipe.issue(s, x + m * a.ldx);
+  }
+  float wr[VPT][E], br[VPT][E];
+  load_affine<T, VPT>(a, tid, NT, wr, br);
+  int cnt[VPT];
+#pragma unroll
+  for (int j = 0; j < VPT; ++j) {
+    const int left = N - (tid + j * NT) * E;
+    cnt[j] = left <= 0 ? 0 : left >= E ? E : left;
+  }
+  const float inv_n = 1.0f / (float)N;
+
+  int s = 0;
+  uint32_t ph = 0, rb = 0;
+  const int64_t ahead = (int64_t)a.stages * step;
+  for (int64_t m = blockIdx.x; m < a.rows; m += step) {
+    const T* xrow = x + m * a.ldx;
+    const bool ok = pipe.wait(s, ph, a.err);
+    const uint8_t* st = pipe.at(s, 0);
+    float xv[VPT][E];
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      const int v = tid + j * NT;
+      if (v < nfull) {
+        V::unpack(*reinterpret_cast<const uint4*>(st + (size_t)v * 16), xv[j]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) xv[j][e] = e < cnt[j] ? V::load1(xrow + v * E + e) : 0.0f;
+      }
+    }
+    float n, mu, M2;
+    thread_stats<VPT, E>(xv, cnt, n, mu, M2);
+    group_stats(n, mu, M2, 32);
+    float4* red = pipe.red + rb * 32;
+    if (lane == 0) red[warp] = make_float4(n, mu, M2, 0.0f);
+    if (__syncthreads_or(!ok)) {
+      if (tid == 0) pipe.drain(m, step, a.rows, s, ph, a.err);
+      return;
+    }
+    if (tid == 0 && m + ahead < a.rows) pipe.issue(s, x + (m + ahead) * a.ldx);
+    rb ^= 1u;
+    if (++s == a.stages) {
+      s = 0;
+      ph ^= 1u;
+    }
+    n = 0.0f, mu = 0.0f, M2 = 0.0f;
+    for (int w = 0; w < nwarps; ++w) {
+      const float4 r = red[w];
+      chan_merge(n, mu, M2, r.x, r.y, r.z);
+    }
+    const float rs = rsqrtf(fmaf(M2, inv_n, a.eps));
+    T* yrow = y + m * a.ldy;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      const int v = tid + j * NT;
+      if (v < nvec) {
+        float o[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) o[e] = epi_fwd<EPI, FAST>(fmaf((xv[j][e] - mu) * rs, wr[j][e], br[j][e]));
+        if (v < nfull) {
+          st_stream(yrow + (size_t)v * E, V::pack(o));
+        } else {
+#pragma unroll
+          for (int e = 0; e < E; ++e)
+            if (e < cnt[j]) V::store1(yrow + v * E + e, o[e]);
+        }
+      }
+    }
+    if (tid == 0) {
+      if (a.mean) a.mean[m] = mu;
+      if (a.rstd) a.rstd[m] = rs;
+    }
+  }
+}
+
+template <typename T, int VPT, int EPI>
+__global__ void __launch_bounds__(norm_max_threads(VPT, true)) ln_bwd_cta(const LnBwdArgs a) {
+  using V = Vec<T>;
+  constexpr int E = V::N;
+  constexpr bool FAST = fast_math_for<T>();
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int tid = threadIdx.x, NT = blockDim.x, lane = tid & 31, warp = tid >> 5;
+  const int nwarps = NT >> 5;
+  const int N = a.N, nfull = N / E, nvec = (N + E - 1) / E;
+  const RowPipe pipe(smem, a.stages, 2, (int64_t)N * sizeof(T));
+  const int64_t step = gridDim.x;
+  const T* x = static_cast<const T*>(a.x);
+  const T* dy = static_cast<const T*>(a.dy);
+  T* dx = static_cast<T*>(a.dx);
+
+  if (tid == 0) pipe.init();
+  __syncthreads();
+  if (tid == 0) {
+    int64_t m = blockIdx.x;
+    for (int s = 0; s < a.stages && m < a.rows; ++s, m += step) pipe.issue(s, x + m * a.ldx, dy + m * a.lddy);
+  }
+  float wr[VPT][E], br[VPT][E], dwa[VPT][E], dba[VPT][E];
+#pragma unroll
+  for (int j = 0; j < VPT; ++j)
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int col = (tid + j * NT) * E + e;
+      const bool in = col < N;
+      wr[j][e] = in ? ld_param(static_cast<const T*>(a.w), col, 1.0f) : 0.0f;
+      br[j][e] = in ? ld_param(static_cast<const T*>(a.b), col, 0.0f) : 0.0f;
+      dwa[j][e] = 0.0f;
+      dba[j][e] = 0.0f;
+    }
+  const float inv_n = 1.0f / (float)N;
+
+  int s = 0;
+  uint32_t ph = 0, rb = 0;
+  const int64_t ahead = (int64_t)a.stages * step;
+  for (int64_t m = blockIdx.x; m < a.rows; m += step) {
+    const float mu = __ldg(a.mean + m), rs = __ldg(a.rstd + m);
+    const T* xrow = x + m * a.ldx;
+    const T* gyrow = dy + m * a.lddy;
+    const bool ok = pipe.wait(s, ph, a.err);
+    const uint8_t* sx = pipe.at(s, 0);
+    const uint8_t* sg = pipe.at(s, 1);
+    float xv[VPT][E], gv[VPT][E];
+    float s1 = 0.0f, s2 = 0.0f;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      const int v = tid + j * NT;
+      if (v < nfull) {
+        V::unpack(*reinterpret_cast<const uint4*>(sx + (size_t)v * 16), xv[j]);
+        V::unpack(*reinterpret_cast<const uint4*>(sg + (size_t)v * 16), gv[j]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int col = v * E + e;
+          const bool in = v < nvec && col < N;
+          xv[j][e] = in ? V::load1(xrow + col) : 0.0f;
+          gv[j][e] = in ? V::load1(gyrow + col) : 0.0f;
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const float xh = (xv[j][e] - mu) * rs;
+        const float g = gv[j][e] * epi_grad<EPI, FAST>(fmaf(xh, wr[j][e], br[j][e]));
+        const float gw = g * wr[j][e];
+        gv[j][e] = g;
+        s1 += gw;
+        s2 = fmaf(gw, xh, s2);
+        dwa[j][e] = fmaf(g, xh, dwa[j][e]);
+        dba[j][e] += g;
+      }
+    }
+    s1 = group_sum<32>(s1);
+    s2 = group_sum<32>(s2);
+    float4* red = pipe.red + rb * 32;
+    if (lane == 0) red[warp] = make_float4(s1, s2, 0.0f, 0.0f);
+    if (__syncthreads_or(!ok)) {
+      if (tid == 0) pipe.drain(m, step, a.rows, s, ph, a.err);
+      return;
+    }
+    if (tid == 0 && m + ahead < a.rows) pipe.issue(s, x + (m + ahead) * a.ldx, dy + (m + ahead) * a.lddy);
+    rb ^= 1u;
+    if (++s == a.stages) {
+      s = 0;
+      ph ^= 1u;
+    }
+    float t1 = 0.0f, t2 = 0.0f;
+    for (int w = 0; w < nwarps; ++w) {
+      t1 += red[w].x;
+      t2 += red[w].y;
+    }
+    const float c1 = t1 * inv_n, c2 = t2 * inv_n;
+    T* dxrow = dx + m * a.lddx;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      const int v = tid + j * NT;
+      if (v < nvec) {
+        float o[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const float xh = (xv[j][e] - mu) * rs;
+          o[e] = rs * (fmaf(gv[j][e], wr[j][e], -c1) - xh * c2);
+        }
+        if (v < nfull) {
+          st_stream(dxrow + (size_t)v * E, V::pack(o));
+        } else {
+#pragma unroll
+          for (int e = 0; e < E; ++e)
+            if (v * E + e < N) V::store1(dxrow + v * E + e, o[e]);
+        }
+      }
+    }
+  }
+  if (a.ws) {
+    float* part = a.ws + (int64_t)blockIdx.x * 2 * N;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j)
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const int col = (tid + j * NT) * E + e;
+        if (col < N) {
+          part[col] = dwa[j][e];
+          part[N + col] = dba[j][e];
+        }
+      }
+  }
+}
+
+// ---------------------------------------------------------------- group path (short rows)
+
+template <typename T, int VPT, int EPI>
+__global__ void __launch_bounds__(kGroupThreads) ln_fwd_grp(const LnFwdArgs a, int lanes) {
+  using V = Vec<T>;
+  constexpr int E = V::N;
+  constexpr bool FAST = fast_math_for<T>();
+  const int N = a.N, nfull = N / E, nvec = (N + E - 1) / E;
+  const int li = threadIdx.x % lanes, gi = threadIdx.x / lanes;
+  const int64_t gpc = kGroupThreads / lanes;
+  const int64_t gstep = (int64_t)gridDim.x * gpc;
+  const T* x = static_cast<const T*>(a.x);
+  T* y = static_cast<T*>(a.y);
+  float wr[VPT][E], br[VPT][E];
+  load_affine<T, VPT>(a, li, lanes, wr, br);
+  int cnt[VPT];
+#pragma unroll
+  for (int j = 0; j < VPT; ++j) {
+    const int left = N - (li + j * lanes) * E;
+    cnt[j] = left <= 0 ? 0 : left >= E ? E : left;
+  }
+  const float inv_n = 1.0f / (float)N;
+  for (int64_t m0 = (int64_t)blockIdx.x * gpc; m0 < a.rows; m0 += gstep) {
+    const int64_t m = m0 + gi;
+    const bool live = m < a.rows;
+    const T* xrow = x + (live ? m : 0) * a.ldx;
+    float xv[VPT][E];
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      const int v = li + j * lanes;
+      if (live && v < nfull) {
+        V::unpack(ld_stream(xrow + (size_t)v * E), xv[j]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) xv[j][e] = (live && e < cnt[j]) ? V::load1(xrow + v * E + e) : 0.0f;
+      }
+    }
+    float n, mu, M2;
+    thread_stats<VPT, E>(xv, cnt, n, mu, M2);
+    group_stats(n, mu, M2, lanes);
+    mu = __shfl_sync(0xffffffffu, mu, 0, lanes);
+    M2 = __shfl_sync(0xffffffffu, M2, 0, lanes);
+    if (!live) continue;
+    const float rs = rsqrtf(fmaf(M2, inv_n, a.eps));
+    T* yrow = y + m * a.ldy;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      const int v = li + j * lanes;
+      if (v < nvec) {
+        float o[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) o[e] = epi_fwd<EPI, FAST>(fmaf((xv[j][e] - mu) * rs, wr[j][e], br[j][e]));
+        if (v < nfull) {
+          st_stream(yrow + (size_t)v * E, V::pack(o));
+        } else {
+#pragma unroll
+          for (int e = 0; e < E; ++e)
+            if (e < cnt[j]) V::store1(yrow + v * E + e, o[e]);
+        }
+      }
+    }
+    if (li == 0) {
+      if (a.mean) a.mean[m] = mu;
+      if (a.rstd) a.rstd[m] = rs;
+    }
+  }
+}
+
+template <typename T, int VPT, int EPI>
+__global__ void __launch_bounds__(kGroupThreads) ln_bwd_grp(const LnBwdArgs a, int lanes) {
+  using V = Vec<T>;
+  constexpr int E = V::N;
+  constexpr bool FAST = fast_math_for<T>();
+  extern __shared__ __align__(16) float gsm[];  // [groups per CTA][2N] dw, db partials
+  const int N = a.N, nfull = N / E, nvec = (N + E - 1) / E;
+  const int li = threadIdx.x % lanes, gi = threadIdx.x / lanes;
+  const int gpc = kGroupThreads / lanes;
+  const int64_t gstep = (int64_t)gridDim.x * gpc;
+  const T* x = static_cast<const T*>(a.x);
+  const T* dy = static_cast<const T*>(a.dy);
+  T* dx = static_cast<T*>(a.dx);
+  float wr[VPT][E], br[VPT][E], dwa[VPT][E], dba[VPT][E];
+#pragma unroll
+  for (int j = 0; j < VPT; ++j)
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int col = (li + j * lanes) * E + e;
+      const bool in = col < N;
+      wr[j][e] = in ? ld_param(static_cast<const T*>(a.w), col, 1.0f) : 0.0f;
+      br[j][e] = in ? ld_param(static_cast<const T*>(a.b), col, 0.0f) : 0.0f;
+      dwa[j][e] = 0.0f;
+      dba[j][e] = 0.0f;
+    }
+  const float inv_n = 1.0f / (float)N;
+  for (int64_t m0 = (int64_t)blockIdx.x * gpc; m0 < a.rows; m0 += gstep) {
+    const int64_t m = m0 + gi;
+    const bool live = m < a.rows;
+    const int64_t mm = live ? m : 0;
+    const float mu = live ? __ldg(a.mean + m) : 0.0f;
+    const float rs = live ? __ldg(a.rstd + m) : 0.0f;
+    const T* xrow = x + mm * a.ldx;
+    const T* gyrow = dy + mm * a.lddy;
+    float xv[VPT][E], gv[VPT][E];
+    float s1 = 0.0f, s2 = 0.0f;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      const int v = li + j * lanes;
+      if (live && v < nfull) {
+        V::unpack(ld_stream(xrow + (size_t)v * E), xv[j]);
+        V::unpack(ld_stream(gyrow + (size_t)v * E), gv[j]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int col = v * E + e;
+          const bool in = live && v < nvec && col < N;
+          xv[j][e] = in ? V::load1(xrow + col) : 0.0f;
+          gv[j][e] = in ? V::load1(gyrow + col) : 0.0f;
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const float xh = (xv[j][e] - mu) * rs;
+        const float g = gv[j][e] * epi_grad<EPI, FAST>(fmaf(xh, wr[j][e], br[j][e]));
+        const float gw = g * wr[j][e];
+        gv[j][e] = g;
+        s1 += gw;
+        s2 = fmaf(gw, xh, s2);
+        dwa[j][e] = fmaf(g, xh, dwa[j][e]);
+        dba[j][e] += g;
+      }
+    }
+    s1 = group_sum_rt(s1, lanes);
+    s2 = group_sum_rt(s2, lanes);
+    if (!live) continue;
+    const float c1 = s1 * inv_n, c2 = s2 * inv_n;
+    T* dxrow = dx + m * a.lddx;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      const int v = li + j * lanes;
+      if (v < nvec) {
+        float o[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const float xh = (xv[j][e] - mu) * rs;
+          o[e] = rs * (fmaf(gv[j][e], wr[j][e], -c1) - xh * c2);
+        }
+        if (v < nfull) {
+          st_stream(dxrow + (size_t)v * E, V::pack(o));
+        } else {
+#pragma unroll
+          for (int e = 0; e < E; ++e)
+            if (v * E + e < N) V::store1(dxrow + v * E + e, o[e]);
+        }
+      }
+    }
+  }
+  if (!a.ws) return;
+#pragma unroll
+  for (int j = 0; j < VPT; ++j)
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int col = (li + j * lanes) * E + e;
+      if (col < N) {
+        gsm[gi * 2 * N + col] = dwa[j][e];
+        gsm[gi * 2 * N + N + col] = dba[j][e];
+      }
+    }
+  __syncthreads();
+  float* part = a.ws + (int64_t)blockIdx.x * 2 * N;
+  for (int col = threadIdx.x; col < 2 * N; col += kGroupThreads) {
+    float t = 0.0f;
+    for (int g = 0; g < gpc; ++g) t += gsm[g * 2 * N + col];
+    part[col] = t;
+  }
+}
+
+// ---------------------------------------------------------------- dispatch
+
+template <typename T, int VPT, bool CTA, bool BWD>
+void* pick_ln(int epi) {
+#define GN_PICK(E_)                                                              \
+  if constexpr (BWD) {                                                           \
+    if constexpr (CTA) return (void*)ln_bwd_cta<T, VPT, E_>;                     \
+    else return (void*)ln_bwd_grp<T, VPT, E_>;                                   \
+  } else {                                                                       \
+    if constexpr (CTA) return (void*)ln_fwd_cta<T, VPT, E_>;                     \
+    else return (void*)ln_fwd_grp<T, VPT, E_>;                                   \
+  }
+  if (epi == EPI_GELU_TANH) { GN_PICK(EPI_GELU_TANH) }
+  if (epi == EPI_SILU) { GN_PICK(EPI_SILU) }
+  GN_PICK(EPI_NONE)
+#undef GN_PICK
+}
+
+template <typename T, bool BWD>
+void* pick_ln_t(int vpt, bool cta, int epi) {
+  switch (vpt) {
+    case 1: return cta ? pick_ln<T, 1, true, BWD>(epi) : pick_ln<T, 1, false, BWD>(epi);
+    case 2: return cta ? pick_ln<T, 2, true, BWD>(epi) : pick_ln<T, 2, false, BWD>(epi);
+    case 4: return cta ? pick_ln<T, 4, true, BWD>(epi) : pick_ln<T, 4, false, BWD>(epi);
+    case 8:
+      if constexpr (!BWD) return cta ? pick_ln<T, 8, true, false>(epi) : nullptr;
+      return nullptr;
+  }
+  return nullptr;
+}
+
+constexpr int kFwdThreads = 256;
+constexpr int kBwdThreads = 512;
+
+gn_status ln_plan(int64_t rows, int64_t hidden, gn_dtype dt, bool bwd, int epi, NormPlan* p, void** kern,
+                  int* grid) {
+  gn_status st = plan_norm(hidden, dt_size(dt), bwd ? 2 : 1, bwd ? 4 : 8, bwd ? kBwdThreads : kFwdThreads, p);
+  if (st != GN_OK) return st;
+  if (dt == GN_BF16)
+    *kern = bwd ? pick_ln_t<__nv_bfloat16, true>(p->vpt, p->cta, epi) : pick_ln_t<__nv_bfloat16, false>(p->vpt, p->cta, epi);
+  else
+    *kern = bwd ? pick_ln_t<float, true>(p->vpt, p->cta, epi) : pick_ln_t<float, false>(p->vpt, p->cta, epi);
+  if (!*kern) return GN_ERR_UNSUPPORTED;
+  const int cap = g_tune.ctas_per_sm ? g_tune.ctas_per_sm : 8;
+  int g = persistent_grid(*kern, p->threads, p->smem, cap);
+  if (g <= 0) return GN_ERR_CUDA;
+  const int64_t units = p->cta ? rows : (rows + (kGroupThreads / p->lanes) - 1) / (kGroupThreads / p->lanes);
+  if (units < g) g = (int)(units > 0 ? units : 1);
+  *grid = g;
+  return GN_OK;
+}
+
+}  // namespace
+}  // namespace gn
+
+using namespace gn;
+
+extern "C" gn_status gn_layernorm_fwd(const void* x, const void* w, const void* b, void* y, float* mean,
+                                      float* rstd, int64_t rows, int64_t hidden, int64_t ld_x, int64_t ld_y,
+                                      float eps, gn_epilogue epi, gn_dtype dt, void* stream) {
+  if (!dt_ok(dt) || !epi_ok(epi)) return GN_ERR_DTYPE;
+  if (rows < 0 || hidden <= 0 || ld_x < hidden || ld_y < hidden || hidden > (1 << 20)) return GN_ERR_SHAPE;
+  if (rows == 0) return GN_OK;
+  if (!x || !y) return GN_ERR_NULL;
+  const size_t es = dt_size(dt);
+  if (!aligned16(x) || !aligned16(y) || (ld_x * es) % 16 || (ld_y * es) % 16) return GN_ERR_ALIGN;
+  NormPlan p;
+  void* kern = nullptr;
+  int grid = 0;
+  gn_status st = ln_plan(rows, hidden, dt, false, epi, &p, &kern, &grid);
+  if (st != GN_OK) return st;
+  unsigned* err = device_err_word();
+  if (!err) return GN_ERR_CUDA;
+  LnFwdArgs a{x, w, b, y, mean, rstd, rows, ld_x, ld_y, (int)hidden, eps, p.stages, err};
+  int lanes = p.lanes;
+  void* args_cta[] = {&a};
+  void* args_grp[] = {&a, &lanes};
+  if (cudaLaunchKernel(kern, dim3(grid), dim3(p.threads), p.cta ? args_cta : args_grp, p.smem,
+                       (cudaStream_t)stream) != cudaSuccess)
+    return GN_ERR_CUDA;
+  count_launches(1);
+  return launch_status();
+}
+
+extern "C" size_t gn_layernorm_bwd_workspace(int64_t rows, int64_t hidden, gn_dtype dt) {
+  if (rows <= 0 || hidden <= 0 || !dt_ok(dt)) return 0;
+  NormPlan p;
+  void* kern = nullptr;
+  int grid = 0;
+  if (ln_plan(rows, hidden, dt, true, GN_EPI_NONE, &p, &kern, &grid) != GN_OK) return 0;
+  return (size_t)grid * 2 * (size_t)hidden * sizeof(float);
+}
+
+extern "C" gn_status gn_layernorm_bwd(const void* x, const void* w, const void* b, const float* mean,
+                                      const float* rstd, const void* dy, void* dx, float* dw, float* db,
+                                      void* ws, size_t ws_bytes, int64_t rows, int64_t hidden, int64_t ld_x,
+                                      int64_t ld_dy, int64_t ld_dx, gn_epilogue epi, gn_dtype dt,
+                                      void* stream) {
+  if (!dt_ok(dt) || !epi_ok(epi)) return GN_ERR_DTYPE;
+  if (rows < 0 || hidden <= 0 || ld_x < hidden || ld_dy < hidden || ld_dx < hidden || hidden > (1 << 20))
+    return GN_ERR_SHAPE;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (rows == 0) {
+    if (dw && cudaMemsetAsync(dw, 0, (size_t)hidden * sizeof(float), s) != cudaSuccess) return GN_ERR_CUDA;
+    if (db && cudaMemsetAsync(db, 0, (size_t)hidden * sizeof(float), s) != cudaSuccess) return GN_ERR_CUDA;
+    return GN_OK;
+  }
+  if (!x || !mean || !rstd || !dy || !dx) return GN_ERR_NULL;
+  const size_t es = dt_size(dt);
+  if (!aligned16(x) || !aligned16(dy) || !aligned16(dx) || (ld_x * es) % 16 || (ld_dy * es) % 16 ||
+      (ld_dx * es) % 16)
+    return GN_ERR_ALIGN;
+  NormPlan p;
+  void* kern = nullptr;
+  int grid = 0;
+  gn_status st = ln_plan(rows, hidden, dt, true, epi, &p, &kern, &grid);
+  if (st != GN_OK) return st;
+  const bool wgrad = dw || db;
+  if (wgrad) {
+    if (!ws) return GN_ERR_WORKSPACE;
+    if (!aligned16(ws)) return GN_ERR_ALIGN;
+    if (ws_bytes < (size_t)grid * 2 * (size_t)hidden * sizeof(float)) return GN_ERR_WORKSPACE;
+  }
+  unsigned* err = device_err_word();
+  if (!err) return GN_ERR_CUDA;
+  LnBwdArgs a{x, w, b, mean, rstd, dy, dx, wgrad ? static_cast<float*>(ws) : nullptr, rows, ld_x, ld_dy, ld_dx,
+              (int)hidden, p.stages, err};
+  int lanes = p.lanes;
+  void* args_cta[] = {&a};
+  void* args_grp[] = {&a, &lanes};
+  if (cudaLaunchKernel(kern, dim3(grid), dim3(p.threads), p.cta ? args_cta : args_grp, p.smem, s) !=
+      cudaSuccess)
+    return GN_ERR_CUDA;
+  count_launches(1);
+  if ((st = launch_status()) != GN_OK) return st;
+  if (wgrad) return launch_colsum(static_cast<const float*>(ws), grid, 2 * hidden, hidden, dw, db, s);
+  return GN_OK;
+}

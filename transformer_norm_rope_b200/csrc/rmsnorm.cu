@@ -1,0 +1,577 @@
+// rmsnorm.cu - RMSNorm forward and backward (Helios kernels article, section
+// "内核一 FlashNorm": one pass over each row, sum of squares and its inverse root, times the
+// weight; Gemma +1 offset as a compile-time branch; the forward saves the per-row inverse
+// RMS and the backward reuses it).
+//
+//   forward : r = rsqrt(mean(x^2) + eps), y = epi(x r w'), inv_rms = r
+//   backward: g = dy epi'(x r w'), dx = r (g w' - x r mean(g w' x r)), dw = sum_rows g x r
+//
+// Both directions read each input byte from HBM once and write each output byte once. The
+// weight gradient is accumulated per thread in fp32 registers over the rows a CTA owns,
+// written as one partial row per CTA, and summed in a fixed order by launch_colsum.
+#include "norm_plan.h"
+
+namespace gn {
+namespace {
+
+struct RmsFwdArgs {
+  const void* x;
+  const void* w;
+  void* y;
+  float* inv_rms;
+  int64_t rows;
+  int64_t ldx, ldy;
+  int N;
+  float eps;
+  int stages;
+  unsigned* err;
+};
+
+struct RmsBwdArgs {
+  const void* x;
+  const void* w;
+  const float* inv_rms;
+  const void* dy;
+  void* dx;
+  float* ws;  // [gridDim.x, N] partial dw, or null
+  int64_t rows;
+  int64_t ldx, lddy, lddx;
+  int N;
+  int stages;
+  unsigned* err;
+};
+
+// ---------------------------------------------------------------- CTA path
+
+template <typename T, int VPT, int EPI, bool GEMMA>
+__global__ void __launch_bounds__(norm_max_threads(VPT)) rms_fwd_cta(const RmsFwdArgs a) {
+  using V = Vec<T>;
+  constexpr int E = V::N;
+  constexpr bool FAST = fast_math_for<T>();
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int tid = threadIdx.x, NT = blockDim.x, lane = tid & 31, warp = tid >> 5;
+  const int nwarps = NT >> 5;
+  const int N = a.N, nfull = N / E, nvec = (N + E - 1) / E;
+  const RowPipe pipe(smem, a.stages, 1, (int64_t)N * sizeof(T));
+  const int64_t step = gridDim.x;
+  const T* x = static_cast<const T*>(a.x);
+  T* y = static_cast<T*>(a.y);
+
+  if (tid == 0) pipe.init();
+  __syncthreads();
+  if (tid == 0) {
+    int64_t m = blockIdx.x;
+    for (int s = 0; s < a.stages && m < a.rows; ++s, m += step) pipe.issue(s, x + m * a.ldx);
+  }
+
+  float wr[VPT][E];
+#pragma unroll
+  for (int j = 0; j < VPT; ++j)
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int col = (tid + j * NT) * E + e;
+      wr[j][e] = col < N ? (GEMMA ? 1.0f : 0.0f) + ld_param(static_cast<const T*>(a.w), col, 0.0f) : 0.0f;
+    }
+  const float inv_n = 1.0f / (float)N;
+
+  int s = 0;         // stage of row m
+  uint32_t ph = 0;   // barrier parity of that stage's current use
+  uint32_t rb = 0;   // reduction buffer, alternating per row
+  const int64_t ahead = (int64_t)a.stages * step;
+  for (int64_t m = blockIdx.x; m < a.rows; m += step) {
+    const T* xrow = x + m * a.ldx;
+    const bool ok = pipe.wait(s, ph, a.err);
+    const uint8_t* st = pipe.at(s, 0);
+    float xv[VPT][E];
+    float ss = 0.0f;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      const int v = tid + j * NT;
+      if (v < nfull) {
+        V::unpack(*reinterpret_cast<const uint4*>(st + (size_t)v * 16), xv[j]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int col = v * E + e;
+          xv[j][e] = (v < nvec && col < N) ? V::load1(xrow + col) : 0.0f;
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < E; ++e) ss = fmaf(xv[j][e], xv[j][e], ss);
+    }
+    ss = group_sum<32>(ss);
+    float4* red = pipe.red + rb * 32;
+    if (lane == 0) red[warp].x = ss;
+    if (__syncthreads_or(!ok)) {
+      if (tid == 0) pipe.drain(m, step, a.rows, s, ph, a.err);
+      return;
+    }
+    if (tid == 0 && m + ahead < a.rows) pipe.issue(s, x + (m + ahead) * a.ldx);
+    rb ^= 1u;
+    if (++s == a.stages) {
+      s = 0;
+      ph ^= 1u;
+    }
+    float tot = 0.0f;
+    for (int w = 0; w < nwarps; ++w) tot += red[w].x;
+    const float r = rsqrtf(fmaf(tot, inv_n, a.eps));
+    T* yrow = y + m * a.ldy;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      const int v = tid + j * NT;
+      if (v < nvec) {
+        float o[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) o[e] = epi_fwd<EPI, FAST>(xv[j][e] * r * wr[j][e]);
+        if (v < nfull) {
+          st_stream(yrow + (size_t)v * E, V::pack(o));
+        } else {
+#pragma unroll
+          for (int e = 0; e < E; ++e)
+            if (v * E + e < N) V::store1(yrow + v * E + e, o[e]);
+        }
+      }
+    }
+    if (tid == 0 && a.inv_rms) a.inv_rms[m] = r;
+  }
+}
+
+template <typename T, int VPT, int EPI, bool GEMMA>
+__global__ void __launch_bounds__(norm_max_threads(VPT, true)) rms_bwd_cta(const RmsBwdArgs a) {
+  using V = Vec<T>;
+  constexpr int E = V::N;
+  constexpr bool FAST = fast_math_for<T>();
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int tid = threadIdx.x, NT = blockDim.x, lane = tid & 31, warp = tid >> 5;
+  const int nwarps = NT >> 5;
+  const int N = a.N, nfull = N / E, nvec = (N + E - 1) / E;
+  const RowPipe pipe(smem, a.stages, 2, (int64_t)N * sizeof(T));
+  const int64_t step = gridDim.x;
+  const T* x = static_cast<const T*>(a.x);
+  const T* dy = static_cast<const T*>(a.dy);
+  T* dx = static_cast<T*>(a.dx);
+
+  if (tid == 0) pipe.init();
+  __syncthreads();
+  if (tid == 0) {
+    int64_t m = blockIdx.x;
+    for (int s = 0; s < a.stages && m < a.rows; ++s, m += step) pipe.issue(s, x + m * a.ldx, dy + m * a.lddy);
+  }
+
+  float wr[VPT][E], dwa[VPT][E];
+#pragma unroll
+  for (int j = 0; j < VPT; ++j)
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int col = (tid + j * NT) * E + e;
+      wr[j][e] = col < N ? (GEMMA ? 1.0f : 0.0f) + ld_param(static_cast<const T*>(a.w), col, 0.0f) : 0.0f;
+      dwa[j][e] = 0.0f;
+    }
+  const float inv_n = 1.0f / (float)N;
+
+  int s = 0;         // stage of row m
+  uint32_t ph = 0;   // barrier parity of that stage's current use
+  uint32_t rb = 0;   // reduction buffer, alternating per row
+  const int64_t ahead = (int64_t)a.stages * step;
+  for (int64_t m = blockIdx.x; m < a.rows; m += step) {
+    const float r = __ldg(a.inv_rms + m);
+    const T* xrow = x + m * a.ldx;
+    const T* gyrow = dy + m * a.lddy;
+    const bool ok = pipe.wait(s, ph, a.err);
+    const uint8_t* sx = pipe.at(s, 0);
+    const uint8_t* sg = pipe.at(s, 1);
+    float xv[VPT][E], gv[VPT][E];
+    float c = 0.0f;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      const int v = tid + j * NT;
+      if (v < nfull) {
+        V::unpack(*reinterpret_cast<const uint4*>(sx + (size_t)v * 16), xv[j]);
+        V::unpack(*reinterpret_cast<const uint4*>(sg + (size_t)v * 16), gv[j]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int col = v * E + e;
+          const bool in = v < nvec && col < N;
+          xv[j][e] = in ? V::load1(xrow + col) : 0.0f;
+          gv[j][e] = in ? V::load1(gyrow + col) : 0.0f;
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const float xh = xv[j][e] * r;
+        const float g = gv[j][e] * epi_grad<EPI, FAST>(xh * wr[j][e]);
+        gv[j][e] = g;
+        c = fmaf(g * wr[j][e], xh, c);
+        dwa[j][e] = fmaf(g, xh, dwa[j][e]);
+      }
+    }
+    c = group_sum<32>(c);
+    float4* red = pipe.red + rb * 32;
+    if (lane == 0) red[warp].x = c;
+    if (__syncthreads_or(!ok)) {
+      if (tid == 0) pipe.drain(m, step, a.rows, s, ph, a.err);
+      return;
+    }
+    if (tid == 0 && m + ahead < a.rows) pipe.issue(s, x + (m + ahead) * a.ldx, dy + (m + ahead) * a.lddy);
+    rb ^= 1u;
+    if (++s == a.stages) {
+      s = 0;
+      ph ^= 1u;
+    }
+    float tot = 0.0f;
+    for (int w = 0; w < nwarps; ++w) tot += red[w].x;
+    const float cm = tot * inv_n;
+    T* dxrow = dx + m * a.lddx;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      const int v = tid + j * NT;
+      if (v < nvec) {
+        float o[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) o[e] = r * fmaf(gv[j][e], wr[j][e], -(xv[j][e] * r) * cm);
+        if (v < nfull) {
+          st_stream(dxrow + (size_t)v * E, V::pack(o));
+        } else {
+#pragma unroll
+          for (int e = 0; e < E; ++e)
+            if (v * E + e < N) V::store1(dxrow + v * E + e, o[e]);
+        }
+      }
+    }
+  }
+  if (a.ws) {
+    float* part = a.ws + (int64_t)blockIdx.x * N;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j)
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const int col = (tid + j * NT) * E + e;
+        if (col < N) part[col] = dwa[j][e];
+      }
+  }
+}
+
+// ---------------------------------------------------------------- group path (short rows)
+// `lanes` consecutive threads own one row; rows are walked grid-stride by lane groups.
+
+template <typename T, int VPT, int EPI, bool GEMMA>
+__global__ void __launch_bounds__(kGroupThreads) rms_fwd_grp(const RmsFwdArgs a, int lanes) {
+  using V = Vec<T>;
+  constexpr int E = V::N;
+  constexpr bool FAST = fast_math_for<T>();
+  const int N = a.N, nfull = N / E, nvec = (N + E - 1) / E;
+  const int li = threadIdx.x % lanes;
+  const int64_t gpc = kGroupThreads / lanes;
+  const int gi = threadIdx.x / lanes;
+  const int64_t gstep = (int64_t)gridDim.x * gpc;
+  const T* x = static_cast<const T*>(a.x);
+  T* y = static_cast<T*>(a.y);
+  float wr[VPT][E];
+#pragma unroll
+  for (int j = 0; j < VPT; ++j)
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int col = (li + j * lanes) * E + e;
+      wr[j][e] = col < N ? (GEMMA ? 1.0f : 0.0f) + ld_param(static_cast<const T*>(a.w), col, 0.0f) : 0.0f;
+    }
+  const float inv_n = 1.0f / (float)N;
+  // the loop bound is the CTA's first row (uniform over the CTA), so every lane runs the
+  // same iterations and the shuffles below always see the full warp
+  for (int64_t m0 = (int64_t)blockIdx.x * gpc; m0 < a.rows; m0 += gstep) {
+    const int64_t m = m0 + gi;
+    const bool live = m < a.rows;
+    const T* xrow = x + (live ? m : 0) * a.ldx;
+    float xv[VPT][E];
+    float ss = 0.0f;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      const int v = li + j * lanes;
+      if (live && v < nfull) {
+        V::unpack(ld_stream(xrow + (size_t)v * E), xv[j]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int col = v * E + e;
+          xv[j][e] = (live && v < nvec && col < N) ? V::load1(xrow + col) : 0.0f;
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < E; ++e) ss = fmaf(xv[j][e], xv[j][e], ss);
+    }
+    ss = group_sum_rt(ss, lanes);
+    if (!live) continue;
+    const float r = rsqrtf(fmaf(ss, inv_n, a.eps));
+    T* yrow = y + m * a.ldy;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      const int v = li + j * lanes;
+      if (v < nvec) {
+        float o[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) o[e] = epi_fwd<EPI, FAST>(xv[j][e] * r * wr[j][e]);
+        if (v < nfull) {
+          st_stream(yrow + (size_t)v * E, V::pack(o));
+        } else {
+#pragma unroll
+          for (int e = 0; e < E; ++e)
+            if (v * E + e < N) V::store1(yrow + v * E + e, o[e]);
+        }
+      }
+    }
+    if (li == 0 && a.inv_rms) a.inv_rms[m] = r;
+  }
+}
+
+template <typename T, int VPT, int EPI, bool GEMMA>
+__global__ void __launch_bounds__(kGroupThreads) rms_bwd_grp(const RmsBwdArgs a, int lanes) {
+  using V = Vec<T>;
+  constexpr int E = V::N;
+  constexpr bool FAST = fast_math_for<T>();
+  extern __shared__ __align__(16) float gsm[];  // [groups per CTA][N] dw partials
+  const int N = a.N, nfull = N / E, nvec = (N + E - 1) / E;
+  const int li = threadIdx.x % lanes;
+  const int gi = threadIdx.x / lanes;
+  const int gpc = kGroupThreads / lanes;
+  const int64_t gstep = (int64_t)gridDim.x * gpc;
+  const T* x = static_cast<const T*>(a.x);
+  const T* dy = static_cast<const T*>(a.dy);
+  T* dx = static_cast<T*>(a.dx);
+  float wr[VPT][E], dwa[VPT][E];
+#pragma unroll
+  for (int j = 0; j < VPT; ++j)
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int col = (li + j * lanes) * E + e;
+      wr[j][e] = col < N ? (GEMMA ? 1.0f : 0.0f) + ld_param(static_cast<const T*>(a.w), col, 0.0f) : 0.0f;
+      dwa[j][e] = 0.0f;
+    }
+  const float inv_n = 1.0f / (float)N;
+  for (int64_t m0 = (int64_t)blockIdx.x * gpc; m0 < a.rows; m0 += gstep) {
+    const int64_t m = m0 + gi;
+    const bool live = m < a.rows;
+    const int64_t mm = live ? m : 0;
+    const float r = live ? __ldg(a.inv_rms + m) : 0.0f;
+    const T* xrow = x + mm * a.ldx;
+    const T* gyrow = dy + mm * a.lddy;
+    float xv[VPT][E], gv[VPT][E];
+    float c = 0.0f;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      const int v = li + j * lanes;
+      if (live && v < nfull) {
+        V::unpack(ld_stream(xrow + (size_t)v * E), xv[j]);
+        V::unpack(ld_stream(gyrow + (size_t)v * E), gv[j]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int col = v * E + e;
+          const bool in = live && v < nvec && col < N;
+          xv[j][e] = in ? V::load1(xrow + col) : 0.0f;
+          gv[j][e] = in ? V::load1(gyrow + col) : 0.0f;
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const float xh = xv[j][e] * r;
+        const float g = gv[j][e] * epi_grad<EPI, FAST>(xh * wr[j][e]);
+        gv[j][e] = g;
+        c = fmaf(g * wr[j][e], xh, c);
+        dwa[j][e] = fmaf(g, xh, dwa[j][e]);
+      }
+    }
+    c = group_sum_rt(c, lanes);
+    if (!live) continue;
+    const float cm = c * inv_n;
+    T* dxrow = dx + m * a.lddx;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      const int v = li + j * lanes;
+      if (v < nvec) {
+        float o[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) o[e] = r * fmaf(gv[j][e], wr[j][e], -(xv[j][e] * r) * cm);
+        if (v < nfull) {
+          st_stream(dxrow + (size_t)v * E, V::pack(o));
+        } else {
+#pragma unroll
+          for (int e = 0; e < E; ++e)
+            if (v * E + e < N) V::store1(dxrow + v * E + e, o[e]);
+        }
+      }
+    }
+  }
+  if (!a.ws) return;
+  // combine the groups of this CTA in group order, then write one partial row
+#pragma unroll
+  for (int j = 0; j < VPT; ++j)
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int col = (li + j * lanes) * E + e;
+      if (col < N) gsm[gi * N + col] = dwa[j][e];
+    }
+  __syncthreads();
+  float* part = a.ws + (int64_t)blockIdx.x * N;
+  for (int col = threadIdx.x; col < N; col += kGroupThreads) {
+    float t = 0.0f;
+    for (int g = 0; g < gpc; ++g) t += gsm[g * N + col];
+    part[col] = t;
+  }
+}
+
+// ---------------------------------------------------------------- dispatch
+
+template <typename T, int VPT, bool CTA>
+void* pick_fwd(int epi, bool gemma) {
+#define GN_PICK(E_, G_) \
+  if constexpr (CTA) return (void*)rms_fwd_cta<T, VPT, E_, G_>; \
+  else return (void*)rms_fwd_grp<T, VPT, E_, G_>
+  if (epi == EPI_GELU_TANH) { if (gemma) GN_PICK(EPI_GELU_TANH, true); else GN_PICK(EPI_GELU_TANH, false); }
+  if (epi == EPI_SILU) { if (gemma) GN_PICK(EPI_SILU, true); else GN_PICK(EPI_SILU, false); }
+  if (gemma) GN_PICK(EPI_NONE, true);
+  GN_PICK(EPI_NONE, false);
+#undef GN_PICK
+}
+
+template <typename T, int VPT, bool CTA>
+void* pick_bwd(int epi, bool gemma) {
+#define GN_PICK(E_, G_) \
+  if constexpr (CTA) return (void*)rms_bwd_cta<T, VPT, E_, G_>; \
+  else return (void*)rms_bwd_grp<T, VPT, E_, G_>
+  if (epi == EPI_GELU_TANH) { if (gemma) GN_PICK(EPI_GELU_TANH, true); else GN_PICK(EPI_GELU_TANH, false); }
+  if (epi == EPI_SILU) { if (gemma) GN_PICK(EPI_SILU, true); else GN_PICK(EPI_SILU, false); }
+  if (gemma) GN_PICK(EPI_NONE, true);
+  GN_PICK(EPI_NONE, false);
+#undef GN_PICK
+}
+
+template <typename T>
+void* pick_fwd_t(int vpt, bool cta, int epi, bool gemma) {
+  switch (vpt) {
+    case 1: return cta ? pick_fwd<T, 1, true>(epi, gemma) : pick_fwd<T, 1, false>(epi, gemma);
+    case 2: return cta ? pick_fwd<T, 2, true>(epi, gemma) : pick_fwd<T, 2, false>(epi, gemma);
+    case 4: return cta ? pick_fwd<T, 4, true>(epi, gemma) : pick_fwd<T, 4, false>(epi, gemma);
+    case 8: return cta ? pick_fwd<T, 8, true>(epi, gemma) : nullptr;
+  }
+  return nullptr;
+}
+
+template <typename T>
+void* pick_bwd_t(int vpt, bool cta, int epi, bool gemma) {
+  switch (vpt) {
+    case 1: return cta ? pick_bwd<T, 1, true>(epi, gemma) : pick_bwd<T, 1, false>(epi, gemma);
+    case 2: return cta ? pick_bwd<T, 2, true>(epi, gemma) : pick_bwd<T, 2, false>(epi, gemma);
+    case 4: return cta ? pick_bwd<T, 4, true>(epi, gemma) : pick_bwd<T, 4, false>(epi, gemma);
+  }
+  return nullptr;
+}
+
+constexpr int kFwdThreads = 256;  // preferred CTA size when choosing vpt (forward)
+constexpr int kBwdThreads = 512;  // (backward)
+
+gn_status rms_bwd_plan(int64_t rows, int64_t hidden, gn_dtype dt, NormPlan* p, void** kern, int epi,
+                       bool gemma, int* grid) {
+  gn_status st = plan_norm(hidden, dt_size(dt), 2, 4, kBwdThreads, p);
+  if (st != GN_OK) return st;
+  *kern = dt == GN_BF16 ? pick_bwd_t<__nv_bfloat16>(p->vpt, p->cta, epi, gemma)
+                        : pick_bwd_t<float>(p->vpt, p->cta, epi, gemma);
+  if (!*kern) return GN_ERR_UNSUPPORTED;
+  const int cap = g_tune.ctas_per_sm ? g_tune.ctas_per_sm : 8;
+  int g = persistent_grid(*kern, p->threads, p->smem, cap);
+  if (g <= 0) return GN_ERR_CUDA;
+  const int64_t units = p->cta ? rows : (rows + (kGroupThreads / p->lanes) - 1) / (kGroupThreads / p->lanes);
+  if (units < g) g = (int)(units > 0 ? units : 1);
+  *grid = g;
+  return GN_OK;
+}
+
+}  // namespace
+}  // namespace gn
+
+using namespace gn;
+
+extern "C" gn_status gn_rmsnorm_fwd(const void* x, const void* w, void* y, float* inv_rms,
+                                    int64_t rows, int64_t hidden, int64_t ld_x, int64_t ld_y,
+                                    float eps, int gemma, gn_epilogue epi, gn_dtype dt,
+                                    void* stream) {
+  if (!dt_ok(dt) || !epi_ok(epi)) return GN_ERR_DTYPE;
+  if (rows < 0 || hidden <= 0 || ld_x < hidden || ld_y < hidden || hidden > (1 << 20)) return GN_ERR_SHAPE;
+  if (rows == 0) return GN_OK;
+  if (!x || !w || !y) return GN_ERR_NULL;
+  const size_t es = dt_size(dt);
+  if (!aligned16(x) || !aligned16(y) || (ld_x * es) % 16 || (ld_y * es) % 16) return GN_ERR_ALIGN;
+  NormPlan p;
+  gn_status st = plan_norm(hidden, es, 1, 8, kFwdThreads, &p);
+  if (st != GN_OK) return st;
+  void* kern = dt == GN_BF16 ? pick_fwd_t<__nv_bfloat16>(p.vpt, p.cta, epi, gemma != 0)
+                             : pick_fwd_t<float>(p.vpt, p.cta, epi, gemma != 0);
+  if (!kern) return GN_ERR_UNSUPPORTED;
+  const int cap = g_tune.ctas_per_sm ? g_tune.ctas_per_sm : 8;
+  int grid = persistent_grid(kern, p.threads, p.smem, cap);
+  if (grid <= 0) return GN_ERR_CUDA;
+  const int64_t units = p.cta ? rows : (rows + (kGroupThreads / p.lanes) - 1) / (kGroupThreads / p.lanes);
+  if (units < grid) grid = (int)units;
+  unsigned* err = device_err_word();
+  if (!err) return GN_ERR_CUDA;
+  RmsFwdArgs a{x, w, y, inv_rms, rows, ld_x, ld_y, (int)hidden, eps, p.stages, err};
+  int lanes = p.lanes;
+  void* args_cta[] = {&a};
+  void* args_grp[] = {&a, &lanes};
+  if (cudaLaunchKernel(kern, dim3(grid), dim3(p.threads), p.cta ? args_cta : args_grp, p.smem,
+                       (cudaStream_t)stream) != cudaSuccess)
+    return GN_ERR_CUDA;
+  count_launches(1);
+  return launch_status();
+}
+
+extern "C" size_t gn_rmsnorm_bwd_workspace(int64_t rows, int64_t hidden, gn_dtype dt) {
+  if (rows <= 0 || hidden <= 0 || !dt_ok(dt)) return 0;
+  NormPlan p;
+  void* kern = nullptr;
+  int grid = 0;
+  if (rms_bwd_plan(rows, hidden, dt, &p, &kern, GN_EPI_NONE, false, &grid) != GN_OK) return 0;
+  return (size_t)grid * (size_t)hidden * sizeof(float);
+}
+
+extern "C" gn_status gn_rmsnorm_bwd(const void* x, const void* w, const float* inv_rms,
+                                    const void* dy, void* dx, float* dw, void* ws, size_t ws_bytes,
+                                    int64_t rows, int64_t hidden, int64_t ld_x, int64_t ld_dy,
+                                    int64_t ld_dx, int gemma, gn_epilogue epi, gn_dtype dt,
+                                    void* stream) {
+  if (!dt_ok(dt) || !epi_ok(epi)) return GN_ERR_DTYPE;
+  if (rows < 0 || hidden <= 0 || ld_x < hidden || ld_dy < hidden || ld_dx < hidden || hidden > (1 << 20))
+    return GN_ERR_SHAPE;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (rows == 0) {
+    if (dw && cudaMemsetAsync(dw, 0, (size_t)hidden * sizeof(float), s) != cudaSuccess) return GN_ERR_CUDA;
+    return GN_OK;
+  }
+  if (!x || !w || !inv_rms || !dy || !dx) return GN_ERR_NULL;
+  const size_t es = dt_size(dt);
+  if (!aligned16(x) || !aligned16(dy) || !aligned16(dx) || (ld_x * es) % 16 || (ld_dy * es) % 16 ||
+      (ld_dx * es) % 16)
+    return GN_ERR_ALIGN;
+  NormPlan p;
+  void* kern = nullptr;
+  int grid = 0;
+  gn_status st = rms_bwd_plan(rows, hidden, dt, &p, &kern, epi, gemma != 0, &grid);
+  if (st != GN_OK) return st;
+  if (dw) {
+    if (!ws || !aligned16(ws)) return ws ? GN_ERR_ALIGN : GN_ERR_WORKSPACE;
+    if (ws_bytes < (size_t)grid * (size_t)hidden * sizeof(float)) return GN_ERR_WORKSPACE;
+  }
+  unsigned* err = device_err_word();
+  if (!err) return GN_ERR_CUDA;
+  RmsBwdArgs a{x, w, inv_rms, dy, dx, dw ? static_cast<float*>(ws) : nullptr, rows, ld_x, ld_dy, ld_dx,
+               (int)hidden, p.stages, err};
+  int lanes = p.lanes;
+  void* args_cta[] = {&a};
+  void* args_grp[] = {&a, &lanes};
+  if (cudaLaunchKernel(kern, dim3(grid), dim3(p.threads), p.cta ? args_cta : args_grp, p.smem, s) !=
+      cudaSuccess)
+    return GN_ERR_CUDA;
+  count_launches(1);
+  if ((st = launch_status()) != GN_OK) return st;
+  if (dw) return launch_colsum(static_cast<const float*>(ws), grid, hidden, hidden, dw, nullptr, s);
+  return GN_OK;
+}

@@ -1,0 +1,489 @@
+// rope.cu - interleaved rotary position embedding, in place (Helios kernels article, section
+// "内核二 FlashRoPE": pair i of a head at offsets 2i and 2i+1, rotated in one pass and written
+// back in place, no intermediate tensors; the backward is the same kernel with sin negated),
+// and the fused per-head RMSNorm + RoPE ("内核一 FlashNorm" and "内核二 FlashRoPE" applied to
+// q and k together, section "基准实测").
+//
+// One kernel template serves the three operations. The work unit is a slab of HC consecutive
+// heads of one token (b, s) of q and of k: HC*D contiguous elements per tensor. A persistent
+// CTA walks the units grid-stride; each unit's slabs and its cos/sin table rows arrive in a
+// shared-memory stage through 1-D TMA bulk copies (multi-stage pipeline, bounded waits).
+// Units are ordered token-major, so the table row of token s is fetched by neighbouring CTAs
+// at about the same time and HBM delivers it once per token.
+//
+//   ROPE    : x <- rot(x, cos, sign*sin)                                   (in place)
+//   QK_FWD  : r = rsqrt(mean_d x^2 + eps), out = rot(x r w', cos, sin), inv_rms = r
+//   QK_BWD  : u = rot(dy, cos, -sin), g = u w', dx = r (g - x r mean_d(g x r)),
+//             dw_d += u_d x_d r   (per tensor, fixed-order partials + column reduction)
+// Lanes of one head (D*size/16 of them, a power of two <= 32) reduce with xor shuffles.
+#include "gn_host.h"
+#include "row_pipe.cuh"
+
+namespace gn {
+namespace {
+
+enum Mode { ROPE = 0, QK_FWD = 1, QK_BWD = 2 };
+
+constexpr int kRopeMaxThreads = 512;
+
+struct RopeArgs {
+  const void* x[2];   // q, k inputs (k may be null: one tensor)
+  const void* dy[2];  // QK_BWD: gradients of the outputs
+  void* out[2];       // outputs (ROPE: == x, in place)
+  const void* w[2];   // QK: weights [D]
+  float* stat[2];     // QK_FWD: inv_rms out; QK_BWD: inv_rms in (cast)
+  const float* cos;
+  const float* sin;
+  float* ws;          // QK_BWD: [gridDim.x][2*D] partial dw, or null
+  int B, S, H, D, HC, NC;  // NC = H / HC slabs per token
+  int ntens;               // 1 or 2
+  int stages;
+  float eps;
+  float sign;
+  uint32_t units;          // B * S * NC
+  uint32_t tslot, tabslot; // bytes of one tensor slot / the table slot in a stage
+  unsigned* err;
+};
+
+__host__ __device__ inline uint32_t round128(uint32_t v) { return (v + 127u) / 128u * 128u; }
+
+template <typename T, int VPT, int MODE, bool GEMMA>
+__global__ void __launch_bounds__(kRopeMaxThreads) rope_kernel(const RopeArgs a) {
+  using V = Vec<T>;
+  constexpr int E = V::N;      // elements per vector
+  constexpr int P = E / 2;     // pairs per vector
+  constexpr bool BWD = MODE == QK_BWD;
+  constexpr bool NORM = MODE != ROPE;
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem);
+  uint8_t* data = smem + 128;
+  const int tid = threadIdx.x, NT = blockDim.x;
+  const int D = a.D, HC = a.HC, lph = D / E;          // lanes (vectors) per head
+  const int nv_t = HC * lph;                          // vectors per tensor slab
+  const int NV = a.ntens * nv_t;
+  const uint32_t nslots = (uint32_t)a.ntens * (BWD ? 2u : 1u);
+  const uint32_t sstride = nslots * a.tslot + a.tabslot;
+  const uint32_t slab_bytes = (uint32_t)(HC * D * (int)sizeof(T));
+  const uint32_t tab_bytes = (uint32_t)(D / 2 * 4);
+  const int64_t step = gridDim.x;
+
+  // this thread's vectors: tensor, head within the slab, element offset within the slab
+  int tt[VPT], hh[VPT], off[VPT];
+  bool valid[VPT];
+#pragma unroll
+  for (int j = 0; j < VPT; ++j) {
+    const int v = tid + j * NT;
+    valid[j] = v < NV;
+    const int vv = valid[j] ? v : 0;
+    tt[j] = vv / nv_t;
+    const int w = vv - tt[j] * nv_t;
+    hh[j] = w / lph;
+    off[j] = w * E;
+  }
+  const int li = tid % lph;  // lane within the head (same for every j when NORM)
+  float wq[E], wk[E];
+  if constexpr (NORM) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int d = li * E + e;
+      wq[e] = (GEMMA ? 1.0f : 0.0f) + Vec<T>::load1(static_cast<const T*>(a.w[0]) + d);
+      wk[e] = a.ntens > 1 ? (GEMMA ? 1.0f : 0.0f) + Vec<T>::load1(static_cast<const T*>(a.w[1]) + d) : 0.0f;
+    }
+  }
+  float dwa[2][E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) dwa[0][e] = dwa[1][e] = 0.0f;
+
+  auto unit_origin = [&](uint32_t u, int64_t& bs, int& c, int& s) {
+    c = (int)(u % (uint32_t)a.NC);
+    const uint32_t t2 = u / (uint32_t)a.NC;
+    const int b = (int)(t2 % (uint32_t)a.B);
+    s = (int)(t2 / (uint32_t)a.B);
+    bs = (int64_t)b * a.S + s;
+  };
+  auto issue = [&](int st, uint32_t u) {
+    int64_t bs;
+    int c, s;
+    unit_origin(u, bs, c, s);
+    const int64_t eoff = (bs * a.H + (int64_t)c * HC) * D;
+    uint8_t* sb = data + (size_t)st * sstride;
+    mbar_expect_tx(&bar[st], nslots * slab_bytes + 2 * tab_bytes);
+    for (int t = 0; t < a.ntens; ++t) {
+      bulk_g2s(sb + t * a.tslot, static_cast<const T*>(a.x[t]) + eoff, slab_bytes, &bar[st]);
+      if constexpr (BWD)
+        bulk_g2s(sb + (a.ntens + t) * a.tslot, static_cast<const T*>(a.dy[t]) + eoff, slab_bytes, &bar[st]);
+    }
+    uint8_t* tb = sb + nslots * a.tslot;
+    bulk_g2s(tb, a.cos + (int64_t)s * (D / 2), tab_bytes, &bar[st]);
+    bulk_g2s(tb + tab_bytes, a.sin + (int64_t)s * (D / 2), tab_bytes, &bar[st]);
+  };
+
+  if (tid == 0) {
+    for (int st = 0; st < a.stages; ++st) mbar_init(&bar[st], 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    uint32_t u = blockIdx.x;
+    for (int st = 0; st < a.stages && u < a.units; ++st, u += (uint32_t)step) issue(st, u);
+  }
+
+  const float inv_d = 1.0f / (float)D;
+  int st = 0;
+  uint32_t ph = 0;
+  for (uint32_t u = blockIdx.x; u < a.units; u += (uint32_t)step) {
+    int64_t bs;
+    int c, s;
+    unit_origin(u, bs, c, s);
+    const int64_t row0 = bs * a.H + (int64_t)c * HC;  // first head row of the unit
+    const int64_t eoff = row0 * D;
+    float rin[VPT];
+    if constexpr (BWD) {
+#pragma unroll
+      for (int j = 0; j < VPT; ++j) rin[j] = valid[j] ? __ldg(a.stat[tt[j]] + row0 + hh[j]) : 0.0f;
+    }
+    const bool ok = mbar_wait(&bar[st], ph, a.err);
+    const uint8_t* sb = data + (size_t)st * sstride;
+    const float* tcos = reinterpret_cast<const float*>(sb + nslots * a.tslot);
+    const float* tsin = tcos + D / 2;
+    float xv[VPT][E], gv[VPT][E], cs[VPT][P], sn[VPT][P];
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      if (valid[j]) {
+        V::unpack(*reinterpret_cast<const uint4*>(sb + tt[j] * a.tslot + off[j] * sizeof(T)), xv[j]);
+        if constexpr (BWD)
+          V::unpack(*reinterpret_cast<const uint4*>(sb + (a.ntens + tt[j]) * a.tslot + off[j] * sizeof(T)), gv[j]);
+        const int p0 = (off[j] % D) / 2;
+#pragma unroll
+        for (int p = 0; p < P; ++p) {
+          cs[j][p] = tcos[p0 + p];
+          sn[j][p] = tsin[p0 + p];
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) xv[j][e] = gv[j][e] = 0.0f;
+#pragma unroll
+        for (int p = 0; p < P; ++p) cs[j][p] = sn[j][p] = 0.0f;
+      }
+    }
+    // every thread has read the stage: release it and refill it with the unit `stages` ahead
+    if (__syncthreads_or(!ok)) {
+      if (tid == 0) {
+        uint32_t uu = u;
+        int s2 = st;
+        uint32_t p2 = ph;
+        for (int k = 0; k < a.stages && uu < a.units; ++k, uu += (uint32_t)step) {
+          (void)mbar_wait(&bar[s2], p2, a.err);
+          if (++s2 == a.stages) s2 = 0, p2 ^= 1u;
+        }
+      }
+      return;
+    }
+    if (tid == 0 && (uint64_t)u + (uint64_t)a.stages * step < a.units) issue(st, u + (uint32_t)(a.stages * step));
+    if (++st == a.stages) st = 0, ph ^= 1u;
+
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      float o[E];
+      if constexpr (MODE == ROPE) {
+#pragma unroll
+        for (int p = 0; p < P; ++p) {
+          const float x0 = xv[j][2 * p], x1 = xv[j][2 * p + 1];
+          const float si = a.sign * sn[j][p];
+          o[2 * p] = fmaf(x0, cs[j][p], -x1 * si);
+          o[2 * p + 1] = fmaf(x0, si, x1 * cs[j][p]);
+        }
+      } else if constexpr (MODE == QK_FWD) {
+        float ss = 0.0f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) ss = fmaf(xv[j][e], xv[j][e], ss);
+        ss = group_sum_rt(ss, lph);
+        const float r = rsqrtf(fmaf(ss, inv_d, a.eps));
+        float n[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) n[e] = xv[j][e] * r * (tt[j] ? wk[e] : wq[e]);
+#pragma unroll
+        for (int p = 0; p < P; ++p) {
+          o[2 * p] = fmaf(n[2 * p], cs[j][p], -n[2 * p + 1] * sn[j][p]);
+          o[2 * p + 1] = fmaf(n[2 * p], sn[j][p], n[2 * p + 1] * cs[j][p]);
+        }
+        if (li == 0 && valid[j] && a.stat[tt[j]]) a.stat[tt[j]][row0 + hh[j]] = r;
+      } else {  // QK_BWD
+        const float r = rin[j];
+        float g[E];
+#pragma unroll
+        for (int p = 0; p < P; ++p) {  // inverse rotation of the output gradient
+          const float d0 = gv[j][2 * p], d1 = gv[j][2 * p + 1];
+          g[2 * p] = fmaf(d0, cs[j][p], d1 * sn[j][p]);
+          g[2 * p + 1] = fmaf(-d0, sn[j][p], d1 * cs[j][p]);
+        }
+        float cdot = 0.0f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const float xh = xv[j][e] * r;
+          const float wv = tt[j] ? wk[e] : wq[e];
+          cdot = fmaf(g[e] * wv, xh, cdot);
+          if (valid[j]) {
+            if (tt[j]) dwa[1][e] = fmaf(g[e], xh, dwa[1][e]);
+            else dwa[0][e] = fmaf(g[e], xh, dwa[0][e]);
+          }
+        }
+        cdot = group_sum_rt(cdot, lph) * inv_d;
+#pragma unroll
+        for (int e = 0; e < E; ++e) o[e] = r * fmaf(g[e], tt[j] ? wk[e] : wq[e], -(xv[j][e] * r) * cdot);
+      }
+      if (valid[j]) st_stream(static_cast<T*>(a.out[tt[j]]) + eoff + off[j], V::pack(o));
+    }
+  }
+
+  if constexpr (BWD) {
+    if (!a.ws) return;
+    // combine the per-thread partials of the CTA in thread order (stages are idle now)
+    __syncthreads();
+    float* red = reinterpret_cast<float*>(data);  // [NT][2][E]
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      red[(tid * 2 + 0) * E + e] = dwa[0][e];
+      red[(tid * 2 + 1) * E + e] = dwa[1][e];
+    }
+    __syncthreads();
+    float* part = a.ws + (int64_t)blockIdx.x * 2 * D;
+    for (int col = tid; col < 2 * D; col += NT) {
+      const int t = col / D, d = col - t * D, l = d / E, e = d - l * E;
+      float acc = 0.0f;
+      for (int th = l; th < NT; th += lph) acc += red[(th * 2 + t) * E + e];
+      part[col] = acc;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- planning
+
+struct RopePlan {
+  int HC, NC, vpt, threads, stages;
+  uint32_t tslot, tabslot;
+  size_t smem;
+};
+
+gn_status plan_rope(int64_t B, int64_t S, int64_t H, int64_t D, int ntens, int mode, size_t es, RopePlan* p) {
+  const int vec = (int)(16 / es);
+  const int lph = (int)(D / vec);
+  const int nslots = ntens * (mode == QK_BWD ? 2 : 1);
+  const int64_t budget = g_tune.unit_bytes ? g_tune.unit_bytes : 24 * 1024;
+  // the backward holds x, dy and the table values of each vector: two vectors per thread
+  const int vpt = g_tune.vpt ? (g_tune.vpt > 4 ? 4 : g_tune.vpt) : (mode == QK_BWD ? 2 : 4);
+  int HC = 0;
+  for (int hc = (int)H; hc >= 1; --hc) {
+    if (H % hc) continue;
+    const int64_t nv = (int64_t)ntens * hc * lph;
+    if ((nv + vpt - 1) / vpt > kRopeMaxThreads) continue;
+    if ((int64_t)nslots * hc * D * (int64_t)es > budget && hc > 1) continue;
+    HC = hc;
+    break;
+  }
+  if (HC == 0) return GN_ERR_UNSUPPORTED;
+  p->HC = HC;
+  p->NC = (int)(H / HC);
+  p->vpt = vpt;
+  const int64_t nv = (int64_t)ntens * HC * lph;
+  p->threads = (int)(((nv + vpt - 1) / vpt + 31) / 32 * 32);
+  if (p->threads > kRopeMaxThreads) return GN_ERR_UNSUPPORTED;
+  p->tslot = round128((uint32_t)(HC * D * (int64_t)es));
+  p->tabslot = round128((uint32_t)(D * 4));
+  const size_t sstride = (size_t)nslots * p->tslot + p->tabslot;
+  int stages = g_tune.stages ? g_tune.stages : (int)(96 * 1024 / sstride);
+  stages = stages < 2 ? 2 : stages > 8 ? 8 : stages;
+  const size_t limit = smem_optin();
+  while (stages > 1 && 128 + stages * sstride > limit) --stages;
+  p->stages = stages;
+  p->smem = 128 + stages * sstride;
+  // the backward reuses the stages for the [threads][2][vec] partial-sum table
+  const size_t red = (size_t)p->threads * 2 * vec * 4;
+  if (mode == QK_BWD && red > stages * sstride) p->smem = 128 + red;
+  if (p->smem > limit) return GN_ERR_UNSUPPORTED;
+  if (B * S * p->NC >= (int64_t)1 << 31) return GN_ERR_UNSUPPORTED;
+  return GN_OK;
+}
+
+template <typename T, int MODE>
+void* pick_rope(int vpt, bool gemma) {
+#define GN_V(V_)                                                       \
+  if (vpt == V_) {                                                     \
+    return gemma ? (void*)rope_kernel<T, V_, MODE, (MODE != ROPE)>     \
+                 : (void*)rope_kernel<T, V_, MODE, false>;             \
+  }
+  GN_V(1) GN_V(2) GN_V(4)
+#undef GN_V
+  return nullptr;
+}
+
+void* pick(gn_dtype dt, int mode, int vpt, bool gemma) {
+  if (dt == GN_BF16) {
+    if (mode == ROPE) return pick_rope<__nv_bfloat16, ROPE>(vpt, false);
+    if (mode == QK_FWD) return pick_rope<__nv_bfloat16, QK_FWD>(vpt, gemma);
+    return pick_rope<__nv_bfloat16, QK_BWD>(vpt, gemma);
+  }
+  if (mode == ROPE) return pick_rope<float, ROPE>(vpt, false);
+  if (mode == QK_FWD) return pick_rope<float, QK_FWD>(vpt, gemma);
+  return pick_rope<float, QK_BWD>(vpt, gemma);
+}
+
+gn_status setup(int64_t B, int64_t S, int64_t H, int64_t D, int ntens, int mode, gn_dtype dt, bool gemma,
+                RopePlan* p, void** kern, int* grid) {
+  gn_status st = plan_rope(B, S, H, D, ntens, mode, dt_size(dt), p);
+  if (st != GN_OK) return st;
+  *kern = pick(dt, mode, p->vpt, gemma);
+  if (!*kern) return GN_ERR_UNSUPPORTED;
+  const int cap = g_tune.ctas_per_sm ? g_tune.ctas_per_sm : 8;
+  int g = persistent_grid(*kern, p->threads, p->smem, cap);
+  if (g <= 0) return GN_ERR_CUDA;
+  const int64_t units = B * S * p->NC;
+  if (units < g) g = (int)(units > 0 ? units : 1);
+  *grid = g;
+  return GN_OK;
+}
+
+gn_status check_common(int64_t B, int64_t S, int64_t H, int64_t D, gn_dtype dt) {
+  if (!dt_ok(dt)) return GN_ERR_DTYPE;
+  if (B < 0 || S < 0 || H < 0 || D <= 0 || D % 8 || D > 4096) return GN_ERR_SHAPE;
+  return GN_OK;
+}
+
+bool norm_head_ok(int64_t D, gn_dtype dt) {
+  const int64_t lph = D * (int64_t)dt_size(dt) / 16;
+  return lph >= 1 && lph <= 32 && (lph & (lph - 1)) == 0;
+}
+
+gn_status launch(void* kern, int grid, const RopePlan& p, RopeArgs& a, cudaStream_t s) {
+  a.HC = p.HC;
+  a.NC = p.NC;
+  a.stages = p.stages;
+  a.tslot = p.tslot;
+  a.tabslot = p.tabslot;
+  a.units = (uint32_t)((int64_t)a.B * a.S * p.NC);
+  a.err = device_err_word();
+  if (!a.err) return GN_ERR_CUDA;
+  void* args[] = {&a};
+  if (cudaLaunchKernel(kern, dim3(grid), dim3(p.threads), args, p.smem, s) != cudaSuccess) return GN_ERR_CUDA;
+  count_launches(1);
+  return launch_status();
+}
+
+}  // namespace
+}  // namespace gn
+
+using namespace gn;
+
+extern "C" gn_status gn_rope_apply_inplace(void* q, void* k, const float* cos, const float* sin, int64_t B,
+                                           int64_t S, int64_t H, int64_t D, int sign, gn_dtype dt,
+                                           void* stream) {
+  gn_status st = check_common(B, S, H, D, dt);
+  if (st != GN_OK) return st;
+  if (sign != 1 && sign != -1) return GN_ERR_SHAPE;
+  if (B * S * H == 0) return GN_OK;
+  if (!q || !cos || !sin) return GN_ERR_NULL;
+  if (!aligned16(q) || (k && !aligned16(k)) || !aligned16(cos) || !aligned16(sin)) return GN_ERR_ALIGN;
+  const int ntens = k ? 2 : 1;
+  RopePlan p;
+  void* kern = nullptr;
+  int grid = 0;
+  if ((st = setup(B, S, H, D, ntens, ROPE, dt, false, &p, &kern, &grid)) != GN_OK) return st;
+  RopeArgs a{};
+  a.x[0] = q;
+  a.x[1] = k;
+  a.out[0] = q;
+  a.out[1] = k;
+  a.cos = cos;
+  a.sin = sin;
+  a.B = (int)B, a.S = (int)S, a.H = (int)H, a.D = (int)D;
+  a.ntens = ntens;
+  a.sign = (float)sign;
+  return launch(kern, grid, p, a, (cudaStream_t)stream);
+}
+
+extern "C" gn_status gn_qknorm_rope_fwd(const void* q, const void* k, const void* wq, const void* wk,
+                                        const float* cos, const float* sin, void* q_out, void* k_out,
+                                        float* inv_rms_q, float* inv_rms_k, int64_t B, int64_t S, int64_t H,
+                                        int64_t D, float eps, int gemma, gn_dtype dt, void* stream) {
+  gn_status st = check_common(B, S, H, D, dt);
+  if (st != GN_OK) return st;
+  if (!norm_head_ok(D, dt)) return GN_ERR_UNSUPPORTED;
+  if (B * S * H == 0) return GN_OK;
+  if (!q || !wq || !cos || !sin || !q_out) return GN_ERR_NULL;
+  if (k && (!wk || !k_out)) return GN_ERR_NULL;
+  if (!aligned16(q) || !aligned16(q_out) || (k && (!aligned16(k) || !aligned16(k_out))) || !aligned16(cos) ||
+      !aligned16(sin))
+    return GN_ERR_ALIGN;
+  const int ntens = k ? 2 : 1;
+  RopePlan p;
+  void* kern = nullptr;
+  int grid = 0;
+  if ((st = setup(B, S, H, D, ntens, QK_FWD, dt, gemma != 0, &p, &kern, &grid)) != GN_OK) return st;
+  RopeArgs a{};
+  a.x[0] = q, a.x[1] = k;
+  a.out[0] = q_out, a.out[1] = k_out;
+  a.w[0] = wq, a.w[1] = wk;
+  a.stat[0] = inv_rms_q, a.stat[1] = inv_rms_k;
+  a.cos = cos, a.sin = sin;
+  a.B = (int)B, a.S = (int)S, a.H = (int)H, a.D = (int)D;
+  a.ntens = ntens;
+  a.eps = eps;
+  a.sign = 1.0f;
+  return launch(kern, grid, p, a, (cudaStream_t)stream);
+}
+
+extern "C" size_t gn_qknorm_rope_bwd_workspace(int64_t B, int64_t S, int64_t H, int64_t D, gn_dtype dt) {
+  if (check_common(B, S, H, D, dt) != GN_OK || !norm_head_ok(D, dt) || B * S * H == 0) return 0;
+  RopePlan p;
+  void* kern = nullptr;
+  int grid = 0;
+  if (setup(B, S, H, D, 2, QK_BWD, dt, false, &p, &kern, &grid) != GN_OK) return 0;
+  // sized for two tensors; a call with k == NULL uses no more
+  return (size_t)grid * 2 * (size_t)D * sizeof(float);
+}
+
+extern "C" gn_status gn_qknorm_rope_bwd(const void* q, const void* k, const void* wq, const void* wk,
+                                        const float* cos, const float* sin, const float* inv_rms_q,
+                                        const float* inv_rms_k, const void* dq_out, const void* dk_out, void* dq,
+                                        void* dk, float* dwq, float* dwk, void* ws, size_t ws_bytes, int64_t B,
+                                        int64_t S, int64_t H, int64_t D, int gemma, gn_dtype dt, void* stream) {
+  gn_status st = check_common(B, S, H, D, dt);
+  if (st != GN_OK) return st;
+  if (!norm_head_ok(D, dt)) return GN_ERR_UNSUPPORTED;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (B * S * H == 0) {
+    if (dwq && cudaMemsetAsync(dwq, 0, (size_t)D * sizeof(float), s) != cudaSuccess) return GN_ERR_CUDA;
+    if (dwk && cudaMemsetAsync(dwk, 0, (size_t)D * sizeof(float), s) != cudaSuccess) return GN_ERR_CUDA;
+    return GN_OK;
+  }
+  if (!q || !wq || !cos || !sin || !inv_rms_q || !dq_out || !dq) return GN_ERR_NULL;
+  if (k && (!wk || !inv_rms_k || !dk_out || !dk)) return GN_ERR_NULL;
+  if (!aligned16(q) || !aligned16(dq_out) || !aligned16(dq) || !aligned16(cos) || !aligned16(sin) ||
+      (k && (!aligned16(k) || !aligned16(dk_out) || !aligned16(dk))))
+    return GN_ERR_ALIGN;
+  const int ntens = k ? 2 : 1;
+  RopePlan p;
+  void* kern = nullptr;
+  int grid = 0;
+  if ((st = setup(B, S, H, D, ntens, QK_BWD, dt, gemma != 0, &p, &kern, &grid)) != GN_OK) return st;
+  const bool wgrad = dwq || (k && dwk);
+  if (wgrad) {
+    if (!ws) return GN_ERR_WORKSPACE;
+    if (!aligned16(ws)) return GN_ERR_ALIGN;
+    if (ws_bytes < (size_t)grid * 2 * (size_t)D * sizeof(float)) return GN_ERR_WORKSPACE;
+  }
+  RopeArgs a{};
+  a.x[0] = q, a.x[1] = k;
+  a.dy[0] = dq_out, a.dy[1] = dk_out;
+  a.out[0] = dq, a.out[1] = dk;
+  a.w[0] = wq, a.w[1] = wk;
+  a.stat[0] = const_cast<float*>(inv_rms_q), a.stat[1] = const_cast<float*>(inv_rms_k);
+  a.cos = cos, a.sin = sin;
+  a.ws = wgrad ? static_cast<float*>(ws) : nullptr;
+  a.B = (int)B, a.S = (int)S, a.H = (int)H, a.D = (int)D;
+  a.ntens = ntens;
+  a.sign = 1.0f;
+  if ((st = launch(kern, grid, p, a, s)) != GN_OK) return st;
+  if (wgrad) return launch_colsum(a.ws, grid, 2 * D, D, dwq, k ? dwk : nullptr, s);
+  return GN_OK;
+}
