@@ -110,57 +110,76 @@ def workload_config(z, l2_note=True):
     }
 
 
-def gen_inputs(z, seed):
+FAMILY = {"rmsnorm_fwd": "rms", "rmsnorm_gemma_fwd": "rms", "rmsnorm_bwd": "rms", "rmsnorm_gemma_bwd": "rms",
+          "layernorm_fwd": "ln", "layernorm_bwd": "ln", "rope_fwd": "rope", "rope_bwd": "rope",
+          "qknorm_rope_fwd": "qk", "qknorm_rope_bwd": "qk"}
+
+
+def gen_inputs(z, seed, families=("rms", "ln", "rope", "qk")):
     r, l, o, q = z["rms"], z["ln"], z["rope"], z["qk"]
-    d = {"rms": wl.rmsnorm(M=r["M"], N=r["N"], dtype="bf16", seed=seed)}
-    d["rms_gemma_w"] = wl.normal(seed, wl.S_W, r["N"], "bf16", scale=0.1)
-    d["ln"] = wl.layernorm(M=l["M"], N=l["N"], dtype="bf16", seed=seed)
-    d["rope"] = wl.rope(**o, dtype="bf16", seed=seed)
-    d["qk"] = wl.qknorm_rope(**q, dtype="bf16", seed=seed)
+    d = {}
+    if "rms" in families:
+        d["rms"] = wl.rmsnorm(M=r["M"], N=r["N"], dtype="bf16", seed=seed)
+        d["rms_gemma_w"] = wl.normal(seed, wl.S_W, r["N"], "bf16", scale=0.1)
+    if "ln" in families:
+        d["ln"] = wl.layernorm(M=l["M"], N=l["N"], dtype="bf16", seed=seed)
+    if "rope" in families:
+        d["rope"] = wl.rope(**o, dtype="bf16", seed=seed)
+    if "qk" in families:
+        d["qk"] = wl.qknorm_rope(**q, dtype="bf16", seed=seed)
     return d
 
 
 # ---------------------------------------------------------------- our arm
 
 class Suite:
-    """Device buffers and C-ABI launch closures for one step of the path."""
+    """Device buffers and C-ABI launch closures for one step of the path (only the workloads
+    of the selected kernels are generated and allocated)."""
 
-    def __init__(self, gn, torch, z, host, dev):
+    def __init__(self, gn, torch, z, host, dev, kernels):
         self.gn, self.torch, self.z, self.dev = gn, torch, z, dev
+        fams = {FAMILY[k] for k in kernels}
         T = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)  # noqa
         F = lambda a: torch.from_numpy(np.ascontiguousarray(a))  # noqa: E731
-        self.h = {  # host tensors (pageable); inputs of the step
-            "rx": T(host["rms"]["x"]), "rdy": T(host["rms"]["dy"]), "rw": T(host["rms"]["w"]),
-            "rwg": T(host["rms_gemma_w"]),
-            "lx": T(host["ln"]["x"]), "ldy": T(host["ln"]["dy"]), "lw": T(host["ln"]["w"]), "lb": T(host["ln"]["b"]),
-            "oq": T(host["rope"]["q"]), "ok": T(host["rope"]["k"]), "ocos": F(host["rope"]["cos"]),
-            "osin": F(host["rope"]["sin"]),
-            "qq": T(host["qk"]["q"]), "qk": T(host["qk"]["k"]), "qwq": T(host["qk"]["wq"]), "qwk": T(host["qk"]["wk"]),
-            "qcos": F(host["qk"]["cos"]), "qsin": F(host["qk"]["sin"]), "qdq": T(host["qk"]["dq_out"]),
-            "qdk": T(host["qk"]["dk_out"]),
-        }
-        self.inputs = list(self.h)
-        self.d = {k: v.to(dev) for k, v in self.h.items()}
-        E = lambda ref, dt=None: torch.empty_like(ref) if dt is None else torch.empty(ref.shape[:-1], dtype=dt, device=dev)  # noqa
-        d = self.d
+        h = {}  # host tensors (pageable): the inputs of the step
+        if "rms" in fams:
+            r = host["rms"]
+            h.update(rx=T(r["x"]), rdy=T(r["dy"]), rw=T(r["w"]), rwg=T(host["rms_gemma_w"]))
+        if "ln" in fams:
+            l = host["ln"]  # noqa: E741
+            h.update(lx=T(l["x"]), ldy=T(l["dy"]), lw=T(l["w"]), lb=T(l["b"]))
+        if "rope" in fams:
+            o = host["rope"]
+            h.update(oq=T(o["q"]), ok=T(o["k"]), ocos=F(o["cos"]), osin=F(o["sin"]))
+        if "qk" in fams:
+            q = host["qk"]
+            h.update(qq=T(q["q"]), qk=T(q["k"]), qwq=T(q["wq"]), qwk=T(q["wk"]), qcos=F(q["cos"]),
+                     qsin=F(q["sin"]), qdq=T(q["dq_out"]), qdk=T(q["dk_out"]))
+        self.h = h
+        self.inputs = list(h)
+        self.d = d = {k: v.to(dev) for k, v in h.items()}
         f32 = torch.float32
-        d.update({
-            "ry": E(d["rx"]), "rr": E(d["rx"], f32), "rdx": E(d["rx"]), "rdw": torch.empty(z["rms"]["N"], dtype=f32, device=dev),
-            "ryg": E(d["rx"]), "rrg": E(d["rx"], f32), "rdxg": E(d["rx"]), "rdwg": torch.empty(z["rms"]["N"], dtype=f32, device=dev),
-            "ly": E(d["lx"]), "lmu": E(d["lx"], f32), "lrs": E(d["lx"], f32), "ldx": E(d["lx"]),
-            "ldw": torch.empty(z["ln"]["N"], dtype=f32, device=dev), "ldb": torch.empty(z["ln"]["N"], dtype=f32, device=dev),
-            "qqo": E(d["qq"]), "qko": E(d["qk"]), "qrq": E(d["qq"], f32), "qrk": E(d["qk"], f32),
-            "qdxq": E(d["qq"]), "qdxk": E(d["qk"]), "qdwq": torch.empty(128, dtype=f32, device=dev),
-            "qdwk": torch.empty(128, dtype=f32, device=dev),
-        })
+        E = lambda ref, dt=None: torch.empty_like(ref) if dt is None else torch.empty(ref.shape[:-1], dtype=dt, device=dev)  # noqa
+        V = lambda n: torch.empty(n, dtype=f32, device=dev)  # noqa: E731
+        if "rms" in fams:
+            N = z["rms"]["N"]
+            d.update(ry=E(d["rx"]), rr=E(d["rx"], f32), rdx=E(d["rx"]), rdw=V(N), ryg=E(d["rx"]), rrg=E(d["rx"], f32),
+                     rdxg=E(d["rx"]), rdwg=V(N))
+        if "ln" in fams:
+            N = z["ln"]["N"]
+            d.update(ly=E(d["lx"]), lmu=E(d["lx"], f32), lrs=E(d["lx"], f32), ldx=E(d["lx"]), ldw=V(N), ldb=V(N))
+        if "qk" in fams:
+            d.update(qqo=E(d["qq"]), qko=E(d["qk"]), qrq=E(d["qq"], f32), qrk=E(d["qk"], f32), qdxq=E(d["qq"]),
+                     qdxk=E(d["qk"]), qdwq=V(z["qk"]["D"]), qdwk=V(z["qk"]["D"]))
         r, l, q = z["rms"], z["ln"], z["qk"]
-        self.ws_r = gn.gn_rmsnorm_bwd_workspace(r["M"], r["N"], gn.GN_BF16)
-        self.ws_l = gn.gn_layernorm_bwd_workspace(l["M"], l["N"], gn.GN_BF16)
-        self.ws_q = gn.gn_qknorm_rope_bwd_workspace(q["B"], q["S"], q["H"], q["D"], gn.GN_BF16)
+        self.ws_r = gn.gn_rmsnorm_bwd_workspace(r["M"], r["N"], gn.GN_BF16) if "rms" in fams else 0
+        self.ws_l = gn.gn_layernorm_bwd_workspace(l["M"], l["N"], gn.GN_BF16) if "ln" in fams else 0
+        self.ws_q = gn.gn_qknorm_rope_bwd_workspace(q["B"], q["S"], q["H"], q["D"], gn.GN_BF16) if "qk" in fams else 0
         self.ws = torch.empty(max(self.ws_r, self.ws_l, self.ws_q, 16), dtype=torch.uint8, device=dev)
         # outputs read back by the end-to-end measurement (final value of each output tensor)
-        self.outputs = ["ry", "rr", "rdx", "rdw", "ryg", "rrg", "rdxg", "rdwg", "ly", "lmu", "lrs", "ldx", "ldw",
-                        "ldb", "oq", "ok", "qqo", "qko", "qrq", "qrk", "qdxq", "qdxk", "qdwq", "qdwk"]
+        self.outputs = [k for k in ("ry", "rr", "rdx", "rdw", "ryg", "rrg", "rdxg", "rdwg", "ly", "lmu", "lrs", "ldx",
+                                    "ldw", "ldb", "oq", "ok", "qqo", "qko", "qrq", "qrk", "qdxq", "qdxk", "qdwq",
+                                    "qdwk") if k in d]
         self.stream = torch.cuda.current_stream(dev)
 
     def launch(self, name):
@@ -335,8 +354,8 @@ def run_ours(args):
     gn.load()
     z = sizes(args.scale)
     kernels = [k for k in ORDER if not args.only or k in args.only.split(",")]
-    host = gen_inputs(z, args.seed + rank)
-    suite = Suite(gn, torch, z, host, dev)
+    host = gen_inputs(z, args.seed + rank, {FAMILY[k] for k in kernels})
+    suite = Suite(gn, torch, z, host, dev, kernels)
     nbytes = algorithmic_bytes(z)
     step_bytes = sum(nbytes[k] for k in kernels)
     # the backward kernels read the forward statistics: run each forward once before timing
@@ -533,7 +552,7 @@ def run_reference(args):
         return
     z = sizes(args.scale)
     kernels = [k for k in ORDER if not args.only or k in args.only.split(",")]
-    host = gen_inputs(z, args.seed)
+    host = gen_inputs(z, args.seed, {FAMILY[k] for k in kernels})
     # size each step's sample so that warmup + steps stay within about two minutes
     t, _ = oracle_step(host, z, kernels, 1.0 / 8192)
     frac = (1.0 / 8192) * max(1.0, min(64.0, 120.0 / max(1, args.steps + args.warmup) / max(t, 1e-3)))

@@ -5,11 +5,16 @@
 // q and k together, section "基准实测").
 //
 // One kernel template serves the three operations. The work unit is a slab of HC consecutive
-// heads of one token (b, s) of q and of k: HC*D contiguous elements per tensor. A persistent
-// CTA walks the units grid-stride; each unit's slabs and its cos/sin table rows arrive in a
-// shared-memory stage through 1-D TMA bulk copies (multi-stage pipeline, bounded waits).
-// Units are ordered token-major, so the table row of token s is fetched by neighbouring CTAs
-// at about the same time and HBM delivers it once per token.
+// heads of one token (b, s) of q and of k: HC*D contiguous elements per tensor, plus the
+// token's cos/sin table rows. A persistent CTA is warp-specialised:
+//   * warp 0 (one lane) is the producer: it walks the CTA's units grid-stride and moves each
+//     unit into a shared-memory stage with 1-D TMA bulk copies, counted on the stage's `full`
+//     mbarrier; before reusing a stage it waits on the stage's `empty` mbarrier;
+//   * the other C warps are consumers: they wait on `full`, compute straight from shared
+//     memory one 16-byte vector at a time (few live registers, so several CTAs share an SM),
+//     store the results with 16-byte streaming stores, and each warp arrives on `empty`.
+// No CTA-wide barrier sits on the per-unit path. Units are ordered token-major, so the table
+// row of token s is fetched by neighbouring CTAs at about the same time. Every wait is bounded.
 //
 //   ROPE    : x <- rot(x, cos, sign*sin)                                   (in place)
 //   QK_FWD  : r = rsqrt(mean_d x^2 + eps), out = rot(x r w', cos, sin), inv_rms = r
@@ -24,7 +29,9 @@ namespace {
 
 enum Mode { ROPE = 0, QK_FWD = 1, QK_BWD = 2 };
 
-constexpr int kRopeMaxThreads = 512;
+constexpr int kMaxConsumerWarps = 10;
+constexpr int kRopeMaxThreads = 32 * (1 + kMaxConsumerWarps);
+constexpr int kRopeMaxStages = 8;
 
 struct RopeArgs {
   const void* x[2];   // q, k inputs (k may be null: one tensor)
@@ -38,6 +45,7 @@ struct RopeArgs {
   int B, S, H, D, HC, NC;  // NC = H / HC slabs per token
   int ntens;               // 1 or 2
   int stages;
+  int lph_shift;           // log2(lanes per head) when that is a power of two, else -1
   float eps;
   float sign;
   uint32_t units;          // B * S * NC
@@ -47,211 +55,235 @@ struct RopeArgs {
 
 __host__ __device__ inline uint32_t round128(uint32_t v) { return (v + 127u) / 128u * 128u; }
 
-template <typename T, int VPT, int MODE, bool GEMMA>
-__global__ void __launch_bounds__(kRopeMaxThreads) rope_kernel(const RopeArgs a) {
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+// named barrier 1 over the consumer warps only (the producer warp never joins it)
+__device__ __forceinline__ void consumers_sync(int nthreads) {
+  asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+}
+
+// OR of `pred` over the consumer warps (named barrier 2)
+__device__ __forceinline__ int consumers_any(int nthreads, int pred) {
+  int r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.s32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 2, %2, p;\n\t"
+      "selp.s32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(pred), "r"(nthreads)
+      : "memory");
+  return r;
+}
+
+__device__ __forceinline__ void unit_origin(const RopeArgs& a, uint32_t u, int64_t& bs, int& c, int& s) {
+  c = (int)(u % (uint32_t)a.NC);
+  const uint32_t t2 = u / (uint32_t)a.NC;
+  const int b = (int)(t2 % (uint32_t)a.B);
+  s = (int)(t2 / (uint32_t)a.B);
+  bs = (int64_t)b * a.S + s;
+}
+
+template <typename T, int MODE, bool GEMMA>
+__global__ void __launch_bounds__(kRopeMaxThreads, 2) rope_kernel(const RopeArgs a) {
   using V = Vec<T>;
-  constexpr int E = V::N;      // elements per vector
+  constexpr int E = V::N;      // elements per 16-byte vector
   constexpr int P = E / 2;     // pairs per vector
   constexpr bool BWD = MODE == QK_BWD;
   constexpr bool NORM = MODE != ROPE;
   extern __shared__ __align__(128) uint8_t smem[];
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+  uint64_t* empty = full + kRopeMaxStages;
   uint8_t* data = smem + 128;
-  const int tid = threadIdx.x, NT = blockDim.x;
-  const int D = a.D, HC = a.HC, lph = D / E;          // lanes (vectors) per head
-  const int nv_t = HC * lph;                          // vectors per tensor slab
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ncw = (int)(blockDim.x >> 5) - 1;  // consumer warps
+  const int D = a.D, HC = a.HC;
+  const int lph = D / E;                       // vectors (lanes) per head
+  const int nv_t = HC * lph;                   // vectors per tensor slab
   const int NV = a.ntens * nv_t;
   const uint32_t nslots = (uint32_t)a.ntens * (BWD ? 2u : 1u);
   const uint32_t sstride = nslots * a.tslot + a.tabslot;
   const uint32_t slab_bytes = (uint32_t)(HC * D * (int)sizeof(T));
   const uint32_t tab_bytes = (uint32_t)(D / 2 * 4);
-  const int64_t step = gridDim.x;
+  const uint32_t step = gridDim.x;
 
-  // this thread's vectors: tensor, head within the slab, element offset within the slab
-  int tt[VPT], hh[VPT], off[VPT];
-  bool valid[VPT];
-#pragma unroll
-  for (int j = 0; j < VPT; ++j) {
-    const int v = tid + j * NT;
-    valid[j] = v < NV;
-    const int vv = valid[j] ? v : 0;
-    tt[j] = vv / nv_t;
-    const int w = vv - tt[j] * nv_t;
-    hh[j] = w / lph;
-    off[j] = w * E;
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < a.stages; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], (uint32_t)ncw);
+    }
+    mbar_fence_init();
   }
-  const int li = tid % lph;  // lane within the head (same for every j when NORM)
-  float wq[E], wk[E];
+  __syncthreads();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane != 0) return;
+    int st = 0;
+    uint32_t ph = 0, used = 0, lastph = 0;
+    uint32_t k = 0;
+    for (uint32_t u = blockIdx.x; u < a.units; u += step, ++k) {
+      if (k >= (uint32_t)a.stages && !mbar_wait(&empty[st], ph ^ 1u, a.err)) break;
+      int64_t bs;
+      int c, s;
+      unit_origin(a, u, bs, c, s);
+      const int64_t eoff = (bs * a.H + (int64_t)c * HC) * D;
+      uint8_t* sb = data + (size_t)st * sstride;
+      mbar_expect_tx(&full[st], nslots * slab_bytes + 2 * tab_bytes);
+      for (int t = 0; t < a.ntens; ++t) {
+        bulk_g2s(sb + t * a.tslot, static_cast<const T*>(a.x[t]) + eoff, slab_bytes, &full[st]);
+        if constexpr (BWD)
+          bulk_g2s(sb + (a.ntens + t) * a.tslot, static_cast<const T*>(a.dy[t]) + eoff, slab_bytes, &full[st]);
+      }
+      uint8_t* tb = sb + nslots * a.tslot;
+      bulk_g2s(tb, a.cos + (int64_t)s * (D / 2), tab_bytes, &full[st]);
+      bulk_g2s(tb + tab_bytes, a.sin + (int64_t)s * (D / 2), tab_bytes, &full[st]);
+      used |= 1u << st;
+      lastph = (lastph & ~(1u << st)) | (ph << st);
+      if (++st == a.stages) st = 0, ph ^= 1u;
+    }
+    // every copy this CTA issued has landed before the CTA may exit (immediate when the
+    // consumers consumed them all)
+    for (int t = 0; t < a.stages; ++t)
+      if (used & (1u << t)) (void)mbar_wait(&full[t], (lastph >> t) & 1u, a.err);
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int ct = threadIdx.x - 32, nct = ncw * 32;
+  const int li = a.lph_shift >= 0 ? (ct & (lph - 1)) : 0;  // NORM: lane within the head (fixed)
+  float wq[E], wk[E], dwa[2][E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    wq[e] = wk[e] = 0.0f;
+    dwa[0][e] = dwa[1][e] = 0.0f;
+  }
   if constexpr (NORM) {
 #pragma unroll
     for (int e = 0; e < E; ++e) {
       const int d = li * E + e;
-      wq[e] = (GEMMA ? 1.0f : 0.0f) + Vec<T>::load1(static_cast<const T*>(a.w[0]) + d);
-      wk[e] = a.ntens > 1 ? (GEMMA ? 1.0f : 0.0f) + Vec<T>::load1(static_cast<const T*>(a.w[1]) + d) : 0.0f;
+      wq[e] = (GEMMA ? 1.0f : 0.0f) + V::load1(static_cast<const T*>(a.w[0]) + d);
+      if (a.ntens > 1) wk[e] = (GEMMA ? 1.0f : 0.0f) + V::load1(static_cast<const T*>(a.w[1]) + d);
     }
   }
-  float dwa[2][E];
-#pragma unroll
-  for (int e = 0; e < E; ++e) dwa[0][e] = dwa[1][e] = 0.0f;
-
-  auto unit_origin = [&](uint32_t u, int64_t& bs, int& c, int& s) {
-    c = (int)(u % (uint32_t)a.NC);
-    const uint32_t t2 = u / (uint32_t)a.NC;
-    const int b = (int)(t2 % (uint32_t)a.B);
-    s = (int)(t2 / (uint32_t)a.B);
-    bs = (int64_t)b * a.S + s;
-  };
-  auto issue = [&](int st, uint32_t u) {
-    int64_t bs;
-    int c, s;
-    unit_origin(u, bs, c, s);
-    const int64_t eoff = (bs * a.H + (int64_t)c * HC) * D;
-    uint8_t* sb = data + (size_t)st * sstride;
-    mbar_expect_tx(&bar[st], nslots * slab_bytes + 2 * tab_bytes);
-    for (int t = 0; t < a.ntens; ++t) {
-      bulk_g2s(sb + t * a.tslot, static_cast<const T*>(a.x[t]) + eoff, slab_bytes, &bar[st]);
-      if constexpr (BWD)
-        bulk_g2s(sb + (a.ntens + t) * a.tslot, static_cast<const T*>(a.dy[t]) + eoff, slab_bytes, &bar[st]);
-    }
-    uint8_t* tb = sb + nslots * a.tslot;
-    bulk_g2s(tb, a.cos + (int64_t)s * (D / 2), tab_bytes, &bar[st]);
-    bulk_g2s(tb + tab_bytes, a.sin + (int64_t)s * (D / 2), tab_bytes, &bar[st]);
-  };
-
-  if (tid == 0) {
-    for (int st = 0; st < a.stages; ++st) mbar_init(&bar[st], 1);
-    mbar_fence_init();
-  }
-  __syncthreads();
-  if (tid == 0) {
-    uint32_t u = blockIdx.x;
-    for (int st = 0; st < a.stages && u < a.units; ++st, u += (uint32_t)step) issue(st, u);
-  }
-
   const float inv_d = 1.0f / (float)D;
+  int failed = 0;
   int st = 0;
   uint32_t ph = 0;
-  for (uint32_t u = blockIdx.x; u < a.units; u += (uint32_t)step) {
+  for (uint32_t u = blockIdx.x; u < a.units; u += step) {
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&full[st], ph, a.err));
+    if (!ok) {
+      failed = 1;
+      break;
+    }
     int64_t bs;
     int c, s;
-    unit_origin(u, bs, c, s);
+    unit_origin(a, u, bs, c, s);
     const int64_t row0 = bs * a.H + (int64_t)c * HC;  // first head row of the unit
     const int64_t eoff = row0 * D;
-    float rin[VPT];
-    if constexpr (BWD) {
-#pragma unroll
-      for (int j = 0; j < VPT; ++j) rin[j] = valid[j] ? __ldg(a.stat[tt[j]] + row0 + hh[j]) : 0.0f;
-    }
-    const bool ok = mbar_wait(&bar[st], ph, a.err);
     const uint8_t* sb = data + (size_t)st * sstride;
     const float* tcos = reinterpret_cast<const float*>(sb + nslots * a.tslot);
     const float* tsin = tcos + D / 2;
-    float xv[VPT][E], gv[VPT][E], cs[VPT][P], sn[VPT][P];
-#pragma unroll
-    for (int j = 0; j < VPT; ++j) {
-      if (valid[j]) {
-        V::unpack(*reinterpret_cast<const uint4*>(sb + tt[j] * a.tslot + off[j] * sizeof(T)), xv[j]);
-        if constexpr (BWD)
-          V::unpack(*reinterpret_cast<const uint4*>(sb + (a.ntens + tt[j]) * a.tslot + off[j] * sizeof(T)), gv[j]);
-        const int p0 = (off[j] % D) / 2;
-#pragma unroll
-        for (int p = 0; p < P; ++p) {
-          cs[j][p] = tcos[p0 + p];
-          sn[j][p] = tsin[p0 + p];
-        }
+    // the trip count is the same for every lane of a warp, so the head shuffles see full warps
+    for (int vb = 0; vb < NV; vb += nct) {
+      const int v = vb + ct;
+      const bool valid = v < NV;
+      const int vv = valid ? v : 0;
+      const int tt = vv >= nv_t ? 1 : 0;
+      const int w = vv - tt * nv_t;  // vector index within the tensor slab
+      int hh, l;
+      if (a.lph_shift >= 0) {
+        hh = w >> a.lph_shift;
+        l = w & (lph - 1);
       } else {
-#pragma unroll
-        for (int e = 0; e < E; ++e) xv[j][e] = gv[j][e] = 0.0f;
-#pragma unroll
-        for (int p = 0; p < P; ++p) cs[j][p] = sn[j][p] = 0.0f;
+        hh = w / lph;
+        l = w - hh * lph;
       }
-    }
-    // every thread has read the stage: release it and refill it with the unit `stages` ahead
-    if (__syncthreads_or(!ok)) {
-      if (tid == 0) {
-        uint32_t uu = u;
-        int s2 = st;
-        uint32_t p2 = ph;
-        for (int k = 0; k < a.stages && uu < a.units; ++k, uu += (uint32_t)step) {
-          (void)mbar_wait(&bar[s2], p2, a.err);
-          if (++s2 == a.stages) s2 = 0, p2 ^= 1u;
-        }
+      float xv[E], o[E], cs[P], sn[P];
+      V::unpack(*reinterpret_cast<const uint4*>(sb + tt * a.tslot + (size_t)w * 16), xv);
+      if constexpr (P == 4) {
+        const float4 c4 = *reinterpret_cast<const float4*>(tcos + l * P);
+        const float4 s4 = *reinterpret_cast<const float4*>(tsin + l * P);
+        cs[0] = c4.x, cs[1] = c4.y, cs[2] = c4.z, cs[3] = c4.w;
+        sn[0] = s4.x, sn[1] = s4.y, sn[2] = s4.z, sn[3] = s4.w;
+      } else {
+        const float2 c2 = *reinterpret_cast<const float2*>(tcos + l * P);
+        const float2 s2 = *reinterpret_cast<const float2*>(tsin + l * P);
+        cs[0] = c2.x, cs[1] = c2.y;
+        sn[0] = s2.x, sn[1] = s2.y;
       }
-      return;
-    }
-    if (tid == 0 && (uint64_t)u + (uint64_t)a.stages * step < a.units) issue(st, u + (uint32_t)(a.stages * step));
-    if (++st == a.stages) st = 0, ph ^= 1u;
-
-#pragma unroll
-    for (int j = 0; j < VPT; ++j) {
-      float o[E];
       if constexpr (MODE == ROPE) {
 #pragma unroll
         for (int p = 0; p < P; ++p) {
-          const float x0 = xv[j][2 * p], x1 = xv[j][2 * p + 1];
-          const float si = a.sign * sn[j][p];
-          o[2 * p] = fmaf(x0, cs[j][p], -x1 * si);
-          o[2 * p + 1] = fmaf(x0, si, x1 * cs[j][p]);
+          const float x0 = xv[2 * p], x1 = xv[2 * p + 1];
+          const float si = a.sign * sn[p];
+          o[2 * p] = fmaf(x0, cs[p], -x1 * si);
+          o[2 * p + 1] = fmaf(x0, si, x1 * cs[p]);
         }
       } else if constexpr (MODE == QK_FWD) {
         float ss = 0.0f;
 #pragma unroll
-        for (int e = 0; e < E; ++e) ss = fmaf(xv[j][e], xv[j][e], ss);
+        for (int e = 0; e < E; ++e) ss = fmaf(xv[e], xv[e], ss);
         ss = group_sum_rt(ss, lph);
         const float r = rsqrtf(fmaf(ss, inv_d, a.eps));
         float n[E];
 #pragma unroll
-        for (int e = 0; e < E; ++e) n[e] = xv[j][e] * r * (tt[j] ? wk[e] : wq[e]);
+        for (int e = 0; e < E; ++e) n[e] = xv[e] * r * (tt ? wk[e] : wq[e]);
 #pragma unroll
         for (int p = 0; p < P; ++p) {
-          o[2 * p] = fmaf(n[2 * p], cs[j][p], -n[2 * p + 1] * sn[j][p]);
-          o[2 * p + 1] = fmaf(n[2 * p], sn[j][p], n[2 * p + 1] * cs[j][p]);
+          o[2 * p] = fmaf(n[2 * p], cs[p], -n[2 * p + 1] * sn[p]);
+          o[2 * p + 1] = fmaf(n[2 * p], sn[p], n[2 * p + 1] * cs[p]);
         }
-        if (li == 0 && valid[j] && a.stat[tt[j]]) a.stat[tt[j]][row0 + hh[j]] = r;
+        if (valid && l == 0 && a.stat[tt]) a.stat[tt][row0 + hh] = r;
       } else {  // QK_BWD
-        const float r = rin[j];
-        float g[E];
+        const float r = valid ? __ldg(a.stat[tt] + row0 + hh) : 0.0f;
+        float gv[E], g[E];
+        V::unpack(*reinterpret_cast<const uint4*>(sb + (a.ntens + tt) * a.tslot + (size_t)w * 16), gv);
 #pragma unroll
         for (int p = 0; p < P; ++p) {  // inverse rotation of the output gradient
-          const float d0 = gv[j][2 * p], d1 = gv[j][2 * p + 1];
-          g[2 * p] = fmaf(d0, cs[j][p], d1 * sn[j][p]);
-          g[2 * p + 1] = fmaf(-d0, sn[j][p], d1 * cs[j][p]);
+          const float d0 = gv[2 * p], d1 = gv[2 * p + 1];
+          g[2 * p] = fmaf(d0, cs[p], d1 * sn[p]);
+          g[2 * p + 1] = fmaf(-d0, sn[p], d1 * cs[p]);
         }
         float cdot = 0.0f;
 #pragma unroll
         for (int e = 0; e < E; ++e) {
-          const float xh = xv[j][e] * r;
-          const float wv = tt[j] ? wk[e] : wq[e];
-          cdot = fmaf(g[e] * wv, xh, cdot);
-          if (valid[j]) {
-            if (tt[j]) dwa[1][e] = fmaf(g[e], xh, dwa[1][e]);
+          const float xh = xv[e] * r;
+          cdot = fmaf(g[e] * (tt ? wk[e] : wq[e]), xh, cdot);
+          if (valid) {
+            if (tt) dwa[1][e] = fmaf(g[e], xh, dwa[1][e]);
             else dwa[0][e] = fmaf(g[e], xh, dwa[0][e]);
           }
         }
         cdot = group_sum_rt(cdot, lph) * inv_d;
 #pragma unroll
-        for (int e = 0; e < E; ++e) o[e] = r * fmaf(g[e], tt[j] ? wk[e] : wq[e], -(xv[j][e] * r) * cdot);
+        for (int e = 0; e < E; ++e) o[e] = r * fmaf(g[e], tt ? wk[e] : wq[e], -(xv[e] * r) * cdot);
       }
-      if (valid[j]) st_stream(static_cast<T*>(a.out[tt[j]]) + eoff + off[j], V::pack(o));
+      if (valid) st_stream(static_cast<T*>(a.out[tt]) + eoff + (int64_t)w * E, V::pack(o));
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[st]);
+    if (++st == a.stages) st = 0, ph ^= 1u;
   }
 
   if constexpr (BWD) {
-    if (!a.ws) return;
-    // combine the per-thread partials of the CTA in thread order (stages are idle now)
-    __syncthreads();
-    float* red = reinterpret_cast<float*>(data);  // [NT][2][E]
+    // combine the consumers' dw partials in thread order (the stages are idle now)
+    if (consumers_any(nct, failed) || !a.ws) return;
+    consumers_sync(nct);
+    float* red = reinterpret_cast<float*>(data);  // [nct][2][E]
 #pragma unroll
     for (int e = 0; e < E; ++e) {
-      red[(tid * 2 + 0) * E + e] = dwa[0][e];
-      red[(tid * 2 + 1) * E + e] = dwa[1][e];
+      red[(ct * 2 + 0) * E + e] = dwa[0][e];
+      red[(ct * 2 + 1) * E + e] = dwa[1][e];
     }
-    __syncthreads();
+    consumers_sync(nct);
     float* part = a.ws + (int64_t)blockIdx.x * 2 * D;
-    for (int col = tid; col < 2 * D; col += NT) {
+    for (int col = ct; col < 2 * D; col += nct) {
       const int t = col / D, d = col - t * D, l = d / E, e = d - l * E;
       float acc = 0.0f;
-      for (int th = l; th < NT; th += lph) acc += red[(th * 2 + t) * E + e];
+      for (int th = l; th < nct; th += lph) acc += red[(th * 2 + t) * E + e];
       part[col] = acc;
     }
   }
@@ -260,7 +292,7 @@ __global__ void __launch_bounds__(kRopeMaxThreads) rope_kernel(const RopeArgs a)
 // ---------------------------------------------------------------- planning
 
 struct RopePlan {
-  int HC, NC, vpt, threads, stages;
+  int HC, NC, cwarps, threads, stages, lph_shift;
   uint32_t tslot, tabslot;
   size_t smem;
 };
@@ -269,71 +301,64 @@ gn_status plan_rope(int64_t B, int64_t S, int64_t H, int64_t D, int ntens, int m
   const int vec = (int)(16 / es);
   const int lph = (int)(D / vec);
   const int nslots = ntens * (mode == QK_BWD ? 2 : 1);
-  const int64_t budget = g_tune.unit_bytes ? g_tune.unit_bytes : 24 * 1024;
-  // the backward holds x, dy and the table values of each vector: two vectors per thread
-  const int vpt = g_tune.vpt ? (g_tune.vpt > 4 ? 4 : g_tune.vpt) : (mode == QK_BWD ? 2 : 4);
-  int HC = 0;
+  const int64_t budget = g_tune.unit_bytes ? g_tune.unit_bytes : 48 * 1024;
+  int HC = 1;
   for (int hc = (int)H; hc >= 1; --hc) {
     if (H % hc) continue;
-    const int64_t nv = (int64_t)ntens * hc * lph;
-    if ((nv + vpt - 1) / vpt > kRopeMaxThreads) continue;
     if ((int64_t)nslots * hc * D * (int64_t)es > budget && hc > 1) continue;
     HC = hc;
     break;
   }
-  if (HC == 0) return GN_ERR_UNSUPPORTED;
   p->HC = HC;
   p->NC = (int)(H / HC);
-  p->vpt = vpt;
   const int64_t nv = (int64_t)ntens * HC * lph;
-  p->threads = (int)(((nv + vpt - 1) / vpt + 31) / 32 * 32);
-  if (p->threads > kRopeMaxThreads) return GN_ERR_UNSUPPORTED;
+  // consumer warps: 8 by default; prefer a count whose 32*C divides the unit's vectors
+  int cw = 8;
+  if (nv % (32 * cw)) {
+    for (int c = kMaxConsumerWarps; c >= 4; --c)
+      if (nv % (32 * c) == 0) {
+        cw = c;
+        break;
+      }
+  }
+  if (g_tune.group_rows) cw = g_tune.group_rows > kMaxConsumerWarps ? kMaxConsumerWarps : g_tune.group_rows;
+  p->cwarps = cw;
+  p->threads = 32 * (1 + cw);
+  p->lph_shift = (lph & (lph - 1)) == 0 ? __builtin_ctz((unsigned)lph) : -1;
   p->tslot = round128((uint32_t)(HC * D * (int64_t)es));
   p->tabslot = round128((uint32_t)(D * 4));
   const size_t sstride = (size_t)nslots * p->tslot + p->tabslot;
   int stages = g_tune.stages ? g_tune.stages : (int)(96 * 1024 / sstride);
-  stages = stages < 2 ? 2 : stages > 8 ? 8 : stages;
+  stages = stages < 2 ? 2 : stages > kRopeMaxStages ? kRopeMaxStages : stages;
   const size_t limit = smem_optin();
   while (stages > 1 && 128 + stages * sstride > limit) --stages;
   p->stages = stages;
   p->smem = 128 + stages * sstride;
-  // the backward reuses the stages for the [threads][2][vec] partial-sum table
-  const size_t red = (size_t)p->threads * 2 * vec * 4;
+  // the backward reuses the stages for the [consumers][2][vec] partial-sum table
+  const size_t red = (size_t)32 * cw * 2 * vec * 4;
   if (mode == QK_BWD && red > stages * sstride) p->smem = 128 + red;
   if (p->smem > limit) return GN_ERR_UNSUPPORTED;
   if (B * S * p->NC >= (int64_t)1 << 31) return GN_ERR_UNSUPPORTED;
   return GN_OK;
 }
 
-template <typename T, int MODE>
-void* pick_rope(int vpt, bool gemma) {
-#define GN_V(V_)                                                       \
-  if (vpt == V_) {                                                     \
-    return gemma ? (void*)rope_kernel<T, V_, MODE, (MODE != ROPE)>     \
-                 : (void*)rope_kernel<T, V_, MODE, false>;             \
-  }
-  GN_V(1) GN_V(2) GN_V(4)
-#undef GN_V
-  return nullptr;
-}
-
-void* pick(gn_dtype dt, int mode, int vpt, bool gemma) {
+void* pick(gn_dtype dt, int mode, bool gemma) {
   if (dt == GN_BF16) {
-    if (mode == ROPE) return pick_rope<__nv_bfloat16, ROPE>(vpt, false);
-    if (mode == QK_FWD) return pick_rope<__nv_bfloat16, QK_FWD>(vpt, gemma);
-    return pick_rope<__nv_bfloat16, QK_BWD>(vpt, gemma);
+    if (mode == ROPE) return (void*)rope_kernel<__nv_bfloat16, ROPE, false>;
+    if (mode == QK_FWD)
+      return gemma ? (void*)rope_kernel<__nv_bfloat16, QK_FWD, true> : (void*)rope_kernel<__nv_bfloat16, QK_FWD, false>;
+    return gemma ? (void*)rope_kernel<__nv_bfloat16, QK_BWD, true> : (void*)rope_kernel<__nv_bfloat16, QK_BWD, false>;
   }
-  if (mode == ROPE) return pick_rope<float, ROPE>(vpt, false);
-  if (mode == QK_FWD) return pick_rope<float, QK_FWD>(vpt, gemma);
-  return pick_rope<float, QK_BWD>(vpt, gemma);
+  if (mode == ROPE) return (void*)rope_kernel<float, ROPE, false>;
+  if (mode == QK_FWD) return gemma ? (void*)rope_kernel<float, QK_FWD, true> : (void*)rope_kernel<float, QK_FWD, false>;
+  return gemma ? (void*)rope_kernel<float, QK_BWD, true> : (void*)rope_kernel<float, QK_BWD, false>;
 }
 
 gn_status setup(int64_t B, int64_t S, int64_t H, int64_t D, int ntens, int mode, gn_dtype dt, bool gemma,
                 RopePlan* p, void** kern, int* grid) {
   gn_status st = plan_rope(B, S, H, D, ntens, mode, dt_size(dt), p);
   if (st != GN_OK) return st;
-  *kern = pick(dt, mode, p->vpt, gemma);
-  if (!*kern) return GN_ERR_UNSUPPORTED;
+  *kern = pick(dt, mode, gemma);
   const int cap = g_tune.ctas_per_sm ? g_tune.ctas_per_sm : 8;
   int g = persistent_grid(*kern, p->threads, p->smem, cap);
   if (g <= 0) return GN_ERR_CUDA;
@@ -360,6 +385,7 @@ gn_status launch(void* kern, int grid, const RopePlan& p, RopeArgs& a, cudaStrea
   a.stages = p.stages;
   a.tslot = p.tslot;
   a.tabslot = p.tabslot;
+  a.lph_shift = p.lph_shift;
   a.units = (uint32_t)((int64_t)a.B * a.S * p.NC);
   a.err = device_err_word();
   if (!a.err) return GN_ERR_CUDA;
