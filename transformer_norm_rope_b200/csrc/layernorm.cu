@@ -60,7 +60,7 @@ __device__ __forceinline__ void chan_merge(float& n, float& m, float& M2, float 
   }
   const float nn = n + nb;
   const float d = mb - m;
-  const float f = nb / nn;
+  const float f = __fdividef(nb, nn);
   m = fmaf(d, f, m);
   M2 = M2 + M2b + d * d * n * f;
   n = nn;
@@ -117,85 +117,95 @@ __device__ __forceinline__ void load_affine(const LnFwdArgs& a, int base, int st
     }
 }
 
-// ---------------------------------------------------------------- CTA path
+// ---------------------------------------------------------------- CTA path (long rows)
+// Warp 0 produces (row_pipe.cuh); warps 1.. consume. Consumer thread ct owns the vectors
+// v = ct + j * nct (j < VPT) of every row. Weight and bias live in shared memory.
+
+template <typename T>
+__device__ __forceinline__ void stage_param(uint8_t* dst, const T* src, int N, int nvec, float dflt, int ct,
+                                            int nct) {
+  T* d = reinterpret_cast<T*>(dst);
+  const int n = nvec * Vec<T>::N;  // padded to whole vectors; the padding holds 0
+  for (int i = ct; i < n; i += nct) {
+    float v = i < N ? ld_param(src, i, dflt) : 0.0f;
+    Vec<T>::store1(d + i, v);
+  }
+}
 
 template <typename T, int VPT, int EPI>
-__global__ void __launch_bounds__(norm_max_threads(VPT)) ln_fwd_cta(const LnFwdArgs a) {
+__global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT)) ln_fwd_cta(const LnFwdArgs a) {
   using V = Vec<T>;
   constexpr int E = V::N;
   constexpr bool FAST = fast_math_for<T>();
   extern __shared__ __align__(128) uint8_t smem[];
-  const int tid = threadIdx.x, NT = blockDim.x, lane = tid & 31, warp = tid >> 5;
-  const int nwarps = NT >> 5;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int N = a.N, nfull = N / E, nvec = (N + E - 1) / E;
-  const RowPipe pipe(smem, a.stages, 1, (int64_t)N * sizeof(T));
-  const int64_t step = gridDim.x;
+  const RowPipe pipe(smem, a.stages, 1, 2, (int64_t)N * sizeof(T));
   const T* x = static_cast<const T*>(a.x);
   T* y = static_cast<T*>(a.y);
-
-  if (tid == 0) pipe.init();
+  const int ncw = (int)(blockDim.x >> 5) - 1;
+  if (tid == 0) pipe.init(ncw);
   __syncthreads();
-  if (tid == 0) {
-    int64_t m = blockIdx.x;
-    for (int s = 0; s < a.stages && m < a.rows; ++s, m += step) pipe.issue(s, x + m * a.ldx);
+  if (warp == 0) {
+    if (lane == 0) pipe.produce(a.rows, [&](int64_t m, int) -> const void* { return x + m * a.ldx; }, a.err);
+    return;
   }
-  float wr[VPT][E], br[VPT][E];
-  load_affine<T, VPT>(a, tid, NT, wr, br);
+  const int ct = tid - 32, nct = ncw * 32, cw = warp - 1;
+  stage_param(pipe.param(0), static_cast<const T*>(a.w), N, nvec, 1.0f, ct, nct);
+  stage_param(pipe.param(1), static_cast<const T*>(a.b), N, nvec, 0.0f, ct, nct);
+  consumers_sync(nct);
   int cnt[VPT];
 #pragma unroll
   for (int j = 0; j < VPT; ++j) {
-    const int left = N - (tid + j * NT) * E;
+    const int left = N - (ct + j * nct) * E;
     cnt[j] = left <= 0 ? 0 : left >= E ? E : left;
   }
   const float inv_n = 1.0f / (float)N;
-
+  const int64_t step = gridDim.x;
   int s = 0;
   uint32_t ph = 0, rb = 0;
-  const int64_t ahead = (int64_t)a.stages * step;
   for (int64_t m = blockIdx.x; m < a.rows; m += step) {
     const T* xrow = x + m * a.ldx;
-    const bool ok = pipe.wait(s, ph, a.err);
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&pipe.full[s], ph, a.err));
     const uint8_t* st = pipe.at(s, 0);
     float xv[VPT][E];
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
-      const int v = tid + j * NT;
-      if (v < nfull) {
+      const int v = ct + j * nct;
+      if (ok && v < nfull) {
         V::unpack(*reinterpret_cast<const uint4*>(st + (size_t)v * 16), xv[j]);
       } else {
 #pragma unroll
-        for (int e = 0; e < E; ++e) xv[j][e] = e < cnt[j] ? V::load1(xrow + v * E + e) : 0.0f;
+        for (int e = 0; e < E; ++e) xv[j][e] = (ok && e < cnt[j]) ? V::load1(xrow + v * E + e) : 0.0f;
       }
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&pipe.empty[s]);
     float n, mu, M2;
     thread_stats<VPT, E>(xv, cnt, n, mu, M2);
     group_stats(n, mu, M2, 32);
     float4* red = pipe.red + rb * 32;
-    if (lane == 0) red[warp] = make_float4(n, mu, M2, 0.0f);
-    if (__syncthreads_or(!ok)) {
-      if (tid == 0) pipe.drain(m, step, a.rows, s, ph, a.err);
-      return;
-    }
-    if (tid == 0 && m + ahead < a.rows) pipe.issue(s, x + (m + ahead) * a.ldx);
+    if (lane == 0) red[cw] = make_float4(n, mu, M2, 0.0f);
+    if (consumers_sync_or(nct, !ok)) return;
     rb ^= 1u;
-    if (++s == a.stages) {
-      s = 0;
-      ph ^= 1u;
-    }
+    if (++s == a.stages) s = 0, ph ^= 1u;
     n = 0.0f, mu = 0.0f, M2 = 0.0f;
-    for (int w = 0; w < nwarps; ++w) {
+    for (int w = 0; w < ncw; ++w) {
       const float4 r = red[w];
       chan_merge(n, mu, M2, r.x, r.y, r.z);
     }
     const float rs = rsqrtf(fmaf(M2, inv_n, a.eps));
+    const float nmr = -mu * rs;
     T* yrow = y + m * a.ldy;
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
-      const int v = tid + j * NT;
+      const int v = ct + j * nct;
       if (v < nvec) {
-        float o[E];
+        float wv[E], bv[E], o[E];
+        V::unpack(*reinterpret_cast<const uint4*>(pipe.param(0) + (size_t)v * 16), wv);
+        V::unpack(*reinterpret_cast<const uint4*>(pipe.param(1) + (size_t)v * 16), bv);
 #pragma unroll
-        for (int e = 0; e < E; ++e) o[e] = epi_fwd<EPI, FAST>(fmaf((xv[j][e] - mu) * rs, wr[j][e], br[j][e]));
+        for (int e = 0; e < E; ++e) o[e] = epi_fwd<EPI, FAST>(fmaf(fmaf(xv[j][e], rs, nmr), wv[e], bv[e]));
         if (v < nfull) {
           st_stream(yrow + (size_t)v * E, V::pack(o));
         } else {
@@ -205,7 +215,7 @@ __global__ void __launch_bounds__(norm_max_threads(VPT)) ln_fwd_cta(const LnFwdA
         }
       }
     }
-    if (tid == 0) {
+    if (ct == 0) {
       if (a.mean) a.mean[m] = mu;
       if (a.rstd) a.rstd[m] = rs;
     }
@@ -213,72 +223,82 @@ __global__ void __launch_bounds__(norm_max_threads(VPT)) ln_fwd_cta(const LnFwdA
 }
 
 template <typename T, int VPT, int EPI>
-__global__ void __launch_bounds__(norm_max_threads(VPT, true)) ln_bwd_cta(const LnBwdArgs a) {
+__global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT, true)) ln_bwd_cta(const LnBwdArgs a) {
   using V = Vec<T>;
   constexpr int E = V::N;
   constexpr bool FAST = fast_math_for<T>();
   extern __shared__ __align__(128) uint8_t smem[];
-  const int tid = threadIdx.x, NT = blockDim.x, lane = tid & 31, warp = tid >> 5;
-  const int nwarps = NT >> 5;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int N = a.N, nfull = N / E, nvec = (N + E - 1) / E;
-  const RowPipe pipe(smem, a.stages, 2, (int64_t)N * sizeof(T));
-  const int64_t step = gridDim.x;
+  const RowPipe pipe(smem, a.stages, 2, 2, (int64_t)N * sizeof(T));
   const T* x = static_cast<const T*>(a.x);
   const T* dy = static_cast<const T*>(a.dy);
   T* dx = static_cast<T*>(a.dx);
-
-  if (tid == 0) pipe.init();
+  const int ncw = (int)(blockDim.x >> 5) - 1;
+  if (tid == 0) pipe.init(ncw);
   __syncthreads();
-  if (tid == 0) {
-    int64_t m = blockIdx.x;
-    for (int s = 0; s < a.stages && m < a.rows; ++s, m += step) pipe.issue(s, x + m * a.ldx, dy + m * a.lddy);
+  if (warp == 0) {
+    if (lane == 0)
+      pipe.produce(
+          a.rows,
+          [&](int64_t m, int t) -> const void* { return t == 0 ? (const void*)(x + m * a.ldx) : (const void*)(dy + m * a.lddy); },
+          a.err);
+    return;
   }
-  float wr[VPT][E], br[VPT][E], dwa[VPT][E], dba[VPT][E];
+  const int ct = tid - 32, nct = ncw * 32, cw = warp - 1;
+  stage_param(pipe.param(0), static_cast<const T*>(a.w), N, nvec, 1.0f, ct, nct);
+  stage_param(pipe.param(1), static_cast<const T*>(a.b), N, nvec, 0.0f, ct, nct);
+  consumers_sync(nct);
+  float dwa[VPT][E], dba[VPT][E];
 #pragma unroll
   for (int j = 0; j < VPT; ++j)
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const int col = (tid + j * NT) * E + e;
-      const bool in = col < N;
-      wr[j][e] = in ? ld_param(static_cast<const T*>(a.w), col, 1.0f) : 0.0f;
-      br[j][e] = in ? ld_param(static_cast<const T*>(a.b), col, 0.0f) : 0.0f;
-      dwa[j][e] = 0.0f;
-      dba[j][e] = 0.0f;
-    }
+    for (int e = 0; e < E; ++e) dwa[j][e] = dba[j][e] = 0.0f;
   const float inv_n = 1.0f / (float)N;
-
+  const int64_t step = gridDim.x;
   int s = 0;
   uint32_t ph = 0, rb = 0;
-  const int64_t ahead = (int64_t)a.stages * step;
+  bool failed = false;
   for (int64_t m = blockIdx.x; m < a.rows; m += step) {
     const float mu = __ldg(a.mean + m), rs = __ldg(a.rstd + m);
     const T* xrow = x + m * a.ldx;
     const T* gyrow = dy + m * a.lddy;
-    const bool ok = pipe.wait(s, ph, a.err);
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&pipe.full[s], ph, a.err));
     const uint8_t* sx = pipe.at(s, 0);
     const uint8_t* sg = pipe.at(s, 1);
     float xv[VPT][E], gv[VPT][E];
-    float s1 = 0.0f, s2 = 0.0f;
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
-      const int v = tid + j * NT;
-      if (v < nfull) {
+      const int v = ct + j * nct;
+      if (ok && v < nfull) {
         V::unpack(*reinterpret_cast<const uint4*>(sx + (size_t)v * 16), xv[j]);
         V::unpack(*reinterpret_cast<const uint4*>(sg + (size_t)v * 16), gv[j]);
       } else {
 #pragma unroll
         for (int e = 0; e < E; ++e) {
           const int col = v * E + e;
-          const bool in = v < nvec && col < N;
+          const bool in = ok && v < nvec && col < N;
           xv[j][e] = in ? V::load1(xrow + col) : 0.0f;
           gv[j][e] = in ? V::load1(gyrow + col) : 0.0f;
         }
       }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&pipe.empty[s]);
+    const float nmr = -mu * rs;
+    float s1 = 0.0f, s2 = 0.0f;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      const int v = ct + j * nct;
+      const size_t vo = (size_t)(v < nvec ? v : 0) * 16;
+      float wv[E], bv[E];
+      V::unpack(*reinterpret_cast<const uint4*>(pipe.param(0) + vo), wv);
+      V::unpack(*reinterpret_cast<const uint4*>(pipe.param(1) + vo), bv);
 #pragma unroll
       for (int e = 0; e < E; ++e) {
-        const float xh = (xv[j][e] - mu) * rs;
-        const float g = gv[j][e] * epi_grad<EPI, FAST>(fmaf(xh, wr[j][e], br[j][e]));
-        const float gw = g * wr[j][e];
+        const float xh = fmaf(xv[j][e], rs, nmr);
+        const float g = gv[j][e] * epi_grad<EPI, FAST>(fmaf(xh, wv[e], bv[e]));
+        const float gw = g * wv[e];
         gv[j][e] = g;
         s1 += gw;
         s2 = fmaf(gw, xh, s2);
@@ -289,19 +309,15 @@ __global__ void __launch_bounds__(norm_max_threads(VPT, true)) ln_bwd_cta(const 
     s1 = group_sum<32>(s1);
     s2 = group_sum<32>(s2);
     float4* red = pipe.red + rb * 32;
-    if (lane == 0) red[warp] = make_float4(s1, s2, 0.0f, 0.0f);
-    if (__syncthreads_or(!ok)) {
-      if (tid == 0) pipe.drain(m, step, a.rows, s, ph, a.err);
-      return;
+    if (lane == 0) red[cw] = make_float4(s1, s2, 0.0f, 0.0f);
+    if (consumers_sync_or(nct, !ok)) {
+      failed = true;
+      break;
     }
-    if (tid == 0 && m + ahead < a.rows) pipe.issue(s, x + (m + ahead) * a.ldx, dy + (m + ahead) * a.lddy);
     rb ^= 1u;
-    if (++s == a.stages) {
-      s = 0;
-      ph ^= 1u;
-    }
+    if (++s == a.stages) s = 0, ph ^= 1u;
     float t1 = 0.0f, t2 = 0.0f;
-    for (int w = 0; w < nwarps; ++w) {
+    for (int w = 0; w < ncw; ++w) {
       t1 += red[w].x;
       t2 += red[w].y;
     }
@@ -309,13 +325,14 @@ __global__ void __launch_bounds__(norm_max_threads(VPT, true)) ln_bwd_cta(const 
     T* dxrow = dx + m * a.lddx;
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
-      const int v = tid + j * NT;
+      const int v = ct + j * nct;
       if (v < nvec) {
-        float o[E];
+        float wv[E], o[E];
+        V::unpack(*reinterpret_cast<const uint4*>(pipe.param(0) + (size_t)v * 16), wv);
 #pragma unroll
         for (int e = 0; e < E; ++e) {
-          const float xh = (xv[j][e] - mu) * rs;
-          o[e] = rs * (fmaf(gv[j][e], wr[j][e], -c1) - xh * c2);
+          const float xh = fmaf(xv[j][e], rs, nmr);
+          o[e] = rs * (fmaf(gv[j][e], wv[e], -c1) - xh * c2);
         }
         if (v < nfull) {
           st_stream(dxrow + (size_t)v * E, V::pack(o));
@@ -327,13 +344,13 @@ __global__ void __launch_bounds__(norm_max_threads(VPT, true)) ln_bwd_cta(const 
       }
     }
   }
-  if (a.ws) {
+  if (a.ws && !failed) {
     float* part = a.ws + (int64_t)blockIdx.x * 2 * N;
 #pragma unroll
     for (int j = 0; j < VPT; ++j)
 #pragma unroll
       for (int e = 0; e < E; ++e) {
-        const int col = (tid + j * NT) * E + e;
+        const int col = (ct + j * nct) * E + e;
         if (col < N) {
           part[col] = dwa[j][e];
           part[N + col] = dba[j][e];
@@ -549,12 +566,10 @@ void* pick_ln_t(int vpt, bool cta, int epi) {
   return nullptr;
 }
 
-constexpr int kFwdThreads = 256;
-constexpr int kBwdThreads = 512;
 
 gn_status ln_plan(int64_t rows, int64_t hidden, gn_dtype dt, bool bwd, int epi, NormPlan* p, void** kern,
                   int* grid) {
-  gn_status st = plan_norm(hidden, dt_size(dt), bwd ? 2 : 1, bwd ? 4 : 8, bwd ? kBwdThreads : kFwdThreads, p);
+  gn_status st = plan_norm(hidden, dt_size(dt), bwd ? 2 : 1, 2, bwd ? 4 : 8, p);
   if (st != GN_OK) return st;
   if (dt == GN_BF16)
     *kern = bwd ? pick_ln_t<__nv_bfloat16, true>(p->vpt, p->cta, epi) : pick_ln_t<__nv_bfloat16, false>(p->vpt, p->cta, epi);

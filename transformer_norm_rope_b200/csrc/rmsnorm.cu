@@ -41,88 +41,88 @@ struct RmsBwdArgs {
   unsigned* err;
 };
 
-// ---------------------------------------------------------------- CTA path
+// ---------------------------------------------------------------- CTA path (long rows)
+// Warp 0 produces (row_pipe.cuh); warps 1.. consume. Consumer thread ct owns the vectors
+// v = ct + j * nct (j < VPT) of every row, so its columns - and its share of the weight
+// gradient - never change. The weight lives in shared memory (one copy per CTA).
+
+template <typename T>
+__device__ __forceinline__ void stage_param(uint8_t* dst, const T* src, int N, int nvec, float dflt, int ct,
+                                            int nct) {
+  T* d = reinterpret_cast<T*>(dst);
+  const int n = nvec * Vec<T>::N;  // padded to whole vectors; the padding holds 0
+  for (int i = ct; i < n; i += nct) {
+    float v = i < N ? ld_param(src, i, dflt) : 0.0f;
+    Vec<T>::store1(d + i, v);
+  }
+}
 
 template <typename T, int VPT, int EPI, bool GEMMA>
-__global__ void __launch_bounds__(norm_max_threads(VPT)) rms_fwd_cta(const RmsFwdArgs a) {
+__global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT)) rms_fwd_cta(const RmsFwdArgs a) {
   using V = Vec<T>;
   constexpr int E = V::N;
   constexpr bool FAST = fast_math_for<T>();
   extern __shared__ __align__(128) uint8_t smem[];
-  const int tid = threadIdx.x, NT = blockDim.x, lane = tid & 31, warp = tid >> 5;
-  const int nwarps = NT >> 5;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int N = a.N, nfull = N / E, nvec = (N + E - 1) / E;
-  const RowPipe pipe(smem, a.stages, 1, (int64_t)N * sizeof(T));
-  const int64_t step = gridDim.x;
+  const RowPipe pipe(smem, a.stages, 1, 1, (int64_t)N * sizeof(T));
   const T* x = static_cast<const T*>(a.x);
   T* y = static_cast<T*>(a.y);
-
-  if (tid == 0) pipe.init();
+  const int ncw = (int)(blockDim.x >> 5) - 1;
+  if (tid == 0) pipe.init(ncw);
   __syncthreads();
-  if (tid == 0) {
-    int64_t m = blockIdx.x;
-    for (int s = 0; s < a.stages && m < a.rows; ++s, m += step) pipe.issue(s, x + m * a.ldx);
+  if (warp == 0) {
+    if (lane == 0) pipe.produce(a.rows, [&](int64_t m, int) -> const void* { return x + m * a.ldx; }, a.err);
+    return;
   }
-
-  float wr[VPT][E];
-#pragma unroll
-  for (int j = 0; j < VPT; ++j)
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const int col = (tid + j * NT) * E + e;
-      wr[j][e] = col < N ? (GEMMA ? 1.0f : 0.0f) + ld_param(static_cast<const T*>(a.w), col, 0.0f) : 0.0f;
-    }
+  const int ct = tid - 32, nct = ncw * 32, cw = warp - 1;
+  stage_param(pipe.param(0), static_cast<const T*>(a.w), N, nvec, 0.0f, ct, nct);
+  consumers_sync(nct);
   const float inv_n = 1.0f / (float)N;
-
-  int s = 0;         // stage of row m
-  uint32_t ph = 0;   // barrier parity of that stage's current use
-  uint32_t rb = 0;   // reduction buffer, alternating per row
-  const int64_t ahead = (int64_t)a.stages * step;
+  const int64_t step = gridDim.x;
+  int s = 0;
+  uint32_t ph = 0, rb = 0;
   for (int64_t m = blockIdx.x; m < a.rows; m += step) {
     const T* xrow = x + m * a.ldx;
-    const bool ok = pipe.wait(s, ph, a.err);
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&pipe.full[s], ph, a.err));
     const uint8_t* st = pipe.at(s, 0);
     float xv[VPT][E];
     float ss = 0.0f;
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
-      const int v = tid + j * NT;
-      if (v < nfull) {
+      const int v = ct + j * nct;
+      if (ok && v < nfull) {
         V::unpack(*reinterpret_cast<const uint4*>(st + (size_t)v * 16), xv[j]);
       } else {
 #pragma unroll
         for (int e = 0; e < E; ++e) {
           const int col = v * E + e;
-          xv[j][e] = (v < nvec && col < N) ? V::load1(xrow + col) : 0.0f;
+          xv[j][e] = (ok && v < nvec && col < N) ? V::load1(xrow + col) : 0.0f;
         }
       }
 #pragma unroll
       for (int e = 0; e < E; ++e) ss = fmaf(xv[j][e], xv[j][e], ss);
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&pipe.empty[s]);
     ss = group_sum<32>(ss);
     float4* red = pipe.red + rb * 32;
-    if (lane == 0) red[warp].x = ss;
-    if (__syncthreads_or(!ok)) {
-      if (tid == 0) pipe.drain(m, step, a.rows, s, ph, a.err);
-      return;
-    }
-    if (tid == 0 && m + ahead < a.rows) pipe.issue(s, x + (m + ahead) * a.ldx);
+    if (lane == 0) red[cw].x = ss;
+    if (consumers_sync_or(nct, !ok)) return;
     rb ^= 1u;
-    if (++s == a.stages) {
-      s = 0;
-      ph ^= 1u;
-    }
+    if (++s == a.stages) s = 0, ph ^= 1u;
     float tot = 0.0f;
-    for (int w = 0; w < nwarps; ++w) tot += red[w].x;
+    for (int w = 0; w < ncw; ++w) tot += red[w].x;
     const float r = rsqrtf(fmaf(tot, inv_n, a.eps));
     T* yrow = y + m * a.ldy;
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
-      const int v = tid + j * NT;
+      const int v = ct + j * nct;
       if (v < nvec) {
-        float o[E];
+        float wv[E], o[E];
+        V::unpack(*reinterpret_cast<const uint4*>(pipe.param(0) + (size_t)v * 16), wv);
 #pragma unroll
-        for (int e = 0; e < E; ++e) o[e] = epi_fwd<EPI, FAST>(xv[j][e] * r * wr[j][e]);
+        for (int e = 0; e < E; ++e) o[e] = epi_fwd<EPI, FAST>(xv[j][e] * r * ((GEMMA ? 1.0f : 0.0f) + wv[e]));
         if (v < nfull) {
           st_stream(yrow + (size_t)v * E, V::pack(o));
         } else {
@@ -132,104 +132,110 @@ __global__ void __launch_bounds__(norm_max_threads(VPT)) rms_fwd_cta(const RmsFw
         }
       }
     }
-    if (tid == 0 && a.inv_rms) a.inv_rms[m] = r;
+    if (ct == 0 && a.inv_rms) a.inv_rms[m] = r;
   }
 }
 
 template <typename T, int VPT, int EPI, bool GEMMA>
-__global__ void __launch_bounds__(norm_max_threads(VPT, true)) rms_bwd_cta(const RmsBwdArgs a) {
+__global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT, true)) rms_bwd_cta(const RmsBwdArgs a) {
   using V = Vec<T>;
   constexpr int E = V::N;
   constexpr bool FAST = fast_math_for<T>();
   extern __shared__ __align__(128) uint8_t smem[];
-  const int tid = threadIdx.x, NT = blockDim.x, lane = tid & 31, warp = tid >> 5;
-  const int nwarps = NT >> 5;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int N = a.N, nfull = N / E, nvec = (N + E - 1) / E;
-  const RowPipe pipe(smem, a.stages, 2, (int64_t)N * sizeof(T));
-  const int64_t step = gridDim.x;
+  const RowPipe pipe(smem, a.stages, 2, 1, (int64_t)N * sizeof(T));
   const T* x = static_cast<const T*>(a.x);
   const T* dy = static_cast<const T*>(a.dy);
   T* dx = static_cast<T*>(a.dx);
-
-  if (tid == 0) pipe.init();
+  const int ncw = (int)(blockDim.x >> 5) - 1;
+  if (tid == 0) pipe.init(ncw);
   __syncthreads();
-  if (tid == 0) {
-    int64_t m = blockIdx.x;
-    for (int s = 0; s < a.stages && m < a.rows; ++s, m += step) pipe.issue(s, x + m * a.ldx, dy + m * a.lddy);
+  if (warp == 0) {
+    if (lane == 0)
+      pipe.produce(
+          a.rows,
+          [&](int64_t m, int t) -> const void* { return t == 0 ? (const void*)(x + m * a.ldx) : (const void*)(dy + m * a.lddy); },
+          a.err);
+    return;
   }
-
-  float wr[VPT][E], dwa[VPT][E];
+  const int ct = tid - 32, nct = ncw * 32, cw = warp - 1;
+  stage_param(pipe.param(0), static_cast<const T*>(a.w), N, nvec, 0.0f, ct, nct);
+  consumers_sync(nct);
+  float dwa[VPT][E];
 #pragma unroll
   for (int j = 0; j < VPT; ++j)
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const int col = (tid + j * NT) * E + e;
-      wr[j][e] = col < N ? (GEMMA ? 1.0f : 0.0f) + ld_param(static_cast<const T*>(a.w), col, 0.0f) : 0.0f;
-      dwa[j][e] = 0.0f;
-    }
+    for (int e = 0; e < E; ++e) dwa[j][e] = 0.0f;
   const float inv_n = 1.0f / (float)N;
-
-  int s = 0;         // stage of row m
-  uint32_t ph = 0;   // barrier parity of that stage's current use
-  uint32_t rb = 0;   // reduction buffer, alternating per row
-  const int64_t ahead = (int64_t)a.stages * step;
+  const float woff = GEMMA ? 1.0f : 0.0f;
+  const int64_t step = gridDim.x;
+  int s = 0;
+  uint32_t ph = 0, rb = 0;
+  bool failed = false;
   for (int64_t m = blockIdx.x; m < a.rows; m += step) {
     const float r = __ldg(a.inv_rms + m);
     const T* xrow = x + m * a.ldx;
     const T* gyrow = dy + m * a.lddy;
-    const bool ok = pipe.wait(s, ph, a.err);
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&pipe.full[s], ph, a.err));
     const uint8_t* sx = pipe.at(s, 0);
     const uint8_t* sg = pipe.at(s, 1);
     float xv[VPT][E], gv[VPT][E];
-    float c = 0.0f;
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
-      const int v = tid + j * NT;
-      if (v < nfull) {
+      const int v = ct + j * nct;
+      if (ok && v < nfull) {
         V::unpack(*reinterpret_cast<const uint4*>(sx + (size_t)v * 16), xv[j]);
         V::unpack(*reinterpret_cast<const uint4*>(sg + (size_t)v * 16), gv[j]);
       } else {
 #pragma unroll
         for (int e = 0; e < E; ++e) {
           const int col = v * E + e;
-          const bool in = v < nvec && col < N;
+          const bool in = ok && v < nvec && col < N;
           xv[j][e] = in ? V::load1(xrow + col) : 0.0f;
           gv[j][e] = in ? V::load1(gyrow + col) : 0.0f;
         }
       }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&pipe.empty[s]);
+    float c = 0.0f;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      const int v = ct + j * nct;
+      float wv[E];
+      V::unpack(*reinterpret_cast<const uint4*>(pipe.param(0) + (size_t)(v < nvec ? v : 0) * 16), wv);
 #pragma unroll
       for (int e = 0; e < E; ++e) {
+        const float wp = woff + wv[e];
         const float xh = xv[j][e] * r;
-        const float g = gv[j][e] * epi_grad<EPI, FAST>(xh * wr[j][e]);
+        const float g = gv[j][e] * epi_grad<EPI, FAST>(xh * wp);
         gv[j][e] = g;
-        c = fmaf(g * wr[j][e], xh, c);
+        c = fmaf(g * wp, xh, c);
         dwa[j][e] = fmaf(g, xh, dwa[j][e]);
       }
     }
     c = group_sum<32>(c);
     float4* red = pipe.red + rb * 32;
-    if (lane == 0) red[warp].x = c;
-    if (__syncthreads_or(!ok)) {
-      if (tid == 0) pipe.drain(m, step, a.rows, s, ph, a.err);
-      return;
+    if (lane == 0) red[cw].x = c;
+    if (consumers_sync_or(nct, !ok)) {
+      failed = true;
+      break;
     }
-    if (tid == 0 && m + ahead < a.rows) pipe.issue(s, x + (m + ahead) * a.ldx, dy + (m + ahead) * a.lddy);
     rb ^= 1u;
-    if (++s == a.stages) {
-      s = 0;
-      ph ^= 1u;
-    }
+    if (++s == a.stages) s = 0, ph ^= 1u;
     float tot = 0.0f;
-    for (int w = 0; w < nwarps; ++w) tot += red[w].x;
+    for (int w = 0; w < ncw; ++w) tot += red[w].x;
     const float cm = tot * inv_n;
     T* dxrow = dx + m * a.lddx;
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
-      const int v = tid + j * NT;
+      const int v = ct + j * nct;
       if (v < nvec) {
-        float o[E];
+        float wv[E], o[E];
+        V::unpack(*reinterpret_cast<const uint4*>(pipe.param(0) + (size_t)v * 16), wv);
 #pragma unroll
-        for (int e = 0; e < E; ++e) o[e] = r * fmaf(gv[j][e], wr[j][e], -(xv[j][e] * r) * cm);
+        for (int e = 0; e < E; ++e) o[e] = r * fmaf(gv[j][e], woff + wv[e], -(xv[j][e] * r) * cm);
         if (v < nfull) {
           st_stream(dxrow + (size_t)v * E, V::pack(o));
         } else {
@@ -240,13 +246,13 @@ __global__ void __launch_bounds__(norm_max_threads(VPT, true)) rms_bwd_cta(const
       }
     }
   }
-  if (a.ws) {
+  if (a.ws && !failed) {
     float* part = a.ws + (int64_t)blockIdx.x * N;
 #pragma unroll
     for (int j = 0; j < VPT; ++j)
 #pragma unroll
       for (int e = 0; e < E; ++e) {
-        const int col = (tid + j * NT) * E + e;
+        const int col = (ct + j * nct) * E + e;
         if (col < N) part[col] = dwa[j][e];
       }
   }
@@ -466,12 +472,10 @@ void* pick_bwd_t(int vpt, bool cta, int epi, bool gemma) {
   return nullptr;
 }
 
-constexpr int kFwdThreads = 256;  // preferred CTA size when choosing vpt (forward)
-constexpr int kBwdThreads = 512;  // (backward)
 
 gn_status rms_bwd_plan(int64_t rows, int64_t hidden, gn_dtype dt, NormPlan* p, void** kern, int epi,
                        bool gemma, int* grid) {
-  gn_status st = plan_norm(hidden, dt_size(dt), 2, 4, kBwdThreads, p);
+  gn_status st = plan_norm(hidden, dt_size(dt), 2, 1, 4, p);
   if (st != GN_OK) return st;
   *kern = dt == GN_BF16 ? pick_bwd_t<__nv_bfloat16>(p->vpt, p->cta, epi, gemma)
                         : pick_bwd_t<float>(p->vpt, p->cta, epi, gemma);
@@ -501,7 +505,7 @@ extern "C" gn_status gn_rmsnorm_fwd(const void* x, const void* w, void* y, float
   const size_t es = dt_size(dt);
   if (!aligned16(x) || !aligned16(y) || (ld_x * es) % 16 || (ld_y * es) % 16) return GN_ERR_ALIGN;
   NormPlan p;
-  gn_status st = plan_norm(hidden, es, 1, 8, kFwdThreads, &p);
+  gn_status st = plan_norm(hidden, es, 1, 1, 8, &p);
   if (st != GN_OK) return st;
   void* kern = dt == GN_BF16 ? pick_fwd_t<__nv_bfloat16>(p.vpt, p.cta, epi, gemma != 0)
                              : pick_fwd_t<float>(p.vpt, p.cta, epi, gemma != 0);

@@ -1,46 +1,75 @@
-// row_pipe.cuh - the multi-stage TMA row pipeline used by the one-CTA-per-row kernels.
+// row_pipe.cuh - the warp-specialised TMA row pipeline of the one-CTA-per-row kernels.
 //
-// A persistent CTA walks the rows m = blockIdx.x + i * gridDim.x. Row i of the CTA lands in
-// stage i % stages: one thread issues one 1-D bulk copy per input tensor (the row's whole
-// 16-byte vectors; a ragged tail of fewer than 16 bytes is read directly from global memory
-// by the thread that owns it) and every thread waits on the stage's mbarrier. Up to `stages`
-// rows are in flight per CTA, which is what keeps HBM busy without holding the rows in
-// registers while they travel.
+// A persistent CTA walks the rows m = blockIdx.x + i * gridDim.x. Warp 0 is the producer:
+// one lane moves each row (each staged tensor's whole 16-byte vectors; a ragged tail of fewer
+// than 16 bytes is read from global memory by the consumer that owns it) into stage
+// i % stages with 1-D TMA bulk copies counted on the stage's `full` mbarrier, and waits on the
+// stage's `empty` mbarrier before reusing it. The other warps are consumers: they wait on
+// `full`, copy their vectors of the row into registers, and each warp arrives on `empty` at
+// once, so the producer refills the stage while the consumers are still reducing the row.
+// The row statistic is reduced with shuffles within warps and one named barrier over the
+// consumer warps (the producer warp never joins it).
 //
 // Shared memory layout (dynamic, 128-byte aligned):
-//   [0, 128)             mbarriers, one per stage (stages <= 16)
-//   [128, 128 + 1024)    reduction scratch: 2 row parities x 32 warps x float4
-//   [1152, ...)          stages x ntens x slot bytes (slot = row bytes rounded up to 128)
+//   [0, 64)           full mbarriers, one per stage (stages <= 8)
+//   [64, 128)         empty mbarriers
+//   [128, 1152)       reduction scratch: 2 row parities x 32 warps x float4
+//   [1152, ...)       nparams parameter vectors (weight, bias) of the row length
+//   then              stages x ntens row slots (row bytes rounded up to 128)
 #pragma once
 
 #include "gn_common.cuh"
 
 namespace gn {
 
-constexpr int kMaxStages = 16;
+constexpr int kMaxStages = 8;
 constexpr uint32_t kPipeHeader = 128 + 2 * 32 * 16;
 
 __host__ __device__ inline uint32_t pipe_slot_bytes(int64_t row_bytes) {
   return (uint32_t)((row_bytes + 127) / 128 * 128);
 }
 
-__host__ __device__ inline size_t pipe_smem_bytes(int stages, int ntens, int64_t row_bytes) {
-  return kPipeHeader + (size_t)stages * ntens * pipe_slot_bytes(row_bytes);
+__host__ __device__ inline size_t pipe_smem_bytes(int stages, int ntens, int nparams, int64_t row_bytes) {
+  return kPipeHeader + (size_t)(nparams + stages * ntens) * pipe_slot_bytes(row_bytes);
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+// Barrier 1 over the `n` consumer threads, returning the OR of `pred` over them.
+__device__ __forceinline__ int consumers_sync_or(int n, int pred) {
+  int r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.s32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, %2, p;\n\t"
+      "selp.s32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(pred), "r"(n)
+      : "memory");
+  return r;
+}
+
+__device__ __forceinline__ void consumers_sync(int n) { asm volatile("bar.sync 1, %0;" ::"r"(n) : "memory"); }
+
 struct RowPipe {
-  uint64_t* bar;
+  uint64_t* full;
+  uint64_t* empty;
   float4* red;      // [2][32]
+  uint8_t* params;  // nparams slots
   uint8_t* data;
   int stages;
   int ntens;
   uint32_t slot;    // bytes per (stage, tensor) slot
   uint32_t bulk;    // bytes bulk-copied per tensor (whole 16-byte vectors of the row)
 
-  __device__ __forceinline__ RowPipe(uint8_t* smem, int stages_, int ntens_, int64_t row_bytes)
-      : bar(reinterpret_cast<uint64_t*>(smem)),
+  __device__ __forceinline__ RowPipe(uint8_t* smem, int stages_, int ntens_, int nparams, int64_t row_bytes)
+      : full(reinterpret_cast<uint64_t*>(smem)),
+        empty(reinterpret_cast<uint64_t*>(smem) + kMaxStages),
         red(reinterpret_cast<float4*>(smem + 128)),
-        data(smem + kPipeHeader),
+        params(smem + kPipeHeader),
+        data(smem + kPipeHeader + (size_t)nparams * pipe_slot_bytes(row_bytes)),
         stages(stages_),
         ntens(ntens_),
         slot(pipe_slot_bytes(row_bytes)),
@@ -49,41 +78,35 @@ struct RowPipe {
   __device__ __forceinline__ const uint8_t* at(int s, int t) const {
     return data + ((size_t)s * ntens + t) * slot;
   }
+  __device__ __forceinline__ uint8_t* param(int i) const { return params + (size_t)i * slot; }
 
   // thread 0, before the first __syncthreads of the kernel
-  __device__ __forceinline__ void init() const {
-    for (int s = 0; s < stages; ++s) mbar_init(&bar[s], 1);
+  __device__ __forceinline__ void init(int consumer_warps) const {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], (uint32_t)consumer_warps);
+    }
     mbar_fence_init();
   }
 
-  // thread 0: start the copies of one row into stage s (s0..s3 = row start of tensors 0..3;
-  // only the first ntens are used)
-  __device__ __forceinline__ void issue(int s, const void* s0, const void* s1 = nullptr,
-                                        const void* s2 = nullptr, const void* s3 = nullptr) const {
-    mbar_expect_tx(&bar[s], bulk * (uint32_t)ntens);
-    bulk_g2s(const_cast<uint8_t*>(at(s, 0)), s0, bulk, &bar[s]);
-    if (ntens > 1) bulk_g2s(const_cast<uint8_t*>(at(s, 1)), s1, bulk, &bar[s]);
-    if (ntens > 2) bulk_g2s(const_cast<uint8_t*>(at(s, 2)), s2, bulk, &bar[s]);
-    if (ntens > 3) bulk_g2s(const_cast<uint8_t*>(at(s, 3)), s3, bulk, &bar[s]);
-  }
-
-  // wait for the stage-s copy whose completion flips the barrier to phase parity `ph`
-  __device__ __forceinline__ bool wait(int s, uint32_t ph, unsigned* err) const {
-    return mbar_wait(&bar[s], ph, err);
-  }
-
-  // thread 0, after a failed wait for row m (stage s, parity ph) of a grid-stride walk with
-  // stride `step` over `rows`: wait (bounded) for the copies still in flight, so that none
-  // lands in shared memory after the CTA has exited.
-  __device__ __forceinline__ void drain(int64_t m, int64_t step, int64_t rows, int s, uint32_t ph,
-                                        unsigned* err) const {
-    for (int k = 0; k < stages && m < rows; ++k, m += step) {
-      (void)wait(s, ph, err);
-      if (++s == stages) {
-        s = 0;
-        ph ^= 1u;
-      }
+  // Producer lane: stage every row of this CTA's walk; src(m, t) is the start of row m of
+  // staged tensor t. Returns after every copy it issued has landed (bounded waits).
+  template <class Src>
+  __device__ __forceinline__ void produce(int64_t rows, Src src, unsigned* err) const {
+    const int64_t step = gridDim.x;
+    int s = 0;
+    uint32_t ph = 0, used = 0, lastph = 0;
+    int64_t k = 0;
+    for (int64_t m = blockIdx.x; m < rows; m += step, ++k) {
+      if (k >= stages && !mbar_wait(&empty[s], ph ^ 1u, err)) break;
+      mbar_expect_tx(&full[s], bulk * (uint32_t)ntens);
+      for (int t = 0; t < ntens; ++t) bulk_g2s(const_cast<uint8_t*>(at(s, t)), src(m, t), bulk, &full[s]);
+      used |= 1u << s;
+      lastph = (lastph & ~(1u << s)) | (ph << s);
+      if (++s == stages) s = 0, ph ^= 1u;
     }
+    for (int t = 0; t < stages; ++t)
+      if (used & (1u << t)) (void)mbar_wait(&full[t], (lastph >> t) & 1u, err);
   }
 };
 
