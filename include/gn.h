@@ -175,6 +175,28 @@ gn_status gn_qknorm_rope_bwd(const void* q, const void* k, const void* wq, const
                              size_t ws_bytes, int64_t B, int64_t S, int64_t H, int64_t D,
                              int gemma, gn_dtype dt, void* stream);
 
+/* gn_qknorm_rope_bwd without a workspace argument, for callers that cannot allocate device
+ * memory: for example code running inside another framework's callback or plugin whose
+ * device memory is owned and budgeted by that framework, or a process whose whole memory is
+ * reserved by another allocator. The source pages have no counterpart of this call; it only
+ * changes where the per-block weight-gradient partials live.
+ * Arguments, results and errors are those of gn_qknorm_rope_bwd. The library allocates
+ * nothing for it: the partials go to a fixed 1 MiB array inside the library (256-byte
+ * aligned) that every GPU which loads the library holds until the process exits. A call
+ * that would need more (2 * D * 4 bytes per block of the persistent grid, e.g. more than
+ * 1024 blocks at D = 128) returns GN_ERR_WORKSPACE; use gn_qknorm_rope_bwd then.
+ * The first call on a device looks up that array's device address (cudaGetSymbolAddress)
+ * with the device current and caches it: make that first call before any stream capture.
+ * All calls share the array, so calls whose kernels overlap on the GPU (other streams,
+ * other threads) race on it and must be serialised by the caller. Nothing in the array has
+ * to start at zero: each call writes every partial it later reads. */
+gn_status gn_qknorm_rope_bwd_noalloc(const void* q, const void* k, const void* wq,
+                                     const void* wk, const float* cos, const float* sin,
+                                     const float* inv_rms_q, const float* inv_rms_k,
+                                     const void* dq_out, const void* dk_out, void* dq, void* dk,
+                                     float* dwq, float* dwk, int64_t B, int64_t S, int64_t H,
+                                     int64_t D, int gemma, gn_dtype dt, void* stream);
+
 /* ---------------------------------------------------------------- runtime queries
  * Number of kernels this process has launched through libgn (all devices, all threads). */
 uint64_t gn_launch_count(void);

@@ -48,6 +48,8 @@ SIGNATURES = {
     "gn_qknorm_rope_bwd_workspace": (_sz, [_i64, _i64, _i64, _i64, _int]),
     "gn_qknorm_rope_bwd": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                  _vp, _sz, _i64, _i64, _i64, _i64, _int, _int, _vp]),
+    "gn_qknorm_rope_bwd_noalloc": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                         _i64, _i64, _i64, _i64, _int, _int, _vp]),
     "gn_launch_count": (C.c_uint64, []),
     "gn_device_error": (_st, [C.POINTER(C.c_uint), _int]),
     "gn_tune": (_st, [C.c_char_p, _int]),

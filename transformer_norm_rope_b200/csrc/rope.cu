@@ -21,6 +21,8 @@
 //   QK_BWD  : u = rot(dy, cos, -sin), g = u w', dx = r (g - x r mean_d(g x r)),
 //             dw_d += u_d x_d r   (per tensor, fixed-order partials + column reduction)
 // Lanes of one head (D*size/16 of them, a power of two <= 32) reduce with xor shuffles.
+#include <mutex>
+
 #include "gn_host.h"
 #include "row_pipe.cuh"
 
@@ -511,5 +513,84 @@ extern "C" gn_status gn_qknorm_rope_bwd(const void* q, const void* k, const void
   a.sign = 1.0f;
   if ((st = launch(kern, grid, p, a, s)) != GN_OK) return st;
   if (wgrad) return launch_colsum(a.ws, grid, 2 * D, D, dwq, k ? dwk : nullptr, s);
+  return GN_OK;
+}
+
+// ---------------------------------------------------------------- fixed-scratch backward
+// gn_qknorm_rope_bwd_noalloc: the same backward for callers that cannot allocate device
+// memory. Its weight-gradient partials go to this file-scope array instead of a caller
+// workspace. Every device that loads the library holds the array until the process exits.
+// In host code the array's name is only a host-side stand-in; the device address comes from
+// cudaGetSymbolAddress, taken once per device with that device current.
+
+static constexpr size_t kQkFixedScratchBytes = 1u << 20;  // 1 MiB
+static __device__ __align__(256) float gn_qk_fixed_scratch[kQkFixedScratchBytes / sizeof(float)];
+
+namespace gn {
+namespace {
+constexpr int kScratchDevices = 64;
+std::mutex g_scratch_mu;
+float* g_scratch_ptr[kScratchDevices];
+
+// device address of gn_qk_fixed_scratch on the current device (nullptr on error)
+float* fixed_scratch() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kScratchDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, gn_qk_fixed_scratch) != cudaSuccess || !p) return nullptr;
+    g_scratch_ptr[dev] = static_cast<float*>(p);
+  }
+  return g_scratch_ptr[dev];
+}
+}  // namespace
+}  // namespace gn
+
+extern "C" gn_status gn_qknorm_rope_bwd_noalloc(const void* q, const void* k, const void* wq, const void* wk,
+                                                const float* cos, const float* sin, const float* inv_rms_q,
+                                                const float* inv_rms_k, const void* dq_out, const void* dk_out,
+                                                void* dq, void* dk, float* dwq, float* dwk, int64_t B, int64_t S,
+                                                int64_t H, int64_t D, int gemma, gn_dtype dt, void* stream) {
+  gn_status st = check_common(B, S, H, D, dt);
+  if (st != GN_OK) return st;
+  if (!norm_head_ok(D, dt)) return GN_ERR_UNSUPPORTED;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (B * S * H == 0) {
+    if (dwq && cudaMemsetAsync(dwq, 0, (size_t)D * sizeof(float), s) != cudaSuccess) return GN_ERR_CUDA;
+    if (dwk && cudaMemsetAsync(dwk, 0, (size_t)D * sizeof(float), s) != cudaSuccess) return GN_ERR_CUDA;
+    return GN_OK;
+  }
+  if (!q || !wq || !cos || !sin || !inv_rms_q || !dq_out || !dq) return GN_ERR_NULL;
+  if (k && (!wk || !inv_rms_k || !dk_out || !dk)) return GN_ERR_NULL;
+  if (!aligned16(q) || !aligned16(dq_out) || !aligned16(dq) || !aligned16(cos) || !aligned16(sin) ||
+      (k && (!aligned16(k) || !aligned16(dk_out) || !aligned16(dk))))
+    return GN_ERR_ALIGN;
+  const int ntens = k ? 2 : 1;
+  RopePlan p;
+  void* kern = nullptr;
+  int grid = 0;
+  if ((st = setup(B, S, H, D, ntens, QK_BWD, dt, gemma != 0, &p, &kern, &grid)) != GN_OK) return st;
+  const bool wgrad = dwq || (k && dwk);
+  float* scratch = nullptr;
+  if (wgrad) {
+    // one partial row of 2*D floats per block; every row read afterwards is written first
+    if ((size_t)grid * 2 * (size_t)D * sizeof(float) > kQkFixedScratchBytes) return GN_ERR_WORKSPACE;
+    scratch = fixed_scratch();
+    if (!scratch) return GN_ERR_CUDA;
+  }
+  RopeArgs a{};
+  a.x[0] = q, a.x[1] = k;
+  a.dy[0] = dq_out, a.dy[1] = dk_out;
+  a.out[0] = dq, a.out[1] = dk;
+  a.w[0] = wq, a.w[1] = wk;
+  a.stat[0] = const_cast<float*>(inv_rms_q), a.stat[1] = const_cast<float*>(inv_rms_k);
+  a.cos = cos, a.sin = sin;
+  a.ws = scratch;
+  a.B = (int)B, a.S = (int)S, a.H = (int)H, a.D = (int)D;
+  a.ntens = ntens;
+  a.sign = 1.0f;
+  if ((st = launch(kern, grid, p, a, s)) != GN_OK) return st;
+  if (wgrad) return launch_colsum(scratch, grid, 2 * D, D, dwq, k ? dwk : nullptr, s);
   return GN_OK;
 }
