@@ -62,6 +62,44 @@ struct Vec<__nv_bfloat16> {
   __device__ __forceinline__ static void store1(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
 };
 
+// ---------------------------------------------------------------- packed fp32 pairs
+// sm_100 executes one FMA / MUL / ADD on two fp32 lanes per instruction (CUDA's __ffma2_rn,
+// __fmul2_rn, __fadd2_rn; round to nearest even per lane, like the scalar forms).
+
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 dup2(float a) { return make_float2(a, a); }
+
+// a 16-byte vector as E/2 element pairs (elements 2i, 2i+1 in .x, .y)
+template <typename T>
+__device__ __forceinline__ void unpack2(const uint4& u, float2 (&f)[Vec<T>::N / 2]) {
+  if constexpr (sizeof(T) == 2) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) f[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u));
+  } else {
+    f[0] = make_float2(__uint_as_float(u.x), __uint_as_float(u.y));
+    f[1] = make_float2(__uint_as_float(u.z), __uint_as_float(u.w));
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ uint4 pack2(const float2 (&f)[Vec<T>::N / 2]) {
+  if constexpr (sizeof(T) == 2) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __nv_bfloat162 h = __float22bfloat162_rn(f[i]);
+      w[i] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+  } else {
+    return make_uint4(__float_as_uint(f[0].x), __float_as_uint(f[0].y), __float_as_uint(f[1].x),
+                      __float_as_uint(f[1].y));
+  }
+}
+
 // streaming 16-byte global access (read-once / write-once data)
 __device__ __forceinline__ uint4 ld_stream(const void* p) { return __ldcs(reinterpret_cast<const uint4*>(p)); }
 __device__ __forceinline__ void st_stream(void* p, const uint4& v) { __stcs(reinterpret_cast<uint4*>(p), v); }
@@ -204,6 +242,41 @@ __device__ __forceinline__ float epi_grad(float z) {
     return s * fmaf(z, 1.0f - s, 1.0f);
   } else {
     return 1.0f;
+  }
+}
+
+// The same epilogues on a pair of lanes with packed fp32x2 arithmetic (tanh / exp per lane).
+template <int EPI, bool FAST>
+__device__ __forceinline__ float2 epi_fwd2(float2 z) {
+  if constexpr (EPI == EPI_GELU_TANH) {
+    const float2 z2 = mul2(z, z);
+    const float2 arg = mul2(fma2(z2, dup2(kGeluK * kGeluC), dup2(kGeluK)), z);  // k (z + c z^3)
+    const float2 t = make_float2(tanh_f<FAST>(arg.x), tanh_f<FAST>(arg.y));
+    const float2 h = mul2(z, dup2(0.5f));
+    return fma2(h, t, h);
+  } else if constexpr (EPI == EPI_SILU) {
+    return mul2(z, make_float2(sigmoid_f<FAST>(z.x), sigmoid_f<FAST>(z.y)));
+  } else {
+    return z;
+  }
+}
+
+template <int EPI, bool FAST>
+__device__ __forceinline__ float2 epi_grad2(float2 z) {
+  if constexpr (EPI == EPI_GELU_TANH) {
+    // 0.5 (1 + t) + 0.5 z (1 - t^2) k (1 + 3 c z^2)
+    const float2 z2 = mul2(z, z);
+    const float2 arg = mul2(fma2(z2, dup2(kGeluK * kGeluC), dup2(kGeluK)), z);
+    const float2 t = make_float2(tanh_f<FAST>(arg.x), tanh_f<FAST>(arg.y));
+    const float2 dt = fma2(mul2(t, dup2(-1.0f)), t, dup2(1.0f));
+    const float2 k3 = fma2(z2, dup2(3.0f * kGeluK * kGeluC), dup2(kGeluK));
+    const float2 a = fma2(t, dup2(0.5f), dup2(0.5f));
+    return fma2(mul2(mul2(z, dt), k3), dup2(0.5f), a);
+  } else if constexpr (EPI == EPI_SILU) {
+    const float2 s = make_float2(sigmoid_f<FAST>(z.x), sigmoid_f<FAST>(z.y));
+    return mul2(s, fma2(z, add2(dup2(1.0f), mul2(s, dup2(-1.0f))), dup2(1.0f)));
+  } else {
+    return dup2(1.0f);
   }
 }
 

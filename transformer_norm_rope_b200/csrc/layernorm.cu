@@ -10,9 +10,9 @@
 //             dx = s (g w - mean(g w) - xhat mean(g w xhat)), dw = sum g xhat, db = sum g
 //
 // The row is read from HBM once and kept in registers, so the variance is taken around the
-// mean (no E[x^2] - E[x]^2 cancellation): every thread forms (count, mean, M2) of its own
-// elements in two register passes, and the triples are combined with Chan et al.'s pairwise
-// update (warp tree, then the per-warp results in warp order after one CTA barrier).
+// mean (no E[x^2] - E[x]^2 cancellation): the long-row kernel reduces the sum, then the
+// centred sum of squares (two barriers over the consumer warps); the short-row kernel forms
+// (count, mean, M2) per thread and combines the triples with Chan et al.'s pairwise update.
 #include "norm_plan.h"
 
 namespace gn {
@@ -119,7 +119,8 @@ __device__ __forceinline__ void load_affine(const LnFwdArgs& a, int base, int st
 
 // ---------------------------------------------------------------- CTA path (long rows)
 // Warp 0 produces (row_pipe.cuh); warps 1.. consume. Consumer thread ct owns the vectors
-// v = ct + j * nct (j < VPT) of every row. Weight and bias live in shared memory.
+// v = ct + j * nct (j < VPT) of every row. Weight and bias live in shared memory. The
+// arithmetic runs on element pairs with packed fp32x2 instructions.
 
 template <typename T>
 __device__ __forceinline__ void stage_param(uint8_t* dst, const T* src, int N, int nvec, float dflt, int ct,
@@ -132,10 +133,40 @@ __device__ __forceinline__ void stage_param(uint8_t* dst, const T* src, int N, i
   }
 }
 
+template <typename T>
+__device__ __forceinline__ void load_pairs(const uint8_t* st, const T* row, int v, int nfull, int N, bool ok,
+                                           float2 (&f)[Vec<T>::N / 2]) {
+  constexpr int E = Vec<T>::N;
+  if (ok && v < nfull) {
+    unpack2<T>(*reinterpret_cast<const uint4*>(st + (size_t)v * 16), f);
+  } else {
+#pragma unroll
+    for (int h = 0; h < E / 2; ++h) {
+      const int col = v * E + 2 * h;
+      f[h].x = (ok && col < N) ? Vec<T>::load1(row + col) : 0.0f;
+      f[h].y = (ok && col + 1 < N) ? Vec<T>::load1(row + col + 1) : 0.0f;
+    }
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ void store_pairs(T* row, int v, int nfull, int N, const float2 (&f)[Vec<T>::N / 2]) {
+  constexpr int E = Vec<T>::N;
+  if (v < nfull) {
+    st_stream(row + (size_t)v * E, pack2<T>(f));
+  } else {
+#pragma unroll
+    for (int h = 0; h < E / 2; ++h) {
+      const int col = v * E + 2 * h;
+      if (col < N) Vec<T>::store1(row + col, f[h].x);
+      if (col + 1 < N) Vec<T>::store1(row + col + 1, f[h].y);
+    }
+  }
+}
+
 template <typename T, int VPT, int EPI>
 __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT)) ln_fwd_cta(const LnFwdArgs a) {
-  using V = Vec<T>;
-  constexpr int E = V::N;
+  constexpr int E = Vec<T>::N, H = E / 2;
   constexpr bool FAST = fast_math_for<T>();
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -165,54 +196,66 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT)) ln_fwd_
   int s = 0;
   uint32_t ph = 0, rb = 0;
   for (int64_t m = blockIdx.x; m < a.rows; m += step) {
-    const T* xrow = x + m * a.ldx;
     const bool ok = __all_sync(0xffffffffu, mbar_wait(&pipe.full[s], ph, a.err));
-    const uint8_t* st = pipe.at(s, 0);
-    float xv[VPT][E];
+    float2 xv[VPT][H];
+    float2 sx2 = dup2(0.0f);
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
-      const int v = ct + j * nct;
-      if (ok && v < nfull) {
-        V::unpack(*reinterpret_cast<const uint4*>(st + (size_t)v * 16), xv[j]);
-      } else {
+      load_pairs<T>(pipe.at(s, 0), x + m * a.ldx, ct + j * nct, nfull, N, ok, xv[j]);
 #pragma unroll
-        for (int e = 0; e < E; ++e) xv[j][e] = (ok && e < cnt[j]) ? V::load1(xrow + v * E + e) : 0.0f;
-      }
+      for (int h = 0; h < H; ++h) sx2 = add2(sx2, xv[j][h]);  // invalid elements are 0
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&pipe.empty[s]);
-    float n, mu, M2;
-    thread_stats<VPT, E>(xv, cnt, n, mu, M2);
-    group_stats(n, mu, M2, 32);
+    // two reductions over the register-resident row: the mean, then the sum of squares
+    // around it (no E[x^2] - E[x]^2 cancellation); invalid elements are masked
+    const float sx = group_sum<32>(sx2.x + sx2.y);
     float4* red = pipe.red + rb * 32;
-    if (lane == 0) red[cw] = make_float4(n, mu, M2, 0.0f);
+    if (lane == 0) red[cw].x = sx;
     if (consumers_sync_or(nct, !ok)) return;
+    float tot = 0.0f;
+    for (int w = 0; w < ncw; ++w) tot += red[w].x;
+    const float mu = tot * inv_n;
+    const float2 nmu = dup2(-mu);
+    float2 q2 = dup2(0.0f);
+    float qt = 0.0f;
+#pragma unroll
+    for (int j = 0; j < VPT; ++j) {
+      if (cnt[j] == E) {
+#pragma unroll
+        for (int h = 0; h < H; ++h) {
+          const float2 d = add2(xv[j][h], nmu);
+          q2 = fma2(d, d, q2);
+        }
+      } else {
+#pragma unroll
+        for (int h = 0; h < H; ++h) {
+          const float d0 = xv[j][h].x - mu, d1 = xv[j][h].y - mu;
+          qt = 2 * h < cnt[j] ? fmaf(d0, d0, qt) : qt;
+          qt = 2 * h + 1 < cnt[j] ? fmaf(d1, d1, qt) : qt;
+        }
+      }
+    }
+    const float q = group_sum<32>(q2.x + q2.y + qt);
+    if (lane == 0) red[cw].y = q;
+    consumers_sync(nct);
+    float tq = 0.0f;
+    for (int w = 0; w < ncw; ++w) tq += red[w].y;
     rb ^= 1u;
     if (++s == a.stages) s = 0, ph ^= 1u;
-    n = 0.0f, mu = 0.0f, M2 = 0.0f;
-    for (int w = 0; w < ncw; ++w) {
-      const float4 r = red[w];
-      chan_merge(n, mu, M2, r.x, r.y, r.z);
-    }
-    const float rs = rsqrtf(fmaf(M2, inv_n, a.eps));
-    const float nmr = -mu * rs;
+    const float rs = rsqrtf(fmaf(tq, inv_n, a.eps));
+    const float2 rs2 = dup2(rs), nmr2 = dup2(-mu * rs);
     T* yrow = y + m * a.ldy;
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
       const int v = ct + j * nct;
       if (v < nvec) {
-        float wv[E], bv[E], o[E];
-        V::unpack(*reinterpret_cast<const uint4*>(pipe.param(0) + (size_t)v * 16), wv);
-        V::unpack(*reinterpret_cast<const uint4*>(pipe.param(1) + (size_t)v * 16), bv);
+        float2 wv[H], bv[H], o[H];
+        unpack2<T>(*reinterpret_cast<const uint4*>(pipe.param(0) + (size_t)v * 16), wv);
+        unpack2<T>(*reinterpret_cast<const uint4*>(pipe.param(1) + (size_t)v * 16), bv);
 #pragma unroll
-        for (int e = 0; e < E; ++e) o[e] = epi_fwd<EPI, FAST>(fmaf(fmaf(xv[j][e], rs, nmr), wv[e], bv[e]));
-        if (v < nfull) {
-          st_stream(yrow + (size_t)v * E, V::pack(o));
-        } else {
-#pragma unroll
-          for (int e = 0; e < E; ++e)
-            if (e < cnt[j]) V::store1(yrow + v * E + e, o[e]);
-        }
+        for (int h = 0; h < H; ++h) o[h] = epi_fwd2<EPI, FAST>(fma2(fma2(xv[j][h], rs2, nmr2), wv[h], bv[h]));
+        store_pairs<T>(yrow, v, nfull, N, o);
       }
     }
     if (ct == 0) {
@@ -224,8 +267,7 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT)) ln_fwd_
 
 template <typename T, int VPT, int EPI>
 __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT, true)) ln_bwd_cta(const LnBwdArgs a) {
-  using V = Vec<T>;
-  constexpr int E = V::N;
+  constexpr int E = Vec<T>::N, H = E / 2;
   constexpr bool FAST = fast_math_for<T>();
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -249,11 +291,11 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT, true)) l
   stage_param(pipe.param(0), static_cast<const T*>(a.w), N, nvec, 1.0f, ct, nct);
   stage_param(pipe.param(1), static_cast<const T*>(a.b), N, nvec, 0.0f, ct, nct);
   consumers_sync(nct);
-  float dwa[VPT][E], dba[VPT][E];
+  float2 dwa[VPT][H], dba[VPT][H];
 #pragma unroll
   for (int j = 0; j < VPT; ++j)
 #pragma unroll
-    for (int e = 0; e < E; ++e) dwa[j][e] = dba[j][e] = 0.0f;
+    for (int h = 0; h < H; ++h) dwa[j][h] = dba[j][h] = dup2(0.0f);
   const float inv_n = 1.0f / (float)N;
   const int64_t step = gridDim.x;
   int s = 0;
@@ -261,53 +303,43 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT, true)) l
   bool failed = false;
   for (int64_t m = blockIdx.x; m < a.rows; m += step) {
     const float mu = __ldg(a.mean + m), rs = __ldg(a.rstd + m);
-    const T* xrow = x + m * a.ldx;
-    const T* gyrow = dy + m * a.lddy;
+    const float2 rs2 = dup2(rs), nmr2 = dup2(-mu * rs);
     const bool ok = __all_sync(0xffffffffu, mbar_wait(&pipe.full[s], ph, a.err));
-    const uint8_t* sx = pipe.at(s, 0);
-    const uint8_t* sg = pipe.at(s, 1);
-    float xv[VPT][E], gv[VPT][E];
+    uint4 xr[VPT];  // x stays packed between the two phases (unpacked on use)
+    float2 gv[VPT][H];
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
       const int v = ct + j * nct;
-      if (ok && v < nfull) {
-        V::unpack(*reinterpret_cast<const uint4*>(sx + (size_t)v * 16), xv[j]);
-        V::unpack(*reinterpret_cast<const uint4*>(sg + (size_t)v * 16), gv[j]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-          const int col = v * E + e;
-          const bool in = ok && v < nvec && col < N;
-          xv[j][e] = in ? V::load1(xrow + col) : 0.0f;
-          gv[j][e] = in ? V::load1(gyrow + col) : 0.0f;
-        }
-      }
+      float2 xt[H];
+      load_pairs<T>(pipe.at(s, 0), x + m * a.ldx, v, nfull, N, ok, xt);
+      xr[j] = pack2<T>(xt);  // exact: the values came from T
+      load_pairs<T>(pipe.at(s, 1), dy + m * a.lddy, v, nfull, N, ok, gv[j]);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&pipe.empty[s]);
-    const float nmr = -mu * rs;
-    float s1 = 0.0f, s2 = 0.0f;
+    float2 s12 = dup2(0.0f), s22 = dup2(0.0f);
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
       const int v = ct + j * nct;
       const size_t vo = (size_t)(v < nvec ? v : 0) * 16;
-      float wv[E], bv[E];
-      V::unpack(*reinterpret_cast<const uint4*>(pipe.param(0) + vo), wv);
-      V::unpack(*reinterpret_cast<const uint4*>(pipe.param(1) + vo), bv);
+      float2 wv[H], bv[H], xv[H];
+      unpack2<T>(*reinterpret_cast<const uint4*>(pipe.param(0) + vo), wv);
+      unpack2<T>(*reinterpret_cast<const uint4*>(pipe.param(1) + vo), bv);
+      unpack2<T>(xr[j], xv);
 #pragma unroll
-      for (int e = 0; e < E; ++e) {
-        const float xh = fmaf(xv[j][e], rs, nmr);
-        const float g = gv[j][e] * epi_grad<EPI, FAST>(fmaf(xh, wv[e], bv[e]));
-        const float gw = g * wv[e];
-        gv[j][e] = g;
-        s1 += gw;
-        s2 = fmaf(gw, xh, s2);
-        dwa[j][e] = fmaf(g, xh, dwa[j][e]);
-        dba[j][e] += g;
+      for (int h = 0; h < H; ++h) {
+        const float2 xh = fma2(xv[h], rs2, nmr2);
+        const float2 g = EPI == EPI_NONE ? gv[j][h] : mul2(gv[j][h], epi_grad2<EPI, FAST>(fma2(xh, wv[h], bv[h])));
+        const float2 gw = mul2(g, wv[h]);
+        gv[j][h] = g;
+        s12 = add2(s12, gw);
+        s22 = fma2(gw, xh, s22);
+        dwa[j][h] = fma2(g, xh, dwa[j][h]);
+        dba[j][h] = add2(dba[j][h], g);
       }
     }
-    s1 = group_sum<32>(s1);
-    s2 = group_sum<32>(s2);
+    const float s1 = group_sum<32>(s12.x + s12.y);
+    const float s2 = group_sum<32>(s22.x + s22.y);
     float4* red = pipe.red + rb * 32;
     if (lane == 0) red[cw] = make_float4(s1, s2, 0.0f, 0.0f);
     if (consumers_sync_or(nct, !ok)) {
@@ -321,26 +353,21 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT, true)) l
       t1 += red[w].x;
       t2 += red[w].y;
     }
-    const float c1 = t1 * inv_n, c2 = t2 * inv_n;
+    const float2 nc1 = dup2(-t1 * inv_n), nc2 = dup2(-t2 * inv_n);
     T* dxrow = dx + m * a.lddx;
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
       const int v = ct + j * nct;
       if (v < nvec) {
-        float wv[E], o[E];
-        V::unpack(*reinterpret_cast<const uint4*>(pipe.param(0) + (size_t)v * 16), wv);
+        float2 wv[H], xv[H], o[H];
+        unpack2<T>(*reinterpret_cast<const uint4*>(pipe.param(0) + (size_t)v * 16), wv);
+        unpack2<T>(xr[j], xv);
 #pragma unroll
-        for (int e = 0; e < E; ++e) {
-          const float xh = fmaf(xv[j][e], rs, nmr);
-          o[e] = rs * (fmaf(gv[j][e], wv[e], -c1) - xh * c2);
+        for (int h = 0; h < H; ++h) {
+          const float2 xh = fma2(xv[h], rs2, nmr2);
+          o[h] = mul2(rs2, fma2(gv[j][h], wv[h], fma2(xh, nc2, nc1)));
         }
-        if (v < nfull) {
-          st_stream(dxrow + (size_t)v * E, V::pack(o));
-        } else {
-#pragma unroll
-          for (int e = 0; e < E; ++e)
-            if (v * E + e < N) V::store1(dxrow + v * E + e, o[e]);
-        }
+        store_pairs<T>(dxrow, v, nfull, N, o);
       }
     }
   }
@@ -349,11 +376,15 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT, true)) l
 #pragma unroll
     for (int j = 0; j < VPT; ++j)
 #pragma unroll
-      for (int e = 0; e < E; ++e) {
-        const int col = (ct + j * nct) * E + e;
+      for (int h = 0; h < H; ++h) {
+        const int col = (ct + j * nct) * E + 2 * h;
         if (col < N) {
-          part[col] = dwa[j][e];
-          part[N + col] = dba[j][e];
+          part[col] = dwa[j][h].x;
+          part[N + col] = dba[j][h].x;
+        }
+        if (col + 1 < N) {
+          part[col + 1] = dwa[j][h].y;
+          part[N + col + 1] = dba[j][h].y;
         }
       }
   }
@@ -569,7 +600,7 @@ void* pick_ln_t(int vpt, bool cta, int epi) {
 
 gn_status ln_plan(int64_t rows, int64_t hidden, gn_dtype dt, bool bwd, int epi, NormPlan* p, void** kern,
                   int* grid) {
-  gn_status st = plan_norm(hidden, dt_size(dt), bwd ? 2 : 1, 2, bwd ? 4 : 8, p);
+  gn_status st = plan_norm(hidden, dt_size(dt), bwd ? 2 : 1, 2, bwd ? 4 : 8, bwd ? 320 : 160, p);
   if (st != GN_OK) return st;
   if (dt == GN_BF16)
     *kern = bwd ? pick_ln_t<__nv_bfloat16, true>(p->vpt, p->cta, epi) : pick_ln_t<__nv_bfloat16, false>(p->vpt, p->cta, epi);

@@ -41,8 +41,10 @@ inline int pow2_ceil(int v) {
 }
 
 // ntens: row tensors staged per row (1 forward, 2 backward); nparams: per-column parameter
-// vectors kept in shared memory (weight, bias); max_vpt: 8 forward, 4 backward.
-inline gn_status plan_norm(int64_t N, size_t es, int ntens, int nparams, int max_vpt, NormPlan* p) {
+// vectors kept in shared memory (weight, bias); max_vpt: 8 forward, 4 backward; target:
+// preferred consumer threads (the forward keeps more of the row per thread, which spreads
+// the per-row reduction over more elements).
+inline gn_status plan_norm(int64_t N, size_t es, int ntens, int nparams, int max_vpt, int target, NormPlan* p) {
   const int vec = (int)(16 / es);
   const int64_t nvec = (N + vec - 1) / vec;
   if (nvec <= kGroupMaxVec) {
@@ -59,7 +61,7 @@ inline gn_status plan_norm(int64_t N, size_t es, int ntens, int nparams, int max
   int vpt = g_tune.vpt;
   if (vpt == 0) {
     vpt = 1;
-    while (vpt < max_vpt && (nvec + vpt - 1) / vpt > kNormMaxConsumers) vpt <<= 1;
+    while (vpt < max_vpt && (nvec + vpt - 1) / vpt > target) vpt <<= 1;
   }
   if (vpt > max_vpt) return GN_ERR_UNSUPPORTED;
   const int64_t consumers = ((nvec + vpt - 1) / vpt + 31) / 32 * 32;
@@ -70,7 +72,7 @@ inline gn_status plan_norm(int64_t N, size_t es, int ntens, int nparams, int max
   const size_t slot = pipe_slot_bytes(row_bytes);
   int stages = g_tune.stages;
   if (stages == 0) {
-    stages = (int)(65536 / (slot * ntens));
+    stages = (int)((ntens > 1 ? 65536 : 49152) / (slot * ntens));
     stages = stages < 2 ? 2 : stages > kMaxStages ? kMaxStages : stages;
   }
   if (stages > kMaxStages) stages = kMaxStages;

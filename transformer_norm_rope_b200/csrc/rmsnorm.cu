@@ -44,7 +44,8 @@ struct RmsBwdArgs {
 // ---------------------------------------------------------------- CTA path (long rows)
 // Warp 0 produces (row_pipe.cuh); warps 1.. consume. Consumer thread ct owns the vectors
 // v = ct + j * nct (j < VPT) of every row, so its columns - and its share of the weight
-// gradient - never change. The weight lives in shared memory (one copy per CTA).
+// gradient - never change. The weight lives in shared memory (one copy per CTA). The
+// arithmetic runs on element pairs with packed fp32x2 instructions.
 
 template <typename T>
 __device__ __forceinline__ void stage_param(uint8_t* dst, const T* src, int N, int nvec, float dflt, int ct,
@@ -57,14 +58,46 @@ __device__ __forceinline__ void stage_param(uint8_t* dst, const T* src, int N, i
   }
 }
 
+// vector v of a row as element pairs: whole vectors from the stage, the ragged tail (and
+// vectors past the row) element by element from global memory, zero beyond the row
+template <typename T>
+__device__ __forceinline__ void load_pairs(const uint8_t* st, const T* row, int v, int nfull, int N, bool ok,
+                                           float2 (&f)[Vec<T>::N / 2]) {
+  constexpr int E = Vec<T>::N;
+  if (ok && v < nfull) {
+    unpack2<T>(*reinterpret_cast<const uint4*>(st + (size_t)v * 16), f);
+  } else {
+#pragma unroll
+    for (int h = 0; h < E / 2; ++h) {
+      const int col = v * E + 2 * h;
+      f[h].x = (ok && col < N) ? Vec<T>::load1(row + col) : 0.0f;
+      f[h].y = (ok && col + 1 < N) ? Vec<T>::load1(row + col + 1) : 0.0f;
+    }
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ void store_pairs(T* row, int v, int nfull, int N, const float2 (&f)[Vec<T>::N / 2]) {
+  constexpr int E = Vec<T>::N;
+  if (v < nfull) {
+    st_stream(row + (size_t)v * E, pack2<T>(f));
+  } else {
+#pragma unroll
+    for (int h = 0; h < E / 2; ++h) {
+      const int col = v * E + 2 * h;
+      if (col < N) Vec<T>::store1(row + col, f[h].x);
+      if (col + 1 < N) Vec<T>::store1(row + col + 1, f[h].y);
+    }
+  }
+}
+
 template <typename T, int VPT, int EPI, bool GEMMA>
 __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT)) rms_fwd_cta(const RmsFwdArgs a) {
-  using V = Vec<T>;
-  constexpr int E = V::N;
+  constexpr int H = Vec<T>::N / 2;
   constexpr bool FAST = fast_math_for<T>();
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int N = a.N, nfull = N / E, nvec = (N + E - 1) / E;
+  const int N = a.N, nfull = N / Vec<T>::N, nvec = (N + Vec<T>::N - 1) / Vec<T>::N;
   const RowPipe pipe(smem, a.stages, 1, 1, (int64_t)N * sizeof(T));
   const T* x = static_cast<const T*>(a.x);
   T* y = static_cast<T*>(a.y);
@@ -83,29 +116,18 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT)) rms_fwd
   int s = 0;
   uint32_t ph = 0, rb = 0;
   for (int64_t m = blockIdx.x; m < a.rows; m += step) {
-    const T* xrow = x + m * a.ldx;
     const bool ok = __all_sync(0xffffffffu, mbar_wait(&pipe.full[s], ph, a.err));
-    const uint8_t* st = pipe.at(s, 0);
-    float xv[VPT][E];
-    float ss = 0.0f;
+    float2 xv[VPT][H];
+    float2 ss2 = dup2(0.0f);
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
-      const int v = ct + j * nct;
-      if (ok && v < nfull) {
-        V::unpack(*reinterpret_cast<const uint4*>(st + (size_t)v * 16), xv[j]);
-      } else {
+      load_pairs<T>(pipe.at(s, 0), x + m * a.ldx, ct + j * nct, nfull, N, ok, xv[j]);
 #pragma unroll
-        for (int e = 0; e < E; ++e) {
-          const int col = v * E + e;
-          xv[j][e] = (ok && v < nvec && col < N) ? V::load1(xrow + col) : 0.0f;
-        }
-      }
-#pragma unroll
-      for (int e = 0; e < E; ++e) ss = fmaf(xv[j][e], xv[j][e], ss);
+      for (int h = 0; h < H; ++h) ss2 = fma2(xv[j][h], xv[j][h], ss2);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&pipe.empty[s]);
-    ss = group_sum<32>(ss);
+    const float ss = group_sum<32>(ss2.x + ss2.y);
     float4* red = pipe.red + rb * 32;
     if (lane == 0) red[cw].x = ss;
     if (consumers_sync_or(nct, !ok)) return;
@@ -114,22 +136,20 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT)) rms_fwd
     float tot = 0.0f;
     for (int w = 0; w < ncw; ++w) tot += red[w].x;
     const float r = rsqrtf(fmaf(tot, inv_n, a.eps));
+    const float2 r2 = dup2(r);
     T* yrow = y + m * a.ldy;
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
       const int v = ct + j * nct;
       if (v < nvec) {
-        float wv[E], o[E];
-        V::unpack(*reinterpret_cast<const uint4*>(pipe.param(0) + (size_t)v * 16), wv);
+        float2 wv[H], o[H];
+        unpack2<T>(*reinterpret_cast<const uint4*>(pipe.param(0) + (size_t)v * 16), wv);
 #pragma unroll
-        for (int e = 0; e < E; ++e) o[e] = epi_fwd<EPI, FAST>(xv[j][e] * r * ((GEMMA ? 1.0f : 0.0f) + wv[e]));
-        if (v < nfull) {
-          st_stream(yrow + (size_t)v * E, V::pack(o));
-        } else {
-#pragma unroll
-          for (int e = 0; e < E; ++e)
-            if (v * E + e < N) V::store1(yrow + v * E + e, o[e]);
+        for (int h = 0; h < H; ++h) {
+          const float2 wp = GEMMA ? add2(wv[h], dup2(1.0f)) : wv[h];
+          o[h] = epi_fwd2<EPI, FAST>(mul2(mul2(xv[j][h], r2), wp));
         }
+        store_pairs<T>(yrow, v, nfull, N, o);
       }
     }
     if (ct == 0 && a.inv_rms) a.inv_rms[m] = r;
@@ -138,8 +158,7 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT)) rms_fwd
 
 template <typename T, int VPT, int EPI, bool GEMMA>
 __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT, true)) rms_bwd_cta(const RmsBwdArgs a) {
-  using V = Vec<T>;
-  constexpr int E = V::N;
+  constexpr int E = Vec<T>::N, H = E / 2;
   constexpr bool FAST = fast_math_for<T>();
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -162,60 +181,50 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT, true)) r
   const int ct = tid - 32, nct = ncw * 32, cw = warp - 1;
   stage_param(pipe.param(0), static_cast<const T*>(a.w), N, nvec, 0.0f, ct, nct);
   consumers_sync(nct);
-  float dwa[VPT][E];
+  float2 dwa[VPT][H];
 #pragma unroll
   for (int j = 0; j < VPT; ++j)
 #pragma unroll
-    for (int e = 0; e < E; ++e) dwa[j][e] = 0.0f;
+    for (int h = 0; h < H; ++h) dwa[j][h] = dup2(0.0f);
   const float inv_n = 1.0f / (float)N;
-  const float woff = GEMMA ? 1.0f : 0.0f;
   const int64_t step = gridDim.x;
   int s = 0;
   uint32_t ph = 0, rb = 0;
   bool failed = false;
   for (int64_t m = blockIdx.x; m < a.rows; m += step) {
     const float r = __ldg(a.inv_rms + m);
-    const T* xrow = x + m * a.ldx;
-    const T* gyrow = dy + m * a.lddy;
+    const float2 r2 = dup2(r);
     const bool ok = __all_sync(0xffffffffu, mbar_wait(&pipe.full[s], ph, a.err));
-    const uint8_t* sx = pipe.at(s, 0);
-    const uint8_t* sg = pipe.at(s, 1);
-    float xv[VPT][E], gv[VPT][E];
+    uint4 xr[VPT];  // x stays packed between the two phases (unpacked on use)
+    float2 gv[VPT][H];
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
       const int v = ct + j * nct;
-      if (ok && v < nfull) {
-        V::unpack(*reinterpret_cast<const uint4*>(sx + (size_t)v * 16), xv[j]);
-        V::unpack(*reinterpret_cast<const uint4*>(sg + (size_t)v * 16), gv[j]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-          const int col = v * E + e;
-          const bool in = ok && v < nvec && col < N;
-          xv[j][e] = in ? V::load1(xrow + col) : 0.0f;
-          gv[j][e] = in ? V::load1(gyrow + col) : 0.0f;
-        }
-      }
+      float2 xt[H];
+      load_pairs<T>(pipe.at(s, 0), x + m * a.ldx, v, nfull, N, ok, xt);
+      xr[j] = pack2<T>(xt);  // exact: the values came from T
+      load_pairs<T>(pipe.at(s, 1), dy + m * a.lddy, v, nfull, N, ok, gv[j]);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&pipe.empty[s]);
-    float c = 0.0f;
+    float2 c2 = dup2(0.0f);
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
       const int v = ct + j * nct;
-      float wv[E];
-      V::unpack(*reinterpret_cast<const uint4*>(pipe.param(0) + (size_t)(v < nvec ? v : 0) * 16), wv);
+      float2 wv[H], xv[H];
+      unpack2<T>(*reinterpret_cast<const uint4*>(pipe.param(0) + (size_t)(v < nvec ? v : 0) * 16), wv);
+      unpack2<T>(xr[j], xv);
 #pragma unroll
-      for (int e = 0; e < E; ++e) {
-        const float wp = woff + wv[e];
-        const float xh = xv[j][e] * r;
-        const float g = gv[j][e] * epi_grad<EPI, FAST>(xh * wp);
-        gv[j][e] = g;
-        c = fmaf(g * wp, xh, c);
-        dwa[j][e] = fmaf(g, xh, dwa[j][e]);
+      for (int h = 0; h < H; ++h) {
+        const float2 wp = GEMMA ? add2(wv[h], dup2(1.0f)) : wv[h];
+        const float2 xh = mul2(xv[h], r2);
+        const float2 g = EPI == EPI_NONE ? gv[j][h] : mul2(gv[j][h], epi_grad2<EPI, FAST>(mul2(xh, wp)));
+        gv[j][h] = g;
+        c2 = fma2(mul2(g, wp), xh, c2);
+        dwa[j][h] = fma2(g, xh, dwa[j][h]);
       }
     }
-    c = group_sum<32>(c);
+    const float c = group_sum<32>(c2.x + c2.y);
     float4* red = pipe.red + rb * 32;
     if (lane == 0) red[cw].x = c;
     if (consumers_sync_or(nct, !ok)) {
@@ -226,23 +235,21 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT, true)) r
     if (++s == a.stages) s = 0, ph ^= 1u;
     float tot = 0.0f;
     for (int w = 0; w < ncw; ++w) tot += red[w].x;
-    const float cm = tot * inv_n;
+    const float2 ncm = dup2(-tot * inv_n);
     T* dxrow = dx + m * a.lddx;
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
       const int v = ct + j * nct;
       if (v < nvec) {
-        float wv[E], o[E];
-        V::unpack(*reinterpret_cast<const uint4*>(pipe.param(0) + (size_t)v * 16), wv);
+        float2 wv[H], xv[H], o[H];
+        unpack2<T>(*reinterpret_cast<const uint4*>(pipe.param(0) + (size_t)v * 16), wv);
+        unpack2<T>(xr[j], xv);
 #pragma unroll
-        for (int e = 0; e < E; ++e) o[e] = r * fmaf(gv[j][e], woff + wv[e], -(xv[j][e] * r) * cm);
-        if (v < nfull) {
-          st_stream(dxrow + (size_t)v * E, V::pack(o));
-        } else {
-#pragma unroll
-          for (int e = 0; e < E; ++e)
-            if (v * E + e < N) V::store1(dxrow + v * E + e, o[e]);
+        for (int h = 0; h < H; ++h) {
+          const float2 wp = GEMMA ? add2(wv[h], dup2(1.0f)) : wv[h];
+          o[h] = mul2(r2, fma2(gv[j][h], wp, mul2(mul2(xv[h], r2), ncm)));
         }
+        store_pairs<T>(dxrow, v, nfull, N, o);
       }
     }
   }
@@ -251,9 +258,10 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT, true)) r
 #pragma unroll
     for (int j = 0; j < VPT; ++j)
 #pragma unroll
-      for (int e = 0; e < E; ++e) {
-        const int col = (ct + j * nct) * E + e;
-        if (col < N) part[col] = dwa[j][e];
+      for (int h = 0; h < H; ++h) {
+        const int col = (ct + j * nct) * E + 2 * h;
+        if (col < N) part[col] = dwa[j][h].x;
+        if (col + 1 < N) part[col + 1] = dwa[j][h].y;
       }
   }
 }
@@ -475,7 +483,7 @@ void* pick_bwd_t(int vpt, bool cta, int epi, bool gemma) {
 
 gn_status rms_bwd_plan(int64_t rows, int64_t hidden, gn_dtype dt, NormPlan* p, void** kern, int epi,
                        bool gemma, int* grid) {
-  gn_status st = plan_norm(hidden, dt_size(dt), 2, 1, 4, p);
+  gn_status st = plan_norm(hidden, dt_size(dt), 2, 1, 4, 320, p);
   if (st != GN_OK) return st;
   *kern = dt == GN_BF16 ? pick_bwd_t<__nv_bfloat16>(p->vpt, p->cta, epi, gemma)
                         : pick_bwd_t<float>(p->vpt, p->cta, epi, gemma);
@@ -505,7 +513,7 @@ extern "C" gn_status gn_rmsnorm_fwd(const void* x, const void* w, void* y, float
   const size_t es = dt_size(dt);
   if (!aligned16(x) || !aligned16(y) || (ld_x * es) % 16 || (ld_y * es) % 16) return GN_ERR_ALIGN;
   NormPlan p;
-  gn_status st = plan_norm(hidden, es, 1, 1, 8, &p);
+  gn_status st = plan_norm(hidden, es, 1, 1, 8, 160, &p);
   if (st != GN_OK) return st;
   void* kern = dt == GN_BF16 ? pick_fwd_t<__nv_bfloat16>(p.vpt, p.cta, epi, gemma != 0)
                              : pick_fwd_t<float>(p.vpt, p.cta, epi, gemma != 0);

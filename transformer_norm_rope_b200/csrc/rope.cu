@@ -88,6 +88,153 @@ __device__ __forceinline__ void unit_origin(const RopeArgs& a, uint32_t u, int64
   bs = (int64_t)b * a.S + s;
 }
 
+struct VecCtx {
+  const uint8_t* sb;   // the unit's stage
+  const float* tcos;   // the token's table rows in the stage
+  const float* tsin;
+  int64_t row0;        // first head row of the unit
+  int lph, lph_shift;  // vectors per head (and log2 when a power of two, else -1)
+  float inv_d;
+};
+
+// A 16-byte vector as two planes over its consecutive pairs: plane 0 holds the even element
+// of each pair, plane 1 the odd one, two pairs per float2 (bf16: pairs 0-3 -> 2 float2 per
+// plane; fp32: pairs 0-1 -> 1 float2). Element e = 4k + 2*lane + plane sits in plane
+// `plane`, float2 k, component `lane`. In this layout the rotation, scaling and gradient
+// arithmetic of a pair runs on packed fp32x2 instructions.
+template <typename T>
+struct Planes {
+  static constexpr int E = Vec<T>::N;
+  static constexpr int K = E / 4;
+  __device__ __forceinline__ static void load(const uint4& u, float2 (&p0)[K], float2 (&p1)[K]) {
+    if constexpr (sizeof(T) == 2) {
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};  // word i = pair i (even element in the low half)
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        p0[k] = make_float2(__uint_as_float(w[2 * k] << 16), __uint_as_float(w[2 * k + 1] << 16));
+        p1[k] = make_float2(__uint_as_float(w[2 * k] & 0xffff0000u), __uint_as_float(w[2 * k + 1] & 0xffff0000u));
+      }
+    } else {
+      p0[0] = make_float2(__uint_as_float(u.x), __uint_as_float(u.z));
+      p1[0] = make_float2(__uint_as_float(u.y), __uint_as_float(u.w));
+    }
+  }
+  __device__ __forceinline__ static uint4 store(const float2 (&p0)[K], const float2 (&p1)[K]) {
+    if constexpr (sizeof(T) == 2) {
+      uint32_t w[4];
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        w[2 * k] = Vec<T>::join(p0[k].x, p1[k].x);
+        w[2 * k + 1] = Vec<T>::join(p0[k].y, p1[k].y);
+      }
+      return make_uint4(w[0], w[1], w[2], w[3]);
+    } else {
+      return make_uint4(__float_as_uint(p0[0].x), __float_as_uint(p1[0].x), __float_as_uint(p0[0].y),
+                        __float_as_uint(p1[0].y));
+    }
+  }
+  // element order <-> planes (per-column weights and weight gradients)
+  __device__ __forceinline__ static void split(const float (&e)[E], float2 (&p0)[K], float2 (&p1)[K]) {
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      p0[k] = make_float2(e[4 * k], e[4 * k + 2]);
+      p1[k] = make_float2(e[4 * k + 1], e[4 * k + 3]);
+    }
+  }
+  __device__ __forceinline__ static void merge(const float2 (&p0)[K], const float2 (&p1)[K], float (&e)[E]) {
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      e[4 * k] = p0[k].x, e[4 * k + 2] = p0[k].y;
+      e[4 * k + 1] = p1[k].x, e[4 * k + 3] = p1[k].y;
+    }
+  }
+};
+
+// One 16-byte vector w of tensor TT's slab of the current unit (valid when w < nv_t).
+// wt0/wt1: this lane's weights w' in planes; dw0/dw1: its weight-gradient accumulators.
+template <typename T, int MODE, int TT>
+__device__ __forceinline__ void rope_vec(const RopeArgs& a, const VecCtx& c, int w, int nv_t,
+                                         const float2 (&wt0)[Planes<T>::K], const float2 (&wt1)[Planes<T>::K],
+                                         float2 (&dw0)[Planes<T>::K], float2 (&dw1)[Planes<T>::K]) {
+  using PL = Planes<T>;
+  constexpr int K = PL::K;
+  constexpr int P = Vec<T>::N / 2;
+  const bool valid = w < nv_t;
+  if (!valid) w = 0;
+  int hh, l;
+  if (c.lph_shift >= 0) {
+    hh = w >> c.lph_shift;
+    l = w & (c.lph - 1);
+  } else {
+    hh = w / c.lph;
+    l = w - hh * c.lph;
+  }
+  float2 x0[K], x1[K], cs[K], sn[K], o0[K], o1[K];
+  PL::load(*reinterpret_cast<const uint4*>(c.sb + TT * a.tslot + (size_t)w * 16), x0, x1);
+  if constexpr (P == 4) {
+    const float4 c4 = *reinterpret_cast<const float4*>(c.tcos + l * P);
+    const float4 s4 = *reinterpret_cast<const float4*>(c.tsin + l * P);
+    cs[0] = make_float2(c4.x, c4.y), cs[1] = make_float2(c4.z, c4.w);
+    sn[0] = make_float2(s4.x, s4.y), sn[1] = make_float2(s4.z, s4.w);
+  } else {
+    cs[0] = *reinterpret_cast<const float2*>(c.tcos + l * P);
+    sn[0] = *reinterpret_cast<const float2*>(c.tsin + l * P);
+  }
+  if constexpr (MODE == ROPE) {
+    // (x0, x1) -> (x0 c - x1 s', x0 s' + x1 c), s' = sign * s
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      const float2 s = mul2(dup2(a.sign), sn[k]), ns = mul2(dup2(-a.sign), sn[k]);
+      o0[k] = fma2(x1[k], ns, mul2(x0[k], cs[k]));
+      o1[k] = fma2(x0[k], s, mul2(x1[k], cs[k]));
+    }
+  } else if constexpr (MODE == QK_FWD) {
+    float2 ss2 = fma2(x0[0], x0[0], mul2(x1[0], x1[0]));
+#pragma unroll
+    for (int k = 1; k < K; ++k) ss2 = fma2(x1[k], x1[k], fma2(x0[k], x0[k], ss2));
+    const float ss = group_sum_rt(ss2.x + ss2.y, c.lph);
+    const float r = rsqrtf(fmaf(ss, c.inv_d, a.eps));
+    const float2 r2 = dup2(r);
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      const float2 n0 = mul2(x0[k], mul2(r2, wt0[k]));
+      const float2 n1 = mul2(x1[k], mul2(r2, wt1[k]));
+      const float2 ns = mul2(dup2(-1.0f), sn[k]);
+      o0[k] = fma2(n1, ns, mul2(n0, cs[k]));
+      o1[k] = fma2(n0, sn[k], mul2(n1, cs[k]));
+    }
+    if (valid && l == 0 && a.stat[TT]) a.stat[TT][c.row0 + hh] = r;
+  } else {  // QK_BWD
+    const float r = valid ? __ldg(a.stat[TT] + c.row0 + hh) : 0.0f;  // r = 0: invalid lanes add nothing
+    const float2 r2 = dup2(r);
+    float2 d0[K], d1[K];
+    PL::load(*reinterpret_cast<const uint4*>(c.sb + (a.ntens + TT) * a.tslot + (size_t)w * 16), d0, d1);
+    float2 gw0[K], gw1[K], h0[K], h1[K], cd2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      // inverse rotation of the output gradient: (d0 c + d1 s, d1 c - d0 s)
+      const float2 ns = mul2(dup2(-1.0f), sn[k]);
+      const float2 g0 = fma2(d1[k], sn[k], mul2(d0[k], cs[k]));
+      const float2 g1 = fma2(d0[k], ns, mul2(d1[k], cs[k]));
+      h0[k] = mul2(x0[k], r2);
+      h1[k] = mul2(x1[k], r2);
+      gw0[k] = mul2(g0, wt0[k]);
+      gw1[k] = mul2(g1, wt1[k]);
+      cd2 = fma2(gw1[k], h1[k], fma2(gw0[k], h0[k], cd2));
+      dw0[k] = fma2(g0, h0[k], dw0[k]);
+      dw1[k] = fma2(g1, h1[k], dw1[k]);
+    }
+    const float cd = group_sum_rt(cd2.x + cd2.y, c.lph) * c.inv_d;
+    const float2 ncd = dup2(-cd);
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      o0[k] = mul2(r2, fma2(h0[k], ncd, gw0[k]));
+      o1[k] = mul2(r2, fma2(h1[k], ncd, gw1[k]));
+    }
+  }
+  if (valid) st_stream(static_cast<T*>(a.out[TT]) + c.row0 * a.D + (int64_t)w * Vec<T>::N, PL::store(o0, o1));
+}
+
 template <typename T, int MODE, bool GEMMA>
 __global__ void __launch_bounds__(kRopeMaxThreads, 2) rope_kernel(const RopeArgs a) {
   using V = Vec<T>;
@@ -156,19 +303,24 @@ __global__ void __launch_bounds__(kRopeMaxThreads, 2) rope_kernel(const RopeArgs
   // -------------------------------------------------------------- consumers
   const int ct = threadIdx.x - 32, nct = ncw * 32;
   const int li = a.lph_shift >= 0 ? (ct & (lph - 1)) : 0;  // NORM: lane within the head (fixed)
-  float wq[E], wk[E], dwa[2][E];
+  constexpr int K = Planes<T>::K;
+  float2 wq0[K], wq1[K], wk0[K], wk1[K], dq0[K], dq1[K], dk0[K], dk1[K];
+  {
+    float wq[E], wk[E];
 #pragma unroll
-  for (int e = 0; e < E; ++e) {
-    wq[e] = wk[e] = 0.0f;
-    dwa[0][e] = dwa[1][e] = 0.0f;
-  }
-  if constexpr (NORM) {
+    for (int e = 0; e < E; ++e) wq[e] = wk[e] = 0.0f;
+    if constexpr (NORM) {
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const int d = li * E + e;
-      wq[e] = (GEMMA ? 1.0f : 0.0f) + V::load1(static_cast<const T*>(a.w[0]) + d);
-      if (a.ntens > 1) wk[e] = (GEMMA ? 1.0f : 0.0f) + V::load1(static_cast<const T*>(a.w[1]) + d);
+      for (int e = 0; e < E; ++e) {
+        const int d = li * E + e;
+        wq[e] = (GEMMA ? 1.0f : 0.0f) + V::load1(static_cast<const T*>(a.w[0]) + d);
+        if (a.ntens > 1) wk[e] = (GEMMA ? 1.0f : 0.0f) + V::load1(static_cast<const T*>(a.w[1]) + d);
+      }
     }
+    Planes<T>::split(wq, wq0, wq1);
+    Planes<T>::split(wk, wk0, wk1);
+#pragma unroll
+    for (int k = 0; k < K; ++k) dq0[k] = dq1[k] = dk0[k] = dk1[k] = make_float2(0.0f, 0.0f);
   }
   const float inv_d = 1.0f / (float)D;
   int failed = 0;
@@ -184,87 +336,14 @@ __global__ void __launch_bounds__(kRopeMaxThreads, 2) rope_kernel(const RopeArgs
     int c, s;
     unit_origin(a, u, bs, c, s);
     const int64_t row0 = bs * a.H + (int64_t)c * HC;  // first head row of the unit
-    const int64_t eoff = row0 * D;
     const uint8_t* sb = data + (size_t)st * sstride;
     const float* tcos = reinterpret_cast<const float*>(sb + nslots * a.tslot);
-    const float* tsin = tcos + D / 2;
-    // the trip count is the same for every lane of a warp, so the head shuffles see full warps
-    for (int vb = 0; vb < NV; vb += nct) {
-      const int v = vb + ct;
-      const bool valid = v < NV;
-      const int vv = valid ? v : 0;
-      const int tt = vv >= nv_t ? 1 : 0;
-      const int w = vv - tt * nv_t;  // vector index within the tensor slab
-      int hh, l;
-      if (a.lph_shift >= 0) {
-        hh = w >> a.lph_shift;
-        l = w & (lph - 1);
-      } else {
-        hh = w / lph;
-        l = w - hh * lph;
-      }
-      float xv[E], o[E], cs[P], sn[P];
-      V::unpack(*reinterpret_cast<const uint4*>(sb + tt * a.tslot + (size_t)w * 16), xv);
-      if constexpr (P == 4) {
-        const float4 c4 = *reinterpret_cast<const float4*>(tcos + l * P);
-        const float4 s4 = *reinterpret_cast<const float4*>(tsin + l * P);
-        cs[0] = c4.x, cs[1] = c4.y, cs[2] = c4.z, cs[3] = c4.w;
-        sn[0] = s4.x, sn[1] = s4.y, sn[2] = s4.z, sn[3] = s4.w;
-      } else {
-        const float2 c2 = *reinterpret_cast<const float2*>(tcos + l * P);
-        const float2 s2 = *reinterpret_cast<const float2*>(tsin + l * P);
-        cs[0] = c2.x, cs[1] = c2.y;
-        sn[0] = s2.x, sn[1] = s2.y;
-      }
-      if constexpr (MODE == ROPE) {
-#pragma unroll
-        for (int p = 0; p < P; ++p) {
-          const float x0 = xv[2 * p], x1 = xv[2 * p + 1];
-          const float si = a.sign * sn[p];
-          o[2 * p] = fmaf(x0, cs[p], -x1 * si);
-          o[2 * p + 1] = fmaf(x0, si, x1 * cs[p]);
-        }
-      } else if constexpr (MODE == QK_FWD) {
-        float ss = 0.0f;
-#pragma unroll
-        for (int e = 0; e < E; ++e) ss = fmaf(xv[e], xv[e], ss);
-        ss = group_sum_rt(ss, lph);
-        const float r = rsqrtf(fmaf(ss, inv_d, a.eps));
-        float n[E];
-#pragma unroll
-        for (int e = 0; e < E; ++e) n[e] = xv[e] * r * (tt ? wk[e] : wq[e]);
-#pragma unroll
-        for (int p = 0; p < P; ++p) {
-          o[2 * p] = fmaf(n[2 * p], cs[p], -n[2 * p + 1] * sn[p]);
-          o[2 * p + 1] = fmaf(n[2 * p], sn[p], n[2 * p + 1] * cs[p]);
-        }
-        if (valid && l == 0 && a.stat[tt]) a.stat[tt][row0 + hh] = r;
-      } else {  // QK_BWD
-        const float r = valid ? __ldg(a.stat[tt] + row0 + hh) : 0.0f;
-        float gv[E], g[E];
-        V::unpack(*reinterpret_cast<const uint4*>(sb + (a.ntens + tt) * a.tslot + (size_t)w * 16), gv);
-#pragma unroll
-        for (int p = 0; p < P; ++p) {  // inverse rotation of the output gradient
-          const float d0 = gv[2 * p], d1 = gv[2 * p + 1];
-          g[2 * p] = fmaf(d0, cs[p], d1 * sn[p]);
-          g[2 * p + 1] = fmaf(-d0, sn[p], d1 * cs[p]);
-        }
-        float cdot = 0.0f;
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-          const float xh = xv[e] * r;
-          cdot = fmaf(g[e] * (tt ? wk[e] : wq[e]), xh, cdot);
-          if (valid) {
-            if (tt) dwa[1][e] = fmaf(g[e], xh, dwa[1][e]);
-            else dwa[0][e] = fmaf(g[e], xh, dwa[0][e]);
-          }
-        }
-        cdot = group_sum_rt(cdot, lph) * inv_d;
-#pragma unroll
-        for (int e = 0; e < E; ++e) o[e] = r * fmaf(g[e], tt ? wk[e] : wq[e], -(xv[e] * r) * cdot);
-      }
-      if (valid) st_stream(static_cast<T*>(a.out[tt]) + eoff + (int64_t)w * E, V::pack(o));
-    }
+    const VecCtx ctx{sb, tcos, tcos + D / 2, row0, lph, a.lph_shift, inv_d};
+    // Each pass covers one tensor (the tensor is a compile-time argument of the body); the
+    // trip count is the same for every lane of a warp, so the head shuffles see full warps.
+    for (int vb = 0; vb < nv_t; vb += nct) rope_vec<T, MODE, 0>(a, ctx, vb + ct, nv_t, wq0, wq1, dq0, dq1);
+    if (a.ntens > 1)
+      for (int vb = 0; vb < nv_t; vb += nct) rope_vec<T, MODE, 1>(a, ctx, vb + ct, nv_t, wk0, wk1, dk0, dk1);
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[st]);
     if (++st == a.stages) st = 0, ph ^= 1u;
@@ -275,10 +354,13 @@ __global__ void __launch_bounds__(kRopeMaxThreads, 2) rope_kernel(const RopeArgs
     if (consumers_any(nct, failed) || !a.ws) return;
     consumers_sync(nct);
     float* red = reinterpret_cast<float*>(data);  // [nct][2][E]
+    float dwq[E], dwk[E];
+    Planes<T>::merge(dq0, dq1, dwq);
+    Planes<T>::merge(dk0, dk1, dwk);
 #pragma unroll
     for (int e = 0; e < E; ++e) {
-      red[(ct * 2 + 0) * E + e] = dwa[0][e];
-      red[(ct * 2 + 1) * E + e] = dwa[1][e];
+      red[(ct * 2 + 0) * E + e] = dwq[e];
+      red[(ct * 2 + 1) * E + e] = dwk[e];
     }
     consumers_sync(nct);
     float* part = a.ws + (int64_t)blockIdx.x * 2 * D;
@@ -313,16 +395,15 @@ gn_status plan_rope(int64_t B, int64_t S, int64_t H, int64_t D, int ntens, int m
   }
   p->HC = HC;
   p->NC = (int)(H / HC);
-  const int64_t nv = (int64_t)ntens * HC * lph;
-  // consumer warps: 8 by default; prefer a count whose 32*C divides the unit's vectors
+  // consumer warps: the most (10 down to 4) whose 32*C threads divide one tensor slab's
+  // vectors, so that no pass over a slab leaves lanes idle; 8 when none does
+  const int64_t nv_t = (int64_t)HC * lph;
   int cw = 8;
-  if (nv % (32 * cw)) {
-    for (int c = kMaxConsumerWarps; c >= 4; --c)
-      if (nv % (32 * c) == 0) {
-        cw = c;
-        break;
-      }
-  }
+  for (int c = kMaxConsumerWarps; c >= 4; --c)
+    if (nv_t % (32 * c) == 0) {
+      cw = c;
+      break;
+    }
   if (g_tune.group_rows) cw = g_tune.group_rows > kMaxConsumerWarps ? kMaxConsumerWarps : g_tune.group_rows;
   p->cwarps = cw;
   p->threads = 32 * (1 + cw);
@@ -330,7 +411,11 @@ gn_status plan_rope(int64_t B, int64_t S, int64_t H, int64_t D, int ntens, int m
   p->tslot = round128((uint32_t)(HC * D * (int64_t)es));
   p->tabslot = round128((uint32_t)(D * 4));
   const size_t sstride = (size_t)nslots * p->tslot + p->tabslot;
-  int stages = g_tune.stages ? g_tune.stages : (int)(96 * 1024 / sstride);
+  // stage depth per CTA (measured on B200): the plain rotation computes so little that one
+  // CTA with a deep pipeline streams best; the qk-norm passes keep ~64-96 KiB per CTA so that
+  // 2-3 CTAs share an SM
+  const size_t depth = mode == ROPE ? 128 * 1024 : mode == QK_FWD ? 64 * 1024 : 96 * 1024;
+  int stages = g_tune.stages ? g_tune.stages : (int)(depth / sstride);
   stages = stages < 2 ? 2 : stages > kRopeMaxStages ? kRopeMaxStages : stages;
   const size_t limit = smem_optin();
   while (stages > 1 && 128 + stages * sstride > limit) --stages;
