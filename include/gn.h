@@ -206,6 +206,12 @@ uint64_t gn_launch_count(void);
  * error. */
 gn_status gn_device_error(unsigned* word, int clear);
 
+/* Self-test of the bounded waits (no counterpart on the source pages): enqueues a one-thread
+ * kernel that waits on an mbarrier phase nothing completes, gives up after limit_us
+ * microseconds (1 .. 1000000), sets GN_DEVERR_WAIT_TIMEOUT in the device error word and
+ * returns, leaving the context usable. GN_ERR_SHAPE for a limit out of range. */
+gn_status gn_selftest_wait_timeout(uint32_t limit_us, void* stream);
+
 /* Tuning knobs of the launch planner, for benchmarking sweeps. key is one of "stages",
  * "ctas_per_sm", "vpt", "unit_bytes", "group_rows"; value 0 restores the default. Returns
  * GN_ERR_SHAPE for an unknown key or a negative value. Not thread-safe with concurrent

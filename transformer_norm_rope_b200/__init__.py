@@ -52,6 +52,7 @@ SIGNATURES = {
                                          _i64, _i64, _i64, _i64, _int, _int, _vp]),
     "gn_launch_count": (C.c_uint64, []),
     "gn_device_error": (_st, [C.POINTER(C.c_uint), _int]),
+    "gn_selftest_wait_timeout": (_st, [C.c_uint32, _vp]),
     "gn_tune": (_st, [C.c_char_p, _int]),
 }
 

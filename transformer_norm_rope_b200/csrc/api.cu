@@ -5,6 +5,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "gn_common.cuh"
 #include "gn_host.h"
 
 namespace gn {
@@ -113,6 +114,15 @@ __global__ void __launch_bounds__(256) colsum_kernel(const float* __restrict__ w
   }
 }
 
+// Self-test of the bounded wait: one thread waits for a phase of an mbarrier that nothing
+// will complete, gives up after limit_ns and records the timeout in the error word.
+__global__ void wait_timeout_selftest_kernel(unsigned* err, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  mbar_init(&bar, 1);
+  mbar_fence_init();
+  (void)mbar_wait(&bar, 0, err, limit_ns);  // phase 0 never completes: no arrival comes
+}
+
 gn_status launch_colsum(const float* ws, int64_t G, int64_t ncols, int64_t split, float* out0,
                         float* out1, cudaStream_t s) {
   if (!out0 && !out1) return GN_OK;
@@ -151,6 +161,15 @@ extern "C" gn_status gn_device_error(unsigned* word, int clear) {
   if (clear && cudaMemset(p, 0, sizeof(unsigned)) != cudaSuccess) return GN_ERR_CUDA;
   if (clear && cudaDeviceSynchronize() != cudaSuccess) return GN_ERR_CUDA;
   return GN_OK;
+}
+
+extern "C" gn_status gn_selftest_wait_timeout(uint32_t limit_us, void* stream) {
+  if (limit_us == 0 || limit_us > 1000000) return GN_ERR_SHAPE;
+  unsigned* err = device_err_word();
+  if (!err) return GN_ERR_CUDA;
+  wait_timeout_selftest_kernel<<<1, 1, 0, (cudaStream_t)stream>>>(err, (uint64_t)limit_us * 1000u);
+  count_launches(1);
+  return launch_status();
 }
 
 extern "C" gn_status gn_tune(const char* key, int value) {

@@ -131,14 +131,18 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
                : "memory");
 }
 
+// The thread may be suspended inside try_wait until the phase completes or about
+// kSuspendHintNs pass, so a waiting warp does not spend issue slots polling.
+constexpr uint32_t kSuspendHintNs = 100000;
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_addr(bar)), "r"(parity)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(kSuspendHintNs)
       : "memory");
   return ok != 0;
 }
@@ -149,13 +153,14 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// Wait for phase `parity` of `bar` to complete, for at most kWaitLimitNs. On timeout the
-// error word gets GN_DEVERR_WAIT_TIMEOUT and the function returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* err) {
+// Wait for phase `parity` of `bar` to complete, for at most limit_ns. On timeout the error
+// word gets GN_DEVERR_WAIT_TIMEOUT and the function returns false.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* err,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       if (err) atomicOr(err, kDevErrWaitTimeout);
       return false;
     }
@@ -182,10 +187,17 @@ __device__ __forceinline__ float group_sum(float v) {
   return v;
 }
 
-// runtime-width variant (width a power of two <= 32); every lane gets the same total
+// runtime-width variant (width a power of two <= 32); every lane gets the same total. The
+// width is uniform across the warp, so the dispatch to the unrolled forms costs one branch.
 __device__ __forceinline__ float group_sum_rt(float v, int width) {
-  for (int o = width / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o, width);
-  return v;
+  switch (width) {
+    case 32: return group_sum<32>(v);
+    case 16: return group_sum<16>(v);
+    case 8: return group_sum<8>(v);
+    case 4: return group_sum<4>(v);
+    case 2: return group_sum<2>(v);
+    default: return v;
+  }
 }
 
 // ---------------------------------------------------------------- epilogues
@@ -221,8 +233,10 @@ __device__ __forceinline__ float sigmoid_f(float x) {
 template <int EPI, bool FAST>
 __device__ __forceinline__ float epi_fwd(float z) {
   if constexpr (EPI == EPI_GELU_TANH) {
-    const float t = tanh_f<FAST>(kGeluK * fmaf(kGeluC * z, z * z, z));
-    return 0.5f * z * (1.0f + t);
+    const float z2 = z * z;
+    const float t = tanh_f<FAST>(z * fmaf(kGeluK * kGeluC, z2, kGeluK));  // k (z + c z^3)
+    const float h = 0.5f * z;
+    return fmaf(h, t, h);
   } else if constexpr (EPI == EPI_SILU) {
     return z * sigmoid_f<FAST>(z);
   } else {
@@ -235,8 +249,10 @@ template <int EPI, bool FAST>
 __device__ __forceinline__ float epi_grad(float z) {
   if constexpr (EPI == EPI_GELU_TANH) {
     const float z2 = z * z;
-    const float t = tanh_f<FAST>(kGeluK * fmaf(kGeluC * z, z2, z));
-    return 0.5f * (1.0f + t) + 0.5f * z * (1.0f - t * t) * kGeluK * fmaf(3.0f * kGeluC, z2, 1.0f);
+    const float t = tanh_f<FAST>(z * fmaf(kGeluK * kGeluC, z2, kGeluK));
+    // 0.5 (1 + t) + 0.5 z (1 - t^2) k (1 + 3 c z^2)
+    const float k3 = fmaf(3.0f * 0.5f * kGeluK * kGeluC, z2, 0.5f * kGeluK);  // 0.5 k (1 + 3 c z^2)
+    return fmaf(z * fmaf(-t, t, 1.0f), k3, fmaf(0.5f, t, 0.5f));
   } else if constexpr (EPI == EPI_SILU) {
     const float s = sigmoid_f<FAST>(z);
     return s * fmaf(z, 1.0f - s, 1.0f);
@@ -245,38 +261,23 @@ __device__ __forceinline__ float epi_grad(float z) {
   }
 }
 
-// The same epilogues on a pair of lanes with packed fp32x2 arithmetic (tanh / exp per lane).
+// The same epilogues on a pair of lanes. They run as two scalar evaluations: the constants of
+// the tanh-GeLU fold into scalar FMA immediates, which packed fp32x2 instructions cannot take.
 template <int EPI, bool FAST>
 __device__ __forceinline__ float2 epi_fwd2(float2 z) {
-  if constexpr (EPI == EPI_GELU_TANH) {
-    const float2 z2 = mul2(z, z);
-    const float2 arg = mul2(fma2(z2, dup2(kGeluK * kGeluC), dup2(kGeluK)), z);  // k (z + c z^3)
-    const float2 t = make_float2(tanh_f<FAST>(arg.x), tanh_f<FAST>(arg.y));
-    const float2 h = mul2(z, dup2(0.5f));
-    return fma2(h, t, h);
-  } else if constexpr (EPI == EPI_SILU) {
-    return mul2(z, make_float2(sigmoid_f<FAST>(z.x), sigmoid_f<FAST>(z.y)));
-  } else {
+  if constexpr (EPI == EPI_NONE) {
     return z;
+  } else {
+    return make_float2(epi_fwd<EPI, FAST>(z.x), epi_fwd<EPI, FAST>(z.y));
   }
 }
 
 template <int EPI, bool FAST>
 __device__ __forceinline__ float2 epi_grad2(float2 z) {
-  if constexpr (EPI == EPI_GELU_TANH) {
-    // 0.5 (1 + t) + 0.5 z (1 - t^2) k (1 + 3 c z^2)
-    const float2 z2 = mul2(z, z);
-    const float2 arg = mul2(fma2(z2, dup2(kGeluK * kGeluC), dup2(kGeluK)), z);
-    const float2 t = make_float2(tanh_f<FAST>(arg.x), tanh_f<FAST>(arg.y));
-    const float2 dt = fma2(mul2(t, dup2(-1.0f)), t, dup2(1.0f));
-    const float2 k3 = fma2(z2, dup2(3.0f * kGeluK * kGeluC), dup2(kGeluK));
-    const float2 a = fma2(t, dup2(0.5f), dup2(0.5f));
-    return fma2(mul2(mul2(z, dt), k3), dup2(0.5f), a);
-  } else if constexpr (EPI == EPI_SILU) {
-    const float2 s = make_float2(sigmoid_f<FAST>(z.x), sigmoid_f<FAST>(z.y));
-    return mul2(s, fma2(z, add2(dup2(1.0f), mul2(s, dup2(-1.0f))), dup2(1.0f)));
-  } else {
+  if constexpr (EPI == EPI_NONE) {
     return dup2(1.0f);
+  } else {
+    return make_float2(epi_grad<EPI, FAST>(z.x), epi_grad<EPI, FAST>(z.y));
   }
 }
 

@@ -122,15 +122,18 @@ __device__ __forceinline__ void load_affine(const LnFwdArgs& a, int base, int st
 // v = ct + j * nct (j < VPT) of every row. Weight and bias live in shared memory. The
 // arithmetic runs on element pairs with packed fp32x2 instructions.
 
+// per-column parameters (weight, bias) copied once into shared memory, padded with zeros
 template <typename T>
-__device__ __forceinline__ void stage_param(uint8_t* dst, const T* src, int N, int nvec, float dflt, int ct,
-                                            int nct) {
+__device__ __forceinline__ void stage_param(uint8_t* dst, const T* src, int N, int nvec, float dflt, int ct, int nct) {
   T* d = reinterpret_cast<T*>(dst);
-  const int n = nvec * Vec<T>::N;  // padded to whole vectors; the padding holds 0
-  for (int i = ct; i < n; i += nct) {
-    float v = i < N ? ld_param(src, i, dflt) : 0.0f;
-    Vec<T>::store1(d + i, v);
-  }
+  const int n = nvec * Vec<T>::N;
+  for (int i = ct; i < n; i += nct) Vec<T>::store1(d + i, i < N ? ld_param(src, i, dflt) : 0.0f);
+}
+
+// the parameters of vector v as element pairs
+template <typename T>
+__device__ __forceinline__ void param_pairs(const uint8_t* p, int v, float2 (&f)[Vec<T>::N / 2]) {
+  unpack2<T>(*reinterpret_cast<const uint4*>(p + (size_t)v * 16), f);
 }
 
 template <typename T>
@@ -171,7 +174,7 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT)) ln_fwd_
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int N = a.N, nfull = N / E, nvec = (N + E - 1) / E;
-  const RowPipe pipe(smem, a.stages, 1, 2, (int64_t)N * sizeof(T));
+  const RowPipe pipe(smem, a.stages, 1, 2, N, sizeof(T));
   const T* x = static_cast<const T*>(a.x);
   T* y = static_cast<T*>(a.y);
   const int ncw = (int)(blockDim.x >> 5) - 1;
@@ -251,8 +254,8 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT)) ln_fwd_
       const int v = ct + j * nct;
       if (v < nvec) {
         float2 wv[H], bv[H], o[H];
-        unpack2<T>(*reinterpret_cast<const uint4*>(pipe.param(0) + (size_t)v * 16), wv);
-        unpack2<T>(*reinterpret_cast<const uint4*>(pipe.param(1) + (size_t)v * 16), bv);
+        param_pairs<T>(pipe.param(0), v, wv);
+        param_pairs<T>(pipe.param(1), v, bv);
 #pragma unroll
         for (int h = 0; h < H; ++h) o[h] = epi_fwd2<EPI, FAST>(fma2(fma2(xv[j][h], rs2, nmr2), wv[h], bv[h]));
         store_pairs<T>(yrow, v, nfull, N, o);
@@ -272,7 +275,7 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT, true)) l
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int N = a.N, nfull = N / E, nvec = (N + E - 1) / E;
-  const RowPipe pipe(smem, a.stages, 2, 2, (int64_t)N * sizeof(T));
+  const RowPipe pipe(smem, a.stages, 2, 2, N, sizeof(T));
   const T* x = static_cast<const T*>(a.x);
   const T* dy = static_cast<const T*>(a.dy);
   T* dx = static_cast<T*>(a.dx);
@@ -321,17 +324,17 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT, true)) l
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
       const int v = ct + j * nct;
-      const size_t vo = (size_t)(v < nvec ? v : 0) * 16;
+      const int vv = v < nvec ? v : 0;
       float2 wv[H], bv[H], xv[H];
-      unpack2<T>(*reinterpret_cast<const uint4*>(pipe.param(0) + vo), wv);
-      unpack2<T>(*reinterpret_cast<const uint4*>(pipe.param(1) + vo), bv);
+      param_pairs<T>(pipe.param(0), vv, wv);
+      param_pairs<T>(pipe.param(1), vv, bv);
       unpack2<T>(xr[j], xv);
 #pragma unroll
       for (int h = 0; h < H; ++h) {
         const float2 xh = fma2(xv[h], rs2, nmr2);
         const float2 g = EPI == EPI_NONE ? gv[j][h] : mul2(gv[j][h], epi_grad2<EPI, FAST>(fma2(xh, wv[h], bv[h])));
         const float2 gw = mul2(g, wv[h]);
-        gv[j][h] = g;
+        gv[j][h] = gw;  // phase 2 needs only g w
         s12 = add2(s12, gw);
         s22 = fma2(gw, xh, s22);
         dwa[j][h] = fma2(g, xh, dwa[j][h]);
@@ -359,14 +362,10 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT, true)) l
     for (int j = 0; j < VPT; ++j) {
       const int v = ct + j * nct;
       if (v < nvec) {
-        float2 wv[H], xv[H], o[H];
-        unpack2<T>(*reinterpret_cast<const uint4*>(pipe.param(0) + (size_t)v * 16), wv);
+        float2 xv[H], o[H];
         unpack2<T>(xr[j], xv);
 #pragma unroll
-        for (int h = 0; h < H; ++h) {
-          const float2 xh = fma2(xv[h], rs2, nmr2);
-          o[h] = mul2(rs2, fma2(gv[j][h], wv[h], fma2(xh, nc2, nc1)));
-        }
+        for (int h = 0; h < H; ++h) o[h] = mul2(rs2, add2(gv[j][h], fma2(fma2(xv[h], rs2, nmr2), nc2, nc1)));
         store_pairs<T>(dxrow, v, nfull, N, o);
       }
     }
@@ -600,7 +599,9 @@ void* pick_ln_t(int vpt, bool cta, int epi) {
 
 gn_status ln_plan(int64_t rows, int64_t hidden, gn_dtype dt, bool bwd, int epi, NormPlan* p, void** kern,
                   int* grid) {
-  gn_status st = plan_norm(hidden, dt_size(dt), bwd ? 2 : 1, 2, bwd ? 4 : 8, bwd ? 320 : 160, p);
+  // 4 vectors per thread in both directions (measured: the backward's per-row overhead
+  // outweighs its extra registers)
+  gn_status st = plan_norm(hidden, dt_size(dt), bwd ? 2 : 1, 2, bwd ? 4 : 8, 160, p);
   if (st != GN_OK) return st;
   if (dt == GN_BF16)
     *kern = bwd ? pick_ln_t<__nv_bfloat16, true>(p->vpt, p->cta, epi) : pick_ln_t<__nv_bfloat16, false>(p->vpt, p->cta, epi);
@@ -650,10 +651,16 @@ extern "C" gn_status gn_layernorm_fwd(const void* x, const void* w, const void* 
 
 extern "C" size_t gn_layernorm_bwd_workspace(int64_t rows, int64_t hidden, gn_dtype dt) {
   if (rows <= 0 || hidden <= 0 || !dt_ok(dt)) return 0;
-  NormPlan p;
-  void* kern = nullptr;
+  // the epilogue variants may differ in occupancy, hence in persistent grid size: size for
+  // the largest
   int grid = 0;
-  if (ln_plan(rows, hidden, dt, true, GN_EPI_NONE, &p, &kern, &grid) != GN_OK) return 0;
+  for (int epi = GN_EPI_NONE; epi <= GN_EPI_SILU; ++epi) {
+    NormPlan p;
+    void* kern = nullptr;
+    int g = 0;
+    if (ln_plan(rows, hidden, dt, true, epi, &p, &kern, &g) != GN_OK) return 0;
+    if (g > grid) grid = g;
+  }
   return (size_t)grid * 2 * (size_t)hidden * sizeof(float);
 }
 

@@ -72,15 +72,17 @@ inline gn_status plan_norm(int64_t N, size_t es, int ntens, int nparams, int max
   const size_t slot = pipe_slot_bytes(row_bytes);
   int stages = g_tune.stages;
   if (stages == 0) {
-    stages = (int)((ntens > 1 ? 65536 : 49152) / (slot * ntens));
+    // forward: shallow pipelines leave room for more CTAs per SM, which hides the per-row
+    // reduction latency better (measured on B200); backward: ~64 KiB in flight per CTA
+    stages = (int)((ntens > 1 ? 65536 : 24576) / (slot * ntens));
     stages = stages < 2 ? 2 : stages > kMaxStages ? kMaxStages : stages;
   }
   if (stages > kMaxStages) stages = kMaxStages;
   const size_t limit = smem_optin();
-  while (stages > 1 && pipe_smem_bytes(stages, ntens, nparams, row_bytes) > limit) --stages;
-  if (pipe_smem_bytes(stages, ntens, nparams, row_bytes) > limit) return GN_ERR_UNSUPPORTED;
+  while (stages > 1 && pipe_smem_bytes(stages, ntens, nparams, N, (int64_t)es) > limit) --stages;
+  if (pipe_smem_bytes(stages, ntens, nparams, N, (int64_t)es) > limit) return GN_ERR_UNSUPPORTED;
   p->stages = stages;
-  p->smem = pipe_smem_bytes(stages, ntens, nparams, row_bytes);
+  p->smem = pipe_smem_bytes(stages, ntens, nparams, N, (int64_t)es);
   return GN_OK;
 }
 

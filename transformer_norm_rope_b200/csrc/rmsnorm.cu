@@ -47,19 +47,20 @@ struct RmsBwdArgs {
 // gradient - never change. The weight lives in shared memory (one copy per CTA). The
 // arithmetic runs on element pairs with packed fp32x2 instructions.
 
+// per-column parameters (weight, bias) copied once into shared memory, padded with zeros
 template <typename T>
-__device__ __forceinline__ void stage_param(uint8_t* dst, const T* src, int N, int nvec, float dflt, int ct,
-                                            int nct) {
+__device__ __forceinline__ void stage_param(uint8_t* dst, const T* src, int N, int nvec, float dflt, int ct, int nct) {
   T* d = reinterpret_cast<T*>(dst);
-  const int n = nvec * Vec<T>::N;  // padded to whole vectors; the padding holds 0
-  for (int i = ct; i < n; i += nct) {
-    float v = i < N ? ld_param(src, i, dflt) : 0.0f;
-    Vec<T>::store1(d + i, v);
-  }
+  const int n = nvec * Vec<T>::N;
+  for (int i = ct; i < n; i += nct) Vec<T>::store1(d + i, i < N ? ld_param(src, i, dflt) : 0.0f);
 }
 
-// vector v of a row as element pairs: whole vectors from the stage, the ragged tail (and
-// vectors past the row) element by element from global memory, zero beyond the row
+// the parameters of vector v as element pairs
+template <typename T>
+__device__ __forceinline__ void param_pairs(const uint8_t* p, int v, float2 (&f)[Vec<T>::N / 2]) {
+  unpack2<T>(*reinterpret_cast<const uint4*>(p + (size_t)v * 16), f);
+}
+
 template <typename T>
 __device__ __forceinline__ void load_pairs(const uint8_t* st, const T* row, int v, int nfull, int N, bool ok,
                                            float2 (&f)[Vec<T>::N / 2]) {
@@ -98,7 +99,7 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT)) rms_fwd
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int N = a.N, nfull = N / Vec<T>::N, nvec = (N + Vec<T>::N - 1) / Vec<T>::N;
-  const RowPipe pipe(smem, a.stages, 1, 1, (int64_t)N * sizeof(T));
+  const RowPipe pipe(smem, a.stages, 1, 1, N, sizeof(T));
   const T* x = static_cast<const T*>(a.x);
   T* y = static_cast<T*>(a.y);
   const int ncw = (int)(blockDim.x >> 5) - 1;
@@ -143,7 +144,7 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT)) rms_fwd
       const int v = ct + j * nct;
       if (v < nvec) {
         float2 wv[H], o[H];
-        unpack2<T>(*reinterpret_cast<const uint4*>(pipe.param(0) + (size_t)v * 16), wv);
+        param_pairs<T>(pipe.param(0), v, wv);
 #pragma unroll
         for (int h = 0; h < H; ++h) {
           const float2 wp = GEMMA ? add2(wv[h], dup2(1.0f)) : wv[h];
@@ -163,7 +164,7 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT, true)) r
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int N = a.N, nfull = N / E, nvec = (N + E - 1) / E;
-  const RowPipe pipe(smem, a.stages, 2, 1, (int64_t)N * sizeof(T));
+  const RowPipe pipe(smem, a.stages, 2, 1, N, sizeof(T));
   const T* x = static_cast<const T*>(a.x);
   const T* dy = static_cast<const T*>(a.dy);
   T* dx = static_cast<T*>(a.dx);
@@ -212,15 +213,16 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT, true)) r
     for (int j = 0; j < VPT; ++j) {
       const int v = ct + j * nct;
       float2 wv[H], xv[H];
-      unpack2<T>(*reinterpret_cast<const uint4*>(pipe.param(0) + (size_t)(v < nvec ? v : 0) * 16), wv);
+      param_pairs<T>(pipe.param(0), v < nvec ? v : 0, wv);
       unpack2<T>(xr[j], xv);
 #pragma unroll
       for (int h = 0; h < H; ++h) {
         const float2 wp = GEMMA ? add2(wv[h], dup2(1.0f)) : wv[h];
         const float2 xh = mul2(xv[h], r2);
         const float2 g = EPI == EPI_NONE ? gv[j][h] : mul2(gv[j][h], epi_grad2<EPI, FAST>(mul2(xh, wp)));
-        gv[j][h] = g;
-        c2 = fma2(mul2(g, wp), xh, c2);
+        const float2 gw = mul2(g, wp);
+        gv[j][h] = gw;  // phase 2 needs only g w'
+        c2 = fma2(gw, xh, c2);
         dwa[j][h] = fma2(g, xh, dwa[j][h]);
       }
     }
@@ -241,14 +243,10 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT, true)) r
     for (int j = 0; j < VPT; ++j) {
       const int v = ct + j * nct;
       if (v < nvec) {
-        float2 wv[H], xv[H], o[H];
-        unpack2<T>(*reinterpret_cast<const uint4*>(pipe.param(0) + (size_t)v * 16), wv);
+        float2 xv[H], o[H];
         unpack2<T>(xr[j], xv);
 #pragma unroll
-        for (int h = 0; h < H; ++h) {
-          const float2 wp = GEMMA ? add2(wv[h], dup2(1.0f)) : wv[h];
-          o[h] = mul2(r2, fma2(gv[j][h], wp, mul2(mul2(xv[h], r2), ncm)));
-        }
+        for (int h = 0; h < H; ++h) o[h] = mul2(r2, fma2(mul2(xv[h], r2), ncm, gv[j][h]));
         store_pairs<T>(dxrow, v, nfull, N, o);
       }
     }
@@ -538,10 +536,17 @@ extern "C" gn_status gn_rmsnorm_fwd(const void* x, const void* w, void* y, float
 
 extern "C" size_t gn_rmsnorm_bwd_workspace(int64_t rows, int64_t hidden, gn_dtype dt) {
   if (rows <= 0 || hidden <= 0 || !dt_ok(dt)) return 0;
-  NormPlan p;
-  void* kern = nullptr;
+  // the epilogue and Gemma variants may differ in occupancy, hence in persistent grid size:
+  // size for the largest
   int grid = 0;
-  if (rms_bwd_plan(rows, hidden, dt, &p, &kern, GN_EPI_NONE, false, &grid) != GN_OK) return 0;
+  for (int epi = GN_EPI_NONE; epi <= GN_EPI_SILU; ++epi)
+    for (int gemma = 0; gemma < 2; ++gemma) {
+      NormPlan p;
+      void* kern = nullptr;
+      int g = 0;
+      if (rms_bwd_plan(rows, hidden, dt, &p, &kern, epi, gemma != 0, &g) != GN_OK) return 0;
+      if (g > grid) grid = g;
+    }
   return (size_t)grid * (size_t)hidden * sizeof(float);
 }
 

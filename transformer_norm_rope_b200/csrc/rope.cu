@@ -547,11 +547,16 @@ extern "C" gn_status gn_qknorm_rope_fwd(const void* q, const void* k, const void
 
 extern "C" size_t gn_qknorm_rope_bwd_workspace(int64_t B, int64_t S, int64_t H, int64_t D, gn_dtype dt) {
   if (check_common(B, S, H, D, dt) != GN_OK || !norm_head_ok(D, dt) || B * S * H == 0) return 0;
-  RopePlan p;
-  void* kern = nullptr;
+  // sized for two tensors (a call with k == NULL uses no more) and for the larger grid of
+  // the plain and Gemma variants, whose occupancy may differ
   int grid = 0;
-  if (setup(B, S, H, D, 2, QK_BWD, dt, false, &p, &kern, &grid) != GN_OK) return 0;
-  // sized for two tensors; a call with k == NULL uses no more
+  for (int gemma = 0; gemma < 2; ++gemma) {
+    RopePlan p;
+    void* kern = nullptr;
+    int g = 0;
+    if (setup(B, S, H, D, 2, QK_BWD, dt, gemma != 0, &p, &kern, &g) != GN_OK) return 0;
+    if (g > grid) grid = g;
+  }
   return (size_t)grid * 2 * (size_t)D * sizeof(float);
 }
 

@@ -29,8 +29,11 @@ __host__ __device__ inline uint32_t pipe_slot_bytes(int64_t row_bytes) {
   return (uint32_t)((row_bytes + 127) / 128 * 128);
 }
 
-__host__ __device__ inline size_t pipe_smem_bytes(int stages, int ntens, int nparams, int64_t row_bytes) {
-  return kPipeHeader + (size_t)(nparams + stages * ntens) * pipe_slot_bytes(row_bytes);
+// parameter vectors are kept in the row type, padded to whole 16-byte vectors and 128 bytes
+__host__ __device__ inline uint32_t pipe_param_bytes(int64_t n, int64_t es) { return pipe_slot_bytes((n * es + 15) / 16 * 16); }
+
+__host__ __device__ inline size_t pipe_smem_bytes(int stages, int ntens, int nparams, int64_t n, int64_t es) {
+  return kPipeHeader + (size_t)nparams * pipe_param_bytes(n, es) + (size_t)stages * ntens * pipe_slot_bytes(n * es);
 }
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
@@ -57,28 +60,30 @@ struct RowPipe {
   uint64_t* full;
   uint64_t* empty;
   float4* red;      // [2][32]
-  uint8_t* params;  // nparams slots
+  uint8_t* params;  // nparams parameter vectors
   uint8_t* data;
   int stages;
   int ntens;
   uint32_t slot;    // bytes per (stage, tensor) slot
+  uint32_t pslot;   // bytes per parameter vector
   uint32_t bulk;    // bytes bulk-copied per tensor (whole 16-byte vectors of the row)
 
-  __device__ __forceinline__ RowPipe(uint8_t* smem, int stages_, int ntens_, int nparams, int64_t row_bytes)
+  __device__ __forceinline__ RowPipe(uint8_t* smem, int stages_, int ntens_, int nparams, int64_t n, int64_t es)
       : full(reinterpret_cast<uint64_t*>(smem)),
         empty(reinterpret_cast<uint64_t*>(smem) + kMaxStages),
         red(reinterpret_cast<float4*>(smem + 128)),
         params(smem + kPipeHeader),
-        data(smem + kPipeHeader + (size_t)nparams * pipe_slot_bytes(row_bytes)),
+        data(smem + kPipeHeader + (size_t)nparams * pipe_param_bytes(n, es)),
         stages(stages_),
         ntens(ntens_),
-        slot(pipe_slot_bytes(row_bytes)),
-        bulk((uint32_t)(row_bytes / 16 * 16)) {}
+        slot(pipe_slot_bytes(n * es)),
+        pslot(pipe_param_bytes(n, es)),
+        bulk((uint32_t)(n * es / 16 * 16)) {}
 
   __device__ __forceinline__ const uint8_t* at(int s, int t) const {
     return data + ((size_t)s * ntens + t) * slot;
   }
-  __device__ __forceinline__ uint8_t* param(int i) const { return params + (size_t)i * slot; }
+  __device__ __forceinline__ uint8_t* param(int i) const { return params + (size_t)i * pslot; }
 
   // thread 0, before the first __syncthreads of the kernel
   __device__ __forceinline__ void init(int consumer_warps) const {
