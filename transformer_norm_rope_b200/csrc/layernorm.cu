@@ -14,6 +14,7 @@
 // centred sum of squares (two barriers over the consumer warps); the short-row kernel forms
 // (count, mean, M2) per thread and combines the triples with Chan et al.'s pairwise update.
 #include "norm_plan.h"
+#include "norm_rows.cuh"
 
 namespace gn {
 namespace {
@@ -122,50 +123,6 @@ __device__ __forceinline__ void load_affine(const LnFwdArgs& a, int base, int st
 // v = ct + j * nct (j < VPT) of every row. Weight and bias live in shared memory. The
 // arithmetic runs on element pairs with packed fp32x2 instructions.
 
-// per-column parameters (weight, bias) copied once into shared memory, padded with zeros
-template <typename T>
-__device__ __forceinline__ void stage_param(uint8_t* dst, const T* src, int N, int nvec, float dflt, int ct, int nct) {
-  T* d = reinterpret_cast<T*>(dst);
-  const int n = nvec * Vec<T>::N;
-  for (int i = ct; i < n; i += nct) Vec<T>::store1(d + i, i < N ? ld_param(src, i, dflt) : 0.0f);
-}
-
-// the parameters of vector v as element pairs
-template <typename T>
-__device__ __forceinline__ void param_pairs(const uint8_t* p, int v, float2 (&f)[Vec<T>::N / 2]) {
-  unpack2<T>(*reinterpret_cast<const uint4*>(p + (size_t)v * 16), f);
-}
-
-template <typename T>
-__device__ __forceinline__ void load_pairs(const uint8_t* st, const T* row, int v, int nfull, int N, bool ok,
-                                           float2 (&f)[Vec<T>::N / 2]) {
-  constexpr int E = Vec<T>::N;
-  if (ok && v < nfull) {
-    unpack2<T>(*reinterpret_cast<const uint4*>(st + (size_t)v * 16), f);
-  } else {
-#pragma unroll
-    for (int h = 0; h < E / 2; ++h) {
-      const int col = v * E + 2 * h;
-      f[h].x = (ok && col < N) ? Vec<T>::load1(row + col) : 0.0f;
-      f[h].y = (ok && col + 1 < N) ? Vec<T>::load1(row + col + 1) : 0.0f;
-    }
-  }
-}
-
-template <typename T>
-__device__ __forceinline__ void store_pairs(T* row, int v, int nfull, int N, const float2 (&f)[Vec<T>::N / 2]) {
-  constexpr int E = Vec<T>::N;
-  if (v < nfull) {
-    st_stream(row + (size_t)v * E, pack2<T>(f));
-  } else {
-#pragma unroll
-    for (int h = 0; h < E / 2; ++h) {
-      const int col = v * E + 2 * h;
-      if (col < N) Vec<T>::store1(row + col, f[h].x);
-      if (col + 1 < N) Vec<T>::store1(row + col + 1, f[h].y);
-    }
-  }
-}
 
 template <typename T, int VPT, int EPI>
 __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT)) ln_fwd_cta(const LnFwdArgs a) {
@@ -304,8 +261,13 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT, true)) l
   int s = 0;
   uint32_t ph = 0, rb = 0;
   bool failed = false;
+  // the statistics of the next row are loaded one row ahead: their global-memory latency
+  // then overlaps the current row instead of stalling the start of the next
+  float mu_n = 0.0f, rs_n = 0.0f;
+  if (blockIdx.x < a.rows) mu_n = __ldg(a.mean + blockIdx.x), rs_n = __ldg(a.rstd + blockIdx.x);
   for (int64_t m = blockIdx.x; m < a.rows; m += step) {
-    const float mu = __ldg(a.mean + m), rs = __ldg(a.rstd + m);
+    const float mu = mu_n, rs = rs_n;
+    if (m + step < a.rows) mu_n = __ldg(a.mean + m + step), rs_n = __ldg(a.rstd + m + step);
     const float2 rs2 = dup2(rs), nmr2 = dup2(-mu * rs);
     const bool ok = __all_sync(0xffffffffu, mbar_wait(&pipe.full[s], ph, a.err));
     uint4 xr[VPT];  // x stays packed between the two phases (unpacked on use)
@@ -313,9 +275,7 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT, true)) l
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
       const int v = ct + j * nct;
-      float2 xt[H];
-      load_pairs<T>(pipe.at(s, 0), x + m * a.ldx, v, nfull, N, ok, xt);
-      xr[j] = pack2<T>(xt);  // exact: the values came from T
+      xr[j] = load_raw<T>(pipe.at(s, 0), x + m * a.ldx, v, nfull, N, ok);
       load_pairs<T>(pipe.at(s, 1), dy + m * a.lddy, v, nfull, N, ok, gv[j]);
     }
     __syncwarp();

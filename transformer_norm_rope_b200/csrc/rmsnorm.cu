@@ -10,6 +10,7 @@
 // weight gradient is accumulated per thread in fp32 registers over the rows a CTA owns,
 // written as one partial row per CTA, and summed in a fixed order by launch_colsum.
 #include "norm_plan.h"
+#include "norm_rows.cuh"
 
 namespace gn {
 namespace {
@@ -47,50 +48,6 @@ struct RmsBwdArgs {
 // gradient - never change. The weight lives in shared memory (one copy per CTA). The
 // arithmetic runs on element pairs with packed fp32x2 instructions.
 
-// per-column parameters (weight, bias) copied once into shared memory, padded with zeros
-template <typename T>
-__device__ __forceinline__ void stage_param(uint8_t* dst, const T* src, int N, int nvec, float dflt, int ct, int nct) {
-  T* d = reinterpret_cast<T*>(dst);
-  const int n = nvec * Vec<T>::N;
-  for (int i = ct; i < n; i += nct) Vec<T>::store1(d + i, i < N ? ld_param(src, i, dflt) : 0.0f);
-}
-
-// the parameters of vector v as element pairs
-template <typename T>
-__device__ __forceinline__ void param_pairs(const uint8_t* p, int v, float2 (&f)[Vec<T>::N / 2]) {
-  unpack2<T>(*reinterpret_cast<const uint4*>(p + (size_t)v * 16), f);
-}
-
-template <typename T>
-__device__ __forceinline__ void load_pairs(const uint8_t* st, const T* row, int v, int nfull, int N, bool ok,
-                                           float2 (&f)[Vec<T>::N / 2]) {
-  constexpr int E = Vec<T>::N;
-  if (ok && v < nfull) {
-    unpack2<T>(*reinterpret_cast<const uint4*>(st + (size_t)v * 16), f);
-  } else {
-#pragma unroll
-    for (int h = 0; h < E / 2; ++h) {
-      const int col = v * E + 2 * h;
-      f[h].x = (ok && col < N) ? Vec<T>::load1(row + col) : 0.0f;
-      f[h].y = (ok && col + 1 < N) ? Vec<T>::load1(row + col + 1) : 0.0f;
-    }
-  }
-}
-
-template <typename T>
-__device__ __forceinline__ void store_pairs(T* row, int v, int nfull, int N, const float2 (&f)[Vec<T>::N / 2]) {
-  constexpr int E = Vec<T>::N;
-  if (v < nfull) {
-    st_stream(row + (size_t)v * E, pack2<T>(f));
-  } else {
-#pragma unroll
-    for (int h = 0; h < E / 2; ++h) {
-      const int col = v * E + 2 * h;
-      if (col < N) Vec<T>::store1(row + col, f[h].x);
-      if (col + 1 < N) Vec<T>::store1(row + col + 1, f[h].y);
-    }
-  }
-}
 
 template <typename T, int VPT, int EPI, bool GEMMA>
 __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT)) rms_fwd_cta(const RmsFwdArgs a) {
@@ -192,8 +149,12 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT, true)) r
   int s = 0;
   uint32_t ph = 0, rb = 0;
   bool failed = false;
+  // the statistic of the next row is loaded one row ahead: its global-memory latency then
+  // overlaps the current row instead of stalling the start of the next
+  float r_n = blockIdx.x < a.rows ? __ldg(a.inv_rms + blockIdx.x) : 0.0f;
   for (int64_t m = blockIdx.x; m < a.rows; m += step) {
-    const float r = __ldg(a.inv_rms + m);
+    const float r = r_n;
+    if (m + step < a.rows) r_n = __ldg(a.inv_rms + m + step);
     const float2 r2 = dup2(r);
     const bool ok = __all_sync(0xffffffffu, mbar_wait(&pipe.full[s], ph, a.err));
     uint4 xr[VPT];  // x stays packed between the two phases (unpacked on use)
@@ -201,9 +162,7 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT, true)) r
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
       const int v = ct + j * nct;
-      float2 xt[H];
-      load_pairs<T>(pipe.at(s, 0), x + m * a.ldx, v, nfull, N, ok, xt);
-      xr[j] = pack2<T>(xt);  // exact: the values came from T
+      xr[j] = load_raw<T>(pipe.at(s, 0), x + m * a.ldx, v, nfull, N, ok);
       load_pairs<T>(pipe.at(s, 1), dy + m * a.lddy, v, nfull, N, ok, gv[j]);
     }
     __syncwarp();

@@ -251,7 +251,6 @@ __global__ void __launch_bounds__(kRopeMaxThreads, 2) rope_kernel(const RopeArgs
   const int D = a.D, HC = a.HC;
   const int lph = D / E;                       // vectors (lanes) per head
   const int nv_t = HC * lph;                   // vectors per tensor slab
-  const int NV = a.ntens * nv_t;
   const uint32_t nslots = (uint32_t)a.ntens * (BWD ? 2u : 1u);
   const uint32_t sstride = nslots * a.tslot + a.tabslot;
   const uint32_t slab_bytes = (uint32_t)(HC * D * (int)sizeof(T));
