@@ -261,17 +261,41 @@ __device__ __forceinline__ float epi_grad(float z) {
   }
 }
 
-// The same epilogues on a pair of lanes. They run as two scalar evaluations: the constants of
-// the tanh-GeLU fold into scalar FMA immediates, which packed fp32x2 instructions cannot take.
+// The same epilogues on a pair of lanes. The forward tanh-GeLU runs on packed fp32x2
+// instructions with the scalar form's operations, operand order and constants lane by lane, so
+// each lane rounds exactly as epi_fwd; SiLU runs as two scalar evaluations.
+template <bool FAST>
+__device__ __forceinline__ float2 tanh2(float2 u) {
+  return make_float2(tanh_f<FAST>(u.x), tanh_f<FAST>(u.y));
+}
+
 template <int EPI, bool FAST>
 __device__ __forceinline__ float2 epi_fwd2(float2 z) {
   if constexpr (EPI == EPI_NONE) {
     return z;
+  } else if constexpr (EPI == EPI_GELU_TANH) {
+    const float2 z2 = mul2(z, z);
+    const float2 t = tanh2<FAST>(mul2(z, fma2(dup2(kGeluK * kGeluC), z2, dup2(kGeluK))));
+    const float2 h = mul2(dup2(0.5f), z);
+    return fma2(h, t, h);
   } else {
     return make_float2(epi_fwd<EPI, FAST>(z.x), epi_fwd<EPI, FAST>(z.y));
   }
 }
 
+// tanh-GeLU of z = 2 h, given h: callers whose pre-activation is an affine map fold the 1/2 into
+// its parameters (scaling by a power of two is exact). With h2 = h h = z^2 / 4 the argument
+// k (z + c z^3) = h (2k + 8kc h2) and GeLU(z) = h + h tanh(.) take the same roundings as
+// epi_fwd(z), one multiplication fewer.
+template <bool FAST>
+__device__ __forceinline__ float2 gelu_of_half2(float2 h) {
+  const float2 h2 = mul2(h, h);
+  const float2 t = tanh2<FAST>(mul2(h, fma2(dup2(8.0f * (kGeluK * kGeluC)), h2, dup2(2.0f * kGeluK))));
+  return fma2(h, t, h);
+}
+
+// the gradient runs as two scalar evaluations: its packed form needs more registers for the
+// constants, which the long-row backward kernels cannot spare
 template <int EPI, bool FAST>
 __device__ __forceinline__ float2 epi_grad2(float2 z) {
   if constexpr (EPI == EPI_NONE) {

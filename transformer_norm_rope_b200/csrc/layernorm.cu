@@ -142,8 +142,11 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT)) ln_fwd_
     return;
   }
   const int ct = tid - 32, nct = ncw * 32, cw = warp - 1;
-  stage_param(pipe.param(0), static_cast<const T*>(a.w), N, nvec, 1.0f, ct, nct);
-  stage_param(pipe.param(1), static_cast<const T*>(a.b), N, nvec, 0.0f, ct, nct);
+  // with the tanh-GeLU epilogue the weight and bias are staged halved (exact): the affine map
+  // then yields z / 2, which gelu_of_half2 takes directly
+  constexpr float kParamScale = EPI == EPI_GELU_TANH ? 0.5f : 1.0f;
+  stage_param(pipe.param(0), static_cast<const T*>(a.w), N, nvec, 1.0f, ct, nct, kParamScale);
+  stage_param(pipe.param(1), static_cast<const T*>(a.b), N, nvec, 0.0f, ct, nct, kParamScale);
   consumers_sync(nct);
   int cnt[VPT];
 #pragma unroll
@@ -214,7 +217,13 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT)) ln_fwd_
         param_pairs<T>(pipe.param(0), v, wv);
         param_pairs<T>(pipe.param(1), v, bv);
 #pragma unroll
-        for (int h = 0; h < H; ++h) o[h] = epi_fwd2<EPI, FAST>(fma2(fma2(xv[j][h], rs2, nmr2), wv[h], bv[h]));
+        for (int h = 0; h < H; ++h) {
+          const float2 z = fma2(fma2(xv[j][h], rs2, nmr2), wv[h], bv[h]);
+          if constexpr (EPI == EPI_GELU_TANH)
+            o[h] = gelu_of_half2<FAST>(z);
+          else
+            o[h] = epi_fwd2<EPI, FAST>(z);
+        }
         store_pairs<T>(yrow, v, nfull, N, o);
       }
     }

@@ -10,11 +10,13 @@
 namespace gn {
 
 // per-column parameters (weight, bias) copied once into shared memory, padded with zeros
+// (times `scale`, a power of two, so the stored values stay exact)
 template <typename T>
-__device__ __forceinline__ void stage_param(uint8_t* dst, const T* src, int N, int nvec, float dflt, int ct, int nct) {
+__device__ __forceinline__ void stage_param(uint8_t* dst, const T* src, int N, int nvec, float dflt, int ct, int nct,
+                                            float scale = 1.0f) {
   T* d = reinterpret_cast<T*>(dst);
   const int n = nvec * Vec<T>::N;
-  for (int i = ct; i < n; i += nct) Vec<T>::store1(d + i, i < N ? ld_param(src, i, dflt) : 0.0f);
+  for (int i = ct; i < n; i += nct) Vec<T>::store1(d + i, i < N ? scale * ld_param(src, i, dflt) : 0.0f);
 }
 
 // the parameters of vector v as element pairs

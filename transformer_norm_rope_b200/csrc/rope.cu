@@ -52,6 +52,8 @@ struct RopeArgs {
   float sign;
   uint32_t units;          // B * S * NC
   uint32_t tslot, tabslot; // bytes of one tensor slot / the table slot in a stage
+  uint32_t statslot;       // QK_BWD: bytes of one tensor's inv_rms slot in a stage
+  int stat_staged;         // QK_BWD: the producer copies the unit's inv_rms values into the stage
   unsigned* err;
 };
 
@@ -92,6 +94,8 @@ struct VecCtx {
   const uint8_t* sb;   // the unit's stage
   const float* tcos;   // the token's table rows in the stage
   const float* tsin;
+  const float* tstat;  // QK_BWD: the unit's inv_rms values in the stage (null: read from global)
+  int sstat;           // floats between the tensors' inv_rms slots
   int64_t row0;        // first head row of the unit
   int lph, lph_shift;  // vectors per head (and log2 when a power of two, else -1)
   float inv_d;
@@ -205,7 +209,8 @@ __device__ __forceinline__ void rope_vec(const RopeArgs& a, const VecCtx& c, int
     }
     if (valid && l == 0 && a.stat[TT]) a.stat[TT][c.row0 + hh] = r;
   } else {  // QK_BWD
-    const float r = valid ? __ldg(a.stat[TT] + c.row0 + hh) : 0.0f;  // r = 0: invalid lanes add nothing
+    // r = 0: invalid lanes add nothing
+    const float r = !valid ? 0.0f : c.tstat ? c.tstat[TT * c.sstat + hh] : __ldg(a.stat[TT] + c.row0 + hh);
     const float2 r2 = dup2(r);
     float2 d0[K], d1[K];
     PL::load(*reinterpret_cast<const uint4*>(c.sb + (a.ntens + TT) * a.tslot + (size_t)w * 16), d0, d1);
@@ -239,7 +244,6 @@ template <typename T, int MODE, bool GEMMA>
 __global__ void __launch_bounds__(kRopeMaxThreads, 2) rope_kernel(const RopeArgs a) {
   using V = Vec<T>;
   constexpr int E = V::N;      // elements per 16-byte vector
-  constexpr int P = E / 2;     // pairs per vector
   constexpr bool BWD = MODE == QK_BWD;
   constexpr bool NORM = MODE != ROPE;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -252,9 +256,11 @@ __global__ void __launch_bounds__(kRopeMaxThreads, 2) rope_kernel(const RopeArgs
   const int lph = D / E;                       // vectors (lanes) per head
   const int nv_t = HC * lph;                   // vectors per tensor slab
   const uint32_t nslots = (uint32_t)a.ntens * (BWD ? 2u : 1u);
-  const uint32_t sstride = nslots * a.tslot + a.tabslot;
+  const uint32_t sstride = nslots * a.tslot + a.tabslot + (BWD ? (uint32_t)a.ntens * a.statslot : 0u);
   const uint32_t slab_bytes = (uint32_t)(HC * D * (int)sizeof(T));
   const uint32_t tab_bytes = (uint32_t)(D / 2 * 4);
+  const bool stat_staged = BWD && a.stat_staged;
+  const uint32_t stat_bytes = stat_staged ? (uint32_t)(HC * 4) : 0u;
   const uint32_t step = gridDim.x;
 
   if (threadIdx.x == 0) {
@@ -279,7 +285,7 @@ __global__ void __launch_bounds__(kRopeMaxThreads, 2) rope_kernel(const RopeArgs
       unit_origin(a, u, bs, c, s);
       const int64_t eoff = (bs * a.H + (int64_t)c * HC) * D;
       uint8_t* sb = data + (size_t)st * sstride;
-      mbar_expect_tx(&full[st], nslots * slab_bytes + 2 * tab_bytes);
+      mbar_expect_tx(&full[st], nslots * slab_bytes + 2 * tab_bytes + (uint32_t)a.ntens * stat_bytes);
       for (int t = 0; t < a.ntens; ++t) {
         bulk_g2s(sb + t * a.tslot, static_cast<const T*>(a.x[t]) + eoff, slab_bytes, &full[st]);
         if constexpr (BWD)
@@ -288,6 +294,9 @@ __global__ void __launch_bounds__(kRopeMaxThreads, 2) rope_kernel(const RopeArgs
       uint8_t* tb = sb + nslots * a.tslot;
       bulk_g2s(tb, a.cos + (int64_t)s * (D / 2), tab_bytes, &full[st]);
       bulk_g2s(tb + tab_bytes, a.sin + (int64_t)s * (D / 2), tab_bytes, &full[st]);
+      if (stat_staged)  // the HC saved statistics of the unit's head rows, per tensor
+        for (int t = 0; t < a.ntens; ++t)
+          bulk_g2s(tb + a.tabslot + t * a.statslot, a.stat[t] + eoff / D, stat_bytes, &full[st]);
       used |= 1u << st;
       lastph = (lastph & ~(1u << st)) | (ph << st);
       if (++st == a.stages) st = 0, ph ^= 1u;
@@ -337,7 +346,8 @@ __global__ void __launch_bounds__(kRopeMaxThreads, 2) rope_kernel(const RopeArgs
     const int64_t row0 = bs * a.H + (int64_t)c * HC;  // first head row of the unit
     const uint8_t* sb = data + (size_t)st * sstride;
     const float* tcos = reinterpret_cast<const float*>(sb + nslots * a.tslot);
-    const VecCtx ctx{sb, tcos, tcos + D / 2, row0, lph, a.lph_shift, inv_d};
+    const float* tstat = stat_staged ? reinterpret_cast<const float*>(sb + nslots * a.tslot + a.tabslot) : nullptr;
+    const VecCtx ctx{sb, tcos, tcos + D / 2, tstat, (int)(a.statslot / 4), row0, lph, a.lph_shift, inv_d};
     // Each pass covers one tensor (the tensor is a compile-time argument of the body); the
     // trip count is the same for every lane of a warp, so the head shuffles see full warps.
     for (int vb = 0; vb < nv_t; vb += nct) rope_vec<T, MODE, 0>(a, ctx, vb + ct, nv_t, wq0, wq1, dq0, dq1);
@@ -376,7 +386,7 @@ __global__ void __launch_bounds__(kRopeMaxThreads, 2) rope_kernel(const RopeArgs
 
 struct RopePlan {
   int HC, NC, cwarps, threads, stages, lph_shift;
-  uint32_t tslot, tabslot;
+  uint32_t tslot, tabslot, statslot;
   size_t smem;
 };
 
@@ -409,7 +419,8 @@ gn_status plan_rope(int64_t B, int64_t S, int64_t H, int64_t D, int ntens, int m
   p->lph_shift = (lph & (lph - 1)) == 0 ? __builtin_ctz((unsigned)lph) : -1;
   p->tslot = round128((uint32_t)(HC * D * (int64_t)es));
   p->tabslot = round128((uint32_t)(D * 4));
-  const size_t sstride = (size_t)nslots * p->tslot + p->tabslot;
+  p->statslot = mode == QK_BWD ? round128((uint32_t)(HC * 4)) : 0u;
+  const size_t sstride = (size_t)nslots * p->tslot + p->tabslot + (size_t)ntens * p->statslot;
   // stage depth per CTA (measured on B200): the plain rotation computes so little that one
   // CTA with a deep pipeline streams best; the qk-norm passes keep ~64-96 KiB per CTA so that
   // 2-3 CTAs share an SM
@@ -471,6 +482,12 @@ gn_status launch(void* kern, int grid, const RopePlan& p, RopeArgs& a, cudaStrea
   a.stages = p.stages;
   a.tslot = p.tslot;
   a.tabslot = p.tabslot;
+  a.statslot = p.statslot;
+  // the unit's saved statistics move with the unit when each unit's HC values start on a
+  // 16-byte boundary (bulk copies need 16-byte aligned addresses and sizes); otherwise the
+  // consumers read them from global memory
+  a.stat_staged = p.statslot && p.HC % 4 == 0 && a.H % 4 == 0 && aligned16(a.stat[0]) &&
+                  (a.ntens < 2 || aligned16(a.stat[1]));
   a.lph_shift = p.lph_shift;
   a.units = (uint32_t)((int64_t)a.B * a.S * p.NC);
   a.err = device_err_word();
