@@ -82,13 +82,39 @@ __device__ __forceinline__ int consumers_any(int nthreads, int pred) {
   return r;
 }
 
-__device__ __forceinline__ void unit_origin(const RopeArgs& a, uint32_t u, int64_t& bs, int& c, int& s) {
-  c = (int)(u % (uint32_t)a.NC);
-  const uint32_t t2 = u / (uint32_t)a.NC;
-  const int b = (int)(t2 % (uint32_t)a.B);
-  s = (int)(t2 / (uint32_t)a.B);
-  bs = (int64_t)b * a.S + s;
-}
+// The CTA's walk over the units u = blockIdx.x + i * gridDim.x, u = (s * B + b) * NC + c (slab c
+// of batch b, token s). The decode takes divisions once per CTA; each step then adds the
+// decoded stride with carries.
+struct UnitWalk {
+  uint32_t u;
+  int c, b, s;     // decode of u
+  int dc, db, ds;  // decode of the stride gridDim.x
+
+  __device__ __forceinline__ static void decode(const RopeArgs& a, uint32_t v, int& c, int& b, int& s) {
+    c = (int)(v % (uint32_t)a.NC);
+    const uint32_t t = v / (uint32_t)a.NC;
+    b = (int)(t % (uint32_t)a.B);
+    s = (int)(t / (uint32_t)a.B);
+  }
+  __device__ __forceinline__ explicit UnitWalk(const RopeArgs& a) : u(blockIdx.x) {
+    decode(a, blockIdx.x, c, b, s);
+    decode(a, gridDim.x, dc, db, ds);
+  }
+  __device__ __forceinline__ void next(const RopeArgs& a) {
+    u += gridDim.x;
+    c += dc;
+    int carry = c >= a.NC;
+    if (carry) c -= a.NC;
+    b += db + carry;
+    carry = b >= a.B;
+    if (carry) b -= a.B;
+    s += ds + carry;
+  }
+  __device__ __forceinline__ int64_t token() const { return s; }
+  __device__ __forceinline__ int64_t first_row(const RopeArgs& a) const {  // first head row
+    return ((int64_t)b * a.S + s) * a.H + (int64_t)c * a.HC;
+  }
+};
 
 struct VecCtx {
   const uint8_t* sb;   // the unit's stage
@@ -261,7 +287,6 @@ __global__ void __launch_bounds__(kRopeMaxThreads, 2) rope_kernel(const RopeArgs
   const uint32_t tab_bytes = (uint32_t)(D / 2 * 4);
   const bool stat_staged = BWD && a.stat_staged;
   const uint32_t stat_bytes = stat_staged ? (uint32_t)(HC * 4) : 0u;
-  const uint32_t step = gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int st = 0; st < a.stages; ++st) {
@@ -278,12 +303,10 @@ __global__ void __launch_bounds__(kRopeMaxThreads, 2) rope_kernel(const RopeArgs
     int st = 0;
     uint32_t ph = 0, used = 0, lastph = 0;
     uint32_t k = 0;
-    for (uint32_t u = blockIdx.x; u < a.units; u += step, ++k) {
+    for (UnitWalk uw(a); uw.u < a.units; uw.next(a), ++k) {
       if (k >= (uint32_t)a.stages && !mbar_wait(&empty[st], ph ^ 1u, a.err)) break;
-      int64_t bs;
-      int c, s;
-      unit_origin(a, u, bs, c, s);
-      const int64_t eoff = (bs * a.H + (int64_t)c * HC) * D;
+      const int64_t row0 = uw.first_row(a), s = uw.token();
+      const int64_t eoff = row0 * D;
       uint8_t* sb = data + (size_t)st * sstride;
       mbar_expect_tx(&full[st], nslots * slab_bytes + 2 * tab_bytes + (uint32_t)a.ntens * stat_bytes);
       for (int t = 0; t < a.ntens; ++t) {
@@ -296,7 +319,7 @@ __global__ void __launch_bounds__(kRopeMaxThreads, 2) rope_kernel(const RopeArgs
       bulk_g2s(tb + tab_bytes, a.sin + (int64_t)s * (D / 2), tab_bytes, &full[st]);
       if (stat_staged)  // the HC saved statistics of the unit's head rows, per tensor
         for (int t = 0; t < a.ntens; ++t)
-          bulk_g2s(tb + a.tabslot + t * a.statslot, a.stat[t] + eoff / D, stat_bytes, &full[st]);
+          bulk_g2s(tb + a.tabslot + t * a.statslot, a.stat[t] + row0, stat_bytes, &full[st]);
       used |= 1u << st;
       lastph = (lastph & ~(1u << st)) | (ph << st);
       if (++st == a.stages) st = 0, ph ^= 1u;
@@ -334,16 +357,13 @@ __global__ void __launch_bounds__(kRopeMaxThreads, 2) rope_kernel(const RopeArgs
   int failed = 0;
   int st = 0;
   uint32_t ph = 0;
-  for (uint32_t u = blockIdx.x; u < a.units; u += step) {
+  for (UnitWalk uw(a); uw.u < a.units; uw.next(a)) {
     const bool ok = __all_sync(0xffffffffu, mbar_wait(&full[st], ph, a.err));
     if (!ok) {
       failed = 1;
       break;
     }
-    int64_t bs;
-    int c, s;
-    unit_origin(a, u, bs, c, s);
-    const int64_t row0 = bs * a.H + (int64_t)c * HC;  // first head row of the unit
+    const int64_t row0 = uw.first_row(a);  // first head row of the unit
     const uint8_t* sb = data + (size_t)st * sstride;
     const float* tcos = reinterpret_cast<const float*>(sb + nslots * a.tslot);
     const float* tstat = stat_staged ? reinterpret_cast<const float*>(sb + nslots * a.tslot + a.tabslot) : nullptr;
