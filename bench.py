@@ -13,7 +13,9 @@ launched through the C ABI of libgn:
 once) divided by the device time of a step, in GB/s (1e9 bytes), summed over all ranks.
 Every input is larger than the 126 MB L2, and consecutive kernels touch different tensors,
 so no L2 flush is inserted. Launch with torchrun for several GPUs: each rank runs the same
-per-GPU workload on its own seeded data (weak scaling, no collective on the data path).
+per-GPU workload on its own seeded data as its shard of a data-parallel step (weak scaling); no
+activation crosses GPUs, and the step's weight gradients (views of one fp32 bucket) are summed
+over the ranks by one NCCL all-reduce per step inside the timed region.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--only KERNEL[,KERNEL]] [--scale F] [--no-e2e] [--no-cpu-baseline]
@@ -137,7 +139,10 @@ class Suite:
     of the selected kernels are generated and allocated)."""
 
     def __init__(self, gn, torch, z, host, dev, kernels):
+        from transformer_norm_rope_b200.shard import GradBucket
+
         self.gn, self.torch, self.z, self.dev = gn, torch, z, dev
+        self.kernels = list(kernels)
         fams = {FAMILY[k] for k in kernels}
         T = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)  # noqa
         F = lambda a: torch.from_numpy(np.ascontiguousarray(a))  # noqa: E731
@@ -160,17 +165,26 @@ class Suite:
         self.d = d = {k: v.to(dev) for k, v in h.items()}
         f32 = torch.float32
         E = lambda ref, dt=None: torch.empty_like(ref) if dt is None else torch.empty(ref.shape[:-1], dtype=dt, device=dev)  # noqa
-        V = lambda n: torch.empty(n, dtype=f32, device=dev)  # noqa: E731
+        # the weight gradients of the step are views of one bucket: with several ranks one
+        # all-reduce per step sums them (the data-parallel exchange of a training step)
+        gsz = {}
         if "rms" in fams:
-            N = z["rms"]["N"]
-            d.update(ry=E(d["rx"]), rr=E(d["rx"], f32), rdx=E(d["rx"]), rdw=V(N), ryg=E(d["rx"]), rrg=E(d["rx"], f32),
-                     rdxg=E(d["rx"]), rdwg=V(N))
+            gsz.update(rdw=z["rms"]["N"], rdwg=z["rms"]["N"])
         if "ln" in fams:
-            N = z["ln"]["N"]
-            d.update(ly=E(d["lx"]), lmu=E(d["lx"], f32), lrs=E(d["lx"], f32), ldx=E(d["lx"]), ldw=V(N), ldb=V(N))
+            gsz.update(ldw=z["ln"]["N"], ldb=z["ln"]["N"])
+        if "qk" in fams:
+            gsz.update(qdwq=z["qk"]["D"], qdwk=z["qk"]["D"])
+        self.grads = GradBucket(gsz, dev) if gsz else None
+        if self.grads is not None:
+            d.update(self.grads.views)
+        if "rms" in fams:
+            d.update(ry=E(d["rx"]), rr=E(d["rx"], f32), rdx=E(d["rx"]), ryg=E(d["rx"]), rrg=E(d["rx"], f32),
+                     rdxg=E(d["rx"]))
+        if "ln" in fams:
+            d.update(ly=E(d["lx"]), lmu=E(d["lx"], f32), lrs=E(d["lx"], f32), ldx=E(d["lx"]))
         if "qk" in fams:
             d.update(qqo=E(d["qq"]), qko=E(d["qk"]), qrq=E(d["qq"], f32), qrk=E(d["qk"], f32), qdxq=E(d["qq"]),
-                     qdxk=E(d["qk"]), qdwq=V(z["qk"]["D"]), qdwk=V(z["qk"]["D"]))
+                     qdxk=E(d["qk"]))
         r, l, q = z["rms"], z["ln"], z["qk"]
         self.ws_r = gn.gn_rmsnorm_bwd_workspace(r["M"], r["N"], gn.GN_BF16) if "rms" in fams else 0
         self.ws_l = gn.gn_layernorm_bwd_workspace(l["M"], l["N"], gn.GN_BF16) if "ln" in fams else 0
@@ -181,6 +195,11 @@ class Suite:
                                     "ldw", "ldb", "oq", "ok", "qqo", "qko", "qrq", "qrk", "qdxq", "qdxk", "qdwq",
                                     "qdwk") if k in d]
         self.stream = torch.cuda.current_stream(dev)
+
+    def reduce_grads(self):
+        """Sum the step's weight gradients over the ranks (one collective; no-op on one rank)."""
+        if self.grads is not None and any(k.endswith("_bwd") for k in self.kernels):
+            self.grads.allreduce()
 
     def launch(self, name):
         gn, d, z, s = self.gn, self.d, self.z, self.stream.cuda_stream
@@ -303,7 +322,7 @@ def dist_setup(args):
         import torch.distributed as dist
 
         torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=torch.device("cuda", local))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
     return ws, rank, local
 
 
@@ -342,6 +361,13 @@ def throughput_gbs(bytes_per_rank, elapsed_s, ws, device):
     return tot / el / 1e9, el
 
 
+def parallelism(ws):
+    if ws == 1:
+        return "single GPU"
+    return (f"data parallel x{ws} (weak): each GPU runs the step on its own shard of the same shapes; "
+            "the step's weight gradients are summed by one NCCL all-reduce")
+
+
 def run_ours(args):
     import torch
 
@@ -371,6 +397,8 @@ def run_ours(args):
             suite.launch(k)
             if ev is not None:
                 ev[i][1].record(stream)
+        if ws > 1:
+            suite.reduce_grads()
 
     for _ in range(args.warmup):
         step()
@@ -401,8 +429,7 @@ def run_ours(args):
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(elapsed / args.steps * 1e3, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded generator, seed = rank)",
-        "config": dict(workload_config(z), parallelism=f"replica per GPU x{ws} (weak, no collective)",
-                       bytes_per_step_per_gpu=step_bytes),
+        "config": dict(workload_config(z), parallelism=parallelism(ws), bytes_per_step_per_gpu=step_bytes),
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(ach / peak, 4), "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs"},
         "kernels": {k: {"ms": round(per_kernel[k] * 1e3, 4), "GB_s": round(nbytes[k] / per_kernel[k] / 1e9, 1),
@@ -447,6 +474,8 @@ def e2e(args, suite, kernels, step_bytes, ws, dev):
             suite.d[k].copy_(pin_in[k], non_blocking=True)
         for k in kernels:
             suite.launch(k)
+        if ws > 1:
+            suite.reduce_grads()
         for k in outs:
             pin_out[k].copy_(suite.d[k], non_blocking=True)
 
