@@ -19,6 +19,7 @@ from . import build as _build
 
 F64, F32, BF16 = 0, 1, 2
 ACT_NONE, ACT_GELU_TANH, ACT_SILU = 0, 1, 2
+NORM_RMS, NORM_LN = 0, 1
 _ACTS = {"none": ACT_NONE, "gelu_tanh": ACT_GELU_TANH, "silu": ACT_SILU}
 
 _lib = None
@@ -41,9 +42,11 @@ def _load():
         lib.oracle_rope.argtypes = [vp, ci, vp, vp, ci, i64, i64, i64, i64, ci, vp]
         lib.oracle_qknorm_rope_fwd.argtypes = [vp, ci, vp, ci, vp, vp, ci, i64, i64, i64, i64, dbl, ci, vp, vp]
         lib.oracle_qknorm_rope_bwd.argtypes = [vp, ci, vp, ci, vp, vp, ci, vp, ci, i64, i64, i64, i64, dbl, ci, vp, vp]
+        lib.oracle_norm_linear.argtypes = [vp, ci, vp, vp, ci, vp, ci, vp, ci, i64, i64, i64, dbl, ci, ci, ci,
+                                           vp, vp, vp]
         for f in ("oracle_rmsnorm_fwd", "oracle_rmsnorm_bwd", "oracle_layernorm_fwd",
                   "oracle_layernorm_bwd", "oracle_rope", "oracle_qknorm_rope_fwd",
-                  "oracle_qknorm_rope_bwd"):
+                  "oracle_qknorm_rope_bwd", "oracle_norm_linear"):
             getattr(lib, f).restype = None
         _lib = lib
     return _lib
@@ -179,3 +182,26 @@ def qknorm_rope_bwd(x, w, cos, sin, dy, eps, gemma=False, want_dx=True):
     _load().oracle_qknorm_rope_bwd(_p(x), xd, _p(w), wd, _p(cos), _p(sin), td, _p(dy), gd, B, S, H,
                                    D, eps, int(gemma), _p(dx), _p(dw))
     return dx, dw
+
+
+def norm_linear(x, g, beta, W, bias, eps, norm="ln", gemma=False, act="none"):
+    """y[M,N] = act(norm(x) W^T + bias), mean[M], rstd[M] for x[M,K], W[N,K]: the normalized
+    row (LayerNorm with weight g and bias beta, or RMSNorm with weight g), then the linear layer.
+    beta (RMSNorm: ignored) and bias may be None."""
+    x, xd = _in(x)
+    g, gd = _in(g)
+    beta, bd = _in(beta)
+    W, wd = _in(W)
+    bias, bsd = _in(bias)
+    if norm == "ln" and beta is not None and gd != bd:
+        raise TypeError("g and beta must share a dtype")
+    M, K = x.shape
+    N = W.shape[0]
+    assert W.shape == (N, K)
+    y = np.empty((M, N))
+    mu = np.empty(M)
+    rs = np.empty(M)
+    _load().oracle_norm_linear(_p(x), xd, _p(g), _p(beta if norm == "ln" else None), gd, _p(W), wd, _p(bias), bsd,
+                               M, N, K, eps, NORM_LN if norm == "ln" else NORM_RMS, int(gemma), _act(act),
+                               _p(y), _p(mu), _p(rs))
+    return y, mu, rs

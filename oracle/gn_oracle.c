@@ -339,3 +339,49 @@ void oracle_qknorm_rope_bwd(const void* x, int x_dt, const void* w, int w_dt, co
   free(row);
   free(wp);
 }
+
+/* ---- Normalization followed by the linear layer after it -------------------------------------
+ * [J] section 4.1: LayerNorm, then a linear projection, then SiLU, in one pass; the HY-Motion
+ * optimization page (section 3.1) merges LayerNorm with the matrix multiplication that follows
+ * it. Plain reading: xn = the normalized row without an activation (LayerNorm
+ * (x - mean) s g + beta, or RMSNorm x r g'), then y[m,n] = act(sum_k xn[k] W[n,k] + bias[n])
+ * with W[N,K] the layer's weight (output feature n in row n). */
+void oracle_norm_linear(const void* x, int x_dt, const void* g, const void* beta, int p_dt,
+                        const void* W, int w_dt, const void* bias, int bias_dt, int64_t M,
+                        int64_t N, int64_t K, double eps, int norm, int gemma, int act, double* y,
+                        double* mean, double* rstd) {
+  double* gv = scratch(K);
+  double* bv = scratch(K);
+  double* row = scratch(K);
+  double* xn = scratch(K);
+  double* wt = scratch(N * K);
+  if (norm == ORC_NORM_LN) {
+    load_affine(g, beta, p_dt, K, gv, bv);
+  } else {
+    load_weight(g, p_dt, K, gemma, gv);
+    for (int64_t k = 0; k < K; ++k) bv[k] = 0.0;
+  }
+  rd_row(W, w_dt, 0, N * K, wt);
+  for (int64_t m = 0; m < M; ++m) {
+    rd_row(x, x_dt, m * K, K, row);
+    double mu = 0.0, s;
+    if (norm == ORC_NORM_LN)
+      ln_row_stats(row, K, eps, &mu, &s);
+    else
+      s = rms_row_inv(row, K, eps);
+    for (int64_t k = 0; k < K; ++k) xn[k] = (row[k] - mu) * s * gv[k] + bv[k];
+    if (y)
+      for (int64_t n = 0; n < N; ++n) {
+        double acc = bias ? rd(bias, bias_dt, n) : 0.0;
+        for (int64_t k = 0; k < K; ++k) acc += xn[k] * wt[n * K + k];
+        y[m * N + n] = oracle_act(act, acc);
+      }
+    if (mean) mean[m] = mu;
+    if (rstd) rstd[m] = s;
+  }
+  free(wt);
+  free(xn);
+  free(row);
+  free(bv);
+  free(gv);
+}

@@ -20,6 +20,8 @@
  *        times weight plus bias, tanh-GeLU with constant 0.79788456 and cubic 0.044715).
  *   [J]  "Janus-Pro-7B模型推理加速实战", section 4.1 (fused LayerNorm + linear + SiLU,
  *        SiLU = x * sigmoid(x)).
+ *   [Y]  "HY-Motion 1.0性能优化从算法到硬件的全方位调优策略", section 3.1 (LayerNorm merged
+ *        with the linear layer that follows it).
  *
  * Parity pins: every function here is pinned by the CPU tests (closed forms, invariants,
  * library special cases and central finite differences); none is "parity unpinned".
@@ -85,6 +87,18 @@ void oracle_qknorm_rope_bwd(const void* x, int x_dt, const void* w, int w_dt, co
                             const void* sin_t, int tab_dt, const void* dy, int dy_dt, int64_t B,
                             int64_t S, int64_t H, int64_t D, double eps, int gemma, double* dx,
                             double* dw);
+
+/* which normalization precedes the linear layer */
+enum { ORC_NORM_RMS = 0, ORC_NORM_LN = 1 };
+
+/* Normalization (RMSNorm with weight g and optional gemma offset, or LayerNorm with weight g and
+ * bias beta; no activation) followed by the linear layer y = act(xn W^T + bias): x[M,K],
+ * W[N,K] (row n = output feature n), bias[N] or NULL, y[M*N]. mean[M] (LayerNorm; 0 for
+ * RMSNorm) and rstd[M] (1/sqrt(var + eps), or the RMSNorm inverse rms) may be NULL. */
+void oracle_norm_linear(const void* x, int x_dt, const void* g, const void* beta, int p_dt,
+                        const void* W, int w_dt, const void* bias, int bias_dt, int64_t M,
+                        int64_t N, int64_t K, double eps, int norm, int gemma, int act, double* y,
+                        double* mean, double* rstd);
 
 #ifdef __cplusplus
 }

@@ -37,6 +37,9 @@ MUTANTS = {
     "qk_bwd_forward_rotation": ("rope_row(grow, cs, sn, D, -1, u);", "rope_row(grow, cs, sn, D, +1, u);"),
     "dw_without_xhat": ("if (dw_acc) dw_acc[j] += g * xh;", "if (dw_acc) dw_acc[j] += g;"),
     "bf16_widen_wrong_shift": ("[i]) << 16;", "[i]) << 15;"),
+    "norm_linear_transposed_weight": ("acc += xn[k] * wt[n * K + k];", "acc += xn[k] * wt[k * N + n];"),
+    "norm_linear_drops_bias": ("double acc = bias ? rd(bias, bias_dt, n) : 0.0;", "double acc = 0.0;"),
+    "norm_linear_uncentred": ("xn[k] = (row[k] - mu) * s * gv[k] + bv[k];", "xn[k] = row[k] * s * gv[k] + bv[k];"),
 }
 
 

@@ -427,3 +427,59 @@ def test_qknorm_rope_is_composition_of_norm_and_rope():
     n, r2 = oracle.rmsnorm_fwd(x.reshape(-1, D), w, 1e-6)
     np.testing.assert_array_equal(out, oracle.rope(n.reshape(x.shape), cos, sin, +1))
     np.testing.assert_array_equal(r.ravel(), r2)
+
+
+# ---- normalization followed by the linear layer (Janus-Pro page, section 4.1; HY-Motion page,
+# section 3.1) -------------------------------------------------------------------------------
+
+
+def test_hand_norm_linear():
+    # LayerNorm of [1, 3]: mean 2, variance 1 (eps 0), xn = [-1, 1]; W = [[1, 2]], bias 0.5
+    y, mu, rs = oracle.norm_linear(np.array([[1.0, 3.0]]), np.ones(2), np.zeros(2), np.array([[1.0, 2.0]]),
+                                   np.array([0.5]), 0.0, "ln")
+    assert y[0, 0] == 1.5 and mu[0] == 2.0 and rs[0] == 1.0
+    # RMSNorm of [3, 4]: mean square 12.5; W = [[1, 1]] -> 7 / sqrt(12.5); with SiLU on top
+    y, mu, rs = oracle.norm_linear(np.array([[3.0, 4.0]]), np.ones(2), None, np.array([[1.0, 1.0]]), None, 0.0, "rms")
+    assert y[0, 0] == pytest.approx(7 / math.sqrt(12.5), rel=1e-15) and mu[0] == 0.0
+    z = 7 / math.sqrt(12.5) + 0.25
+    y, _, _ = oracle.norm_linear(np.array([[3.0, 4.0]]), np.ones(2), None, np.array([[1.0, 1.0]]), np.array([0.25]),
+                                 0.0, "rms", act="silu")
+    assert y[0, 0] == pytest.approx(z / (1 + math.exp(-z)), rel=1e-14)
+
+
+@pytest.mark.parametrize("norm,act,gemma", [("ln", "none", False), ("ln", "silu", False), ("ln", "gelu_tanh", False),
+                                            ("rms", "silu", False), ("rms", "none", True)])
+def test_norm_linear_is_the_norm_then_a_matmul(norm, act, gemma):
+    # the normalization (pinned above) followed by numpy's fp64 matrix product, bias and the
+    # activation; W is deliberately not square, so a transposed operand cannot pass
+    M, N, K, eps = 7, 5, 24, 1e-5
+    x = rng.standard_normal((M, K)) * 2 + 0.7
+    g = 1 + 0.2 * rng.standard_normal(K)
+    beta = 0.3 * rng.standard_normal(K)
+    W = rng.standard_normal((N, K)) / math.sqrt(K)
+    bias = rng.standard_normal(N)
+    y, mu, rs = oracle.norm_linear(x, g, beta, W, bias, eps, norm, gemma=gemma, act=act)
+    if norm == "ln":
+        xn, m2, r2 = oracle.layernorm_fwd(x, g, beta, eps)
+        np.testing.assert_array_equal(mu, m2)
+    else:
+        xn, r2 = oracle.rmsnorm_fwd(x, g, eps, gemma=gemma)
+        assert not mu.any()
+    np.testing.assert_array_equal(rs, r2)
+    z = xn @ W.T + bias
+    ref = np.vectorize(lambda v: oracle.act(act, v))(z)
+    np.testing.assert_allclose(y, ref, rtol=1e-13, atol=1e-13)
+
+
+def test_norm_linear_with_identity_weight_is_the_norm():
+    M, K = 4, 16
+    x = rng.standard_normal((M, K))
+    g, beta = 1 + 0.1 * rng.standard_normal(K), 0.1 * rng.standard_normal(K)
+    y, _, _ = oracle.norm_linear(x, g, beta, np.eye(K), None, 1e-6, "ln")
+    np.testing.assert_allclose(y, oracle.layernorm_fwd(x, g, beta, 1e-6)[0], rtol=1e-15, atol=1e-15)
+    # output feature n reads row n of W: a one-hot row picks one normalized column
+    W = np.zeros((3, K))
+    W[0, 5], W[1, 0], W[2, K - 1] = 1.0, 1.0, 1.0
+    y, _, _ = oracle.norm_linear(x, g, beta, W, None, 1e-6, "ln")
+    xn = oracle.layernorm_fwd(x, g, beta, 1e-6)[0]
+    np.testing.assert_array_equal(y, xn[:, [5, 0, K - 1]])
