@@ -15,7 +15,11 @@
  *         points combine them per attention head).
  *   [L] "LLM层的优化算子", section "编写定制融合算子": LayerNorm fused with a tanh-GeLU epilogue
  *       (centre, biased variance, divide by sqrt(var + eps), times weight plus bias, GeLU).
- *   [J] "Janus-Pro-7B模型推理加速实战", section 4.1: LayerNorm fused with SiLU = x * sigmoid(x).
+ *   [J] "Janus-Pro-7B模型推理加速实战", section 4.1: LayerNorm fused with SiLU = x * sigmoid(x),
+ *       and LayerNorm, the first linear projection and SiLU fused into one kernel.
+ *   [Y] "HY-Motion 1.0性能优化从算法到硬件的全方位调优策略", section 3.1: LayerNorm merged with
+ *       the matrix multiplication that follows it (no round trip of the normalized activations
+ *       through memory).
  *
  * Conventions for every entry point:
  *   - Pointers are DEVICE pointers owned by the caller, except where stated. The library
@@ -71,6 +75,9 @@ typedef enum { GN_F32 = 0, GN_BF16 = 1 } gn_dtype;
 
 /* epilogue applied to z = normalized * weight (+ bias) before the store */
 typedef enum { GN_EPI_NONE = 0, GN_EPI_GELU_TANH = 1, GN_EPI_SILU = 2 } gn_epilogue;
+
+/* the normalization in front of the fused linear layer */
+typedef enum { GN_NORM_RMS = 0, GN_NORM_LN = 1 } gn_norm;
 
 /* device error word bits */
 #define GN_DEVERR_WAIT_TIMEOUT 1u
@@ -196,6 +203,40 @@ gn_status gn_qknorm_rope_bwd_noalloc(const void* q, const void* k, const void* w
                                      const void* dq_out, const void* dk_out, void* dq, void* dk,
                                      float* dwq, float* dwk, int64_t B, int64_t S, int64_t H,
                                      int64_t D, int gemma, gn_dtype dt, void* stream);
+
+/* ---- normalization + linear layer on the tensor cores ([J] section 4.1, [Y] section 3.1) ----
+ * y[m,n] = act( sum_k xn[m,k] W[n,k] + bias[n] ) with xn the normalized row of x[M,K]:
+ *   GN_NORM_LN : xn = (x - mean) rstd g + beta   (biased variance, rstd = 1/sqrt(var + eps))
+ *   GN_NORM_RMS: xn = x rstd g',  g' = g or 1 + g (gemma),  rstd = 1/sqrt(mean(x^2) + eps)
+ * The normalization is folded into the layer instead of being materialised: the forward
+ * multiplies the raw x by Wf = bf16(g' W) on the tcgen05 tensor cores and corrects each output
+ * with the row statistics, which it accumulates from the same x tiles:
+ *   y[m,n] = act( rstd_m (x Wf^T)[m,n] - rstd_m mean_m c[n] + d[n] ),
+ *   c[n] = sum_k Wf[n,k],  d[n] = sum_k beta[k] W[n,k] + bias[n]   (RMSNorm: mean = 0, d = bias).
+ * bf16 only (GN_BF16; GN_F32 returns GN_ERR_UNSUPPORTED). */
+
+/* Builds Wf [N, K] (bf16, row n = output feature n, contiguous), c [N] fp32 (LayerNorm; may be
+ * NULL for RMSNorm) and d [N] fp32 (may be NULL when beta and bias are both absent) from the
+ * layer weight W [N, K] (bf16, contiguous), the norm weight g [K] (NULL = ones), the LayerNorm
+ * bias beta [K] (NULL = zeros; ignored for RMSNorm) and the layer bias [N] (NULL = zeros), all
+ * bf16. Run it once per weight update; Wf, c and d are then read by every forward. The sums run
+ * in a fixed order: the results are the same on every run.
+ * Errors: GN_ERR_NULL (W, Wf, or c for LayerNorm), GN_ERR_SHAPE (N < 0, K <= 0, unknown norm). */
+gn_status gn_norm_linear_prepare(const void* W, const void* g, const void* beta, const void* bias,
+                                 void* Wf, float* c, float* d, int64_t N, int64_t K, gn_norm norm,
+                                 int gemma, gn_dtype dt, void* stream);
+
+/* Forward: y [M, N] (bf16, row stride ldy) from x [M, K] (bf16, row stride ldx) and the
+ * prepared Wf, c, d. mean and rstd (fp32 [M], each may be NULL) receive the row statistics
+ * (mean = 0 for RMSNorm). K, ldx and ldy must be multiples of 8; x, Wf, y, c and d 16-byte
+ * aligned; M up to 8388480. Ragged M, N and K are handled (tiles of 128 x 256 outputs, 64 k).
+ * Errors: GN_ERR_SHAPE (sizes, strides, norm), GN_ERR_DTYPE (epilogue), GN_ERR_ALIGN,
+ * GN_ERR_NULL (x, Wf, y, or c for LayerNorm), GN_ERR_CUDA (tensor-map encoding or launch).
+ * M == 0 or N == 0: nothing is launched. */
+gn_status gn_norm_linear_fwd(const void* x, const void* Wf, const float* c, const float* d, void* y,
+                             float* mean, float* rstd, int64_t M, int64_t N, int64_t K, int64_t ldx,
+                             int64_t ldy, float eps, gn_norm norm, gn_epilogue epi, gn_dtype dt,
+                             void* stream);
 
 /* ---------------------------------------------------------------- runtime queries
  * Number of kernels this process has launched through libgn (all devices, all threads). */

@@ -1,0 +1,85 @@
+"""Normalization + linear layer on the tensor cores (gn_norm_linear_prepare / gn_norm_linear_fwd)
+against the fp64 oracle: y = act(norm(x) W^T + bias) for LayerNorm and RMSNorm, the three
+epilogues, the Gemma offset, ragged M, N and K, and the benchmark size on sampled rows.
+
+Tolerance: the bf16 output tolerance (1.6e-2 relative + 1e-2 absolute). The kernel multiplies by
+Wf = bf16(g W), one bf16 rounding per weight, where the unfused layer rounds the normalized
+activations instead; with W ~ N(0, 1/K) and unit-scale outputs either rounding perturbs an output
+by about 1e-3 (random over K terms), an order of magnitude inside the bound. The row statistics
+(fp32, shifted one-pass moments over the streamed tiles) are checked at 1e-5 relative."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests._util import assert_close, to_dev, to_np
+from transformer_norm_rope_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+
+def _inputs(M, N, K, seed, norm, gemma=False):
+    d = wl.layernorm(M=M, N=K, dtype="bf16", seed=seed)  # rows with their own mean and scale
+    g = np.random.default_rng(seed + 100)
+    bf = lambda a: wl.bf16_bits(np.asarray(a, dtype=np.float32))  # noqa: E731
+    W = bf(g.standard_normal((N, K)) / math.sqrt(K))
+    gw = bf(0.1 * g.standard_normal(K) + (0.0 if gemma else 1.0))  # Gemma stores w with w' = 1 + w
+    beta = bf(0.1 * g.standard_normal(K)) if norm == "ln" else None
+    bias = bf(0.1 * g.standard_normal(N))
+    return d["x"], gw, beta, W, bias
+
+
+def _run(gpu, x, gw, beta, W, bias, eps, norm, gemma, epi):
+    Wf, c, dd = gpu.norm_linear_prepare(to_dev(W), to_dev(gw), None if beta is None else to_dev(beta), to_dev(bias),
+                                        norm=norm, gemma=gemma)
+    y, mu, rs = gpu.norm_linear_fwd(to_dev(x), Wf, c, dd, eps=eps, norm=norm, epilogue=epi)
+    torch.cuda.synchronize()
+    return y, mu, rs
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (300, 520, 1024), (257, 264, 1000), (64, 40, 136)])
+@pytest.mark.parametrize("norm,epi,gemma", [("ln", "silu", False), ("ln", "none", False), ("rms", "gelu_tanh", False),
+                                            ("rms", "none", True)])
+def test_norm_linear_matches_oracle(gpu, M, N, K, norm, epi, gemma):
+    x, gw, beta, W, bias = _inputs(M, N, K, seed=M + N + K, norm=norm, gemma=gemma)
+    eps = 1e-5
+    y, mu, rs = _run(gpu, x, gw, beta, W, bias, eps, norm, gemma, epi)
+    ref, rmu, rrs = oracle.norm_linear(x, gw, beta, W, bias, eps, norm, gemma=gemma, act=epi)
+    assert_close(to_np(y), ref, "bf16", f"y {norm} {epi} {M}x{N}x{K}")
+    assert_close(to_np(rs), rrs, (1e-5, 0.0), "rstd")
+    if norm == "ln":
+        assert_close(to_np(mu), rmu, (1e-5, 1e-6), "mean")
+    assert gpu.device_error(clear=True) == 0
+
+
+def test_norm_linear_repeat_calls_are_identical(gpu):
+    x, gw, beta, W, bias = _inputs(256, 512, 512, seed=5, norm="ln")
+    a = _run(gpu, x, gw, beta, W, bias, 1e-5, "ln", False, "silu")[0]
+    b = _run(gpu, x, gw, beta, W, bias, 1e-5, "ln", False, "silu")[0]
+    assert torch.equal(a, b)
+
+
+def test_norm_linear_empty_and_unsupported(gpu):
+    x = torch.zeros((0, 64), dtype=torch.bfloat16, device="cuda")
+    W = torch.zeros((256, 64), dtype=torch.bfloat16, device="cuda")
+    Wf, c, d = gpu.norm_linear_prepare(W, norm="ln")
+    y, _, _ = gpu.norm_linear_fwd(x, Wf, c, d)
+    assert y.shape == (0, 256)
+    with pytest.raises(gpu.GnError):
+        gpu.norm_linear_fwd(torch.zeros((4, 60), dtype=torch.bfloat16, device="cuda"), Wf, c, d)  # K % 8
+
+
+@pytest.mark.slow
+def test_norm_linear_full_size_sampled_rows(gpu):
+    # the benchmark shape: x [32768, 5120] (LayerNorm rows), W [5120, 5120], SiLU; the oracle
+    # checks 48 rows spread over the tiles (first, last, ragged positions inside tiles)
+    M, N, K = 32768, 5120, 5120
+    x, gw, beta, W, bias = _inputs(M, N, K, seed=0, norm="ln")
+    y, mu, rs = _run(gpu, x, gw, beta, W, bias, 1e-5, "ln", False, "silu")
+    rows = np.unique(np.concatenate([np.arange(0, M, M // 40), [1, 127, 128, 129, M - 129, M - 2, M - 1]]))
+    ref, rmu, rrs = oracle.norm_linear(x[rows], gw, beta, W, bias, 1e-5, "ln", act="silu")
+    assert_close(to_np(y)[rows], ref, "bf16", "full-size y")
+    assert_close(to_np(rs)[rows], rrs, (1e-5, 0.0), "full-size rstd")
+    assert gpu.device_error(clear=True) == 0

@@ -24,6 +24,7 @@ GN_OK, GN_ERR_NULL, GN_ERR_SHAPE, GN_ERR_ALIGN, GN_ERR_DTYPE, GN_ERR_WORKSPACE, 
     GN_ERR_UNSUPPORTED, GN_ERR_CUDA = range(8)
 GN_F32, GN_BF16 = 0, 1
 GN_EPI_NONE, GN_EPI_GELU_TANH, GN_EPI_SILU = 0, 1, 2
+GN_NORM_RMS, GN_NORM_LN = 0, 1
 GN_DEVERR_WAIT_TIMEOUT = 1
 EPILOGUES = {"none": GN_EPI_NONE, "gelu_tanh": GN_EPI_GELU_TANH, "silu": GN_EPI_SILU}
 
@@ -50,6 +51,9 @@ SIGNATURES = {
                                  _vp, _sz, _i64, _i64, _i64, _i64, _int, _int, _vp]),
     "gn_qknorm_rope_bwd_noalloc": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                          _i64, _i64, _i64, _i64, _int, _int, _vp]),
+    "gn_norm_linear_prepare": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _int, _int, _int, _vp]),
+    "gn_norm_linear_fwd": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _f32, _int,
+                                 _int, _int, _vp]),
     "gn_launch_count": (C.c_uint64, []),
     "gn_device_error": (_st, [C.POINTER(C.c_uint), _int]),
     "gn_selftest_wait_timeout": (_st, [C.c_uint32, _vp]),
@@ -273,6 +277,38 @@ def qknorm_rope_bwd(q, k, wq, wk, cos, sin, inv_rms_q, inv_rms_k, dq_out, dk_out
                              _ptr(dwk), _ptr(ws), nws, B, S, H, D, int(gemma), _dt(q), _stream(stream)),
           "gn_qknorm_rope_bwd")
     return dq, dk, dwq, dwk
+
+
+def _norm(norm) -> int:
+    return {"rms": GN_NORM_RMS, "ln": GN_NORM_LN}[norm] if isinstance(norm, str) else int(norm)
+
+
+def norm_linear_prepare(W, g=None, beta=None, bias=None, norm="ln", gemma=False, stream=None):
+    """Fold the norm weight into the layer weight W [N, K] (bf16): -> (Wf [N, K] bf16, c [N] fp32
+    or None, d [N] fp32)."""
+    torch = _torch()
+    N, K = W.shape
+    Wf = torch.empty_like(W)
+    c = torch.empty(N, dtype=torch.float32, device=W.device) if _norm(norm) == GN_NORM_LN else None
+    d = torch.empty(N, dtype=torch.float32, device=W.device)
+    check(gn_norm_linear_prepare(_ptr(W), _ptr(g), _ptr(beta), _ptr(bias), _ptr(Wf), _ptr(c), _ptr(d), N, K,
+                                 _norm(norm), int(gemma), _dt(W), _stream(stream)), "gn_norm_linear_prepare")
+    return Wf, c, d
+
+
+def norm_linear_fwd(x, Wf, c, d, eps=1e-5, norm="ln", epilogue="none", save_stats=True, stream=None):
+    """y [M, N] = act(norm(x) W^T + bias) from x [M, K] and the prepared (Wf, c, d):
+    -> (y, mean, rstd) (statistics fp32 [M], or None)."""
+    torch = _torch()
+    M, K = x.shape
+    N = Wf.shape[0]
+    y = torch.empty((M, N), dtype=x.dtype, device=x.device)
+    mk = (lambda: torch.empty(M, dtype=torch.float32, device=x.device)) if save_stats else (lambda: None)
+    mu, rs = mk(), mk()
+    check(gn_norm_linear_fwd(_ptr(x), _ptr(Wf), _ptr(c), _ptr(d), _ptr(y), _ptr(mu), _ptr(rs), M, N, K,
+                             x.stride(0), y.stride(0), eps, _norm(norm), _epi(epilogue), _dt(x),
+                             _stream(stream)), "gn_norm_linear_fwd")
+    return y, mu, rs
 
 
 def device_error(clear: bool = False) -> int:

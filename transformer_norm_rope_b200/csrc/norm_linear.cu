@@ -1,0 +1,516 @@
+// norm_linear.cu - normalization fused into the linear layer that follows it, on the tcgen05
+// tensor cores (Janus-Pro inference page, section 4.1: LayerNorm, the first linear projection
+// and SiLU in one kernel; HY-Motion optimization page, section 3.1: LayerNorm merged with the
+// matrix multiplication after it, which saves the round trip of the normalized activations
+// through HBM).
+//
+// The normalization is folded into the operands instead of being applied to the A tiles:
+//   LayerNorm: xn[k] = (x[k] - mu) s g[k] + beta[k], so
+//     y[m,n] = act( s_m * sum_k x[m,k] Wf[n,k] - s_m mu_m c[n] + d[n] )
+//     with Wf[n,k] = bf16(g[k] W[n,k]), c[n] = sum_k Wf[n,k], d[n] = sum_k beta[k] W[n,k] + bias[n];
+//   RMSNorm:   y[m,n] = act( r_m * sum_k x[m,k] Wf[n,k] + d[n] ), Wf = bf16(g'[k] W[n,k]), d = bias.
+// gn_norm_linear_prepare builds Wf, c and d once per weight (a memory-bound pass over W). The
+// forward kernel then streams the raw bf16 x and Wf through TMA straight into the tensor
+// cores; the per-row statistics (mu, s or r) are accumulated by the epilogue warps from the
+// same A tiles while they sit in shared memory, and applied with the column terms and the
+// activation when the fp32 accumulator is read back from tensor memory.
+//
+// Forward kernel, one 128 x 256 output tile per CTA (6 warps):
+//   warp 0      TMA producer: A tile [128 rows x 64 k] and B tile [256 rows x 64 k] per stage,
+//               128-byte swizzled, 4 stages (48 KiB each);
+//   warp 1      allocates 256 tensor-memory columns; one lane issues tcgen05.mma (M=128,
+//               N=256, K=16, bf16 in, fp32 accumulate) and commits each stage back to the
+//               producer, then the finished accumulator to the epilogue;
+//   warps 2..5  per-row statistics from the A tiles (thread = row; each copies its row's 128
+//               bytes of the tile to registers and releases the stage), then the epilogue:
+//               tcgen05.ld of 32 accumulator columns at a time, corrections, activation,
+//               bf16 stores. A warp may only read the tensor-memory lanes 32*(warp%4)..+31,
+//               so warp w owns rows 32*(w%4)..+31 of the tile.
+// Every mbarrier wait is bounded (kWaitLimitNs); a timeout records the error bit, the CTA
+// skips its stores, waits for its own tensor-core work and copies, frees its tensor memory
+// and exits.
+#include <cuda.h>  // CUtensorMap and the cuTensorMapEncodeTiled prototype (types only)
+
+#include <mutex>
+
+#include "gn_common.cuh"
+#include "gn_host.h"
+
+namespace gn {
+namespace {
+
+constexpr int kBM = 128, kBN = 256, kBK = 64, kUK = 16;  // tile and instruction shapes
+constexpr int kStages = 4;
+constexpr int kThreads = 192;
+constexpr uint32_t kABytes = kBM * kBK * 2;  // 16 KiB
+constexpr uint32_t kBBytes = kBN * kBK * 2;  // 32 KiB
+constexpr uint32_t kStageBytes = kABytes + kBBytes;
+constexpr uint32_t kTmemCols = kBN;  // fp32 accumulator: one column per output column
+constexpr size_t kSmemBytes = 1024 /* alignment slack */ + (size_t)kStages * kStageBytes + 256;
+
+// instruction descriptor of tcgen05.mma kind::f16: D fp32 (bits 4-5 = 1), A and B bf16 (bits 7-9,
+// 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 at bit 17, M >> 4 at bit 24
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) |
+                            ((uint32_t)(kBM >> 4) << 24);
+
+struct NlArgs {
+  const float* c;  // [N] (LayerNorm)
+  const float* d;  // [N] or null
+  __nv_bfloat16* y;
+  float* mean;  // [M] or null
+  float* rstd;  // [M] or null
+  int M, N, K;
+  int64_t ldy;
+  float eps;
+  unsigned* err;
+};
+
+// ---------------------------------------------------------------- PTX wrappers
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {  // whole warp
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(slot)), "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {  // whole warp
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// D[tmem] (+)= A[smem] * B[smem]^T for one M=128, N=256, K=16 step
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
+      : "memory");
+}
+
+// arrive once on `bar` when every tcgen05.mma this thread issued before has completed
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+               : "memory");
+}
+
+// shared-memory matrix descriptor of a K-major tile of 128-byte rows in the 128-byte swizzle
+// layout: start address >> 4 (bits 0-13), leading-dimension offset 16 B (encoded 1, bits
+// 16-29; unused by this layout), stride between 8-row groups 1024 B (encoded 64, bits 32-45),
+// descriptor version 1 (bits 46-47), layout SWIZZLE_128B = 2 (bits 61-63). Tiles start on
+// 1024-byte boundaries, so the base offset (bits 49-51) is 0.
+__device__ __forceinline__ uint64_t sw128_desc(const void* tile) {
+  return (uint64_t)((smem_addr(tile) & 0x3FFFFu) >> 4) | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void mbar_arrive1(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+// ---------------------------------------------------------------- forward kernel
+
+template <int NORM, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    norm_linear_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                       const NlArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* accf = empty + kStages;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(accf + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * kBN, m0 = blockIdx.y * kBM;
+  const int nk = (a.K + kBK - 1) / kBK;
+  auto A = [&](int s) { return smem + s * kStageBytes; };
+  auto B = [&](int s) { return smem + s * kStageBytes + kABytes; };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1 + 4);  // the MMA commit and the four statistics warps
+    }
+    mbar_init(accf, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 1) tmem_alloc(tslot, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t lastph = 0, used = 0;
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % kStages;
+        const uint32_t ph = (uint32_t)(kb / kStages) & 1u;
+        if (kb >= kStages && !mbar_wait(&empty[s], ph ^ 1u, a.err)) {
+          *abort_flag = 1;
+          break;
+        }
+        if (*abort_flag) break;
+        mbar_expect_tx(&full[s], kStageBytes);
+        tma_load_2d(A(s), &tmA, kb * kBK, m0, &full[s]);
+        tma_load_2d(B(s), &tmB, kb * kBK, n0, &full[s]);
+        used |= 1u << s;
+        lastph = (lastph & ~(1u << s)) | (ph << s);
+      }
+      // every copy issued has landed before the CTA may exit
+      for (int s = 0; s < kStages; ++s)
+        if (used & (1u << s)) (void)mbar_wait(&full[s], (lastph >> s) & 1u, a.err);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % kStages;
+        const uint32_t ph = (uint32_t)(kb / kStages) & 1u;
+        if (!mbar_wait(&full[s], ph, a.err) || *abort_flag) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t ad = sw128_desc(A(s)), bd = sw128_desc(B(s));
+#pragma unroll
+        for (int k = 0; k < kBK / kUK; ++k)  // +32 bytes along K inside the swizzled rows
+          umma_bf16(tmem, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k), (kb | k) != 0);
+        umma_commit(&empty[s]);
+      }
+      umma_commit(accf);  // also after an abort: the epilogue waits for the work in flight
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ statistics + epilogue
+    const int q = warp & 3;
+    const int r = 32 * q + lane;  // row of the tile (= tensor-memory lane)
+    const uint32_t sw = (uint32_t)(r & 7);  // 16-byte chunk permutation of this row
+    // Row statistics over the streamed tiles. LayerNorm: each k-tile's mean and centred sum of
+    // squares (two passes over the 64 register-resident values), merged into the running
+    // (count, mean, M2) with Chan's update - two-pass accuracy in one sweep. RMSNorm: sum of
+    // squares, one partial per k-tile added to the running total.
+    float cnt = 0.0f, mean = 0.0f, m2 = 0.0f;
+    bool ok = true;
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % kStages;
+      const uint32_t ph = (uint32_t)(kb / kStages) & 1u;
+      ok = __all_sync(0xffffffffu, mbar_wait(&full[s], ph, a.err)) && !*abort_flag;
+      if (!ok) {
+        *abort_flag = 1;
+        break;
+      }
+      // logical chunk c of the row sits at position c ^ (r % 8) of its 128-byte line: reading
+      // in logical order spreads the 8 rows of a bank group over all 32 banks
+      const uint8_t* line = A(s) + r * 128;
+      uint4 u[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) u[c] = *reinterpret_cast<const uint4*>(line + (((uint32_t)c ^ sw) << 4));
+      const int kleft = a.K - kb * kBK;  // valid elements of this row in the tile
+      const bool whole = kleft >= kBK;
+      auto pair = [&](int c, int i) {  // element pair i of logical chunk c, invalid -> 0
+        const uint32_t w = i == 0 ? u[c].x : i == 1 ? u[c].y : i == 2 ? u[c].z : u[c].w;
+        float2 v = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+        if (!whole) {
+          const int valid = kleft - 8 * c;
+          v.x = 2 * i < valid ? v.x : 0.0f;
+          v.y = 2 * i + 1 < valid ? v.y : 0.0f;
+        }
+        return v;
+      };
+      // every loaded value is consumed before the stage is released (the next TMA write into
+      // this stage must not overtake a load still in flight)
+      float2 t = make_float2(0.0f, 0.0f);
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 v = pair(c, i);
+          t = NORM == GN_NORM_LN ? add2(t, v) : fma2(v, v, t);
+        }
+      __syncwarp();
+      if (lane == 0) mbar_arrive1(&empty[s]);
+      if (NORM == GN_NORM_LN) {
+        const float nb = whole ? (float)kBK : (float)max(kleft, 0);
+        const float bm = nb > 0.0f ? (t.x + t.y) / nb : 0.0f;
+        const float2 nbm = dup2(-bm);
+        float2 q2 = make_float2(0.0f, 0.0f);
+        float qt = 0.0f;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 dv = add2(pair(c, i), nbm);
+            if (whole) {
+              q2 = fma2(dv, dv, q2);
+            } else {  // zero-filled elements past the row are not centred values: skip them
+              const int valid = kleft - 8 * c;
+              qt = 2 * i < valid ? fmaf(dv.x, dv.x, qt) : qt;
+              qt = 2 * i + 1 < valid ? fmaf(dv.y, dv.y, qt) : qt;
+            }
+          }
+        if (nb > 0.0f) {
+          const float n = cnt + nb, dlt = bm - mean;
+          mean = fmaf(dlt, nb / n, mean);
+          m2 += q2.x + q2.y + qt + dlt * dlt * (cnt * nb / n);
+          cnt = n;
+        }
+      } else {
+        m2 += t.x + t.y;
+      }
+    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(accf, 0, a.err));
+    tc_fence_after();
+    if (ok && !*abort_flag) {
+      const float inv_k = 1.0f / (float)a.K;
+      float mu = 0.0f, rs;
+      if (NORM == GN_NORM_LN) {
+        mu = mean;
+        rs = rsqrtf(fmaf(m2, inv_k, a.eps));  // biased variance M2 / K
+      } else {
+        rs = rsqrtf(fmaf(m2, inv_k, a.eps));
+      }
+      const float nsm = -rs * mu;
+      const int m = m0 + r;
+      __nv_bfloat16* yrow = a.y + (int64_t)m * a.ldy;
+      for (int j = 0; j < kBN / 32; ++j) {
+        const int col0 = n0 + 32 * j;
+        if (col0 >= a.N) break;  // uniform over the warp
+        float v[32];
+        tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(32 * j), v);
+        const bool whole = col0 + 32 <= a.N;
+        float o[32];
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+          float4 c4 = make_float4(0.f, 0.f, 0.f, 0.f), d4 = c4;
+          if (whole) {
+            if (NORM == GN_NORM_LN) c4 = __ldg(reinterpret_cast<const float4*>(a.c + col0 + i));
+            if (a.d) d4 = __ldg(reinterpret_cast<const float4*>(a.d + col0 + i));
+          } else {
+            const float* cp = a.c;
+            const float* dp = a.d;
+            float cc[4] = {0.f, 0.f, 0.f, 0.f}, dd[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (col0 + i + e < a.N) {
+                if (NORM == GN_NORM_LN) cc[e] = cp[col0 + i + e];
+                if (dp) dd[e] = dp[col0 + i + e];
+              }
+            c4 = make_float4(cc[0], cc[1], cc[2], cc[3]);
+            d4 = make_float4(dd[0], dd[1], dd[2], dd[3]);
+          }
+          o[i + 0] = epi_fwd<EPI, true>(fmaf(rs, v[i + 0], fmaf(nsm, c4.x, d4.x)));
+          o[i + 1] = epi_fwd<EPI, true>(fmaf(rs, v[i + 1], fmaf(nsm, c4.y, d4.y)));
+          o[i + 2] = epi_fwd<EPI, true>(fmaf(rs, v[i + 2], fmaf(nsm, c4.z, d4.z)));
+          o[i + 3] = epi_fwd<EPI, true>(fmaf(rs, v[i + 3], fmaf(nsm, c4.w, d4.w)));
+        }
+        if (m < a.M) {
+          if (whole) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+              const float f8[8] = {o[i], o[i + 1], o[i + 2], o[i + 3], o[i + 4], o[i + 5], o[i + 6], o[i + 7]};
+              st_stream(yrow + col0 + i, Vec<__nv_bfloat16>::pack(f8));
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (col0 + i < a.N) yrow[col0 + i] = __float2bfloat16_rn(o[i]);
+          }
+        }
+      }
+      if (blockIdx.x == 0 && m < a.M) {
+        if (a.mean) a.mean[m] = mu;
+        if (a.rstd) a.rstd[m] = rs;
+      }
+    }
+  }
+
+  // teardown: tensor memory is freed after every warp is done with it
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- weight preparation
+// One CTA per output feature n: Wf[n,k] = bf16(g'[k] W[n,k]); c[n] = sum_k Wf[n,k] (of the
+// rounded values the GEMM multiplies); d[n] = sum_k beta[k] W[n,k] + bias[n]. The sums run in a
+// fixed order (per-thread strided partials, then a fixed tree), so they are deterministic.
+template <int NORM>
+__global__ void __launch_bounds__(256) norm_linear_prepare_kernel(const __nv_bfloat16* __restrict__ W,
+                                                                   const __nv_bfloat16* __restrict__ g,
+                                                                   const __nv_bfloat16* __restrict__ beta,
+                                                                   const __nv_bfloat16* __restrict__ bias,
+                                                                   __nv_bfloat16* __restrict__ Wf, float* __restrict__ c,
+                                                                   float* __restrict__ d, int K, int gemma) {
+  __shared__ float red[2][256];
+  const int n = blockIdx.x, t = threadIdx.x;
+  const __nv_bfloat16* wrow = W + (int64_t)n * K;
+  __nv_bfloat16* frow = Wf + (int64_t)n * K;
+  float cs = 0.0f, ds = 0.0f;
+  for (int k = t; k < K; k += 256) {
+    const float w = __bfloat162float(wrow[k]);
+    const float gk = (g ? __bfloat162float(g[k]) : 1.0f) + (NORM == GN_NORM_RMS && gemma ? 1.0f : 0.0f);
+    const __nv_bfloat16 f = __float2bfloat16_rn(gk * w);
+    frow[k] = f;
+    cs += __bfloat162float(f);
+    if (NORM == GN_NORM_LN && beta) ds = fmaf(__bfloat162float(beta[k]), w, ds);
+  }
+  red[0][t] = cs;
+  red[1][t] = ds;
+  __syncthreads();
+  for (int h = 128; h > 0; h >>= 1) {
+    if (t < h) {
+      red[0][t] += red[0][t + h];
+      red[1][t] += red[1][t + h];
+    }
+    __syncthreads();
+  }
+  if (t == 0) {
+    if (c) c[n] = red[0][0];
+    if (d) d[n] = red[1][0] + (bias ? __bfloat162float(bias[n]) : 0.0f);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encode_fn() {
+  static std::once_flag once;
+  static EncodeTiled fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiled>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor map of rows x cols (row stride ld elements), box box_rows x 64 columns,
+// 128-byte swizzle; reads outside the tensor return zeros
+bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t ld, uint32_t box_rows) {
+  EncodeTiled enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
+  const cuuint32_t box[2] = {(cuuint32_t)kBK, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int NORM>
+void* pick_epi(int epi) {
+  if (epi == GN_EPI_GELU_TANH) return (void*)norm_linear_kernel<NORM, EPI_GELU_TANH>;
+  if (epi == GN_EPI_SILU) return (void*)norm_linear_kernel<NORM, EPI_SILU>;
+  return (void*)norm_linear_kernel<NORM, EPI_NONE>;
+}
+
+}  // namespace
+}  // namespace gn
+
+using namespace gn;
+
+extern "C" gn_status gn_norm_linear_prepare(const void* W, const void* g, const void* beta, const void* bias, void* Wf,
+                                            float* c, float* d, int64_t N, int64_t K, gn_norm norm, int gemma,
+                                            gn_dtype dt, void* stream) {
+  if (dt != GN_BF16) return dt_ok(dt) ? GN_ERR_UNSUPPORTED : GN_ERR_DTYPE;
+  if (norm != GN_NORM_RMS && norm != GN_NORM_LN) return GN_ERR_SHAPE;
+  if (N < 0 || K <= 0 || K > INT32_MAX || N > INT32_MAX) return GN_ERR_SHAPE;
+  if (N == 0) return GN_OK;
+  if (!W || !Wf) return GN_ERR_NULL;
+  if (norm == GN_NORM_LN && !c) return GN_ERR_NULL;
+  cudaStream_t s = (cudaStream_t)stream;
+  const auto* Wb = static_cast<const __nv_bfloat16*>(W);
+  const auto* gb = static_cast<const __nv_bfloat16*>(g);
+  const auto* bb = static_cast<const __nv_bfloat16*>(beta);
+  const auto* cb = static_cast<const __nv_bfloat16*>(bias);
+  auto* fb = static_cast<__nv_bfloat16*>(Wf);
+  if (norm == GN_NORM_LN)
+    norm_linear_prepare_kernel<GN_NORM_LN><<<(unsigned)N, 256, 0, s>>>(Wb, gb, bb, cb, fb, c, d, (int)K, 0);
+  else
+    norm_linear_prepare_kernel<GN_NORM_RMS><<<(unsigned)N, 256, 0, s>>>(Wb, gb, nullptr, cb, fb, c, d, (int)K,
+                                                                        gemma != 0);
+  count_launches(1);
+  return launch_status();
+}
+
+extern "C" gn_status gn_norm_linear_fwd(const void* x, const void* Wf, const float* c, const float* d, void* y,
+                                        float* mean, float* rstd, int64_t M, int64_t N, int64_t K, int64_t ldx,
+                                        int64_t ldy, float eps, gn_norm norm, gn_epilogue epi, gn_dtype dt,
+                                        void* stream) {
+  if (dt != GN_BF16) return dt_ok(dt) ? GN_ERR_UNSUPPORTED : GN_ERR_DTYPE;
+  if (!epi_ok(epi)) return GN_ERR_DTYPE;
+  if (norm != GN_NORM_RMS && norm != GN_NORM_LN) return GN_ERR_SHAPE;
+  if (M < 0 || N < 0 || K <= 0 || ldx < K || ldy < N || K % 8 || ldx % 8 || ldy % 8) return GN_ERR_SHAPE;
+  if (M > (int64_t)65535 * kBM || N > INT32_MAX || K > INT32_MAX) return GN_ERR_SHAPE;
+  if (M == 0 || N == 0) return GN_OK;
+  if (!x || !Wf || !y || (norm == GN_NORM_LN && !c)) return GN_ERR_NULL;
+  if (!aligned16(x) || !aligned16(Wf) || !aligned16(y) || (c && !aligned16(c)) || (d && !aligned16(d)))
+    return GN_ERR_ALIGN;
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, x, M, K, ldx, kBM) || !make_map(&tb, Wf, N, K, K, kBN)) return GN_ERR_CUDA;
+  void* kern = norm == GN_NORM_LN ? pick_epi<GN_NORM_LN>(epi) : pick_epi<GN_NORM_RMS>(epi);
+  static std::once_flag attr_once;
+  static bool attr_ok = true;
+  std::call_once(attr_once, [] {
+    const void* ks[] = {(void*)norm_linear_kernel<GN_NORM_LN, EPI_NONE>, (void*)norm_linear_kernel<GN_NORM_LN, EPI_GELU_TANH>,
+                        (void*)norm_linear_kernel<GN_NORM_LN, EPI_SILU>, (void*)norm_linear_kernel<GN_NORM_RMS, EPI_NONE>,
+                        (void*)norm_linear_kernel<GN_NORM_RMS, EPI_GELU_TANH>, (void*)norm_linear_kernel<GN_NORM_RMS, EPI_SILU>};
+    for (const void* k : ks)
+      if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) != cudaSuccess)
+        attr_ok = false;
+  });
+  if (!attr_ok) return GN_ERR_CUDA;
+  NlArgs a{};
+  a.c = c, a.d = d;
+  a.y = static_cast<__nv_bfloat16*>(y);
+  a.mean = mean, a.rstd = rstd;
+  a.M = (int)M, a.N = (int)N, a.K = (int)K;
+  a.ldy = ldy;
+  a.eps = eps;
+  a.err = device_err_word();
+  if (!a.err) return GN_ERR_CUDA;
+  const dim3 grid((unsigned)((N + kBN - 1) / kBN), (unsigned)((M + kBM - 1) / kBM));
+  void* args[] = {&ta, &tb, &a};
+  if (cudaLaunchKernel(kern, grid, dim3(kThreads), args, kSmemBytes, (cudaStream_t)stream) != cudaSuccess)
+    return GN_ERR_CUDA;
+  count_launches(1);
+  return launch_status();
+}
