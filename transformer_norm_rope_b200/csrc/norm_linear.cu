@@ -39,19 +39,33 @@
 namespace gn {
 namespace {
 
-constexpr int kBM = 128, kBN = 256, kBK = 64, kUK = 16;  // tile and instruction shapes
-constexpr int kStages = 4;
-constexpr int kThreads = 192;
-constexpr uint32_t kABytes = kBM * kBK * 2;  // 16 KiB
-constexpr uint32_t kBBytes = kBN * kBK * 2;  // 32 KiB
-constexpr uint32_t kStageBytes = kABytes + kBBytes;
-constexpr uint32_t kTmemCols = kBN;  // fp32 accumulator: one column per output column
-constexpr size_t kSmemBytes = 1024 /* alignment slack */ + (size_t)kStages * kStageBytes + 256;
+#ifndef GN_NL_BK
+#define GN_NL_BK 64
+#endif
+constexpr int kUM = 128, kBN = 256, kBK = GN_NL_BK, kUK = 16;  // instruction M, tile N, tile K, instruction K
+constexpr uint32_t kLine = kBK * 2;  // bytes of one tile row: 64 (BK 32, 64-byte swizzle) or 128
+constexpr int kChunks = kLine / 16;  // 16-byte chunks per tile row
+constexpr uint32_t kBBytes = kBN * kLine;
+
+// A CTA computes MH x 128 rows by 256 columns: MH instructions of M = 128 share each B tile, so
+// MH = 2 moves 64 KiB of operands per 8.4 MFLOP where MH = 1 moves 48 KiB per 4.2 MFLOP (the
+// copies in flight per SM then cover the L2 latency at full tensor rate). Accumulator h sits in
+// tensor-memory columns 256h..256h+255, lanes = rows 128h.. of the tile.
+template <int MH>
+struct Tile {
+  static constexpr int BM = kUM * MH;
+  static constexpr int Stages = (MH == 1 ? 4 : 3) * (128 / kLine) + (kLine == 64 && MH == 2 ? 1 : 0);
+  static constexpr int Threads = 64 + 128 * MH;  // producer, MMA, 4*MH statistics/epilogue warps
+  static constexpr uint32_t ABytes = BM * kLine;
+  static constexpr uint32_t StageBytes = ABytes + kBBytes;
+  static constexpr uint32_t TmemCols = kBN * MH;  // fp32 accumulators: one column per output column
+  static constexpr size_t Smem = 1024 /* alignment slack */ + (size_t)Stages * StageBytes + 256 + 2 * kBN * 4;
+};
 
 // instruction descriptor of tcgen05.mma kind::f16: D fp32 (bits 4-5 = 1), A and B bf16 (bits 7-9,
 // 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 at bit 17, M >> 4 at bit 24
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) |
-                            ((uint32_t)(kBM >> 4) << 24);
+                            ((uint32_t)(kUM >> 4) << 24);
 
 struct NlArgs {
   const float* c;  // [N] (LayerNorm)
@@ -73,6 +87,13 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
           smem_addr(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
       : "memory");
+}
+
+// bring a tile into L2 ahead of its load (no shared memory involved)
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y)
+               : "memory");
 }
 
 __device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {  // whole warp
@@ -104,13 +125,21 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
                : "memory");
 }
 
-// shared-memory matrix descriptor of a K-major tile of 128-byte rows in the 128-byte swizzle
-// layout: start address >> 4 (bits 0-13), leading-dimension offset 16 B (encoded 1, bits
-// 16-29; unused by this layout), stride between 8-row groups 1024 B (encoded 64, bits 32-45),
-// descriptor version 1 (bits 46-47), layout SWIZZLE_128B = 2 (bits 61-63). Tiles start on
-// 1024-byte boundaries, so the base offset (bits 49-51) is 0.
-__device__ __forceinline__ uint64_t sw128_desc(const void* tile) {
-  return (uint64_t)((smem_addr(tile) & 0x3FFFFu) >> 4) | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
+// Shared-memory matrix descriptor of a K-major tile of kLine-byte rows in the matching swizzle
+// layout (the one TMA writes): start address >> 4 (bits 0-13), leading-dimension offset 16 B
+// (encoded 1, bits 16-29; unused by these layouts), stride between 8-row groups 8 * kLine bytes
+// (bits 32-45, in 16-byte units), descriptor version 1 (bits 46-47), layout (bits 61-63):
+// SWIZZLE_128B = 2, SWIZZLE_64B = 4. Tiles start on 1024-byte boundaries (base offset 0).
+__device__ __forceinline__ uint64_t tile_desc(const void* tile) {
+  constexpr uint64_t layout = kLine == 128 ? 2 : 4;
+  return (uint64_t)((smem_addr(tile) & 0x3FFFFu) >> 4) | (1ull << 16) | ((uint64_t)(8 * kLine / 16) << 32) |
+         (1ull << 46) | (layout << 61);
+}
+
+// 16-byte chunk c of row r sits at chunk position c ^ swz(r) of the row: the swizzle XORs
+// address bits 4.. with bits 7.. of the offset inside the tile
+__device__ __forceinline__ uint32_t swz(int r) {
+  return kLine == 128 ? (uint32_t)(r & 7) : (uint32_t)((r >> 1) & 3);
 }
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
@@ -133,12 +162,26 @@ __device__ __forceinline__ void mbar_arrive1(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
+// the epilogue's activation: the tanh-GeLU of gn_common; SiLU with the approximate divide
+// (relative error ~1e-7, far below the bf16 rounding of the output)
+template <int EPI>
+__device__ __forceinline__ float nl_act(float z) {
+  if constexpr (EPI == EPI_SILU)
+    return __fdividef(z, 1.0f + __expf(-z));
+  else
+    return epi_fwd<EPI, true>(z);
+}
+
 // ---------------------------------------------------------------- forward kernel
 
-template <int NORM, int EPI>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int MH, int NORM, int EPI>
+__global__ void __launch_bounds__(Tile<MH>::Threads, 1)
     norm_linear_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const NlArgs a) {
+  using TL = Tile<MH>;
+  constexpr int kStages = TL::Stages;
+  constexpr int kPrefetch = 2 * kStages;
+  constexpr uint32_t kABytes = TL::ABytes, kStageBytes = TL::StageBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
@@ -146,8 +189,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* accf = empty + kStages;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(accf + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+  float* col_c = reinterpret_cast<float*>(smem + kStages * kStageBytes + 256);  // c, d of the tile's columns
+  float* col_d = col_c + kBN;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * kBN, m0 = blockIdx.y * kBM;
+  const int n0 = blockIdx.x * kBN, m0 = blockIdx.y * TL::BM;
   const int nk = (a.K + kBK - 1) / kBK;
   auto A = [&](int s) { return smem + s * kStageBytes; };
   auto B = [&](int s) { return smem + s * kStageBytes + kABytes; };
@@ -155,13 +200,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + 4);  // the MMA commit and the four statistics warps
+      mbar_init(&empty[s], 1 + 4 * MH);  // the MMA commit and the statistics warps
     }
     mbar_init(accf, 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
-  if (warp == 1) tmem_alloc(tslot, kTmemCols);
+  if (warp == 1) tmem_alloc(tslot, TL::TmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -180,6 +225,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (*abort_flag) break;
         mbar_expect_tx(&full[s], kStageBytes);
+        // x is read from DRAM once per row block (the other column tiles hit in L2, W stays in
+        // L2): fetch it into L2 a ring of stages ahead so the loads wait for L2, not DRAM
+        if (kb + kPrefetch < nk) tma_prefetch_2d(&tmA, (kb + kPrefetch) * kBK, m0);
         tma_load_2d(A(s), &tmA, kb * kBK, m0, &full[s]);
         tma_load_2d(B(s), &tmB, kb * kBK, n0, &full[s]);
         used |= 1u << s;
@@ -200,10 +248,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint64_t ad = sw128_desc(A(s)), bd = sw128_desc(B(s));
+        const uint64_t ad = tile_desc(A(s)), bd = tile_desc(B(s));
 #pragma unroll
         for (int k = 0; k < kBK / kUK; ++k)  // +32 bytes along K inside the swizzled rows
-          umma_bf16(tmem, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k), (kb | k) != 0);
+#pragma unroll
+          for (int h = 0; h < MH; ++h)  // rows 128h.. of the A tile start 128 * kLine bytes further
+            umma_bf16(tmem + (uint32_t)(kBN * h), ad + (uint64_t)(2 * k + 8 * kLine * h), bd + (uint64_t)(2 * k),
+                      (kb | k) != 0);
         umma_commit(&empty[s]);
       }
       umma_commit(accf);  // also after an abort: the epilogue waits for the work in flight
@@ -211,13 +262,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ statistics + epilogue
-    const int q = warp & 3;
-    const int r = 32 * q + lane;  // row of the tile (= tensor-memory lane)
-    const uint32_t sw = (uint32_t)(r & 7);  // 16-byte chunk permutation of this row
+    const int q = warp & 3;          // tensor-memory lane quadrant this warp may read
+    const int h = (warp - 2) >> 2;   // accumulator (row half) of this warp
+    const int r = kUM * h + 32 * q + lane;  // row of the tile
+    const uint32_t sw = swz(r);  // 16-byte chunk permutation of this row
     // Row statistics over the streamed tiles. LayerNorm: each k-tile's mean and centred sum of
     // squares (two passes over the 64 register-resident values), merged into the running
     // (count, mean, M2) with Chan's update - two-pass accuracy in one sweep. RMSNorm: sum of
     // squares, one partial per k-tile added to the running total.
+    // the tile's column terms, staged once (zero past N); read back after the mainloop
+    for (int i = threadIdx.x - 64; i < kBN; i += 128 * MH) {
+      const int n = n0 + i;
+      col_c[i] = (NORM == GN_NORM_LN && n < a.N) ? a.c[n] : 0.0f;
+      col_d[i] = (a.d && n < a.N) ? a.d[n] : 0.0f;
+    }
+    asm volatile("bar.sync 1, %0;" ::"r"(128 * MH) : "memory");  // the statistics warps only
     float cnt = 0.0f, mean = 0.0f, m2 = 0.0f;
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
@@ -228,12 +287,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 1;
         break;
       }
-      // logical chunk c of the row sits at position c ^ (r % 8) of its 128-byte line: reading
-      // in logical order spreads the 8 rows of a bank group over all 32 banks
-      const uint8_t* line = A(s) + r * 128;
-      uint4 u[8];
+      // reading the row's chunks in logical order (position c ^ swz(r)) spreads the rows that
+      // share a bank group over all 32 banks
+      const uint8_t* line = A(s) + r * kLine;
+      uint4 u[kChunks];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) u[c] = *reinterpret_cast<const uint4*>(line + (((uint32_t)c ^ sw) << 4));
+      for (int c = 0; c < kChunks; ++c) u[c] = *reinterpret_cast<const uint4*>(line + (((uint32_t)c ^ sw) << 4));
       const int kleft = a.K - kb * kBK;  // valid elements of this row in the tile
       const bool whole = kleft >= kBK;
       auto pair = [&](int c, int i) {  // element pair i of logical chunk c, invalid -> 0
@@ -250,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // this stage must not overtake a load still in flight)
       float2 t = make_float2(0.0f, 0.0f);
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
+      for (int c = 0; c < kChunks; ++c)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const float2 v = pair(c, i);
@@ -265,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float2 q2 = make_float2(0.0f, 0.0f);
         float qt = 0.0f;
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
+        for (int c = 0; c < kChunks; ++c)
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const float2 dv = add2(pair(c, i), nbm);
@@ -305,32 +364,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int col0 = n0 + 32 * j;
         if (col0 >= a.N) break;  // uniform over the warp
         float v[32];
-        tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(32 * j), v);
+        tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(kBN * h + 32 * j), v);
         const bool whole = col0 + 32 <= a.N;
         float o[32];
 #pragma unroll
         for (int i = 0; i < 32; i += 4) {
-          float4 c4 = make_float4(0.f, 0.f, 0.f, 0.f), d4 = c4;
-          if (whole) {
-            if (NORM == GN_NORM_LN) c4 = __ldg(reinterpret_cast<const float4*>(a.c + col0 + i));
-            if (a.d) d4 = __ldg(reinterpret_cast<const float4*>(a.d + col0 + i));
-          } else {
-            const float* cp = a.c;
-            const float* dp = a.d;
-            float cc[4] = {0.f, 0.f, 0.f, 0.f}, dd[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              if (col0 + i + e < a.N) {
-                if (NORM == GN_NORM_LN) cc[e] = cp[col0 + i + e];
-                if (dp) dd[e] = dp[col0 + i + e];
-              }
-            c4 = make_float4(cc[0], cc[1], cc[2], cc[3]);
-            d4 = make_float4(dd[0], dd[1], dd[2], dd[3]);
-          }
-          o[i + 0] = epi_fwd<EPI, true>(fmaf(rs, v[i + 0], fmaf(nsm, c4.x, d4.x)));
-          o[i + 1] = epi_fwd<EPI, true>(fmaf(rs, v[i + 1], fmaf(nsm, c4.y, d4.y)));
-          o[i + 2] = epi_fwd<EPI, true>(fmaf(rs, v[i + 2], fmaf(nsm, c4.z, d4.z)));
-          o[i + 3] = epi_fwd<EPI, true>(fmaf(rs, v[i + 3], fmaf(nsm, c4.w, d4.w)));
+          const float4 c4 = *reinterpret_cast<const float4*>(col_c + 32 * j + i);
+          const float4 d4 = *reinterpret_cast<const float4*>(col_d + 32 * j + i);
+          o[i + 0] = nl_act<EPI>(fmaf(rs, v[i + 0], fmaf(nsm, c4.x, d4.x)));
+          o[i + 1] = nl_act<EPI>(fmaf(rs, v[i + 1], fmaf(nsm, c4.y, d4.y)));
+          o[i + 2] = nl_act<EPI>(fmaf(rs, v[i + 2], fmaf(nsm, c4.z, d4.z)));
+          o[i + 3] = nl_act<EPI>(fmaf(rs, v[i + 3], fmaf(nsm, c4.w, d4.w)));
         }
         if (m < a.M) {
           if (whole) {
@@ -358,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, TL::TmemCols);
   }
 }
 
@@ -431,16 +475,37 @@ bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, in
   const cuuint32_t box[2] = {(cuuint32_t)kBK, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, kLine == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int NORM>
+template <int MH, int NORM>
 void* pick_epi(int epi) {
-  if (epi == GN_EPI_GELU_TANH) return (void*)norm_linear_kernel<NORM, EPI_GELU_TANH>;
-  if (epi == GN_EPI_SILU) return (void*)norm_linear_kernel<NORM, EPI_SILU>;
-  return (void*)norm_linear_kernel<NORM, EPI_NONE>;
+  if (epi == GN_EPI_GELU_TANH) return (void*)norm_linear_kernel<MH, NORM, EPI_GELU_TANH>;
+  if (epi == GN_EPI_SILU) return (void*)norm_linear_kernel<MH, NORM, EPI_SILU>;
+  return (void*)norm_linear_kernel<MH, NORM, EPI_NONE>;
 }
+
+template <int MH>
+void* pick(int norm, int epi) {
+  return norm == GN_NORM_LN ? pick_epi<MH, GN_NORM_LN>(epi) : pick_epi<MH, GN_NORM_RMS>(epi);
+}
+
+template <int MH>
+bool set_smem_attr() {
+  const void* ks[] = {pick<MH>(GN_NORM_LN, GN_EPI_NONE), pick<MH>(GN_NORM_LN, GN_EPI_GELU_TANH),
+                      pick<MH>(GN_NORM_LN, GN_EPI_SILU), pick<MH>(GN_NORM_RMS, GN_EPI_NONE),
+                      pick<MH>(GN_NORM_RMS, GN_EPI_GELU_TANH), pick<MH>(GN_NORM_RMS, GN_EPI_SILU)};
+  for (const void* k : ks)
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Tile<MH>::Smem) != cudaSuccess)
+      return false;
+  return true;
+}
+
+#ifndef GN_NL_MH
+#define GN_NL_MH 2
+#endif
 
 }  // namespace
 }  // namespace gn
@@ -479,24 +544,20 @@ extern "C" gn_status gn_norm_linear_fwd(const void* x, const void* Wf, const flo
   if (!epi_ok(epi)) return GN_ERR_DTYPE;
   if (norm != GN_NORM_RMS && norm != GN_NORM_LN) return GN_ERR_SHAPE;
   if (M < 0 || N < 0 || K <= 0 || ldx < K || ldy < N || K % 8 || ldx % 8 || ldy % 8) return GN_ERR_SHAPE;
-  if (M > (int64_t)65535 * kBM || N > INT32_MAX || K > INT32_MAX) return GN_ERR_SHAPE;
+  if (M > (int64_t)65535 * kUM || N > INT32_MAX || K > INT32_MAX) return GN_ERR_SHAPE;
   if (M == 0 || N == 0) return GN_OK;
   if (!x || !Wf || !y || (norm == GN_NORM_LN && !c)) return GN_ERR_NULL;
   if (!aligned16(x) || !aligned16(Wf) || !aligned16(y) || (c && !aligned16(c)) || (d && !aligned16(d)))
     return GN_ERR_ALIGN;
+  // two accumulators (256-row tiles) once there are more than 128 rows
+  const int mh = M > kUM ? GN_NL_MH : 1;
+  const int bm = kUM * mh;
   CUtensorMap ta, tb;
-  if (!make_map(&ta, x, M, K, ldx, kBM) || !make_map(&tb, Wf, N, K, K, kBN)) return GN_ERR_CUDA;
-  void* kern = norm == GN_NORM_LN ? pick_epi<GN_NORM_LN>(epi) : pick_epi<GN_NORM_RMS>(epi);
+  if (!make_map(&ta, x, M, K, ldx, (uint32_t)bm) || !make_map(&tb, Wf, N, K, K, kBN)) return GN_ERR_CUDA;
+  void* kern = mh == 2 ? pick<2>(norm, epi) : pick<1>(norm, epi);
   static std::once_flag attr_once;
   static bool attr_ok = true;
-  std::call_once(attr_once, [] {
-    const void* ks[] = {(void*)norm_linear_kernel<GN_NORM_LN, EPI_NONE>, (void*)norm_linear_kernel<GN_NORM_LN, EPI_GELU_TANH>,
-                        (void*)norm_linear_kernel<GN_NORM_LN, EPI_SILU>, (void*)norm_linear_kernel<GN_NORM_RMS, EPI_NONE>,
-                        (void*)norm_linear_kernel<GN_NORM_RMS, EPI_GELU_TANH>, (void*)norm_linear_kernel<GN_NORM_RMS, EPI_SILU>};
-    for (const void* k : ks)
-      if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) != cudaSuccess)
-        attr_ok = false;
-  });
+  std::call_once(attr_once, [] { attr_ok = set_smem_attr<1>() && set_smem_attr<2>(); });
   if (!attr_ok) return GN_ERR_CUDA;
   NlArgs a{};
   a.c = c, a.d = d;
@@ -507,9 +568,11 @@ extern "C" gn_status gn_norm_linear_fwd(const void* x, const void* Wf, const flo
   a.eps = eps;
   a.err = device_err_word();
   if (!a.err) return GN_ERR_CUDA;
-  const dim3 grid((unsigned)((N + kBN - 1) / kBN), (unsigned)((M + kBM - 1) / kBM));
+  const dim3 grid((unsigned)((N + kBN - 1) / kBN), (unsigned)((M + bm - 1) / bm));
   void* args[] = {&ta, &tb, &a};
-  if (cudaLaunchKernel(kern, grid, dim3(kThreads), args, kSmemBytes, (cudaStream_t)stream) != cudaSuccess)
+  const int threads = mh == 2 ? Tile<2>::Threads : Tile<1>::Threads;
+  const size_t smem = mh == 2 ? Tile<2>::Smem : Tile<1>::Smem;
+  if (cudaLaunchKernel(kern, grid, dim3(threads), args, smem, (cudaStream_t)stream) != cudaSuccess)
     return GN_ERR_CUDA;
   count_launches(1);
   return launch_status();
