@@ -53,6 +53,7 @@ def parse():
     ap.add_argument("--scale", type=float, default=1.0, help="fraction of rows/tokens (profiling)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-next", action="store_true", help="skip the fused norm + linear measurement")
     ap.add_argument("--seed", type=int, default=0)
     return ap.parse_args()
 
@@ -368,6 +369,57 @@ def parallelism(ws):
             "the step's weight gradients are summed by one NCCL all-reduce")
 
 
+def norm_linear_measure(gn, torch, dev, scale, seed, reps=10):
+    """The fused LayerNorm + linear + SiLU (tcgen05 tensor cores) on x[32768, 5120] and a
+    5120 x 5120 layer, timed alone with CUDA events (median of `reps` after 3 warm-ups), beside
+    the unfused sequence it replaces: the LayerNorm kernel writing bf16 activations, a cuBLAS
+    matmul (torch) and the bias + SiLU (torch). Tensor-bound: reported against the measured bf16
+    burst peak. Not part of the HBM step."""
+    M, N, K = max(256, int(32768 * scale)), 5120, 5120
+    d = wl.norm_linear(M, N, K, seed)
+    T = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)  # noqa
+    x, g, beta, W, bias = T(d["x"]), T(d["g"]), T(d["beta"]), T(d["W"]), T(d["bias"])
+    Wf, c, dd = gn.norm_linear_prepare(W, g, beta, bias, norm="ln")
+    stream = torch.cuda.current_stream(dev)
+
+    def fused():
+        gn.norm_linear_fwd(x, Wf, c, dd, eps=d["eps"], norm="ln", epilogue="silu", save_stats=False)
+
+    def unfused():
+        xn, _, _ = gn.layernorm_fwd(x, g, beta, d["eps"], save_stats=False)
+        torch.nn.functional.silu(torch.addmm(bias, xn, W.t()))
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize(dev)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for a, b in ev:
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        return statistics.median(a.elapsed_time(b) for a, b in ev) * 1e-3
+
+    t_f, t_u = timed(fused), timed(unfused)
+    flops = 2.0 * M * N * K
+    tf = flops / t_f / 1e12
+    peak = None
+    try:
+        peak = float(json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["bf16_tflops"])
+        kind = "measured bf16_tflops (burst)"
+    except Exception:  # noqa: BLE001
+        peak, kind = 1590.0, "fallback"
+    gn.check(0 if gn.device_error(clear=True) == 0 else gn.GN_ERR_CUDA, "norm_linear device error")
+    return {"workload": f"LayerNorm + linear {K}->{N} + SiLU, x[{M},{K}] bf16 (tcgen05, one launch)",
+            "ms": round(t_f * 1e3, 4), "TFLOP_s": round(tf, 1),
+            "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(tf / peak, 4), "peak_source": kind},
+            "unfused_ms": round(t_u * 1e3, 4),
+            "unfused": "LayerNorm kernel (bf16 activations) + cuBLAS addmm + SiLU (torch)",
+            "speedup_vs_unfused": round(t_u / t_f, 3)}
+
+
 def run_ours(args):
     import torch
 
@@ -442,6 +494,10 @@ def run_ours(args):
     }
     if not args.no_e2e:
         out["e2e"] = e2e(args, suite, kernels, step_bytes, ws, dev)
+    if not args.no_next and not args.only:
+        del suite  # free the step's buffers first
+        torch.cuda.empty_cache()
+        out["next_norm_linear"] = norm_linear_measure(gn, torch, dev, args.scale, args.seed + rank)
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(host, z, kernels, budget_s=15.0)
     if rank == 0:

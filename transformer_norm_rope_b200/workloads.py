@@ -29,12 +29,14 @@ from __future__ import annotations
 import os
 from concurrent.futures import ThreadPoolExecutor
 
+import math
+
 import numpy as np
 
 CHUNK = 1 << 22
 
 # stream ids: one per tensor role, fixed forever so inputs never change meaning
-S_X, S_W, S_B, S_DY, S_ROWS, S_MU, S_SIGMA, S_Q, S_K, S_WQ, S_WK, S_DQ, S_DK = range(1, 14)
+S_X, S_W, S_B, S_DY, S_ROWS, S_MU, S_SIGMA, S_Q, S_K, S_WQ, S_WK, S_DQ, S_DK, S_LW, S_LB = range(1, 16)
 
 
 def _threads() -> int:
@@ -180,3 +182,16 @@ RMSNORM_MAIN = dict(M=15360, N=5120, dtype="bf16")
 LAYERNORM_MAIN = dict(M=32768, N=5120, dtype="bf16")
 ROPE_MAIN = dict(B=1, S=32760, H=40, D=128, dtype="bf16")
 QKNORM_MAIN = dict(B=2, S=76800, H=40, D=128, dtype="bf16")
+
+
+def norm_linear(M: int = 32768, N: int = 5120, K: int = 5120, seed: int = 0) -> dict:
+    """LayerNorm rows x[M, K] (the layernorm recipe: row mean ~ U(-2, 2), row scale ~ U(0.5, 3)),
+    norm weight g = 1 + 0.1 N(0, 1) and bias beta = 0.1 N(0, 1) over K, then the linear layer
+    W[N, K] ~ N(0, 1/K) (unit-scale outputs) with bias 0.1 N(0, 1) over N; all bf16."""
+    d = layernorm(M=M, N=K, dtype="bf16", seed=seed)
+    return {
+        "x": d["x"], "g": d["w"], "beta": d["b"],
+        "W": normal(seed, S_LW, N * K, "bf16", scale=1.0 / math.sqrt(K)).reshape(N, K),
+        "bias": normal(seed, S_LB, N, "bf16", scale=0.1),
+        "eps": 1e-5,
+    }
