@@ -227,12 +227,14 @@ gn_status gn_norm_linear_prepare(const void* W, const void* g, const void* beta,
                                  int gemma, gn_dtype dt, void* stream);
 
 /* Forward: y [M, N] (bf16, row stride ldy) from x [M, K] (bf16, row stride ldx) and the
- * prepared Wf, c, d. mean and rstd (fp32 [M], each may be NULL) receive the row statistics
- * (mean = 0 for RMSNorm). K, ldx and ldy must be multiples of 8; x, Wf, y, c and d 16-byte
- * aligned; M up to 8388480. Ragged M, N and K are handled (tiles of 128 x 256 outputs, 64 k).
+ * prepared Wf, c, d. mean [M] (LayerNorm; may be NULL for RMSNorm) and rstd [M] (fp32) receive
+ * the row statistics and are required: beyond 128 rows and 256 columns a streaming pre-pass
+ * writes them and the matrix kernel (pairs of SMs, 256 x 512 tiles) reads them back; below that
+ * one kernel computes them from its own tiles. K, ldx and ldy must be multiples of 8; x, Wf, y, c
+ * and d 16-byte aligned; M up to 8388480. Ragged M, N and K are handled.
  * Errors: GN_ERR_SHAPE (sizes, strides, norm), GN_ERR_DTYPE (epilogue), GN_ERR_ALIGN,
- * GN_ERR_NULL (x, Wf, y, or c for LayerNorm), GN_ERR_CUDA (tensor-map encoding or launch).
- * M == 0 or N == 0: nothing is launched. */
+ * GN_ERR_NULL (x, Wf, y, rstd, or c and mean for LayerNorm), GN_ERR_CUDA (tensor-map encoding
+ * or launch). M == 0 or N == 0: nothing is launched. */
 gn_status gn_norm_linear_fwd(const void* x, const void* Wf, const float* c, const float* d, void* y,
                              float* mean, float* rstd, int64_t M, int64_t N, int64_t K, int64_t ldx,
                              int64_t ldy, float eps, gn_norm norm, gn_epilogue epi, gn_dtype dt,

@@ -123,19 +123,21 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
 def test_norm_linear_argument_checks(lib):
     f = gn.gn_norm_linear_fwd
     LN, RMS = gn.GN_NORM_LN, gn.GN_NORM_RMS
-    ok = (P, P, P, P, P, None, None, 256, 512, 1024, 1024, 512, 1e-5)
+    ok = (P, P, P, P, P, P, P, 256, 512, 1024, 1024, 512, 1e-5)
     assert f(*ok, LN, 0, gn.GN_F32, None) == gn.GN_ERR_UNSUPPORTED
     assert f(*ok, LN, 0, 7, None) == gn.GN_ERR_DTYPE
     assert f(*ok, LN, 9, gn.GN_BF16, None) == gn.GN_ERR_DTYPE
     assert f(*ok, 5, 0, gn.GN_BF16, None) == gn.GN_ERR_SHAPE
-    assert f(P, P, P, P, P, None, None, 256, 512, 1020, 1024, 512, 1e-5, LN, 0, gn.GN_BF16, None) == gn.GN_ERR_SHAPE
-    assert f(P, P, P, P, P, None, None, 256, 512, 1024, 1000, 512, 1e-5, LN, 0, gn.GN_BF16, None) == gn.GN_ERR_SHAPE
-    assert f(None, P, P, P, P, None, None, 256, 512, 1024, 1024, 512, 1e-5, LN, 0, gn.GN_BF16, None) == gn.GN_ERR_NULL
-    assert f(P, P, None, P, P, None, None, 256, 512, 1024, 1024, 512, 1e-5, LN, 0, gn.GN_BF16, None) == gn.GN_ERR_NULL
-    assert f(P + 8, P, P, P, P, None, None, 256, 512, 1024, 1024, 512, 1e-5, LN, 0, gn.GN_BF16,
+    assert f(P, P, P, P, P, P, P, 256, 512, 1020, 1024, 512, 1e-5, LN, 0, gn.GN_BF16, None) == gn.GN_ERR_SHAPE
+    assert f(P, P, P, P, P, P, P, 256, 512, 1024, 1000, 512, 1e-5, LN, 0, gn.GN_BF16, None) == gn.GN_ERR_SHAPE
+    assert f(None, P, P, P, P, P, P, 256, 512, 1024, 1024, 512, 1e-5, LN, 0, gn.GN_BF16, None) == gn.GN_ERR_NULL
+    assert f(P, P, None, P, P, P, P, 256, 512, 1024, 1024, 512, 1e-5, LN, 0, gn.GN_BF16, None) == gn.GN_ERR_NULL
+    assert f(P, P, P, P, P, None, P, 256, 512, 1024, 1024, 512, 1e-5, LN, 0, gn.GN_BF16, None) == gn.GN_ERR_NULL
+    assert f(P, P, P, P, P, P, None, 256, 512, 1024, 1024, 512, 1e-5, LN, 0, gn.GN_BF16, None) == gn.GN_ERR_NULL
+    assert f(P + 8, P, P, P, P, P, P, 256, 512, 1024, 1024, 512, 1e-5, LN, 0, gn.GN_BF16,
              None) == gn.GN_ERR_ALIGN
     # RMSNorm needs no c; empty inputs launch nothing
-    assert f(P, P, None, None, P, None, None, 0, 512, 1024, 1024, 512, 1e-5, RMS, 0, gn.GN_BF16, None) == gn.GN_OK
+    assert f(P, P, None, None, P, None, P, 0, 512, 1024, 1024, 512, 1e-5, RMS, 0, gn.GN_BF16, None) == gn.GN_OK
     p = gn.gn_norm_linear_prepare
     assert p(None, None, None, None, P, P, P, 8, 64, LN, 0, gn.GN_BF16, None) == gn.GN_ERR_NULL
     assert p(P, None, None, None, P, None, P, 8, 64, LN, 0, gn.GN_BF16, None) == gn.GN_ERR_NULL

@@ -303,12 +303,12 @@ def norm_linear_fwd(x, Wf, c, d, eps=1e-5, norm="ln", epilogue="none", save_stat
     M, K = x.shape
     N = Wf.shape[0]
     y = torch.empty((M, N), dtype=x.dtype, device=x.device)
-    mk = (lambda: torch.empty(M, dtype=torch.float32, device=x.device)) if save_stats else (lambda: None)
-    mu, rs = mk(), mk()
+    mu = torch.empty(M, dtype=torch.float32, device=x.device)  # the kernels need both
+    rs = torch.empty(M, dtype=torch.float32, device=x.device)
     check(gn_norm_linear_fwd(_ptr(x), _ptr(Wf), _ptr(c), _ptr(d), _ptr(y), _ptr(mu), _ptr(rs), M, N, K,
                              x.stride(0), y.stride(0), eps, _norm(norm), _epi(epilogue), _dt(x),
                              _stream(stream)), "gn_norm_linear_fwd")
-    return y, mu, rs
+    return (y, mu, rs) if save_stats else (y, None, None)
 
 
 def device_error(clear: bool = False) -> int:

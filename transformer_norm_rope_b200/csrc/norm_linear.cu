@@ -42,7 +42,11 @@ namespace {
 #ifndef GN_NL_BK
 #define GN_NL_BK 64
 #endif
-constexpr int kUM = 128, kBN = 256, kBK = GN_NL_BK, kUK = 16;  // instruction M, tile N, tile K, instruction K
+#ifndef GN_NL_BN
+#define GN_NL_BN 256
+#endif
+constexpr int kUM = 128, kBN = GN_NL_BN, kBK = GN_NL_BK, kUK = 16;  // instruction M, tile N, tile K, instruction K
+constexpr int kAccCols = 256;  // tensor-memory columns between the two accumulators
 constexpr uint32_t kLine = kBK * 2;  // bytes of one tile row: 64 (BK 32, 64-byte swizzle) or 128
 constexpr int kChunks = kLine / 16;  // 16-byte chunks per tile row
 constexpr uint32_t kBBytes = kBN * kLine;
@@ -54,11 +58,13 @@ constexpr uint32_t kBBytes = kBN * kLine;
 template <int MH>
 struct Tile {
   static constexpr int BM = kUM * MH;
-  static constexpr int Stages = (MH == 1 ? 4 : 3) * (128 / kLine) + (kLine == 64 && MH == 2 ? 1 : 0);
+  // as many stages as fit in 227 KiB next to the barriers and column terms (at most 8)
+  static constexpr int StagesFit = (int)((232448 - 1024 - 256 - 2 * kBN * 4) / (BM * kLine + kBN * kLine));
+  static constexpr int Stages = StagesFit > 8 ? 8 : StagesFit;
   static constexpr int Threads = 64 + 128 * MH;  // producer, MMA, 4*MH statistics/epilogue warps
   static constexpr uint32_t ABytes = BM * kLine;
   static constexpr uint32_t StageBytes = ABytes + kBBytes;
-  static constexpr uint32_t TmemCols = kBN * MH;  // fp32 accumulators: one column per output column
+  static constexpr uint32_t TmemCols = MH == 1 ? (kBN <= 128 ? 128 : 256) : 512;  // power of two >= kAccCols*(MH-1)+kBN
   static constexpr size_t Smem = 1024 /* alignment slack */ + (size_t)Stages * StageBytes + 256 + 2 * kBN * 4;
 };
 
@@ -253,7 +259,7 @@ __global__ void __launch_bounds__(Tile<MH>::Threads, 1)
         for (int k = 0; k < kBK / kUK; ++k)  // +32 bytes along K inside the swizzled rows
 #pragma unroll
           for (int h = 0; h < MH; ++h)  // rows 128h.. of the A tile start 128 * kLine bytes further
-            umma_bf16(tmem + (uint32_t)(kBN * h), ad + (uint64_t)(2 * k + 8 * kLine * h), bd + (uint64_t)(2 * k),
+            umma_bf16(tmem + (uint32_t)(kAccCols * h), ad + (uint64_t)(2 * k + 8 * kLine * h), bd + (uint64_t)(2 * k),
                       (kb | k) != 0);
         umma_commit(&empty[s]);
       }
@@ -364,7 +370,7 @@ __global__ void __launch_bounds__(Tile<MH>::Threads, 1)
         const int col0 = n0 + 32 * j;
         if (col0 >= a.N) break;  // uniform over the warp
         float v[32];
-        tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(kBN * h + 32 * j), v);
+        tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(kAccCols * h + 32 * j), v);
         const bool whole = col0 + 32 <= a.N;
         float o[32];
 #pragma unroll
@@ -403,6 +409,297 @@ __global__ void __launch_bounds__(Tile<MH>::Threads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, TL::TmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- pair-of-SMs forward kernel
+// The same computation on a pair of CTAs on two SMs (a cluster of 2) that share each MMA: the
+// leader CTA issues tcgen05.mma.cta_group::2 with M = 256 (rows 0-127 from its own shared memory,
+// 128-255 from its peer's) and N = 256 (columns 0-127 of the B tile from the leader, 128-255
+// from the peer), twice per k-step for a 256 x 512 pair tile. Each SM then loads 16 KiB of x and
+// 32 KiB of W per 8.4 MFLOP (the single-SM 256 x 256 tile loads 64 KiB), and each SM's tensor
+// memory holds its own 128 rows x 512 columns. Both CTAs' TMA loads count on the leader's `full`
+// barrier; the MMA commits arrive on both CTAs' `empty` and accumulator barriers. The row
+// statistics come from norm_stats_kernel, run just before: reading them from the x tiles here
+// would need a signal from the leader to the peer on every stage, and a remote arrive on the
+// pipeline's critical path cost more than the whole pre-pass (measured on B200).
+constexpr int kPairN = 512;            // output columns of a pair tile
+constexpr int kPairStages = 4;         // 48 KiB per stage and SM
+constexpr uint32_t kPairABytes = kUM * kLine;           // 16 KiB: this CTA's 128 rows
+constexpr uint32_t kPairBBytes = 2 * 128 * kLine;       // 32 KiB: this CTA's 2 x 128 B rows
+constexpr uint32_t kPairStageBytes = kPairABytes + kPairBBytes;
+constexpr int kPairThreads = 320;      // producer, MMA, 8 statistics/epilogue warps
+constexpr size_t kPairSmem = 1024 + (size_t)kPairStages * kPairStageBytes + 256 + 2 * kPairN * 4;
+// instruction descriptor: as kIdesc with M = 256 (the pair)
+constexpr uint32_t kIdescPair = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) |
+                                ((uint32_t)(256 >> 4) << 24);
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// shared::cluster address of the same shared-memory offset in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// TMA load into this CTA's shared memory whose completion counts on an mbarrier of either CTA
+// of the pair (here: the leader's)
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, int x, int y, uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cluster)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* slot, uint32_t ncols) {  // whole warp, both CTAs
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(slot)), "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {  // whole warp, both CTAs
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(kIdescPair), "r"(accumulate)
+      : "memory");
+}
+
+// arrive once on the barrier at this offset in both CTAs when the issued MMAs have completed
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
+  const uint16_t mask = 0x3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_addr(bar)),
+      "h"(mask)
+      : "memory");
+}
+
+template <int NORM, int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
+    norm_linear_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                            const NlArgs a) {
+  constexpr int kPrefetch = 2 * kPairStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* tail = smem + kPairStages * kPairStageBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(tail);   // leader: both CTAs' tiles landed
+  uint64_t* empty = full + kPairStages;                   // the pair's MMAs done with the stage
+  uint64_t* accf = empty + kPairStages;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(accf + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+  float* col_c = reinterpret_cast<float*>(tail + 256);
+  float* col_d = col_c + kPairN;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int n0 = (blockIdx.x >> 1) * kPairN;         // the pair's first output column
+  const int m0 = blockIdx.y * 256 + kUM * (int)rank;  // this CTA's first row
+  const int nk = (a.K + kBK - 1) / kBK;
+  auto A = [&](int s) { return smem + s * kPairStageBytes; };
+  auto B = [&](int s) { return smem + s * kPairStageBytes + kPairABytes; };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPairStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accf, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 1) tmem_alloc_pair(tslot, 512);
+  tc_fence_before();
+  cluster_sync_all();  // both CTAs' barriers exist before any load counts on them
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      uint32_t lastph = 0, used = 0;
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % kPairStages;
+        const uint32_t ph = (uint32_t)(kb / kPairStages) & 1u;
+        if (kb >= kPairStages && !mbar_wait(&empty[s], ph ^ 1u, a.err)) {
+          *abort_flag = 1;
+          break;
+        }
+        if (*abort_flag) break;
+        const uint32_t bar = cluster_addr(&full[s], 0);
+        if (leader) mbar_expect_tx(&full[s], 2 * kPairStageBytes);  // both CTAs' bytes
+        if (kb + kPrefetch < nk) tma_prefetch_2d(&tmA, (kb + kPrefetch) * kBK, m0);
+        tma_load_2d_pair(A(s), &tmA, kb * kBK, m0, bar);
+        tma_load_2d_pair(B(s), &tmB, kb * kBK, n0 + 128 * (int)rank, bar);
+        tma_load_2d_pair(B(s) + 128 * kLine, &tmB, kb * kBK, n0 + 256 + 128 * (int)rank, bar);
+        used |= 1u << s;
+        lastph = (lastph & ~(1u << s)) | (ph << s);
+      }
+      // the leader's barriers count both CTAs' copies: every copy issued has landed once they
+      // complete (bounded waits)
+      if (leader)
+        for (int s = 0; s < kPairStages; ++s)
+          if (used & (1u << s)) (void)mbar_wait(&full[s], (lastph >> s) & 1u, a.err);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (leader && lane == 0) {
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % kPairStages;
+        const uint32_t ph = (uint32_t)(kb / kPairStages) & 1u;
+        if (!mbar_wait(&full[s], ph, a.err) || *abort_flag) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t ad = tile_desc(A(s)), bd = tile_desc(B(s));
+#pragma unroll
+        for (int k = 0; k < kBK / kUK; ++k)
+#pragma unroll
+          for (int j = 0; j < 2; ++j)  // B rows 128j.. of each CTA's tile: columns 256j.. of the pair
+            umma_bf16_pair(tmem + (uint32_t)(kAccCols * j), ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k + 8 * kLine * j),
+                           (kb | k) != 0);
+        umma_commit_pair(&empty[s]);
+      }
+      umma_commit_pair(accf);  // also after an abort: both epilogues wait for the work in flight
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;          // tensor-memory lane quadrant
+    const int j = (warp - 2) >> 2;   // accumulator (512 columns = 2 x 256) this warp drains
+    const int r = 32 * q + lane;     // row of this CTA's 128
+    const int m = m0 + r;
+    for (int i = threadIdx.x - 64; i < kPairN; i += 256) {
+      const int n = n0 + i;
+      col_c[i] = (NORM == GN_NORM_LN && n < a.N) ? a.c[n] : 0.0f;
+      col_d[i] = (a.d && n < a.N) ? a.d[n] : 0.0f;
+    }
+    const float mu = (NORM == GN_NORM_LN && m < a.M) ? __ldg(a.mean + m) : 0.0f;
+    const float rs = m < a.M ? __ldg(a.rstd + m) : 0.0f;
+    asm volatile("bar.sync 1, 256;" ::: "memory");  // column terms in place
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(accf, 0, a.err)) && !*abort_flag;
+    tc_fence_after();
+    if (ok) {
+      const float nsm = -rs * mu;
+      __nv_bfloat16* yrow = a.y + (int64_t)m * a.ldy;
+      for (int cb = 0; cb < 256 / 32; ++cb) {
+        const int lc = 256 * j + 32 * cb;  // column of the pair tile
+        const int col0 = n0 + lc;
+        if (col0 >= a.N) break;  // uniform over the warp
+        float v[32];
+        tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(kAccCols * j + 32 * cb), v);
+        const bool whole = col0 + 32 <= a.N;
+        float o[32];
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+          const float4 c4 = *reinterpret_cast<const float4*>(col_c + lc + i);
+          const float4 d4 = *reinterpret_cast<const float4*>(col_d + lc + i);
+          o[i + 0] = nl_act<EPI>(fmaf(rs, v[i + 0], fmaf(nsm, c4.x, d4.x)));
+          o[i + 1] = nl_act<EPI>(fmaf(rs, v[i + 1], fmaf(nsm, c4.y, d4.y)));
+          o[i + 2] = nl_act<EPI>(fmaf(rs, v[i + 2], fmaf(nsm, c4.z, d4.z)));
+          o[i + 3] = nl_act<EPI>(fmaf(rs, v[i + 3], fmaf(nsm, c4.w, d4.w)));
+        }
+        if (m < a.M) {
+          if (whole) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+              const float f8[8] = {o[i], o[i + 1], o[i + 2], o[i + 3], o[i + 4], o[i + 5], o[i + 6], o[i + 7]};
+              st_stream(yrow + col0 + i, Vec<__nv_bfloat16>::pack(f8));
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (col0 + i < a.N) yrow[col0 + i] = __float2bfloat16_rn(o[i]);
+          }
+        }
+      }
+    }
+  }
+
+  // teardown: neither CTA leaves while the pair's MMAs may still touch its shared or tensor
+  // memory; then both free the pair's tensor memory
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- row statistics pre-pass
+// One warp per row of x [M, K] bf16: each lane folds its 16-byte vectors (lane, lane + 32, ...)
+// into (count, mean, M2) - per vector a two-pass mean and centred sum of squares of the 8
+// values, merged with Chan's update - then the lanes merge with xor shuffles (Chan's update
+// again) so every lane holds the row's statistics. RMSNorm needs only the sum of squares.
+// Writes mean (LayerNorm) and rstd = 1/sqrt(var + eps) (RMSNorm: 1/sqrt(mean(x^2) + eps)).
+template <int NORM>
+__global__ void __launch_bounds__(256) norm_stats_kernel(const __nv_bfloat16* __restrict__ x, int64_t ldx, int M, int K,
+                                                          float eps, float* __restrict__ mean, float* __restrict__ rstd) {
+  const int lane = threadIdx.x & 31;
+  const int64_t m = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (m >= M) return;
+  const __nv_bfloat16* row = x + m * ldx;
+  const int nv = K / 8;  // whole 16-byte vectors (K is a multiple of 8)
+  float cnt = 0.0f, mu = 0.0f, m2 = 0.0f;
+#pragma unroll 4
+  for (int v = lane; v < nv; v += 32) {
+    const uint4 u = ld_stream(row + (int64_t)v * 8);
+    float f[8];
+    Vec<__nv_bfloat16>::unpack(u, f);
+    if (NORM == GN_NORM_LN) {
+      float t = 0.0f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) t += f[e];
+      const float bm = t * 0.125f;
+      float q = 0.0f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) q = fmaf(f[e] - bm, f[e] - bm, q);
+      const float n = cnt + 8.0f, dlt = bm - mu;
+      mu = fmaf(dlt, 8.0f / n, mu);
+      m2 += q + dlt * dlt * (cnt * 8.0f / n);
+      cnt = n;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) m2 = fmaf(f[e], f[e], m2);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float c2 = __shfl_xor_sync(0xffffffffu, cnt, o);
+    const float mu2 = __shfl_xor_sync(0xffffffffu, mu, o);
+    const float q2 = __shfl_xor_sync(0xffffffffu, m2, o);
+    if (NORM == GN_NORM_LN) {
+      const float n = cnt + c2;
+      if (n > 0.0f) {
+        const float dlt = mu2 - mu;
+        m2 += q2 + dlt * dlt * (cnt * c2 / n);
+        mu = fmaf(dlt, c2 / n, mu);
+      }
+      cnt = n;
+    } else {
+      m2 += q2;
+    }
+  }
+  if (lane == 0) {
+    if (NORM == GN_NORM_LN) mean[m] = mu;
+    rstd[m] = rsqrtf(fmaf(m2, 1.0f / (float)K, eps));
   }
 }
 
@@ -503,8 +800,32 @@ bool set_smem_attr() {
   return true;
 }
 
+template <int NORM>
+void* pick_pair_epi(int epi) {
+  if (epi == GN_EPI_GELU_TANH) return (void*)norm_linear_pair_kernel<NORM, EPI_GELU_TANH>;
+  if (epi == GN_EPI_SILU) return (void*)norm_linear_pair_kernel<NORM, EPI_SILU>;
+  return (void*)norm_linear_pair_kernel<NORM, EPI_NONE>;
+}
+
+void* pick_pair(int norm, int epi) {
+  return norm == GN_NORM_LN ? pick_pair_epi<GN_NORM_LN>(epi) : pick_pair_epi<GN_NORM_RMS>(epi);
+}
+
+bool set_pair_smem_attr() {
+  const void* ks[] = {pick_pair(GN_NORM_LN, GN_EPI_NONE), pick_pair(GN_NORM_LN, GN_EPI_GELU_TANH),
+                      pick_pair(GN_NORM_LN, GN_EPI_SILU), pick_pair(GN_NORM_RMS, GN_EPI_NONE),
+                      pick_pair(GN_NORM_RMS, GN_EPI_GELU_TANH), pick_pair(GN_NORM_RMS, GN_EPI_SILU)};
+  for (const void* k : ks)
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPairSmem) != cudaSuccess)
+      return false;
+  return true;
+}
+
 #ifndef GN_NL_MH
 #define GN_NL_MH 2
+#endif
+#ifndef GN_NL_PAIR
+#define GN_NL_PAIR 1
 #endif
 
 }  // namespace
@@ -546,18 +867,22 @@ extern "C" gn_status gn_norm_linear_fwd(const void* x, const void* Wf, const flo
   if (M < 0 || N < 0 || K <= 0 || ldx < K || ldy < N || K % 8 || ldx % 8 || ldy % 8) return GN_ERR_SHAPE;
   if (M > (int64_t)65535 * kUM || N > INT32_MAX || K > INT32_MAX) return GN_ERR_SHAPE;
   if (M == 0 || N == 0) return GN_OK;
-  if (!x || !Wf || !y || (norm == GN_NORM_LN && !c)) return GN_ERR_NULL;
+  if (!x || !Wf || !y || !rstd || (norm == GN_NORM_LN && (!c || !mean))) return GN_ERR_NULL;
   if (!aligned16(x) || !aligned16(Wf) || !aligned16(y) || (c && !aligned16(c)) || (d && !aligned16(d)))
     return GN_ERR_ALIGN;
-  // two accumulators (256-row tiles) once there are more than 128 rows
+  // pairs of SMs sharing 256 x 512 tiles once there are more than 128 rows and 256 columns;
+  // one SM per 256 x 256 tile (two accumulators) for fewer columns; 128 x 256 for few rows
+  const bool pair = GN_NL_PAIR && M > kUM && N > kBN;
   const int mh = M > kUM ? GN_NL_MH : 1;
-  const int bm = kUM * mh;
+  const int bm = pair ? 2 * kUM : kUM * mh;
   CUtensorMap ta, tb;
-  if (!make_map(&ta, x, M, K, ldx, (uint32_t)bm) || !make_map(&tb, Wf, N, K, K, kBN)) return GN_ERR_CUDA;
-  void* kern = mh == 2 ? pick<2>(norm, epi) : pick<1>(norm, epi);
+  if (!make_map(&ta, x, M, K, ldx, pair ? (uint32_t)kUM : (uint32_t)bm) ||
+      !make_map(&tb, Wf, N, K, K, pair ? 128u : (uint32_t)kBN))
+    return GN_ERR_CUDA;
+  void* kern = pair ? pick_pair(norm, epi) : mh == 2 ? pick<2>(norm, epi) : pick<1>(norm, epi);
   static std::once_flag attr_once;
   static bool attr_ok = true;
-  std::call_once(attr_once, [] { attr_ok = set_smem_attr<1>() && set_smem_attr<2>(); });
+  std::call_once(attr_once, [] { attr_ok = set_smem_attr<1>() && set_smem_attr<2>() && set_pair_smem_attr(); });
   if (!attr_ok) return GN_ERR_CUDA;
   NlArgs a{};
   a.c = c, a.d = d;
@@ -568,10 +893,22 @@ extern "C" gn_status gn_norm_linear_fwd(const void* x, const void* Wf, const flo
   a.eps = eps;
   a.err = device_err_word();
   if (!a.err) return GN_ERR_CUDA;
-  const dim3 grid((unsigned)((N + kBN - 1) / kBN), (unsigned)((M + bm - 1) / bm));
+  if (pair) {  // the pair kernel reads the row statistics: compute them first
+    const unsigned sblocks = (unsigned)((M + 7) / 8);
+    if (norm == GN_NORM_LN)
+      norm_stats_kernel<GN_NORM_LN><<<sblocks, 256, 0, (cudaStream_t)stream>>>(
+          static_cast<const __nv_bfloat16*>(x), ldx, (int)M, (int)K, eps, mean, rstd);
+    else
+      norm_stats_kernel<GN_NORM_RMS><<<sblocks, 256, 0, (cudaStream_t)stream>>>(
+          static_cast<const __nv_bfloat16*>(x), ldx, (int)M, (int)K, eps, mean, rstd);
+    count_launches(1);
+    if (launch_status() != GN_OK) return GN_ERR_CUDA;
+  }
+  const dim3 grid(pair ? (unsigned)(2 * ((N + kPairN - 1) / kPairN)) : (unsigned)((N + kBN - 1) / kBN),
+                  (unsigned)((M + bm - 1) / bm));
   void* args[] = {&ta, &tb, &a};
-  const int threads = mh == 2 ? Tile<2>::Threads : Tile<1>::Threads;
-  const size_t smem = mh == 2 ? Tile<2>::Smem : Tile<1>::Smem;
+  const int threads = pair ? kPairThreads : mh == 2 ? Tile<2>::Threads : Tile<1>::Threads;
+  const size_t smem = pair ? kPairSmem : mh == 2 ? Tile<2>::Smem : Tile<1>::Smem;
   if (cudaLaunchKernel(kern, grid, dim3(threads), args, smem, (cudaStream_t)stream) != cudaSuccess)
     return GN_ERR_CUDA;
   count_launches(1);
