@@ -411,7 +411,7 @@ def norm_linear_measure(gn, torch, dev, scale, seed, reps=10):
     except Exception:  # noqa: BLE001
         peak, kind = 1590.0, "fallback"
     gn.check(0 if gn.device_error(clear=True) == 0 else gn.GN_ERR_CUDA, "norm_linear device error")
-    return {"workload": f"LayerNorm + linear {K}->{N} + SiLU, x[{M},{K}] bf16 (tcgen05, one launch)",
+    return {"workload": f"LayerNorm + linear {K}->{N} + SiLU, x[{M},{K}] bf16 (statistics pre-pass + tcgen05 GEMM on pairs of SMs)",
             "ms": round(t_f * 1e3, 4), "TFLOP_s": round(tf, 1),
             "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peak, "unit": "TFLOP/s",
                          "frac": round(tf / peak, 4), "peak_source": kind},
