@@ -420,6 +420,55 @@ def norm_linear_measure(gn, torch, dev, scale, seed, reps=10):
             "speedup_vs_unfused": round(t_u / t_f, 3)}
 
 
+def tiled_linear_measure(gn, torch, dev, scale, seed, reps=5):
+    """The token-chunked linear + SiLU (TiledLinear) on x[32768, 5120] and a 5120 x 5120 layer:
+    forward + backward time and the peak memory the step allocates beyond its inputs, for the
+    default chunk count (ceil(tokens / hidden) = 7), one chunk, and torch autograd keeping the
+    pre-activation (the layer TiledLinear replaces)."""
+    from transformer_norm_rope_b200 import tiled_linear as tl
+
+    M, N, K = max(256, int(32768 * scale)), 5120, 5120
+    d = wl.norm_linear(M, N, K, seed)
+    T = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)  # noqa
+    x, W, bias = T(d["x"]), T(d["W"]), T(d["bias"])
+    dy = torch.randn((M, N), device=dev).to(torch.bfloat16)
+    stream = torch.cuda.current_stream(dev)
+    Wf, dd = tl.prepare(W, bias)
+
+    def tiled(chunks):
+        def f():
+            tl.forward(x, Wf, dd, "silu", chunks)
+            tl.backward(x, Wf, dd, dy, "silu", chunks)
+        return f
+
+    def autograd():
+        xa, Wa, ba = x.detach().requires_grad_(), W.detach().requires_grad_(), bias.detach().requires_grad_()
+        torch.nn.functional.silu(torch.nn.functional.linear(xa, Wa, ba)).backward(dy)
+
+    def measure(fn):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize(dev)
+        base = torch.cuda.memory_allocated(dev)
+        torch.cuda.reset_peak_memory_stats(dev)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for a, b in ev:
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        peak = torch.cuda.max_memory_allocated(dev) - base
+        return statistics.median(a.elapsed_time(b) for a, b in ev), peak / 2**20
+
+    out = {"workload": f"linear {K}->{N} + SiLU forward + backward, x[{M},{K}] bf16",
+           "default_chunks": tl.default_chunks(M, K)}
+    for name, fn in (("tiled", tiled(None)), ("one_chunk", tiled(1)), ("torch_autograd", autograd)):
+        ms, mib = measure(fn)
+        out[name] = {"ms": round(ms, 3), "peak_extra_MiB": round(mib, 1)}
+    gn.check(0 if gn.device_error(clear=True) == 0 else gn.GN_ERR_CUDA, "tiled_linear device error")
+    return out
+
+
 def run_ours(args):
     import torch
 
@@ -498,6 +547,8 @@ def run_ours(args):
         del suite  # free the step's buffers first
         torch.cuda.empty_cache()
         out["next_norm_linear"] = norm_linear_measure(gn, torch, dev, args.scale, args.seed + rank)
+        torch.cuda.empty_cache()
+        out["next_tiled_linear"] = tiled_linear_measure(gn, torch, dev, args.scale, args.seed + rank)
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(host, z, kernels, budget_s=15.0)
     if rank == 0:

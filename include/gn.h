@@ -17,6 +17,9 @@
  *       (centre, biased variance, divide by sqrt(var + eps), times weight plus bias, GeLU).
  *   [J] "Janus-Pro-7B模型推理加速实战", section 4.1: LayerNorm fused with SiLU = x * sigmoid(x),
  *       and LayerNorm, the first linear projection and SiLU fused into one kernel.
+ *       - "内核三 TiledLinear": a linear layer run chunk by chunk along the tokens, the backward
+ *         recomputing each chunk instead of keeping its activations (gn_act_grad and
+ *         GN_NORM_NONE serve it).
  *   [Y] "HY-Motion 1.0性能优化从算法到硬件的全方位调优策略", section 3.1: LayerNorm merged with
  *       the matrix multiplication that follows it (no round trip of the normalized activations
  *       through memory).
@@ -76,8 +79,8 @@ typedef enum { GN_F32 = 0, GN_BF16 = 1 } gn_dtype;
 /* epilogue applied to z = normalized * weight (+ bias) before the store */
 typedef enum { GN_EPI_NONE = 0, GN_EPI_GELU_TANH = 1, GN_EPI_SILU = 2 } gn_epilogue;
 
-/* the normalization in front of the fused linear layer */
-typedef enum { GN_NORM_RMS = 0, GN_NORM_LN = 1 } gn_norm;
+/* the normalization in front of the fused linear layer (GN_NORM_NONE: a plain linear layer) */
+typedef enum { GN_NORM_RMS = 0, GN_NORM_LN = 1, GN_NORM_NONE = 2 } gn_norm;
 
 /* device error word bits */
 #define GN_DEVERR_WAIT_TIMEOUT 1u
@@ -213,6 +216,8 @@ gn_status gn_qknorm_rope_bwd_noalloc(const void* q, const void* k, const void* w
  * with the row statistics, which it accumulates from the same x tiles:
  *   y[m,n] = act( rstd_m (x Wf^T)[m,n] - rstd_m mean_m c[n] + d[n] ),
  *   c[n] = sum_k Wf[n,k],  d[n] = sum_k beta[k] W[n,k] + bias[n]   (RMSNorm: mean = 0, d = bias).
+ * GN_NORM_NONE: no normalization, y = act(x W^T + bias) (a plain linear layer on the tensor
+ * cores; g, beta, c, mean and rstd are not used).
  * bf16 only (GN_BF16; GN_F32 returns GN_ERR_UNSUPPORTED). */
 
 /* Builds Wf [N, K] (bf16, row n = output feature n, contiguous), c [N] fp32 (LayerNorm; may be
@@ -239,6 +244,16 @@ gn_status gn_norm_linear_fwd(const void* x, const void* Wf, const float* c, cons
                              float* mean, float* rstd, int64_t M, int64_t N, int64_t K, int64_t ldx,
                              int64_t ldy, float eps, gn_norm norm, gn_epilogue epi, gn_dtype dt,
                              void* stream);
+
+/* Gradient of the epilogue activation, elementwise over n elements: dz = dy * act'(z) (act as
+ * in the gn_epilogue values; GN_EPI_NONE gives dz = dy). z is the pre-activation, dy the
+ * gradient of act(z). The backward of a linear layer with an activation needs it before its two
+ * gradient products; the token-chunked linear layer ([H] "内核三 TiledLinear": the forward runs
+ * chunk by chunk, the backward recomputes each chunk's z instead of keeping it) calls it per
+ * chunk. z, dy, dz: contiguous, dt, 16-byte aligned; dz may alias z or dy (elementwise).
+ * Errors: GN_ERR_DTYPE, GN_ERR_SHAPE (n < 0), GN_ERR_NULL, GN_ERR_ALIGN, GN_ERR_CUDA. */
+gn_status gn_act_grad(const void* z, const void* dy, void* dz, int64_t n, gn_epilogue epi, gn_dtype dt,
+                      void* stream);
 
 /* ---------------------------------------------------------------- runtime queries
  * Number of kernels this process has launched through libgn (all devices, all threads). */

@@ -19,7 +19,7 @@ from . import build as _build
 
 F64, F32, BF16 = 0, 1, 2
 ACT_NONE, ACT_GELU_TANH, ACT_SILU = 0, 1, 2
-NORM_RMS, NORM_LN = 0, 1
+NORM_RMS, NORM_LN, NORM_NONE = 0, 1, 2
 _ACTS = {"none": ACT_NONE, "gelu_tanh": ACT_GELU_TANH, "silu": ACT_SILU}
 
 _lib = None
@@ -44,9 +44,10 @@ def _load():
         lib.oracle_qknorm_rope_bwd.argtypes = [vp, ci, vp, ci, vp, vp, ci, vp, ci, i64, i64, i64, i64, dbl, ci, vp, vp]
         lib.oracle_norm_linear.argtypes = [vp, ci, vp, vp, ci, vp, ci, vp, ci, i64, i64, i64, dbl, ci, ci, ci,
                                            vp, vp, vp]
+        lib.oracle_linear_act_bwd.argtypes = [vp, ci, vp, ci, vp, ci, vp, ci, i64, i64, i64, ci, vp, vp, vp]
         for f in ("oracle_rmsnorm_fwd", "oracle_rmsnorm_bwd", "oracle_layernorm_fwd",
                   "oracle_layernorm_bwd", "oracle_rope", "oracle_qknorm_rope_fwd",
-                  "oracle_qknorm_rope_bwd", "oracle_norm_linear"):
+                  "oracle_qknorm_rope_bwd", "oracle_norm_linear", "oracle_linear_act_bwd"):
             getattr(lib, f).restype = None
         _lib = lib
     return _lib
@@ -201,7 +202,21 @@ def norm_linear(x, g, beta, W, bias, eps, norm="ln", gemma=False, act="none"):
     y = np.empty((M, N))
     mu = np.empty(M)
     rs = np.empty(M)
+    code = {"ln": NORM_LN, "rms": NORM_RMS, "none": NORM_NONE}[norm]
     _load().oracle_norm_linear(_p(x), xd, _p(g), _p(beta if norm == "ln" else None), gd, _p(W), wd, _p(bias), bsd,
-                               M, N, K, eps, NORM_LN if norm == "ln" else NORM_RMS, int(gemma), _act(act),
-                               _p(y), _p(mu), _p(rs))
+                               M, N, K, eps, code, int(gemma), _act(act), _p(y), _p(mu), _p(rs))
     return y, mu, rs
+
+
+def linear_act_bwd(x, W, bias, dy, act="none"):
+    """Gradients of sum(dy * act(x W^T + bias)): dx[M,K], dW[N,K], dbias[N]."""
+    x, xd = _in(x)
+    W, wd = _in(W)
+    bias, bd = _in(bias)
+    dy, gd = _in(dy)
+    M, K = x.shape
+    N = W.shape[0]
+    dx, dW, db = np.empty((M, K)), np.empty((N, K)), np.empty(N)
+    _load().oracle_linear_act_bwd(_p(x), xd, _p(W), wd, _p(bias), bd, _p(dy), gd, M, N, K, _act(act), _p(dx),
+                                  _p(dW), _p(db))
+    return dx, dW, db

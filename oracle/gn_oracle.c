@@ -357,17 +357,19 @@ void oracle_norm_linear(const void* x, int x_dt, const void* g, const void* beta
   double* wt = scratch(N * K);
   if (norm == ORC_NORM_LN) {
     load_affine(g, beta, p_dt, K, gv, bv);
-  } else {
+  } else if (norm == ORC_NORM_RMS) {
     load_weight(g, p_dt, K, gemma, gv);
     for (int64_t k = 0; k < K; ++k) bv[k] = 0.0;
+  } else {  /* no normalization: xn = x */
+    for (int64_t k = 0; k < K; ++k) gv[k] = 1.0, bv[k] = 0.0;
   }
   rd_row(W, w_dt, 0, N * K, wt);
   for (int64_t m = 0; m < M; ++m) {
     rd_row(x, x_dt, m * K, K, row);
-    double mu = 0.0, s;
+    double mu = 0.0, s = 1.0;
     if (norm == ORC_NORM_LN)
       ln_row_stats(row, K, eps, &mu, &s);
-    else
+    else if (norm == ORC_NORM_RMS)
       s = rms_row_inv(row, K, eps);
     for (int64_t k = 0; k < K; ++k) xn[k] = (row[k] - mu) * s * gv[k] + bv[k];
     if (y)
@@ -384,4 +386,44 @@ void oracle_norm_linear(const void* x, int x_dt, const void* g, const void* beta
   free(row);
   free(bv);
   free(gv);
+}
+
+/* ---- Backward of the linear layer with an activation -----------------------------------------
+ * [H] "内核三 TiledLinear": the layer y = act(z), z = x W^T + bias runs chunk by chunk along the
+ * tokens and its backward recomputes each chunk; chunking changes no arithmetic of the result,
+ * so the oracle is the plain gradient: g = dy act'(z), dx = g W, dW = g^T x, dbias = sum_m g.
+ * x[M,K], W[N,K], dy[M,N]; dx[M*K], dW[N*K], db[N] may each be NULL. */
+void oracle_linear_act_bwd(const void* x, int x_dt, const void* W, int w_dt, const void* bias, int bias_dt,
+                           const void* dy, int dy_dt, int64_t M, int64_t N, int64_t K, int act, double* dx,
+                           double* dW, double* db) {
+  double* wt = scratch(N * K);
+  double* row = scratch(K);
+  double* gr = scratch(N);
+  rd_row(W, w_dt, 0, N * K, wt);
+  if (dW)
+    for (int64_t i = 0; i < N * K; ++i) dW[i] = 0.0;
+  if (db)
+    for (int64_t n = 0; n < N; ++n) db[n] = 0.0;
+  for (int64_t m = 0; m < M; ++m) {
+    rd_row(x, x_dt, m * K, K, row);
+    for (int64_t n = 0; n < N; ++n) {
+      double z = bias ? rd(bias, bias_dt, n) : 0.0;
+      for (int64_t k = 0; k < K; ++k) z += row[k] * wt[n * K + k];
+      gr[n] = rd(dy, dy_dt, m * N + n) * oracle_act_grad(act, z);
+    }
+    if (dx)
+      for (int64_t k = 0; k < K; ++k) {
+        double acc = 0.0;
+        for (int64_t n = 0; n < N; ++n) acc += gr[n] * wt[n * K + k];
+        dx[m * K + k] = acc;
+      }
+    if (dW)
+      for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) dW[n * K + k] += gr[n] * row[k];
+    if (db)
+      for (int64_t n = 0; n < N; ++n) db[n] += gr[n];
+  }
+  free(gr);
+  free(row);
+  free(wt);
 }

@@ -18,6 +18,8 @@
  *   [L]  "LLM层的优化算子" (optimized kernels for LLM layers), section "编写定制融合算子"
  *        (fused LayerNorm + GeLU example: centre, biased variance, divide by sqrt(var+eps),
  *        times weight plus bias, tanh-GeLU with constant 0.79788456 and cubic 0.044715).
+ *        section "内核三 TiledLinear" (linear layer run chunk by chunk along the tokens, the
+ *        backward recomputing each chunk).
  *   [J]  "Janus-Pro-7B模型推理加速实战", section 4.1 (fused LayerNorm + linear + SiLU,
  *        SiLU = x * sigmoid(x)).
  *   [Y]  "HY-Motion 1.0性能优化从算法到硬件的全方位调优策略", section 3.1 (LayerNorm merged
@@ -88,8 +90,8 @@ void oracle_qknorm_rope_bwd(const void* x, int x_dt, const void* w, int w_dt, co
                             int64_t S, int64_t H, int64_t D, double eps, int gemma, double* dx,
                             double* dw);
 
-/* which normalization precedes the linear layer */
-enum { ORC_NORM_RMS = 0, ORC_NORM_LN = 1 };
+/* which normalization precedes the linear layer (ORC_NORM_NONE: none, a plain linear layer) */
+enum { ORC_NORM_RMS = 0, ORC_NORM_LN = 1, ORC_NORM_NONE = 2 };
 
 /* Normalization (RMSNorm with weight g and optional gemma offset, or LayerNorm with weight g and
  * bias beta; no activation) followed by the linear layer y = act(xn W^T + bias): x[M,K],
@@ -99,6 +101,12 @@ void oracle_norm_linear(const void* x, int x_dt, const void* g, const void* beta
                         const void* W, int w_dt, const void* bias, int bias_dt, int64_t M,
                         int64_t N, int64_t K, double eps, int norm, int gemma, int act, double* y,
                         double* mean, double* rstd);
+
+/* Backward of y = act(x W^T + bias): g = dy act'(z); dx[M*K] = g W; dW[N*K] = g^T x;
+ * db[N] = sum over rows of g (each output may be NULL; dW and db are overwritten). */
+void oracle_linear_act_bwd(const void* x, int x_dt, const void* W, int w_dt, const void* bias, int bias_dt,
+                           const void* dy, int dy_dt, int64_t M, int64_t N, int64_t K, int act, double* dx,
+                           double* dW, double* db);
 
 #ifdef __cplusplus
 }

@@ -40,6 +40,9 @@ MUTANTS = {
     "norm_linear_transposed_weight": ("acc += xn[k] * wt[n * K + k];", "acc += xn[k] * wt[k * N + n];"),
     "norm_linear_drops_bias": ("double acc = bias ? rd(bias, bias_dt, n) : 0.0;", "double acc = 0.0;"),
     "norm_linear_uncentred": ("xn[k] = (row[k] - mu) * s * gv[k] + bv[k];", "xn[k] = row[k] * s * gv[k] + bv[k];"),
+    "linear_bwd_drops_act_grad": ("gr[n] = rd(dy, dy_dt, m * N + n) * oracle_act_grad(act, z);",
+                                  "gr[n] = rd(dy, dy_dt, m * N + n);"),
+    "linear_bwd_dx_from_wrong_column": ("acc += gr[n] * wt[n * K + k];", "acc += gr[n] * wt[n * K + (K - 1 - k)];"),
 }
 
 

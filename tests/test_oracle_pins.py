@@ -483,3 +483,35 @@ def test_norm_linear_with_identity_weight_is_the_norm():
     y, _, _ = oracle.norm_linear(x, g, beta, W, None, 1e-6, "ln")
     xn = oracle.layernorm_fwd(x, g, beta, 1e-6)[0]
     np.testing.assert_array_equal(y, xn[:, [5, 0, K - 1]])
+
+
+# ---- the linear layer with an activation, forward and backward (Helios kernels article,
+# section "内核三 TiledLinear": chunking along the tokens changes none of these values) ----------
+
+
+@pytest.mark.parametrize("act", ["none", "silu", "gelu_tanh"])
+def test_linear_act_matches_torch_fp64(act):
+    M, N, K = 6, 5, 7
+    x, W, b = rng.standard_normal((M, K)), rng.standard_normal((N, K)), rng.standard_normal(N)
+    dy = rng.standard_normal((M, N))
+    xt, Wt, bt = t64(x).requires_grad_(), t64(W).requires_grad_(), t64(b).requires_grad_()
+    z = F.linear(xt, Wt, bt)
+    y = {"none": lambda v: v, "silu": F.silu, "gelu_tanh": lambda v: F.gelu(v, approximate="tanh")}[act](z)
+    (y * t64(dy)).sum().backward()
+    yo, _, _ = oracle.norm_linear(x, None, None, W, b, 0.0, "none", act=act)
+    np.testing.assert_allclose(yo, y.detach().numpy(), rtol=1e-12, atol=1e-12)
+    dx, dW, db = oracle.linear_act_bwd(x, W, b, dy, act)
+    np.testing.assert_allclose(dx, xt.grad.numpy(), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(dW, Wt.grad.numpy(), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(db, bt.grad.numpy(), rtol=1e-11, atol=1e-12)
+
+
+def test_linear_act_bwd_finite_differences():
+    M, N, K = 3, 4, 5
+    x, W, b = rng.standard_normal((M, K)), rng.standard_normal((N, K)), rng.standard_normal(N)
+    dy = rng.standard_normal((M, N))
+    loss = lambda: float((oracle.norm_linear(x, None, None, W, b, 0.0, "none", act="silu")[0] * dy).sum())
+    dx, dW, db = oracle.linear_act_bwd(x, W, b, dy, "silu")
+    np.testing.assert_allclose(dx, _fd_grad(loss, x), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dW, _fd_grad(loss, W), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(db, _fd_grad(loss, b), rtol=1e-6, atol=1e-8)

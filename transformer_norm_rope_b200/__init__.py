@@ -24,7 +24,7 @@ GN_OK, GN_ERR_NULL, GN_ERR_SHAPE, GN_ERR_ALIGN, GN_ERR_DTYPE, GN_ERR_WORKSPACE, 
     GN_ERR_UNSUPPORTED, GN_ERR_CUDA = range(8)
 GN_F32, GN_BF16 = 0, 1
 GN_EPI_NONE, GN_EPI_GELU_TANH, GN_EPI_SILU = 0, 1, 2
-GN_NORM_RMS, GN_NORM_LN = 0, 1
+GN_NORM_RMS, GN_NORM_LN, GN_NORM_NONE = 0, 1, 2
 GN_DEVERR_WAIT_TIMEOUT = 1
 EPILOGUES = {"none": GN_EPI_NONE, "gelu_tanh": GN_EPI_GELU_TANH, "silu": GN_EPI_SILU}
 
@@ -54,6 +54,7 @@ SIGNATURES = {
     "gn_norm_linear_prepare": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _int, _int, _int, _vp]),
     "gn_norm_linear_fwd": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _f32, _int,
                                  _int, _int, _vp]),
+    "gn_act_grad": (_st, [_vp, _vp, _vp, _i64, _int, _int, _vp]),
     "gn_launch_count": (C.c_uint64, []),
     "gn_device_error": (_st, [C.POINTER(C.c_uint), _int]),
     "gn_selftest_wait_timeout": (_st, [C.c_uint32, _vp]),
@@ -280,7 +281,7 @@ def qknorm_rope_bwd(q, k, wq, wk, cos, sin, inv_rms_q, inv_rms_k, dq_out, dk_out
 
 
 def _norm(norm) -> int:
-    return {"rms": GN_NORM_RMS, "ln": GN_NORM_LN}[norm] if isinstance(norm, str) else int(norm)
+    return {"rms": GN_NORM_RMS, "ln": GN_NORM_LN, "none": GN_NORM_NONE}[norm] if isinstance(norm, str) else int(norm)
 
 
 def norm_linear_prepare(W, g=None, beta=None, bias=None, norm="ln", gemma=False, stream=None):
@@ -296,19 +297,33 @@ def norm_linear_prepare(W, g=None, beta=None, bias=None, norm="ln", gemma=False,
     return Wf, c, d
 
 
-def norm_linear_fwd(x, Wf, c, d, eps=1e-5, norm="ln", epilogue="none", save_stats=True, stream=None):
+def norm_linear_fwd(x, Wf, c, d, eps=1e-5, norm="ln", epilogue="none", save_stats=True, out=None, stream=None):
     """y [M, N] = act(norm(x) W^T + bias) from x [M, K] and the prepared (Wf, c, d):
-    -> (y, mean, rstd) (statistics fp32 [M], or None)."""
+    -> (y, mean, rstd) (statistics fp32 [M], or None). `out` may give y (rows of a larger
+    tensor included: its row stride is passed on)."""
     torch = _torch()
     M, K = x.shape
     N = Wf.shape[0]
-    y = torch.empty((M, N), dtype=x.dtype, device=x.device)
-    mu = torch.empty(M, dtype=torch.float32, device=x.device)  # the kernels need both
-    rs = torch.empty(M, dtype=torch.float32, device=x.device)
+    y = torch.empty((M, N), dtype=x.dtype, device=x.device) if out is None else out
+    plain = _norm(norm) == GN_NORM_NONE
+    mu = None if plain else torch.empty(M, dtype=torch.float32, device=x.device)  # the kernels need both
+    rs = None if plain else torch.empty(M, dtype=torch.float32, device=x.device)
     check(gn_norm_linear_fwd(_ptr(x), _ptr(Wf), _ptr(c), _ptr(d), _ptr(y), _ptr(mu), _ptr(rs), M, N, K,
                              x.stride(0), y.stride(0), eps, _norm(norm), _epi(epilogue), _dt(x),
                              _stream(stream)), "gn_norm_linear_fwd")
     return (y, mu, rs) if save_stats else (y, None, None)
+
+
+def act_grad(z, dy, epilogue="silu", out=None, stream=None):
+    """dz = dy * act'(z), elementwise (contiguous tensors of one dtype)."""
+    dz = torch_empty_like(dy) if out is None else out
+    check(gn_act_grad(_ptr(z), _ptr(dy), _ptr(dz), dy.numel(), _epi(epilogue), _dt(dy), _stream(stream)),
+          "gn_act_grad")
+    return dz
+
+
+def torch_empty_like(t):
+    return _torch().empty_like(t)
 
 
 def device_error(clear: bool = False) -> int:

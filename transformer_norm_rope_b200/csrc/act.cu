@@ -1,0 +1,65 @@
+// act.cu - gradient of the epilogue activation, elementwise: dz = dy * act'(z).
+//
+// The backward of a linear layer with an activation (y = act(z), z = x W^T + b) needs dz before
+// its two gradient products; the token-chunked linear layer (TiledLinear, Helios kernels
+// article, section "内核三 TiledLinear") recomputes z chunk by chunk and calls this on each
+// chunk. The derivative is the one the normalization kernels' backward uses (epi_grad: the
+// tanh-GeLU with the same constants, SiLU). 16-byte vectors per thread, grid-stride; a ragged
+// tail of fewer than one vector is handled element by element.
+#include "gn_common.cuh"
+#include "gn_host.h"
+
+namespace gn {
+namespace {
+
+template <typename T, int EPI>
+__global__ void __launch_bounds__(256) act_grad_kernel(const T* __restrict__ z, const T* __restrict__ dy,
+                                                       T* __restrict__ dz, int64_t n) {
+  constexpr int E = Vec<T>::N;
+  constexpr bool FAST = fast_math_for<T>();
+  const int64_t nvec = n / E;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < nvec; v += stride) {
+    float fz[E], fg[E];
+    Vec<T>::unpack(ld_stream(z + v * E), fz);
+    Vec<T>::unpack(ld_stream(dy + v * E), fg);
+#pragma unroll
+    for (int e = 0; e < E; ++e) fg[e] *= epi_grad<EPI, FAST>(fz[e]);
+    st_stream(dz + v * E, Vec<T>::pack(fg));
+  }
+  // the ragged tail, by the first threads of the grid
+  const int64_t t = nvec * E + (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t < n) Vec<T>::store1(dz + t, Vec<T>::load1(dy + t) * epi_grad<EPI, FAST>(Vec<T>::load1(z + t)));
+}
+
+template <typename T>
+void* pick(int epi) {
+  if (epi == GN_EPI_GELU_TANH) return (void*)act_grad_kernel<T, EPI_GELU_TANH>;
+  if (epi == GN_EPI_SILU) return (void*)act_grad_kernel<T, EPI_SILU>;
+  return (void*)act_grad_kernel<T, EPI_NONE>;
+}
+
+}  // namespace
+}  // namespace gn
+
+using namespace gn;
+
+extern "C" gn_status gn_act_grad(const void* z, const void* dy, void* dz, int64_t n, gn_epilogue epi, gn_dtype dt,
+                                 void* stream) {
+  if (!dt_ok(dt) || !epi_ok(epi)) return GN_ERR_DTYPE;
+  if (n < 0) return GN_ERR_SHAPE;
+  if (n == 0) return GN_OK;
+  if (!z || !dy || !dz) return GN_ERR_NULL;
+  if (!aligned16(z) || !aligned16(dy) || !aligned16(dz)) return GN_ERR_ALIGN;
+  void* kern = dt == GN_BF16 ? pick<__nv_bfloat16>(epi) : pick<float>(epi);
+  const int64_t nvec = n / (int64_t)(16 / dt_size(dt));
+  int64_t blocks = (nvec + 255) / 256;
+  const int64_t cap = (int64_t)(sm_count() > 0 ? sm_count() : 148) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  void* args[] = {&z, &dy, &dz, &n};
+  if (cudaLaunchKernel(kern, dim3((unsigned)blocks), dim3(256), args, 0, (cudaStream_t)stream) != cudaSuccess)
+    return GN_ERR_CUDA;
+  count_launches(1);
+  return launch_status();
+}

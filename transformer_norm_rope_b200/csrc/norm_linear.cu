@@ -206,7 +206,7 @@ __global__ void __launch_bounds__(Tile<MH>::Threads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + 4 * MH);  // the MMA commit and the statistics warps
+      mbar_init(&empty[s], NORM == GN_NORM_NONE ? 1 : 1 + 4 * MH);  // the MMA commit and the statistics warps
     }
     mbar_init(accf, 1);
     *abort_flag = 0;
@@ -285,7 +285,7 @@ __global__ void __launch_bounds__(Tile<MH>::Threads, 1)
     asm volatile("bar.sync 1, %0;" ::"r"(128 * MH) : "memory");  // the statistics warps only
     float cnt = 0.0f, mean = 0.0f, m2 = 0.0f;
     bool ok = true;
-    for (int kb = 0; kb < nk; ++kb) {
+    for (int kb = 0; kb < (NORM == GN_NORM_NONE ? 0 : nk); ++kb) {  // no statistics without a norm
       const int s = kb % kStages;
       const uint32_t ph = (uint32_t)(kb / kStages) & 1u;
       ok = __all_sync(0xffffffffu, mbar_wait(&full[s], ph, a.err)) && !*abort_flag;
@@ -360,8 +360,10 @@ __global__ void __launch_bounds__(Tile<MH>::Threads, 1)
       if (NORM == GN_NORM_LN) {
         mu = mean;
         rs = rsqrtf(fmaf(m2, inv_k, a.eps));  // biased variance M2 / K
-      } else {
+      } else if (NORM == GN_NORM_RMS) {
         rs = rsqrtf(fmaf(m2, inv_k, a.eps));
+      } else {
+        rs = 1.0f;  // plain linear layer
       }
       const float nsm = -rs * mu;
       const int m = m0 + r;
@@ -396,7 +398,7 @@ __global__ void __launch_bounds__(Tile<MH>::Threads, 1)
           }
         }
       }
-      if (blockIdx.x == 0 && m < a.M) {
+      if (NORM != GN_NORM_NONE && blockIdx.x == 0 && m < a.M) {
         if (a.mean) a.mean[m] = mu;
         if (a.rstd) a.rstd[m] = rs;
       }
@@ -591,7 +593,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       col_d[i] = (a.d && n < a.N) ? a.d[n] : 0.0f;
     }
     const float mu = (NORM == GN_NORM_LN && m < a.M) ? __ldg(a.mean + m) : 0.0f;
-    const float rs = m < a.M ? __ldg(a.rstd + m) : 0.0f;
+    const float rs = NORM == GN_NORM_NONE ? 1.0f : m < a.M ? __ldg(a.rstd + m) : 0.0f;
     asm volatile("bar.sync 1, 256;" ::: "memory");  // column terms in place
     const bool ok = __all_sync(0xffffffffu, mbar_wait(accf, 0, a.err)) && !*abort_flag;
     tc_fence_after();
@@ -721,7 +723,8 @@ __global__ void __launch_bounds__(256) norm_linear_prepare_kernel(const __nv_bfl
   float cs = 0.0f, ds = 0.0f;
   for (int k = t; k < K; k += 256) {
     const float w = __bfloat162float(wrow[k]);
-    const float gk = (g ? __bfloat162float(g[k]) : 1.0f) + (NORM == GN_NORM_RMS && gemma ? 1.0f : 0.0f);
+    const float gk = NORM == GN_NORM_NONE ? 1.0f
+                                          : (g ? __bfloat162float(g[k]) : 1.0f) + (NORM == GN_NORM_RMS && gemma ? 1.0f : 0.0f);
     const __nv_bfloat16 f = __float2bfloat16_rn(gk * w);
     frow[k] = f;
     cs += __bfloat162float(f);
@@ -786,17 +789,18 @@ void* pick_epi(int epi) {
 
 template <int MH>
 void* pick(int norm, int epi) {
-  return norm == GN_NORM_LN ? pick_epi<MH, GN_NORM_LN>(epi) : pick_epi<MH, GN_NORM_RMS>(epi);
+  return norm == GN_NORM_LN    ? pick_epi<MH, GN_NORM_LN>(epi)
+         : norm == GN_NORM_RMS ? pick_epi<MH, GN_NORM_RMS>(epi)
+                               : pick_epi<MH, GN_NORM_NONE>(epi);
 }
 
 template <int MH>
 bool set_smem_attr() {
-  const void* ks[] = {pick<MH>(GN_NORM_LN, GN_EPI_NONE), pick<MH>(GN_NORM_LN, GN_EPI_GELU_TANH),
-                      pick<MH>(GN_NORM_LN, GN_EPI_SILU), pick<MH>(GN_NORM_RMS, GN_EPI_NONE),
-                      pick<MH>(GN_NORM_RMS, GN_EPI_GELU_TANH), pick<MH>(GN_NORM_RMS, GN_EPI_SILU)};
-  for (const void* k : ks)
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Tile<MH>::Smem) != cudaSuccess)
-      return false;
+  for (int norm = 0; norm < 3; ++norm)
+    for (int epi = 0; epi < 3; ++epi)
+      if (cudaFuncSetAttribute(pick<MH>(norm, epi), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)Tile<MH>::Smem) != cudaSuccess)
+        return false;
   return true;
 }
 
@@ -808,16 +812,17 @@ void* pick_pair_epi(int epi) {
 }
 
 void* pick_pair(int norm, int epi) {
-  return norm == GN_NORM_LN ? pick_pair_epi<GN_NORM_LN>(epi) : pick_pair_epi<GN_NORM_RMS>(epi);
+  return norm == GN_NORM_LN    ? pick_pair_epi<GN_NORM_LN>(epi)
+         : norm == GN_NORM_RMS ? pick_pair_epi<GN_NORM_RMS>(epi)
+                               : pick_pair_epi<GN_NORM_NONE>(epi);
 }
 
 bool set_pair_smem_attr() {
-  const void* ks[] = {pick_pair(GN_NORM_LN, GN_EPI_NONE), pick_pair(GN_NORM_LN, GN_EPI_GELU_TANH),
-                      pick_pair(GN_NORM_LN, GN_EPI_SILU), pick_pair(GN_NORM_RMS, GN_EPI_NONE),
-                      pick_pair(GN_NORM_RMS, GN_EPI_GELU_TANH), pick_pair(GN_NORM_RMS, GN_EPI_SILU)};
-  for (const void* k : ks)
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPairSmem) != cudaSuccess)
-      return false;
+  for (int norm = 0; norm < 3; ++norm)
+    for (int epi = 0; epi < 3; ++epi)
+      if (cudaFuncSetAttribute(pick_pair(norm, epi), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPairSmem) !=
+          cudaSuccess)
+        return false;
   return true;
 }
 
@@ -837,7 +842,7 @@ extern "C" gn_status gn_norm_linear_prepare(const void* W, const void* g, const 
                                             float* c, float* d, int64_t N, int64_t K, gn_norm norm, int gemma,
                                             gn_dtype dt, void* stream) {
   if (dt != GN_BF16) return dt_ok(dt) ? GN_ERR_UNSUPPORTED : GN_ERR_DTYPE;
-  if (norm != GN_NORM_RMS && norm != GN_NORM_LN) return GN_ERR_SHAPE;
+  if (norm != GN_NORM_RMS && norm != GN_NORM_LN && norm != GN_NORM_NONE) return GN_ERR_SHAPE;
   if (N < 0 || K <= 0 || K > INT32_MAX || N > INT32_MAX) return GN_ERR_SHAPE;
   if (N == 0) return GN_OK;
   if (!W || !Wf) return GN_ERR_NULL;
@@ -850,6 +855,8 @@ extern "C" gn_status gn_norm_linear_prepare(const void* W, const void* g, const 
   auto* fb = static_cast<__nv_bfloat16*>(Wf);
   if (norm == GN_NORM_LN)
     norm_linear_prepare_kernel<GN_NORM_LN><<<(unsigned)N, 256, 0, s>>>(Wb, gb, bb, cb, fb, c, d, (int)K, 0);
+  else if (norm == GN_NORM_NONE)
+    norm_linear_prepare_kernel<GN_NORM_NONE><<<(unsigned)N, 256, 0, s>>>(Wb, nullptr, nullptr, cb, fb, c, d, (int)K, 0);
   else
     norm_linear_prepare_kernel<GN_NORM_RMS><<<(unsigned)N, 256, 0, s>>>(Wb, gb, nullptr, cb, fb, c, d, (int)K,
                                                                         gemma != 0);
@@ -863,11 +870,11 @@ extern "C" gn_status gn_norm_linear_fwd(const void* x, const void* Wf, const flo
                                         void* stream) {
   if (dt != GN_BF16) return dt_ok(dt) ? GN_ERR_UNSUPPORTED : GN_ERR_DTYPE;
   if (!epi_ok(epi)) return GN_ERR_DTYPE;
-  if (norm != GN_NORM_RMS && norm != GN_NORM_LN) return GN_ERR_SHAPE;
+  if (norm != GN_NORM_RMS && norm != GN_NORM_LN && norm != GN_NORM_NONE) return GN_ERR_SHAPE;
   if (M < 0 || N < 0 || K <= 0 || ldx < K || ldy < N || K % 8 || ldx % 8 || ldy % 8) return GN_ERR_SHAPE;
   if (M > (int64_t)65535 * kUM || N > INT32_MAX || K > INT32_MAX) return GN_ERR_SHAPE;
   if (M == 0 || N == 0) return GN_OK;
-  if (!x || !Wf || !y || !rstd || (norm == GN_NORM_LN && (!c || !mean))) return GN_ERR_NULL;
+  if (!x || !Wf || !y || (norm != GN_NORM_NONE && !rstd) || (norm == GN_NORM_LN && (!c || !mean))) return GN_ERR_NULL;
   if (!aligned16(x) || !aligned16(Wf) || !aligned16(y) || (c && !aligned16(c)) || (d && !aligned16(d)))
     return GN_ERR_ALIGN;
   // pairs of SMs sharing 256 x 512 tiles once there are more than 128 rows and 256 columns;
@@ -893,7 +900,7 @@ extern "C" gn_status gn_norm_linear_fwd(const void* x, const void* Wf, const flo
   a.eps = eps;
   a.err = device_err_word();
   if (!a.err) return GN_ERR_CUDA;
-  if (pair) {  // the pair kernel reads the row statistics: compute them first
+  if (pair && norm != GN_NORM_NONE) {  // the pair kernel reads the row statistics: compute them first
     const unsigned sblocks = (unsigned)((M + 7) / 8);
     if (norm == GN_NORM_LN)
       norm_stats_kernel<GN_NORM_LN><<<sblocks, 256, 0, (cudaStream_t)stream>>>(
