@@ -8,27 +8,32 @@
 //   LayerNorm: xn[k] = (x[k] - mu) s g[k] + beta[k], so
 //     y[m,n] = act( s_m * sum_k x[m,k] Wf[n,k] - s_m mu_m c[n] + d[n] )
 //     with Wf[n,k] = bf16(g[k] W[n,k]), c[n] = sum_k Wf[n,k], d[n] = sum_k beta[k] W[n,k] + bias[n];
-//   RMSNorm:   y[m,n] = act( r_m * sum_k x[m,k] Wf[n,k] + d[n] ), Wf = bf16(g'[k] W[n,k]), d = bias.
+//   RMSNorm:   y[m,n] = act( r_m * sum_k x[m,k] Wf[n,k] + d[n] ), Wf = bf16(g'[k] W[n,k]), d = bias;
+//   no norm:   y[m,n] = act( sum_k x[m,k] W[n,k] + bias[n] )   (the plain layer; TiledLinear).
 // gn_norm_linear_prepare builds Wf, c and d once per weight (a memory-bound pass over W). The
-// forward kernel then streams the raw bf16 x and Wf through TMA straight into the tensor
-// cores; the per-row statistics (mu, s or r) are accumulated by the epilogue warps from the
-// same A tiles while they sit in shared memory, and applied with the column terms and the
-// activation when the fp32 accumulator is read back from tensor memory.
+// forward kernels stream the raw bf16 x and Wf through TMA straight into the tensor cores and
+// apply the row statistics, the column terms and the activation when the fp32 accumulators
+// are read back from tensor memory.
 //
-// Forward kernel, one 128 x 256 output tile per CTA (6 warps):
-//   warp 0      TMA producer: A tile [128 rows x 64 k] and B tile [256 rows x 64 k] per stage,
-//               128-byte swizzled, 4 stages (48 KiB each);
-//   warp 1      allocates 256 tensor-memory columns; one lane issues tcgen05.mma (M=128,
-//               N=256, K=16, bf16 in, fp32 accumulate) and commits each stage back to the
-//               producer, then the finished accumulator to the epilogue;
-//   warps 2..5  per-row statistics from the A tiles (thread = row; each copies its row's 128
-//               bytes of the tile to registers and releases the stage), then the epilogue:
-//               tcgen05.ld of 32 accumulator columns at a time, corrections, activation,
-//               bf16 stores. A warp may only read the tensor-memory lanes 32*(warp%4)..+31,
-//               so warp w owns rows 32*(w%4)..+31 of the tile.
-// Every mbarrier wait is bounded (kWaitLimitNs); a timeout records the error bit, the CTA
-// skips its stores, waits for its own tensor-core work and copies, frees its tensor memory
-// and exits.
+// Three kernels, by shape:
+//   * norm_linear_pair_kernel (more than 128 rows and 256 columns): a cluster of two CTAs on
+//     two SMs per 256 x 512 tile, tcgen05.mma.cta_group::2; the row statistics come from
+//     norm_stats_kernel, a streaming pre-pass (see the comment above the pair kernel);
+//   * norm_linear_kernel<MH> (otherwise): one CTA per 128 x 256 (MH = 1) or 256 x 256 (MH = 2)
+//     tile, 2 + 4*MH warps:
+//       warp 0      TMA producer: A tile [128*MH rows x 64 k] and B tile [256 rows x 64 k] per
+//                   stage, 128-byte swizzled, as many stages as fit in shared memory;
+//       warp 1      allocates the tensor memory; one lane issues tcgen05.mma (M=128, N=256,
+//                   K=16, bf16 in, fp32 accumulate; MH instructions share each B tile) and
+//                   commits each stage back to the producer, then the accumulators to the
+//                   epilogue;
+//       warps 2..   per-row statistics from the A tiles (thread = row; each copies its row of
+//                   the tile to registers, consumes it and releases the stage), then the
+//                   epilogue: tcgen05.ld of 32 accumulator columns at a time, corrections,
+//                   activation, bf16 stores. A warp may only read the tensor-memory lanes
+//                   32*(warp%4)..+31, so warp w owns rows 128h + 32*(w%4).. of the tile.
+// Every mbarrier wait is bounded (kWaitLimitNs); a timeout records the error bit, the CTA skips
+// its stores, waits for its own tensor-core work and copies, frees its tensor memory and exits.
 #include <cuda.h>  // CUtensorMap and the cuTensorMapEncodeTiled prototype (types only)
 
 #include <mutex>
