@@ -470,7 +470,7 @@ extern "C" gn_status gn_rmsnorm_fwd(const void* x, const void* w, void* y, float
   const size_t es = dt_size(dt);
   if (!aligned16(x) || !aligned16(y) || (ld_x * es) % 16 || (ld_y * es) % 16) return GN_ERR_ALIGN;
   NormPlan p;
-  gn_status st = plan_norm(hidden, es, 1, 1, 8, 160, &p);
+  gn_status st = plan_norm(hidden, es, 1, 1, 8, 320, &p);
   if (st != GN_OK) return st;
   void* kern = dt == GN_BF16 ? pick_fwd_t<__nv_bfloat16>(p.vpt, p.cta, epi, gemma != 0)
                              : pick_fwd_t<float>(p.vpt, p.cta, epi, gemma != 0);
