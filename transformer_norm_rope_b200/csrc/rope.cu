@@ -442,9 +442,10 @@ gn_status plan_rope(int64_t B, int64_t S, int64_t H, int64_t D, int ntens, int m
   p->statslot = mode == QK_BWD ? round128((uint32_t)(HC * 4)) : 0u;
   const size_t sstride = (size_t)nslots * p->tslot + p->tabslot + (size_t)ntens * p->statslot;
   // stage depth per CTA (measured on B200): the plain rotation computes so little that one
-  // CTA with a deep pipeline streams best; the qk-norm passes keep ~64-96 KiB per CTA so that
-  // 2-3 CTAs share an SM
-  const size_t depth = mode == ROPE ? 128 * 1024 : mode == QK_FWD ? 64 * 1024 : 96 * 1024;
+  // CTA per SM with ~4 stages of q and k streams best (deeper pipelines and more CTAs per SM
+  // were slower: ~5750 against ~6340 GB/s at [1, 32760, 40, 128]); the qk-norm passes keep
+  // ~64-96 KiB per CTA so that 2-3 CTAs share an SM
+  const size_t depth = mode == ROPE ? 84 * 1024 : mode == QK_FWD ? 64 * 1024 : 96 * 1024;
   int stages = g_tune.stages ? g_tune.stages : (int)(depth / sstride);
   stages = stages < 2 ? 2 : stages > kRopeMaxStages ? kRopeMaxStages : stages;
   const size_t limit = smem_optin();
@@ -476,7 +477,7 @@ gn_status setup(int64_t B, int64_t S, int64_t H, int64_t D, int ntens, int mode,
   gn_status st = plan_rope(B, S, H, D, ntens, mode, dt_size(dt), p);
   if (st != GN_OK) return st;
   *kern = pick(dt, mode, gemma);
-  const int cap = g_tune.ctas_per_sm ? g_tune.ctas_per_sm : 8;
+  const int cap = g_tune.ctas_per_sm ? g_tune.ctas_per_sm : mode == ROPE ? 1 : 8;
   int g = persistent_grid(*kern, p->threads, p->smem, cap);
   if (g <= 0) return GN_ERR_CUDA;
   const int64_t units = B * S * p->NC;
