@@ -73,8 +73,9 @@ inline gn_status plan_norm(int64_t N, size_t es, int ntens, int nparams, int max
   int stages = g_tune.stages;
   if (stages == 0) {
     // forward: shallow pipelines leave room for more CTAs per SM, which hides the per-row
-    // reduction latency better (measured on B200); backward: ~64 KiB in flight per CTA
-    stages = (int)((ntens > 1 ? 65536 : 24576) / (slot * ntens));
+    // reduction latency better; backward: ~40 KiB in flight per CTA (2 stages of x and dy at
+    // hidden 5120 bf16; 3 or 4 were 1-2 % slower). Measured on B200.
+    stages = (int)((ntens > 1 ? 40960 : 24576) / (slot * ntens));
     stages = stages < 2 ? 2 : stages > kMaxStages ? kMaxStages : stages;
   }
   if (stages > kMaxStages) stages = kMaxStages;
