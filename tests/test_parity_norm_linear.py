@@ -6,7 +6,8 @@ Tolerance: the bf16 output tolerance (1.6e-2 relative + 1e-2 absolute). The kern
 Wf = bf16(g W), one bf16 rounding per weight, where the unfused layer rounds the normalized
 activations instead; with W ~ N(0, 1/K) and unit-scale outputs either rounding perturbs an output
 by about 1e-3 (random over K terms), an order of magnitude inside the bound. The row statistics
-(fp32, shifted one-pass moments over the streamed tiles) are checked at 1e-5 relative."""
+(fp32: each piece of the row centred on its own mean, the pieces combined with Chan's pairwise
+update) are checked at 1e-5 relative."""
 import math
 
 import numpy as np
