@@ -68,8 +68,10 @@ def test_norm_linear_empty_and_unsupported(gpu):
     Wf, c, d = gpu.norm_linear_prepare(W, norm="ln")
     y, _, _ = gpu.norm_linear_fwd(x, Wf, c, d)
     assert y.shape == (0, 256)
-    with pytest.raises(gpu.GnError):
-        gpu.norm_linear_fwd(torch.zeros((4, 60), dtype=torch.bfloat16, device="cuda"), Wf, c, d)  # K % 8
+    W60 = torch.zeros((256, 60), dtype=torch.bfloat16, device="cuda")
+    Wf60, c60, d60 = gpu.norm_linear_prepare(W60, norm="ln")
+    with pytest.raises(gpu.GnError):  # K % 8: the rows of x and W are not 16-byte tiles
+        gpu.norm_linear_fwd(torch.zeros((4, 60), dtype=torch.bfloat16, device="cuda"), Wf60, c60, d60)
 
 
 @pytest.mark.slow

@@ -142,11 +142,39 @@ def _epi(epi) -> int:
     return EPILOGUES[epi] if isinstance(epi, str) else int(epi)
 
 
-def _rows(x):
-    """(rows, hidden, ld) of a tensor whose last dim is contiguous and whose leading dims
+def _on_gpu(t) -> bool:
+    return t.is_cuda
+
+
+def _need(t, name, *, like=None, shape=None, numel=None, dtype=None, contiguous=True, optional=False):
+    """Validate a tensor argument before its pointer reaches the library, which sees raw
+    pointers only: a wrong size, dtype or layout there would read or write out of bounds.
+    Checks (in this order) presence, shape or element count, dtype, contiguity, and that it
+    lives on the device of `like` (always a CUDA device)."""
+    if t is None:
+        if optional:
+            return
+        raise ValueError(f"{name} is required")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if numel is not None and t.numel() != numel:
+        raise ValueError(f"{name} has {t.numel()} elements, expected {numel}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if contiguous and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if not _on_gpu(t):
+        raise ValueError(f"{name} must be a CUDA tensor (the library runs on the GPU only)")
+    if like is not None and t.device != like.device:
+        raise ValueError(f"{name} is on {t.device}, the other operands on {like.device}")
+
+
+def _rows(x, name="x", like=None, dtype=None):
+    """(rows, hidden, ld) of a CUDA tensor whose last dim is contiguous and whose leading dims
     collapse to one row stride."""
+    _need(x, name, like=like, dtype=dtype, contiguous=False)
     if x.dim() < 1 or x.stride(-1) != 1:
-        raise ValueError("last dimension must be contiguous")
+        raise ValueError(f"last dimension of {name} must be contiguous")
     hidden = x.shape[-1]
     x2 = x.reshape(-1, hidden) if x.dim() != 2 else x
     if x2.data_ptr() != x.data_ptr():
@@ -178,8 +206,10 @@ def rmsnorm_fwd(x, w, eps=1e-6, gemma=False, epilogue="none", out=None, save_sta
     """y = epi(x * rsqrt(mean(x^2) + eps) * w') -> (y, inv_rms[rows] fp32 or None)."""
     torch = _torch()
     rows, hidden, ld = _rows(x)
+    _need(w, "w", like=x, shape=(hidden,), dtype=x.dtype)
     y = empty_rows(x.shape, x.dtype, x.device) if out is None else out
-    _, _, ldy = _rows(y)
+    _need(y, "out", like=x, shape=x.shape, contiguous=False)
+    _, _, ldy = _rows(y, "out", like=x, dtype=x.dtype)
     r = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device) if save_stats else None
     check(gn_rmsnorm_fwd(_ptr(x), _ptr(w), _ptr(y), _ptr(r), rows, hidden, ld, ldy, eps, int(gemma),
                          _epi(epilogue), _dt(x), _stream(stream)), "gn_rmsnorm_fwd")
@@ -190,7 +220,10 @@ def rmsnorm_bwd(x, w, inv_rms, dy, gemma=False, epilogue="none", want_dw=True, s
     """-> (dx, dw fp32 or None)."""
     torch = _torch()
     rows, hidden, ld = _rows(x)
-    _, _, lddy = _rows(dy)
+    _need(w, "w", like=x, shape=(hidden,), dtype=x.dtype)
+    _need(inv_rms, "inv_rms", like=x, numel=rows, dtype=torch.float32)
+    _need(dy, "dy", like=x, shape=x.shape, contiguous=False)
+    _, _, lddy = _rows(dy, "dy", like=x, dtype=x.dtype)
     dx = empty_rows(x.shape, x.dtype, x.device)
     _, _, lddx = _rows(dx)
     dw = torch.empty(hidden, dtype=torch.float32, device=x.device) if want_dw else None
@@ -206,8 +239,11 @@ def layernorm_fwd(x, w=None, b=None, eps=1e-5, epilogue="none", out=None, save_s
     """y = epi((x - mean) * rstd * w + b) -> (y, mean, rstd)."""
     torch = _torch()
     rows, hidden, ld = _rows(x)
+    _need(w, "w", like=x, shape=(hidden,), dtype=x.dtype, optional=True)
+    _need(b, "b", like=x, shape=(hidden,), dtype=x.dtype, optional=True)
     y = empty_rows(x.shape, x.dtype, x.device) if out is None else out
-    _, _, ldy = _rows(y)
+    _need(y, "out", like=x, shape=x.shape, contiguous=False)
+    _, _, ldy = _rows(y, "out", like=x, dtype=x.dtype)
     mk = (lambda: torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device))
     mu, rs = (mk(), mk()) if save_stats else (None, None)
     check(gn_layernorm_fwd(_ptr(x), _ptr(w), _ptr(b), _ptr(y), _ptr(mu), _ptr(rs), rows, hidden, ld, ldy,
@@ -219,7 +255,12 @@ def layernorm_bwd(x, w, b, mean, rstd, dy, epilogue="none", want_wgrad=True, str
     """-> (dx, dw, db) (dw, db fp32 or None)."""
     torch = _torch()
     rows, hidden, ld = _rows(x)
-    _, _, lddy = _rows(dy)
+    _need(w, "w", like=x, shape=(hidden,), dtype=x.dtype, optional=True)
+    _need(b, "b", like=x, shape=(hidden,), dtype=x.dtype, optional=True)
+    _need(mean, "mean", like=x, numel=rows, dtype=torch.float32)
+    _need(rstd, "rstd", like=x, numel=rows, dtype=torch.float32)
+    _need(dy, "dy", like=x, shape=x.shape, contiguous=False)
+    _, _, lddy = _rows(dy, "dy", like=x, dtype=x.dtype)
     dx = empty_rows(x.shape, x.dtype, x.device)
     _, _, lddx = _rows(dx)
     mk = (lambda: torch.empty(hidden, dtype=torch.float32, device=x.device))
@@ -233,16 +274,24 @@ def layernorm_bwd(x, w, b, mean, rstd, dy, epilogue="none", want_wgrad=True, str
 
 
 def _bshd(q):
-    if q.dim() != 4 or not q.is_contiguous():
+    _need(q, "q")
+    if q.dim() != 4:
         raise ValueError("rotary tensors must be contiguous [B, S, H, D]")
     return q.shape
+
+
+def _tables(q, cos, sin):
+    torch = _torch()
+    _, S, _, D = q.shape
+    _need(cos, "cos", like=q, shape=(S, D // 2), dtype=torch.float32)
+    _need(sin, "sin", like=q, shape=(S, D // 2), dtype=torch.float32)
 
 
 def rope_apply_(q, k, cos, sin, sign=+1, stream=None):
     """In-place interleaved RoPE of q (and k, may be None); sign=-1 is the backward."""
     B, S, H, D = _bshd(q)
-    if k is not None and k.shape != q.shape:
-        raise ValueError("q and k must have the same shape")
+    _need(k, "k", like=q, shape=q.shape, dtype=q.dtype, optional=True)
+    _tables(q, cos, sin)
     check(gn_rope_apply_inplace(_ptr(q), _ptr(k), _ptr(cos), _ptr(sin), B, S, H, D, int(sign), _dt(q),
                                 _stream(stream)), "gn_rope_apply_inplace")
     return q, k
@@ -252,6 +301,10 @@ def qknorm_rope_fwd(q, k, wq, wk, cos, sin, eps=1e-6, gemma=False, stream=None):
     """-> (q_out, k_out, inv_rms_q, inv_rms_k); k may be None."""
     torch = _torch()
     B, S, H, D = _bshd(q)
+    _need(k, "k", like=q, shape=q.shape, dtype=q.dtype, optional=True)
+    _need(wq, "wq", like=q, shape=(D,), dtype=q.dtype)
+    _need(wk, "wk", like=q, shape=(D,), dtype=q.dtype, optional=k is None)
+    _tables(q, cos, sin)
     qo = torch.empty_like(q)
     ko = torch.empty_like(k) if k is not None else None
     rq = torch.empty((B, S, H), dtype=torch.float32, device=q.device)
@@ -267,6 +320,15 @@ def qknorm_rope_bwd(q, k, wq, wk, cos, sin, inv_rms_q, inv_rms_k, dq_out, dk_out
     """-> (dq, dk, dwq, dwk)."""
     torch = _torch()
     B, S, H, D = _bshd(q)
+    _need(k, "k", like=q, shape=q.shape, dtype=q.dtype, optional=True)
+    _need(wq, "wq", like=q, shape=(D,), dtype=q.dtype)
+    _need(wk, "wk", like=q, shape=(D,), dtype=q.dtype, optional=k is None)
+    _tables(q, cos, sin)
+    _need(inv_rms_q, "inv_rms_q", like=q, numel=B * S * H, dtype=torch.float32)
+    _need(dq_out, "dq_out", like=q, shape=q.shape, dtype=q.dtype)
+    if k is not None:
+        _need(inv_rms_k, "inv_rms_k", like=q, numel=B * S * H, dtype=torch.float32)
+        _need(dk_out, "dk_out", like=q, shape=q.shape, dtype=q.dtype)
     dq = torch.empty_like(q)
     dk = torch.empty_like(k) if k is not None else None
     dwq = torch.empty(D, dtype=torch.float32, device=q.device) if want_dw else None
@@ -288,7 +350,13 @@ def norm_linear_prepare(W, g=None, beta=None, bias=None, norm="ln", gemma=False,
     """Fold the norm weight into the layer weight W [N, K] (bf16): -> (Wf [N, K] bf16, c [N] fp32
     or None, d [N] fp32)."""
     torch = _torch()
+    _need(W, "W")
+    if W.dim() != 2:
+        raise ValueError("W must be [N, K]")
     N, K = W.shape
+    _need(g, "g", like=W, shape=(K,), dtype=W.dtype, optional=True)
+    _need(beta, "beta", like=W, shape=(K,), dtype=W.dtype, optional=True)
+    _need(bias, "bias", like=W, shape=(N,), dtype=W.dtype, optional=True)
     Wf = torch.empty_like(W)
     c = torch.empty(N, dtype=torch.float32, device=W.device) if _norm(norm) == GN_NORM_LN else None
     d = torch.empty(N, dtype=torch.float32, device=W.device)
@@ -302,9 +370,19 @@ def norm_linear_fwd(x, Wf, c, d, eps=1e-5, norm="ln", epilogue="none", save_stat
     -> (y, mean, rstd) (statistics fp32 [M], or None). `out` may give y (rows of a larger
     tensor included: its row stride is passed on)."""
     torch = _torch()
+    if x.dim() != 2:
+        raise ValueError("x must be [M, K]")
     M, K = x.shape
+    _rows(x)
+    _need(Wf, "Wf", like=x, dtype=x.dtype)
+    if Wf.dim() != 2 or Wf.shape[1] != K:
+        raise ValueError(f"Wf has shape {tuple(Wf.shape)}, expected [N, {K}]")
     N = Wf.shape[0]
+    _need(c, "c", like=x, shape=(N,), dtype=torch.float32, optional=_norm(norm) != GN_NORM_LN)
+    _need(d, "d", like=x, shape=(N,), dtype=torch.float32, optional=True)
     y = torch.empty((M, N), dtype=x.dtype, device=x.device) if out is None else out
+    _need(y, "out", like=x, shape=(M, N), contiguous=False)
+    _rows(y, "out", like=x, dtype=x.dtype)
     plain = _norm(norm) == GN_NORM_NONE
     mu = None if plain else torch.empty(M, dtype=torch.float32, device=x.device)  # the kernels need both
     rs = None if plain else torch.empty(M, dtype=torch.float32, device=x.device)
@@ -316,7 +394,10 @@ def norm_linear_fwd(x, Wf, c, d, eps=1e-5, norm="ln", epilogue="none", save_stat
 
 def act_grad(z, dy, epilogue="silu", out=None, stream=None):
     """dz = dy * act'(z), elementwise (contiguous tensors of one dtype)."""
+    _need(dy, "dy")
+    _need(z, "z", like=dy, shape=dy.shape, dtype=dy.dtype)
     dz = torch_empty_like(dy) if out is None else out
+    _need(dz, "out", like=dy, shape=dy.shape, dtype=dy.dtype)
     check(gn_act_grad(_ptr(z), _ptr(dy), _ptr(dz), dy.numel(), _epi(epilogue), _dt(dy), _stream(stream)),
           "gn_act_grad")
     return dz
