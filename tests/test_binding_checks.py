@@ -129,3 +129,29 @@ def test_linear_helpers(stub):
         with pytest.raises((ValueError, TypeError)):
             f()
     assert len(stub) == 5
+
+
+def test_tiled_linear_autograd_plumbing(stub, monkeypatch):
+    # with the kernels stubbed, the values are meaningless; the test checks that the autograd
+    # form saves what it needs and returns one gradient per input, of the input's dtype and shape
+    from transformer_norm_rope_b200 import tiled_linear as tl
+
+    def addmm_f32(c, a, b, out_dtype, out):  # the fp32-output addmm exists for CUDA only
+        assert out_dtype == f32 and out is c and c.dtype == f32
+        return out.add_(a.float() @ b.float())
+
+    monkeypatch.setattr(torch, "addmm", addmm_f32)
+
+    M, N, K = 24, 16, 32
+    x = z(M, K).requires_grad_()
+    W = z(N, K).requires_grad_()
+    b = z(N).requires_grad_()
+    y = tl.TiledLinearFunction.apply(x, W, b, "silu", 3)
+    assert y.shape == (M, N) and y.dtype == bf
+    y.backward(z(M, N))
+    assert x.grad.shape == x.shape and W.grad.shape == W.shape and b.grad.shape == b.shape
+    assert x.grad.dtype == W.grad.dtype == b.grad.dtype == bf
+    x2 = z(M, K).requires_grad_()
+    tl.TiledLinearFunction.apply(x2, W, None, "gelu_tanh", None).backward(z(M, N))
+    assert x2.grad.shape == x2.shape
+    assert stub.count("gn_norm_linear_fwd") == 2 * 3 + 2 * 1  # forward + recompute, per chunk

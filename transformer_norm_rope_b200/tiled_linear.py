@@ -10,7 +10,8 @@ Where each step runs:
   * forward and recompute: ``gn_norm_linear_fwd`` with ``GN_NORM_NONE`` (the tcgen05 kernels of
     this library; the bias and activation in their epilogue);
   * dz = dy * act'(z): ``gn_act_grad``;
-  * dx = dz W and dW += dz^T x: plain GEMMs, done by cuBLAS (``torch.matmul``); db by a sum.
+  * dx = dz W and dW += dz^T x: plain GEMMs, done by cuBLAS (``torch.matmul``, and
+    ``torch.addmm`` with an fp32 output accumulating dW across the chunks); db by a sum.
 This module only orchestrates chunks (host logic); every elementwise and fused step is a kernel
 of the library.
 """
@@ -71,9 +72,36 @@ def backward(x, Wf, d, dy, act: str = "silu", chunks: Optional[int] = None) -> T
         z = gn.norm_linear_fwd(xc, Wf, None, d, norm="none", epilogue="none", save_stats=False)[0]
         dz = gn.act_grad(z, dy[r0:r1].contiguous(), epilogue=act, out=z)  # z is not needed after this
         torch.matmul(dz, Wf, out=dx[r0:r1])
-        dW += torch.matmul(dz.t(), xc).float()
+        # bf16 operands, fp32 accumulator updated in place (beta = 1): no bf16 rounding of the
+        # per-chunk partial and no extra pass over a converted copy
+        torch.addmm(dW, dz.t(), xc, out_dtype=torch.float32, out=dW)
         db += dz.sum(0, dtype=torch.float32)
     return dx, dW, db
+
+
+def _function_class():
+    torch = gn._torch()
+
+    class _TiledLinear(torch.autograd.Function):
+        @staticmethod
+        def forward(ctx, x, W, bias, act, chunks):
+            Wf, d = prepare(W, bias)
+            ctx.save_for_backward(x, Wf, d)
+            ctx.act, ctx.chunks = act, chunks
+            ctx.w_dtype = W.dtype
+            ctx.b_dtype = None if bias is None else bias.dtype
+            return forward(x, Wf, d, act, chunks)
+
+        @staticmethod
+        def backward(ctx, dy):
+            x, Wf, d = ctx.saved_tensors
+            dx, dW, db = backward(x, Wf, d, dy.contiguous(), ctx.act, ctx.chunks)
+            return dx, dW.to(ctx.w_dtype), (None if ctx.b_dtype is None else db.to(ctx.b_dtype)), None, None
+
+    return _TiledLinear
+
+
+_FUNCTION = None
 
 
 class TiledLinearFunction:
@@ -81,19 +109,7 @@ class TiledLinearFunction:
 
     @staticmethod
     def apply(x, W, bias, act: str = "silu", chunks: Optional[int] = None):
-        torch = gn._torch()
-
-        class _F(torch.autograd.Function):
-            @staticmethod
-            def forward(ctx, x_, W_, b_):
-                Wf, d = prepare(W_, b_)
-                ctx.save_for_backward(x_, Wf, d)
-                return forward(x_, Wf, d, act, chunks)
-
-            @staticmethod
-            def backward(ctx, dy):
-                x_, Wf, d = ctx.saved_tensors
-                dx, dW, db = backward(x_, Wf, d, dy.contiguous(), act, chunks)
-                return dx, dW.to(W.dtype), (db.to(bias.dtype) if bias is not None else None)
-
-        return _F.apply(x, W, bias)
+        global _FUNCTION
+        if _FUNCTION is None:
+            _FUNCTION = _function_class()
+        return _FUNCTION.apply(x, W, bias, act, chunks)
