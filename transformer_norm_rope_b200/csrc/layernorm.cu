@@ -145,8 +145,8 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT)) ln_fwd_
   // with the tanh-GeLU epilogue the weight and bias are staged halved (exact): the affine map
   // then yields z / 2, which gelu_of_half2 takes directly
   constexpr float kParamScale = EPI == EPI_GELU_TANH ? 0.5f : 1.0f;
-  stage_param(pipe.param(0), static_cast<const T*>(a.w), N, nvec, 1.0f, ct, nct, kParamScale);
-  stage_param(pipe.param(1), static_cast<const T*>(a.b), N, nvec, 0.0f, ct, nct, kParamScale);
+  stage_param<T, VPT>(pipe.param(0), static_cast<const T*>(a.w), N, nvec, 1.0f, ct, nct, kParamScale);
+  stage_param<T, VPT>(pipe.param(1), static_cast<const T*>(a.b), N, nvec, 0.0f, ct, nct, kParamScale);
   consumers_sync(nct);
   int cnt[VPT];
 #pragma unroll
@@ -257,8 +257,8 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT, true)) l
     return;
   }
   const int ct = tid - 32, nct = ncw * 32, cw = warp - 1;
-  stage_param(pipe.param(0), static_cast<const T*>(a.w), N, nvec, 1.0f, ct, nct);
-  stage_param(pipe.param(1), static_cast<const T*>(a.b), N, nvec, 0.0f, ct, nct);
+  stage_param<T, VPT>(pipe.param(0), static_cast<const T*>(a.w), N, nvec, 1.0f, ct, nct);
+  stage_param<T, VPT>(pipe.param(1), static_cast<const T*>(a.b), N, nvec, 0.0f, ct, nct);
   consumers_sync(nct);
   float2 dwa[VPT][H], dba[VPT][H];
 #pragma unroll

@@ -9,14 +9,39 @@
 
 namespace gn {
 
-// per-column parameters (weight, bias) copied once into shared memory, padded with zeros
-// (times `scale`, a power of two, so the stored values stay exact)
-template <typename T>
+// Per-column parameters (weight, bias) copied once into shared memory, padded with zeros,
+// times `scale` (a power of two, so the stored values stay exact); `dflt` stands for a null
+// src. Consumer thread ct writes vectors ct + j * nct (j < VPT), which covers the row. The
+// whole 16-byte vectors of an aligned src are fetched with one load each, all of a thread's
+// loads issued before the first is used: an element-strided loop paid one L2 round trip per
+// element at the start of every CTA. A ragged tail or an unaligned src goes element by element.
+template <typename T, int VPT>
 __device__ __forceinline__ void stage_param(uint8_t* dst, const T* src, int N, int nvec, float dflt, int ct, int nct,
                                             float scale = 1.0f) {
-  T* d = reinterpret_cast<T*>(dst);
-  const int n = nvec * Vec<T>::N;
-  for (int i = ct; i < n; i += nct) Vec<T>::store1(d + i, i < N ? scale * ld_param(src, i, dflt) : 0.0f);
+  constexpr int E = Vec<T>::N;
+  const int nfull = (src && (reinterpret_cast<uintptr_t>(src) & 15u) == 0) ? N / E : 0;
+  uint4 raw[VPT];
+#pragma unroll
+  for (int j = 0; j < VPT; ++j) {
+    const int v = ct + j * nct;
+    raw[j] = v < nfull ? __ldg(reinterpret_cast<const uint4*>(src) + v) : make_uint4(0u, 0u, 0u, 0u);
+  }
+#pragma unroll
+  for (int j = 0; j < VPT; ++j) {
+    const int v = ct + j * nct;
+    if (v < nvec) {
+      float f[E];
+      if (v < nfull) {
+        Vec<T>::unpack(raw[j], f);
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) f[e] = v * E + e < N ? ld_param(src, v * E + e, dflt) : 0.0f;
+      }
+#pragma unroll
+      for (int e = 0; e < E; ++e) f[e] *= scale;
+      *reinterpret_cast<uint4*>(dst + (size_t)v * 16) = Vec<T>::pack(f);
+    }
+  }
 }
 
 // the parameters of vector v as element pairs

@@ -67,7 +67,7 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT)) rms_fwd
     return;
   }
   const int ct = tid - 32, nct = ncw * 32, cw = warp - 1;
-  stage_param(pipe.param(0), static_cast<const T*>(a.w), N, nvec, 0.0f, ct, nct);
+  stage_param<T, VPT>(pipe.param(0), static_cast<const T*>(a.w), N, nvec, 0.0f, ct, nct);
   consumers_sync(nct);
   const float inv_n = 1.0f / (float)N;
   const int64_t step = gridDim.x;
@@ -137,7 +137,7 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT, true)) r
     return;
   }
   const int ct = tid - 32, nct = ncw * 32, cw = warp - 1;
-  stage_param(pipe.param(0), static_cast<const T*>(a.w), N, nvec, 0.0f, ct, nct);
+  stage_param<T, VPT>(pipe.param(0), static_cast<const T*>(a.w), N, nvec, 0.0f, ct, nct);
   consumers_sync(nct);
   float2 dwa[VPT][H];
 #pragma unroll
