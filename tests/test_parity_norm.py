@@ -183,3 +183,43 @@ def test_layernorm_full_size(gpu):
     assert_close(to_np(rs), rrs, "stat", "full ln rstd")
     assert_close(to_np(dw), rdw, "grad_bf16", "full ln dw")
     assert_close(to_np(db), rdb, "grad_bf16", "full ln db")
+
+
+def _shifted(t):
+    """The same values in storage that starts 2 bytes past a 16-byte boundary."""
+    buf = torch.empty(t.numel() + 8, dtype=t.dtype, device=t.device)
+    off = (2 - buf.data_ptr() % 16) % 16 // t.element_size() if t.element_size() == 2 else 1
+    out = buf[off:off + t.numel()]
+    out.copy_(t)
+    return out
+
+
+@pytest.mark.parametrize("hidden", [2051, 5120])
+def test_unaligned_weights_give_the_aligned_result(gpu, hidden):
+    # weights need no alignment: whole 16-byte vectors of an aligned weight are staged with one
+    # load each, an unaligned one element by element; the staged values, hence every output,
+    # must be the same bits
+    d = wl.layernorm(M=300, N=hidden, dtype="bf16")
+    x, dy = to_rows(d["x"]), to_rows(d["dy"])
+    w, b = to_dev(d["w"]), to_dev(d["b"])
+    ws, bs = _shifted(w), _shifted(b)
+    assert ws.data_ptr() % 16 != 0 and torch.equal(ws, w)
+    for epi in ("gelu_tanh", "none"):
+        a = gpu.layernorm_fwd(x, w, b, d["eps"], epilogue=epi)
+        u = gpu.layernorm_fwd(x, ws, bs, d["eps"], epilogue=epi)
+        ga = gpu.layernorm_bwd(x, w, b, a[1], a[2], dy, epilogue=epi)
+        gu = gpu.layernorm_bwd(x, ws, bs, a[1], a[2], dy, epilogue=epi)
+        torch.cuda.synchronize()
+        for p, q in zip(a + ga, u + gu):
+            assert torch.equal(p, q), f"layernorm {epi} {hidden}"
+    r = wl.rmsnorm(M=300, N=hidden, dtype="bf16", gemma=True)
+    xr, dyr, wr = to_rows(r["x"]), to_rows(r["dy"]), to_dev(r["w"])
+    wrs = _shifted(wr)
+    a = gpu.rmsnorm_fwd(xr, wr, r["eps"], gemma=True, epilogue="silu")
+    u = gpu.rmsnorm_fwd(xr, wrs, r["eps"], gemma=True, epilogue="silu")
+    ga = gpu.rmsnorm_bwd(xr, wr, a[1], dyr, gemma=True, epilogue="silu")
+    gu = gpu.rmsnorm_bwd(xr, wrs, a[1], dyr, gemma=True, epilogue="silu")
+    torch.cuda.synchronize()
+    for p, q in zip(a + ga, u + gu):
+        assert torch.equal(p, q), f"rmsnorm {hidden}"
+    assert gpu.device_error(clear=True) == 0
