@@ -13,13 +13,13 @@
  *         is the same kernel with sin negated.
  *       - "基准实测": FlashNorm and FlashRoPE applied together (the fused qk-norm + RoPE entry
  *         points combine them per attention head).
+ *       - "内核三 TiledLinear": a linear layer run chunk by chunk along the tokens, the backward
+ *         recomputing each chunk instead of keeping its activations (gn_act_grad and
+ *         GN_NORM_NONE serve it).
  *   [L] "LLM层的优化算子", section "编写定制融合算子": LayerNorm fused with a tanh-GeLU epilogue
  *       (centre, biased variance, divide by sqrt(var + eps), times weight plus bias, GeLU).
  *   [J] "Janus-Pro-7B模型推理加速实战", section 4.1: LayerNorm fused with SiLU = x * sigmoid(x),
  *       and LayerNorm, the first linear projection and SiLU fused into one kernel.
- *       - "内核三 TiledLinear": a linear layer run chunk by chunk along the tokens, the backward
- *         recomputing each chunk instead of keeping its activations (gn_act_grad and
- *         GN_NORM_NONE serve it).
  *   [Y] "HY-Motion 1.0性能优化从算法到硬件的全方位调优策略", section 3.1: LayerNorm merged with
  *       the matrix multiplication that follows it (no round trip of the normalized activations
  *       through memory).
