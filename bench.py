@@ -562,11 +562,14 @@ def run_ours(args):
 def e2e(args, suite, kernels, step_bytes, ws, dev):
     """Same metric through host buffers: each step copies its inputs from pinned host memory,
     runs the path, and copies every output back to pinned host memory, as a caller streaming
-    batches through the API would: on three streams, so that step i's download overlaps step
-    i+1's upload (PCIe moves both directions at once). Step i+1 overwrites its inputs only after
-    step i's kernels have read them, its outputs only after step i's download has read them, and
-    the in-place tensors (RoPE q, k) only after both."""
+    batches through the API would. Uploads, kernels and downloads run on three streams over two
+    sets of device buffers used by alternate steps, so that step i+1's upload overlaps step i's
+    download (PCIe moves both directions at once) and neither waits for the other: a set is
+    overwritten only after the step that used it two steps earlier has been read by its
+    kernels (inputs) and by its download (outputs, in-place tensors included)."""
     import torch
+
+    from transformer_norm_rope_b200.shard import GradBucket
 
     steps = max(1, min(args.steps, 5))
     need = set()
@@ -579,31 +582,47 @@ def e2e(args, suite, kernels, step_bytes, ws, dev):
     pin_out = {k: torch.empty(suite.d[k].shape, dtype=suite.d[k].dtype, pin_memory=True) for k in outs}
     h2d = sum(v.numel() * v.element_size() for v in pin_in.values())
     d2h = sum(v.numel() * v.element_size() for v in pin_out.values())
+    # the second buffer set: its own copy of every tensor a step uploads or downloads, and its
+    # own gradient bucket (the all-reduce of a step sums that step's gradients)
+    grad_names = set(suite.grads.names()) if suite.grads is not None else set()
+    alt = dict(suite.d)
+    for k in set(ins) | set(outs):
+        if k not in grad_names:
+            alt[k] = torch.empty_like(suite.d[k])
+    alt_grads = None
+    if suite.grads is not None:
+        alt_grads = GradBucket({k: suite.grads[k].numel() for k in suite.grads.names()}, dev)
+        alt.update(alt_grads.views)
+    sets = [(suite.d, suite.grads), (alt, alt_grads)]
     comp = suite.stream
     s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     Ev = lambda: torch.cuda.Event(enable_timing=False)  # noqa: E731
 
     def run(n, t0=None, t1=None):
-        prev_comp = prev_out = None
+        done = [None, None]  # per set: (kernels read its inputs, download read its outputs)
+        last_out = None
         if t0 is not None:
             t0.record(comp)
             s_in.wait_event(t0)
-        for _ in range(n):
+        for i in range(n):
+            d, grads = sets[i % 2]
+            prev = done[i % 2]
             ev_in, ev_comp, ev_out = Ev(), Ev(), Ev()
             with torch.cuda.stream(s_in):
-                if prev_comp is not None:
-                    s_in.wait_event(prev_comp)  # the previous step's kernels have read the inputs
+                if prev is not None:
+                    s_in.wait_event(prev[0])  # the set's last kernels have read its inputs
                 for k in ins:
                     if k not in inplace:
-                        suite.d[k].copy_(pin_in[k], non_blocking=True)
-                if prev_out is not None and inplace:
-                    s_in.wait_event(prev_out)  # ... and its download has read the in-place tensors
+                        d[k].copy_(pin_in[k], non_blocking=True)
+                if prev is not None and inplace:
+                    s_in.wait_event(prev[1])  # ... and its download has read the in-place tensors
                 for k in inplace:
-                    suite.d[k].copy_(pin_in[k], non_blocking=True)
+                    d[k].copy_(pin_in[k], non_blocking=True)
                 ev_in.record(s_in)
             comp.wait_event(ev_in)
-            if prev_out is not None:
-                comp.wait_event(prev_out)  # outputs are overwritten only after their download
+            if prev is not None:
+                comp.wait_event(prev[1])  # the set's outputs are overwritten only after their download
+            suite.d, suite.grads = d, grads
             for k in kernels:
                 suite.launch(k)
             if ws > 1:
@@ -612,24 +631,28 @@ def e2e(args, suite, kernels, step_bytes, ws, dev):
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_comp)
                 for k in outs:
-                    pin_out[k].copy_(suite.d[k], non_blocking=True)
+                    pin_out[k].copy_(d[k], non_blocking=True)
                 ev_out.record(s_out)
-            prev_comp, prev_out = ev_comp, ev_out
-        comp.wait_event(prev_out)
+            done[i % 2] = (ev_comp, ev_out)
+            last_out = ev_out
+        comp.wait_event(last_out)
         if t1 is not None:
             t1.record(comp)
 
-    run(1)
-    torch.cuda.synchronize(dev)
-    barrier(ws, dev)
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    run(steps, a, b)
-    b.synchronize()
-    barrier(ws, dev)
+    try:
+        run(2)
+        torch.cuda.synchronize(dev)
+        barrier(ws, dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        run(steps, a, b)
+        b.synchronize()
+        barrier(ws, dev)
+    finally:
+        suite.d, suite.grads = sets[0]
     v, _ = throughput_gbs(step_bytes * steps, a.elapsed_time(b) * 1e-3, ws, dev)
     return {"value": round(v, 2), "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "steps": steps,
-            "schedule": "uploads of step i+1 overlap downloads of step i (3 streams)"}
+            "schedule": "two device buffer sets on alternate steps; uploads of step i+1 overlap downloads of step i (3 streams)"}
 
 
 INPUTS = {
