@@ -60,3 +60,18 @@ def test_qknorm_recipe_shapes():
     assert d["q"].shape == (2, 16, 4, 128) and d["q"].dtype == np.uint16
     assert d["dq_out"].shape == d["q"].shape and d["wq"].shape == (128,)
     assert not np.array_equal(d["q"], d["k"])
+
+
+def test_norm_linear_recipe():
+    d = wl.norm_linear(M=64, N=96, K=512, seed=3)
+    assert d["x"].shape == (64, 512) and d["W"].shape == (96, 512) and d["bias"].shape == (96,)
+    assert all(d[k].dtype == np.uint16 for k in ("x", "g", "beta", "W", "bias"))  # bf16 bit patterns
+    W = wl.bf16_to_f32(d["W"]).astype(np.float64)
+    assert abs(W.std() * np.sqrt(512) - 1) < 0.05  # W ~ N(0, 1/K): unit-scale outputs
+    g = wl.bf16_to_f32(d["g"])
+    assert abs(g.mean() - 1) < 0.03 and abs(g.std() - 0.1) < 0.02
+    # the rows are the LayerNorm recipe's rows with the same seed, the layer weights their own streams
+    np.testing.assert_array_equal(d["x"], wl.layernorm(M=64, N=512, dtype="bf16", seed=3)["x"])
+    e = wl.norm_linear(M=8, N=96, K=512, seed=3)
+    np.testing.assert_array_equal(e["W"], d["W"])  # weights do not depend on the row count
+    assert not np.array_equal(wl.norm_linear(M=8, N=96, K=512, seed=4)["W"], d["W"])
