@@ -12,10 +12,12 @@ launched through the C ABI of libgn:
 `value` is the algorithmic HBM bytes of a step (each input read once, each output written
 once) divided by the device time of a step, in GB/s (1e9 bytes), summed over all ranks.
 Every input is larger than the 126 MB L2, and consecutive kernels touch different tensors,
-so no L2 flush is inserted. Launch with torchrun for several GPUs: each rank runs the same
-per-GPU workload on its own seeded data as its shard of a data-parallel step (weak scaling); no
-activation crosses GPUs, and the step's weight gradients (views of one fp32 bucket) are summed
-over the ranks by one NCCL all-reduce per step inside the timed region.
+so no L2 flush is inserted. Launch with torchrun for several GPUs: the ranks share one global
+problem of N times the per-GPU rows and tokens, and rank r owns the r-th contiguous range of
+rows (norms) and tokens (RoPE, qk-norm; with the table rows of its positions), generated from
+the same seed (weak scaling: the work per GPU is fixed). No activation crosses GPUs; the step's
+weight gradients (views of one fp32 bucket) are summed over the ranks by one NCCL all-reduce
+per step inside the timed region.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--only KERNEL[,KERNEL]] [--scale F] [--no-e2e] [--no-cpu-baseline]
@@ -109,7 +111,7 @@ def workload_config(z, l2_note=True):
                                                   z["rope"]["S"], z["qk"]["S"]),
         "l2": "no flush: every input tensor is larger than the 126 MB L2 and consecutive kernels touch "
               "different tensors" if l2_note else "n/a",
-        "seed": "seed = rank",
+        "seed": "seed 0 on every rank; rank r holds shard r of one global problem",
     }
 
 
@@ -118,18 +120,38 @@ FAMILY = {"rmsnorm_fwd": "rms", "rmsnorm_gemma_fwd": "rms", "rmsnorm_bwd": "rms"
           "qknorm_rope_fwd": "qk", "qknorm_rope_bwd": "qk"}
 
 
-def gen_inputs(z, seed, families=("rms", "ln", "rope", "qk")):
-    r, l, o, q = z["rms"], z["ln"], z["rope"], z["qk"]
+def global_sizes(z, ws):
+    """The global problem of a run on ws ranks: ws times the per-GPU rows and tokens."""
+    return {"rms": dict(z["rms"], M=z["rms"]["M"] * ws), "ln": dict(z["ln"], M=z["ln"]["M"] * ws),
+            "rope": dict(z["rope"], S=z["rope"]["S"] * ws), "qk": dict(z["qk"], S=z["qk"]["S"] * ws)}
+
+
+def shard_ranges(z, ws, rank):
+    """Rank `rank`'s contiguous shard of the global problem (the token partition of the path):
+    rows of the norm workloads, tokens of the rotary workloads (each with the table rows of its
+    positions). With the global sizes ws times the per-GPU ones, every shard has the per-GPU
+    size."""
+    from transformer_norm_rope_b200.shard import shard_bounds
+
+    g = global_sizes(z, ws)
+    return {"rms": shard_bounds(g["rms"]["M"], ws, rank), "ln": shard_bounds(g["ln"]["M"], ws, rank),
+            "rope": shard_bounds(g["rope"]["S"], ws, rank), "qk": shard_bounds(g["qk"]["S"], ws, rank)}
+
+
+def gen_inputs(z, seed, families=("rms", "ln", "rope", "qk"), ws=1, rank=0):
+    """Host inputs of rank `rank` of `ws`: its shard of the global problem, from `seed`."""
+    g, sh = global_sizes(z, ws), shard_ranges(z, ws, rank)
+    r, l, o, q = g["rms"], g["ln"], g["rope"], g["qk"]
     d = {}
     if "rms" in families:
-        d["rms"] = wl.rmsnorm(M=r["M"], N=r["N"], dtype="bf16", seed=seed)
+        d["rms"] = wl.rmsnorm(M=r["M"], N=r["N"], dtype="bf16", seed=seed, rows=sh["rms"])
         d["rms_gemma_w"] = wl.normal(seed, wl.S_W, r["N"], "bf16", scale=0.1)
     if "ln" in families:
-        d["ln"] = wl.layernorm(M=l["M"], N=l["N"], dtype="bf16", seed=seed)
+        d["ln"] = wl.layernorm(M=l["M"], N=l["N"], dtype="bf16", seed=seed, rows=sh["ln"])
     if "rope" in families:
-        d["rope"] = wl.rope(**o, dtype="bf16", seed=seed)
+        d["rope"] = wl.rope(**o, dtype="bf16", seed=seed, tokens=sh["rope"])
     if "qk" in families:
-        d["qk"] = wl.qknorm_rope(**q, dtype="bf16", seed=seed)
+        d["qk"] = wl.qknorm_rope(**q, dtype="bf16", seed=seed, tokens=sh["qk"])
     return d
 
 
@@ -365,8 +387,9 @@ def throughput_gbs(bytes_per_rank, elapsed_s, ws, device):
 def parallelism(ws):
     if ws == 1:
         return "single GPU"
-    return (f"data parallel x{ws} (weak): each GPU runs the step on its own shard of the same shapes; "
-            "the step's weight gradients are summed by one NCCL all-reduce")
+    return (f"token-sharded data parallel x{ws} (weak): one global problem of {ws}x the per-GPU rows and "
+            "tokens; rank r owns its r-th contiguous range of rows and tokens (RoPE tables sliced to its "
+            "positions); the step's weight gradients are summed by one NCCL all-reduce")
 
 
 def norm_linear_measure(gn, torch, dev, scale, seed, reps=10):
@@ -481,7 +504,7 @@ def run_ours(args):
     gn.load()
     z = sizes(args.scale)
     kernels = [k for k in ORDER if not args.only or k in args.only.split(",")]
-    host = gen_inputs(z, args.seed + rank, {FAMILY[k] for k in kernels})
+    host = gen_inputs(z, args.seed, {FAMILY[k] for k in kernels}, ws, rank)
     suite = Suite(gn, torch, z, host, dev, kernels)
     nbytes = algorithmic_bytes(z)
     step_bytes = sum(nbytes[k] for k in kernels)
@@ -529,7 +552,7 @@ def run_ours(args):
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(elapsed / args.steps * 1e3, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded generator, seed = rank)",
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded generator, seed 0; rank r generates shard r of one global problem)",
         "config": dict(workload_config(z), parallelism=parallelism(ws), bytes_per_step_per_gpu=step_bytes),
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(ach / peak, 4), "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs"},
@@ -543,14 +566,14 @@ def run_ours(args):
     }
     if not args.no_e2e:
         out["e2e"] = e2e(args, suite, kernels, step_bytes, ws, dev)
-    if not args.no_next and not args.only:
+    if not args.no_next and not args.only and ws == 1:  # single-GPU measurements, not part of the step
         del suite  # free the step's buffers first
         torch.cuda.empty_cache()
-        out["next_norm_linear"] = norm_linear_measure(gn, torch, dev, args.scale, args.seed + rank)
+        out["next_norm_linear"] = norm_linear_measure(gn, torch, dev, args.scale, args.seed)
         torch.cuda.empty_cache()
-        out["next_tiled_linear"] = tiled_linear_measure(gn, torch, dev, args.scale, args.seed + rank)
+        out["next_tiled_linear"] = tiled_linear_measure(gn, torch, dev, args.scale, args.seed)
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(host, z, kernels, budget_s=15.0)
+        out["cpu_baseline"] = cpu_baseline(host, z, kernels, budget_s=15.0, seed=args.seed)
     if rank == 0:
         print(json.dumps(out), flush=True)
     if ws > 1:
@@ -673,67 +696,158 @@ OUTPUTS = {
 
 # ---------------------------------------------------------------- the fp64 CPU oracle arm
 
+def _units(z, k):
+    fam = FAMILY[k]
+    return z[fam]["M"] if fam in ("rms", "ln") else z[fam]["S"]
+
+
+def oracle_range(host, z, k, lo, hi):
+    """Runs the oracle for kernel k on rows (norms) or tokens (rotary) [lo, hi) of the host
+    inputs; returns the algorithmic bytes of that range (the kernel's bytes pro rata)."""
+    import oracle
+
+    if hi <= lo:
+        return 0.0
+    if k.startswith("rmsnorm"):
+        r = host["rms"]
+        w = host["rms_gemma_w"] if "gemma" in k else r["w"]
+        g = "gemma" in k
+        if k.endswith("fwd"):
+            oracle.rmsnorm_fwd(r["x"][lo:hi], w, 1e-6, gemma=g)
+        else:
+            oracle.rmsnorm_bwd(r["x"][lo:hi], w, r["dy"][lo:hi], 1e-6, gemma=g)
+    elif k.startswith("layernorm"):
+        l = host["ln"]  # noqa: E741
+        if k.endswith("fwd"):
+            oracle.layernorm_fwd(l["x"][lo:hi], l["w"], l["b"], 1e-5, act="gelu_tanh")
+        else:
+            oracle.layernorm_bwd(l["x"][lo:hi], l["w"], l["b"], l["dy"][lo:hi], 1e-5, act="gelu_tanh")
+    elif k.startswith("rope"):
+        o = host["rope"]
+        sign = 1 if k == "rope_fwd" else -1
+        oracle.rope(o["q"][:, lo:hi], o["cos"][lo:hi], o["sin"][lo:hi], sign)
+        oracle.rope(o["k"][:, lo:hi], o["cos"][lo:hi], o["sin"][lo:hi], sign)
+    else:
+        q = host["qk"]
+        for x, w, dy in (("q", "wq", "dq_out"), ("k", "wk", "dk_out")):
+            if k.endswith("fwd"):
+                oracle.qknorm_rope_fwd(q[x][:, lo:hi], q[w], q["cos"][lo:hi], q["sin"][lo:hi], 1e-6)
+            else:
+                oracle.qknorm_rope_bwd(q[x][:, lo:hi], q[w], q["cos"][lo:hi], q["sin"][lo:hi], q[dy][:, lo:hi], 1e-6)
+    return algorithmic_bytes(z)[k] * (hi - lo) / _units(z, k)
+
+
 def oracle_step(host, z, kernels, frac):
     """Runs the oracle on the first `frac` of the rows/tokens of each kernel; returns
     (seconds, algorithmic bytes of the sample)."""
-    import oracle
-
-    nb = algorithmic_bytes(z)
     done, t = 0.0, 0.0
-    r, l, o, q = host["rms"], host["ln"], host["rope"], host["qk"]
     for k in kernels:
-        if k.startswith("rmsnorm"):
-            M = z["rms"]["M"]
-            m = max(1, int(M * frac))
-            w = host["rms_gemma_w"] if "gemma" in k else r["w"]
-            g = "gemma" in k
-            s = time.perf_counter()
-            if k.endswith("fwd"):
-                oracle.rmsnorm_fwd(r["x"][:m], w, 1e-6, gemma=g)
-            else:
-                oracle.rmsnorm_bwd(r["x"][:m], w, r["dy"][:m], 1e-6, gemma=g)
-            t += time.perf_counter() - s
-            done += nb[k] * m / M
-        elif k.startswith("layernorm"):
-            M = z["ln"]["M"]
-            m = max(1, int(M * frac))
-            s = time.perf_counter()
-            if k.endswith("fwd"):
-                oracle.layernorm_fwd(l["x"][:m], l["w"], l["b"], 1e-5, act="gelu_tanh")
-            else:
-                oracle.layernorm_bwd(l["x"][:m], l["w"], l["b"], l["dy"][:m], 1e-5, act="gelu_tanh")
-            t += time.perf_counter() - s
-            done += nb[k] * m / M
-        elif k.startswith("rope"):
-            S = z["rope"]["S"]
-            m = max(1, int(S * frac))
-            sign = 1 if k == "rope_fwd" else -1
-            s = time.perf_counter()
-            oracle.rope(o["q"][:, :m], o["cos"][:m], o["sin"][:m], sign)
-            oracle.rope(o["k"][:, :m], o["cos"][:m], o["sin"][:m], sign)
-            t += time.perf_counter() - s
-            done += nb[k] * m / S
-        else:
-            S = z["qk"]["S"]
-            m = max(1, int(S * frac))
-            s = time.perf_counter()
-            for x, w, dy in (("q", "wq", "dq_out"), ("k", "wk", "dk_out")):
-                if k.endswith("fwd"):
-                    oracle.qknorm_rope_fwd(q[x][:, :m], q[w], q["cos"][:m], q["sin"][:m], 1e-6)
-                else:
-                    oracle.qknorm_rope_bwd(q[x][:, :m], q[w], q["cos"][:m], q["sin"][:m], q[dy][:, :m], 1e-6)
-            t += time.perf_counter() - s
-            done += nb[k] * m / S
+        m = max(1, int(_units(z, k) * frac))
+        s = time.perf_counter()
+        done += oracle_range(host, z, k, 0, m)
+        t += time.perf_counter() - s
     return t, done
 
 
-def cpu_baseline(host, z, kernels, budget_s):
+def _oracle_worker(conn, z, seed, jobs):
+    """One host core of the all-cores oracle run: generates the inputs of its (kernel, lo, hi)
+    ranges, reports ready, waits for the start signal, runs the oracle on them and reports
+    (seconds, bytes)."""
+    try:
+        local = []
+        for k, lo, hi in jobs:
+            fam = FAMILY[k]
+            if fam == "rms":
+                h = {"rms": wl.rmsnorm(M=z["rms"]["M"], N=z["rms"]["N"], dtype="bf16", seed=seed, rows=(lo, hi)),
+                     "rms_gemma_w": wl.normal(seed, wl.S_W, z["rms"]["N"], "bf16", scale=0.1)}
+            elif fam == "ln":
+                h = {"ln": wl.layernorm(M=z["ln"]["M"], N=z["ln"]["N"], dtype="bf16", seed=seed, rows=(lo, hi))}
+            elif fam == "rope":
+                h = {"rope": wl.rope(**z["rope"], dtype="bf16", seed=seed, tokens=(lo, hi))}
+            else:
+                h = {"qk": wl.qknorm_rope(**z["qk"], dtype="bf16", seed=seed, tokens=(lo, hi))}
+            local.append((k, h, hi - lo))
+        conn.send("ready")
+        conn.recv()
+        s = time.perf_counter()
+        done = sum(oracle_range(h, z, k, 0, n) for k, h, n in local)
+        conn.send((time.perf_counter() - s, done))
+    except Exception as e:  # noqa: BLE001 - reported to the parent, which raises
+        conn.send(("error", repr(e)))
+    finally:
+        conn.close()
+
+
+def oracle_all_cores(z, seed, kernels, frac, cores):
+    """The unchanged oracle on `cores` host processes at once: the first `frac` of every
+    kernel's rows/tokens split into `cores` contiguous ranges, one per process. Each process
+    generates its own inputs before the clock starts; the wall time runs from the common start
+    signal until the last process is done. Returns (seconds, bytes)."""
+    import multiprocessing as mp
+
+    jobs = [[] for _ in range(cores)]
+    for k in kernels:
+        m = max(1, int(_units(z, k) * frac))
+        for i in range(cores):
+            lo, hi = m * i // cores, m * (i + 1) // cores
+            if hi > lo:
+                jobs[i].append((k, lo, hi))
+    ctx = mp.get_context("spawn")
+    procs, conns = [], []
+    for i in range(cores):
+        a, b = ctx.Pipe()
+        p = ctx.Process(target=_oracle_worker, args=(b, z, seed, jobs[i]), daemon=True)
+        p.start()
+        procs.append(p)
+        conns.append(a)
+    try:
+        for c in conns:
+            msg = c.recv()
+            if msg != "ready":
+                raise RuntimeError(f"oracle worker failed: {msg}")
+        t0 = time.perf_counter()
+        for c in conns:
+            c.send("go")
+        res = [c.recv() for c in conns]
+        wall = time.perf_counter() - t0
+    finally:
+        for p in procs:
+            p.join(60)
+    bad = [r for r in res if r[0] == "error"]
+    if bad:
+        raise RuntimeError(f"oracle worker failed: {bad[0][1]}")
+    return wall, sum(r[1] for r in res)
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(host, z, kernels, budget_s, seed=0):
+    """The oracle as it stands on the host cores: one thread on a sample sized to about
+    `budget_s`, then every core at once (one process per core) on a sample sized to about
+    budget_s / 2 per core."""
     t, done = oracle_step(host, z, kernels, 1.0 / 4096)
     frac = min(1.0, (1.0 / 4096) * max(1.0, budget_s / max(t, 1e-3)))
     t, done = oracle_step(host, z, kernels, frac)
-    return {"value": round(done / t / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"first {frac:.5f} of the rows/tokens of every kernel of the step ({t:.1f} s of fp64 C oracle, "
-                      "single thread, same seeded inputs)"}
+    single = done / t / 1e9
+    cores = host_cores()
+    frac_all = min(1.0, frac * cores * 0.5)
+    t_all, done_all = oracle_all_cores(z, seed, kernels, frac_all, cores)
+    multi = done_all / t_all / 1e9
+    return {"value": round(multi, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "single_core": {"value": round(single, 4), "cores": 1,
+                            "sample": f"first {frac:.5f} of the rows/tokens of every kernel of the step "
+                                      f"({t:.1f} s of fp64 C oracle, one thread)"},
+            "all_cores": {"value": round(multi, 4), "cores": cores,
+                          "sample": f"first {frac_all:.5f} of the rows/tokens of every kernel of the step, split "
+                                    f"into {cores} contiguous ranges run at once by {cores} processes "
+                                    f"({t_all:.1f} s wall)"},
+            "sample": f"all {cores} host cores (one oracle process each) on the first {frac_all:.5f} of the "
+                      f"rows/tokens of every kernel of the step; same seeded inputs"}
 
 
 def run_reference(args):

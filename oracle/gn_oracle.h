@@ -14,12 +14,12 @@
  *        section "内核一 FlashNorm" (one row per block, one load, sum of squares and its
  *        inverse, times the weight; Gemma +1 offset; per-row inverse statistic saved for the
  *        backward) and section "内核二 FlashRoPE" (interleaved even/odd pairs, in-place
- *        rotation; the inverse rotation is the same kernel with sin negated).
+ *        rotation; the inverse rotation is the same kernel with sin negated), and section
+ *        "内核三 TiledLinear" (linear layer run chunk by chunk along the tokens, the
+ *        backward recomputing each chunk).
  *   [L]  "LLM层的优化算子" (optimized kernels for LLM layers), section "编写定制融合算子"
  *        (fused LayerNorm + GeLU example: centre, biased variance, divide by sqrt(var+eps),
  *        times weight plus bias, tanh-GeLU with constant 0.79788456 and cubic 0.044715).
- *        section "内核三 TiledLinear" (linear layer run chunk by chunk along the tokens, the
- *        backward recomputing each chunk).
  *   [J]  "Janus-Pro-7B模型推理加速实战", section 4.1 (fused LayerNorm + linear + SiLU,
  *        SiLU = x * sigmoid(x)).
  *   [Y]  "HY-Motion 1.0性能优化从算法到硬件的全方位调优策略", section 3.1 (LayerNorm merged

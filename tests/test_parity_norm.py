@@ -3,15 +3,15 @@
 Small cases span several CTAs and row tiles, ragged tails (hidden not a multiple of the
 16-byte vector), both launch shapes (lane group per row for short rows, CTA per row with the
 TMA pipeline for long rows), strided rows, in-place outputs and empty inputs. The full-size
-cases run the exact launch configuration the benchmark times and compare sampled rows, every
-saved statistic and the complete weight gradients.
+cases run the exact launch configuration the benchmark times and compare every output element,
+every saved statistic and the complete weight gradients with the oracle.
 """
-import numpy as np
 import pytest
 import torch
 
 import oracle
 from transformer_norm_rope_b200 import workloads as wl
+from tests import _fullsize as fs
 from tests._util import assert_close, grad_tol, io_tol, to_dev, to_np, wgrad_tol
 
 
@@ -134,55 +134,53 @@ def test_deterministic_weight_gradients(gpu):
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
 
 
-def _sample_rows(M, outlier_scale, k=48, seed=7):
-    rows = set(np.random.default_rng(seed).choice(M, k, replace=False).tolist())
-    rows |= {0, 1, M - 1}
-    rows |= set(np.nonzero(outlier_scale > 1)[0][:8].tolist())
-    return np.array(sorted(rows))
-
-
 @pytest.mark.slow
 @pytest.mark.parametrize("gemma", [False, True])
 def test_rmsnorm_full_size(gpu, gemma):
+    """The benchmark's launch (x[15360, 5120] bf16, 1% outlier rows): y, inv_rms and dx on every
+    row against the oracle (chunks of rows on host worker processes), dw complete."""
     cfg = wl.RMSNORM_MAIN
     d = wl.rmsnorm(M=cfg["M"], N=cfg["N"], dtype="bf16", gemma=gemma)
     x, w, dy = to_dev(d["x"]), to_dev(d["w"]), to_dev(d["dy"])
     y, r = gpu.rmsnorm_fwd(x, w, d["eps"], gemma=gemma)
     dx, dw = gpu.rmsnorm_bwd(x, w, r, dy, gemma=gemma)
     torch.cuda.synchronize()
-    rows = _sample_rows(cfg["M"], wl.outlier_rows(0, cfg["M"]))
-    ry, _ = oracle.rmsnorm_fwd(d["x"][rows], d["w"], d["eps"], gemma=gemma)
-    rdx, _ = oracle.rmsnorm_bwd(d["x"][rows], d["w"], d["dy"][rows], d["eps"], gemma=gemma)
-    _, rr = oracle.rmsnorm_fwd(d["x"], d["w"], d["eps"], gemma=gemma)
-    _, rdw = oracle.rmsnorm_bwd(d["x"], d["w"], d["dy"], d["eps"], gemma=gemma, want_dx=False)
-    idx = torch.from_numpy(rows).cuda()
-    assert_close(to_np(y[idx]), ry, "bf16", "full rms y")
-    assert_close(to_np(dx[idx]), rdx, "grad_bf16", "full rms dx")
-    assert_close(to_np(r), rr, "stat", "full rms inv_rms (all rows)")
-    assert_close(to_np(dw), rdw, "grad_bf16", "full rms dw")
+    M, N = x.shape
+
+    def jobs():
+        for r0, r1 in fs.row_chunks(M, N):
+            yield fs.job_rms, (d["x"][r0:r1], d["w"], d["dy"][r0:r1], d["eps"], gemma, fs.bits(y[r0:r1]),
+                               fs.bits(r[r0:r1]), fs.bits(dx[r0:r1]), f"rows {r0}:{r1}")
+
+    v = fs.run(jobs(), f"full rms gemma={gemma}")
+    n = v.assert_ok()
+    assert n == {"y": M * N, "inv_rms": M, "dx": M * N}
+    assert_close(to_np(dw), v.parts["dw"], "grad_bf16", "full rms dw")
 
 
 @pytest.mark.slow
 def test_layernorm_full_size(gpu):
+    """The benchmark's launch (x[32768, 5120] bf16, tanh-GeLU): y, mean, rstd and dx on every row
+    against the oracle, dw and db complete."""
     cfg = wl.LAYERNORM_MAIN
     d = wl.layernorm(M=cfg["M"], N=cfg["N"], dtype="bf16")
     x, w, b, dy = (to_dev(d[k]) for k in ("x", "w", "b", "dy"))
     y, mu, rs = gpu.layernorm_fwd(x, w, b, d["eps"], epilogue="gelu_tanh")
     dx, dw, db = gpu.layernorm_bwd(x, w, b, mu, rs, dy, epilogue="gelu_tanh")
     torch.cuda.synchronize()
-    rows = _sample_rows(cfg["M"], np.ones(cfg["M"]))
-    ry, _, _ = oracle.layernorm_fwd(d["x"][rows], d["w"], d["b"], d["eps"], act="gelu_tanh")
-    rdx, _, _ = oracle.layernorm_bwd(d["x"][rows], d["w"], d["b"], d["dy"][rows], d["eps"], act="gelu_tanh")
-    _, rmu, rrs = oracle.layernorm_fwd(d["x"], d["w"], d["b"], d["eps"], act="gelu_tanh")
-    _, rdw, rdb = oracle.layernorm_bwd(d["x"], d["w"], d["b"], d["dy"], d["eps"], act="gelu_tanh",
-                                       want_dx=False)
-    idx = torch.from_numpy(rows).cuda()
-    assert_close(to_np(y[idx]), ry, "bf16", "full ln y")
-    assert_close(to_np(dx[idx]), rdx, "grad_bf16", "full ln dx")
-    assert_close(to_np(mu), rmu, (1e-5, 1e-6), "full ln mean")
-    assert_close(to_np(rs), rrs, "stat", "full ln rstd")
-    assert_close(to_np(dw), rdw, "grad_bf16", "full ln dw")
-    assert_close(to_np(db), rdb, "grad_bf16", "full ln db")
+    M, N = x.shape
+
+    def jobs():
+        for r0, r1 in fs.row_chunks(M, N):
+            yield fs.job_ln, (d["x"][r0:r1], d["w"], d["b"], d["dy"][r0:r1], d["eps"], "gelu_tanh",
+                              fs.bits(y[r0:r1]), fs.bits(mu[r0:r1]), fs.bits(rs[r0:r1]), fs.bits(dx[r0:r1]),
+                              f"rows {r0}:{r1}")
+
+    v = fs.run(jobs(), "full ln")
+    n = v.assert_ok()
+    assert n == {"y": M * N, "mean": M, "rstd": M, "dx": M * N}
+    assert_close(to_np(dw), v.parts["dw"], "grad_bf16", "full ln dw")
+    assert_close(to_np(db), v.parts["db"], "grad_bf16", "full ln db")
 
 
 def _shifted(t):

@@ -4,7 +4,7 @@ Small cases cover several units per CTA and several CTAs, one or two tensors (k 
 absent), head dims from 8 to 264 (including widths whose lanes per head are not a power of
 two, for the plain rotation), slabs split across heads (the backward stages four tensors),
 and empty inputs. The full-size cases run the benchmark's launch configuration and compare
-sampled tokens, every saved statistic and the complete weight gradients.
+every output element, every saved statistic and the complete weight gradients with the oracle.
 """
 import numpy as np
 import pytest
@@ -12,6 +12,7 @@ import torch
 
 import oracle
 from transformer_norm_rope_b200 import workloads as wl
+from tests import _fullsize as fs
 from tests._util import assert_close, grad_tol, io_tol, to_dev, to_np, wgrad_tol
 
 pytestmark = pytest.mark.gpu
@@ -69,11 +70,7 @@ def test_rope_empty(gpu):
 
 
 QK_SHAPES = [(2, 37, 5, 128, "bf16"), (1, 64, 40, 128, "bf16"), (1, 50, 8, 128, "f32"), (2, 21, 3, 64, "bf16"),
-             (1, 30, 4, 8, "bf16"), (1, 19, 7, 32, "f32")]
-
-
-def _bits(t, dtype):
-    return t.cpu().view(torch.int16).numpy().view(np.uint16) if dtype == "bf16" else t.cpu().numpy()
+             (1, 30, 4, 8, "bf16"), (1, 19, 7, 32, "f32"), (1, 24, 4, 256, "bf16")]
 
 
 @pytest.mark.parametrize("B,S,H,D,dtype", QK_SHAPES)
@@ -124,40 +121,39 @@ def test_qknorm_unsupported_head_dim(gpu):
     assert e.value.status == gpu.GN_ERR_UNSUPPORTED
 
 
-def _sample_tokens(B, S, k=24, seed=11):
-    rng = np.random.default_rng(seed)
-    toks = {(0, 0), (B - 1, S - 1), (0, 1)}
-    toks |= {(int(b), int(s)) for b, s in zip(rng.integers(0, B, k), rng.integers(0, S, k))}
-    return sorted(toks)
-
-
 @pytest.mark.slow
 def test_rope_full_size(gpu):
+    """The benchmark's launch (q, k [1, 32760, 40, 128] bf16): the forward on every element
+    against the oracle, the backward on every element against the oracle applied to the
+    forward's bf16 output (the backward's actual input), and the round-trip bound on every
+    element."""
     c = wl.ROPE_MAIN
     d = wl.rope(**c)
     q, k = to_dev(d["q"]), to_dev(d["k"])
     cos, sin = to_dev(d["cos"]), to_dev(d["sin"])
     gpu.rope_apply_(q, k, cos, sin, +1)
-    torch.cuda.synchronize()
-    for b, s in _sample_tokens(c["B"], c["S"]):
-        for name, t in (("q", q), ("k", k)):
-            ref = oracle.rope(d[name][b:b + 1, s:s + 1], d["cos"][s:s + 1], d["sin"][s:s + 1], +1)
-            assert_close(to_np(t[b:b + 1, s:s + 1]), ref, "bf16", f"full rope {name} token {b},{s}")
-    # the backward: against the oracle applied to the forward's bf16 output on sampled
-    # tokens, and the round-trip bound on every element
-    toks = _sample_tokens(c["B"], c["S"])
-    fwd = {name: [_bits(t[b:b + 1, s:s + 1], "bf16") for b, s in toks] for name, t in (("q", q), ("k", k))}
+    qf, kf = q.clone(), k.clone()
     gpu.rope_apply_(q, k, cos, sin, -1)
     torch.cuda.synchronize()
+    B, S, H, D = q.shape
+
+    def jobs():
+        for name, fwd, bwd in (("q", qf, q), ("k", kf, k)):
+            for s0, s1 in fs.token_chunks(S, B * H * D):
+                yield fs.job_rope, (d[name][:, s0:s1], d["cos"][s0:s1], d["sin"][s0:s1], fs.bits(fwd[:, s0:s1]),
+                                    fs.bits(bwd[:, s0:s1]), f"{name} tokens {s0}:{s1}")
+
+    n = fs.run(jobs(), "full rope").assert_ok()
+    assert n == {"fwd": 2 * B * S * H * D, "bwd": 2 * B * S * H * D}
     for name, t in (("q", q), ("k", k)):
-        for (b, s), f in zip(toks, fwd[name]):
-            ref = oracle.rope(f, d["cos"][s:s + 1], d["sin"][s:s + 1], -1)
-            assert_close(to_np(t[b:b + 1, s:s + 1]), ref, "bf16", f"full rope bwd {name} token {b},{s}")
         assert_undone(t, to_dev(d[name]), "bf16", f"full rope bwd(fwd) {name}")
 
 
 @pytest.mark.slow
 def test_qknorm_rope_full_size(gpu):
+    """The benchmark's launch (q, k [2, 76800, 40, 128] bf16): out, inv_rms and dx of both
+    tensors on every element against the oracle (chunks of tokens on host worker processes),
+    dw_q and dw_k complete."""
     c = wl.QKNORM_MAIN
     d = wl.qknorm_rope(**c)
     q, k, wq, wk = (to_dev(d[n]) for n in ("q", "k", "wq", "wk"))
@@ -165,18 +161,16 @@ def test_qknorm_rope_full_size(gpu):
     qo, ko, rq, rk = gpu.qknorm_rope_fwd(q, k, wq, wk, cos, sin, d["eps"])
     dq, dk, dwq, dwk = gpu.qknorm_rope_bwd(q, k, wq, wk, cos, sin, rq, rk, to_dev(d["dq_out"]), to_dev(d["dk_out"]))
     torch.cuda.synchronize()
+    B, S, H, D = q.shape
     for name, x, w, dy, out, r, dx, dw in (("q", "q", "wq", "dq_out", qo, rq, dq, dwq),
                                            ("k", "k", "wk", "dk_out", ko, rk, dk, dwk)):
-        for b, s in _sample_tokens(c["B"], c["S"]):
-            xs = d[x][b:b + 1, s:s + 1]
-            ro, rr = oracle.qknorm_rope_fwd(xs, d[w], d["cos"][s:s + 1], d["sin"][s:s + 1], d["eps"])
-            rdx, _ = oracle.qknorm_rope_bwd(xs, d[w], d["cos"][s:s + 1], d["sin"][s:s + 1], d[dy][b:b + 1, s:s + 1],
-                                            d["eps"])
-            tag = f"full qk {name} token {b},{s}"
-            assert_close(to_np(out[b:b + 1, s:s + 1]), ro, "bf16", tag + " out")
-            assert_close(to_np(r[b:b + 1, s:s + 1]), rr, "stat", tag + " inv_rms")
-            assert_close(to_np(dx[b:b + 1, s:s + 1]), rdx, "grad_bf16", tag + " dx")
-        _, rr_all = oracle.qknorm_rope_fwd(d[x], d[w], d["cos"], d["sin"], d["eps"], want_out=False)
-        assert_close(to_np(r), rr_all, "stat", f"full qk {name} inv_rms (all rows)")
-        _, rdw = oracle.qknorm_rope_bwd(d[x], d[w], d["cos"], d["sin"], d[dy], d["eps"], want_dx=False)
-        assert_close(to_np(dw), rdw, "grad_bf16", f"full qk {name} dw")
+        def jobs():
+            for s0, s1 in fs.token_chunks(S, B * H * D):
+                yield fs.job_qk, (d[x][:, s0:s1], d[w], d["cos"][s0:s1], d["sin"][s0:s1], d[dy][:, s0:s1], d["eps"],
+                                  False, fs.bits(out[:, s0:s1]), fs.bits(r[:, s0:s1]), fs.bits(dx[:, s0:s1]),
+                                  f"{name} tokens {s0}:{s1}")
+
+        v = fs.run(jobs(), f"full qk {name}")
+        n = v.assert_ok()
+        assert n == {"out": B * S * H * D, "inv_rms": B * S * H, "dx": B * S * H * D}
+        assert_close(to_np(dw), v.parts["dw"], "grad_bf16", f"full qk {name} dw")

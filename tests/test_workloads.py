@@ -75,3 +75,30 @@ def test_norm_linear_recipe():
     e = wl.norm_linear(M=8, N=96, K=512, seed=3)
     np.testing.assert_array_equal(e["W"], d["W"])  # weights do not depend on the row count
     assert not np.array_equal(wl.norm_linear(M=8, N=96, K=512, seed=4)["W"], d["W"])
+
+
+def test_row_and_token_ranges_are_slices_of_the_whole():
+    # ranges cross chunk boundaries (CHUNK = 4 Mi elements) and keep the global outlier rows,
+    # row statistics and table positions
+    M, N = 1000, 5120
+    full = wl.rmsnorm(M=M, N=N, seed=2)
+    part = wl.rmsnorm(M=M, N=N, seed=2, rows=(811, 997))
+    np.testing.assert_array_equal(part["x"], full["x"][811:997])
+    np.testing.assert_array_equal(part["dy"], full["dy"][811:997])
+    np.testing.assert_array_equal(part["w"], full["w"])
+    full = wl.layernorm(M=900, N=5120, seed=1)
+    part = wl.layernorm(M=900, N=5120, seed=1, rows=(3, 850))
+    np.testing.assert_array_equal(part["x"], full["x"][3:850])
+    np.testing.assert_array_equal(part["dy"], full["dy"][3:850])
+    full = wl.rope(B=2, S=900, H=40, D=128, seed=5)
+    part = wl.rope(B=2, S=900, H=40, D=128, seed=5, tokens=(450, 900))
+    for k in ("q", "k"):
+        np.testing.assert_array_equal(part[k], full[k][:, 450:900])
+    for k in ("cos", "sin"):
+        np.testing.assert_array_equal(part[k], full[k][450:900])
+    full = wl.qknorm_rope(B=2, S=900, H=40, D=128, seed=6)
+    part = wl.qknorm_rope(B=2, S=900, H=40, D=128, seed=6, tokens=(1, 420))
+    for k in ("q", "k", "dq_out", "dk_out"):
+        np.testing.assert_array_equal(part[k], full[k][:, 1:420])
+    for k in ("cos", "sin", "wq", "wk"):
+        np.testing.assert_array_equal(part[k], full[k][1:420] if k in ("cos", "sin") else full[k])

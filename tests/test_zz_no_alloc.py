@@ -3,54 +3,116 @@
 allocator owns). It keeps its per-block partial sums in a fixed array inside the library
 instead of a caller workspace. This file is collected last on purpose.
 
-The test calls both C entry points directly (ctypes, raw device pointers) on the same inputs
-and requires the no-allocation variant to match the workspace variant within the gradient
-tolerance, on two calls in a row (the second call reuses the array the first one filled).
+The tests call both C entry points directly (ctypes, raw device pointers) on the same inputs.
+Both run the same kernel on the same grid and sum the partials in the same fixed order, so the
+no-allocation variant must give the workspace variant's results bit for bit: on two calls in a
+row (the second call reuses the array the first one filled), with and without k, and it must
+refuse, before launching anything, a call whose partials would not fit the array.
 """
-import numpy as np
 import pytest
 import torch
 
 from transformer_norm_rope_b200 import workloads as wl
-from tests._util import assert_close, to_dev, to_np
+from tests._util import to_dev
 
 pytestmark = pytest.mark.gpu
 
+FIXED_BYTES = 1 << 20  # size of the library's fixed partial-sum array
 
-def test_noalloc_backward_matches_workspace_backward(gpu):
-    d = wl.qknorm_rope(B=2, S=96, H=40, D=128, dtype="bf16", seed=3)
-    q, k, wq, wk = (to_dev(d[n]) for n in ("q", "k", "wq", "wk"))
-    cos, sin = to_dev(d["cos"]), to_dev(d["sin"])
-    dqo, dko = to_dev(d["dq_out"]), to_dev(d["dk_out"])
-    _, _, rq, rk = gpu.qknorm_rope_fwd(q, k, wq, wk, cos, sin, d["eps"])
+
+def _inputs(gpu, B, S, H, D, seed):
+    d = wl.qknorm_rope(B=B, S=S, H=H, D=D, dtype="bf16", seed=seed)
+    t = {n: to_dev(d[n]) for n in ("q", "k", "wq", "wk", "cos", "sin", "dq_out", "dk_out")}
+    _, _, t["rq"], t["rk"] = gpu.qknorm_rope_fwd(t["q"], t["k"], t["wq"], t["wk"], t["cos"], t["sin"], d["eps"])
+    return t
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _outputs(q, with_k, D):
+    nan = float("nan")
+    dq = torch.full_like(q, nan)
+    dk = torch.full_like(q, nan) if with_k else None
+    dwq = torch.full((D,), nan, dtype=torch.float32, device=q.device)
+    dwk = torch.full((D,), nan, dtype=torch.float32, device=q.device) if with_k else None
+    return dq, dk, dwq, dwk
+
+
+def _call_ws(gpu, t, with_k, stream):
+    q = t["q"]
     B, S, H, D = q.shape
-    stream = torch.cuda.current_stream().cuda_stream
-
-    # reference: the entry point with a caller-owned workspace
-    dq0, dk0 = torch.empty_like(q), torch.empty_like(k)
-    dwq0 = torch.empty(D, dtype=torch.float32, device="cuda")
-    dwk0 = torch.empty(D, dtype=torch.float32, device="cuda")
+    k = t["k"] if with_k else None
+    dq, dk, dwq, dwk = _outputs(q, with_k, D)
     nws = gpu.gn_qknorm_rope_bwd_workspace(B, S, H, D, gpu.GN_BF16)
-    ws = torch.empty(nws, dtype=torch.uint8, device="cuda")
-    gpu.check(gpu.gn_qknorm_rope_bwd(q.data_ptr(), k.data_ptr(), wq.data_ptr(), wk.data_ptr(), cos.data_ptr(),
-                                     sin.data_ptr(), rq.data_ptr(), rk.data_ptr(), dqo.data_ptr(), dko.data_ptr(),
-                                     dq0.data_ptr(), dk0.data_ptr(), dwq0.data_ptr(), dwk0.data_ptr(),
-                                     ws.data_ptr(), nws, B, S, H, D, 0, gpu.GN_BF16, stream))
-    torch.cuda.synchronize()
+    ws = torch.empty(nws, dtype=torch.uint8, device=q.device)
+    gpu.check(gpu.gn_qknorm_rope_bwd(q.data_ptr(), _ptr(k), t["wq"].data_ptr(), _ptr(t["wk"] if with_k else None),
+                                     t["cos"].data_ptr(), t["sin"].data_ptr(), t["rq"].data_ptr(),
+                                     _ptr(t["rk"] if with_k else None), t["dq_out"].data_ptr(),
+                                     _ptr(t["dk_out"] if with_k else None), dq.data_ptr(), _ptr(dk), dwq.data_ptr(),
+                                     _ptr(dwk), ws.data_ptr(), nws, B, S, H, D, 0, gpu.GN_BF16, stream),
+              "gn_qknorm_rope_bwd")
+    return dq, dk, dwq, dwk
 
+
+def _call_noalloc(gpu, t, with_k, stream, outs=None):
+    q = t["q"]
+    B, S, H, D = q.shape
+    k = t["k"] if with_k else None
+    dq, dk, dwq, dwk = outs if outs is not None else _outputs(q, with_k, D)
+    st = gpu.gn_qknorm_rope_bwd_noalloc(q.data_ptr(), _ptr(k), t["wq"].data_ptr(),
+                                        _ptr(t["wk"] if with_k else None), t["cos"].data_ptr(), t["sin"].data_ptr(),
+                                        t["rq"].data_ptr(), _ptr(t["rk"] if with_k else None),
+                                        t["dq_out"].data_ptr(), _ptr(t["dk_out"] if with_k else None), dq.data_ptr(),
+                                        _ptr(dk), dwq.data_ptr(), _ptr(dwk), B, S, H, D, 0, gpu.GN_BF16, stream)
+    return st, (dq, dk, dwq, dwk)
+
+
+@pytest.mark.parametrize("with_k", [True, False])
+def test_noalloc_backward_matches_workspace_backward(gpu, with_k):
+    t = _inputs(gpu, B=2, S=96, H=40, D=128, seed=3)
+    stream = torch.cuda.current_stream().cuda_stream
+    ref = _call_ws(gpu, t, with_k, stream)
+    torch.cuda.synchronize()
     for call in range(2):
-        dq, dk = torch.full_like(q, float("nan")), torch.full_like(k, float("nan"))
-        dwq = torch.full((D,), float("nan"), dtype=torch.float32, device="cuda")
-        dwk = torch.full((D,), float("nan"), dtype=torch.float32, device="cuda")
-        gpu.check(gpu.gn_qknorm_rope_bwd_noalloc(q.data_ptr(), k.data_ptr(), wq.data_ptr(), wk.data_ptr(),
-                                                 cos.data_ptr(), sin.data_ptr(), rq.data_ptr(), rk.data_ptr(),
-                                                 dqo.data_ptr(), dko.data_ptr(), dq.data_ptr(), dk.data_ptr(),
-                                                 dwq.data_ptr(), dwk.data_ptr(), B, S, H, D, 0, gpu.GN_BF16,
-                                                 stream), "gn_qknorm_rope_bwd_noalloc")
+        st, got = _call_noalloc(gpu, t, with_k, stream)
+        gpu.check(st, "gn_qknorm_rope_bwd_noalloc")
         torch.cuda.synchronize()
-        tag = f"no-alloc call {call + 1}"
-        assert_close(to_np(dq), to_np(dq0), "grad_bf16", tag + " dq")
-        assert_close(to_np(dk), to_np(dk0), "grad_bf16", tag + " dk")
-        assert_close(to_np(dwq), to_np(dwq0), "grad_bf16", tag + " dwq")
-        assert_close(to_np(dwk), to_np(dwk0), "grad_bf16", tag + " dwk")
+        for name, a, b in zip(("dq", "dk", "dwq", "dwk"), got, ref):
+            if b is None:
+                assert a is None
+                continue
+            assert torch.equal(a, b), f"no-alloc call {call + 1} (k {'given' if with_k else 'absent'}): {name} differs"
+    assert gpu.device_error() == 0
+
+
+def test_noalloc_refuses_partials_beyond_the_fixed_array(gpu):
+    """A call whose per-block partials (2 * D * 4 bytes for each block of the persistent grid)
+    exceed the fixed array returns GN_ERR_WORKSPACE and leaves every output untouched. Head dim
+    256 with short units and four consumer warps per block makes a grid of more than 512 blocks
+    (found through the workspace query, which reports grid * 2 * D * 4 bytes)."""
+    B, S, H, D = 1, 4096, 4, 256
+    t = _inputs(gpu, B=B, S=S, H=H, D=D, seed=5)
+    stream = torch.cuda.current_stream().cuda_stream
+    found = None
+    try:
+        for unit_bytes, group_rows, stages in ((0, 0, 0), (2048, 4, 0), (2048, 4, 2), (1024, 4, 2)):
+            gpu.tune("unit_bytes", unit_bytes)
+            gpu.tune("group_rows", group_rows)
+            gpu.tune("stages", stages)
+            need = gpu.gn_qknorm_rope_bwd_workspace(B, S, H, D, gpu.GN_BF16)
+            if need > FIXED_BYTES * 5 // 4:
+                found = (unit_bytes, group_rows, stages, need)
+                break
+        assert found is not None, "no launch shape on this device needs more than the fixed array"
+        outs = _outputs(t["q"], True, D)
+        st, outs = _call_noalloc(gpu, t, True, stream, outs)
+        torch.cuda.synchronize()
+        assert st == gpu.GN_ERR_WORKSPACE, f"{found}: status {st}"
+        for o in outs:  # nothing was launched: the NaN fill is intact
+            assert torch.isnan(o).all()
+    finally:
+        for key in ("unit_bytes", "group_rows", "stages"):
+            gpu.tune(key, 0)
     assert gpu.device_error() == 0

@@ -892,10 +892,17 @@ extern "C" gn_status gn_norm_linear_fwd(const void* x, const void* Wf, const flo
       !make_map(&tb, Wf, N, K, K, pair ? 128u : (uint32_t)kBN))
     return GN_ERR_CUDA;
   void* kern = pair ? pick_pair(norm, epi) : mh == 2 ? pick<2>(norm, epi) : pick<1>(norm, epi);
-  static std::once_flag attr_once;
-  static bool attr_ok = true;
-  std::call_once(attr_once, [] { attr_ok = set_smem_attr<1>() && set_smem_attr<2>() && set_pair_smem_attr(); });
-  if (!attr_ok) return GN_ERR_CUDA;
+  // the dynamic shared-memory limits are attributes of the kernels on the current device: set
+  // them once per device (0 = not yet, 1 = set, -1 = failed)
+  static std::mutex attr_mu;
+  static signed char attr_state[64];
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GN_ERR_CUDA;
+  {
+    std::lock_guard<std::mutex> lk(attr_mu);
+    if (!attr_state[dev]) attr_state[dev] = set_smem_attr<1>() && set_smem_attr<2>() && set_pair_smem_attr() ? 1 : -1;
+    if (attr_state[dev] < 0) return GN_ERR_CUDA;
+  }
   NlArgs a{};
   a.c = c, a.d = d;
   a.y = static_cast<__nv_bfloat16*>(y);

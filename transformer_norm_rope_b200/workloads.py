@@ -59,33 +59,45 @@ def _gen(seed: int, stream: int, chunk: int) -> np.random.Generator:
     return np.random.Generator(np.random.Philox(key=[int(seed), (int(stream) << 32) | int(chunk)]))
 
 
-def normal(seed: int, stream: int, n: int, dtype: str = "bf16", scale: float = 1.0,
-           offset: float = 0.0, row_len: int = 0, row_scale=None) -> np.ndarray:
-    """n draws of offset + scale * N(0,1) from one stream, as bf16 bits or float32.
-
-    ``row_scale`` (length n // row_len, float32) multiplies row r after the scale and offset,
-    before the single rounding to the output type."""
-    out = np.empty(n, dtype=np.uint16 if dtype == "bf16" else np.float32)
+def _draw(seed: int, stream: int, start: int, n: int, fill) -> None:
+    """Elements [start, start + n) of a stream, chunk by chunk: fill(lo, hi, a) receives the
+    float32 draws a of the global element range [lo, hi). A chunk is always drawn from its own
+    start, so a range gives exactly the elements the whole-tensor draw has there."""
+    if n <= 0:
+        return
+    c0, c1 = start // CHUNK, (start + n - 1) // CHUNK
 
     def work(c):
-        s, e = c * CHUNK, min(n, (c + 1) * CHUNK)
-        a = _gen(seed, stream, c).standard_normal(e - s, dtype=np.float32)
+        lo, hi = max(start, c * CHUNK), min(start + n, (c + 1) * CHUNK)
+        a = _gen(seed, stream, c).standard_normal(hi - c * CHUNK, dtype=np.float32)
+        fill(lo, hi, a[lo - c * CHUNK:])
+
+    if c1 == c0:
+        work(c0)
+    else:
+        with ThreadPoolExecutor(_threads()) as ex:
+            list(ex.map(work, range(c0, c1 + 1)))
+
+
+def normal(seed: int, stream: int, n: int, dtype: str = "bf16", scale: float = 1.0,
+           offset: float = 0.0, row_len: int = 0, row_scale=None, start: int = 0) -> np.ndarray:
+    """Elements [start, start + n) of offset + scale * N(0,1) from one stream, as bf16 bits or
+    float32.
+
+    ``row_scale`` (indexed by the global row, element index // row_len, float32) multiplies each
+    row after the scale and offset, before the single rounding to the output type."""
+    out = np.empty(n, dtype=np.uint16 if dtype == "bf16" else np.float32)
+
+    def fill(lo, hi, a):
         if scale != 1.0:
             a *= np.float32(scale)
         if offset != 0.0:
             a += np.float32(offset)
         if row_scale is not None:
-            rows = np.arange(s, e, dtype=np.int64) // row_len
-            a *= row_scale[rows]
-        out[s:e] = bf16_bits(a) if dtype == "bf16" else a
+            a *= row_scale[np.arange(lo, hi, dtype=np.int64) // row_len]
+        out[lo - start:hi - start] = bf16_bits(a) if dtype == "bf16" else a
 
-    nchunks = (n + CHUNK - 1) // CHUNK
-    if nchunks <= 1:
-        for c in range(nchunks):
-            work(c)
-    else:
-        with ThreadPoolExecutor(_threads()) as ex:
-            list(ex.map(work, range(nchunks)))
+    _draw(seed, stream, start, n, fill)
     return out
 
 
@@ -113,65 +125,85 @@ def rope_tables(S: int, D: int, theta: float = 10000.0, p0: int = 0):
 # ---- the workloads ----------------------------------------------------------------------------
 
 
+def _range(total: int, part) -> tuple:
+    lo, hi = (0, total) if part is None else (int(part[0]), int(part[1]))
+    if not 0 <= lo <= hi <= total:
+        raise ValueError(f"range {part} outside [0, {total}]")
+    return lo, hi
+
+
 def rmsnorm(M: int = 15360, N: int = 5120, dtype: str = "bf16", gemma: bool = False,
-            outliers: bool = True, seed: int = 0) -> dict:
+            outliers: bool = True, seed: int = 0, rows=None) -> dict:
+    """``rows=(r0, r1)`` gives rows r0..r1-1 of the M-row workload (the outlier rows are still
+    chosen among all M rows)."""
+    r0, r1 = _range(M, rows)
     rs = outlier_rows(seed, M) if outliers else None
     return {
-        "x": normal(seed, S_X, M * N, dtype, row_len=N, row_scale=rs).reshape(M, N),
+        "x": normal(seed, S_X, (r1 - r0) * N, dtype, row_len=N, row_scale=rs, start=r0 * N).reshape(r1 - r0, N),
         "w": normal(seed, S_W, N, dtype, scale=0.1, offset=0.0 if gemma else 1.0),
-        "dy": normal(seed, S_DY, M * N, dtype).reshape(M, N),
+        "dy": normal(seed, S_DY, (r1 - r0) * N, dtype, start=r0 * N).reshape(r1 - r0, N),
         "eps": 1e-6, "gemma": gemma, "dtype": dtype,
     }
 
 
-def layernorm(M: int = 32768, N: int = 5120, dtype: str = "bf16", seed: int = 0) -> dict:
+def layernorm(M: int = 32768, N: int = 5120, dtype: str = "bf16", seed: int = 0, rows=None) -> dict:
+    """``rows=(r0, r1)`` gives rows r0..r1-1 of the M-row workload."""
+    r0, r1 = _range(M, rows)
     mu = uniform(seed, S_MU, M, -2.0, 2.0)
     sg = uniform(seed, S_SIGMA, M, 0.5, 3.0)
-    x = np.empty(M * N, dtype=np.uint16 if dtype == "bf16" else np.float32)
+    x = np.empty((r1 - r0) * N, dtype=np.uint16 if dtype == "bf16" else np.float32)
 
-    def work(c):
-        s, e = c * CHUNK, min(M * N, (c + 1) * CHUNK)
-        a = _gen(seed, S_X, c).standard_normal(e - s, dtype=np.float32)
-        rows = np.arange(s, e, dtype=np.int64) // N
-        a = mu[rows] + sg[rows] * a
-        x[s:e] = bf16_bits(a) if dtype == "bf16" else a
+    def fill(lo, hi, a):
+        rr = np.arange(lo, hi, dtype=np.int64) // N
+        a = mu[rr] + sg[rr] * a
+        x[lo - r0 * N:hi - r0 * N] = bf16_bits(a) if dtype == "bf16" else a
 
-    with ThreadPoolExecutor(_threads()) as ex:
-        list(ex.map(work, range((M * N + CHUNK - 1) // CHUNK)))
+    _draw(seed, S_X, r0 * N, (r1 - r0) * N, fill)
     return {
-        "x": x.reshape(M, N),
+        "x": x.reshape(r1 - r0, N),
         "w": normal(seed, S_W, N, dtype, scale=0.1, offset=1.0),
         "b": normal(seed, S_B, N, dtype, scale=0.1),
-        "dy": normal(seed, S_DY, M * N, dtype).reshape(M, N),
+        "dy": normal(seed, S_DY, (r1 - r0) * N, dtype, start=r0 * N).reshape(r1 - r0, N),
         "eps": 1e-5, "dtype": dtype,
     }
 
 
+def _tokens(seed: int, stream: int, B: int, S: int, H: int, D: int, s0: int, s1: int, dtype: str) -> np.ndarray:
+    """Tokens s0..s1-1 of every batch entry of a [B, S, H, D] stream tensor."""
+    per = H * D
+    return np.stack([normal(seed, stream, (s1 - s0) * per, dtype, start=(b * S + s0) * per)
+                     for b in range(B)]).reshape(B, s1 - s0, H, D)
+
+
 def rope(B: int = 1, S: int = 32760, H: int = 40, D: int = 128, dtype: str = "bf16",
-         theta: float = 10000.0, seed: int = 0) -> dict:
-    n = B * S * H * D
-    cos, sin = rope_tables(S, D, theta)
+         theta: float = 10000.0, seed: int = 0, tokens=None) -> dict:
+    """``tokens=(s0, s1)`` gives tokens s0..s1-1 of the S-token workload, with the table rows of
+    their positions s0..s1-1."""
+    s0, s1 = _range(S, tokens)
+    cos, sin = rope_tables(s1 - s0, D, theta, p0=s0)
     return {
-        "q": normal(seed, S_Q, n, dtype).reshape(B, S, H, D),
-        "k": normal(seed, S_K, n, dtype).reshape(B, S, H, D),
+        "q": _tokens(seed, S_Q, B, S, H, D, s0, s1, dtype),
+        "k": _tokens(seed, S_K, B, S, H, D, s0, s1, dtype),
         "cos": cos, "sin": sin, "dtype": dtype,
     }
 
 
 def qknorm_rope(B: int = 2, S: int = 76800, H: int = 40, D: int = 128, dtype: str = "bf16",
-                theta: float = 10000.0, seed: int = 0, grads: bool = True) -> dict:
-    n = B * S * H * D
-    cos, sin = rope_tables(S, D, theta)
+                theta: float = 10000.0, seed: int = 0, grads: bool = True, tokens=None) -> dict:
+    """``tokens=(s0, s1)`` gives tokens s0..s1-1 of the S-token workload, with the table rows of
+    their positions s0..s1-1."""
+    s0, s1 = _range(S, tokens)
+    cos, sin = rope_tables(s1 - s0, D, theta, p0=s0)
     d = {
-        "q": normal(seed, S_Q, n, dtype).reshape(B, S, H, D),
-        "k": normal(seed, S_K, n, dtype).reshape(B, S, H, D),
+        "q": _tokens(seed, S_Q, B, S, H, D, s0, s1, dtype),
+        "k": _tokens(seed, S_K, B, S, H, D, s0, s1, dtype),
         "wq": normal(seed, S_WQ, D, dtype, scale=0.1, offset=1.0),
         "wk": normal(seed, S_WK, D, dtype, scale=0.1, offset=1.0),
         "cos": cos, "sin": sin, "eps": 1e-6, "dtype": dtype,
     }
     if grads:
-        d["dq_out"] = normal(seed, S_DQ, n, dtype).reshape(B, S, H, D)
-        d["dk_out"] = normal(seed, S_DK, n, dtype).reshape(B, S, H, D)
+        d["dq_out"] = _tokens(seed, S_DQ, B, S, H, D, s0, s1, dtype)
+        d["dk_out"] = _tokens(seed, S_DK, B, S, H, D, s0, s1, dtype)
     return d
 
 
