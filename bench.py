@@ -558,7 +558,8 @@ def run_ours(args):
                      "frac": round(ach / peak, 4), "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs"},
         "kernels": {k: {"ms": round(per_kernel[k] * 1e3, 4), "GB_s": round(nbytes[k] / per_kernel[k] / 1e9, 1),
                         "frac_of_peak": round(nbytes[k] / per_kernel[k] / 1e9 / peak, 4),
-                        "rows_per_s": round(rows_of(z)[k] / per_kernel[k], 1)} for k in kernels},
+                        "rows_per_s": round(rows_of(z)[k] / per_kernel[k], 1),
+                        "algorithmic_bytes": nbytes[k], "traffic": ncu_traffic(k, z)} for k in kernels},
         "frac_of_peak": round(value / ws / peak, 4),
         "frac_of_8TBs": round(value / ws / 8000.0, 4),
         "clocks": clk.report(),

@@ -90,28 +90,40 @@ def test_noalloc_backward_matches_workspace_backward(gpu, with_k):
 def test_noalloc_refuses_partials_beyond_the_fixed_array(gpu):
     """A call whose per-block partials (2 * D * 4 bytes for each block of the persistent grid)
     exceed the fixed array returns GN_ERR_WORKSPACE and leaves every output untouched. Head dim
-    256 with short units and four consumer warps per block makes a grid of more than 512 blocks
-    (found through the workspace query, which reports grid * 2 * D * 4 bytes)."""
+    256 with one head per unit and four consumer warps per block gives a grid of more than 512
+    blocks; the workspace query reports grid * 2 * D * 4 bytes for the larger grid of the plain
+    and Gemma variants, so the variant with that grid must be refused (the other may run)."""
     B, S, H, D = 1, 4096, 4, 256
     t = _inputs(gpu, B=B, S=S, H=H, D=D, seed=5)
     stream = torch.cuda.current_stream().cuda_stream
     found = None
     try:
-        for unit_bytes, group_rows, stages in ((0, 0, 0), (2048, 4, 0), (2048, 4, 2), (1024, 4, 2)):
+        for unit_bytes, group_rows, stages in ((0, 0, 0), (2048, 4, 0), (2048, 4, 2), (1024, 4, 2), (512, 4, 2)):
             gpu.tune("unit_bytes", unit_bytes)
             gpu.tune("group_rows", group_rows)
             gpu.tune("stages", stages)
             need = gpu.gn_qknorm_rope_bwd_workspace(B, S, H, D, gpu.GN_BF16)
-            if need > FIXED_BYTES * 5 // 4:
+            if need > FIXED_BYTES:
                 found = (unit_bytes, group_rows, stages, need)
                 break
         assert found is not None, "no launch shape on this device needs more than the fixed array"
-        outs = _outputs(t["q"], True, D)
-        st, outs = _call_noalloc(gpu, t, True, stream, outs)
-        torch.cuda.synchronize()
-        assert st == gpu.GN_ERR_WORKSPACE, f"{found}: status {st}"
-        for o in outs:  # nothing was launched: the NaN fill is intact
-            assert torch.isnan(o).all()
+        refused = 0
+        for gemma in (0, 1):
+            q = t["q"]
+            dq, dk, dwq, dwk = _outputs(q, True, D)
+            st = gpu.gn_qknorm_rope_bwd_noalloc(q.data_ptr(), t["k"].data_ptr(), t["wq"].data_ptr(),
+                                                t["wk"].data_ptr(), t["cos"].data_ptr(), t["sin"].data_ptr(),
+                                                t["rq"].data_ptr(), t["rk"].data_ptr(), t["dq_out"].data_ptr(),
+                                                t["dk_out"].data_ptr(), dq.data_ptr(), dk.data_ptr(), dwq.data_ptr(),
+                                                dwk.data_ptr(), B, S, H, D, gemma, gpu.GN_BF16, stream)
+            torch.cuda.synchronize()
+            if st == gpu.GN_ERR_WORKSPACE:
+                refused += 1
+                for o in (dq, dk, dwq, dwk):  # nothing was launched: the NaN fill is intact
+                    assert torch.isnan(o).all()
+            else:
+                assert st == gpu.GN_OK, f"{found} gemma={gemma}: status {st}"
+        assert refused >= 1, f"{found}: no variant refused"
     finally:
         for key in ("unit_bytes", "group_rows", "stages"):
             gpu.tune(key, 0)

@@ -10,7 +10,7 @@
 
 namespace gn {
 
-Tuning g_tune = {0, 0, 0, 0, 0};
+Tuning g_tune = {0, 0, 0, 0, 0, 0, 0, 0};
 
 static std::atomic<uint64_t> g_launches{0};
 
@@ -71,12 +71,46 @@ size_t smem_optin() {
 
 gn_status launch_status() { return cudaGetLastError() == cudaSuccess ? GN_OK : GN_ERR_CUDA; }
 
+// Every kernel of the library asks for the same L1 / shared-memory split (the most shared
+// memory): an SM whose split differs from the next kernel's must be reconfigured between the two
+// kernels, which costs the next launch several microseconds.
+#ifndef GN_CARVEOUT
+#define GN_CARVEOUT 100
+#endif
+
+bool kernel_attrs(const void* kernel, size_t smem) {
+  const int d = current_device();
+  if (d < 0) return false;
+  struct Seen {
+    const void* k;
+    int d;
+    size_t smem;
+  };
+  static std::mutex mu;
+  static Seen seen[512];
+  static int nseen = 0;
+  std::lock_guard<std::mutex> lk(mu);
+  for (int i = 0; i < nseen; ++i)
+    if (seen[i].k == kernel && seen[i].d == d && seen[i].smem >= smem) return true;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return false;
+  if (GN_CARVEOUT >= 0 &&
+      cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, GN_CARVEOUT) != cudaSuccess)
+    return false;
+  for (int i = 0; i < nseen; ++i)
+    if (seen[i].k == kernel && seen[i].d == d) {
+      seen[i].smem = smem;
+      return true;
+    }
+  if (nseen < 512) seen[nseen++] = Seen{kernel, d, smem};
+  return true;
+}
+
 int persistent_grid(const void* kernel, int threads, size_t smem, int cap) {
   const int sms = sm_count();
   if (sms <= 0) return 0;
-  if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return 0;
+  if (!kernel_attrs(kernel, smem)) return 0;
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) != cudaSuccess) return 0;
   if (per_sm <= 0) return 0;
@@ -93,6 +127,7 @@ __global__ void __launch_bounds__(256) colsum_kernel(const float* __restrict__ w
                                                      float* __restrict__ out0,
                                                      float* __restrict__ out1) {
   __shared__ float part[8][33];
+  pdl_wait();  // the partial rows are complete: the backward grid before this one has finished
   const int cl = threadIdx.x & 31, sl = threadIdx.x >> 5;
   const int64_t c = (int64_t)blockIdx.x * 32 + cl;
   float acc = 0.f;
@@ -127,7 +162,20 @@ gn_status launch_colsum(const float* ws, int64_t G, int64_t ncols, int64_t split
                         float* out1, cudaStream_t s) {
   if (!out0 && !out1) return GN_OK;
   const int64_t blocks = (ncols + 31) / 32;
-  colsum_kernel<<<(unsigned)blocks, 256, 0, s>>>(ws, G, ncols, split, out0, out1);
+  if (!kernel_attrs((const void*)colsum_kernel, 0)) return GN_ERR_CUDA;
+  // launched with programmatic stream serialization: its launch overlaps the tail of the
+  // backward grid before it, which it waits for on the device (pdl_wait)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = GN_PDL;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, colsum_kernel, ws, G, ncols, split, out0, out1) != cudaSuccess) return GN_ERR_CUDA;
   count_launches(1);
   return launch_status();
 }
@@ -186,6 +234,15 @@ extern "C" gn_status gn_tune(const char* key, int value) {
     g_tune.unit_bytes = value;
   } else if (!strcmp(key, "group_rows")) {
     g_tune.group_rows = value;
+  } else if (!strcmp(key, "fwd_warps")) {
+    if (value > 16) return GN_ERR_SHAPE;
+    g_tune.fwd_warps = value;
+  } else if (!strcmp(key, "fwd_path")) {
+    if (value > 3) return GN_ERR_SHAPE;
+    g_tune.fwd_path = value;
+  } else if (!strcmp(key, "bwd_tmem")) {
+    if (value > 2) return GN_ERR_SHAPE;
+    g_tune.bwd_tmem = value;
   } else {
     return GN_ERR_SHAPE;
   }

@@ -133,7 +133,10 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
 
 // The thread may be suspended inside try_wait until the phase completes or about
 // kSuspendHintNs pass, so a waiting warp does not spend issue slots polling.
-constexpr uint32_t kSuspendHintNs = 100000;
+#ifndef GN_SUSPEND_HINT_NS
+#define GN_SUSPEND_HINT_NS 100000
+#endif
+constexpr uint32_t kSuspendHintNs = GN_SUSPEND_HINT_NS;
 
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
@@ -176,6 +179,21 @@ __device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src, uint32
           smem_addr(dst_smem)),
       "l"(src), "r"(bytes), "r"(smem_addr(bar))
       : "memory");
+}
+
+// ---------------------------------------------------------------- programmatic dependent launch
+// A backward kernel lets the launch of the grid that follows it in the stream (the weight-gradient
+// column reduction, launched with programmatic stream serialization) start before it completes;
+// that grid waits in pdl_wait() for this grid's completion and memory before it reads anything.
+
+#ifndef GN_PDL
+#define GN_PDL 1
+#endif
+__device__ __forceinline__ void pdl_launch_dependents() {
+  if (GN_PDL) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() {
+  if (GN_PDL) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // ---------------------------------------------------------------- reductions
@@ -224,7 +242,9 @@ __device__ __forceinline__ float tanh_f(float x) {
 template <bool FAST>
 __device__ __forceinline__ float sigmoid_f(float x) {
   if constexpr (FAST) {
-    return __frcp_rn(1.0f + __expf(-x));
+    // approximate reciprocal (2 ulp): far below the bf16 rounding of the outputs; the correctly
+    // rounded __frcp_rn is a multi-instruction sequence that made the SiLU kernels ALU-bound
+    return __fdividef(1.0f, 1.0f + __expf(-x));
   } else {
     return 1.0f / (1.0f + expf(-x));
   }
@@ -294,12 +314,19 @@ __device__ __forceinline__ float2 gelu_of_half2(float2 h) {
   return fma2(h, t, h);
 }
 
-// the gradient runs as two scalar evaluations: its packed form needs more registers for the
-// constants, which the long-row backward kernels cannot spare
+// The tanh-GeLU gradient runs on packed fp32x2 instructions with the scalar form's operations,
+// operand order and constants lane by lane (each lane rounds exactly as epi_grad); SiLU runs as
+// two scalar evaluations.
 template <int EPI, bool FAST>
 __device__ __forceinline__ float2 epi_grad2(float2 z) {
   if constexpr (EPI == EPI_NONE) {
     return dup2(1.0f);
+  } else if constexpr (EPI == EPI_GELU_TANH) {
+    const float2 z2 = mul2(z, z);
+    const float2 t = tanh2<FAST>(mul2(z, fma2(dup2(kGeluK * kGeluC), z2, dup2(kGeluK))));
+    const float2 k3 = fma2(dup2(3.0f * 0.5f * kGeluK * kGeluC), z2, dup2(0.5f * kGeluK));
+    const float2 s = fma2(make_float2(-t.x, -t.y), t, dup2(1.0f));  // 1 - t^2
+    return fma2(mul2(z, s), k3, fma2(dup2(0.5f), t, dup2(0.5f)));
   } else {
     return make_float2(epi_grad<EPI, FAST>(z.x), epi_grad<EPI, FAST>(z.y));
   }

@@ -16,6 +16,10 @@ struct Tuning {
   int vpt;
   int unit_bytes;
   int group_rows;
+  int fwd_warps;  // warps per CTA of the one-warp-per-row forward
+  int fwd_path;   // norm forward of long rows: 1 = CTA-per-row pipeline, 2 = one warp per row,
+                  // 3 = one warp per row with one-pass LayerNorm statistics
+  int bwd_tmem;   // LayerNorm backward of bf16 long rows: 1 = accumulators in registers, 2 = in TMEM
 };
 extern Tuning g_tune;
 
@@ -41,6 +45,10 @@ inline bool epi_ok(int e) { return e == GN_EPI_NONE || e == GN_EPI_GELU_TANH || 
 // c < split, out1[c - split] for c >= split (either output may be null to skip its part).
 gn_status launch_colsum(const float* ws, int64_t G, int64_t ncols, int64_t split, float* out0,
                         float* out1, cudaStream_t s);
+
+// Sets a kernel's launch attributes on the current device once (the dynamic shared-memory limit
+// when smem exceeds 48 KiB, and the L1 / shared-memory split every kernel of the library shares).
+bool kernel_attrs(const void* kernel, size_t smem);
 
 // Largest grid of a persistent kernel: sm_count() * min(occupancy, cap).
 int persistent_grid(const void* kernel, int threads, size_t smem, int cap);

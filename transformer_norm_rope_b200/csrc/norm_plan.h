@@ -41,10 +41,13 @@ inline int pow2_ceil(int v) {
 }
 
 // ntens: row tensors staged per row (1 forward, 2 backward); nparams: per-column parameter
-// vectors kept in shared memory (weight, bias); max_vpt: 8 forward, 4 backward; target:
-// preferred consumer threads (the forward keeps more of the row per thread, which spreads
-// the per-row reduction over more elements).
-inline gn_status plan_norm(int64_t N, size_t es, int ntens, int nparams, int max_vpt, int target, NormPlan* p) {
+// vectors kept in shared memory (weight, bias), pes bytes per element (the row type's size, or 4
+// for fp32 copies); max_vpt: 8 forward, 4 backward; target: preferred consumer threads (the
+// forward keeps more of the row per thread, which spreads the per-row reduction over more
+// elements).
+inline gn_status plan_norm(int64_t N, size_t es, int ntens, int nparams, int max_vpt, int target, NormPlan* p,
+                           size_t pes = 0) {
+  if (!pes) pes = es;
   const int vec = (int)(16 / es);
   const int64_t nvec = (N + vec - 1) / vec;
   if (nvec <= kGroupMaxVec) {
@@ -80,11 +83,19 @@ inline gn_status plan_norm(int64_t N, size_t es, int ntens, int nparams, int max
   }
   if (stages > kMaxStages) stages = kMaxStages;
   const size_t limit = smem_optin();
-  while (stages > 1 && pipe_smem_bytes(stages, ntens, nparams, N, (int64_t)es) > limit) --stages;
-  if (pipe_smem_bytes(stages, ntens, nparams, N, (int64_t)es) > limit) return GN_ERR_UNSUPPORTED;
+  while (stages > 1 && pipe_smem_bytes(stages, ntens, nparams, N, (int64_t)es, (int64_t)pes) > limit) --stages;
+  if (pipe_smem_bytes(stages, ntens, nparams, N, (int64_t)es, (int64_t)pes) > limit) return GN_ERR_UNSUPPORTED;
   p->stages = stages;
-  p->smem = pipe_smem_bytes(stages, ntens, nparams, N, (int64_t)es);
+  p->smem = pipe_smem_bytes(stages, ntens, nparams, N, (int64_t)es, (int64_t)pes);
   return GN_OK;
 }
+
+// Forward of long rows with one warp per row (norm_fwd_warp.cu): RMSNorm (ln = false: stat0 =
+// inv_rms) or LayerNorm (ln = true: stat0 = mean, stat1 = rstd, b = bias). Arguments validated by
+// the caller. GN_ERR_UNSUPPORTED when the row does not fit its shared-memory stages (the caller
+// then uses the CTA-per-row kernel).
+gn_status launch_norm_fwd_warp(bool ln, const void* x, const void* w, const void* b, void* y, float* stat0,
+                               float* stat1, int64_t rows, int64_t N, int64_t ldx, int64_t ldy, float eps, bool gemma,
+                               int epi, gn_dtype dt, cudaStream_t stream);
 
 }  // namespace gn

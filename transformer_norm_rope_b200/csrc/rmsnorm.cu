@@ -56,7 +56,7 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT)) rms_fwd
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int N = a.N, nfull = N / Vec<T>::N, nvec = (N + Vec<T>::N - 1) / Vec<T>::N;
-  const RowPipe pipe(smem, a.stages, 1, 1, N, sizeof(T));
+  const RowPipe pipe(smem, a.stages, 1, 1, N, sizeof(T), sizeof(T));
   const T* x = static_cast<const T*>(a.x);
   T* y = static_cast<T*>(a.y);
   const int ncw = (int)(blockDim.x >> 5) - 1;
@@ -68,6 +68,7 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT)) rms_fwd
   }
   const int ct = tid - 32, nct = ncw * 32, cw = warp - 1;
   stage_param<T, VPT>(pipe.param(0), static_cast<const T*>(a.w), N, nvec, 0.0f, ct, nct);
+  pipe.red_zero(ct, nct);
   consumers_sync(nct);
   const float inv_n = 1.0f / (float)N;
   const int64_t step = gridDim.x;
@@ -86,13 +87,11 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT)) rms_fwd
     __syncwarp();
     if (lane == 0) mbar_arrive(&pipe.empty[s]);
     const float ss = group_sum<32>(ss2.x + ss2.y);
-    float4* red = pipe.red + rb * 32;
-    if (lane == 0) red[cw].x = ss;
+    if (lane == 0) pipe.red_at(rb, 0)[cw] = ss;
     if (consumers_sync_or(nct, !ok)) return;
+    const float tot = pipe.red_sum(rb, 0, ncw);
     rb ^= 1u;
     if (++s == a.stages) s = 0, ph ^= 1u;
-    float tot = 0.0f;
-    for (int w = 0; w < ncw; ++w) tot += red[w].x;
     const float r = rsqrtf(fmaf(tot, inv_n, a.eps));
     const float2 r2 = dup2(r);
     T* yrow = y + m * a.ldy;
@@ -116,12 +115,13 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT)) rms_fwd
 
 template <typename T, int VPT, int EPI, bool GEMMA>
 __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT, true)) rms_bwd_cta(const RmsBwdArgs a) {
+  pdl_launch_dependents();  // the column reduction that follows may launch early
   constexpr int E = Vec<T>::N, H = E / 2;
   constexpr bool FAST = fast_math_for<T>();
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int N = a.N, nfull = N / E, nvec = (N + E - 1) / E;
-  const RowPipe pipe(smem, a.stages, 2, 1, N, sizeof(T));
+  const RowPipe pipe(smem, a.stages, 2, 1, N, sizeof(T), 4);
   const T* x = static_cast<const T*>(a.x);
   const T* dy = static_cast<const T*>(a.dy);
   T* dx = static_cast<T*>(a.dx);
@@ -137,7 +137,10 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT, true)) r
     return;
   }
   const int ct = tid - 32, nct = ncw * 32, cw = warp - 1;
-  stage_param<T, VPT>(pipe.param(0), static_cast<const T*>(a.w), N, nvec, 0.0f, ct, nct);
+  // w' = w (+1 Gemma) as fp32: the per-row passes read it with no conversion
+  stage_param_f32<T, VPT>(reinterpret_cast<float*>(pipe.param(0)), static_cast<const T*>(a.w), N, nvec,
+                          GEMMA ? 1.0f : 0.0f, 1.0f, 0.0f, ct, nct);
+  pipe.red_zero(ct, nct);
   consumers_sync(nct);
   float2 dwa[VPT][H];
 #pragma unroll
@@ -172,11 +175,11 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT, true)) r
     for (int j = 0; j < VPT; ++j) {
       const int v = ct + j * nct;
       float2 wv[H], xv[H];
-      param_pairs<T>(pipe.param(0), v < nvec ? v : 0, wv);
+      prm_pairs<H>(reinterpret_cast<const float*>(pipe.param(0)), v < nvec ? v : 0, nvec, wv);
       unpack2<T>(xr[j], xv);
 #pragma unroll
       for (int h = 0; h < H; ++h) {
-        const float2 wp = GEMMA ? add2(wv[h], dup2(1.0f)) : wv[h];
+        const float2 wp = wv[h];
         const float2 xh = mul2(xv[h], r2);
         const float2 g = EPI == EPI_NONE ? gv[j][h] : mul2(gv[j][h], epi_grad2<EPI, FAST>(mul2(xh, wp)));
         const float2 gw = mul2(g, wp);
@@ -186,16 +189,14 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT, true)) r
       }
     }
     const float c = group_sum<32>(c2.x + c2.y);
-    float4* red = pipe.red + rb * 32;
-    if (lane == 0) red[cw].x = c;
+    if (lane == 0) pipe.red_at(rb, 0)[cw] = c;
     if (consumers_sync_or(nct, !ok)) {
       failed = true;
       break;
     }
+    const float tot = pipe.red_sum(rb, 0, ncw);
     rb ^= 1u;
     if (++s == a.stages) s = 0, ph ^= 1u;
-    float tot = 0.0f;
-    for (int w = 0; w < ncw; ++w) tot += red[w].x;
     const float2 ncm = dup2(-tot * inv_n);
     T* dxrow = dx + m * a.lddx;
 #pragma unroll
@@ -296,6 +297,7 @@ __global__ void __launch_bounds__(kGroupThreads) rms_fwd_grp(const RmsFwdArgs a,
 
 template <typename T, int VPT, int EPI, bool GEMMA>
 __global__ void __launch_bounds__(kGroupThreads) rms_bwd_grp(const RmsBwdArgs a, int lanes) {
+  pdl_launch_dependents();  // the column reduction that follows may launch early
   using V = Vec<T>;
   constexpr int E = V::N;
   constexpr bool FAST = fast_math_for<T>();
@@ -440,7 +442,7 @@ void* pick_bwd_t(int vpt, bool cta, int epi, bool gemma) {
 
 gn_status rms_bwd_plan(int64_t rows, int64_t hidden, gn_dtype dt, NormPlan* p, void** kern, int epi,
                        bool gemma, int* grid) {
-  gn_status st = plan_norm(hidden, dt_size(dt), 2, 1, 4, 320, p);
+  gn_status st = plan_norm(hidden, dt_size(dt), 2, 1, 4, 320, p, 4);
   if (st != GN_OK) return st;
   *kern = dt == GN_BF16 ? pick_bwd_t<__nv_bfloat16>(p->vpt, p->cta, epi, gemma)
                         : pick_bwd_t<float>(p->vpt, p->cta, epi, gemma);
@@ -472,6 +474,11 @@ extern "C" gn_status gn_rmsnorm_fwd(const void* x, const void* w, void* y, float
   NormPlan p;
   gn_status st = plan_norm(hidden, es, 1, 1, 8, 320, &p);
   if (st != GN_OK) return st;
+  if (p.cta && g_tune.fwd_path != 1) {  // long rows: one warp per row unless the row does not fit
+    st = launch_norm_fwd_warp(false, x, w, nullptr, y, inv_rms, nullptr, rows, hidden, ld_x, ld_y, eps, gemma != 0,
+                              epi, dt, (cudaStream_t)stream);
+    if (st != GN_ERR_UNSUPPORTED) return st;
+  }
   void* kern = dt == GN_BF16 ? pick_fwd_t<__nv_bfloat16>(p.vpt, p.cta, epi, gemma != 0)
                              : pick_fwd_t<float>(p.vpt, p.cta, epi, gemma != 0);
   if (!kern) return GN_ERR_UNSUPPORTED;

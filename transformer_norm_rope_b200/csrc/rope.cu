@@ -287,6 +287,7 @@ __global__ void __launch_bounds__(kRopeMaxThreads, 2) rope_kernel(const RopeArgs
   const uint32_t tab_bytes = (uint32_t)(D / 2 * 4);
   const bool stat_staged = BWD && a.stat_staged;
   const uint32_t stat_bytes = stat_staged ? (uint32_t)(HC * 4) : 0u;
+  if constexpr (BWD) pdl_launch_dependents();  // the column reduction that follows may launch early
 
   if (threadIdx.x == 0) {
     for (int st = 0; st < a.stages; ++st) {

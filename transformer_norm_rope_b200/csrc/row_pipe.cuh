@@ -13,8 +13,9 @@
 // Shared memory layout (dynamic, 128-byte aligned):
 //   [0, 64)           full mbarriers, one per stage (stages <= 8)
 //   [64, 128)         empty mbarriers
-//   [128, 1152)       reduction scratch: 2 row parities x 32 warps x float4
-//   [1152, ...)       nparams parameter vectors (weight, bias) of the row length
+//   [128, 1152)       reduction scratch: 2 row parities x 4 quantities x 32 warps of float
+//   [1152, ...)       nparams parameter vectors (weight, bias) of the row length, in the row type
+//                     (forward) or as fp32 (backward)
 //   then              stages x ntens row slots (row bytes rounded up to 128)
 #pragma once
 
@@ -29,11 +30,15 @@ __host__ __device__ inline uint32_t pipe_slot_bytes(int64_t row_bytes) {
   return (uint32_t)((row_bytes + 127) / 128 * 128);
 }
 
-// parameter vectors are kept in the row type, padded to whole 16-byte vectors and 128 bytes
-__host__ __device__ inline uint32_t pipe_param_bytes(int64_t n, int64_t es) { return pipe_slot_bytes((n * es + 15) / 16 * 16); }
+// parameter vectors: one element of pes bytes (the row type's size, or 4 for fp32 copies) per
+// row element, padded to whole 16-byte row vectors and to 128 bytes
+__host__ __device__ inline uint32_t pipe_param_bytes(int64_t n, int64_t es, int64_t pes) {
+  return pipe_slot_bytes((n * es + 15) / 16 * (16 / es) * pes);
+}
 
-__host__ __device__ inline size_t pipe_smem_bytes(int stages, int ntens, int nparams, int64_t n, int64_t es) {
-  return kPipeHeader + (size_t)nparams * pipe_param_bytes(n, es) + (size_t)stages * ntens * pipe_slot_bytes(n * es);
+__host__ __device__ inline size_t pipe_smem_bytes(int stages, int ntens, int nparams, int64_t n, int64_t es,
+                                                  int64_t pes) {
+  return kPipeHeader + (size_t)nparams * pipe_param_bytes(n, es, pes) + (size_t)stages * ntens * pipe_slot_bytes(n * es);
 }
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
@@ -68,17 +73,38 @@ struct RowPipe {
   uint32_t pslot;   // bytes per parameter vector
   uint32_t bulk;    // bytes bulk-copied per tensor (whole 16-byte vectors of the row)
 
-  __device__ __forceinline__ RowPipe(uint8_t* smem, int stages_, int ntens_, int nparams, int64_t n, int64_t es)
+  __device__ __forceinline__ RowPipe(uint8_t* smem, int stages_, int ntens_, int nparams, int64_t n, int64_t es,
+                                     int64_t pes)
       : full(reinterpret_cast<uint64_t*>(smem)),
         empty(reinterpret_cast<uint64_t*>(smem) + kMaxStages),
         red(reinterpret_cast<float4*>(smem + 128)),
         params(smem + kPipeHeader),
-        data(smem + kPipeHeader + (size_t)nparams * pipe_param_bytes(n, es)),
+        data(smem + kPipeHeader + (size_t)nparams * pipe_param_bytes(n, es, pes)),
         stages(stages_),
         ntens(ntens_),
         slot(pipe_slot_bytes(n * es)),
-        pslot(pipe_param_bytes(n, es)),
+        pslot(pipe_param_bytes(n, es, pes)),
         bulk((uint32_t)(n * es / 16 * 16)) {}
+
+  // Cross-warp partials of the per-row reductions, as float [2 row parities][4 quantities][32
+  // warps]: warp w's partial of quantity q sits at index w, so a sum over the consumer warps reads
+  // four partials per 16-byte load. Slots past the consumer warps stay zero (red_zero).
+  __device__ __forceinline__ float* red_at(uint32_t rb, int q) const {
+    return reinterpret_cast<float*>(red) + (rb * 4 + q) * 32;
+  }
+  __device__ __forceinline__ void red_zero(int ct, int nct) const {
+    for (int i = ct; i < 256; i += nct) reinterpret_cast<float*>(red)[i] = 0.0f;
+  }
+  // the fixed-order sum of quantity q over the ncw consumer warps (same order in every thread)
+  __device__ __forceinline__ float red_sum(uint32_t rb, int q, int ncw) const {
+    const float4* p = reinterpret_cast<const float4*>(red_at(rb, q));
+    float t = 0.0f;
+    for (int i = 0; i < ((ncw + 3) >> 2); ++i) {
+      const float4 v = p[i];
+      t += (v.x + v.y) + (v.z + v.w);
+    }
+    return t;
+  }
 
   __device__ __forceinline__ const uint8_t* at(int s, int t) const {
     return data + ((size_t)s * ntens + t) * slot;
