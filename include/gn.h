@@ -273,9 +273,8 @@ gn_status gn_selftest_wait_timeout(uint32_t limit_us, void* stream);
 /* Tuning knobs of the launch planner, for benchmarking sweeps. key is one of "stages",
  * "ctas_per_sm", "vpt", "unit_bytes", "group_rows", "fwd_warps" (warps per CTA of the
  * one-warp-per-row norm forward, at most 16), "fwd_path" (norm forward of long rows: 1 = the
- * CTA-per-row pipeline, 2 = one warp per row, 3 = one warp per row with the LayerNorm statistics
- * in one pass), "bwd_tmem" (LayerNorm backward of bf16 long rows: 1 = weight-gradient
- * accumulators in registers, 2 = in tensor memory); value 0 restores the default. Returns
+ * CTA-per-row pipeline, 2 = one warp per row with two-pass LayerNorm statistics, 3 = one warp per
+ * row with one shifted pass; by default RMSNorm takes the first and LayerNorm the third); value 0 restores the default. Returns
  * GN_ERR_SHAPE for an unknown key or a value out of range. Not thread-safe with concurrent
  * launches. */
 gn_status gn_tune(const char* key, int value);

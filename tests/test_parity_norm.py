@@ -85,18 +85,20 @@ def test_layernorm_fwd_bwd(gpu, rows, hidden, dtype):
         assert_close(to_np(db), rdb, wgrad_tol(dtype, rdb), tag + " db")
 
 
-@pytest.mark.parametrize("path,warps,stages", [(1, 0, 0), (2, 4, 3), (2, 0, 4), (2, 5, 2), (3, 0, 0), (3, 6, 3)])
+@pytest.mark.parametrize("path,warps,stages", [(0, 0, 0), (1, 0, 0), (1, 0, 4), (2, 4, 3), (2, 0, 4), (2, 5, 2),
+                                               (3, 0, 0), (3, 6, 3)])
 def test_norm_forward_kernels_of_long_rows(gpu, path, warps, stages):
     """The forward kernels of long rows - the CTA-per-row pipeline (fwd_path 1), one warp per row
-    with the LayerNorm statistics in two passes (fwd_path 2) or in one pass with Chan et al.'s
-    update (fwd_path 3), at several warp and stage counts - against the oracle, ragged tails
-    included. A row whose stages do not fit the warp kernel falls back to the CTA kernel."""
+    with the LayerNorm statistics in two passes (fwd_path 2) or one shifted pass (fwd_path 3), and
+    the default (RMSNorm: the CTA kernel, LayerNorm: the shifted warp kernel) - at several warp and
+    stage counts, against the oracle, ragged tails included. A row whose stages do not fit the
+    warp kernel falls back to the CTA kernel."""
     try:
         gpu.tune("fwd_path", path)
         gpu.tune("fwd_warps", warps)
         gpu.tune("stages", stages)
         for rows, hidden, dtype in ((300, 5120, "bf16"), (65, 2051, "bf16"), (77, 1000, "f32"), (129, 8192, "bf16"),
-                                    (41, 1027, "f32")):
+                                    (41, 1027, "f32"), (50, 3500, "bf16"), (30, 6000, "bf16")):
             d = wl.rmsnorm(M=rows, N=hidden, dtype=dtype, gemma=True, outliers=False)
             y, r = gpu.rmsnorm_fwd(to_rows(d["x"]), to_dev(d["w"]), d["eps"], gemma=True, epilogue="gelu_tanh")
             ry, rr = oracle.rmsnorm_fwd(d["x"], d["w"], d["eps"], gemma=True, act="gelu_tanh")
@@ -113,34 +115,6 @@ def test_norm_forward_kernels_of_long_rows(gpu, path, warps, stages):
     finally:
         for key in ("fwd_path", "fwd_warps", "stages"):
             gpu.tune(key, 0)
-    assert gpu.device_error(clear=True) == 0
-
-
-@pytest.mark.parametrize("tmem", [1, 2])
-def test_layernorm_backward_kernels_of_long_rows(gpu, tmem):
-    """Both LayerNorm backward kernels of bf16 long rows - weight-gradient accumulators in
-    registers (bwd_tmem 1) or in tensor memory (bwd_tmem 2) - against the oracle, ragged tails,
-    several consumer-warp counts and all three epilogues included; rows too long for the
-    tensor-memory kernel fall back to the register kernel."""
-    try:
-        gpu.tune("bwd_tmem", tmem)
-        for rows, hidden in ((300, 5120), (65, 2051), (777, 1100), (129, 4000), (5, 8192)):
-            d = wl.layernorm(M=rows, N=hidden, dtype="bf16")
-            x, dy, w, b = to_rows(d["x"]), to_rows(d["dy"]), to_dev(d["w"]), to_dev(d["b"])
-            for epi in ("gelu_tanh", "silu", "none"):
-                _, mu, rs = gpu.layernorm_fwd(x, w, b, d["eps"], epilogue=epi)
-                dx, dw, db = gpu.layernorm_bwd(x, w, b, mu, rs, dy, epilogue=epi)
-                rdx, rdw, rdb = oracle.layernorm_bwd(d["x"], d["w"], d["b"], d["dy"], d["eps"], act=epi)
-                tag = f"bwd_tmem {tmem} {rows}x{hidden} {epi}"
-                assert_close(to_np(dx), rdx, "grad_bf16", tag + " dx")
-                assert_close(to_np(dw), rdw, "grad_bf16", tag + " dw")
-                assert_close(to_np(db), rdb, "grad_bf16", tag + " db")
-            a = gpu.layernorm_bwd(x, w, b, mu, rs, dy)
-            c = gpu.layernorm_bwd(x, w, b, mu, rs, dy)
-            torch.cuda.synchronize()
-            assert all(torch.equal(p, q) for p, q in zip(a, c)), f"bwd_tmem {tmem}: not deterministic"
-    finally:
-        gpu.tune("bwd_tmem", 0)
     assert gpu.device_error(clear=True) == 0
 
 

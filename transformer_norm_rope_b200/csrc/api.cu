@@ -10,7 +10,7 @@
 
 namespace gn {
 
-Tuning g_tune = {0, 0, 0, 0, 0, 0, 0, 0};
+Tuning g_tune = {0, 0, 0, 0, 0, 0, 0};
 
 static std::atomic<uint64_t> g_launches{0};
 
@@ -240,9 +240,7 @@ extern "C" gn_status gn_tune(const char* key, int value) {
   } else if (!strcmp(key, "fwd_path")) {
     if (value > 3) return GN_ERR_SHAPE;
     g_tune.fwd_path = value;
-  } else if (!strcmp(key, "bwd_tmem")) {
-    if (value > 2) return GN_ERR_SHAPE;
-    g_tune.bwd_tmem = value;
+
   } else {
     return GN_ERR_SHAPE;
   }

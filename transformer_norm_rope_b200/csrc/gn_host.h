@@ -17,9 +17,8 @@ struct Tuning {
   int unit_bytes;
   int group_rows;
   int fwd_warps;  // warps per CTA of the one-warp-per-row forward
-  int fwd_path;   // norm forward of long rows: 1 = CTA-per-row pipeline, 2 = one warp per row,
-                  // 3 = one warp per row with one-pass LayerNorm statistics
-  int bwd_tmem;   // LayerNorm backward of bf16 long rows: 1 = accumulators in registers, 2 = in TMEM
+  int fwd_path;   // norm forward of long rows: 1 = CTA-per-row pipeline, 2 = one warp per row with
+                  // two-pass LayerNorm statistics, 3 = one warp per row with one shifted pass
 };
 extern Tuning g_tune;
 

@@ -15,7 +15,6 @@
 // (count, mean, M2) per thread and combines the triples with Chan et al.'s pairwise update.
 #include "norm_plan.h"
 #include "norm_rows.cuh"
-#include "tmem.cuh"
 
 namespace gn {
 namespace {
@@ -356,162 +355,6 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT, true)) l
   }
 }
 
-// ---------------------------------------------------------------- CTA path, accumulators in TMEM
-// The same backward with each thread's dw and db accumulators (2 x 32 fp32 at 4 vectors of bf16)
-// kept in tensor memory instead of registers: read, updated and written back once per row and
-// vector with 16-column tcgen05.ld / tcgen05.st. That takes ~64 registers off every thread, so
-// three CTAs of six warps fit an SM (register budget 112 a thread) where the register-resident
-// form fits two. The weight and bias stay bf16 in shared memory (three CTAs' stages and
-// parameters must fit the SM's 228 KiB). bf16 rows only, up to 5 consumer warps.
-constexpr int kTmemThreads = 192;
-
-template <typename T, int VPT, int EPI>
-__global__ void __maxnreg__(112) ln_bwd_tmem(const LnBwdArgs a, uint32_t tmem_cols) {
-  pdl_launch_dependents();  // the column reduction that follows may launch early
-  constexpr int E = Vec<T>::N, H = E / 2;
-  static_assert(E == 8, "one 16-column TMEM access holds one bf16 vector's dw and db");
-  constexpr int W = 2 * VPT * E;  // TMEM columns of one thread: dw then db of each vector
-  constexpr bool FAST = fast_math_for<T>();
-  extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ uint32_t tmem_slot;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int N = a.N, nfull = N / E, nvec = (N + E - 1) / E;
-  const RowPipe pipe(smem, a.stages, 2, 2, N, sizeof(T), sizeof(T));
-  const T* x = static_cast<const T*>(a.x);
-  const T* dy = static_cast<const T*>(a.dy);
-  T* dx = static_cast<T*>(a.dx);
-  const int ncw = (int)(blockDim.x >> 5) - 1;
-  if (tid == 0) pipe.init(ncw);
-  __syncthreads();
-  if (warp == 0) {
-    if (lane == 0)
-      pipe.produce(
-          a.rows,
-          [&](int64_t m, int t) -> const void* { return t == 0 ? (const void*)(x + m * a.ldx) : (const void*)(dy + m * a.lddy); },
-          a.err);
-    return;
-  }
-  const int ct = tid - 32, nct = ncw * 32, cw = warp - 1;
-  if (warp == 1) tmem_alloc_warp(&tmem_slot, tmem_cols);
-  stage_param<T, VPT>(pipe.param(0), static_cast<const T*>(a.w), N, nvec, 1.0f, ct, nct);
-  stage_param<T, VPT>(pipe.param(1), static_cast<const T*>(a.b), N, nvec, 0.0f, ct, nct);
-  pipe.red_zero(ct, nct);
-  tmem_fence_before_sync();
-  consumers_sync(nct);
-  tmem_fence_after_sync();
-  // this warp's lanes and columns: warps that share a lane quadrant take successive column blocks
-  const uint32_t tacc = tmem_slot + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(((warp - 1) >> 2) * W);
-  {
-    uint32_t z[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) z[i] = 0u;
-#pragma unroll
-    for (int j = 0; j < VPT; ++j) tmem_st16(tacc + 16 * j, z);
-  }
-  const float inv_n = 1.0f / (float)N;
-  const int64_t step = gridDim.x;
-  int s = 0;
-  uint32_t ph = 0, rb = 0;
-  bool failed = false;
-  float mu_n = 0.0f, rs_n = 0.0f;
-  if (blockIdx.x < a.rows) mu_n = __ldg(a.mean + blockIdx.x), rs_n = __ldg(a.rstd + blockIdx.x);
-  for (int64_t m = blockIdx.x; m < a.rows; m += step) {
-    const float mu = mu_n, rs = rs_n;
-    if (m + step < a.rows) mu_n = __ldg(a.mean + m + step), rs_n = __ldg(a.rstd + m + step);
-    const float2 rs2 = dup2(rs), nmr2 = dup2(-mu * rs);
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(&pipe.full[s], ph, a.err));
-    uint4 xr[VPT];
-    float2 gv[VPT][H];
-#pragma unroll
-    for (int j = 0; j < VPT; ++j) {
-      const int v = ct + j * nct;
-      xr[j] = load_raw<T>(pipe.at(s, 0), x + m * a.ldx, v, nfull, N, ok);
-      load_pairs<T>(pipe.at(s, 1), dy + m * a.lddy, v, nfull, N, ok, gv[j]);
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&pipe.empty[s]);
-    float2 s12 = dup2(0.0f), s22 = dup2(0.0f);
-#pragma unroll
-    for (int j = 0; j < VPT; ++j) {
-      const int v = ct + j * nct;
-      const int vv = v < nvec ? v : 0;
-      uint32_t acc[16];
-      tmem_wait_st();  // this thread's last store of these columns has landed
-      tmem_ld16(tacc + 16 * j, acc);
-      // weight, bias and x stay packed (one 32-bit word per element pair) and are widened pair by
-      // pair: the register budget of three CTAs per SM has no room for whole widened vectors
-      const uint4 wr = *reinterpret_cast<const uint4*>(pipe.param(0) + (size_t)vv * 16);
-      const uint4 br = *reinterpret_cast<const uint4*>(pipe.param(1) + (size_t)vv * 16);
-      const uint32_t ww[4] = {wr.x, wr.y, wr.z, wr.w}, bw[4] = {br.x, br.y, br.z, br.w};
-      const uint32_t xw[4] = {xr[j].x, xr[j].y, xr[j].z, xr[j].w};
-      tmem_wait_ld();  // the load's latency overlaps the shared-memory reads above
-#pragma unroll
-      for (int h = 0; h < H; ++h) {
-        const float2 wvh = make_float2(__uint_as_float(ww[h] << 16), __uint_as_float(ww[h] & 0xffff0000u));
-        const float2 bvh = make_float2(__uint_as_float(bw[h] << 16), __uint_as_float(bw[h] & 0xffff0000u));
-        const float2 xvh = make_float2(__uint_as_float(xw[h] << 16), __uint_as_float(xw[h] & 0xffff0000u));
-        const float2 xh = fma2(xvh, rs2, nmr2);
-        const float2 g = EPI == EPI_NONE ? gv[j][h] : mul2(gv[j][h], epi_grad2<EPI, FAST>(fma2(xh, wvh, bvh)));
-        const float2 gw = mul2(g, wvh);
-        gv[j][h] = gw;  // phase 2 needs only g w
-        s12 = add2(s12, gw);
-        s22 = fma2(gw, xh, s22);
-        const float2 dwp = fma2(g, xh, make_float2(__uint_as_float(acc[2 * h]), __uint_as_float(acc[2 * h + 1])));
-        const float2 dbp = add2(g, make_float2(__uint_as_float(acc[8 + 2 * h]), __uint_as_float(acc[9 + 2 * h])));
-        acc[2 * h] = __float_as_uint(dwp.x), acc[2 * h + 1] = __float_as_uint(dwp.y);
-        acc[8 + 2 * h] = __float_as_uint(dbp.x), acc[9 + 2 * h] = __float_as_uint(dbp.y);
-      }
-      tmem_st16(tacc + 16 * j, acc);
-    }
-    const float s1 = group_sum<32>(s12.x + s12.y);
-    const float s2 = group_sum<32>(s22.x + s22.y);
-    if (lane == 0) pipe.red_at(rb, 0)[cw] = s1, pipe.red_at(rb, 1)[cw] = s2;
-    if (consumers_sync_or(nct, !ok)) {
-      failed = true;
-      break;
-    }
-    const float t1 = pipe.red_sum(rb, 0, ncw), t2 = pipe.red_sum(rb, 1, ncw);
-    rb ^= 1u;
-    if (++s == a.stages) s = 0, ph ^= 1u;
-    const float2 nc1 = dup2(-t1 * inv_n), nc2 = dup2(-t2 * inv_n);
-    T* dxrow = dx + m * a.lddx;
-#pragma unroll
-    for (int j = 0; j < VPT; ++j) {
-      const int v = ct + j * nct;
-      if (v < nvec) {
-        float2 xv[H], o[H];
-        unpack2<T>(xr[j], xv);
-#pragma unroll
-        for (int h = 0; h < H; ++h) o[h] = mul2(rs2, add2(gv[j][h], fma2(fma2(xv[h], rs2, nmr2), nc2, nc1)));
-        store_pairs<T>(dxrow, v, nfull, N, o);
-      }
-    }
-  }
-  tmem_wait_st();
-  if (a.ws && !failed) {
-    float* part = a.ws + (int64_t)blockIdx.x * 2 * N;
-#pragma unroll
-    for (int j = 0; j < VPT; ++j) {
-      uint32_t acc[16];
-      tmem_ld16(tacc + 16 * j, acc);
-      tmem_wait_ld();
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        const int col = (ct + j * nct) * E + e;
-        if (col < N) {
-          part[col] = __uint_as_float(acc[e]);
-          part[N + col] = __uint_as_float(acc[8 + e]);
-        }
-      }
-    }
-  }
-  // every warp's tensor-memory accesses are complete before the allocating warp frees it
-  tmem_fence_before_sync();
-  consumers_sync(nct);
-  tmem_fence_after_sync();
-  if (warp == 1) tmem_dealloc_warp(tmem_slot, tmem_cols);
-}
-
 // ---------------------------------------------------------------- group path (short rows)
 
 template <typename T, int VPT, int EPI>
@@ -741,37 +584,6 @@ gn_status ln_plan(int64_t rows, int64_t hidden, gn_dtype dt, bool bwd, int epi, 
   return GN_OK;
 }
 
-void* pick_ln_tmem(int epi) {
-  if (epi == EPI_GELU_TANH) return (void*)ln_bwd_tmem<__nv_bfloat16, 4, EPI_GELU_TANH>;
-  if (epi == EPI_SILU) return (void*)ln_bwd_tmem<__nv_bfloat16, 4, EPI_SILU>;
-  return (void*)ln_bwd_tmem<__nv_bfloat16, 4, EPI_NONE>;
-}
-
-// The backward with its weight-gradient accumulators in tensor memory: bf16 rows of 129 .. 640
-// vectors (4 vectors a thread, at most 5 consumer warps). GN_ERR_UNSUPPORTED otherwise.
-gn_status ln_plan_tmem(int64_t rows, int64_t hidden, gn_dtype dt, int epi, NormPlan* p, void** kern, int* grid,
-                       uint32_t* cols) {
-  if (dt != GN_BF16 || g_tune.bwd_tmem == 1) return GN_ERR_UNSUPPORTED;
-  const int saved_vpt = g_tune.vpt;
-  g_tune.vpt = 4;
-  gn_status st = plan_norm(hidden, 2, 2, 2, 4, 160, p, 2);
-  g_tune.vpt = saved_vpt;
-  if (st != GN_OK || !p->cta || p->threads > kTmemThreads) return GN_ERR_UNSUPPORTED;
-  *kern = pick_ln_tmem(epi);
-  const int ncw = p->threads / 32 - 1;
-  uint32_t c = (uint32_t)((ncw + 3) / 4) * 2 * 4 * 8;
-  uint32_t c2 = 32;
-  while (c2 < c) c2 <<= 1;
-  *cols = c2;
-  int cap = g_tune.ctas_per_sm ? g_tune.ctas_per_sm : 8;
-  if (cap > (int)(512 / c2)) cap = (int)(512 / c2);  // every resident CTA's allocation fits the SM
-  int g = persistent_grid(*kern, p->threads, p->smem, cap);
-  if (g <= 0) return GN_ERR_CUDA;
-  if (rows < g) g = (int)(rows > 0 ? rows : 1);
-  *grid = g;
-  return GN_OK;
-}
-
 }  // namespace
 }  // namespace gn
 
@@ -820,10 +632,8 @@ extern "C" size_t gn_layernorm_bwd_workspace(int64_t rows, int64_t hidden, gn_dt
     NormPlan p;
     void* kern = nullptr;
     int g = 0;
-    uint32_t cols = 0;
     if (ln_plan(rows, hidden, dt, true, epi, &p, &kern, &g) != GN_OK) return 0;
     if (g > grid) grid = g;
-    if (ln_plan_tmem(rows, hidden, dt, epi, &p, &kern, &g, &cols) == GN_OK && g > grid) grid = g;
   }
   return (size_t)grid * 2 * (size_t)hidden * sizeof(float);
 }
@@ -850,9 +660,7 @@ extern "C" gn_status gn_layernorm_bwd(const void* x, const void* w, const void* 
   NormPlan p;
   void* kern = nullptr;
   int grid = 0;
-  uint32_t tmem_cols = 0;
-  gn_status st = ln_plan_tmem(rows, hidden, dt, epi, &p, &kern, &grid, &tmem_cols);
-  if (st == GN_ERR_UNSUPPORTED) st = ln_plan(rows, hidden, dt, true, epi, &p, &kern, &grid);
+  gn_status st = ln_plan(rows, hidden, dt, true, epi, &p, &kern, &grid);
   if (st != GN_OK) return st;
   const bool wgrad = dw || db;
   if (wgrad) {
@@ -867,9 +675,7 @@ extern "C" gn_status gn_layernorm_bwd(const void* x, const void* w, const void* 
   int lanes = p.lanes;
   void* args_cta[] = {&a};
   void* args_grp[] = {&a, &lanes};
-  void* args_tmem[] = {&a, &tmem_cols};
-  if (cudaLaunchKernel(kern, dim3(grid), dim3(p.threads), tmem_cols ? args_tmem : p.cta ? args_cta : args_grp, p.smem,
-                       s) != cudaSuccess)
+  if (cudaLaunchKernel(kern, dim3(grid), dim3(p.threads), p.cta ? args_cta : args_grp, p.smem, s) != cudaSuccess)
     return GN_ERR_CUDA;
   count_launches(1);
   if ((st = launch_status()) != GN_OK) return st;

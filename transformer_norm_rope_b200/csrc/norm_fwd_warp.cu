@@ -54,20 +54,10 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// Chan et al.'s combination of two (count, mean, M2) summaries, a before b in a fixed order
-__device__ __forceinline__ void chan_merge2(float& n, float& m, float& M2, float nb, float mb, float M2b) {
-  const float nn = n + nb;
-  if (nb == 0.0f || nn == 0.0f) return;
-  const float d = mb - m;
-  const float f = __fdividef(nb, nn);
-  M2 = M2 + M2b + d * d * n * f;
-  m = fmaf(d, f, m);
-  n = nn;
-}
-
 // MODE: 0 RMSNorm; 1 LayerNorm, statistics in two passes (mean, then centred squares); 2 LayerNorm,
-// statistics in one pass (each lane's row share in chunks of four vectors: chunk mean and centred
-// squares from registers, chunks and then lanes combined with Chan et al.'s update)
+// statistics in one pass around a shift K (the mean of each lane's first vector over the warp):
+// mean = K + S1 / N, var = S2 / N - (S1 / N)^2 with S1 = sum (x - K), S2 = sum (x - K)^2; |mean - K|
+// is of the order of the row's deviation over sqrt(256), so the subtraction loses nothing measurable
 template <typename T, int MODE, int EPI, bool GEMMA>
 __global__ void __launch_bounds__(kWarpFwdMaxWarps * 32, 1) norm_fwd_warp(const WarpFwdArgs a) {
   constexpr bool LN = MODE != 0;
@@ -172,67 +162,47 @@ __global__ void __launch_bounds__(kWarpFwdMaxWarps * 32, 1) norm_fwd_warp(const 
       stat_a = rsqrtf(fmaf(ss, inv_n, a.eps));
       stat_b = 0.0f;
     } else if constexpr (MODE == 2) {
-      float n = 0.0f, M2 = 0.0f;
-      for (int v0 = lane; v0 < nfull; v0 += 128) {
-        float2 f[4][H];
-        float2 s2 = dup2(0.0f);
-        int cnt = 0;
+      // one pass with a shift: K = the mean of the first vector of every lane that has a whole one
+      float k0;
+      {
+        float2 f[H];
+        unpack2<T>(*reinterpret_cast<const uint4*>(st + (size_t)(lane < nfull ? lane : 0) * 16), f);
+        float2 t = f[0];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int v = v0 + 32 * i;
-          if (v < nfull) {
-            unpack2<T>(*reinterpret_cast<const uint4*>(st + (size_t)v * 16), f[i]);
-            cnt += E;
-          } else {
-#pragma unroll
-            for (int h = 0; h < H; ++h) f[i][h] = dup2(0.0f);
-          }
-#pragma unroll
-          for (int h = 0; h < H; ++h) s2 = add2(s2, f[i][h]);
-        }
-        const float cm = __fdividef(s2.x + s2.y, (float)cnt);
-        const float2 ncm = dup2(-cm);
-        float2 q2 = dup2(0.0f);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          if (v0 + 32 * i < nfull)
-#pragma unroll
-            for (int h = 0; h < H; ++h) {
-              const float2 d = add2(f[i][h], ncm);
-              q2 = fma2(d, d, q2);
-            }
-        chan_merge2(n, mu, M2, (float)cnt, cm, q2.x + q2.y);
+        for (int h = 1; h < H; ++h) t = add2(t, f[h]);
+        const int nk = nfull < 32 ? nfull : 32;
+        k0 = warp_sum(lane < nfull ? t.x + t.y : 0.0f) / (float)(nk * E);
       }
-      if (tcnt && lane == (tv & 31)) {
-        float ts = 0.0f;
+      const float2 nk2 = dup2(-k0);
+      float2 s1[H], s2[H];
 #pragma unroll
-        for (int h = 0; h < H; ++h) ts += tail[h].x + tail[h].y;  // zero past N
-        const float tm = ts / (float)tcnt;
-        float tq = 0.0f;
+      for (int h = 0; h < H; ++h) s1[h] = s2[h] = dup2(0.0f);
+#pragma unroll 4
+      for (int v = lane; v < nfull; v += 32) {
+        float2 f[H];
+        unpack2<T>(*reinterpret_cast<const uint4*>(st + (size_t)v * 16), f);
 #pragma unroll
         for (int h = 0; h < H; ++h) {
-          const float d0 = 2 * h < tcnt ? tail[h].x - tm : 0.0f;
-          const float d1 = 2 * h + 1 < tcnt ? tail[h].y - tm : 0.0f;
-          tq = fmaf(d0, d0, fmaf(d1, d1, tq));
+          const float2 d = add2(f[h], nk2);
+          s1[h] = add2(s1[h], d);
+          s2[h] = fma2(d, d, s2[h]);
         }
-        chan_merge2(n, mu, M2, (float)tcnt, tm, tq);
       }
-      // lanes: xor butterfly with the lower lane's summary always first, so both partners
-      // compute the same merge and every lane ends with the same statistics
+      if (tcnt && lane == (tv & 31))
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float pn = __shfl_xor_sync(0xffffffffu, n, o);
-        const float pm = __shfl_xor_sync(0xffffffffu, mu, o);
-        const float pq = __shfl_xor_sync(0xffffffffu, M2, o);
-        if (lane & o) {
-          float an = pn, am = pm, aq = pq;
-          chan_merge2(an, am, aq, n, mu, M2);
-          n = an, mu = am, M2 = aq;
-        } else {
-          chan_merge2(n, mu, M2, pn, pm, pq);
+        for (int h = 0; h < H; ++h) {
+          const float d0 = 2 * h < tcnt ? tail[h].x - k0 : 0.0f;
+          const float d1 = 2 * h + 1 < tcnt ? tail[h].y - k0 : 0.0f;
+          s1[h].x += d0, s1[h].y += d1;
+          s2[h].x = fmaf(d0, d0, s2[h].x), s2[h].y = fmaf(d1, d1, s2[h].y);
         }
-      }
-      stat_a = rsqrtf(fmaf(M2, inv_n, a.eps));
+      float2 t1 = s1[0], t2 = s2[0];
+#pragma unroll
+      for (int h = 1; h < H; ++h) t1 = add2(t1, s1[h]), t2 = add2(t2, s2[h]);
+      const float m1 = warp_sum(t1.x + t1.y) * inv_n;  // mean - K
+      const float m2 = warp_sum(t2.x + t2.y) * inv_n;
+      mu = k0 + m1;
+      stat_a = rsqrtf(fmaxf(fmaf(-m1, m1, m2), 0.0f) + a.eps);
       stat_b = -mu * stat_a;
     } else {
       float2 acc[H];
@@ -345,10 +315,11 @@ void* pick_warp_fwd(int epi, bool gemma) {
   }
 }
 
+// LayerNorm: the one-pass shifted statistics unless fwd_path 2 asks for the two-pass form
 template <typename T>
 void* pick_warp_fwd_t(bool ln, int epi, bool gemma) {
   if (!ln) return pick_warp_fwd<T, 0>(epi, gemma);
-  return g_tune.fwd_path == 3 ? pick_warp_fwd<T, 2>(epi, gemma) : pick_warp_fwd<T, 1>(epi, gemma);
+  return g_tune.fwd_path == 2 ? pick_warp_fwd<T, 1>(epi, gemma) : pick_warp_fwd<T, 2>(epi, gemma);
 }
 
 }  // namespace
@@ -362,6 +333,8 @@ gn_status launch_norm_fwd_warp(bool ln, const void* x, const void* w, const void
   if (nfull < 1) return GN_ERR_UNSUPPORTED;
   const uint32_t slot = pipe_slot_bytes(nfull * 16);
   const uint32_t pbytes = pipe_slot_bytes((N + E - 1) / E * E * 4);
+  unsigned* err = device_err_word();
+  if (!err) return GN_ERR_CUDA;
   const size_t limit = smem_optin();
   const size_t fixed = kWarpFwdHeader + (ln ? 2u : 1u) * (size_t)pbytes;
   int stages = g_tune.stages ? g_tune.stages : 2;
@@ -377,8 +350,6 @@ gn_status launch_norm_fwd_warp(bool ln, const void* x, const void* w, const void
   if (grid <= 0) return GN_ERR_CUDA;
   const int64_t need = (rows + warps - 1) / warps;
   if (need < grid) grid = (int)need;
-  unsigned* err = device_err_word();
-  if (!err) return GN_ERR_CUDA;
   WarpFwdArgs a{x, w, b, y, stat0, stat1, rows, ldx, ldy, (int)N, stages, slot, pbytes, eps, err};
   void* args[] = {&a};
   if (cudaLaunchKernel(kern, dim3(grid), dim3(warps * 32), args, smem, stream) != cudaSuccess) return GN_ERR_CUDA;

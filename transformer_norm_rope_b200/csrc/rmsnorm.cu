@@ -474,7 +474,7 @@ extern "C" gn_status gn_rmsnorm_fwd(const void* x, const void* w, void* y, float
   NormPlan p;
   gn_status st = plan_norm(hidden, es, 1, 1, 8, 320, &p);
   if (st != GN_OK) return st;
-  if (p.cta && g_tune.fwd_path != 1) {  // long rows: one warp per row unless the row does not fit
+  if (p.cta && (g_tune.fwd_path == 2 || g_tune.fwd_path == 3)) {  // long rows, one warp per row on request
     st = launch_norm_fwd_warp(false, x, w, nullptr, y, inv_rms, nullptr, rows, hidden, ld_x, ld_y, eps, gemma != 0,
                               epi, dt, (cudaStream_t)stream);
     if (st != GN_ERR_UNSUPPORTED) return st;
