@@ -245,6 +245,47 @@ gn_status gn_norm_linear_fwd(const void* x, const void* Wf, const float* c, cons
                              int64_t ldy, float eps, gn_norm norm, gn_epilogue epi, gn_dtype dt,
                              void* stream);
 
+/* ---- TiledLinear backward ([H] "内核三 TiledLinear": per chunk of tokens the backward recomputes
+ * the pre-activation z = x W^T + b, forms dz = dy * act'(z), then dx = dz W, dW += dz^T x,
+ * db += sum dz; the calls below run these steps on this library's kernels) ---- */
+
+/* dz [M, N] = dy [M, N] * act'(x [M, K] Wf^T + d): the chunk's recompute on the tensor-core
+ * kernels (as gn_norm_linear_fwd with GN_NORM_NONE) with the activation gradient applied where the
+ * accumulators are read back, so z is never written. Wf [N, K] from gn_norm_linear_prepare
+ * (GN_NORM_NONE), d [N] fp32 (may be NULL = 0). bf16 only. Row strides ldx, lddy, lddz in
+ * elements, multiples of 8; K a multiple of 8; x, Wf, dy, dz, d 16-byte aligned.
+ * Errors: GN_ERR_SHAPE, GN_ERR_DTYPE (epilogue), GN_ERR_NULL, GN_ERR_ALIGN, GN_ERR_UNSUPPORTED
+ * (fp32), GN_ERR_CUDA. M == 0 or N == 0: nothing is launched. */
+gn_status gn_linear_act_grad(const void* x, const void* Wf, const float* d, const void* dy, void* dz,
+                             int64_t M, int64_t N, int64_t K, int64_t ldx, int64_t lddy, int64_t lddz,
+                             gn_epilogue epi, gn_dtype dt, void* stream);
+
+/* C [M, N] += A [M, K] B [N, K]^T with C fp32 (updated in place: a weight gradient summed over
+ * chunks), A and B bf16 with the contraction index K contiguous (row strides lda, ldb, multiples
+ * of 8; K a multiple of 8), on the tensor-core kernels. ldc a multiple of 4; A, B, C 16-byte
+ * aligned. Errors as gn_linear_act_grad. */
+gn_status gn_linear_acc_f32(const void* A, const void* B, float* C, int64_t M, int64_t N, int64_t K,
+                            int64_t lda, int64_t ldb, int64_t ldc, gn_dtype dt, void* stream);
+
+/* dst [cols, rows] = src [rows, cols]^T (bf16; cols and both row strides multiples of 8; both
+ * pointers 16-byte aligned). A row count that is not a multiple of 8 is padded: each output row
+ * is written up to the next multiple of 8 columns, with zeros past the input rows (ld_dst must
+ * cover them). The weight gradient contracts over the tokens, so its operands are transposed to
+ * put the tokens contiguous.
+ * Errors: GN_ERR_SHAPE, GN_ERR_NULL, GN_ERR_ALIGN, GN_ERR_UNSUPPORTED (fp32), GN_ERR_CUDA. */
+gn_status gn_transpose(const void* src, void* dst, int64_t rows, int64_t cols, int64_t ld_src,
+                       int64_t ld_dst, gn_dtype dt, void* stream);
+
+/* Column sums of a bf16 matrix src [rows, cols] (row stride ld; cols and ld even; src 4-byte
+ * aligned) into fp32 out [cols]: out = sum (accumulate == 0) or out += sum (accumulate != 0), in
+ * a fixed order (the same bits on every run): 64 row slices summed into the caller's workspace
+ * ws (gn_colsum_bf16_workspace(cols) bytes, 16-byte aligned), then the slices in order.
+ * Errors: GN_ERR_SHAPE, GN_ERR_NULL, GN_ERR_ALIGN, GN_ERR_WORKSPACE, GN_ERR_UNSUPPORTED (fp32),
+ * GN_ERR_CUDA. */
+size_t gn_colsum_bf16_workspace(int64_t cols);
+gn_status gn_colsum_bf16(const void* src, float* out, void* ws, size_t ws_bytes, int64_t rows,
+                         int64_t cols, int64_t ld, int accumulate, gn_dtype dt, void* stream);
+
 /* Gradient of the epilogue activation, elementwise over n elements: dz = dy * act'(z) (act as
  * in the gn_epilogue values; GN_EPI_NONE gives dz = dy). z is the pre-activation, dy the
  * gradient of act(z). The backward of a linear layer with an activation needs it before its two

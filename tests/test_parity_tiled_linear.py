@@ -83,3 +83,40 @@ def test_act_grad_matches_oracle_derivative(gpu):
             gf = dy.astype(np.float64) if dt == "f32" else wl.bf16_to_f32(dy).astype(np.float64)
             ref = gf * np.array([oracle.act_grad(act, v) for v in zf])
             assert_close(to_np(dz), ref, tol, f"act_grad {dt} {act}")
+
+
+@pytest.mark.parametrize("rows,cols", [(300, 264), (64, 5120), (1000, 72), (8, 8)])
+def test_transpose_and_column_sums(gpu, rows, cols):
+    """The backward's memory-bound steps: the transpose is exact (bit for bit, zero-padded up to
+    a multiple of 8 rows) and the column sums match the fp64 sums of the same bf16 values."""
+    g = np.random.default_rng(rows)
+    a = wl.bf16_bits(g.standard_normal((rows, cols)).astype(np.float32))
+    t = to_dev(a)
+    tt = gpu.transpose(t)
+    r8 = (rows + 7) // 8 * 8
+    assert tuple(tt.shape) == (cols, r8)
+    assert torch.equal(tt[:, :rows], t.t()) and bool((tt[:, rows:] == 0).all())
+    out = torch.full((cols,), 1.5, dtype=torch.float32, device="cuda")
+    gpu.colsum_bf16(t, out, accumulate=True)
+    ref = wl.bf16_to_f32(a).astype(np.float64).sum(0) + 1.5
+    assert_close(to_np(out), ref, (1e-5, 1e-5 * float(np.abs(ref).max())), "colsum")
+    a2 = gpu.colsum_bf16(t, torch.empty(cols, dtype=torch.float32, device="cuda"))
+    b2 = gpu.colsum_bf16(t, torch.empty(cols, dtype=torch.float32, device="cuda"))
+    assert torch.equal(a2, b2)  # fixed order
+
+
+@pytest.mark.parametrize("M,N,K", [(300, 264, 1024), (5120, 512, 1000), (100, 600, 200)])
+def test_fp32_accumulating_product(gpu, M, N, K):
+    """C += A B^T on the tensor cores with an fp32 accumulator updated in place, against the fp64
+    product of the same bf16 operands (K padded with zeros to a multiple of 8 by the transpose
+    path where the caller needs it; here K is a multiple of 8)."""
+    g = np.random.default_rng(M + N + K)
+    A = wl.bf16_bits(g.standard_normal((M, K)).astype(np.float32))
+    B = wl.bf16_bits(g.standard_normal((N, K)).astype(np.float32))
+    C0 = g.standard_normal((M, N)).astype(np.float32)
+    C = to_dev(C0)
+    gpu.linear_acc_f32(to_dev(A), to_dev(B), C)
+    torch.cuda.synchronize()
+    ref = C0.astype(np.float64) + wl.bf16_to_f32(A).astype(np.float64) @ wl.bf16_to_f32(B).astype(np.float64).T
+    assert_close(to_np(C), ref, (1e-5, 1e-4 * math.sqrt(K)), "C += A B^T")
+    assert gpu.device_error(clear=True) == 0

@@ -54,6 +54,11 @@ SIGNATURES = {
     "gn_norm_linear_prepare": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _int, _int, _int, _vp]),
     "gn_norm_linear_fwd": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _f32, _int,
                                  _int, _int, _vp]),
+    "gn_linear_act_grad": (_st, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _int, _int, _vp]),
+    "gn_linear_acc_f32": (_st, [_vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _int, _vp]),
+    "gn_transpose": (_st, [_vp, _vp, _i64, _i64, _i64, _i64, _int, _vp]),
+    "gn_colsum_bf16_workspace": (_sz, [_i64]),
+    "gn_colsum_bf16": (_st, [_vp, _vp, _vp, _sz, _i64, _i64, _i64, _int, _int, _vp]),
     "gn_act_grad": (_st, [_vp, _vp, _vp, _i64, _int, _int, _vp]),
     "gn_launch_count": (C.c_uint64, []),
     "gn_device_error": (_st, [C.POINTER(C.c_uint), _int]),
@@ -401,6 +406,69 @@ def act_grad(z, dy, epilogue="silu", out=None, stream=None):
     check(gn_act_grad(_ptr(z), _ptr(dy), _ptr(dz), dy.numel(), _epi(epilogue), _dt(dy), _stream(stream)),
           "gn_act_grad")
     return dz
+
+
+def linear_act_grad(x, Wf, d, dy, epilogue="silu", out=None, stream=None):
+    """dz = dy * act'(x Wf^T + d) [M, N] (bf16) on the tensor-core kernels (z never stored)."""
+    _rows(x)
+    M, K = x.shape
+    _need(Wf, "Wf", like=x, dtype=x.dtype)
+    if Wf.dim() != 2 or Wf.shape[1] != K:
+        raise ValueError(f"Wf has shape {tuple(Wf.shape)}, expected [N, {K}]")
+    N = Wf.shape[0]
+    _need(d, "d", like=x, shape=(N,), dtype=_torch().float32, optional=True)
+    _need(dy, "dy", like=x, shape=(M, N), dtype=x.dtype, contiguous=False)
+    _rows(dy, "dy", like=x, dtype=x.dtype)
+    dz = _torch().empty((M, N), dtype=x.dtype, device=x.device) if out is None else out
+    _need(dz, "out", like=x, shape=(M, N), dtype=x.dtype, contiguous=False)
+    _rows(dz, "out", like=x, dtype=x.dtype)
+    check(gn_linear_act_grad(_ptr(x), _ptr(Wf), _ptr(d), _ptr(dy), _ptr(dz), M, N, K, x.stride(0), dy.stride(0),
+                             dz.stride(0), _epi(epilogue), _dt(x), _stream(stream)), "gn_linear_act_grad")
+    return dz
+
+
+def linear_acc_f32(A, B, C, stream=None):
+    """C [M, N] (fp32, in place) += A [M, K] B [N, K]^T (bf16, K contiguous)."""
+    torch = _torch()
+    _rows(A, "A")
+    _rows(B, "B", like=A, dtype=A.dtype)
+    M, K = A.shape
+    if B.dim() != 2 or B.shape[1] != K:
+        raise ValueError(f"B has shape {tuple(B.shape)}, expected [N, {K}]")
+    N = B.shape[0]
+    _need(C, "C", like=A, shape=(M, N), dtype=torch.float32, contiguous=False)
+    _rows(C, "C", like=A, dtype=torch.float32)
+    check(gn_linear_acc_f32(_ptr(A), _ptr(B), _ptr(C), M, N, K, A.stride(0), B.stride(0), C.stride(0), _dt(A),
+                            _stream(stream)), "gn_linear_acc_f32")
+    return C
+
+
+def transpose(src, out=None, stream=None):
+    """src [rows, cols] -> [cols, rows8] (bf16), rows8 = rows rounded up to 8: the columns past
+    rows are zero."""
+    rows, cols, ld = _rows(src, "src")
+    if src.dim() != 2:
+        raise ValueError("transpose takes a matrix")
+    rows8 = (rows + 7) // 8 * 8
+    dst = _torch().empty((cols, rows8), dtype=src.dtype, device=src.device) if out is None else out
+    _need(dst, "out", like=src, shape=(cols, rows8), dtype=src.dtype, contiguous=False)
+    _, _, ldd = _rows(dst, "out", like=src, dtype=src.dtype)
+    check(gn_transpose(_ptr(src), _ptr(dst), rows, cols, ld, ldd, _dt(src), _stream(stream)), "gn_transpose")
+    return dst
+
+
+def colsum_bf16(src, out, accumulate=False, ws=None, stream=None):
+    """out [cols] (fp32) = (or +=) column sums of src [rows, cols] (bf16), fixed order."""
+    torch = _torch()
+    rows, cols, ld = _rows(src, "src")
+    _need(out, "out", like=src, shape=(cols,), dtype=torch.float32)
+    nws = gn_colsum_bf16_workspace(cols)
+    if ws is None:
+        ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=src.device)
+    _need(ws, "ws", like=src, numel=ws.numel(), dtype=torch.uint8)
+    check(gn_colsum_bf16(_ptr(src), _ptr(out), _ptr(ws), ws.numel(), rows, cols, ld, int(accumulate), _dt(src),
+                         _stream(stream)), "gn_colsum_bf16")
+    return out
 
 
 def torch_empty_like(t):

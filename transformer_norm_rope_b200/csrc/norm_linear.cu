@@ -88,7 +88,73 @@ struct NlArgs {
   int64_t ldy;
   float eps;
   unsigned* err;
+  const __nv_bfloat16* dy;  // OUT_DGRAD: gradient of the activation's output [M, N], row stride lddy
+  int64_t lddy;
+  float* y32;               // OUT_ACC32: fp32 accumulator [M, N], row stride ldy
 };
+
+// What the epilogue writes:
+//   OUT_BF16  : y = act(rstd (x Wf^T) - rstd mean c + d) in bf16 (the layer's forward);
+//   OUT_DGRAD : y = dy * act'(x Wf^T + d) in bf16 (no norm: the TiledLinear recompute of a chunk's
+//               pre-activation with its gradient applied; the pre-activation is never stored);
+//   OUT_ACC32 : y32 += x Wf^T in fp32 (no norm, no bias, no activation: a weight gradient summed
+//               over token chunks).
+enum NlOut { OUT_BF16 = 0, OUT_DGRAD = 1, OUT_ACC32 = 2 };
+
+// The 32 columns col0.. of row m of the epilogue's output from the 32 accumulator values v:
+// o = the corrected pre-activation (OUT_BF16: already activated).
+template <int OUT, int EPI>
+__device__ __forceinline__ void nl_store32(const NlArgs& a, int m, int col0, const float (&o)[32]) {
+  const bool whole = col0 + 32 <= a.N;
+  if constexpr (OUT == OUT_ACC32) {
+    float* row = a.y32 + (int64_t)m * a.ldy + col0;
+    if (whole) {
+#pragma unroll
+      for (int i = 0; i < 32; i += 4) {
+        float4 t = *reinterpret_cast<const float4*>(row + i);
+        t.x += o[i], t.y += o[i + 1], t.z += o[i + 2], t.w += o[i + 3];
+        *reinterpret_cast<float4*>(row + i) = t;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (col0 + i < a.N) row[i] += o[i];
+    }
+  } else {
+    float r[32];
+    if constexpr (OUT == OUT_DGRAD) {
+      const __nv_bfloat16* g = a.dy + (int64_t)m * a.lddy + col0;
+      if (whole) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 8) {
+          float f8[8];
+          Vec<__nv_bfloat16>::unpack(ld_stream(g + i), f8);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) r[i + e] = f8[e] * epi_grad<EPI, true>(o[i + e]);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          r[i] = col0 + i < a.N ? __bfloat162float(g[i]) * epi_grad<EPI, true>(o[i]) : 0.0f;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) r[i] = o[i];
+    }
+    __nv_bfloat16* yrow = a.y + (int64_t)m * a.ldy;
+    if (whole) {
+#pragma unroll
+      for (int i = 0; i < 32; i += 8) {
+        const float f8[8] = {r[i], r[i + 1], r[i + 2], r[i + 3], r[i + 4], r[i + 5], r[i + 6], r[i + 7]};
+        st_stream(yrow + col0 + i, Vec<__nv_bfloat16>::pack(f8));
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (col0 + i < a.N) yrow[col0 + i] = __float2bfloat16_rn(r[i]);
+    }
+  }
+}
 
 // ---------------------------------------------------------------- PTX wrappers
 
@@ -185,7 +251,7 @@ __device__ __forceinline__ float nl_act(float z) {
 
 // ---------------------------------------------------------------- forward kernel
 
-template <int MH, int NORM, int EPI>
+template <int MH, int NORM, int EPI, int OUT = OUT_BF16>
 __global__ void __launch_bounds__(Tile<MH>::Threads, 1)
     norm_linear_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const NlArgs a) {
@@ -372,36 +438,25 @@ __global__ void __launch_bounds__(Tile<MH>::Threads, 1)
       }
       const float nsm = -rs * mu;
       const int m = m0 + r;
-      __nv_bfloat16* yrow = a.y + (int64_t)m * a.ldy;
       for (int j = 0; j < kBN / 32; ++j) {
         const int col0 = n0 + 32 * j;
         if (col0 >= a.N) break;  // uniform over the warp
         float v[32];
         tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(kAccCols * h + 32 * j), v);
-        const bool whole = col0 + 32 <= a.N;
         float o[32];
 #pragma unroll
         for (int i = 0; i < 32; i += 4) {
           const float4 c4 = *reinterpret_cast<const float4*>(col_c + 32 * j + i);
           const float4 d4 = *reinterpret_cast<const float4*>(col_d + 32 * j + i);
-          o[i + 0] = nl_act<EPI>(fmaf(rs, v[i + 0], fmaf(nsm, c4.x, d4.x)));
-          o[i + 1] = nl_act<EPI>(fmaf(rs, v[i + 1], fmaf(nsm, c4.y, d4.y)));
-          o[i + 2] = nl_act<EPI>(fmaf(rs, v[i + 2], fmaf(nsm, c4.z, d4.z)));
-          o[i + 3] = nl_act<EPI>(fmaf(rs, v[i + 3], fmaf(nsm, c4.w, d4.w)));
+          o[i + 0] = fmaf(rs, v[i + 0], fmaf(nsm, c4.x, d4.x));
+          o[i + 1] = fmaf(rs, v[i + 1], fmaf(nsm, c4.y, d4.y));
+          o[i + 2] = fmaf(rs, v[i + 2], fmaf(nsm, c4.z, d4.z));
+          o[i + 3] = fmaf(rs, v[i + 3], fmaf(nsm, c4.w, d4.w));
         }
-        if (m < a.M) {
-          if (whole) {
+        if constexpr (OUT == OUT_BF16)
 #pragma unroll
-            for (int i = 0; i < 32; i += 8) {
-              const float f8[8] = {o[i], o[i + 1], o[i + 2], o[i + 3], o[i + 4], o[i + 5], o[i + 6], o[i + 7]};
-              st_stream(yrow + col0 + i, Vec<__nv_bfloat16>::pack(f8));
-            }
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (col0 + i < a.N) yrow[col0 + i] = __float2bfloat16_rn(o[i]);
-          }
-        }
+          for (int i = 0; i < 32; ++i) o[i] = nl_act<EPI>(o[i]);
+        if (m < a.M) nl_store32<OUT, EPI>(a, m, col0, o);
       }
       if (NORM != GN_NORM_NONE && blockIdx.x == 0 && m < a.M) {
         if (a.mean) a.mean[m] = mu;
@@ -497,7 +552,7 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
       : "memory");
 }
 
-template <int NORM, int EPI>
+template <int NORM, int EPI, int OUT = OUT_BF16>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     norm_linear_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const NlArgs a) {
@@ -604,37 +659,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     tc_fence_after();
     if (ok) {
       const float nsm = -rs * mu;
-      __nv_bfloat16* yrow = a.y + (int64_t)m * a.ldy;
       for (int cb = 0; cb < 256 / 32; ++cb) {
         const int lc = 256 * j + 32 * cb;  // column of the pair tile
         const int col0 = n0 + lc;
         if (col0 >= a.N) break;  // uniform over the warp
         float v[32];
         tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(kAccCols * j + 32 * cb), v);
-        const bool whole = col0 + 32 <= a.N;
         float o[32];
 #pragma unroll
         for (int i = 0; i < 32; i += 4) {
           const float4 c4 = *reinterpret_cast<const float4*>(col_c + lc + i);
           const float4 d4 = *reinterpret_cast<const float4*>(col_d + lc + i);
-          o[i + 0] = nl_act<EPI>(fmaf(rs, v[i + 0], fmaf(nsm, c4.x, d4.x)));
-          o[i + 1] = nl_act<EPI>(fmaf(rs, v[i + 1], fmaf(nsm, c4.y, d4.y)));
-          o[i + 2] = nl_act<EPI>(fmaf(rs, v[i + 2], fmaf(nsm, c4.z, d4.z)));
-          o[i + 3] = nl_act<EPI>(fmaf(rs, v[i + 3], fmaf(nsm, c4.w, d4.w)));
+          o[i + 0] = fmaf(rs, v[i + 0], fmaf(nsm, c4.x, d4.x));
+          o[i + 1] = fmaf(rs, v[i + 1], fmaf(nsm, c4.y, d4.y));
+          o[i + 2] = fmaf(rs, v[i + 2], fmaf(nsm, c4.z, d4.z));
+          o[i + 3] = fmaf(rs, v[i + 3], fmaf(nsm, c4.w, d4.w));
         }
-        if (m < a.M) {
-          if (whole) {
+        if constexpr (OUT == OUT_BF16)
 #pragma unroll
-            for (int i = 0; i < 32; i += 8) {
-              const float f8[8] = {o[i], o[i + 1], o[i + 2], o[i + 3], o[i + 4], o[i + 5], o[i + 6], o[i + 7]};
-              st_stream(yrow + col0 + i, Vec<__nv_bfloat16>::pack(f8));
-            }
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (col0 + i < a.N) yrow[col0 + i] = __float2bfloat16_rn(o[i]);
-          }
-        }
+          for (int i = 0; i < 32; ++i) o[i] = nl_act<EPI>(o[i]);
+        if (m < a.M) nl_store32<OUT, EPI>(a, m, col0, o);
       }
     }
   }
@@ -786,48 +830,73 @@ bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, in
 }
 
 template <int MH, int NORM>
-void* pick_epi(int epi) {
+void* pick_epi(int epi, int out) {
+  if constexpr (NORM == GN_NORM_NONE) {  // the gradient modes exist without a norm only
+    if (out == OUT_DGRAD) {
+      if (epi == GN_EPI_GELU_TANH) return (void*)norm_linear_kernel<MH, NORM, EPI_GELU_TANH, OUT_DGRAD>;
+      if (epi == GN_EPI_SILU) return (void*)norm_linear_kernel<MH, NORM, EPI_SILU, OUT_DGRAD>;
+      return (void*)norm_linear_kernel<MH, NORM, EPI_NONE, OUT_DGRAD>;
+    }
+    if (out == OUT_ACC32) return (void*)norm_linear_kernel<MH, NORM, EPI_NONE, OUT_ACC32>;
+  } else if (out != OUT_BF16) {
+    return nullptr;
+  }
   if (epi == GN_EPI_GELU_TANH) return (void*)norm_linear_kernel<MH, NORM, EPI_GELU_TANH>;
   if (epi == GN_EPI_SILU) return (void*)norm_linear_kernel<MH, NORM, EPI_SILU>;
   return (void*)norm_linear_kernel<MH, NORM, EPI_NONE>;
 }
 
 template <int MH>
-void* pick(int norm, int epi) {
-  return norm == GN_NORM_LN    ? pick_epi<MH, GN_NORM_LN>(epi)
-         : norm == GN_NORM_RMS ? pick_epi<MH, GN_NORM_RMS>(epi)
-                               : pick_epi<MH, GN_NORM_NONE>(epi);
+void* pick(int norm, int epi, int out) {
+  return norm == GN_NORM_LN    ? pick_epi<MH, GN_NORM_LN>(epi, out)
+         : norm == GN_NORM_RMS ? pick_epi<MH, GN_NORM_RMS>(epi, out)
+                               : pick_epi<MH, GN_NORM_NONE>(epi, out);
 }
 
 template <int MH>
 bool set_smem_attr() {
   for (int norm = 0; norm < 3; ++norm)
     for (int epi = 0; epi < 3; ++epi)
-      if (cudaFuncSetAttribute(pick<MH>(norm, epi), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)Tile<MH>::Smem) != cudaSuccess)
-        return false;
+      for (int out = 0; out < 3; ++out) {
+        void* k = pick<MH>(norm, epi, out);
+        if (k && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Tile<MH>::Smem) !=
+                     cudaSuccess)
+          return false;
+      }
   return true;
 }
 
 template <int NORM>
-void* pick_pair_epi(int epi) {
+void* pick_pair_epi(int epi, int out) {
+  if constexpr (NORM == GN_NORM_NONE) {
+    if (out == OUT_DGRAD) {
+      if (epi == GN_EPI_GELU_TANH) return (void*)norm_linear_pair_kernel<NORM, EPI_GELU_TANH, OUT_DGRAD>;
+      if (epi == GN_EPI_SILU) return (void*)norm_linear_pair_kernel<NORM, EPI_SILU, OUT_DGRAD>;
+      return (void*)norm_linear_pair_kernel<NORM, EPI_NONE, OUT_DGRAD>;
+    }
+    if (out == OUT_ACC32) return (void*)norm_linear_pair_kernel<NORM, EPI_NONE, OUT_ACC32>;
+  } else if (out != OUT_BF16) {
+    return nullptr;
+  }
   if (epi == GN_EPI_GELU_TANH) return (void*)norm_linear_pair_kernel<NORM, EPI_GELU_TANH>;
   if (epi == GN_EPI_SILU) return (void*)norm_linear_pair_kernel<NORM, EPI_SILU>;
   return (void*)norm_linear_pair_kernel<NORM, EPI_NONE>;
 }
 
-void* pick_pair(int norm, int epi) {
-  return norm == GN_NORM_LN    ? pick_pair_epi<GN_NORM_LN>(epi)
-         : norm == GN_NORM_RMS ? pick_pair_epi<GN_NORM_RMS>(epi)
-                               : pick_pair_epi<GN_NORM_NONE>(epi);
+void* pick_pair(int norm, int epi, int out) {
+  return norm == GN_NORM_LN    ? pick_pair_epi<GN_NORM_LN>(epi, out)
+         : norm == GN_NORM_RMS ? pick_pair_epi<GN_NORM_RMS>(epi, out)
+                               : pick_pair_epi<GN_NORM_NONE>(epi, out);
 }
 
 bool set_pair_smem_attr() {
   for (int norm = 0; norm < 3; ++norm)
     for (int epi = 0; epi < 3; ++epi)
-      if (cudaFuncSetAttribute(pick_pair(norm, epi), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPairSmem) !=
-          cudaSuccess)
-        return false;
+      for (int out = 0; out < 3; ++out) {
+        void* k = pick_pair(norm, epi, out);
+        if (k && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPairSmem) != cudaSuccess)
+          return false;
+      }
   return true;
 }
 
@@ -837,6 +906,73 @@ bool set_pair_smem_attr() {
 #ifndef GN_NL_PAIR
 #define GN_NL_PAIR 1
 #endif
+
+// The launch shared by the forward and the TiledLinear backward products: y (bf16, OUT_BF16 and
+// OUT_DGRAD) or y32 (fp32, OUT_ACC32) [M, N] from x [M, K] (row stride ldx) and Wf [N, K] (row
+// stride ldw), arguments validated by the caller.
+gn_status nl_run(const void* x, int64_t ldx, const void* Wf, int64_t ldw, const float* c, const float* d, void* y,
+                 float* y32, int64_t ldy, const void* dy, int64_t lddy, float* mean, float* rstd, int64_t M,
+                 int64_t N, int64_t K, float eps, int norm, int epi, int out, cudaStream_t stream) {
+  // pairs of SMs sharing 256 x 512 tiles once there are more than 128 rows and 256 columns;
+  // one SM per 256 x 256 tile (two accumulators) for fewer columns; 128 x 256 for few rows
+  const bool pair = GN_NL_PAIR && M > kUM && N > kBN;
+  const int mh = M > kUM ? GN_NL_MH : 1;
+  const int bm = pair ? 2 * kUM : kUM * mh;
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, x, M, K, ldx, pair ? (uint32_t)kUM : (uint32_t)bm) ||
+      !make_map(&tb, Wf, N, K, ldw, pair ? 128u : (uint32_t)kBN))
+    return GN_ERR_CUDA;
+  void* kern = pair ? pick_pair(norm, epi, out) : mh == 2 ? pick<2>(norm, epi, out) : pick<1>(norm, epi, out);
+  if (!kern) return GN_ERR_UNSUPPORTED;
+  // the dynamic shared-memory limits are attributes of the kernels on the current device: set
+  // them once per device (0 = not yet, 1 = set, -1 = failed)
+  static std::mutex attr_mu;
+  static signed char attr_state[64];
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GN_ERR_CUDA;
+  {
+    std::lock_guard<std::mutex> lk(attr_mu);
+    if (!attr_state[dev]) attr_state[dev] = set_smem_attr<1>() && set_smem_attr<2>() && set_pair_smem_attr() ? 1 : -1;
+    if (attr_state[dev] < 0) return GN_ERR_CUDA;
+  }
+  NlArgs a{};
+  a.c = c, a.d = d;
+  a.y = static_cast<__nv_bfloat16*>(y);
+  a.y32 = y32;
+  a.dy = static_cast<const __nv_bfloat16*>(dy);
+  a.lddy = lddy;
+  a.mean = mean, a.rstd = rstd;
+  a.M = (int)M, a.N = (int)N, a.K = (int)K;
+  a.ldy = ldy;
+  a.eps = eps;
+  a.err = device_err_word();
+  if (!a.err) return GN_ERR_CUDA;
+  if (pair && norm != GN_NORM_NONE) {  // the pair kernel reads the row statistics: compute them first
+    const unsigned sblocks = (unsigned)((M + 7) / 8);
+    if (norm == GN_NORM_LN)
+      norm_stats_kernel<GN_NORM_LN><<<sblocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), ldx, (int)M,
+                                                                 (int)K, eps, mean, rstd);
+    else
+      norm_stats_kernel<GN_NORM_RMS><<<sblocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), ldx, (int)M,
+                                                                  (int)K, eps, mean, rstd);
+    count_launches(1);
+    if (launch_status() != GN_OK) return GN_ERR_CUDA;
+  }
+  const dim3 grid(pair ? (unsigned)(2 * ((N + kPairN - 1) / kPairN)) : (unsigned)((N + kBN - 1) / kBN),
+                  (unsigned)((M + bm - 1) / bm));
+  void* args[] = {&ta, &tb, &a};
+  const int threads = pair ? kPairThreads : mh == 2 ? Tile<2>::Threads : Tile<1>::Threads;
+  const size_t smem = pair ? kPairSmem : mh == 2 ? Tile<2>::Smem : Tile<1>::Smem;
+  if (cudaLaunchKernel(kern, grid, dim3(threads), args, smem, stream) != cudaSuccess) return GN_ERR_CUDA;
+  count_launches(1);
+  return launch_status();
+}
+
+// shape checks shared by the entry points: K (the contraction) and every row stride a multiple of
+// 8 elements (16-byte rows for the tensor maps)
+bool nl_shape_ok(int64_t M, int64_t N, int64_t K) {
+  return M >= 0 && N >= 0 && K > 0 && K % 8 == 0 && M <= (int64_t)65535 * kUM && N <= INT32_MAX && K <= INT32_MAX;
+}
 
 }  // namespace
 }  // namespace gn
@@ -876,60 +1012,36 @@ extern "C" gn_status gn_norm_linear_fwd(const void* x, const void* Wf, const flo
   if (dt != GN_BF16) return dt_ok(dt) ? GN_ERR_UNSUPPORTED : GN_ERR_DTYPE;
   if (!epi_ok(epi)) return GN_ERR_DTYPE;
   if (norm != GN_NORM_RMS && norm != GN_NORM_LN && norm != GN_NORM_NONE) return GN_ERR_SHAPE;
-  if (M < 0 || N < 0 || K <= 0 || ldx < K || ldy < N || K % 8 || ldx % 8 || ldy % 8) return GN_ERR_SHAPE;
-  if (M > (int64_t)65535 * kUM || N > INT32_MAX || K > INT32_MAX) return GN_ERR_SHAPE;
+  if (!nl_shape_ok(M, N, K) || ldx < K || ldy < N || ldx % 8 || ldy % 8) return GN_ERR_SHAPE;
   if (M == 0 || N == 0) return GN_OK;
   if (!x || !Wf || !y || (norm != GN_NORM_NONE && !rstd) || (norm == GN_NORM_LN && (!c || !mean))) return GN_ERR_NULL;
   if (!aligned16(x) || !aligned16(Wf) || !aligned16(y) || (c && !aligned16(c)) || (d && !aligned16(d)))
     return GN_ERR_ALIGN;
-  // pairs of SMs sharing 256 x 512 tiles once there are more than 128 rows and 256 columns;
-  // one SM per 256 x 256 tile (two accumulators) for fewer columns; 128 x 256 for few rows
-  const bool pair = GN_NL_PAIR && M > kUM && N > kBN;
-  const int mh = M > kUM ? GN_NL_MH : 1;
-  const int bm = pair ? 2 * kUM : kUM * mh;
-  CUtensorMap ta, tb;
-  if (!make_map(&ta, x, M, K, ldx, pair ? (uint32_t)kUM : (uint32_t)bm) ||
-      !make_map(&tb, Wf, N, K, K, pair ? 128u : (uint32_t)kBN))
-    return GN_ERR_CUDA;
-  void* kern = pair ? pick_pair(norm, epi) : mh == 2 ? pick<2>(norm, epi) : pick<1>(norm, epi);
-  // the dynamic shared-memory limits are attributes of the kernels on the current device: set
-  // them once per device (0 = not yet, 1 = set, -1 = failed)
-  static std::mutex attr_mu;
-  static signed char attr_state[64];
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GN_ERR_CUDA;
-  {
-    std::lock_guard<std::mutex> lk(attr_mu);
-    if (!attr_state[dev]) attr_state[dev] = set_smem_attr<1>() && set_smem_attr<2>() && set_pair_smem_attr() ? 1 : -1;
-    if (attr_state[dev] < 0) return GN_ERR_CUDA;
-  }
-  NlArgs a{};
-  a.c = c, a.d = d;
-  a.y = static_cast<__nv_bfloat16*>(y);
-  a.mean = mean, a.rstd = rstd;
-  a.M = (int)M, a.N = (int)N, a.K = (int)K;
-  a.ldy = ldy;
-  a.eps = eps;
-  a.err = device_err_word();
-  if (!a.err) return GN_ERR_CUDA;
-  if (pair && norm != GN_NORM_NONE) {  // the pair kernel reads the row statistics: compute them first
-    const unsigned sblocks = (unsigned)((M + 7) / 8);
-    if (norm == GN_NORM_LN)
-      norm_stats_kernel<GN_NORM_LN><<<sblocks, 256, 0, (cudaStream_t)stream>>>(
-          static_cast<const __nv_bfloat16*>(x), ldx, (int)M, (int)K, eps, mean, rstd);
-    else
-      norm_stats_kernel<GN_NORM_RMS><<<sblocks, 256, 0, (cudaStream_t)stream>>>(
-          static_cast<const __nv_bfloat16*>(x), ldx, (int)M, (int)K, eps, mean, rstd);
-    count_launches(1);
-    if (launch_status() != GN_OK) return GN_ERR_CUDA;
-  }
-  const dim3 grid(pair ? (unsigned)(2 * ((N + kPairN - 1) / kPairN)) : (unsigned)((N + kBN - 1) / kBN),
-                  (unsigned)((M + bm - 1) / bm));
-  void* args[] = {&ta, &tb, &a};
-  const int threads = pair ? kPairThreads : mh == 2 ? Tile<2>::Threads : Tile<1>::Threads;
-  const size_t smem = pair ? kPairSmem : mh == 2 ? Tile<2>::Smem : Tile<1>::Smem;
-  if (cudaLaunchKernel(kern, grid, dim3(threads), args, smem, (cudaStream_t)stream) != cudaSuccess)
-    return GN_ERR_CUDA;
-  count_launches(1);
-  return launch_status();
+  return nl_run(x, ldx, Wf, K, c, d, y, nullptr, ldy, nullptr, 0, mean, rstd, M, N, K, eps, norm, epi, OUT_BF16,
+                (cudaStream_t)stream);
+}
+
+extern "C" gn_status gn_linear_act_grad(const void* x, const void* Wf, const float* d, const void* dy, void* dz,
+                                        int64_t M, int64_t N, int64_t K, int64_t ldx, int64_t lddy, int64_t lddz,
+                                        gn_epilogue epi, gn_dtype dt, void* stream) {
+  if (dt != GN_BF16) return dt_ok(dt) ? GN_ERR_UNSUPPORTED : GN_ERR_DTYPE;
+  if (!epi_ok(epi)) return GN_ERR_DTYPE;
+  if (!nl_shape_ok(M, N, K) || ldx < K || lddy < N || lddz < N || ldx % 8 || lddy % 8 || lddz % 8)
+    return GN_ERR_SHAPE;
+  if (M == 0 || N == 0) return GN_OK;
+  if (!x || !Wf || !dy || !dz) return GN_ERR_NULL;
+  if (!aligned16(x) || !aligned16(Wf) || !aligned16(dy) || !aligned16(dz) || (d && !aligned16(d))) return GN_ERR_ALIGN;
+  return nl_run(x, ldx, Wf, K, nullptr, d, dz, nullptr, lddz, dy, lddy, nullptr, nullptr, M, N, K, 0.0f, GN_NORM_NONE,
+                epi, OUT_DGRAD, (cudaStream_t)stream);
+}
+
+extern "C" gn_status gn_linear_acc_f32(const void* A, const void* B, float* C, int64_t M, int64_t N, int64_t K,
+                                       int64_t lda, int64_t ldb, int64_t ldc, gn_dtype dt, void* stream) {
+  if (dt != GN_BF16) return dt_ok(dt) ? GN_ERR_UNSUPPORTED : GN_ERR_DTYPE;
+  if (!nl_shape_ok(M, N, K) || lda < K || ldb < K || ldc < N || lda % 8 || ldb % 8 || ldc % 4) return GN_ERR_SHAPE;
+  if (M == 0 || N == 0) return GN_OK;
+  if (!A || !B || !C) return GN_ERR_NULL;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(C)) return GN_ERR_ALIGN;
+  return nl_run(A, lda, B, ldb, nullptr, nullptr, nullptr, C, ldc, nullptr, 0, nullptr, nullptr, M, N, K, 0.0f,
+                GN_NORM_NONE, GN_EPI_NONE, OUT_ACC32, (cudaStream_t)stream);
 }

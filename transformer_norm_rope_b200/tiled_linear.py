@@ -6,12 +6,16 @@ keeps no intermediate activation: it recomputes each chunk's pre-activation z fr
 forms that chunk's gradients. Memory for the layer's intermediates falls with the chunk count;
 the price is the recomputed forward. The default chunk count is ceil(tokens / hidden).
 
-Where each step runs:
-  * forward and recompute: ``gn_norm_linear_fwd`` with ``GN_NORM_NONE`` (the tcgen05 kernels of
-    this library; the bias and activation in their epilogue);
-  * dz = dy * act'(z): ``gn_act_grad``;
-  * dx = dz W and dW += dz^T x: plain GEMMs, done by cuBLAS (``torch.matmul``, and
-    ``torch.addmm`` with an fp32 output accumulating dW across the chunks); db by a sum.
+Where each step runs (all on this library's kernels):
+  * forward and recompute: ``gn_norm_linear_fwd`` with ``GN_NORM_NONE`` (the tcgen05 kernels; the
+    bias and activation in their epilogue);
+  * dz = dy * act'(z): ``gn_linear_act_grad``, the recompute with the activation gradient applied
+    where the accumulators are read back (z never reaches memory);
+  * dx = dz W: ``gn_norm_linear_fwd`` on dz with W^T (``gn_transpose``, once per backward) as the
+    weight operand;
+  * dW += dz^T x: ``gn_linear_acc_f32`` on the transposed chunk operands (the tokens, over which
+    the product contracts, made contiguous by ``gn_transpose``), accumulating in fp32 in place;
+  * db += sum dz: ``gn_colsum_bf16`` (fixed order).
 This module only orchestrates chunks (host logic); every elementwise and fused step is a kernel
 of the library.
 """
@@ -67,15 +71,16 @@ def backward(x, Wf, d, dy, act: str = "silu", chunks: Optional[int] = None) -> T
     dx = torch.empty_like(x)
     dW = torch.zeros((N, K), dtype=torch.float32, device=x.device)
     db = torch.zeros(N, dtype=torch.float32, device=x.device)
+    Wt = gn.transpose(Wf)  # [K, N]: the weight operand of dx = dz W
+    ws = torch.empty(max(gn.gn_colsum_bf16_workspace(N), 16), dtype=torch.uint8, device=x.device)
     for r0, r1 in _bounds(M, chunks):
         xc = x[r0:r1]
-        z = gn.norm_linear_fwd(xc, Wf, None, d, norm="none", epilogue="none", save_stats=False)[0]
-        dz = gn.act_grad(z, dy[r0:r1].contiguous(), epilogue=act, out=z)  # z is not needed after this
-        torch.matmul(dz, Wf, out=dx[r0:r1])
-        # bf16 operands, fp32 accumulator updated in place (beta = 1): no bf16 rounding of the
-        # per-chunk partial and no extra pass over a converted copy
-        torch.addmm(dW, dz.t(), xc, out_dtype=torch.float32, out=dW)
-        db += dz.sum(0, dtype=torch.float32)
+        dz = gn.linear_act_grad(xc, Wf, d, dy[r0:r1], epilogue=act)
+        gn.norm_linear_fwd(dz, Wt, None, None, norm="none", epilogue="none", save_stats=False, out=dx[r0:r1])
+        # dW += dz^T x contracts over the chunk's tokens: both operands with the tokens contiguous
+        # (zero-padded to a multiple of 8 tokens)
+        gn.linear_acc_f32(gn.transpose(dz), gn.transpose(xc), dW)
+        gn.colsum_bf16(dz, db, accumulate=True, ws=ws)
     return dx, dW, db
 
 
