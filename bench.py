@@ -325,7 +325,7 @@ def ncu_traffic(kernel, z):
         t = json.load(open(p))
         from transformer_norm_rope_b200 import _build
 
-        if t.get("sources_sha") != _build.sources_digest():
+        if t.get("sources_sha") != _build.sources_digest(step_only=True):
             return None
         e = t["kernels"][kernel]
         return e["dram_bytes_per_launch"] * (algorithmic_bytes(z)[kernel] / e["algorithmic_bytes"])

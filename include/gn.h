@@ -260,21 +260,28 @@ gn_status gn_linear_act_grad(const void* x, const void* Wf, const float* d, cons
                              int64_t M, int64_t N, int64_t K, int64_t ldx, int64_t lddy, int64_t lddz,
                              gn_epilogue epi, gn_dtype dt, void* stream);
 
-/* C [M, N] += A [M, K] B [N, K]^T with C fp32 (updated in place: a weight gradient summed over
- * chunks), A and B bf16 with the contraction index K contiguous (row strides lda, ldb, multiples
- * of 8; K a multiple of 8), on the tensor-core kernels. ldc a multiple of 4; A, B, C 16-byte
- * aligned. Errors as gn_linear_act_grad. */
-gn_status gn_linear_acc_f32(const void* A, const void* B, float* C, int64_t M, int64_t N, int64_t K,
-                            int64_t lda, int64_t ldb, int64_t ldc, gn_dtype dt, void* stream);
+/* Operand layouts of the plain products below. GN_K_MAJOR: A as [M, K], B as [N, K], the
+ * contraction index contiguous (row strides lda >= K, ldb >= K; K a multiple of 8). GN_MN_MAJOR:
+ * the operand stored transposed, A as [K, M], B as [K, N] (row strides lda >= M, ldb >= N; K
+ * free). The weight gradient dW = dz^T x contracts over the tokens, the rows of dz [tokens, N]
+ * and x [tokens, K]: both operands are MN-major there; dx = dz W reads W [N, K] as an MN-major
+ * B. Row strides are multiples of 8 elements in either layout. */
+typedef enum { GN_K_MAJOR = 0, GN_MN_MAJOR = 1 } gn_layout;
 
-/* dst [cols, rows] = src [rows, cols]^T (bf16; cols and both row strides multiples of 8; both
- * pointers 16-byte aligned). A row count that is not a multiple of 8 is padded: each output row
- * is written up to the next multiple of 8 columns, with zeros past the input rows (ld_dst must
- * cover them). The weight gradient contracts over the tokens, so its operands are transposed to
- * put the tokens contiguous.
- * Errors: GN_ERR_SHAPE, GN_ERR_NULL, GN_ERR_ALIGN, GN_ERR_UNSUPPORTED (fp32), GN_ERR_CUDA. */
-gn_status gn_transpose(const void* src, void* dst, int64_t rows, int64_t cols, int64_t ld_src,
-                       int64_t ld_dst, gn_dtype dt, void* stream);
+/* y [M, N] = A B^T (+ d) in bf16 (fp32 accumulation on the tensor-core kernels; d [N] fp32, may
+ * be NULL = 0). ldy >= N, a multiple of 8; A, B, y, d 16-byte aligned.
+ * Errors: GN_ERR_SHAPE (sizes, strides, layout values), GN_ERR_NULL, GN_ERR_ALIGN,
+ * GN_ERR_UNSUPPORTED (fp32), GN_ERR_CUDA. M == 0 or N == 0: nothing is launched. */
+gn_status gn_linear_bf16(const void* A, const void* B, const float* d, void* y, int64_t M, int64_t N,
+                         int64_t K, int64_t lda, int64_t ldb, int64_t ldy, gn_layout a_layout,
+                         gn_layout b_layout, gn_dtype dt, void* stream);
+
+/* C [M, N] += A B^T with C fp32, updated in place (a weight gradient summed over token chunks:
+ * no partial is rounded), A and B bf16 in the given layouts, on the tensor-core kernels. ldc >=
+ * N, a multiple of 4; A, B, C 16-byte aligned. Errors as gn_linear_bf16. */
+gn_status gn_linear_acc_f32(const void* A, const void* B, float* C, int64_t M, int64_t N, int64_t K,
+                            int64_t lda, int64_t ldb, int64_t ldc, gn_layout a_layout,
+                            gn_layout b_layout, gn_dtype dt, void* stream);
 
 /* Column sums of a bf16 matrix src [rows, cols] (row stride ld; cols and ld even; src 4-byte
  * aligned) into fp32 out [cols]: out = sum (accumulate == 0) or out += sum (accumulate != 0), in
@@ -315,7 +322,8 @@ gn_status gn_selftest_wait_timeout(uint32_t limit_us, void* stream);
  * "ctas_per_sm", "vpt", "unit_bytes", "group_rows", "fwd_warps" (warps per CTA of the
  * one-warp-per-row norm forward, at most 16), "fwd_path" (norm forward of long rows: 1 = the
  * CTA-per-row pipeline, 2 = one warp per row with two-pass LayerNorm statistics, 3 = one warp per
- * row with one shifted pass; by default RMSNorm takes the first and LayerNorm the third); value 0 restores the default. Returns
+ * row with one shifted pass; by default RMSNorm takes the first and LayerNorm the third);
+ * value 0 restores the default. Returns
  * GN_ERR_SHAPE for an unknown key or a value out of range. Not thread-safe with concurrent
  * launches. */
 gn_status gn_tune(const char* key, int value);

@@ -133,15 +133,19 @@ def test_linear_helpers(stub):
 
 def test_tiled_linear_autograd_plumbing(stub, monkeypatch):
     # with the kernels stubbed, the values are meaningless; the test checks that the autograd
-    # form saves what it needs and returns one gradient per input, of the input's dtype and shape
+    # form saves what it needs, returns one gradient per input, of the input's dtype and shape,
+    # and runs every step of every chunk on the library's entry points
     from transformer_norm_rope_b200 import tiled_linear as tl
 
-    def addmm_f32(c, a, b, out_dtype, out):  # the fp32-output addmm exists for CUDA only
-        assert out_dtype == f32 and out is c and c.dtype == f32
-        return out.add_(a.float() @ b.float())
+    class _Sync:  # stands in for a CUDA stream and a CUDA event (no GPU here)
+        def wait_event(self, e):
+            pass
 
-    monkeypatch.setattr(torch, "addmm", addmm_f32)
+        def record(self, s=None):
+            pass
 
+    monkeypatch.setattr(tl, "_stream_pair", lambda device: (_Sync(), _Sync()))
+    monkeypatch.setattr(tl, "_event", _Sync)
     M, N, K = 24, 16, 32
     x = z(M, K).requires_grad_()
     W = z(N, K).requires_grad_()
@@ -154,4 +158,7 @@ def test_tiled_linear_autograd_plumbing(stub, monkeypatch):
     x2 = z(M, K).requires_grad_()
     tl.TiledLinearFunction.apply(x2, W, None, "gelu_tanh", None).backward(z(M, N))
     assert x2.grad.shape == x2.shape
-    assert stub.count("gn_norm_linear_fwd") == 2 * 3 + 2 * 1  # forward + recompute, per chunk
+    chunks = 3 + 1  # 3 chunks, then ceil(24 / 32) = 1
+    assert stub.count("gn_norm_linear_fwd") == 3 + 1  # the forward: chunked on request, else one launch
+    for step in ("gn_linear_act_grad", "gn_linear_bf16", "gn_linear_acc_f32", "gn_colsum_bf16"):
+        assert stub.count(step) == chunks, step  # the backward, per chunk

@@ -86,16 +86,12 @@ def test_act_grad_matches_oracle_derivative(gpu):
 
 
 @pytest.mark.parametrize("rows,cols", [(300, 264), (64, 5120), (1000, 72), (8, 8)])
-def test_transpose_and_column_sums(gpu, rows, cols):
-    """The backward's memory-bound steps: the transpose is exact (bit for bit, zero-padded up to
-    a multiple of 8 rows) and the column sums match the fp64 sums of the same bf16 values."""
+def test_column_sums(gpu, rows, cols):
+    """The backward's memory-bound step: the column sums match the fp64 sums of the same bf16
+    values, and repeat bit for bit (fixed order)."""
     g = np.random.default_rng(rows)
     a = wl.bf16_bits(g.standard_normal((rows, cols)).astype(np.float32))
     t = to_dev(a)
-    tt = gpu.transpose(t)
-    r8 = (rows + 7) // 8 * 8
-    assert tuple(tt.shape) == (cols, r8)
-    assert torch.equal(tt[:, :rows], t.t()) and bool((tt[:, rows:] == 0).all())
     out = torch.full((cols,), 1.5, dtype=torch.float32, device="cuda")
     gpu.colsum_bf16(t, out, accumulate=True)
     ref = wl.bf16_to_f32(a).astype(np.float64).sum(0) + 1.5
@@ -105,18 +101,60 @@ def test_transpose_and_column_sums(gpu, rows, cols):
     assert torch.equal(a2, b2)  # fixed order
 
 
-@pytest.mark.parametrize("M,N,K", [(300, 264, 1024), (5120, 512, 1000), (100, 600, 200)])
-def test_fp32_accumulating_product(gpu, M, N, K):
-    """C += A B^T on the tensor cores with an fp32 accumulator updated in place, against the fp64
-    product of the same bf16 operands (K padded with zeros to a multiple of 8 by the transpose
-    path where the caller needs it; here K is a multiple of 8)."""
-    g = np.random.default_rng(M + N + K)
+# shapes: a single-CTA tile with few rows (M <= 128), two-accumulator tiles (N <= 256), pair
+# tiles (M > 128 and N > 256) with M, N, K not multiples of the tiles (N a multiple of 8: the
+# output rows stay 16-byte aligned); a stored row is a multiple of 8 elements (K for a K-major
+# operand, M or N for an MN-major one), so K is ragged only where both operands are MN-major
+PRODUCT_SHAPES = [(100, 600, 200), (104, 600, 200), (300, 264, 1000), (296, 264, 1000), (5120, 512, 1000),
+                  (1000, 776, 328), (136, 1032, 1001)]
+LAYOUTS = [(False, False), (True, False), (False, True), (True, True)]
+
+
+def _skip_unaligned(M, N, K, a_mn, b_mn):
+    """Stored rows must be whole 16-byte vectors: K for a K-major operand, M / N for MN-major."""
+    if (K % 8 and not (a_mn and b_mn)) or (a_mn and M % 8) or (b_mn and N % 8):
+        pytest.skip("a stored row that is not a multiple of 8 elements")
+
+
+def _product_operands(M, N, K, a_mn, b_mn, seed):
+    """Logical A [M, K], B [N, K] (bf16 bits) and their stored forms in the requested layouts."""
+    g = np.random.default_rng(seed)
     A = wl.bf16_bits(g.standard_normal((M, K)).astype(np.float32))
     B = wl.bf16_bits(g.standard_normal((N, K)).astype(np.float32))
-    C0 = g.standard_normal((M, N)).astype(np.float32)
+    As = np.ascontiguousarray(A.T) if a_mn else A
+    Bs = np.ascontiguousarray(B.T) if b_mn else B
+    return A, B, to_dev(As), to_dev(Bs)
+
+
+@pytest.mark.parametrize("M,N,K", PRODUCT_SHAPES)
+@pytest.mark.parametrize("a_mn,b_mn", LAYOUTS)
+def test_fp32_accumulating_product(gpu, M, N, K, a_mn, b_mn):
+    """C += A B^T on the tensor cores with an fp32 accumulator updated in place, every operand
+    layout, against the oracle's fp64 linear layer (no norm, no activation) of the same bf16
+    operands plus the starting C."""
+    _skip_unaligned(M, N, K, a_mn, b_mn)
+    A, B, As, Bs = _product_operands(M, N, K, a_mn, b_mn, seed=M + N + K)
+    C0 = np.random.default_rng(K).standard_normal((M, N)).astype(np.float32)
     C = to_dev(C0)
-    gpu.linear_acc_f32(to_dev(A), to_dev(B), C)
+    gpu.linear_acc_f32(As, Bs, C, a_mn=a_mn, b_mn=b_mn)
     torch.cuda.synchronize()
-    ref = C0.astype(np.float64) + wl.bf16_to_f32(A).astype(np.float64) @ wl.bf16_to_f32(B).astype(np.float64).T
-    assert_close(to_np(C), ref, (1e-5, 1e-4 * math.sqrt(K)), "C += A B^T")
+    prod, _, _ = oracle.norm_linear(A, None, None, B, None, 0.0, "none")
+    ref = C0.astype(np.float64) + prod
+    assert_close(to_np(C), ref, (1e-5, 1e-4 * math.sqrt(K)), f"C += A B^T (a_mn={a_mn}, b_mn={b_mn})")
+    assert gpu.device_error(clear=True) == 0
+
+
+@pytest.mark.parametrize("M,N,K", PRODUCT_SHAPES)
+@pytest.mark.parametrize("a_mn,b_mn", LAYOUTS)
+def test_bf16_product(gpu, M, N, K, a_mn, b_mn):
+    """y = A B^T + d in bf16, every operand layout, against the oracle's fp64 linear layer of the
+    same operands (tolerance: the bf16 rounding of y)."""
+    _skip_unaligned(M, N, K, a_mn, b_mn)
+    A, B, As, Bs = _product_operands(M, N, K, a_mn, b_mn, seed=3 * M + N + K)
+    bias = wl.bf16_bits((0.1 * np.random.default_rng(N).standard_normal(N)).astype(np.float32))
+    d = torch.from_numpy(wl.bf16_to_f32(bias)).cuda()
+    y = gpu.linear_bf16(As, Bs, d, a_mn=a_mn, b_mn=b_mn)
+    torch.cuda.synchronize()
+    ref, _, _ = oracle.norm_linear(A, None, None, B, bias, 0.0, "none")
+    assert_close(to_np(y), ref, "bf16", f"y = A B^T + d (a_mn={a_mn}, b_mn={b_mn})")
     assert gpu.device_error(clear=True) == 0

@@ -55,8 +55,8 @@ SIGNATURES = {
     "gn_norm_linear_fwd": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _f32, _int,
                                  _int, _int, _vp]),
     "gn_linear_act_grad": (_st, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _int, _int, _vp]),
-    "gn_linear_acc_f32": (_st, [_vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _int, _vp]),
-    "gn_transpose": (_st, [_vp, _vp, _i64, _i64, _i64, _i64, _int, _vp]),
+    "gn_linear_bf16": (_st, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _int, _int, _int, _vp]),
+    "gn_linear_acc_f32": (_st, [_vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _int, _int, _int, _vp]),
     "gn_colsum_bf16_workspace": (_sz, [_i64]),
     "gn_colsum_bf16": (_st, [_vp, _vp, _vp, _sz, _i64, _i64, _i64, _int, _int, _vp]),
     "gn_act_grad": (_st, [_vp, _vp, _vp, _i64, _int, _int, _vp]),
@@ -427,34 +427,49 @@ def linear_act_grad(x, Wf, d, dy, epilogue="silu", out=None, stream=None):
     return dz
 
 
-def linear_acc_f32(A, B, C, stream=None):
-    """C [M, N] (fp32, in place) += A [M, K] B [N, K]^T (bf16, K contiguous)."""
-    torch = _torch()
+GN_K_MAJOR, GN_MN_MAJOR = 0, 1
+
+
+def _operands(A, B, a_mn, b_mn):
+    """(M, N, K) of the product A B^T from the stored operands: A is [M, K], or [K, M] when a_mn
+    (MN-major); B is [N, K], or [K, N] when b_mn."""
     _rows(A, "A")
     _rows(B, "B", like=A, dtype=A.dtype)
-    M, K = A.shape
-    if B.dim() != 2 or B.shape[1] != K:
-        raise ValueError(f"B has shape {tuple(B.shape)}, expected [N, {K}]")
-    N = B.shape[0]
+    if A.dim() != 2 or B.dim() != 2:
+        raise ValueError("A and B must be 2-D")
+    M, K = (A.shape[1], A.shape[0]) if a_mn else A.shape
+    N, KB = (B.shape[1], B.shape[0]) if b_mn else B.shape
+    if KB != K:
+        raise ValueError(f"contraction sizes differ: A gives {K}, B gives {KB}")
+    return M, N, K
+
+
+def linear_bf16(A, B, d=None, out=None, a_mn=False, b_mn=False, stream=None):
+    """y [M, N] = A B^T (+ d) in bf16 on the tensor-core kernels; a_mn / b_mn: the operand is
+    stored transposed ([K, M] / [K, N])."""
+    torch = _torch()
+    M, N, K = _operands(A, B, a_mn, b_mn)
+    _need(d, "d", like=A, shape=(N,), dtype=torch.float32, optional=True)
+    y = torch.empty((M, N), dtype=A.dtype, device=A.device) if out is None else out
+    _need(y, "out", like=A, shape=(M, N), dtype=A.dtype, contiguous=False)
+    _rows(y, "out", like=A, dtype=A.dtype)
+    check(gn_linear_bf16(_ptr(A), _ptr(B), _ptr(d), _ptr(y), M, N, K, A.stride(0), B.stride(0), y.stride(0),
+                         GN_MN_MAJOR if a_mn else GN_K_MAJOR, GN_MN_MAJOR if b_mn else GN_K_MAJOR, _dt(A),
+                         _stream(stream)), "gn_linear_bf16")
+    return y
+
+
+def linear_acc_f32(A, B, C, a_mn=False, b_mn=False, stream=None):
+    """C [M, N] (fp32, in place) += A B^T (bf16) on the tensor-core kernels; a_mn / b_mn: the
+    operand is stored transposed ([K, M] / [K, N])."""
+    torch = _torch()
+    M, N, K = _operands(A, B, a_mn, b_mn)
     _need(C, "C", like=A, shape=(M, N), dtype=torch.float32, contiguous=False)
     _rows(C, "C", like=A, dtype=torch.float32)
-    check(gn_linear_acc_f32(_ptr(A), _ptr(B), _ptr(C), M, N, K, A.stride(0), B.stride(0), C.stride(0), _dt(A),
+    check(gn_linear_acc_f32(_ptr(A), _ptr(B), _ptr(C), M, N, K, A.stride(0), B.stride(0), C.stride(0),
+                            GN_MN_MAJOR if a_mn else GN_K_MAJOR, GN_MN_MAJOR if b_mn else GN_K_MAJOR, _dt(A),
                             _stream(stream)), "gn_linear_acc_f32")
     return C
-
-
-def transpose(src, out=None, stream=None):
-    """src [rows, cols] -> [cols, rows8] (bf16), rows8 = rows rounded up to 8: the columns past
-    rows are zero."""
-    rows, cols, ld = _rows(src, "src")
-    if src.dim() != 2:
-        raise ValueError("transpose takes a matrix")
-    rows8 = (rows + 7) // 8 * 8
-    dst = _torch().empty((cols, rows8), dtype=src.dtype, device=src.device) if out is None else out
-    _need(dst, "out", like=src, shape=(cols, rows8), dtype=src.dtype, contiguous=False)
-    _, _, ldd = _rows(dst, "out", like=src, dtype=src.dtype)
-    check(gn_transpose(_ptr(src), _ptr(dst), rows, cols, ld, ldd, _dt(src), _stream(stream)), "gn_transpose")
-    return dst
 
 
 def colsum_bf16(src, out, accumulate=False, ws=None, stream=None):

@@ -41,12 +41,19 @@ def _deps():
         glob.glob(os.path.join(INCLUDE, "*.h")) + [__file__]
 
 
-def sources_digest() -> str:
-    """sha256 over the kernel sources and headers (identifies the code a profile was taken of)."""
+# the files the row-normalization and RoPE kernels (and their column reduction) are built from;
+# the tensor-core products live in other files
+STEP_SOURCES = ("api.cu", "rmsnorm.cu", "layernorm.cu", "norm_fwd_warp.cu", "rope.cu")
+
+
+def sources_digest(step_only: bool = False) -> str:
+    """sha256 over the kernel sources and headers (identifies the code a profile was taken of);
+    step_only: over the row-normalization and RoPE sources and the headers only."""
     import hashlib
 
+    srcs = [p for p in sources() if not step_only or os.path.basename(p) in STEP_SOURCES]
     h = hashlib.sha256()
-    for p in sorted(sources() + glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh"))):
+    for p in sorted(srcs + glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh"))):
         h.update(os.path.basename(p).encode())
         h.update(open(p, "rb").read())
     return h.hexdigest()[:16]

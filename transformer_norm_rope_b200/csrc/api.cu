@@ -119,28 +119,31 @@ int persistent_grid(const void* kernel, int threads, size_t smem, int cap) {
 }
 
 // ---------------------------------------------------------------- column reduction
-// Block = 32 columns x 8 slices of the partial rows. Slice k sums rows g = k, k+8, ... in
-// order, then slice 0 adds the 8 slice sums in order: a fixed order for a given G, so the
-// result is the same on every run.
-__global__ void __launch_bounds__(256) colsum_kernel(const float* __restrict__ ws, int64_t G,
-                                                     int64_t ncols, int64_t split,
-                                                     float* __restrict__ out0,
-                                                     float* __restrict__ out1) {
-  __shared__ float part[8][33];
+// Block = 32 columns x 32 slices of the partial rows (1024 threads: a whole SM's worth of loads in
+// flight, the partial rows being L2-resident right after the backward wrote them). Slice k sums
+// rows g = k, k+32, ... in order, then the first warp adds the 32 slice sums in order: a fixed
+// order for a given G, so the result is the same on every run.
+constexpr int kColsumSlices = 32;
+
+__global__ void __launch_bounds__(32 * kColsumSlices) colsum_kernel(const float* __restrict__ ws, int64_t G,
+                                                                    int64_t ncols, int64_t split,
+                                                                    float* __restrict__ out0,
+                                                                    float* __restrict__ out1) {
+  __shared__ float part[kColsumSlices][33];
   pdl_wait();  // the partial rows are complete: the backward grid before this one has finished
   const int cl = threadIdx.x & 31, sl = threadIdx.x >> 5;
   const int64_t c = (int64_t)blockIdx.x * 32 + cl;
   float acc = 0.f;
   if (c < ncols) {
 #pragma unroll 4
-    for (int64_t g = sl; g < G; g += 8) acc += ws[g * ncols + c];
+    for (int64_t g = sl; g < G; g += kColsumSlices) acc += ws[g * ncols + c];
   }
   part[sl][cl] = acc;
   __syncthreads();
   if (sl == 0 && c < ncols) {
     float t = 0.f;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) t += part[k][cl];
+    for (int k = 0; k < kColsumSlices; ++k) t += part[k][cl];
     if (c < split) {
       if (out0) out0[c] = t;
     } else if (out1) {
@@ -167,7 +170,7 @@ gn_status launch_colsum(const float* ws, int64_t G, int64_t ncols, int64_t split
   // backward grid before it, which it waits for on the device (pdl_wait)
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)blocks);
-  cfg.blockDim = dim3(256);
+  cfg.blockDim = dim3(32 * kColsumSlices);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];

@@ -73,10 +73,19 @@ struct Tile {
   static constexpr size_t Smem = 1024 /* alignment slack */ + (size_t)Stages * StageBytes + 256 + 2 * kBN * 4;
 };
 
+// Operand layouts in global (and shared) memory, bit 0 for A (x), bit 1 for B (Wf):
+//   K-major  : A [M, K] / B [N, K] with K contiguous (the layer's natural layout);
+//   MN-major : the operand stored transposed, A as [K, M] / B as [K, N] with M / N contiguous (a
+//              product that contracts over the tokens, dW = dz^T x, reads both operands so,
+//              and dx = dz W reads the weight so).
+enum NlMajor { MAJ_A_MN = 1, MAJ_B_MN = 2 };
+
 // instruction descriptor of tcgen05.mma kind::f16: D fp32 (bits 4-5 = 1), A and B bf16 (bits 7-9,
-// 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 at bit 17, M >> 4 at bit 24
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) |
-                            ((uint32_t)(kUM >> 4) << 24);
+// 10-12 = 1), A / B MN-major (bits 15 / 16), N >> 3 at bit 17, M >> 4 at bit 24
+constexpr uint32_t idesc_f16(int m, int n, int maj) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((maj & MAJ_A_MN) ? 1u << 15 : 0u) | ((maj & MAJ_B_MN) ? 1u << 16 : 0u) |
+         ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
 
 struct NlArgs {
   const float* c;  // [N] (LayerNorm)
@@ -187,12 +196,13 @@ __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence:
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
 // D[tmem] (+)= A[smem] * B[smem]^T for one M=128, N=256, K=16 step
+template <int MAJ>
 __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
+      "l"(adesc), "l"(bdesc), "r"(idesc_f16(kUM, kBN, MAJ)), "r"(accumulate)
       : "memory");
 }
 
@@ -211,6 +221,42 @@ __device__ __forceinline__ uint64_t tile_desc(const void* tile) {
   constexpr uint64_t layout = kLine == 128 ? 2 : 4;
   return (uint64_t)((smem_addr(tile) & 0x3FFFFu) >> 4) | (1ull << 16) | ((uint64_t)(8 * kLine / 16) << 32) |
          (1ull << 46) | (layout << 61);
+}
+
+// MN-major tiles (kBK = 64 only): the tile is a row of TMA boxes, each 64 M/N elements (128 bytes,
+// the swizzle span) wide and kBK k-rows deep, 128-byte swizzled. Descriptor: the next 64 M/N
+// elements one box further (leading-dimension offset = box bytes), the next 8 k-rows one 1024-byte
+// swizzle atom further (stride offset), SWIZZLE_128B. One K=16 instruction step is 16 k-rows =
+// 2048 bytes down the tile.
+constexpr uint32_t kMnBox = 64 * kLine;  // bytes of one 64 x kBK box
+__device__ __forceinline__ uint64_t tile_desc_mn(const void* tile) {
+  return (uint64_t)((smem_addr(tile) & 0x3FFFFu) >> 4) | ((uint64_t)(kMnBox >> 4) << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         (1ull << 46) | (2ull << 61);
+}
+// descriptor units (16 bytes) between consecutive K=16 steps of a K-major / MN-major tile
+template <bool MN>
+constexpr uint64_t ksub_step() {
+  return MN ? 2048 / 16 : 32 / 16;
+}
+
+// one stage's tile of an operand: a K-major tile is one box of `rows` x kBK; an MN-major tile is
+// rows / 64 boxes of 64 x kBK at consecutive kMnBox offsets (coordinates: M/N first, then K)
+template <bool MN>
+__device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map, int k0, int r0, int rows, uint64_t* bar) {
+  if constexpr (MN) {
+    for (int i = 0; i < rows / 64; ++i) tma_load_2d(dst + i * kMnBox, map, r0 + 64 * i, k0, bar);
+  } else {
+    tma_load_2d(dst, map, k0, r0, bar);
+  }
+}
+
+template <bool MN>
+__device__ __forceinline__ void prefetch_tile(const CUtensorMap* map, int k0, int r0, int rows) {
+  if constexpr (MN) {
+    for (int i = 0; i < rows / 64; ++i) tma_prefetch_2d(map, r0 + 64 * i, k0);
+  } else {
+    tma_prefetch_2d(map, k0, r0);
+  }
 }
 
 // 16-byte chunk c of row r sits at chunk position c ^ swz(r) of the row: the swizzle XORs
@@ -251,11 +297,13 @@ __device__ __forceinline__ float nl_act(float z) {
 
 // ---------------------------------------------------------------- forward kernel
 
-template <int MH, int NORM, int EPI, int OUT = OUT_BF16>
+template <int MH, int NORM, int EPI, int OUT = OUT_BF16, int MAJ = 0>
 __global__ void __launch_bounds__(Tile<MH>::Threads, 1)
     norm_linear_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const NlArgs a) {
   using TL = Tile<MH>;
+  constexpr bool AMN = (MAJ & MAJ_A_MN) != 0, BMN = (MAJ & MAJ_B_MN) != 0;
+  static_assert(MAJ == 0 || (NORM == GN_NORM_NONE && kLine == 128), "MN-major operands: no norm, 64-wide k tiles");
   constexpr int kStages = TL::Stages;
   constexpr int kPrefetch = 2 * kStages;
   constexpr uint32_t kABytes = TL::ABytes, kStageBytes = TL::StageBytes;
@@ -304,9 +352,9 @@ __global__ void __launch_bounds__(Tile<MH>::Threads, 1)
         mbar_expect_tx(&full[s], kStageBytes);
         // x is read from DRAM once per row block (the other column tiles hit in L2, W stays in
         // L2): fetch it into L2 a ring of stages ahead so the loads wait for L2, not DRAM
-        if (kb + kPrefetch < nk) tma_prefetch_2d(&tmA, (kb + kPrefetch) * kBK, m0);
-        tma_load_2d(A(s), &tmA, kb * kBK, m0, &full[s]);
-        tma_load_2d(B(s), &tmB, kb * kBK, n0, &full[s]);
+        if (kb + kPrefetch < nk) prefetch_tile<AMN>(&tmA, (kb + kPrefetch) * kBK, m0, TL::BM);
+        load_tile<AMN>(A(s), &tmA, kb * kBK, m0, TL::BM, &full[s]);
+        load_tile<BMN>(B(s), &tmB, kb * kBK, n0, kBN, &full[s]);
         used |= 1u << s;
         lastph = (lastph & ~(1u << s)) | (ph << s);
       }
@@ -325,13 +373,14 @@ __global__ void __launch_bounds__(Tile<MH>::Threads, 1)
           break;
         }
         tc_fence_after();
-        const uint64_t ad = tile_desc(A(s)), bd = tile_desc(B(s));
+        const uint64_t ad = AMN ? tile_desc_mn(A(s)) : tile_desc(A(s));
+        const uint64_t bd = BMN ? tile_desc_mn(B(s)) : tile_desc(B(s));
 #pragma unroll
-        for (int k = 0; k < kBK / kUK; ++k)  // +32 bytes along K inside the swizzled rows
+        for (int k = 0; k < kBK / kUK; ++k)  // K-major: +32 bytes inside the swizzled rows
 #pragma unroll
           for (int h = 0; h < MH; ++h)  // rows 128h.. of the A tile start 128 * kLine bytes further
-            umma_bf16(tmem + (uint32_t)(kAccCols * h), ad + (uint64_t)(2 * k + 8 * kLine * h), bd + (uint64_t)(2 * k),
-                      (kb | k) != 0);
+            umma_bf16<MAJ>(tmem + (uint32_t)(kAccCols * h), ad + ksub_step<AMN>() * k + (uint64_t)(8 * kLine * h),
+                           bd + ksub_step<BMN>() * k, (kb | k) != 0);
         umma_commit(&empty[s]);
       }
       umma_commit(accf);  // also after an abort: the epilogue waits for the work in flight
@@ -492,9 +541,6 @@ constexpr uint32_t kPairBBytes = 2 * 128 * kLine;       // 32 KiB: this CTA's 2 
 constexpr uint32_t kPairStageBytes = kPairABytes + kPairBBytes;
 constexpr int kPairThreads = 320;      // producer, MMA, 8 statistics/epilogue warps
 constexpr size_t kPairSmem = 1024 + (size_t)kPairStages * kPairStageBytes + 256 + 2 * kPairN * 4;
-// instruction descriptor: as kIdesc with M = 256 (the pair)
-constexpr uint32_t kIdescPair = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) |
-                                ((uint32_t)(256 >> 4) << 24);
 
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -523,6 +569,16 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
       : "memory");
 }
 
+template <bool MN>
+__device__ __forceinline__ void load_tile_pair(uint8_t* dst, const CUtensorMap* map, int k0, int r0, int rows,
+                                               uint32_t bar_cluster) {
+  if constexpr (MN) {
+    for (int i = 0; i < rows / 64; ++i) tma_load_2d_pair(dst + i * kMnBox, map, r0 + 64 * i, k0, bar_cluster);
+  } else {
+    tma_load_2d_pair(dst, map, k0, r0, bar_cluster);
+  }
+}
+
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* slot, uint32_t ncols) {  // whole warp, both CTAs
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(slot)), "r"(ncols)
                : "memory");
@@ -533,12 +589,14 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
   asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
 
+// instruction shape of the pair: M = 256 (128 rows from each CTA), N = 256
+template <int MAJ>
 __device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(kIdescPair), "r"(accumulate)
+      "l"(adesc), "l"(bdesc), "r"(idesc_f16(256, 256, MAJ)), "r"(accumulate)
       : "memory");
 }
 
@@ -552,10 +610,12 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
       : "memory");
 }
 
-template <int NORM, int EPI, int OUT = OUT_BF16>
+template <int NORM, int EPI, int OUT = OUT_BF16, int MAJ = 0>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     norm_linear_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const NlArgs a) {
+  constexpr bool AMN = (MAJ & MAJ_A_MN) != 0, BMN = (MAJ & MAJ_B_MN) != 0;
+  static_assert(MAJ == 0 || (NORM == GN_NORM_NONE && kLine == 128), "MN-major operands: no norm, 64-wide k tiles");
   constexpr int kPrefetch = 2 * kPairStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -605,10 +665,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         if (*abort_flag) break;
         const uint32_t bar = cluster_addr(&full[s], 0);
         if (leader) mbar_expect_tx(&full[s], 2 * kPairStageBytes);  // both CTAs' bytes
-        if (kb + kPrefetch < nk) tma_prefetch_2d(&tmA, (kb + kPrefetch) * kBK, m0);
-        tma_load_2d_pair(A(s), &tmA, kb * kBK, m0, bar);
-        tma_load_2d_pair(B(s), &tmB, kb * kBK, n0 + 128 * (int)rank, bar);
-        tma_load_2d_pair(B(s) + 128 * kLine, &tmB, kb * kBK, n0 + 256 + 128 * (int)rank, bar);
+        if (kb + kPrefetch < nk) prefetch_tile<AMN>(&tmA, (kb + kPrefetch) * kBK, m0, kUM);
+        load_tile_pair<AMN>(A(s), &tmA, kb * kBK, m0, kUM, bar);
+        load_tile_pair<BMN>(B(s), &tmB, kb * kBK, n0 + 128 * (int)rank, 128, bar);
+        load_tile_pair<BMN>(B(s) + 128 * kLine, &tmB, kb * kBK, n0 + 256 + 128 * (int)rank, 128, bar);
         used |= 1u << s;
         lastph = (lastph & ~(1u << s)) | (ph << s);
       }
@@ -629,13 +689,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint64_t ad = tile_desc(A(s)), bd = tile_desc(B(s));
+        const uint64_t ad = AMN ? tile_desc_mn(A(s)) : tile_desc(A(s));
+        const uint64_t bd = BMN ? tile_desc_mn(B(s)) : tile_desc(B(s));
 #pragma unroll
         for (int k = 0; k < kBK / kUK; ++k)
 #pragma unroll
           for (int j = 0; j < 2; ++j)  // B rows 128j.. of each CTA's tile: columns 256j.. of the pair
-            umma_bf16_pair(tmem + (uint32_t)(kAccCols * j), ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k + 8 * kLine * j),
-                           (kb | k) != 0);
+            umma_bf16_pair<MAJ>(tmem + (uint32_t)(kAccCols * j), ad + ksub_step<AMN>() * k,
+                                bd + ksub_step<BMN>() * k + (uint64_t)(8 * kLine * j), (kb | k) != 0);
         umma_commit_pair(&empty[s]);
       }
       umma_commit_pair(accf);  // also after an abort: both epilogues wait for the work in flight
@@ -829,74 +890,70 @@ bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, in
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int MH, int NORM>
-void* pick_epi(int epi, int out) {
-  if constexpr (NORM == GN_NORM_NONE) {  // the gradient modes exist without a norm only
-    if (out == OUT_DGRAD) {
-      if (epi == GN_EPI_GELU_TANH) return (void*)norm_linear_kernel<MH, NORM, EPI_GELU_TANH, OUT_DGRAD>;
-      if (epi == GN_EPI_SILU) return (void*)norm_linear_kernel<MH, NORM, EPI_SILU, OUT_DGRAD>;
-      return (void*)norm_linear_kernel<MH, NORM, EPI_NONE, OUT_DGRAD>;
+// The kernel instances, by launch shape: one CTA per tile (MH = 1 or 2 accumulators) or a pair.
+template <int MH>
+struct SingleKernels {
+  static constexpr size_t kSmem = Tile<MH>::Smem;
+  template <int NORM, int EPI, int OUT, int MAJ>
+  static void* get() {
+    return (void*)norm_linear_kernel<MH, NORM, EPI, OUT, MAJ>;
+  }
+};
+struct PairKernels {
+  static constexpr size_t kSmem = kPairSmem;
+  template <int NORM, int EPI, int OUT, int MAJ>
+  static void* get() {
+    return (void*)norm_linear_pair_kernel<NORM, EPI, OUT, MAJ>;
+  }
+};
+
+// Built combinations: the layer's forward with every norm and activation (K-major operands);
+// without a norm, the activation-gradient epilogue (K-major), and the plain bf16 product and the
+// fp32-accumulating product in every operand layout. Others return null.
+template <class KS, int MAJ>
+void* pick_plain(int out) {
+  return out == OUT_ACC32 ? KS::template get<GN_NORM_NONE, EPI_NONE, OUT_ACC32, MAJ>()
+                          : KS::template get<GN_NORM_NONE, EPI_NONE, OUT_BF16, MAJ>();
+}
+
+template <class KS, int NORM>
+void* pick_epi(int epi, int out, int maj) {
+  if constexpr (NORM == GN_NORM_NONE) {
+    if (maj != 0) {
+      if (out == OUT_DGRAD || (out == OUT_BF16 && epi != GN_EPI_NONE)) return nullptr;
+      return maj == 1 ? pick_plain<KS, 1>(out) : maj == 2 ? pick_plain<KS, 2>(out) : pick_plain<KS, 3>(out);
     }
-    if (out == OUT_ACC32) return (void*)norm_linear_kernel<MH, NORM, EPI_NONE, OUT_ACC32>;
-  } else if (out != OUT_BF16) {
+    if (out == OUT_DGRAD) {
+      if (epi == GN_EPI_GELU_TANH) return KS::template get<NORM, EPI_GELU_TANH, OUT_DGRAD, 0>();
+      if (epi == GN_EPI_SILU) return KS::template get<NORM, EPI_SILU, OUT_DGRAD, 0>();
+      return KS::template get<NORM, EPI_NONE, OUT_DGRAD, 0>();
+    }
+    if (out == OUT_ACC32) return KS::template get<NORM, EPI_NONE, OUT_ACC32, 0>();
+  } else if (out != OUT_BF16 || maj != 0) {
     return nullptr;
   }
-  if (epi == GN_EPI_GELU_TANH) return (void*)norm_linear_kernel<MH, NORM, EPI_GELU_TANH>;
-  if (epi == GN_EPI_SILU) return (void*)norm_linear_kernel<MH, NORM, EPI_SILU>;
-  return (void*)norm_linear_kernel<MH, NORM, EPI_NONE>;
+  if (epi == GN_EPI_GELU_TANH) return KS::template get<NORM, EPI_GELU_TANH, OUT_BF16, 0>();
+  if (epi == GN_EPI_SILU) return KS::template get<NORM, EPI_SILU, OUT_BF16, 0>();
+  return KS::template get<NORM, EPI_NONE, OUT_BF16, 0>();
 }
 
-template <int MH>
-void* pick(int norm, int epi, int out) {
-  return norm == GN_NORM_LN    ? pick_epi<MH, GN_NORM_LN>(epi, out)
-         : norm == GN_NORM_RMS ? pick_epi<MH, GN_NORM_RMS>(epi, out)
-                               : pick_epi<MH, GN_NORM_NONE>(epi, out);
+template <class KS>
+void* pick(int norm, int epi, int out, int maj) {
+  return norm == GN_NORM_LN    ? pick_epi<KS, GN_NORM_LN>(epi, out, maj)
+         : norm == GN_NORM_RMS ? pick_epi<KS, GN_NORM_RMS>(epi, out, maj)
+                               : pick_epi<KS, GN_NORM_NONE>(epi, out, maj);
 }
 
-template <int MH>
+template <class KS>
 bool set_smem_attr() {
   for (int norm = 0; norm < 3; ++norm)
     for (int epi = 0; epi < 3; ++epi)
-      for (int out = 0; out < 3; ++out) {
-        void* k = pick<MH>(norm, epi, out);
-        if (k && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Tile<MH>::Smem) !=
-                     cudaSuccess)
-          return false;
-      }
-  return true;
-}
-
-template <int NORM>
-void* pick_pair_epi(int epi, int out) {
-  if constexpr (NORM == GN_NORM_NONE) {
-    if (out == OUT_DGRAD) {
-      if (epi == GN_EPI_GELU_TANH) return (void*)norm_linear_pair_kernel<NORM, EPI_GELU_TANH, OUT_DGRAD>;
-      if (epi == GN_EPI_SILU) return (void*)norm_linear_pair_kernel<NORM, EPI_SILU, OUT_DGRAD>;
-      return (void*)norm_linear_pair_kernel<NORM, EPI_NONE, OUT_DGRAD>;
-    }
-    if (out == OUT_ACC32) return (void*)norm_linear_pair_kernel<NORM, EPI_NONE, OUT_ACC32>;
-  } else if (out != OUT_BF16) {
-    return nullptr;
-  }
-  if (epi == GN_EPI_GELU_TANH) return (void*)norm_linear_pair_kernel<NORM, EPI_GELU_TANH>;
-  if (epi == GN_EPI_SILU) return (void*)norm_linear_pair_kernel<NORM, EPI_SILU>;
-  return (void*)norm_linear_pair_kernel<NORM, EPI_NONE>;
-}
-
-void* pick_pair(int norm, int epi, int out) {
-  return norm == GN_NORM_LN    ? pick_pair_epi<GN_NORM_LN>(epi, out)
-         : norm == GN_NORM_RMS ? pick_pair_epi<GN_NORM_RMS>(epi, out)
-                               : pick_pair_epi<GN_NORM_NONE>(epi, out);
-}
-
-bool set_pair_smem_attr() {
-  for (int norm = 0; norm < 3; ++norm)
-    for (int epi = 0; epi < 3; ++epi)
-      for (int out = 0; out < 3; ++out) {
-        void* k = pick_pair(norm, epi, out);
-        if (k && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPairSmem) != cudaSuccess)
-          return false;
-      }
+      for (int out = 0; out < 3; ++out)
+        for (int maj = 0; maj < 4; ++maj) {
+          void* k = pick<KS>(norm, epi, out, maj);
+          if (k && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)KS::kSmem) != cudaSuccess)
+            return false;
+        }
   return true;
 }
 
@@ -908,21 +965,26 @@ bool set_pair_smem_attr() {
 #endif
 
 // The launch shared by the forward and the TiledLinear backward products: y (bf16, OUT_BF16 and
-// OUT_DGRAD) or y32 (fp32, OUT_ACC32) [M, N] from x [M, K] (row stride ldx) and Wf [N, K] (row
-// stride ldw), arguments validated by the caller.
+// OUT_DGRAD) or y32 (fp32, OUT_ACC32) [M, N] from x and Wf: x [M, K] (K-major) or [K, M] (MN-major,
+// maj bit 0), row stride ldx; Wf [N, K] or [K, N] (maj bit 1), row stride ldw. Arguments validated
+// by the caller.
 gn_status nl_run(const void* x, int64_t ldx, const void* Wf, int64_t ldw, const float* c, const float* d, void* y,
                  float* y32, int64_t ldy, const void* dy, int64_t lddy, float* mean, float* rstd, int64_t M,
-                 int64_t N, int64_t K, float eps, int norm, int epi, int out, cudaStream_t stream) {
+                 int64_t N, int64_t K, float eps, int norm, int epi, int out, int maj, cudaStream_t stream) {
   // pairs of SMs sharing 256 x 512 tiles once there are more than 128 rows and 256 columns;
   // one SM per 256 x 256 tile (two accumulators) for fewer columns; 128 x 256 for few rows
   const bool pair = GN_NL_PAIR && M > kUM && N > kBN;
   const int mh = M > kUM ? GN_NL_MH : 1;
   const int bm = pair ? 2 * kUM : kUM * mh;
+  // an MN-major operand is read as boxes of 64 M/N elements x 64 k-rows of the [K, M/N] matrix
   CUtensorMap ta, tb;
-  if (!make_map(&ta, x, M, K, ldx, pair ? (uint32_t)kUM : (uint32_t)bm) ||
-      !make_map(&tb, Wf, N, K, ldw, pair ? 128u : (uint32_t)kBN))
+  const bool amn = (maj & MAJ_A_MN) != 0, bmn = (maj & MAJ_B_MN) != 0;
+  if (!(amn ? make_map(&ta, x, K, M, ldx, 64u) : make_map(&ta, x, M, K, ldx, pair ? (uint32_t)kUM : (uint32_t)bm)) ||
+      !(bmn ? make_map(&tb, Wf, K, N, ldw, 64u) : make_map(&tb, Wf, N, K, ldw, pair ? 128u : (uint32_t)kBN)))
     return GN_ERR_CUDA;
-  void* kern = pair ? pick_pair(norm, epi, out) : mh == 2 ? pick<2>(norm, epi, out) : pick<1>(norm, epi, out);
+  void* kern = pair      ? pick<PairKernels>(norm, epi, out, maj)
+               : mh == 2 ? pick<SingleKernels<2>>(norm, epi, out, maj)
+                         : pick<SingleKernels<1>>(norm, epi, out, maj);
   if (!kern) return GN_ERR_UNSUPPORTED;
   // the dynamic shared-memory limits are attributes of the kernels on the current device: set
   // them once per device (0 = not yet, 1 = set, -1 = failed)
@@ -932,7 +994,9 @@ gn_status nl_run(const void* x, int64_t ldx, const void* Wf, int64_t ldw, const 
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GN_ERR_CUDA;
   {
     std::lock_guard<std::mutex> lk(attr_mu);
-    if (!attr_state[dev]) attr_state[dev] = set_smem_attr<1>() && set_smem_attr<2>() && set_pair_smem_attr() ? 1 : -1;
+    if (!attr_state[dev])
+      attr_state[dev] =
+          set_smem_attr<SingleKernels<1>>() && set_smem_attr<SingleKernels<2>>() && set_smem_attr<PairKernels>() ? 1 : -1;
     if (attr_state[dev] < 0) return GN_ERR_CUDA;
   }
   NlArgs a{};
@@ -1017,7 +1081,7 @@ extern "C" gn_status gn_norm_linear_fwd(const void* x, const void* Wf, const flo
   if (!x || !Wf || !y || (norm != GN_NORM_NONE && !rstd) || (norm == GN_NORM_LN && (!c || !mean))) return GN_ERR_NULL;
   if (!aligned16(x) || !aligned16(Wf) || !aligned16(y) || (c && !aligned16(c)) || (d && !aligned16(d)))
     return GN_ERR_ALIGN;
-  return nl_run(x, ldx, Wf, K, c, d, y, nullptr, ldy, nullptr, 0, mean, rstd, M, N, K, eps, norm, epi, OUT_BF16,
+  return nl_run(x, ldx, Wf, K, c, d, y, nullptr, ldy, nullptr, 0, mean, rstd, M, N, K, eps, norm, epi, OUT_BF16, 0,
                 (cudaStream_t)stream);
 }
 
@@ -1032,16 +1096,45 @@ extern "C" gn_status gn_linear_act_grad(const void* x, const void* Wf, const flo
   if (!x || !Wf || !dy || !dz) return GN_ERR_NULL;
   if (!aligned16(x) || !aligned16(Wf) || !aligned16(dy) || !aligned16(dz) || (d && !aligned16(d))) return GN_ERR_ALIGN;
   return nl_run(x, ldx, Wf, K, nullptr, d, dz, nullptr, lddz, dy, lddy, nullptr, nullptr, M, N, K, 0.0f, GN_NORM_NONE,
-                epi, OUT_DGRAD, (cudaStream_t)stream);
+                epi, OUT_DGRAD, 0, (cudaStream_t)stream);
+}
+
+namespace {
+// operand checks of the plain products: a K-major operand [rows, K] needs K contiguous and a
+// multiple of 8 (16-byte rows); an MN-major one [K, rows] needs its rows within the stride.
+// Returns the layout bits for nl_run, or -1.
+int plain_layouts(int64_t M, int64_t N, int64_t K, int64_t lda, int64_t ldb, gn_layout al, gn_layout bl) {
+  if ((al != GN_K_MAJOR && al != GN_MN_MAJOR) || (bl != GN_K_MAJOR && bl != GN_MN_MAJOR)) return -1;
+  if (M < 0 || N < 0 || K <= 0 || M > (int64_t)65535 * kUM || N > INT32_MAX || K > INT32_MAX) return -1;
+  if ((al == GN_K_MAJOR || bl == GN_K_MAJOR) && K % 8) return -1;
+  if (lda % 8 || ldb % 8) return -1;
+  if (lda < (al == GN_K_MAJOR ? K : M) || ldb < (bl == GN_K_MAJOR ? K : N)) return -1;
+  return (al == GN_MN_MAJOR ? MAJ_A_MN : 0) | (bl == GN_MN_MAJOR ? MAJ_B_MN : 0);
+}
+}  // namespace
+
+extern "C" gn_status gn_linear_bf16(const void* A, const void* B, const float* d, void* y, int64_t M, int64_t N,
+                                    int64_t K, int64_t lda, int64_t ldb, int64_t ldy, gn_layout a_layout,
+                                    gn_layout b_layout, gn_dtype dt, void* stream) {
+  if (dt != GN_BF16) return dt_ok(dt) ? GN_ERR_UNSUPPORTED : GN_ERR_DTYPE;
+  const int maj = plain_layouts(M, N, K, lda, ldb, a_layout, b_layout);
+  if (maj < 0 || ldy < N || ldy % 8) return GN_ERR_SHAPE;
+  if (M == 0 || N == 0) return GN_OK;
+  if (!A || !B || !y) return GN_ERR_NULL;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(y) || (d && !aligned16(d))) return GN_ERR_ALIGN;
+  return nl_run(A, lda, B, ldb, nullptr, d, y, nullptr, ldy, nullptr, 0, nullptr, nullptr, M, N, K, 0.0f, GN_NORM_NONE,
+                GN_EPI_NONE, OUT_BF16, maj, (cudaStream_t)stream);
 }
 
 extern "C" gn_status gn_linear_acc_f32(const void* A, const void* B, float* C, int64_t M, int64_t N, int64_t K,
-                                       int64_t lda, int64_t ldb, int64_t ldc, gn_dtype dt, void* stream) {
+                                       int64_t lda, int64_t ldb, int64_t ldc, gn_layout a_layout, gn_layout b_layout,
+                                       gn_dtype dt, void* stream) {
   if (dt != GN_BF16) return dt_ok(dt) ? GN_ERR_UNSUPPORTED : GN_ERR_DTYPE;
-  if (!nl_shape_ok(M, N, K) || lda < K || ldb < K || ldc < N || lda % 8 || ldb % 8 || ldc % 4) return GN_ERR_SHAPE;
+  const int maj = plain_layouts(M, N, K, lda, ldb, a_layout, b_layout);
+  if (maj < 0 || ldc < N || ldc % 4) return GN_ERR_SHAPE;
   if (M == 0 || N == 0) return GN_OK;
   if (!A || !B || !C) return GN_ERR_NULL;
   if (!aligned16(A) || !aligned16(B) || !aligned16(C)) return GN_ERR_ALIGN;
   return nl_run(A, lda, B, ldb, nullptr, nullptr, nullptr, C, ldc, nullptr, 0, nullptr, nullptr, M, N, K, 0.0f,
-                GN_NORM_NONE, GN_EPI_NONE, OUT_ACC32, (cudaStream_t)stream);
+                GN_NORM_NONE, GN_EPI_NONE, OUT_ACC32, maj, (cudaStream_t)stream);
 }

@@ -1,54 +1,12 @@
-// tiled_aux.cu - the memory-bound steps of the TiledLinear backward around its tensor-core
+// tiled_aux.cu - the memory-bound step of the TiledLinear backward next to its tensor-core
 // products (Helios kernels article, section "内核三 TiledLinear": per chunk of tokens, recompute
-// the pre-activation, then dx = dz W and dW += dz^T x, db += sum dz):
-//   * gn_transpose: a bf16 matrix transposed (the weight gradient contracts over the tokens, so
-//     its two operands are fed to the K-major tensor-core kernel as dz^T and x^T);
-//   * gn_colsum_bf16: column sums of a bf16 matrix into fp32 (db), in a fixed order.
+// the pre-activation, then dx = dz W and dW += dz^T x, db += sum dz): gn_colsum_bf16, the column
+// sums of a bf16 matrix into fp32 (db), in a fixed order.
 #include "gn_common.cuh"
 #include "gn_host.h"
 
 namespace gn {
 namespace {
-
-// 64 x 64 tile per CTA of 256 threads. Loads: thread t reads 16 elements (two 16-byte vectors)
-// of row t / 4 of the tile, four threads per 128-byte row segment. The tile sits in shared memory
-// as 32-bit words (two elements of a row), rows padded to 33 words. Stores: thread t writes 16
-// elements of output row t / 4 (= input column), gathered from 16 input rows, as two 16-byte
-// vectors. Columns are a multiple of 8 (whole vectors); a row count that is not is padded: the
-// output rows are written up to the next multiple of 8 columns, with zeros past the input rows.
-__global__ void __launch_bounds__(256) transpose_bf16_kernel(const __nv_bfloat16* __restrict__ src,
-                                                             __nv_bfloat16* __restrict__ dst, int64_t rows,
-                                                             int64_t cols, int64_t lds, int64_t ldd) {
-  __shared__ uint32_t tile[64][33];
-  const int t = threadIdx.x;
-  const int64_t r0 = (int64_t)blockIdx.y * 64, c0 = (int64_t)blockIdx.x * 64;
-  {
-    const int r = t >> 2, c = (t & 3) * 16;
-    uint4 v[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
-    if (r0 + r < rows) {
-      const __nv_bfloat16* p = src + (r0 + r) * lds + c0 + c;
-      if (c0 + c < cols) v[0] = ld_stream(p);
-      if (c0 + c + 8 < cols) v[1] = ld_stream(p + 8);
-    }
-    const uint32_t w[8] = {v[0].x, v[0].y, v[0].z, v[0].w, v[1].x, v[1].y, v[1].z, v[1].w};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) tile[r][c / 2 + i] = w[i];
-  }
-  __syncthreads();
-  const int oc = t >> 2, seg = (t & 3) * 16;  // output row oc (input column c0 + oc), input rows seg..
-  if (c0 + oc >= cols) return;
-  uint32_t w[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint32_t a = tile[seg + 2 * i][oc >> 1], b = tile[seg + 2 * i + 1][oc >> 1];
-    const uint32_t lo = (oc & 1) ? (a >> 16) : (a & 0xffffu);
-    const uint32_t hi = (oc & 1) ? (b & 0xffff0000u) : (b << 16);
-    w[i] = lo | hi;
-  }
-  __nv_bfloat16* q = dst + (c0 + oc) * ldd + r0 + seg;
-  if (r0 + seg < rows) st_stream(q, make_uint4(w[0], w[1], w[2], w[3]));
-  if (r0 + seg + 8 < rows) st_stream(q + 8, make_uint4(w[4], w[5], w[6], w[7]));  // zeros past rows
-}
 
 constexpr int kColsumSlices = 64;
 
@@ -94,24 +52,6 @@ __global__ void __launch_bounds__(256) colsum_bf16_final(const float* __restrict
 }  // namespace gn
 
 using namespace gn;
-
-extern "C" gn_status gn_transpose(const void* src, void* dst, int64_t rows, int64_t cols, int64_t ld_src,
-                                  int64_t ld_dst, gn_dtype dt, void* stream) {
-  if (dt != GN_BF16) return dt_ok(dt) ? GN_ERR_UNSUPPORTED : GN_ERR_DTYPE;
-  if (rows < 0 || cols < 0 || ld_src < cols || ld_dst < (rows + 7) / 8 * 8 || cols % 8 || ld_src % 8 || ld_dst % 8)
-    return GN_ERR_SHAPE;
-  if (rows == 0 || cols == 0) return GN_OK;
-  if (!src || !dst) return GN_ERR_NULL;
-  if (!aligned16(src) || !aligned16(dst)) return GN_ERR_ALIGN;
-  if ((rows + 63) / 64 > 65535) return GN_ERR_SHAPE;
-  if (!kernel_attrs((const void*)transpose_bf16_kernel, 0)) return GN_ERR_CUDA;
-  const dim3 grid((unsigned)((cols + 63) / 64), (unsigned)((rows + 63) / 64));
-  transpose_bf16_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(static_cast<const __nv_bfloat16*>(src),
-                                                                static_cast<__nv_bfloat16*>(dst), rows, cols, ld_src,
-                                                                ld_dst);
-  count_launches(1);
-  return launch_status();
-}
 
 extern "C" size_t gn_colsum_bf16_workspace(int64_t cols) {
   return cols > 0 ? (size_t)kColsumSlices * (size_t)cols * sizeof(float) : 0;
