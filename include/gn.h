@@ -320,7 +320,7 @@ gn_status gn_selftest_wait_timeout(uint32_t limit_us, void* stream);
 
 /* Tuning knobs of the launch planner, for benchmarking sweeps. key is one of "stages",
  * "ctas_per_sm", "vpt", "unit_bytes", "group_rows", "fwd_warps" (warps per CTA of the
- * one-warp-per-row norm forward, at most 16), "fwd_path" (norm forward of long rows: 1 = the
+ * one-warp-per-row norm forward, at most 20), "fwd_path" (norm forward of long rows: 1 = the
  * CTA-per-row pipeline, 2 = one warp per row with two-pass LayerNorm statistics, 3 = one warp per
  * row with one shifted pass; by default RMSNorm takes the first and LayerNorm the third);
  * value 0 restores the default. Returns

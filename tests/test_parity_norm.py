@@ -86,7 +86,7 @@ def test_layernorm_fwd_bwd(gpu, rows, hidden, dtype):
 
 
 @pytest.mark.parametrize("path,warps,stages", [(0, 0, 0), (1, 0, 0), (1, 0, 4), (2, 4, 3), (2, 0, 4), (2, 5, 2),
-                                               (3, 0, 0), (3, 6, 3)])
+                                               (3, 0, 0), (3, 6, 3), (3, 0, 2), (2, 20, 1), (3, 13, 1)])
 def test_norm_forward_kernels_of_long_rows(gpu, path, warps, stages):
     """The forward kernels of long rows - the CTA-per-row pipeline (fwd_path 1), one warp per row
     with the LayerNorm statistics in two passes (fwd_path 2) or one shifted pass (fwd_path 3), and

@@ -238,7 +238,7 @@ extern "C" gn_status gn_tune(const char* key, int value) {
   } else if (!strcmp(key, "group_rows")) {
     g_tune.group_rows = value;
   } else if (!strcmp(key, "fwd_warps")) {
-    if (value > 16) return GN_ERR_SHAPE;
+    if (value > 20) return GN_ERR_SHAPE;
     g_tune.fwd_warps = value;
   } else if (!strcmp(key, "fwd_path")) {
     if (value > 3) return GN_ERR_SHAPE;
