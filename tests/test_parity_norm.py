@@ -158,6 +158,48 @@ def test_unsupported_hidden_is_reported(gpu):
     assert e.value.status == gpu.GN_ERR_UNSUPPORTED
 
 
+@pytest.mark.parametrize("dtype,fwd_max,bwd_max", [("bf16", 20480, 10240), ("f32", 10240, 5120)])
+def test_widest_rows(gpu, dtype, fwd_max, bwd_max):
+    """The widest rows each path takes (the CTA-per-row kernels: 320 consumer threads, at most 8
+    vectors a thread forward and 4 backward) match the oracle; one 16-byte vector more is
+    refused with GN_ERR_UNSUPPORTED before anything is launched."""
+    vec = 8 if dtype == "bf16" else 4
+    for hidden, bwd in ((fwd_max, False), (bwd_max, True)):
+        d = wl.rmsnorm(M=3, N=hidden, dtype=dtype, gemma=True, outliers=False)
+        x, w = to_rows(d["x"]), to_dev(d["w"])
+        y, r = gpu.rmsnorm_fwd(x, w, d["eps"], gemma=True, epilogue="silu")
+        ry, rr = oracle.rmsnorm_fwd(d["x"], d["w"], d["eps"], gemma=True, act="silu")
+        assert_close(to_np(y), ry, io_tol(dtype), f"rms {dtype} {hidden} y")
+        dl = wl.layernorm(M=3, N=hidden, dtype=dtype)
+        xl, wt, bt = to_rows(dl["x"]), to_dev(dl["w"]), to_dev(dl["b"])
+        yl, mu, rs = gpu.layernorm_fwd(xl, wt, bt, dl["eps"], epilogue="gelu_tanh")
+        ryl, _, _ = oracle.layernorm_fwd(dl["x"], dl["w"], dl["b"], dl["eps"], act="gelu_tanh")
+        assert_close(to_np(yl), ryl, io_tol(dtype), f"ln {dtype} {hidden} y")
+        if bwd:
+            dx, dw = gpu.rmsnorm_bwd(x, w, r, to_rows(d["dy"]), gemma=True, epilogue="silu")
+            rdx, rdw = oracle.rmsnorm_bwd(d["x"], d["w"], d["dy"], d["eps"], gemma=True, act="silu")
+            assert_close(to_np(dx), rdx, grad_tol(dtype), f"rms {dtype} {hidden} dx")
+            assert_close(to_np(dw), rdw, wgrad_tol(dtype, rdw), f"rms {dtype} {hidden} dw")
+            dxl, dwl, dbl = gpu.layernorm_bwd(xl, wt, bt, mu, rs, to_rows(dl["dy"]), epilogue="gelu_tanh")
+            rdxl, rdwl, rdbl = oracle.layernorm_bwd(dl["x"], dl["w"], dl["b"], dl["dy"], dl["eps"], act="gelu_tanh")
+            assert_close(to_np(dxl), rdxl, grad_tol(dtype), f"ln {dtype} {hidden} dx")
+            assert_close(to_np(dwl), rdwl, wgrad_tol(dtype, rdwl), f"ln {dtype} {hidden} dw")
+            assert_close(to_np(dbl), rdbl, wgrad_tol(dtype, rdbl), f"ln {dtype} {hidden} db")
+    torch.cuda.synchronize()
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    for hidden, bwd in ((fwd_max + vec, False), (bwd_max + vec, True)):
+        x = torch.zeros(2, hidden, dtype=tdt, device="cuda")
+        w = torch.ones(hidden, dtype=tdt, device="cuda")
+        st = torch.ones(2, device="cuda")
+        calls = [lambda: gpu.rmsnorm_bwd(x, w, st, x), lambda: gpu.layernorm_bwd(x, w, w, st, st, x)] if bwd else \
+            [lambda: gpu.rmsnorm_fwd(x, w), lambda: gpu.layernorm_fwd(x, w, w)]
+        for call in calls:
+            with pytest.raises(gpu.GnError) as e:
+                call()
+            assert e.value.status == gpu.GN_ERR_UNSUPPORTED, hidden
+    assert gpu.device_error(clear=True) == 0
+
+
 def test_deterministic_weight_gradients(gpu):
     d = wl.rmsnorm(M=3000, N=5120, dtype="bf16")
     x, w, dy = to_dev(d["x"]), to_dev(d["w"]), to_dev(d["dy"])

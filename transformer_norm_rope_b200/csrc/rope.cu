@@ -434,6 +434,11 @@ gn_status plan_rope(int64_t B, int64_t S, int64_t H, int64_t D, int ntens, int m
       cw = c;
       break;
     }
+  // the plain rotation (one CTA per SM) streams best with 8 consumer warps, two per scheduler,
+  // even where a pass over the slab then leaves lanes idle (B200, q and k [1, 32760, 40, 128]:
+  // 10 warps 6250-6390 GB/s, 8 warps 6410-6500); the qk-norm passes do more arithmetic per
+  // vector and keep the divisor rule (8 warps: 5690-5920 against 5860-6050 forward)
+  if (mode == ROPE && nv_t >= 32 * 8) cw = 8;
   if (g_tune.group_rows) cw = g_tune.group_rows > kMaxConsumerWarps ? kMaxConsumerWarps : g_tune.group_rows;
   p->cwarps = cw;
   p->threads = 32 * (1 + cw);
