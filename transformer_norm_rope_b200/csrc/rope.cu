@@ -182,7 +182,10 @@ struct Planes {
 
 // One 16-byte vector w of tensor TT's slab of the current unit (valid when w < nv_t).
 // wt0/wt1: this lane's weights w' in planes; dw0/dw1: its weight-gradient accumulators.
-template <typename T, int MODE, int TT>
+// LPH: lanes (16-byte vectors) per head when known at compile time (16 for bf16 heads of 128,
+// the benchmark's), so that the head index, the lane within the head and the head shuffles
+// fold to constants; 0 = taken from the launch.
+template <typename T, int MODE, int TT, int LPH>
 __device__ __forceinline__ void rope_vec(const RopeArgs& a, const VecCtx& c, int w, int nv_t,
                                          const float2 (&wt0)[Planes<T>::K], const float2 (&wt1)[Planes<T>::K],
                                          float2 (&dw0)[Planes<T>::K], float2 (&dw1)[Planes<T>::K]) {
@@ -192,7 +195,10 @@ __device__ __forceinline__ void rope_vec(const RopeArgs& a, const VecCtx& c, int
   const bool valid = w < nv_t;
   if (!valid) w = 0;
   int hh, l;
-  if (c.lph_shift >= 0) {
+  if constexpr (LPH > 0) {
+    hh = w / LPH;
+    l = w % LPH;
+  } else if (c.lph_shift >= 0) {
     hh = w >> c.lph_shift;
     l = w & (c.lph - 1);
   } else {
@@ -222,7 +228,7 @@ __device__ __forceinline__ void rope_vec(const RopeArgs& a, const VecCtx& c, int
     float2 ss2 = fma2(x0[0], x0[0], mul2(x1[0], x1[0]));
 #pragma unroll
     for (int k = 1; k < K; ++k) ss2 = fma2(x1[k], x1[k], fma2(x0[k], x0[k], ss2));
-    const float ss = group_sum_rt(ss2.x + ss2.y, c.lph);
+    const float ss = LPH > 0 ? group_sum<LPH>(ss2.x + ss2.y) : group_sum_rt(ss2.x + ss2.y, c.lph);
     const float r = rsqrtf(fmaf(ss, c.inv_d, a.eps));
     const float2 r2 = dup2(r);
 #pragma unroll
@@ -255,7 +261,7 @@ __device__ __forceinline__ void rope_vec(const RopeArgs& a, const VecCtx& c, int
       dw0[k] = fma2(g0, h0[k], dw0[k]);
       dw1[k] = fma2(g1, h1[k], dw1[k]);
     }
-    const float cd = group_sum_rt(cd2.x + cd2.y, c.lph) * c.inv_d;
+    const float cd = (LPH > 0 ? group_sum<LPH>(cd2.x + cd2.y) : group_sum_rt(cd2.x + cd2.y, c.lph)) * c.inv_d;
     const float2 ncd = dup2(-cd);
 #pragma unroll
     for (int k = 0; k < K; ++k) {
@@ -266,7 +272,7 @@ __device__ __forceinline__ void rope_vec(const RopeArgs& a, const VecCtx& c, int
   if (valid) st_stream(static_cast<T*>(a.out[TT]) + c.row0 * a.D + (int64_t)w * Vec<T>::N, PL::store(o0, o1));
 }
 
-template <typename T, int MODE, bool GEMMA>
+template <typename T, int MODE, bool GEMMA, int LPH>
 __global__ void __launch_bounds__(kRopeMaxThreads, 2) rope_kernel(const RopeArgs a) {
   using V = Vec<T>;
   constexpr int E = V::N;      // elements per 16-byte vector
@@ -279,7 +285,7 @@ __global__ void __launch_bounds__(kRopeMaxThreads, 2) rope_kernel(const RopeArgs
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ncw = (int)(blockDim.x >> 5) - 1;  // consumer warps
   const int D = a.D, HC = a.HC;
-  const int lph = D / E;                       // vectors (lanes) per head
+  const int lph = LPH > 0 ? LPH : D / E;       // vectors (lanes) per head
   const int nv_t = HC * lph;                   // vectors per tensor slab
   const uint32_t nslots = (uint32_t)a.ntens * (BWD ? 2u : 1u);
   const uint32_t sstride = nslots * a.tslot + a.tabslot + (BWD ? (uint32_t)a.ntens * a.statslot : 0u);
@@ -371,9 +377,9 @@ __global__ void __launch_bounds__(kRopeMaxThreads, 2) rope_kernel(const RopeArgs
     const VecCtx ctx{sb, tcos, tcos + D / 2, tstat, (int)(a.statslot / 4), row0, lph, a.lph_shift, inv_d};
     // Each pass covers one tensor (the tensor is a compile-time argument of the body); the
     // trip count is the same for every lane of a warp, so the head shuffles see full warps.
-    for (int vb = 0; vb < nv_t; vb += nct) rope_vec<T, MODE, 0>(a, ctx, vb + ct, nv_t, wq0, wq1, dq0, dq1);
+    for (int vb = 0; vb < nv_t; vb += nct) rope_vec<T, MODE, 0, LPH>(a, ctx, vb + ct, nv_t, wq0, wq1, dq0, dq1);
     if (a.ntens > 1)
-      for (int vb = 0; vb < nv_t; vb += nct) rope_vec<T, MODE, 1>(a, ctx, vb + ct, nv_t, wk0, wk1, dk0, dk1);
+      for (int vb = 0; vb < nv_t; vb += nct) rope_vec<T, MODE, 1, LPH>(a, ctx, vb + ct, nv_t, wk0, wk1, dk0, dk1);
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[st]);
     if (++st == a.stages) st = 0, ph ^= 1u;
@@ -466,23 +472,25 @@ gn_status plan_rope(int64_t B, int64_t S, int64_t H, int64_t D, int ntens, int m
   return GN_OK;
 }
 
-void* pick(gn_dtype dt, int mode, bool gemma) {
-  if (dt == GN_BF16) {
-    if (mode == ROPE) return (void*)rope_kernel<__nv_bfloat16, ROPE, false>;
-    if (mode == QK_FWD)
-      return gemma ? (void*)rope_kernel<__nv_bfloat16, QK_FWD, true> : (void*)rope_kernel<__nv_bfloat16, QK_FWD, false>;
-    return gemma ? (void*)rope_kernel<__nv_bfloat16, QK_BWD, true> : (void*)rope_kernel<__nv_bfloat16, QK_BWD, false>;
-  }
-  if (mode == ROPE) return (void*)rope_kernel<float, ROPE, false>;
-  if (mode == QK_FWD) return gemma ? (void*)rope_kernel<float, QK_FWD, true> : (void*)rope_kernel<float, QK_FWD, false>;
-  return gemma ? (void*)rope_kernel<float, QK_BWD, true> : (void*)rope_kernel<float, QK_BWD, false>;
+template <typename T, int LPH>
+void* pick_t(int mode, bool gemma) {
+  if (mode == ROPE) return (void*)rope_kernel<T, ROPE, false, LPH>;
+  if (mode == QK_FWD) return gemma ? (void*)rope_kernel<T, QK_FWD, true, LPH> : (void*)rope_kernel<T, QK_FWD, false, LPH>;
+  return gemma ? (void*)rope_kernel<T, QK_BWD, true, LPH> : (void*)rope_kernel<T, QK_BWD, false, LPH>;
+}
+
+// heads of 16 vectors (bf16 D = 128, fp32 D = 64) take the instance with the head geometry
+// folded in
+void* pick(gn_dtype dt, int mode, bool gemma, int64_t D) {
+  if (dt == GN_BF16) return D == 128 ? pick_t<__nv_bfloat16, 16>(mode, gemma) : pick_t<__nv_bfloat16, 0>(mode, gemma);
+  return D == 64 ? pick_t<float, 16>(mode, gemma) : pick_t<float, 0>(mode, gemma);
 }
 
 gn_status setup(int64_t B, int64_t S, int64_t H, int64_t D, int ntens, int mode, gn_dtype dt, bool gemma,
                 RopePlan* p, void** kern, int* grid) {
   gn_status st = plan_rope(B, S, H, D, ntens, mode, dt_size(dt), p);
   if (st != GN_OK) return st;
-  *kern = pick(dt, mode, gemma);
+  *kern = pick(dt, mode, gemma, D);
   const int cap = g_tune.ctas_per_sm ? g_tune.ctas_per_sm : mode == ROPE ? 1 : 8;
   int g = persistent_grid(*kern, p->threads, p->smem, cap);
   if (g <= 0) return GN_ERR_CUDA;
