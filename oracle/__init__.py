@@ -208,6 +208,28 @@ def norm_linear(x, g, beta, W, bias, eps, norm="ln", gemma=False, act="none"):
     return y, mu, rs
 
 
+def norm_linear_bwd(x, g, beta, W, bias, dy, eps, norm="ln", gemma=False, act="none"):
+    """Gradients of sum(dy * act(norm(x) W^T + bias)) for the layer that normalizes the rows of x
+    and feeds them to the linear layer (Janus-Pro inference page, section 4.1; HY-Motion page,
+    section 3.1): -> dx [M,K], dg [K], dbeta [K] (LayerNorm; None for RMSNorm), dW [N,K],
+    dbias [N]. By the chain rule: the normalized rows xn = norm(x) in fp64, the linear layer's
+    gradients at xn (dxn, dW, dbias), then the normalization's backward with dxn as the gradient of
+    its output. RMSNorm needs its weight g."""
+    if norm == "ln":
+        xn, _, _ = layernorm_fwd(x, g, beta, eps)
+        dxn, dW, db = linear_act_bwd(xn, W, bias, dy, act)
+        dx, dg, dbeta = layernorm_bwd(x, g, beta, dxn, eps)
+        return dx, dg, dbeta, dW, db
+    if norm != "rms":
+        raise ValueError(f"norm {norm!r}")
+    if g is None:
+        raise ValueError("RMSNorm needs its weight g")
+    xn, _ = rmsnorm_fwd(x, g, eps, gemma=gemma)
+    dxn, dW, db = linear_act_bwd(xn, W, bias, dy, act)
+    dx, dg = rmsnorm_bwd(x, g, dxn, eps, gemma=gemma)
+    return dx, dg, None, dW, db
+
+
 def linear_act_bwd(x, W, bias, dy, act="none"):
     """Gradients of sum(dy * act(x W^T + bias)): dx[M,K], dW[N,K], dbias[N]."""
     x, xd = _in(x)

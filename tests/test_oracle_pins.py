@@ -515,3 +515,24 @@ def test_linear_act_bwd_finite_differences():
     np.testing.assert_allclose(dx, _fd_grad(loss, x), rtol=1e-6, atol=1e-8)
     np.testing.assert_allclose(dW, _fd_grad(loss, W), rtol=1e-6, atol=1e-8)
     np.testing.assert_allclose(db, _fd_grad(loss, b), rtol=1e-6, atol=1e-8)
+
+
+@pytest.mark.parametrize("norm,act,gemma", [("ln", "silu", False), ("ln", "gelu_tanh", False), ("rms", "silu", True),
+                                            ("rms", "none", False)])
+def test_norm_linear_bwd_finite_differences(norm, act, gemma):
+    """The backward of the normalization followed by the linear layer, against central differences
+    of the oracle's own forward (fp64): every gradient, every element. A dropped term of the
+    norm's backward, a transposed product or a wrong chain-rule order fails here."""
+    M, N, K = 3, 4, 6
+    x = rng.standard_normal((M, K)) * 2.0 + 0.5
+    g = 1.0 + 0.3 * rng.standard_normal(K)
+    beta = 0.2 * rng.standard_normal(K) if norm == "ln" else None
+    W, b = rng.standard_normal((N, K)), rng.standard_normal(N)
+    dy = rng.standard_normal((M, N))
+    eps = 1e-3
+    loss = lambda: float((oracle.norm_linear(x, g, beta, W, b, eps, norm, gemma=gemma, act=act)[0] * dy).sum())
+    dx, dg, dbeta, dW, db = oracle.norm_linear_bwd(x, g, beta, W, b, dy, eps, norm, gemma=gemma, act=act)
+    for got, var in ((dx, x), (dg, g), (dW, W), (db, b)) + (((dbeta, beta),) if norm == "ln" else ()):
+        np.testing.assert_allclose(got, _fd_grad(loss, var), rtol=1e-6, atol=1e-8)
+    if norm != "ln":
+        assert dbeta is None
