@@ -425,6 +425,25 @@ def norm_linear_measure(gn, torch, dev, scale, seed, reps=10):
         return statistics.median(a.elapsed_time(b) for a, b in ev) * 1e-3
 
     t_f, t_u = timed(fused), timed(unfused)
+    # the training backward (this library's kernels only) beside torch autograd of the unfused
+    # layer (torch LayerNorm, cuBLAS, SiLU), both from the same upstream gradient
+    from transformer_norm_rope_b200 import norm_linear as nl
+
+    dy = torch.randn(M, N, device=dev, dtype=torch.bfloat16)
+    _, mu, rs = nl.forward(x, g, beta, W, bias, d["eps"], "ln", False, "silu")
+
+    def bwd():
+        nl.backward(x, g, beta, W, bias, mu, rs, dy, d["eps"], "ln", False, "silu")
+
+    leaves = [t.detach().clone().requires_grad_() for t in (x, g, beta, W, bias)]
+
+    def autograd_fwd_bwd():
+        xa, ga, ba, Wa, bia = leaves
+        ya = torch.nn.functional.silu(torch.nn.functional.linear(
+            torch.nn.functional.layer_norm(xa, (K,), ga, ba, d["eps"]), Wa, bia))
+        ya.backward(dy)
+
+    t_b, t_ab = timed(bwd), timed(autograd_fwd_bwd)
     flops = 2.0 * M * N * K
     tf = flops / t_f / 1e12
     peak = None
@@ -440,7 +459,12 @@ def norm_linear_measure(gn, torch, dev, scale, seed, reps=10):
                          "frac": round(tf / peak, 4), "peak_source": kind},
             "unfused_ms": round(t_u * 1e3, 4),
             "unfused": "LayerNorm kernel (bf16 activations) + cuBLAS addmm + SiLU (torch)",
-            "speedup_vs_unfused": round(t_u / t_f, 3)}
+            "speedup_vs_unfused": round(t_u / t_f, 3),
+            "backward_ms": round(t_b * 1e3, 4),
+            "fwd_bwd_ms": round((t_f + t_b) * 1e3, 4),
+            "torch_autograd_fwd_bwd_ms": round(t_ab * 1e3, 4),
+            "backward": "normalized rows recomputed, activation gradient in the product epilogue, dx and fp32 dW "
+                        "on the tensor cores with MN-major operands, column sums, LayerNorm backward"}
 
 
 def tiled_linear_measure(gn, torch, dev, scale, seed, reps=5):

@@ -86,3 +86,51 @@ def test_norm_linear_full_size_sampled_rows(gpu):
     assert_close(to_np(y)[rows], ref, "bf16", "full-size y")
     assert_close(to_np(rs)[rows], rrs, (1e-5, 0.0), "full-size rstd")
     assert gpu.device_error(clear=True) == 0
+
+
+@pytest.mark.parametrize("M,N,K", [(300, 264, 520), (257, 520, 1000), (64, 40, 136)])
+@pytest.mark.parametrize("norm,act,gemma", [("ln", "silu", False), ("ln", "gelu_tanh", False), ("rms", "silu", True),
+                                            ("rms", "none", False)])
+def test_norm_linear_backward_matches_oracle(gpu, M, N, K, norm, act, gemma):
+    """The training backward of the fused layer (normalized rows recomputed, activation gradient in
+    the product's epilogue, dW and the gradient of the normalized rows on the tensor cores, then the
+    normalization's backward with the forward's saved statistics) against the oracle's chain rule
+    in fp64. dx within the bf16 gradient tolerance; dW, dbias and the norm's dg, dbeta (sums over
+    the rows) relative to their scale."""
+    from transformer_norm_rope_b200 import norm_linear as nl
+
+    x, gw, beta, W, bias = _inputs(M, N, K, seed=M + N + K, norm=norm, gemma=gemma)
+    dy = wl.bf16_bits(np.random.default_rng(M * N).standard_normal((M, N)).astype(np.float32))
+    eps = 1e-5
+    dev = [None if a is None else to_dev(a) for a in (x, gw, beta, W, bias, dy)]
+    xt, gt, bt, Wt, biast, dyt = dev
+    y, mu, rs = nl.forward(xt, gt, bt, Wt, biast, eps, norm, gemma, act)
+    dx, dg, dbeta, dW, db = nl.backward(xt, gt, bt, Wt, biast, mu, rs, dyt, eps, norm, gemma, act)
+    torch.cuda.synchronize()
+    rdx, rdg, rdbeta, rdW, rdb = oracle.norm_linear_bwd(x, gw, beta, W, bias, dy, eps, norm, gemma=gemma, act=act)
+    tag = f"{norm} {act} gemma={gemma} {M}x{N}x{K}"
+    assert_close(to_np(dx), rdx, "grad_bf16", tag + " dx")
+    for name, got, ref in (("dg", dg, rdg), ("dbeta", dbeta, rdbeta), ("dW", dW, rdW), ("dbias", db, rdb)):
+        if ref is None:
+            assert got is None, name
+            continue
+        sc = float(np.abs(ref).max())
+        assert_close(to_np(got), ref, (2e-2, 2e-2 * sc), tag + " " + name)
+    assert gpu.device_error(clear=True) == 0
+
+
+def test_norm_linear_autograd_function_matches_backward(gpu):
+    from transformer_norm_rope_b200 import norm_linear as nl
+
+    x, gw, beta, W, bias = _inputs(256, 264, 512, seed=7, norm="ln")
+    dy = to_dev(wl.bf16_bits(np.random.default_rng(8).standard_normal((256, 264)).astype(np.float32)))
+    leaves = [to_dev(a).requires_grad_() for a in (x, gw, beta, W, bias)]
+    y = nl.NormLinearFunction.apply(*leaves, 1e-5, "ln", False, "silu")
+    y.backward(dy)
+    xt, gt, bt, Wt, biast = (to_dev(a) for a in (x, gw, beta, W, bias))
+    _, mu, rs = nl.forward(xt, gt, bt, Wt, biast, 1e-5, "ln", False, "silu")
+    ref = nl.backward(xt, gt, bt, Wt, biast, mu, rs, dy, 1e-5, "ln", False, "silu")
+    torch.cuda.synchronize()
+    assert torch.equal(leaves[0].grad, ref[0])
+    for leaf, r in zip(leaves[1:], (ref[1], ref[2], ref[3], ref[4])):
+        assert leaf.grad.dtype == leaf.dtype and torch.equal(leaf.grad, r.to(leaf.dtype))
