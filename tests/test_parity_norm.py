@@ -6,6 +6,7 @@ TMA pipeline for long rows), strided rows, in-place outputs and empty inputs. Th
 cases run the exact launch configuration the benchmark times and compare every output element,
 every saved statistic and the complete weight gradients with the oracle.
 """
+import numpy as np
 import pytest
 import torch
 
@@ -197,6 +198,55 @@ def test_widest_rows(gpu, dtype, fwd_max, bwd_max):
             with pytest.raises(gpu.GnError) as e:
                 call()
             assert e.value.status == gpu.GN_ERR_UNSUPPORTED, hidden
+    assert gpu.device_error(clear=True) == 0
+
+
+def _degenerate_rows(hidden, rng):
+    """Rows the statistics can trip on: all zero, constant, a large mean with a small spread (the
+    shifted one-pass variance must not cancel), one outlier, a tiny scale, alternating signs."""
+    j = np.arange(hidden)
+    rows = [np.zeros(hidden), np.full(hidden, 3.5), 1000.0 + 8.0 * (j % 2), np.where(j == hidden // 3, 500.0, 0.25),
+            1e-3 * rng.standard_normal(hidden), np.where(j % 2 == 0, 1.0, -1.0)]
+    return np.stack(rows).astype(np.float32)
+
+
+@pytest.mark.parametrize("hidden,dtype", [(5120, "bf16"), (64, "bf16"), (1000, "f32"), (2051, "bf16")])
+def test_degenerate_rows(gpu, hidden, dtype):
+    """Zero, constant, far-off-centre, outlier, tiny and alternating rows through every norm
+    kernel (CTA, warp and lane-group paths by row width) against the oracle: y and the saved
+    statistics of the forwards, dx and the weight gradients of the backwards."""
+    rng = np.random.default_rng(hidden)
+    xf = _degenerate_rows(hidden, rng)
+    conv = (lambda a: wl.bf16_bits(a)) if dtype == "bf16" else (lambda a: a.astype(np.float32))  # noqa: E731
+    x = conv(xf)
+    w = conv((1.0 + 0.1 * rng.standard_normal(hidden)).astype(np.float32))
+    b = conv((0.1 * rng.standard_normal(hidden)).astype(np.float32))
+    dy = conv(rng.standard_normal(xf.shape).astype(np.float32))
+    xt, wt, bt, dyt = to_rows(x), to_dev(w), to_dev(b), to_rows(dy)
+    for gemma, eps in ((False, 1e-6), (True, 1e-5)):
+        y, r = gpu.rmsnorm_fwd(xt, wt, eps, gemma=gemma, epilogue="silu")
+        dx, dw = gpu.rmsnorm_bwd(xt, wt, r, dyt, gemma=gemma, epilogue="silu")
+        torch.cuda.synchronize()
+        ry, rr = oracle.rmsnorm_fwd(x, w, eps, gemma=gemma, act="silu")
+        rdx, rdw = oracle.rmsnorm_bwd(x, w, dy, eps, gemma=gemma, act="silu")
+        tag = f"rms {dtype} {hidden} gemma={gemma}"
+        assert_close(to_np(y), ry, io_tol(dtype), tag + " y")
+        assert_close(to_np(r), rr, "stat", tag + " inv_rms")
+        assert_close(to_np(dx), rdx, grad_tol(dtype), tag + " dx")
+        assert_close(to_np(dw), rdw, wgrad_tol(dtype, rdw), tag + " dw")
+    eps = 1e-5
+    y, mu, rs = gpu.layernorm_fwd(xt, wt, bt, eps, epilogue="gelu_tanh")
+    dx, dw, db = gpu.layernorm_bwd(xt, wt, bt, mu, rs, dyt, epilogue="gelu_tanh")
+    torch.cuda.synchronize()
+    ry, rmu, rrs = oracle.layernorm_fwd(x, w, b, eps, act="gelu_tanh")
+    rdx, rdw, rdb = oracle.layernorm_bwd(x, w, b, dy, eps, act="gelu_tanh")
+    tag = f"ln {dtype} {hidden}"
+    assert_close(to_np(y), ry, io_tol(dtype), tag + " y")
+    assert_close(to_np(mu), rmu, (1e-5, 1e-6), tag + " mean")
+    assert_close(to_np(rs), rrs, "stat", tag + " rstd")
+    assert_close(to_np(dx), rdx, grad_tol(dtype), tag + " dx")
+    assert_close(to_np(dw), rdw, wgrad_tol(dtype, rdw), tag + " dw")
+    assert_close(to_np(db), rdb, wgrad_tol(dtype, rdb), tag + " db")
     assert gpu.device_error(clear=True) == 0
 
 

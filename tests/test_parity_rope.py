@@ -112,6 +112,36 @@ def test_qknorm_rope_without_k(gpu):
     assert_close(to_np(dwq), rdw, "grad_bf16", "q only dw")
 
 
+@pytest.mark.parametrize("D,dtype", [(128, "bf16"), (64, "f32"), (64, "bf16")])
+def test_qknorm_rope_degenerate_heads(gpu, D, dtype):
+    """Heads the per-head statistic can trip on - all zero (inv_rms = 1/sqrt(eps), output 0),
+    constant, a single large element, a tiny scale - next to ordinary heads, at position 0 (the
+    identity rotation) and beyond, forward and backward against the oracle."""
+    d = wl.qknorm_rope(B=1, S=4, H=6, D=D, dtype=dtype)
+    rng = np.random.default_rng(D)
+    j = np.arange(D)
+    special = [np.zeros(D), np.full(D, -2.0), np.where(j == 5, 300.0, 0.0), 1e-3 * rng.standard_normal(D)]
+    conv = (lambda a: wl.bf16_bits(a.astype(np.float32))) if dtype == "bf16" else (lambda a: a.astype(np.float32))  # noqa
+    for name in ("q", "k"):
+        for s_, row in enumerate(special):
+            d[name][0, s_, s_ % 6] = conv(row)
+    q, k, wq, wk = (to_dev(d[n]) for n in ("q", "k", "wq", "wk"))
+    cos, sin = to_dev(d["cos"]), to_dev(d["sin"])
+    qo, ko, rq, rk = gpu.qknorm_rope_fwd(q, k, wq, wk, cos, sin, d["eps"])
+    dq, dk, dwq, dwk = gpu.qknorm_rope_bwd(q, k, wq, wk, cos, sin, rq, rk, to_dev(d["dq_out"]), to_dev(d["dk_out"]))
+    torch.cuda.synchronize()
+    for name, x, w, dy, out, r, dx, dw in (("q", d["q"], d["wq"], d["dq_out"], qo, rq, dq, dwq),
+                                           ("k", d["k"], d["wk"], d["dk_out"], ko, rk, dk, dwk)):
+        ro, rr = oracle.qknorm_rope_fwd(x, w, d["cos"], d["sin"], d["eps"])
+        rdx, rdw = oracle.qknorm_rope_bwd(x, w, d["cos"], d["sin"], dy, d["eps"])
+        tag = f"qk degenerate {name} {dtype} D={D}"
+        assert_close(to_np(out), ro, io_tol(dtype), tag + " out")
+        assert_close(to_np(r), rr, "stat", tag + " inv_rms")
+        assert_close(to_np(dx), rdx, grad_tol(dtype), tag + " dx")
+        assert_close(to_np(dw), rdw, wgrad_tol(dtype, rdw), tag + " dw")
+    assert gpu.device_error(clear=True) == 0
+
+
 def test_qknorm_unsupported_head_dim(gpu):
     q = torch.zeros(1, 2, 2, 96, dtype=torch.bfloat16, device="cuda")
     w = torch.ones(96, dtype=torch.bfloat16, device="cuda")

@@ -204,7 +204,9 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT)) ln_fwd_
     rb ^= 1u;
     if (++s == a.stages) s = 0, ph ^= 1u;
     const float rs = rsqrtf(fmaf(tq, inv_n, a.eps));
-    const float2 rs2 = dup2(rs), nmr2 = dup2(-mu * rs);
+    // centre, then scale: (x - mu) s keeps near-constant rows (large s) exact where the fused
+    // x s - mu s would round mu s
+    const float2 rs2 = dup2(rs);
     T* yrow = y + m * a.ldy;
 #pragma unroll
     for (int j = 0; j < VPT; ++j) {
@@ -215,7 +217,7 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT)) ln_fwd_
         param_pairs<T>(pipe.param(1), v, bv);
 #pragma unroll
         for (int h = 0; h < H; ++h) {
-          const float2 z = fma2(fma2(xv[j][h], rs2, nmr2), wv[h], bv[h]);
+          const float2 z = fma2(mul2(add2(xv[j][h], nmu), rs2), wv[h], bv[h]);
           if constexpr (EPI == EPI_GELU_TANH)
             o[h] = gelu_of_half2<FAST>(z);
           else
@@ -279,7 +281,8 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT, true)) l
   for (int64_t m = blockIdx.x; m < a.rows; m += step) {
     const float mu = mu_n, rs = rs_n;
     if (m + step < a.rows) mu_n = __ldg(a.mean + m + step), rs_n = __ldg(a.rstd + m + step);
-    const float2 rs2 = dup2(rs), nmr2 = dup2(-mu * rs);
+    // centre, then scale (as the forward): (x - mu) s
+    const float2 rs2 = dup2(rs), nmu2 = dup2(-mu);
     const bool ok = __all_sync(0xffffffffu, mbar_wait(&pipe.full[s], ph, a.err));
     uint4 xr[VPT];  // x stays packed between the two phases (unpacked on use)
     float2 gv[VPT][H];
@@ -302,7 +305,7 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT, true)) l
       unpack2<T>(xr[j], xv);
 #pragma unroll
       for (int h = 0; h < H; ++h) {
-        const float2 xh = fma2(xv[h], rs2, nmr2);
+        const float2 xh = mul2(add2(xv[h], nmu2), rs2);
         const float2 g = EPI == EPI_NONE ? gv[j][h] : mul2(gv[j][h], epi_grad2<EPI, FAST>(fma2(xh, wv[h], bv[h])));
         const float2 gw = mul2(g, wv[h]);
         gv[j][h] = gw;  // phase 2 needs only g w
@@ -331,7 +334,7 @@ __global__ void __launch_bounds__(kNormCtaThreads, norm_min_blocks(VPT, true)) l
         float2 xv[H], o[H];
         unpack2<T>(xr[j], xv);
 #pragma unroll
-        for (int h = 0; h < H; ++h) o[h] = mul2(rs2, add2(gv[j][h], fma2(fma2(xv[h], rs2, nmr2), nc2, nc1)));
+        for (int h = 0; h < H; ++h) o[h] = mul2(rs2, add2(gv[j][h], fma2(mul2(add2(xv[h], nmu2), rs2), nc2, nc1)));
         store_pairs<T>(dxrow, v, nfull, N, o);
       }
     }

@@ -141,7 +141,7 @@ __global__ void __launch_bounds__(kWarpFwdMaxWarps * 32, 1) norm_fwd_warp(const 
         tail[h].y = 2 * h + 1 < tcnt ? V::load1(xrow + tv * E + 2 * h + 1) : 0.0f;
       }
     }
-    float stat_a, stat_b;  // RMSNorm: r, -; LayerNorm: rstd, -mean*rstd
+    float stat_a;  // RMSNorm: r; LayerNorm: rstd
     float mu = 0.0f;
     if constexpr (!LN) {
       float2 acc[H];
@@ -162,7 +162,6 @@ __global__ void __launch_bounds__(kWarpFwdMaxWarps * 32, 1) norm_fwd_warp(const 
       for (int h = 1; h < H; ++h) t = add2(t, acc[h]);
       const float ss = warp_sum(t.x + t.y);
       stat_a = rsqrtf(fmaf(ss, inv_n, a.eps));
-      stat_b = 0.0f;
     } else if constexpr (MODE == 2) {
       // one pass with a shift: K = the mean of the first vector of every lane that has a whole one
       float k0;
@@ -205,7 +204,6 @@ __global__ void __launch_bounds__(kWarpFwdMaxWarps * 32, 1) norm_fwd_warp(const 
       const float m2 = warp_sum(t2.x + t2.y) * inv_n;
       mu = k0 + m1;
       stat_a = rsqrtf(fmaxf(fmaf(-m1, m1, m2), 0.0f) + a.eps);
-      stat_b = -mu * stat_a;
     } else {
       float2 acc[H];
 #pragma unroll
@@ -251,10 +249,11 @@ __global__ void __launch_bounds__(kWarpFwdMaxWarps * 32, 1) norm_fwd_warp(const 
       for (int h = 1; h < H; ++h) t = add2(t, acc[h]);
       const float q = warp_sum(t.x + t.y);
       stat_a = rsqrtf(fmaf(q, inv_n, a.eps));
-      stat_b = -mu * stat_a;
     }
-    // output pass
-    const float2 ra = dup2(stat_a), rb = dup2(stat_b);
+    // output pass. LayerNorm centres first, then scales: (x - mu) s. The fused x s - mu s would
+    // round mu s, an error of up to half an ulp of mu s in every normalized value, which for a
+    // near-constant row (large s) with a mean away from 0 exceeds the output's own rounding.
+    const float2 ra = dup2(stat_a), nmu2 = dup2(-mu);
     T* yrow = y + m * a.ldy;
 #pragma unroll 4
     for (int v = lane; v < nvec; v += 32) {
@@ -271,7 +270,7 @@ __global__ void __launch_bounds__(kWarpFwdMaxWarps * 32, 1) norm_fwd_warp(const 
         prm_pairs<H>(pb, v, nvec, bv);
 #pragma unroll
         for (int h = 0; h < H; ++h) {
-          const float2 z = fma2(fma2(f[h], ra, rb), wv[h], bv[h]);
+          const float2 z = fma2(mul2(add2(f[h], nmu2), ra), wv[h], bv[h]);
           if constexpr (EPI == EPI_GELU_TANH)
             o[h] = gelu_of_half2<FAST>(z);
           else
