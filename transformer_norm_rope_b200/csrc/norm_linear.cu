@@ -112,6 +112,24 @@ enum NlOut { OUT_BF16 = 0, OUT_DGRAD = 1, OUT_ACC32 = 2 };
 
 // The 32 columns col0.. of row m of the epilogue's output from the 32 accumulator values v:
 // o = the corrected pre-activation (OUT_BF16: already activated).
+// OUT_DGRAD: o <- dy[m, col0 ..] * act'(o) for the 32 columns (0 past N; row m < M)
+template <int EPI>
+__device__ __forceinline__ void nl_dgrad32(const NlArgs& a, int m, int col0, float (&o)[32]) {
+  const __nv_bfloat16* g = a.dy + (int64_t)m * a.lddy + col0;
+  if (col0 + 32 <= a.N) {
+#pragma unroll
+    for (int i = 0; i < 32; i += 8) {
+      float f8[8];
+      Vec<__nv_bfloat16>::unpack(ld_stream(g + i), f8);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[i + e] = f8[e] * epi_grad<EPI, true>(o[i + e]);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) o[i] = col0 + i < a.N ? __bfloat162float(g[i]) * epi_grad<EPI, true>(o[i]) : 0.0f;
+  }
+}
+
 template <int OUT, int EPI>
 __device__ __forceinline__ void nl_store32(const NlArgs& a, int m, int col0, const float (&o)[32]) {
   const bool whole = col0 + 32 <= a.N;
@@ -579,6 +597,20 @@ __device__ __forceinline__ void load_tile_pair(uint8_t* dst, const CUtensorMap* 
   }
 }
 
+// TMA store of a box from this CTA's shared memory (bulk-group completion), and the waits on this
+// thread's bulk groups: until at most N remain reading shared memory
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(smem_addr(src))
+               : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* slot, uint32_t ncols) {  // whole warp, both CTAs
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(slot)), "r"(ncols)
                : "memory");
@@ -613,7 +645,7 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
 template <int NORM, int EPI, int OUT = OUT_BF16, int MAJ = 0>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     norm_linear_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                            const NlArgs a) {
+                            const __grid_constant__ CUtensorMap tmY, const NlArgs a) {
   constexpr bool AMN = (MAJ & MAJ_A_MN) != 0, BMN = (MAJ & MAJ_B_MN) != 0;
   static_assert(MAJ == 0 || (NORM == GN_NORM_NONE && kLine == 128), "MN-major operands: no norm, 64-wide k tiles");
   constexpr int kPrefetch = 2 * kPairStages;
@@ -720,6 +752,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     tc_fence_after();
     if (ok) {
       const float nsm = -rs * mu;
+      // bf16 outputs (y, or dz of OUT_DGRAD) leave through shared memory and TMA stores: each
+      // warp turns 64 columns of its 32 rows into one 32 x 128-byte box (128-byte swizzle:
+      // 16-byte chunk c of row r at position c ^ (r % 8)), two boxes in flight per warp, written
+      // to y with the rows and columns past M and N clipped by the store. The pipeline stages
+      // are free once every MMA has completed (accf), so the boxes reuse them. Measured (B200):
+      // the fused LayerNorm + linear + SiLU 1.291 -> 1.258 ms, a dx chunk product 0.191 -> 0.180
+      // ms against one 16-byte store per thread and row.
+      uint8_t* box = smem + (size_t)(warp - 2) * 2 * 4096;
       for (int cb = 0; cb < 256 / 32; ++cb) {
         const int lc = 256 * j + 32 * cb;  // column of the pair tile
         const int col0 = n0 + lc;
@@ -736,11 +776,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           o[i + 2] = fmaf(rs, v[i + 2], fmaf(nsm, c4.z, d4.z));
           o[i + 3] = fmaf(rs, v[i + 3], fmaf(nsm, c4.w, d4.w));
         }
-        if constexpr (OUT == OUT_BF16)
+        if constexpr (OUT != OUT_ACC32) {
+          if constexpr (OUT == OUT_BF16) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = nl_act<EPI>(o[i]);
-        if (m < a.M) nl_store32<OUT, EPI>(a, m, col0, o);
+            for (int i = 0; i < 32; ++i) o[i] = nl_act<EPI>(o[i]);
+          } else if (m < a.M) {  // OUT_DGRAD: the gradient applied (rows past M are clipped anyway)
+            nl_dgrad32<EPI>(a, m, col0, o);
+          }
+          uint8_t* bx = box + (size_t)((cb >> 1) & 1) * 4096;
+          if ((cb & 1) == 0 && cb >= 4) {  // this box's previous store has finished reading it
+            if (lane == 0) bulk_wait_read<1>();
+            __syncwarp();
+          }
+          uint8_t* row = bx + lane * 128;
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            const float f8[8] = {o[i], o[i + 1], o[i + 2], o[i + 3], o[i + 4], o[i + 5], o[i + 6], o[i + 7]};
+            const int c = (cb & 1) * 4 + i / 8;  // 16-byte chunk of the 128-byte box row
+            *reinterpret_cast<uint4*>(row + ((c ^ (lane & 7)) << 4)) = Vec<__nv_bfloat16>::pack(f8);
+          }
+          if ((cb & 1) == 1 || col0 + 32 >= a.N) {  // the box is complete (or the row ends in it)
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) tma_store_2d(&tmY, bx, n0 + 256 * j + 64 * (cb >> 1), m0 + 32 * q);
+          }
+        } else {
+          if (m < a.M) nl_store32<OUT, EPI>(a, m, col0, o);
+        }
       }
+      if constexpr (OUT != OUT_ACC32)
+        if (lane == 0) bulk_wait_read<0>();  // the boxes are read before the CTA may leave
+      __syncwarp();
     }
   }
 
@@ -1024,7 +1090,12 @@ gn_status nl_run(const void* x, int64_t ldx, const void* Wf, int64_t ldw, const 
   }
   const dim3 grid(pair ? (unsigned)(2 * ((N + kPairN - 1) / kPairN)) : (unsigned)((N + kBN - 1) / kBN),
                   (unsigned)((M + bm - 1) / bm));
-  void* args[] = {&ta, &tb, &a};
+  // the pair kernel stores bf16 outputs through TMA: a map of y [M, N] in 32-row x 64-column boxes
+  CUtensorMap ty = ta;
+  if (pair && out != OUT_ACC32 && !make_map(&ty, y, M, N, ldy, 32u)) return GN_ERR_CUDA;
+  void* args_pair[] = {&ta, &tb, &ty, &a};
+  void* args_one[] = {&ta, &tb, &a};
+  void** args = pair ? args_pair : args_one;
   const int threads = pair ? kPairThreads : mh == 2 ? Tile<2>::Threads : Tile<1>::Threads;
   const size_t smem = pair ? kPairSmem : mh == 2 ? Tile<2>::Smem : Tile<1>::Smem;
   if (cudaLaunchKernel(kern, grid, dim3(threads), args, smem, stream) != cudaSuccess) return GN_ERR_CUDA;
