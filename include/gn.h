@@ -14,8 +14,8 @@
  *       - "基准实测": FlashNorm and FlashRoPE applied together (the fused qk-norm + RoPE entry
  *         points combine them per attention head).
  *       - "内核三 TiledLinear": a linear layer run chunk by chunk along the tokens, the backward
- *         recomputing each chunk instead of keeping its activations (gn_act_grad and
- *         GN_NORM_NONE serve it).
+ *         recomputing each chunk instead of keeping its activations (GN_NORM_NONE and the
+ *         plain products below serve it).
  *   [L] "LLM层的优化算子", section "编写定制融合算子": LayerNorm fused with a tanh-GeLU epilogue
  *       (centre, biased variance, divide by sqrt(var + eps), times weight plus bias, GeLU).
  *   [J] "Janus-Pro-7B模型推理加速实战", section 4.1: LayerNorm fused with SiLU = x * sigmoid(x),
@@ -295,10 +295,10 @@ gn_status gn_colsum_bf16(const void* src, float* out, void* ws, size_t ws_bytes,
 
 /* Gradient of the epilogue activation, elementwise over n elements: dz = dy * act'(z) (act as
  * in the gn_epilogue values; GN_EPI_NONE gives dz = dy). z is the pre-activation, dy the
- * gradient of act(z). The backward of a linear layer with an activation needs it before its two
- * gradient products; the token-chunked linear layer ([H] "内核三 TiledLinear": the forward runs
- * chunk by chunk, the backward recomputes each chunk's z instead of keeping it) calls it per
- * chunk. z, dy, dz: contiguous, dt, 16-byte aligned; dz may alias z or dy (elementwise).
+ * gradient of act(z): the step between a layer's activation and its gradient products, for a
+ * caller that holds z. (The token-chunked layer never stores z: gn_linear_act_grad applies the
+ * same derivative where its recompute reads the accumulators back.) z, dy, dz: contiguous, dt,
+ * 16-byte aligned; dz may alias z or dy (elementwise).
  * Errors: GN_ERR_DTYPE, GN_ERR_SHAPE (n < 0), GN_ERR_NULL, GN_ERR_ALIGN, GN_ERR_CUDA. */
 gn_status gn_act_grad(const void* z, const void* dy, void* dz, int64_t n, gn_epilogue epi, gn_dtype dt,
                       void* stream);
