@@ -1,10 +1,11 @@
 // act.cu - gradient of the epilogue activation, elementwise: dz = dy * act'(z).
 //
 // The backward of a linear layer with an activation (y = act(z), z = x W^T + b) needs dz before
-// its two gradient products; the token-chunked linear layer (TiledLinear, Helios kernels
-// article, section "内核三 TiledLinear") recomputes z chunk by chunk and calls this on each
-// chunk. The derivative is the one the normalization kernels' backward uses (epi_grad: the
-// tanh-GeLU with the same constants, SiLU). 16-byte vectors per thread, grid-stride; a ragged
+// its two gradient products; this is that step for a caller that holds z (the token-chunked
+// layer of the Helios kernels article, section "内核三 TiledLinear", never stores z: its
+// recompute applies the same derivative in the tensor-core epilogue). The derivative is the one
+// the normalization kernels' backward uses (epi_grad: the tanh-GeLU with the same constants,
+// SiLU). 16-byte vectors per thread, grid-stride; a ragged
 // tail of fewer than one vector is handled element by element.
 #include "gn_common.cuh"
 #include "gn_host.h"
