@@ -456,9 +456,8 @@ gn_status plan_rope(int64_t B, int64_t S, int64_t H, int64_t D, int ntens, int m
   // stage depth per CTA (measured on B200): the plain rotation computes so little that one
   // CTA per SM with ~4 stages of q and k streams best (deeper pipelines and more CTAs per SM
   // were slower: ~5750 against ~6340 GB/s at [1, 32760, 40, 128]); the qk-norm passes keep
-  // ~84-96 KiB per CTA so that two CTAs share an SM (qk-norm forward at [2, 76800, 40, 128]: 3
-  // stages 5910-5990 GB/s, 4 stages 6080-6100)
-  const size_t depth = mode == ROPE ? 84 * 1024 : mode == QK_FWD ? 84 * 1024 : 96 * 1024;
+  // ~64-96 KiB per CTA so that 2-3 CTAs share an SM
+  const size_t depth = mode == ROPE ? 84 * 1024 : mode == QK_FWD ? 64 * 1024 : 96 * 1024;
   int stages = g_tune.stages ? g_tune.stages : (int)(depth / sstride);
   stages = stages < 2 ? 2 : stages > kRopeMaxStages ? kRopeMaxStages : stages;
   const size_t limit = smem_optin();
