@@ -19,9 +19,10 @@
 // squares in separate passes, three in all), so the row stays in HBM order one 16-byte vector
 // per lane and nothing of it needs to live in registers.
 //
-// The parameters (weight, bias) are widened to fp32 once per CTA in shared memory, with the
-// Gemma +1 offset and, before the tanh-GeLU, the factor 1/2 folded in (exact), so the per-row
-// passes read them with 16-byte loads and no conversion.
+// The parameters (weight, bias) are staged once per CTA in shared memory, before the tanh-GeLU
+// with the factor 1/2 folded in (exact): widened to fp32 with the Gemma +1 offset folded in for
+// RMSNorm and fp32 rows (the per-row passes then read them with no conversion), kept in bf16 for
+// LayerNorm on bf16 rows (half the space, so that more warps fit).
 #include "gn_host.h"
 #include "norm_plan.h"
 #include "norm_rows.cuh"
@@ -45,7 +46,7 @@ struct WarpFwdArgs {
   int N;
   int stages;
   uint32_t slot;    // bytes per stage (one row of whole 16-byte vectors, rounded to 128)
-  uint32_t pbytes;  // bytes per fp32 parameter vector
+  uint32_t pbytes;  // bytes per staged parameter vector
   float eps;
   unsigned* err;
 };
@@ -67,6 +68,9 @@ __global__ void __launch_bounds__(kWarpFwdMaxWarps * 32, 1) norm_fwd_warp(const 
   constexpr int E = V::N, H = E / 2;
   constexpr bool FAST = fast_math_for<T>();
   constexpr bool HALF = LN && EPI == EPI_GELU_TANH;  // parameters staged halved for gelu_of_half2
+  // LayerNorm on bf16 rows keeps its weight and bias in bf16 (unpacked on use): half the shared
+  // memory of fp32 copies, so that 20 warps fit at hidden 5120 instead of 16
+  constexpr bool P16 = LN && sizeof(T) == 2;
   extern __shared__ __align__(128) uint8_t smem[];
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = (int)(blockDim.x >> 5);
   const int S = a.stages;
@@ -97,9 +101,14 @@ __global__ void __launch_bounds__(kWarpFwdMaxWarps * 32, 1) norm_fwd_warp(const 
       }
     }
   }
-  // fp32 parameters, zero past N
-  stage_fp32<T>(pw, static_cast<const T*>(a.w), N, nvec, GEMMA ? 1.0f : 0.0f, HALF ? 0.5f : 1.0f, 1.0f);
-  if constexpr (LN) stage_fp32<T>(pb, static_cast<const T*>(a.b), N, nvec, 0.0f, HALF ? 0.5f : 1.0f, 0.0f);
+  // the parameters, zero past N: fp32 (Gemma offset folded in) or, for P16, the row type
+  if constexpr (P16) {
+    stage_rowtype<T>(reinterpret_cast<uint8_t*>(pw), static_cast<const T*>(a.w), N, nvec, HALF ? 0.5f : 1.0f, 1.0f);
+    stage_rowtype<T>(reinterpret_cast<uint8_t*>(pb), static_cast<const T*>(a.b), N, nvec, HALF ? 0.5f : 1.0f, 0.0f);
+  } else {
+    stage_fp32<T>(pw, static_cast<const T*>(a.w), N, nvec, GEMMA ? 1.0f : 0.0f, HALF ? 0.5f : 1.0f, 1.0f);
+    if constexpr (LN) stage_fp32<T>(pb, static_cast<const T*>(a.b), N, nvec, 0.0f, HALF ? 0.5f : 1.0f, 0.0f);
+  }
   __syncthreads();
 
   const float inv_n = 1.0f / (float)N;
@@ -264,10 +273,16 @@ __global__ void __launch_bounds__(kWarpFwdMaxWarps * 32, 1) norm_fwd_warp(const 
 #pragma unroll
         for (int h = 0; h < H; ++h) f[h] = tail[h];
       }
-      prm_pairs<H>(pw, v, nvec, wv);
+      if constexpr (P16)
+        param_pairs<T>(reinterpret_cast<const uint8_t*>(pw), v, wv);
+      else
+        prm_pairs<H>(pw, v, nvec, wv);
       if constexpr (LN) {
         float2 bv[H];
-        prm_pairs<H>(pb, v, nvec, bv);
+        if constexpr (P16)
+          param_pairs<T>(reinterpret_cast<const uint8_t*>(pb), v, bv);
+        else
+          prm_pairs<H>(pb, v, nvec, bv);
 #pragma unroll
         for (int h = 0; h < H; ++h) {
           const float2 z = fma2(mul2(add2(f[h], nmu2), ra), wv[h], bv[h]);
@@ -333,7 +348,8 @@ gn_status launch_norm_fwd_warp(bool ln, const void* x, const void* w, const void
   const int64_t nfull = N / E;
   if (nfull < 1) return GN_ERR_UNSUPPORTED;
   const uint32_t slot = pipe_slot_bytes(nfull * 16);
-  const uint32_t pbytes = pipe_slot_bytes((N + E - 1) / E * E * 4);
+  // a parameter vector: fp32 copies, or the row type for LayerNorm on bf16 rows (P16 in the kernel)
+  const uint32_t pbytes = pipe_slot_bytes((N + E - 1) / E * E * (ln && dt == GN_BF16 ? 2 : 4));
   unsigned* err = device_err_word();
   if (!err) return GN_ERR_CUDA;
   const size_t limit = smem_optin();

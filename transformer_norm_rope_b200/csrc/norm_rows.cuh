@@ -143,7 +143,29 @@ __device__ __forceinline__ void stage_param_f32(float* dst, const T* src, int N,
   }
 }
 
-// the parameters of vector v as element pairs
+// dst vector v (16 bytes, the row type) = src vector v * scale (a power of two: exact), src == null
+// giving dflt, zero past N. All threads of the CTA take part, one 16-byte load each per vector of
+// an aligned src (element by element for a ragged tail or an unaligned src).
+template <typename T>
+__device__ __forceinline__ void stage_rowtype(uint8_t* dst, const T* src, int N, int nvec, float scale, float dflt) {
+  using V = Vec<T>;
+  constexpr int E = V::N;
+  const int nfull = (src && (reinterpret_cast<uintptr_t>(src) & 15u) == 0) ? N / E : 0;
+  for (int v = (int)threadIdx.x; v < nvec; v += (int)blockDim.x) {
+    float f[E];
+    if (v < nfull) {
+      V::unpack(__ldg(reinterpret_cast<const uint4*>(src) + v), f);
+    } else {
+#pragma unroll
+      for (int e = 0; e < E; ++e) f[e] = v * E + e < N ? ld_param(src, v * E + e, dflt) : 0.0f;
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e) f[e] *= scale;
+    *reinterpret_cast<uint4*>(dst + (size_t)v * 16) = V::pack(f);
+  }
+}
+
+// the parameters of vector v as element pairs// the parameters of vector v as element pairs
 template <typename T>
 __device__ __forceinline__ void param_pairs(const uint8_t* p, int v, float2 (&f)[Vec<T>::N / 2]) {
   unpack2<T>(*reinterpret_cast<const uint4*>(p + (size_t)v * 16), f);
