@@ -134,3 +134,31 @@ def test_norm_linear_autograd_function_matches_backward(gpu):
     assert torch.equal(leaves[0].grad, ref[0])
     for leaf, r in zip(leaves[1:], (ref[1], ref[2], ref[3], ref[4])):
         assert leaf.grad.dtype == leaf.dtype and torch.equal(leaf.grad, r.to(leaf.dtype))
+
+
+def _spread_rows(M):
+    """Rows over the whole range: first, last, tile edges (128 / 256 / 512 row tiles) and a spread."""
+    return np.unique(np.concatenate([np.arange(0, M, M // 40), [1, 127, 128, 129, 255, 256, 511, 512, M - 129, M - 2,
+                                                                 M - 1]]))
+
+
+@pytest.mark.slow
+def test_norm_linear_backward_full_size_sampled_rows(gpu):
+    """The training backward at the benchmark's shape (x [32768, 5120], W [5120, 5120], LayerNorm,
+    SiLU): dx is row-local given the weights, so the oracle's chain rule on sampled rows gives their
+    exact dx; dW, dbias, dg and dbeta sum over all rows and are checked at the small shapes."""
+    from transformer_norm_rope_b200 import norm_linear as nl
+
+    d = wl.norm_linear(seed=0)
+    M, N = d["x"].shape[0], d["W"].shape[0]
+    dy = wl.normal(0, 91, M * N, "bf16").reshape(M, N)
+    xt, gt, bt, Wt, biast = (to_dev(d[k]) for k in ("x", "g", "beta", "W", "bias"))
+    dyt = to_dev(dy)
+    _, mu, rs = nl.forward(xt, gt, bt, Wt, biast, d["eps"], "ln", False, "silu")
+    dx = nl.backward(xt, gt, bt, Wt, biast, mu, rs, dyt, d["eps"], "ln", False, "silu")[0]
+    torch.cuda.synchronize()
+    rows = _spread_rows(M)
+    rdx = oracle.norm_linear_bwd(d["x"][rows], d["g"], d["beta"], d["W"], d["bias"], dy[rows], d["eps"], "ln",
+                                 act="silu")[0]
+    assert_close(to_np(dx)[rows], rdx, "grad_bf16", "full-size norm + linear dx")
+    assert gpu.device_error(clear=True) == 0

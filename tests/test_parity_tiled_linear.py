@@ -158,3 +158,28 @@ def test_bf16_product(gpu, M, N, K, a_mn, b_mn):
     ref, _, _ = oracle.norm_linear(A, None, None, B, bias, 0.0, "none")
     assert_close(to_np(y), ref, "bf16", f"y = A B^T + d (a_mn={a_mn}, b_mn={b_mn})")
     assert gpu.device_error(clear=True) == 0
+
+
+@pytest.mark.slow
+def test_tiled_linear_full_size_sampled_rows(gpu):
+    """The benchmark's TiledLinear (x [32768, 5120], W [5120, 5120], SiLU, 7 backward chunks): y and
+    dx are row-local given the weights, so the oracle on sampled rows - both ends of every chunk,
+    tile edges and a spread - gives their exact values; dW and db sum over all rows and are checked
+    at the small shapes."""
+    M, N, K = 32768, 5120, 5120
+    x = wl.normal(0, 92, M * K, "bf16").reshape(M, K)
+    W = wl.normal(0, 93, N * K, "bf16", scale=1.0 / math.sqrt(K)).reshape(N, K)
+    b = wl.normal(0, 94, N, "bf16", scale=0.1)
+    dy = wl.normal(0, 95, M * N, "bf16").reshape(M, N)
+    Wf, d = tl.prepare(to_dev(W), to_dev(b))
+    y = tl.forward(to_dev(x), Wf, d, "silu")
+    dx = tl.backward(to_dev(x), Wf, d, to_dev(dy), "silu")[0]
+    torch.cuda.synchronize()
+    bounds = list(tl._bounds(M, tl.default_chunks(M, K)))
+    rows = np.unique(np.concatenate([np.arange(0, M, M // 32), [r for b0, b1 in bounds for r in (b0, b0 + 1, b1 - 1)],
+                                     [127, 128, 255, 256, M - 1]]))
+    ry, _, _ = oracle.norm_linear(x[rows], None, None, W, b, 0.0, "none", act="silu")
+    rdx = oracle.linear_act_bwd(x[rows], W, b, dy[rows], "silu")[0]
+    assert_close(to_np(y)[rows], ry, "bf16", "full-size tiled y")
+    assert_close(to_np(dx)[rows], rdx, "grad_bf16", "full-size tiled dx")
+    assert gpu.device_error(clear=True) == 0
