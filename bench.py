@@ -19,8 +19,14 @@ the same seed (weak scaling: the work per GPU is fixed). No activation crosses G
 weight gradients (views of one fp32 bucket) are summed over the ranks by one NCCL all-reduce
 per step inside the timed region.
 
+Besides the step, the line carries per-kernel times, GB/s, roofline fractions and ncu DRAM
+traffic, the end-to-end figure through host buffers (`e2e`), the fp64 CPU oracle on one and on
+all host cores (`cpu_baseline`), SM clocks sampled during the timed region, and (one GPU only,
+outside the step) the fused norm + linear layer (TFLOP/s, forward and training backward) and
+TiledLinear (time and extra peak memory) beside torch autograd.
+
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--only KERNEL[,KERNEL]] [--scale F] [--no-e2e] [--no-cpu-baseline]
+                  [--only KERNEL[,KERNEL]] [--scale F] [--no-e2e] [--no-cpu-baseline] [--no-next]
 """
 from __future__ import annotations
 
@@ -55,7 +61,7 @@ def parse():
     ap.add_argument("--scale", type=float, default=1.0, help="fraction of rows/tokens (profiling)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-next", action="store_true", help="skip the fused norm + linear measurement")
+    ap.add_argument("--no-next", action="store_true", help="skip the norm + linear and TiledLinear measurements")
     ap.add_argument("--seed", type=int, default=0)
     return ap.parse_args()
 
