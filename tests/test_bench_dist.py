@@ -131,6 +131,20 @@ def test_all_cores_oracle_run_covers_the_sample():
     assert t > 0 and done == pytest.approx(sum(nb[k] for k in kernels))
 
 
+def test_oracle_pool_runs_repeat():
+    """A pool's processes keep their inputs between runs: every run covers the same sample."""
+    z = bench.sizes(0.001)
+    kernels = ["rmsnorm_bwd", "rope_bwd"]
+    pool = bench.OraclePool(z, 0, kernels, 0.5, 2)
+    try:
+        runs = [pool.run() for _ in range(3)]
+    finally:
+        pool.close()
+    assert all(t > 0 for t, _ in runs)
+    assert len({b for _, b in runs}) == 1
+    assert all(not p.is_alive() for p in pool.procs)
+
+
 def test_reference_arm_prints_one_json_line():
     env = dict(os.environ, WORLD_SIZE="1", RANK="0")
     r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--scale", "0.002", "--steps", "2",
@@ -140,7 +154,7 @@ def test_reference_arm_prints_one_json_line():
     assert len(lines) == 1
     out = json.loads(lines[0])
     assert out["impl"] == "reference" and out["unit"] == "GB/s" and out["value"] > 0
-    assert out["cpu_baseline"]["kind"] == "oracle" and out["cpu_baseline"]["cores"] == 1
+    assert out["cpu_baseline"]["kind"] == "oracle" and out["cpu_baseline"]["cores"] == bench.host_cores()
     assert out["e2e"]["h2d_bytes_per_step"] == 0 and out["metric"] == bench.METRIC
 
 
