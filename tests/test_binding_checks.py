@@ -162,3 +162,22 @@ def test_tiled_linear_autograd_plumbing(stub, monkeypatch):
     assert stub.count("gn_norm_linear_fwd") == 3 + 1  # the forward: chunked on request, else one launch
     for step in ("gn_linear_act_grad", "gn_linear_bf16", "gn_linear_acc_f32", "gn_colsum_bf16"):
         assert stub.count(step) == chunks, step  # the backward, per chunk
+
+
+@pytest.mark.parametrize("rows,chunks", [(32768, 7), (1000, 2), (300, 2), (64, 1), (5000, 5), (1, 1), (0, 3),
+                                         (4100, 16), (257, 2), (9999, 3)])
+def test_tiled_linear_chunk_bounds(rows, chunks):
+    """Chunks tile the rows in order, start on 8-row boundaries, keep the count that 8-row rounding
+    gives, and start on 256-row tile boundaries whenever that keeps the count."""
+    from transformer_norm_rope_b200 import tiled_linear as tl
+
+    b = list(tl._bounds(rows, chunks))
+    assert all(b[i][1] == b[i + 1][0] for i in range(len(b) - 1))
+    assert (b[0][0], b[-1][1]) == (0, rows) if rows else b == []
+    assert all(r1 > r0 for r0, r1 in b) and all(r0 % 8 == 0 for r0, _ in b)
+    if rows:
+        step8 = -(-(-(-rows // chunks)) // 8) * 8
+        assert len(b) == -(-rows // step8)
+        step256 = -(-(-(-rows // chunks)) // 256) * 256
+        if -(-rows // step256) == len(b):
+            assert all(r0 % 256 == 0 for r0, _ in b)

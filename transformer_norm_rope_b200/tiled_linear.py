@@ -33,13 +33,23 @@ def default_chunks(tokens: int, hidden: int) -> int:
     return max(1, math.ceil(tokens / max(1, hidden)))
 
 
+# rows of one tensor-core output tile (a pair of SMs covers 256 rows)
+_TILE_ROWS = 256
+
+
 def _bounds(rows: int, chunks: int):
+    """Contiguous row ranges of about rows / chunks rows each. Every range starts on a multiple of
+    8 rows (16-byte aligned rows for the kernels) and, where that keeps the number of ranges, on a
+    multiple of the 256-row output tile, so that no chunk's products pay for a partly empty tile
+    row in the middle of the tensor."""
     step = math.ceil(rows / chunks) if rows else 0
-    # 8-row multiples keep every chunk's rows 16-byte aligned for the kernels
-    step = (step + 7) // 8 * 8 if step else 0
+    step8 = (step + 7) // 8 * 8 if step else 0
+    step_t = (step + _TILE_ROWS - 1) // _TILE_ROWS * _TILE_ROWS if step else 0
+    if step and math.ceil(rows / step_t) == math.ceil(rows / step8):
+        step8 = step_t
     r0 = 0
     while r0 < rows:
-        r1 = min(rows, r0 + step)
+        r1 = min(rows, r0 + step8)
         yield r0, r1
         r0 = r1
 
