@@ -449,7 +449,11 @@ def norm_linear_measure(gn, torch, dev, scale, seed, reps=10):
             torch.nn.functional.layer_norm(xa, (K,), ga, ba, d["eps"]), Wa, bia))
         ya.backward(dy)
 
-    t_b, t_ab = timed(bwd), timed(autograd_fwd_bwd)
+    def fwd_bwd_keep_z():  # the training form that stores the pre-activation instead of recomputing it
+        yk, muk, rsk, zk = nl.forward_keeping_z(x, g, beta, W, bias, d["eps"], "ln", False, "silu")
+        nl.backward(x, g, beta, W, bias, muk, rsk, dy, d["eps"], "ln", False, "silu", z=zk)
+
+    t_b, t_ab, t_kz = timed(bwd), timed(autograd_fwd_bwd), timed(fwd_bwd_keep_z)
     flops = 2.0 * M * N * K
     tf = flops / t_f / 1e12
     peak = None
@@ -469,6 +473,9 @@ def norm_linear_measure(gn, torch, dev, scale, seed, reps=10):
             "backward_ms": round(t_b * 1e3, 4),
             "fwd_bwd_ms": round((t_f + t_b) * 1e3, 4),
             "torch_autograd_fwd_bwd_ms": round(t_ab * 1e3, 4),
+            "keep_z_fwd_bwd_ms": round(t_kz * 1e3, 4),
+            "keep_z": "forward keeps the pre-activation (product with no activation, then the activation "
+                      "elementwise); backward forms dz from it instead of recomputing the product",
             "backward": "normalized rows recomputed, activation gradient in the product epilogue, dx and fp32 dW "
                         "on the tensor cores with MN-major operands, column sums, LayerNorm backward"}
 

@@ -303,6 +303,15 @@ gn_status gn_colsum_bf16(const void* src, float* out, void* ws, size_t ws_bytes,
 gn_status gn_act_grad(const void* z, const void* dy, void* dz, int64_t n, gn_epilogue epi, gn_dtype dt,
                       void* stream);
 
+/* The epilogue activation, elementwise over n elements: y = act(z) (act as in the gn_epilogue
+ * values: tanh-GeLU of "LLM层的优化算子" section "编写定制融合算子", SiLU of the Janus-Pro-7B
+ * article section 4.1; GN_EPI_NONE copies). For a caller that keeps the pre-activation z of a
+ * linear layer for its backward (gn_act_grad then forms dz from it) instead of recomputing it:
+ * gn_norm_linear_fwd with GN_EPI_NONE writes z, this call y. z, y: contiguous, dt, 16-byte aligned;
+ * y may alias z (in place).
+ * Errors: GN_ERR_DTYPE, GN_ERR_SHAPE (n < 0), GN_ERR_NULL, GN_ERR_ALIGN, GN_ERR_CUDA. */
+gn_status gn_act_fwd(const void* z, void* y, int64_t n, gn_epilogue epi, gn_dtype dt, void* stream);
+
 /* ---------------------------------------------------------------- runtime queries
  * Number of kernels this process has launched through libgn (all devices, all threads). */
 uint64_t gn_launch_count(void);

@@ -142,3 +142,15 @@ def test_norm_linear_argument_checks(lib):
     assert p(P, None, None, None, P, None, P, 8, 64, LN, 0, gn.GN_BF16, None) == gn.GN_ERR_NULL
     assert p(P, None, None, None, P, P, P, 8, 0, LN, 0, gn.GN_BF16, None) == gn.GN_ERR_SHAPE
     assert p(P, None, None, None, P, P, P, 0, 64, LN, 0, gn.GN_BF16, None) == gn.GN_OK
+
+
+def test_activation_argument_checks(lib):
+    for f, args in ((gn.gn_act_fwd, lambda z, y, n: (z, y, n)), (gn.gn_act_grad, lambda z, y, n: (z, P, y, n))):
+        assert f(*args(P, P, 64), gn.GN_EPI_SILU, 7, None) == gn.GN_ERR_DTYPE
+        assert f(*args(P, P, 64), 9, gn.GN_BF16, None) == gn.GN_ERR_DTYPE
+        assert f(*args(P, P, -1), gn.GN_EPI_SILU, gn.GN_BF16, None) == gn.GN_ERR_SHAPE
+        assert f(*args(P, P, 0), gn.GN_EPI_SILU, gn.GN_BF16, None) == gn.GN_OK  # nothing launched
+        assert f(*args(None, P, 64), gn.GN_EPI_SILU, gn.GN_BF16, None) == gn.GN_ERR_NULL
+        assert f(*args(P, None, 64), gn.GN_EPI_SILU, gn.GN_BF16, None) == gn.GN_ERR_NULL
+        assert f(*args(P + 8, P, 64), gn.GN_EPI_SILU, gn.GN_BF16, None) == gn.GN_ERR_ALIGN
+        assert f(*args(P, P + 4, 64), gn.GN_EPI_SILU, gn.GN_BF16, None) == gn.GN_ERR_ALIGN

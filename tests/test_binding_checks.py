@@ -109,8 +109,9 @@ def test_linear_helpers(stub):
     y = z(M, N)
     gn.norm_linear_fwd(z(M, K)[4:8], Wn, None, dn, norm="none", out=y[4:8])
     gn.act_grad(y, z(M, N), out=y)
+    gn.act_fwd(y, out=y)
     assert stub == ["gn_norm_linear_prepare", "gn_norm_linear_fwd", "gn_norm_linear_prepare",
-                    "gn_norm_linear_fwd", "gn_act_grad"]
+                    "gn_norm_linear_fwd", "gn_act_grad", "gn_act_fwd"]
     bad = [
         lambda: gn.norm_linear_prepare(W, z(N), None, None),  # g is over K
         lambda: gn.norm_linear_prepare(W, None, None, z(K)),  # bias is over N
@@ -124,11 +125,14 @@ def test_linear_helpers(stub):
         lambda: gn.act_grad(z(M, N, dtype=f32), z(M, N)),
         lambda: gn.act_grad(z(N, M).t(), z(M, N)),
         lambda: gn.act_grad(z(M, N), z(M, N), out=z(M, N, dtype=f32)),
+        lambda: gn.act_fwd(z(N, M).t()),
+        lambda: gn.act_fwd(z(M, N), out=z(M, N + 1)),
+        lambda: gn.act_fwd(z(M, N), out=z(M, N, dtype=f32)),
     ]
     for f in bad:
         with pytest.raises((ValueError, TypeError)):
             f()
-    assert len(stub) == 5
+    assert len(stub) == 6
 
 
 def test_tiled_linear_autograd_plumbing(stub, monkeypatch):

@@ -162,3 +162,45 @@ def test_norm_linear_backward_full_size_sampled_rows(gpu):
                                  act="silu")[0]
     assert_close(to_np(dx)[rows], rdx, "grad_bf16", "full-size norm + linear dx")
     assert gpu.device_error(clear=True) == 0
+
+
+@pytest.mark.parametrize("M,N,K", [(300, 264, 520), (64, 40, 136)])
+@pytest.mark.parametrize("norm,act", [("ln", "silu"), ("rms", "gelu_tanh"), ("ln", "none")])
+def test_norm_linear_keeping_z_matches_oracle(gpu, M, N, K, norm, act):
+    """The training form that keeps the pre-activation: the product with no activation writes z,
+    gn_act_fwd forms y from it, and the backward takes dz = dy act'(z) from the stored z
+    (gn_act_grad) instead of recomputing the product. Against the oracle's forward and chain rule,
+    at the tolerances of the recomputing form; the autograd form with keep_z gives the same
+    gradients as the explicit backward."""
+    from transformer_norm_rope_b200 import norm_linear as nl
+
+    x, gw, beta, W, bias = _inputs(M, N, K, seed=M + K, norm=norm)
+    dy = wl.bf16_bits(np.random.default_rng(M + N).standard_normal((M, N)).astype(np.float32))
+    eps = 1e-5
+    xt, gt, bt, Wt, biast, dyt = (None if a is None else to_dev(a) for a in (x, gw, beta, W, bias, dy))
+    y, mu, rs, zt = nl.forward_keeping_z(xt, gt, bt, Wt, biast, eps, norm, False, act)
+    grads = nl.backward(xt, gt, bt, Wt, biast, mu, rs, dyt, eps, norm, False, act, z=zt)
+    torch.cuda.synchronize()
+    ry, _, _ = oracle.norm_linear(x, gw, beta, W, bias, eps, norm, act=act)
+    rz, _, _ = oracle.norm_linear(x, gw, beta, W, bias, eps, norm, act="none")
+    tag = f"keep z {norm} {act} {M}x{N}x{K}"
+    assert_close(to_np(y), ry, "bf16", tag + " y")
+    assert_close(to_np(zt), rz, "bf16", tag + " z")
+    ref = oracle.norm_linear_bwd(x, gw, beta, W, bias, dy, eps, norm, act=act)
+    assert_close(to_np(grads[0]), ref[0], "grad_bf16", tag + " dx")
+    for name, got, r in zip(("dg", "dbeta", "dW", "dbias"), grads[1:], ref[1:]):
+        if r is None:
+            assert got is None, name
+            continue
+        sc = float(np.abs(r).max())
+        assert_close(to_np(got), r, (2e-2, 2e-2 * sc), tag + " " + name)
+    leaves = [None if a is None else to_dev(a).requires_grad_() for a in (x, gw, beta, W, bias)]
+    out = nl.NormLinearFunction.apply(*leaves, eps, norm, False, act, True)
+    out.backward(dyt)
+    torch.cuda.synchronize()
+    assert torch.equal(out.detach(), y)
+    assert torch.equal(leaves[0].grad, grads[0])
+    for leaf, r in zip(leaves[1:], grads[1:]):
+        if leaf is not None:
+            assert torch.equal(leaf.grad, r.to(leaf.dtype))
+    assert gpu.device_error(clear=True) == 0

@@ -183,3 +183,34 @@ def test_tiled_linear_full_size_sampled_rows(gpu):
     assert_close(to_np(y)[rows], ry, "bf16", "full-size tiled y")
     assert_close(to_np(dx)[rows], rdx, "grad_bf16", "full-size tiled dx")
     assert gpu.device_error(clear=True) == 0
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("act", ["silu", "gelu_tanh", "none"])
+def test_elementwise_activation_and_gradient(gpu, dtype, act):
+    """gn_act_fwd (y = act(z)) and gn_act_grad (dz = dy act'(z)) element by element against the
+    oracle's activation and derivative, on a ragged length (a tail shorter than one 16-byte vector)
+    and in place (y over z, dz over dy)."""
+    n = 4099
+    g = np.random.default_rng(n)
+    zf = (3.0 * g.standard_normal(n)).astype(np.float32)
+    dyf = g.standard_normal(n).astype(np.float32)
+    conv = (lambda a: wl.bf16_bits(a)) if dtype == "bf16" else (lambda a: a)  # noqa: E731
+    zh, dyh = conv(zf), conv(dyf)
+    zt, dyt = to_dev(zh), to_dev(dyh)
+    widen = (lambda a: (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)) if dtype == "bf16" else \
+        (lambda a: a.astype(np.float64))  # noqa: E731
+    zr, dyr = widen(zh), widen(dyh)
+    ry = np.array([oracle.act(act, v) for v in zr])
+    rdz = np.array([dv * oracle.act_grad(act, v) for v, dv in zip(zr, dyr)])
+    tol = "bf16" if dtype == "bf16" else "f32"
+    y = gpu.act_fwd(zt, epilogue=act)
+    dz = gpu.act_grad(zt, dyt, epilogue=act)
+    torch.cuda.synchronize()
+    assert_close(to_np(y), ry, tol, f"act {act} {dtype}")
+    assert_close(to_np(dz), rdz, "grad_bf16" if dtype == "bf16" else "f32", f"act' {act} {dtype}")
+    gpu.act_fwd(zt, epilogue=act, out=zt)  # in place
+    gpu.act_grad(to_dev(zh), dyt, epilogue=act, out=dyt)
+    torch.cuda.synchronize()
+    assert torch.equal(zt, y) and torch.equal(dyt, dz)
+    assert gpu.device_error(clear=True) == 0

@@ -60,6 +60,7 @@ SIGNATURES = {
     "gn_colsum_bf16_workspace": (_sz, [_i64]),
     "gn_colsum_bf16": (_st, [_vp, _vp, _vp, _sz, _i64, _i64, _i64, _int, _int, _vp]),
     "gn_act_grad": (_st, [_vp, _vp, _vp, _i64, _int, _int, _vp]),
+    "gn_act_fwd": (_st, [_vp, _vp, _i64, _int, _int, _vp]),
     "gn_launch_count": (C.c_uint64, []),
     "gn_device_error": (_st, [C.POINTER(C.c_uint), _int]),
     "gn_selftest_wait_timeout": (_st, [C.c_uint32, _vp]),
@@ -406,6 +407,15 @@ def act_grad(z, dy, epilogue="silu", out=None, stream=None):
     check(gn_act_grad(_ptr(z), _ptr(dy), _ptr(dz), dy.numel(), _epi(epilogue), _dt(dy), _stream(stream)),
           "gn_act_grad")
     return dz
+
+
+def act_fwd(z, epilogue="silu", out=None, stream=None):
+    """y = act(z), elementwise (contiguous; out may be z itself)."""
+    _need(z, "z")
+    y = torch_empty_like(z) if out is None else out
+    _need(y, "out", like=z, shape=z.shape, dtype=z.dtype)
+    check(gn_act_fwd(_ptr(z), _ptr(y), z.numel(), _epi(epilogue), _dt(z), _stream(stream)), "gn_act_fwd")
+    return y
 
 
 def linear_act_grad(x, Wf, d, dy, epilogue="silu", out=None, stream=None):

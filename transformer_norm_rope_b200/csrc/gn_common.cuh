@@ -221,7 +221,8 @@ __device__ __forceinline__ float group_sum_rt(float v, int width) {
 // ---------------------------------------------------------------- epilogues
 // tanh-GeLU: 0.5 z (1 + tanh(k (z + 0.044715 z^3))), k = sqrt(2/pi). SiLU: z * sigmoid(z).
 // bf16 outputs use the hardware tanh.approx / ex2-based __expf (error far below bf16
-// rounding); fp32 outputs use the accurate tanhf / expf.
+// rounding); fp32 outputs use the accurate expf, the tanh-GeLU through 1 +- tanh(u) formed from
+// exp(-2|u|) (one_pm_tanh).
 
 enum Epi { EPI_NONE = 0, EPI_GELU_TANH = 1, EPI_SILU = 2 };
 
@@ -250,9 +251,25 @@ __device__ __forceinline__ float sigmoid_f(float x) {
   }
 }
 
+// 1 + tanh(u) and 1 - tanh(u) from a = exp(-2|u|): tanh(|u|) = (1 - a) / (1 + a), so the two are
+// 2 / (1 + a) and 2a / (1 + a), the smaller one without cancellation. The fp32 tanh-GeLU and its
+// derivative use this form: with tanh(u) itself, 1 + tanh(u) keeps no significant bits once
+// tanh(u) rounds to -1 (u < -9, z < -5.5), where the derivative is still ~1e-6.
+__device__ __forceinline__ void one_pm_tanh(float u, float& p, float& q) {
+  const float a = expf(-2.0f * fabsf(u));
+  const float r = 2.0f / (1.0f + a);
+  const float ra = r * a;
+  p = u >= 0.0f ? r : ra;  // 1 + tanh(u)
+  q = u >= 0.0f ? ra : r;  // 1 - tanh(u)
+}
+
 template <int EPI, bool FAST>
 __device__ __forceinline__ float epi_fwd(float z) {
-  if constexpr (EPI == EPI_GELU_TANH) {
+  if constexpr (EPI == EPI_GELU_TANH && !FAST) {
+    float p, q;
+    one_pm_tanh(z * fmaf(kGeluK * kGeluC, z * z, kGeluK), p, q);
+    return 0.5f * z * p;
+  } else if constexpr (EPI == EPI_GELU_TANH) {
     const float z2 = z * z;
     const float t = tanh_f<FAST>(z * fmaf(kGeluK * kGeluC, z2, kGeluK));  // k (z + c z^3)
     const float h = 0.5f * z;
@@ -267,7 +284,13 @@ __device__ __forceinline__ float epi_fwd(float z) {
 // d epi / dz
 template <int EPI, bool FAST>
 __device__ __forceinline__ float epi_grad(float z) {
-  if constexpr (EPI == EPI_GELU_TANH) {
+  if constexpr (EPI == EPI_GELU_TANH && !FAST) {
+    // 0.5 (1 + t) + 0.5 z (1 - t)(1 + t) k' = 0.5 (1 + t) (1 + z (1 - t) k'), k' = k (1 + 3 c z^2)
+    const float z2 = z * z;
+    float p, q;
+    one_pm_tanh(z * fmaf(kGeluK * kGeluC, z2, kGeluK), p, q);
+    return 0.5f * p * fmaf(z * q, fmaf(3.0f * kGeluK * kGeluC, z2, kGeluK), 1.0f);
+  } else if constexpr (EPI == EPI_GELU_TANH) {
     const float z2 = z * z;
     const float t = tanh_f<FAST>(z * fmaf(kGeluK * kGeluC, z2, kGeluK));
     // 0.5 (1 + t) + 0.5 z (1 - t^2) k (1 + 3 c z^2)
@@ -281,9 +304,9 @@ __device__ __forceinline__ float epi_grad(float z) {
   }
 }
 
-// The same epilogues on a pair of lanes. The forward tanh-GeLU runs on packed fp32x2
+// The same epilogues on a pair of lanes. On bf16 rows the forward tanh-GeLU runs on packed fp32x2
 // instructions with the scalar form's operations, operand order and constants lane by lane, so
-// each lane rounds exactly as epi_fwd; SiLU runs as two scalar evaluations.
+// each lane rounds exactly as epi_fwd; the fp32 form and SiLU run as two scalar evaluations.
 template <bool FAST>
 __device__ __forceinline__ float2 tanh2(float2 u) {
   return make_float2(tanh_f<FAST>(u.x), tanh_f<FAST>(u.y));
@@ -293,7 +316,7 @@ template <int EPI, bool FAST>
 __device__ __forceinline__ float2 epi_fwd2(float2 z) {
   if constexpr (EPI == EPI_NONE) {
     return z;
-  } else if constexpr (EPI == EPI_GELU_TANH) {
+  } else if constexpr (EPI == EPI_GELU_TANH && FAST) {
     const float2 z2 = mul2(z, z);
     const float2 t = tanh2<FAST>(mul2(z, fma2(dup2(kGeluK * kGeluC), z2, dup2(kGeluK))));
     const float2 h = mul2(dup2(0.5f), z);
@@ -309,19 +332,26 @@ __device__ __forceinline__ float2 epi_fwd2(float2 z) {
 // epi_fwd(z), one multiplication fewer.
 template <bool FAST>
 __device__ __forceinline__ float2 gelu_of_half2(float2 h) {
-  const float2 h2 = mul2(h, h);
-  const float2 t = tanh2<FAST>(mul2(h, fma2(dup2(8.0f * (kGeluK * kGeluC)), h2, dup2(2.0f * kGeluK))));
-  return fma2(h, t, h);
+  if constexpr (!FAST) {  // the fp32 form: GeLU(z) = h (1 + tanh(u)), 1 + tanh(u) without cancellation
+    float p0, p1, q;
+    one_pm_tanh(h.x * fmaf(8.0f * (kGeluK * kGeluC), h.x * h.x, 2.0f * kGeluK), p0, q);
+    one_pm_tanh(h.y * fmaf(8.0f * (kGeluK * kGeluC), h.y * h.y, 2.0f * kGeluK), p1, q);
+    return make_float2(h.x * p0, h.y * p1);
+  } else {
+    const float2 h2 = mul2(h, h);
+    const float2 t = tanh2<FAST>(mul2(h, fma2(dup2(8.0f * (kGeluK * kGeluC)), h2, dup2(2.0f * kGeluK))));
+    return fma2(h, t, h);
+  }
 }
 
-// The tanh-GeLU gradient runs on packed fp32x2 instructions with the scalar form's operations,
-// operand order and constants lane by lane (each lane rounds exactly as epi_grad); SiLU runs as
-// two scalar evaluations.
+// On bf16 rows the tanh-GeLU gradient runs on packed fp32x2 instructions with the scalar form's
+// operations, operand order and constants lane by lane (each lane rounds exactly as epi_grad);
+// the fp32 form and SiLU run as two scalar evaluations.
 template <int EPI, bool FAST>
 __device__ __forceinline__ float2 epi_grad2(float2 z) {
   if constexpr (EPI == EPI_NONE) {
     return dup2(1.0f);
-  } else if constexpr (EPI == EPI_GELU_TANH) {
+  } else if constexpr (EPI == EPI_GELU_TANH && FAST) {
     const float2 z2 = mul2(z, z);
     const float2 t = tanh2<FAST>(mul2(z, fma2(dup2(kGeluK * kGeluC), z2, dup2(kGeluK))));
     const float2 k3 = fma2(dup2(3.0f * 0.5f * kGeluK * kGeluC), z2, dup2(0.5f * kGeluK));
