@@ -346,3 +346,39 @@ def test_unaligned_weights_give_the_aligned_result(gpu, hidden):
     for p, q in zip(a + ga, u + gu):
         assert torch.equal(p, q), f"rmsnorm {hidden}"
     assert gpu.device_error(clear=True) == 0
+
+
+def test_fp32_gelu_far_below_zero(gpu):
+    """fp32 rows whose pre-activations reach far below zero (z down to about -12), where the
+    tanh-GeLU and its derivative are 1e-7 .. 1e-3 and 1 + tanh(u) must not be formed from a
+    tanh(u) that rounds to -1: LayerNorm with a bias near -6 and RMSNorm with a weight near -4,
+    forward and backward through the CTA and warp kernels, against the oracle at the fp32
+    tolerances."""
+    rng = np.random.default_rng(11)
+    for rows, hidden in ((64, 1000), (40, 2051)):
+        x = rng.standard_normal((rows, hidden)).astype(np.float32)
+        dy = rng.standard_normal((rows, hidden)).astype(np.float32)
+        w = (1.0 + 0.1 * rng.standard_normal(hidden)).astype(np.float32)
+        b = (-6.0 + 0.5 * rng.standard_normal(hidden)).astype(np.float32)
+        xt, dyt, wt, bt = to_rows(x), to_rows(dy), to_dev(w), to_dev(b)
+        y, mu, rs = gpu.layernorm_fwd(xt, wt, bt, 1e-5, epilogue="gelu_tanh")
+        dx, dw, db = gpu.layernorm_bwd(xt, wt, bt, mu, rs, dyt, epilogue="gelu_tanh")
+        torch.cuda.synchronize()
+        ry, _, _ = oracle.layernorm_fwd(x, w, b, 1e-5, act="gelu_tanh")
+        rdx, rdw, rdb = oracle.layernorm_bwd(x, w, b, dy, 1e-5, act="gelu_tanh")
+        tag = f"ln f32 {rows}x{hidden} far below zero"
+        assert_close(to_np(y), ry, "f32", tag + " y")
+        assert_close(to_np(dx), rdx, "f32", tag + " dx")
+        assert_close(to_np(dw), rdw, wgrad_tol("f32", rdw), tag + " dw")
+        assert_close(to_np(db), rdb, wgrad_tol("f32", rdb), tag + " db")
+        wr = (-4.0 + 0.1 * rng.standard_normal(hidden)).astype(np.float32)
+        y, r = gpu.rmsnorm_fwd(xt, to_dev(wr), 1e-6, epilogue="gelu_tanh")
+        dx, dw = gpu.rmsnorm_bwd(xt, to_dev(wr), r, dyt, epilogue="gelu_tanh")
+        torch.cuda.synchronize()
+        ry, _ = oracle.rmsnorm_fwd(x, wr, 1e-6, act="gelu_tanh")
+        rdx, rdw = oracle.rmsnorm_bwd(x, wr, dy, 1e-6, act="gelu_tanh")
+        tag = f"rms f32 {rows}x{hidden} far below zero"
+        assert_close(to_np(y), ry, "f32", tag + " y")
+        assert_close(to_np(dx), rdx, "f32", tag + " dx")
+        assert_close(to_np(dw), rdw, wgrad_tol("f32", rdw), tag + " dw")
+    assert gpu.device_error(clear=True) == 0
