@@ -16,9 +16,9 @@
 namespace gn {
 namespace {
 
+// dz may alias z or dy (each element is read before it is written, by the same thread)
 template <typename T, int EPI>
-__global__ void __launch_bounds__(256) act_grad_kernel(const T* __restrict__ z, const T* __restrict__ dy,
-                                                       T* __restrict__ dz, int64_t n) {
+__global__ void __launch_bounds__(256) act_grad_kernel(const T* z, const T* dy, T* dz, int64_t n) {
   constexpr int E = Vec<T>::N;
   constexpr bool FAST = fast_math_for<T>();
   const int64_t nvec = n / E;
