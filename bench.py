@@ -418,19 +418,26 @@ def norm_linear_measure(gn, torch, dev, scale, seed, reps=10):
         xn, _, _ = gn.layernorm_fwd(x, g, beta, d["eps"], save_stats=False)
         torch.nn.functional.silu(torch.addmm(bias, xn, W.t()))
 
-    def timed(fn):
+    def timed(*fns):
+        """Median seconds of each fn over `reps` rounds that run the fns in turn: tensor-core timings
+        drift with the power state within seconds, so variants compared with each other are
+        interleaved rather than timed one after another."""
         for _ in range(3):
-            fn()
+            for fn in fns:
+                fn()
         torch.cuda.synchronize(dev)
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
-        for a, b in ev:
-            a.record(stream)
-            fn()
-            b.record(stream)
+        ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in fns]
+              for _ in range(reps)]
+        for r in ev:
+            for fn, (a, b) in zip(fns, r):
+                a.record(stream)
+                fn()
+                b.record(stream)
         torch.cuda.synchronize(dev)
-        return statistics.median(a.elapsed_time(b) for a, b in ev) * 1e-3
+        out = [statistics.median(r[i][0].elapsed_time(r[i][1]) for r in ev) * 1e-3 for i in range(len(fns))]
+        return out if len(fns) > 1 else out[0]
 
-    t_f, t_u = timed(fused), timed(unfused)
+    t_f, t_u = timed(fused, unfused)
     # the training backward (this library's kernels only) beside torch autograd of the unfused
     # layer (torch LayerNorm, cuBLAS, SiLU), both from the same upstream gradient
     from transformer_norm_rope_b200 import norm_linear as nl
@@ -453,7 +460,7 @@ def norm_linear_measure(gn, torch, dev, scale, seed, reps=10):
         yk, muk, rsk, zk = nl.forward_keeping_z(x, g, beta, W, bias, d["eps"], "ln", False, "silu")
         nl.backward(x, g, beta, W, bias, muk, rsk, dy, d["eps"], "ln", False, "silu", z=zk)
 
-    t_b, t_ab, t_kz = timed(bwd), timed(autograd_fwd_bwd), timed(fwd_bwd_keep_z)
+    t_b, t_ab, t_kz = timed(bwd, autograd_fwd_bwd, fwd_bwd_keep_z)
     flops = 2.0 * M * N * K
     tf = flops / t_f / 1e12
     peak = None
@@ -505,26 +512,31 @@ def tiled_linear_measure(gn, torch, dev, scale, seed, reps=5):
         xa, Wa, ba = x.detach().requires_grad_(), W.detach().requires_grad_(), bias.detach().requires_grad_()
         torch.nn.functional.silu(torch.nn.functional.linear(xa, Wa, ba)).backward(dy)
 
-    def measure(fn):
-        for _ in range(2):
-            fn()
+    variants = (("tiled", tiled(None)), ("one_chunk", tiled(1)), ("torch_autograd", autograd))
+    peaks = {}
+    for name, fn in variants:  # extra peak memory of one call, after a warm-up call
+        fn()
         torch.cuda.synchronize(dev)
         base = torch.cuda.memory_allocated(dev)
         torch.cuda.reset_peak_memory_stats(dev)
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
-        for a, b in ev:
+        fn()
+        torch.cuda.synchronize(dev)
+        peaks[name] = (torch.cuda.max_memory_allocated(dev) - base) / 2**20
+    # times: the variants in turn over `reps` rounds (tensor-core timings drift with the power
+    # state within seconds, so variants compared with each other are interleaved)
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in variants]
+          for _ in range(reps)]
+    for r in ev:
+        for (_, fn), (a, b) in zip(variants, r):
             a.record(stream)
             fn()
             b.record(stream)
-        torch.cuda.synchronize(dev)
-        peak = torch.cuda.max_memory_allocated(dev) - base
-        return statistics.median(a.elapsed_time(b) for a, b in ev), peak / 2**20
-
+    torch.cuda.synchronize(dev)
     out = {"workload": f"linear {K}->{N} + SiLU forward + backward, x[{M},{K}] bf16",
            "default_chunks": tl.default_chunks(M, K)}
-    for name, fn in (("tiled", tiled(None)), ("one_chunk", tiled(1)), ("torch_autograd", autograd)):
-        ms, mib = measure(fn)
-        out[name] = {"ms": round(ms, 3), "peak_extra_MiB": round(mib, 1)}
+    for i, (name, _) in enumerate(variants):
+        ms = statistics.median(r[i][0].elapsed_time(r[i][1]) for r in ev)
+        out[name] = {"ms": round(ms, 3), "peak_extra_MiB": round(peaks[name], 1)}
     gn.check(0 if gn.device_error(clear=True) == 0 else gn.GN_ERR_CUDA, "tiled_linear device error")
     return out
 
